@@ -1,0 +1,206 @@
+"""Float64 CPU oracle for the Comba chunk-wise forward -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package.  The CUDA
+package never imports it and shares no code with it; nothing here is a
+fallback for the GPU path.
+
+Contents (each pinned by the ``-m "not gpu"`` tests against closed forms, a
+hand-worked example, brute-force transition products and invariants):
+
+* ``recurrence``      -- the token-by-token definition in plain C (float64,
+                         OpenMP over the independent (b, h) chains);
+* ``recurrence_np``   -- the same definition in NumPy, for small cases;
+* ``chunked_np``      -- the chunk-wise (inter-chunk recurrent, intra-chunk
+                         parallel) formulation with one unit-lower-triangular
+                         inverse per chunk, in float64.  It is not the oracle
+                         for the GPU; it pins the chunk algebra the kernels use
+                         to the recurrence.
+* ``decode_steps``    -- repeated single-token steps (the recurrence at T=1).
+
+The recurrence (Comba, "Improving Bilinear RNNs with Closed-loop Control";
+PaperWeekly write-up, sections "Comba架构：基于闭环控制理论" and
+"硬件高效的分块并行计算"; arXiv abstract) whose formulas were lost in the
+page extraction, read as:
+
+    S_t = alpha_t S_{t-1} - beta_t S_{t-1} k_t k_t^T + beta_t v_t k_t^T
+    o_t = S_t (q_t - d_h k_t),          alpha_t = exp(log_alpha_t).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "comba_recurrence.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD_DIR, "libcomba_oracle.so")
+_lib = None
+_lock = threading.Lock()
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (float64, no fast-math, no FMA contraction)."""
+    os.makedirs(_BUILD_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or \
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math",
+                               "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            dp = ctypes.POINTER(ctypes.c_double)
+            lib.comba_oracle_recurrence_f64.argtypes = [dp] * 10 + [ctypes.c_long] * 5 + [ctypes.c_int]
+            lib.comba_oracle_recurrence_f64.restype = ctypes.c_int
+            lib.comba_oracle_num_threads.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().comba_oracle_num_threads())
+
+
+def _f64(x) -> np.ndarray:
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor: widen the stored (possibly bf16) values exactly
+        import torch
+        x = x.detach().to("cpu", torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: Optional[np.ndarray]):
+    if a is None:
+        return ctypes.POINTER(ctypes.c_double)()
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def recurrence(q, k, v, log_alpha, beta, d, S0=None, beta_write=None,
+               threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """Token-by-token float64 recurrence (C).  Shapes: q,k [B,T,H,dk], v [B,T,H,dv],
+    log_alpha, beta [B,T,H], d [H], S0 [B,H,dv,dk] or None.
+    ``beta_write`` (self-tests only) replaces beta in the write term.
+    Returns (out [B,T,H,dv], S_final [B,H,dv,dk]) in float64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    la, be, d = _f64(log_alpha), _f64(beta), _f64(d)
+    bw = be if beta_write is None else _f64(beta_write)
+    S0 = _f64(S0)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and v.shape == (B, T, H, dv)
+    assert la.shape == (B, T, H) and be.shape == (B, T, H) and bw.shape == (B, T, H)
+    assert d.shape == (H,)
+    assert S0 is None or S0.shape == (B, H, dv, dk)
+    out = np.empty((B, T, H, dv), dtype=np.float64)
+    S_final = np.empty((B, H, dv, dk), dtype=np.float64)
+    rc = _load().comba_oracle_recurrence_f64(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(be), _ptr(bw), _ptr(d), _ptr(S0),
+        _ptr(out), _ptr(S_final), B, T, H, dk, dv, int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle recurrence failed with status {rc}")
+    return out, S_final
+
+
+def recurrence_np(q, k, v, log_alpha, beta, d, S0=None, beta_write=None):
+    """The same token-by-token definition in NumPy (vectorised over b, h only)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    la, be, d = _f64(log_alpha), _f64(beta), _f64(d)
+    bw = be if beta_write is None else _f64(beta_write)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    S = np.zeros((B, H, dv, dk)) if S0 is None else _f64(S0).copy()
+    out = np.empty((B, T, H, dv))
+    for t in range(T):
+        kt, qv, vt = k[:, t], q[:, t], v[:, t]                      # [B,H,d]
+        a = np.exp(la[:, t])[..., None, None]                       # [B,H,1,1]
+        Sk = np.einsum("bhij,bhj->bhi", S, kt)                      # S_{t-1} k_t
+        S = (a * S
+             - be[:, t][..., None, None] * np.einsum("bhi,bhj->bhij", Sk, kt)
+             + bw[:, t][..., None, None] * np.einsum("bhi,bhj->bhij", vt, kt))
+        qt = qv - d[None, :, None] * kt
+        out[:, t] = np.einsum("bhij,bhj->bhi", S, qt)
+    return out, S
+
+
+def chunked_np(q, k, v, log_alpha, beta, d, S0=None, chunk: int = 64):
+    """Chunk-wise formulation in float64: sequential over chunks of length C,
+    parallel inside a chunk, with one unit-lower-triangular inverse per chunk
+    (the write-up's "block-recurrent, intra-block parallel" form with the single
+    inverse that the scalar-plus-low-rank transition allows).
+
+    Per chunk with chunk-start state S, local positions r, s = 1..L, and
+    g_r = sum_{i<=r} log_alpha_i (g_0 = 0):
+        A_rs  = beta_r exp(g_{r-1} - g_s) (k_r . k_s)      for s < r, else 0
+        Tinv  = (I + A)^{-1}
+        W     = Tinv diag(beta_r exp(g_{r-1})) K,   U~ = Tinv diag(beta_r) V
+        X     = U~ - W S^T                          (rows: beta_r (v_r - S_{r-1} k_r))
+        P_rs  = exp(g_r - g_s) ((q_r - d k_r) . k_s)  for s <= r, else 0
+        O     = diag(exp(g_r)) (Q - d K) S^T + P X
+        S_new = exp(g_L) S + X^T diag(exp(g_L - g_s)) K
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    la, be, d = _f64(log_alpha), _f64(beta), _f64(d)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    S = np.zeros((B, H, dv, dk)) if S0 is None else _f64(S0).copy()
+    out = np.empty((B, T, H, dv))
+    # chain-major views: [B,H,T,*]
+    qh, kh, vh = q.transpose(0, 2, 1, 3), k.transpose(0, 2, 1, 3), v.transpose(0, 2, 1, 3)
+    lah, beh = la.transpose(0, 2, 1), be.transpose(0, 2, 1)
+    dd = d[None, :, None, None]
+    for c0 in range(0, T, chunk):
+        c1 = min(T, c0 + chunk)
+        L = c1 - c0
+        K, Q, V = kh[:, :, c0:c1], qh[:, :, c0:c1], vh[:, :, c0:c1]
+        bt = beh[:, :, c0:c1]
+        g = np.cumsum(lah[:, :, c0:c1], axis=-1)                       # g_1..g_L
+        g_prev = np.concatenate([np.zeros_like(g[..., :1]), g[..., :-1]], axis=-1)
+        KK = np.einsum("bhrd,bhsd->bhrs", K, K)
+        QK = np.einsum("bhrd,bhsd->bhrs", Q, K)
+        strict = np.tril(np.ones((L, L), dtype=bool), k=-1)
+        incl = np.tril(np.ones((L, L), dtype=bool))
+        # exponent differences are only formed where they are <= 0 (s <= r)
+        dg_prev = np.where(strict, g_prev[..., :, None] - g[..., None, :], 0.0)
+        A = np.where(strict, bt[..., :, None] * np.exp(dg_prev) * KK, 0.0)
+        Tinv = np.linalg.solve(np.eye(L) + A, np.broadcast_to(np.eye(L), A.shape))
+        W = Tinv @ ((bt * np.exp(g_prev))[..., None] * K)
+        Ut = Tinv @ (bt[..., None] * V)
+        X = Ut - W @ np.swapaxes(S, -1, -2)
+        dg = np.where(incl, g[..., :, None] - g[..., None, :], 0.0)
+        P = np.where(incl, np.exp(dg) * (QK - dd * KK), 0.0)
+        Qt = Q - dd * K
+        O = np.exp(g)[..., None] * (Qt @ np.swapaxes(S, -1, -2)) + P @ X
+        out[:, c0:c1] = O.transpose(0, 2, 1, 3)
+        gL = g[..., -1:]
+        S = np.exp(gL)[..., None] * S + np.swapaxes(X, -1, -2) @ (np.exp(gL - g)[..., None] * K)
+    return out, S
+
+
+def decode_steps(steps, d, S, threads: int = 0):
+    """Apply single-token steps in order.  ``steps`` yields dicts with q, k [B,H,dk],
+    v [B,H,dv], log_alpha, beta [B,H]; S [B,H,dv,dk] is the state before the first
+    step.  Returns (list of outputs [B,H,dv], final state), float64."""
+    S = _f64(S)
+    outs = []
+    for st in steps:
+        q = _f64(st["q"])[:, None]
+        k = _f64(st["k"])[:, None]
+        v = _f64(st["v"])[:, None]
+        la = _f64(st["log_alpha"])[:, None]
+        be = _f64(st["beta"])[:, None]
+        o, S = recurrence(q, k, v, la, be, d, S, threads=threads)
+        outs.append(o[:, 0])
+    return outs, S
