@@ -1,0 +1,375 @@
+"""Benchmark of the Comba chunk-wise forward on B200.
+
+One step = one chunk-wise forward over the whole workload (every (b, h) chain,
+every token), i.e. one pass of the hot path.  Default workload: the 1.3B-model
+layer shape (B=8, H=16, T=4096, dk=dv=128, chunk=64, bf16 q/k/v/out, fp32
+gates and state), seeded synthetic inputs.
+
+Prints ONE JSON line (rank 0).  ``value`` is device-timed throughput with the
+inputs resident in HBM; ``e2e`` is the same metric through the public Python
+API with the step's inputs copied from pinned host memory and its outputs
+copied back inside the timed region.  Multi-GPU (torchrun): the (b, h) chains
+are independent, so every rank runs its own batch (weak scaling, no
+collective on the data path); time is the max over ranks.
+
+``--impl reference`` times the float64 CPU oracle (the plain token-by-token
+recurrence) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from comba_workloads import CONFIGS, make_chunk_inputs  # noqa: E402
+
+METRIC = "Comba chunk-fwd tokens/s and TFLOP/s on 1 B200, % of roofline"
+L2_BYTES = 126 * 2 ** 20
+
+
+def algorithmic_counts(cfg):
+    """Per-launch algorithmic FLOPs and bytes of the chunk-wise forward.
+
+    FLOPs per head-token (triangle-aware): C(3dk + 2dv) + 6 dk dv
+      (K K^T and Q K^T lower halves, the inverse applied to [K | V], P X lower
+       half; W S^T, (Q - dK) S^T and the X^T K state update).
+    Bytes per head-token: q, k, v and out at their element size plus fp32
+      log(alpha) and beta; plus the fp32 S0 read and S_final write once per chain."""
+    C, dk, dv = cfg.chunk, cfg.dk, cfg.dv
+    el = 2 if cfg.dtype == "bf16" else 4
+    ht = cfg.B * cfg.T * cfg.H
+    flops = ht * (C * (3 * dk + 2 * dv) + 6 * dk * dv)
+    bytes_ = ht * ((2 * dk + 2 * dv) * el + 8) + cfg.B * cfg.H * dv * dk * 4 * 2
+    return flops, bytes_
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "chunk_delta_rule_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    or None when the summary is missing or the kernel source changed since."""
+    path = os.path.join(ROOT, "profiles", f"chunk_fwd_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_h = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m_t or not m_h or m_h.group(1) != kernel_source_hash():
+        return None
+    return float(m_t.group(1))
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi during a region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(cfg, x, target_s: float = 15.0):
+    """Times the float64 oracle (as it stands) on the host cores on a bounded
+    sample of the workload's chains; returns the baseline record."""
+    import oracle
+    import numpy as np
+    threads = oracle.num_threads()
+    B, H = cfg.B, cfg.H
+
+    def run(chains):
+        sl = [(c // H, c % H) for c in chains]
+        xs = {
+            "q": torch.stack([x["q"][b, :, h] for b, h in sl], dim=1)[None],
+            "k": torch.stack([x["k"][b, :, h] for b, h in sl], dim=1)[None],
+            "v": torch.stack([x["v"][b, :, h] for b, h in sl], dim=1)[None],
+            "log_alpha": torch.stack([x["log_alpha"][b, :, h] for b, h in sl], dim=1)[None],
+            "beta": torch.stack([x["beta"][b, :, h] for b, h in sl], dim=1)[None],
+            "d": torch.stack([x["d"][h] for _, h in sl]),
+            "S0": None if x["S0"] is None else torch.stack([x["S0"][b, h] for b, h in sl])[None],
+        }
+        t0 = time.perf_counter()
+        oracle.recurrence(**xs, threads=threads)
+        return time.perf_counter() - t0
+
+    probe = run([0])
+    n = max(1, min(B * H, int(target_s / max(probe, 1e-6)) * threads))
+    n = min(n, B * H)
+    chains = list(range(n))
+    el = run(chains)
+    tokens = n * cfg.T / H  # a token carries all H heads
+    return {"value": tokens / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {B * H} (b,h) chains x {cfg.T} tokens of {cfg.name}, float64 C "
+                      f"recurrence, OpenMP over chains; {el:.1f} s",
+            "seconds": el}
+
+
+def run_reference(args, cfg):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    x = make_chunk_inputs(cfg)
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(cfg, x, target_s=per_step / 4)
+    vals, secs, rec = [], 0.0, None
+    for _ in range(args.steps):
+        rec = cpu_baseline(cfg, x, target_s=per_step)
+        vals.append(rec["value"])
+        secs += rec["seconds"]
+    value = sum(vals) / len(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_record(cfg),
+        "cpu_baseline": {"kind": "oracle", "cores": rec["cores"], "sample": rec["sample"],
+                         "value": value, "unit": "tokens/s"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_record(cfg):
+    return {"workload": cfg.name, "B": cfg.B, "T": cfg.T, "H": cfg.H, "dk": cfg.dk, "dv": cfg.dv,
+            "chunk": cfg.chunk, "tokens_per_step": cfg.B * cfg.T,
+            "l2": "inputs larger than L2 (q,k,v,out %.0f MiB vs 126 MiB L2); no flush"
+                  % (cfg.B * cfg.T * cfg.H * (2 * cfg.dk + 2 * cfg.dv) * (2 if cfg.dtype == "bf16" else 4) / 2 ** 20)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="layer1p3b_bf16", choices=sorted(CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = CONFIGS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+        return
+
+    import chunk_delta_rule_b200 as cdr
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cdr.library()  # fails loudly if the CUDA library is missing
+
+    # Weak scaling: every rank owns a full batch of independent chains.
+    x = make_chunk_inputs(cfg, seed=cfg.seed + 1000 * rank)
+    names = ("q", "k", "v", "log_alpha", "beta", "d", "S0")
+    host = {k: x[k].pin_memory() for k in names if x[k] is not None}
+    dv_ = {k: host[k].to(dev, non_blocking=True) for k in host}
+    S0 = dv_.get("S0")
+    out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.dv), dtype=cfg.torch_dtype, device=dev)
+    S_final = torch.empty((cfg.B, cfg.H, cfg.dv, cfg.dk), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        cdr.chunk_fwd(dv_["q"], dv_["k"], dv_["v"], dv_["log_alpha"], dv_["beta"], dv_["d"], S0,
+                      chunk=cfg.chunk, out=out, S_final=S_final, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert cdr.get_last_error(dev) == 0
+
+    # ---- device-timed region: inputs resident in HBM -------------------------------
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms, world, dev)
+    ms_step = ms / args.steps
+    tokens_all = world * cfg.B * cfg.T
+    value = tokens_all / (ms_step / 1e3)
+    if cdr.get_last_error(dev) != 0:
+        raise RuntimeError("device-side error during the timed region")
+
+    # ---- end-to-end: pinned host -> device, the public API call, results -> host ----
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    S_h = torch.empty(S_final.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size() + S_h.numel() * 4
+
+    def e2e_step():
+        for k in host:
+            dv_[k].copy_(host[k], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        S_h.copy_(S_final, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), world, dev) / args.steps
+    e2e_value = tokens_all / (ms_e2e / 1e3)
+
+    # ---- roofline of the (single) kernel per step ---------------------------------
+    flops, bytes_ = algorithmic_counts(cfg)
+    peaks = load_peaks()
+    achieved_gbs = bytes_ / (ms_step / 1e3) / 1e9
+    tflops = flops / (ms_step / 1e3) / 1e12
+    traffic = profiled_traffic(cfg.name)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": config_record(cfg),
+        "tflops": tflops,
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
+                     "traffic": traffic, "peak_source": peaks["source"] + " hbm_gbs (copy)",
+                     "algorithmic_bytes_per_launch": bytes_,
+                     "algorithmic_flops_per_launch": flops,
+                     "tensor_frac_of_bf16_peak": tflops / peaks["bf16_tflops"]},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+        "clocks": clocks.summary(),
+        "gpu_launches": args.steps,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = {k: v for k, v in cpu_baseline(cfg, x).items() if k != "seconds"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,174 @@
+"""Comba chunk-wise forward and decode step on B200 (sm_100a).
+
+Thin ctypes binding over the C ABI in ``include/comba.h``: it checks tensor
+placement, dtypes and contiguity, allocates outputs with PyTorch when the
+caller does not pass them, and hands raw device pointers and sizes to the
+library.  Every step of the computation runs in the library's CUDA kernels;
+there is no other implementation behind these functions, and they raise if
+the library is missing or a tensor is not on a CUDA device.
+
+Recurrence (Comba, "Improving Bilinear RNNs with Closed-loop Control"):
+    S_t = alpha_t S_{t-1} - beta_t (S_{t-1} k_t) k_t^T + beta_t v_t k_t^T
+    o_t = S_t (q_t - d_h k_t),        alpha_t = exp(log_alpha_t)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = ["chunk_fwd", "recurrent_step", "get_last_error", "CombaError", "library",
+           "library_path", "EXPORTS", "status_string"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libcomba.so")
+_lib = None
+_lock = threading.Lock()
+
+EXPORTS = ("comba_chunk_fwd", "comba_chunk_fwd_f32", "comba_recurrent_step",
+           "comba_get_last_error", "comba_status_string", "comba_version")
+
+
+class CombaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({status_string(status)})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def library():
+    """The loaded ``libcomba.so`` (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                                   "`python -m chunk_delta_rule_b200.build`")
+            lib = ctypes.CDLL(_LIB_PATH)
+            vp, i = ctypes.c_void_p, ctypes.c_int
+            chunk_sig = [vp] * 9 + [i] * 6 + [vp]
+            lib.comba_chunk_fwd.argtypes = chunk_sig
+            lib.comba_chunk_fwd_f32.argtypes = chunk_sig
+            lib.comba_recurrent_step.argtypes = [vp] * 8 + [i] * 4 + [vp]
+            for fn in (lib.comba_chunk_fwd, lib.comba_chunk_fwd_f32, lib.comba_recurrent_step,
+                       lib.comba_get_last_error, lib.comba_version):
+                fn.restype = ctypes.c_int
+            lib.comba_get_last_error.argtypes = []
+            lib.comba_version.argtypes = []
+            lib.comba_status_string.argtypes = [ctypes.c_int]
+            lib.comba_status_string.restype = ctypes.c_char_p
+            _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return library().comba_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(None) if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t: torch.Tensor, name: str, dtype, shape):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype} (got {t.dtype})")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream_handle(device: torch.device, stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+              beta: torch.Tensor, d: torch.Tensor, S0: Optional[torch.Tensor] = None,
+              chunk: int = 64, out: Optional[torch.Tensor] = None,
+              S_final: Optional[torch.Tensor] = None, return_state: bool = True,
+              stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunk-wise forward.  q, k [B,T,H,dk], v [B,T,H,dv] (bf16 or fp32, same
+    dtype); log_alpha, beta [B,T,H] fp32; d [H] fp32; S0 [B,H,dv,dk] fp32 or None.
+    Returns (out [B,T,H,dv] in q's dtype, S_final [B,H,dv,dk] fp32 or None).
+    ``S_final`` may be passed as ``S0`` itself for an in-place state carry."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in (torch.bfloat16, torch.float32):
+        raise TypeError("q, k, v must be bf16 or fp32")
+    _check(q, "q", dt, (B, T, H, dk))
+    _check(k, "k", dt, (B, T, H, dk))
+    _check(v, "v", dt, (B, T, H, dv))
+    _check(log_alpha, "log_alpha", torch.float32, (B, T, H))
+    _check(beta, "beta", torch.float32, (B, T, H))
+    _check(d, "d", torch.float32, (H,))
+    dev = q.device
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (B, H, dv, dk))
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    _check(out, "out", dt, (B, T, H, dv))
+    if S_final is None and return_state:
+        S_final = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _check(S_final, "S_final", torch.float32, (B, H, dv, dk))
+    lib = library()
+    fn = lib.comba_chunk_fwd if dt == torch.bfloat16 else lib.comba_chunk_fwd_f32
+    with torch.cuda.device(dev):
+        st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(d), _ptr(S0),
+                _ptr(out), _ptr(S_final), B, T, H, dk, dv, int(chunk), _stream_handle(dev, stream))
+    if st != 0:
+        raise CombaError(st, "comba_chunk_fwd" + ("" if dt == torch.bfloat16 else "_f32"))
+    return out, S_final
+
+
+def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                   beta: torch.Tensor, d: torch.Tensor, S: torch.Tensor,
+                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One decode token: q, k [B,H,dk] bf16, v [B,H,dv] bf16, log_alpha, beta [B,H]
+    fp32, d [H] fp32, S [B,H,dv,dk] fp32 updated in place.  Returns out [B,H,dv] bf16."""
+    if q.dim() != 3:
+        raise ValueError("q must be [B, H, dk]")
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", torch.bfloat16, (B, H, dk))
+    _check(k, "k", torch.bfloat16, (B, H, dk))
+    _check(v, "v", torch.bfloat16, (B, H, dv))
+    _check(log_alpha, "log_alpha", torch.float32, (B, H))
+    _check(beta, "beta", torch.float32, (B, H))
+    _check(d, "d", torch.float32, (H,))
+    _check(S, "S", torch.float32, (B, H, dv, dk))
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=torch.bfloat16, device=dev)
+    _check(out, "out", torch.bfloat16, (B, H, dv))
+    with torch.cuda.device(dev):
+        st = library().comba_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                            _ptr(beta), _ptr(d), _ptr(S), _ptr(out), B, H, dk,
+                                            dv, _stream_handle(dev, stream))
+    if st != 0:
+        raise CombaError(st, "comba_recurrent_step")
+    return out
+
+
+def get_last_error(device=None) -> int:
+    """Reads and clears the device-side status word (synchronises the device)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(library().comba_get_last_error())

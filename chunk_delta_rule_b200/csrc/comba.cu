@@ -1,0 +1,202 @@
+// C ABI of the Comba chunk-wise forward and decode step (declared in comba.h).
+//
+// The host side validates every argument before anything is enqueued, picks
+// the kernel for the shape, launches on the caller's stream and returns a
+// status.  It owns no device memory.
+#include "comba.h"
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "common.cuh"
+#include "chunk_simt.cuh"
+#include "chunk_tc.cuh"
+#include "recurrent_step.cuh"
+
+namespace {
+
+using comba::SimtSmem;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Byte ranges [a, a + na) and [b, b + nb) intersect.
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+struct ChunkArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta, *d, *S0;
+    void* out;
+    float* S_final;
+    int B, T, H, dk, dv, chunk;
+    size_t elt;  // bytes per q/k/v/out element
+};
+
+int validate_chunk(const ChunkArgs& a) {
+    if (a.B < 0 || a.T < 0 || a.H < 0) return COMBA_EINVAL;
+    if (a.dk < 16 || a.dk > 128 || a.dk % 16) return COMBA_EINVAL;
+    if (a.dv < 16 || a.dv > 128 || a.dv % 16) return COMBA_EINVAL;
+    if (a.chunk != 16 && a.chunk != 32 && a.chunk != 64) return COMBA_EINVAL;
+    if (a.B == 0 || a.H == 0) return COMBA_OK;
+    if (!a.d) return COMBA_EINVAL;
+    if (a.T > 0 && (!a.q || !a.k || !a.v || !a.log_alpha || !a.beta || !a.out)) return COMBA_EINVAL;
+    const size_t bth = (size_t)a.B * a.T * a.H;
+    if (bth > (size_t)1 << 40) return COMBA_EINVAL;
+    const size_t nqk = bth * a.dk * a.elt, nv = bth * a.dv * a.elt;
+    const size_t ng = bth * sizeof(float), nd = (size_t)a.H * sizeof(float);
+    const size_t ns = (size_t)a.B * a.H * a.dv * a.dk * sizeof(float);
+    if (!aligned(a.q, 16) || !aligned(a.k, 16) || !aligned(a.v, 16) || !aligned(a.out, 16) ||
+        !aligned(a.S0, 16) || !aligned(a.S_final, 16) || !aligned(a.log_alpha, 4) ||
+        !aligned(a.beta, 4) || !aligned(a.d, 4))
+        return COMBA_EINVAL;
+    const void* ins[] = {a.q, a.k, a.v, a.log_alpha, a.beta, a.d, a.S0};
+    const size_t nin[] = {nqk, nqk, nv, ng, ng, nd, ns};
+    for (int i = 0; i < 7; ++i) {
+        if (overlap(a.out, nv, ins[i], nin[i])) return COMBA_EINVAL;
+        // S_final may alias S0 exactly (in-place carry), nothing else.
+        if (i == 6 && a.S_final == a.S0) continue;
+        if (overlap(a.S_final, ns, ins[i], nin[i])) return COMBA_EINVAL;
+    }
+    if (overlap(a.S_final, ns, a.out, nv)) return COMBA_EINVAL;
+    return COMBA_OK;
+}
+
+int current_device(int* dev) {
+    if (cudaGetDevice(dev) != cudaSuccess) return COMBA_ECUDA;
+    if (*dev < 0 || *dev >= kMaxDevices) return COMBA_ECUDA;
+    return COMBA_OK;
+}
+
+// T == 0: the final state is the initial one.
+int empty_sequence(const ChunkArgs& a, cudaStream_t stream) {
+    if (!a.S_final) return COMBA_OK;
+    const size_t ns = (size_t)a.B * a.H * a.dv * a.dk * sizeof(float);
+    cudaError_t e = a.S0 ? (a.S0 == a.S_final ? cudaSuccess
+                                              : cudaMemcpyAsync(a.S_final, a.S0, ns,
+                                                                cudaMemcpyDeviceToDevice, stream))
+                         : cudaMemsetAsync(a.S_final, 0, ns, stream);
+    return e == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
+}
+
+template <typename Tin>
+int launch_simt(const ChunkArgs& a, cudaStream_t stream) {
+    static bool attr_set[kMaxDevices] = {};
+    int dev;
+    if (int st = current_device(&dev)) return st;
+    const int dvt = (a.dv % 32 == 0) ? 32 : 16;
+    const SimtSmem m = comba::simt_smem_layout(a.dk, dvt, a.chunk);
+    const size_t smem = m.total * sizeof(float);
+    auto kern = comba::chunk_fwd_simt_kernel<Tin>;
+    if (!attr_set[dev]) {
+        const SimtSmem mx = comba::simt_smem_layout(128, 32, 64);
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(mx.total * sizeof(float))) != cudaSuccess)
+            return COMBA_ECUDA;
+        attr_set[dev] = true;
+    }
+    dim3 grid((a.dv + dvt - 1) / dvt, a.H, a.B);
+    kern<<<grid, comba::kSimtThreads, smem, stream>>>(
+        static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
+        a.log_alpha, a.beta, a.d, a.S0, static_cast<Tin*>(a.out), a.S_final, a.T, a.H, a.dk,
+        a.dv, a.chunk, dvt);
+    return cudaGetLastError() == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
+}
+
+}  // namespace
+
+extern "C" int comba_chunk_fwd(const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta, const float* d,
+                               const float* S0, void* out, float* S_final, int B, int T, int H,
+                               int dk, int dv, int chunk, comba_stream_t stream) {
+    const ChunkArgs a{q, k, v, log_alpha, beta, d, S0, out, S_final, B, T, H, dk, dv, chunk, 2};
+    if (int st = validate_chunk(a)) return st;
+    if (B == 0 || H == 0) return COMBA_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) return empty_sequence(a, s);
+    if (comba::tc_supported(dk, dv, chunk)) return comba::launch_chunk_tc(a.q, a.k, a.v, a.log_alpha, a.beta, a.d, a.S0, a.out, a.S_final, B, T, H, s);
+    return launch_simt<__nv_bfloat16>(a, s);
+}
+
+extern "C" int comba_chunk_fwd_f32(const float* q, const float* k, const float* v,
+                                   const float* log_alpha, const float* beta, const float* d,
+                                   const float* S0, float* out, float* S_final, int B, int T,
+                                   int H, int dk, int dv, int chunk, comba_stream_t stream) {
+    const ChunkArgs a{q, k, v, log_alpha, beta, d, S0, out, S_final, B, T, H, dk, dv, chunk, 4};
+    if (int st = validate_chunk(a)) return st;
+    if (B == 0 || H == 0) return COMBA_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) return empty_sequence(a, s);
+    return launch_simt<float>(a, s);
+}
+
+extern "C" int comba_recurrent_step(const void* q, const void* k, const void* v,
+                                    const float* log_alpha, const float* beta, const float* d,
+                                    float* S, void* out, int B, int H, int dk, int dv,
+                                    comba_stream_t stream) {
+    if (B < 0 || H < 0) return COMBA_EINVAL;
+    if (dk != 32 && dk != 64 && dk != 128) return COMBA_EINVAL;
+    if (dv < 16 || dv > 128 || dv % 16) return COMBA_EINVAL;
+    if (B == 0 || H == 0) return COMBA_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !d || !S || !out) return COMBA_EINVAL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(S, 16) || !aligned(log_alpha, 4) || !aligned(beta, 4) || !aligned(d, 4))
+        return COMBA_EINVAL;
+    const size_t bh = (size_t)B * H;
+    if (bh > (size_t)1 << 31) return COMBA_EINVAL;
+    const size_t nqk = bh * dk * 2, nv = bh * dv * 2, ng = bh * 4, ns = bh * dv * dk * 4;
+    const void* ins[] = {q, k, v, log_alpha, beta, d};
+    const size_t nin[] = {nqk, nqk, nv, ng, ng, (size_t)H * 4};
+    for (int i = 0; i < 6; ++i)
+        if (overlap(out, nv, ins[i], nin[i]) || overlap(S, ns, ins[i], nin[i])) return COMBA_EINVAL;
+    if (overlap(out, nv, S, ns)) return COMBA_EINVAL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const auto* qb = static_cast<const __nv_bfloat16*>(q);
+    const auto* kb = static_cast<const __nv_bfloat16*>(k);
+    const auto* vb = static_cast<const __nv_bfloat16*>(v);
+    auto* ob = static_cast<__nv_bfloat16*>(out);
+    const unsigned grid = (unsigned)bh;
+    switch (dk) {
+        case 32:
+            comba::recurrent_step_kernel<32><<<grid, comba::kStepThreads, 0, s>>>(qb, kb, vb, log_alpha, beta, d, S, ob, H, dv);
+            break;
+        case 64:
+            comba::recurrent_step_kernel<64><<<grid, comba::kStepThreads, 0, s>>>(qb, kb, vb, log_alpha, beta, d, S, ob, H, dv);
+            break;
+        default:
+            comba::recurrent_step_kernel<128><<<grid, comba::kStepThreads, 0, s>>>(qb, kb, vb, log_alpha, beta, d, S, ob, H, dv);
+            break;
+    }
+    return cudaGetLastError() == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
+}
+
+extern "C" int comba_get_last_error(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;
+    int h = 0;
+    if (cudaMemcpyFromSymbol(&h, comba::g_status, sizeof(int)) != cudaSuccess) return COMBA_ECUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(comba::g_status, &zero, sizeof(int)) != cudaSuccess) return COMBA_ECUDA;
+    return h;
+}
+
+extern "C" const char* comba_status_string(int status) {
+    switch (status) {
+        case COMBA_OK: return "ok";
+        case COMBA_EINVAL: return "invalid argument (pointer, size, alignment or aliasing)";
+        case COMBA_EUNSUPPORTED: return "unsupported shape";
+        case COMBA_ECUDA: return "CUDA runtime error";
+        case COMBA_ETIMEOUT: return "device-side bounded wait gave up";
+        case COMBA_EDEVICE: return "device-side inconsistency";
+        default: return "unknown status";
+    }
+}
+
+extern "C" int comba_version(void) { return 100; }

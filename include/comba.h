@@ -1,0 +1,121 @@
+/*
+ * comba.h -- C ABI of the B200 (sm_100a) Comba chunk-wise forward and decode step.
+ *
+ * The method: Comba, "Improving Bilinear RNNs with Closed-loop Control"
+ * (PaperWeekly write-up and arXiv abstract 2506.02475).  Comba's recurrent
+ * state S (dv x dk per batch element and head) follows a scalar-plus-low-rank
+ * (SPLR) transition with the key as state feedback, and its output is read
+ * through a second, output-side feedback on the same key (write-up, section
+ * "Comba架构：基于闭环控制理论"):
+ *
+ *     S_t = alpha_t S_{t-1} - beta_t (S_{t-1} k_t) k_t^T + beta_t v_t k_t^T
+ *     o_t = S_t (q_t - d_h k_t),           alpha_t = exp(log_alpha_t)
+ *
+ * The training/prefill form is chunk-wise: recurrent across chunks of `chunk`
+ * tokens and parallel inside a chunk, with one unit-lower-triangular inverse
+ * per chunk (write-up, section "硬件高效的分块并行计算").  The single-token
+ * form is the constant-memory recurrent step used for decoding (write-up,
+ * section "背景知识和相关工作").
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *    owned by the caller; the library allocates nothing per call and keeps no
+ *    reference after the call is enqueued.
+ *  - Layouts are dense row-major:
+ *        q, k      [B, T, H, dk]      v, out [B, T, H, dv]
+ *        log_alpha, beta  [B, T, H]   fp32 (log_alpha <= 0 expected, not required)
+ *        d         [H]                fp32, the per-head output-correction factor
+ *        S0, S_final [B, H, dv, dk]   fp32 (row i = value index, column j = key index)
+ *  - q, k, v, out, S0 and S_final must be 16-byte aligned; log_alpha, beta and d
+ *    4-byte aligned.
+ *  - S0 == NULL means a zero initial state; S_final == NULL skips the final
+ *    state.  S_final may alias S0 exactly (in-place state carry); no other
+ *    output may overlap any input.
+ *  - Work is enqueued asynchronously on `stream` (NULL = legacy default
+ *    stream).  The return value reports argument and launch errors only;
+ *    errors found on the device (a bounded wait that gave up) are latched in
+ *    a per-device status word read by comba_get_last_error().
+ *  - No C++ exception crosses this boundary.
+ */
+#ifndef COMBA_H_
+#define COMBA_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without pulling in the CUDA headers. */
+typedef struct CUstream_st* comba_stream_t;
+
+enum comba_status {
+    COMBA_OK = 0,
+    COMBA_EINVAL = -1,        /* bad pointer, size, alignment or aliasing; nothing launched */
+    COMBA_EUNSUPPORTED = -2,  /* valid but unsupported shape (see each entry point) */
+    COMBA_ECUDA = -3,         /* a CUDA runtime call failed (launch, attribute, device query) */
+    COMBA_ETIMEOUT = -4,      /* device side: a bounded wait gave up (comba_get_last_error) */
+    COMBA_EDEVICE = -5        /* device side: inconsistent internal state detected */
+};
+
+/*
+ * Chunk-wise forward, bf16 inputs and output, fp32 gates/state/accumulation.
+ *
+ * Computes, for every (b, h) chain independently, out[b, t, h, :] = o_t for
+ * t = 0..T-1 and S_final[b, h] = S_T, starting from S0[b, h] (write-up,
+ * sections "Comba架构：基于闭环控制理论" and "硬件高效的分块并行计算").
+ *
+ * q, k, v, out: __nv_bfloat16.  Sizes: B, H >= 0; T >= 0 (T == 0 copies S0, or
+ * zeros, to S_final); dk, dv multiples of 16 in [16, 128]; chunk in {16, 32,
+ * 64}.  Any T is accepted: a last chunk shorter than `chunk` uses the same
+ * math.  dk == dv == 128 with chunk == 64 runs the tensor-core kernel; other
+ * shapes run the general kernel.
+ */
+int comba_chunk_fwd(const void* q, const void* k, const void* v,
+                    const float* log_alpha, const float* beta, const float* d,
+                    const float* S0, void* out, float* S_final,
+                    int B, int T, int H, int dk, int dv, int chunk,
+                    comba_stream_t stream);
+
+/*
+ * Chunk-wise forward with fp32 q, k, v and out (same math, same layouts, same
+ * size rules as comba_chunk_fwd); every product is an fp32 FMA, no reduced-
+ * precision tensor-core arithmetic.
+ */
+int comba_chunk_fwd_f32(const float* q, const float* k, const float* v,
+                        const float* log_alpha, const float* beta, const float* d,
+                        const float* S0, float* out, float* S_final,
+                        int B, int T, int H, int dk, int dv, int chunk,
+                        comba_stream_t stream);
+
+/*
+ * One recurrent (decode) step for every (b, h): the recurrence above at a
+ * single token, updating the resident state in place (write-up, section
+ * "背景知识和相关工作": constant memory and O(1) work per token).
+ *
+ * q, k [B, H, dk] and v [B, H, dv]: __nv_bfloat16; log_alpha, beta [B, H] fp32;
+ * d [H] fp32; S [B, H, dv, dk] fp32, read and overwritten with S_t; out
+ * [B, H, dv] __nv_bfloat16 receives o_t = S_t (q - d_h k).  dk in {32, 64,
+ * 128}; dv a multiple of 16 in [16, 128].  B or H == 0 is a no-op.
+ */
+int comba_recurrent_step(const void* q, const void* k, const void* v,
+                         const float* log_alpha, const float* beta, const float* d,
+                         float* S, void* out, int B, int H, int dk, int dv,
+                         comba_stream_t stream);
+
+/*
+ * Reads and clears the current device's status word (synchronises the
+ * device first).  Returns COMBA_OK, COMBA_ETIMEOUT, COMBA_EDEVICE, or
+ * COMBA_ECUDA if the synchronisation or the read itself failed.
+ */
+int comba_get_last_error(void);
+
+/* Static, NUL-terminated description of a status code. */
+const char* comba_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int comba_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* COMBA_H_ */

@@ -1,0 +1,126 @@
+"""The C ABI library on the host: it loads without a GPU, exports every function
+the public header declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import chunk_delta_rule_b200 as cdr
+from chunk_delta_rule_b200 import build as cbuild
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "comba.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    cbuild.build()
+    return cdr.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(comba_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("comba_chunk_fwd", "comba_chunk_fwd_f32", "comba_recurrent_step",
+              "comba_get_last_error", "comba_status_string", "comba_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) <= set(cdr.EXPORTS) | set(declared_functions())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.comba_version() == 100
+    assert cdr.status_string(0) == "ok"
+    for code in (-1, -2, -3, -4, -5):
+        assert cdr.status_string(code) not in ("ok", "unknown status")
+    assert cdr.status_string(12345) == "unknown status"
+
+
+# Fake, well-aligned, non-overlapping "device" addresses: validation rejects
+# before any CUDA call, so they are never dereferenced.
+BASE = 1 << 40
+GB = 1 << 30
+
+
+def _chunk_args(**kw):
+    a = dict(q=BASE, k=BASE + GB, v=BASE + 2 * GB, log_alpha=BASE + 3 * GB, beta=BASE + 4 * GB,
+             d=BASE + 5 * GB, S0=BASE + 6 * GB, out=BASE + 7 * GB, S_final=BASE + 8 * GB,
+             B=2, T=128, H=4, dk=64, dv=64, chunk=64)
+    a.update(kw)
+    return a
+
+
+def _call_chunk(lib, a, f32=False):
+    fn = lib.comba_chunk_fwd_f32 if f32 else lib.comba_chunk_fwd
+    p = lambda x: ctypes.c_void_p(x)
+    return fn(p(a["q"]), p(a["k"]), p(a["v"]), p(a["log_alpha"]), p(a["beta"]), p(a["d"]),
+              p(a["S0"]), p(a["out"]), p(a["S_final"]), a["B"], a["T"], a["H"], a["dk"],
+              a["dv"], a["chunk"], ctypes.c_void_p(None))
+
+
+@pytest.mark.parametrize("bad", [
+    dict(dk=7), dict(dk=0), dict(dk=144), dict(dv=24), dict(dv=256), dict(chunk=48),
+    dict(chunk=128), dict(chunk=0), dict(B=-1), dict(T=-3), dict(H=-2),
+    dict(q=None), dict(k=None), dict(v=None), dict(log_alpha=None), dict(beta=None),
+    dict(d=None), dict(out=None),
+    dict(q=BASE + 8), dict(out=BASE + 7 * GB + 2), dict(S0=BASE + 6 * GB + 4),
+    dict(log_alpha=BASE + 3 * GB + 2),
+    dict(out=BASE + 16),                  # out overlaps q
+    dict(S_final=BASE + 2 * GB + 64),     # S_final overlaps v
+    dict(S_final=BASE + 6 * GB + 16),     # partial overlap with S0
+    dict(S_final=BASE + 7 * GB + 256),    # S_final overlaps out
+])
+@pytest.mark.parametrize("f32", [False, True])
+def test_chunk_rejects_bad_arguments(lib, bad, f32):
+    assert _call_chunk(lib, _chunk_args(**bad), f32) == -1
+
+
+@pytest.mark.parametrize("empty", [dict(B=0), dict(H=0)])
+def test_chunk_empty_batch_is_noop(lib, empty):
+    # Nothing to compute and nothing enqueued: succeeds without a device.
+    assert _call_chunk(lib, _chunk_args(**empty, q=None, k=None, v=None)) == 0
+
+
+def _step_args(**kw):
+    a = dict(q=BASE, k=BASE + GB, v=BASE + 2 * GB, log_alpha=BASE + 3 * GB, beta=BASE + 4 * GB,
+             d=BASE + 5 * GB, S=BASE + 6 * GB, out=BASE + 7 * GB, B=4, H=2, dk=128, dv=128)
+    a.update(kw)
+    return a
+
+
+def _call_step(lib, a):
+    p = lambda x: ctypes.c_void_p(x)
+    return lib.comba_recurrent_step(p(a["q"]), p(a["k"]), p(a["v"]), p(a["log_alpha"]),
+                                    p(a["beta"]), p(a["d"]), p(a["S"]), p(a["out"]), a["B"],
+                                    a["H"], a["dk"], a["dv"], ctypes.c_void_p(None))
+
+
+@pytest.mark.parametrize("bad", [
+    dict(dk=16), dict(dk=96), dict(dv=8), dict(dv=200), dict(B=-1), dict(H=-1),
+    dict(S=None), dict(out=None), dict(q=None), dict(S=BASE + 6 * GB + 8),
+    dict(out=BASE + 6 * GB + 64),         # out inside S
+    dict(S=BASE + 512),                   # S overlaps q
+])
+def test_step_rejects_bad_arguments(lib, bad):
+    assert _call_step(lib, _step_args(**bad)) == -1
+
+
+def test_step_empty_is_noop(lib):
+    assert _call_step(lib, _step_args(B=0)) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 1, 16)
+    g = torch.zeros(1, 4, 1)
+    with pytest.raises(ValueError):
+        cdr.chunk_fwd(x, x, x, g, g, torch.zeros(1))
