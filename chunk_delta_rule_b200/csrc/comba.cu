@@ -200,3 +200,14 @@ extern "C" const char* comba_status_string(int status) {
 }
 
 extern "C" int comba_version(void) { return 100; }
+
+#ifdef COMBA_TRACE_PHASES
+// Tracing builds only: copies and clears the per-phase cycle counters.
+extern "C" int comba_trace_read_phases(unsigned long long* host16) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;
+    if (cudaMemcpyFromSymbol(host16, comba::g_phase_cycles, 16 * sizeof(unsigned long long)) != cudaSuccess)
+        return COMBA_ECUDA;
+    static const unsigned long long zeros[16] = {};
+    return cudaMemcpyToSymbol(comba::g_phase_cycles, zeros, sizeof(zeros)) == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
+}
+#endif

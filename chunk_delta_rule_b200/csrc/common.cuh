@@ -13,6 +13,25 @@ __device__ int g_status = 0;
 
 __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0, code); }
 
+// Optional phase tracing (compile with -DCOMBA_TRACE_PHASES): thread 0 of CTA 0
+// accumulates clock64() deltas between consecutive COMBA_PHASE marks.  Off by
+// default; the marks then compile to nothing.
+#ifdef COMBA_TRACE_PHASES
+__device__ unsigned long long g_phase_cycles[16];
+#define COMBA_PHASE_BEGIN() long long comba_phase_t = clock64()
+#define COMBA_PHASE(i)                                                              \
+    do {                                                                            \
+        if (blockIdx.x == 0 && threadIdx.x == 0) {                                  \
+            const long long comba_phase_now = clock64();                            \
+            g_phase_cycles[(i)] += (unsigned long long)(comba_phase_now - comba_phase_t); \
+            comba_phase_t = comba_phase_now;                                        \
+        }                                                                           \
+    } while (0)
+#else
+#define COMBA_PHASE_BEGIN() do {} while (0)
+#define COMBA_PHASE(i) do {} while (0)
+#endif
+
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 

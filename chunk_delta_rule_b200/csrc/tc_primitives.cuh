@@ -46,6 +46,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
          | ((uint32_t)(M >> 4) << 24);
 }
 
+// Instruction descriptor for kind::tf32 (fp32 storage, tf32 products, fp32
+// accumulation).  An A operand taken from TMEM is always K-major.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4)                         // D format: f32
+         | (2u << 7)                         // A format: tf32
+         | (2u << 10)                        // B format: tf32
+         | ((a_mn ? 1u : 0u) << 15)
+         | ((b_mn ? 1u : 0u) << 16)
+         | ((uint32_t)(N >> 3) << 17)
+         | ((uint32_t)(M >> 4) << 24);
+}
+
 // ---------------------------------------------------------------- mbarriers
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
@@ -123,6 +135,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
         "}\n"
         ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, tf32 (A: lane = row, one fp32 per column)
+__device__ __forceinline__ void mma_tf32_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "setp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n"
+        "}\n"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
 // Arrives on `bar` once all previously issued MMAs of this thread complete.
@@ -253,6 +277,38 @@ __device__ __forceinline__ void mma_ak_bmn(uint32_t d, uint32_t a, uint32_t a_at
         const uint64_t bd = sdesc_sw128(b + (ks % kwrap) * 2048, b_lbo, 1024);
         mma_bf16(d, ad, bd, idesc, (ks > 0) ? 1u : acc0);
     }
+}
+
+// tf32, A from TMEM (K = 8 columns per MMA), B K-major fp32 (N rows; 32-element
+// K atoms `b_atom` bytes apart).
+__device__ __forceinline__ void mma_tf32_ta_bk(uint32_t d, uint32_t a_tmem, uint32_t b,
+                                               uint32_t b_atom, uint32_t idesc, int ksteps,
+                                               uint32_t acc0) {
+    for (int ks = 0; ks < ksteps; ++ks) {
+        const uint64_t bd = sdesc_sw128(b + (ks >> 2) * b_atom + (ks & 3) * 32, 16, 1024);
+        mma_tf32_ta(d, a_tmem + ks * 8, bd, idesc, (ks > 0) ? 1u : acc0);
+    }
+}
+
+// ---------------------------------------------------------------- warp MMA (legacy)
+__device__ __forceinline__ uint32_t f32_to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// d[16x8] += a[16x8] * b[8x8], tf32 inputs, fp32 accumulation, one warp.
+__device__ __forceinline__ void mma_sync_tf32(float (&d)[4], const uint32_t (&a)[4],
+                                              const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ void named_barrier(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ---------------------------------------------------------------- swizzle

@@ -38,6 +38,20 @@ __global__ void umma_check_kernel(int mode, const float* A, const float* B, cons
     int M = 128, N = 64, K = 128;
     if (mode == 1 || mode == 2) K = 64;
     if (mode == 4) N = 128;
+    if (mode == 6 || mode == 7) {
+        // tf32 with A in TMEM (fp32, lane = row, column = k); B fp32 in smem:
+        // 6: K-major, N = 64, K = 64 in two 32-element atoms 8 KB apart
+        // 7: K-major, N = 128, K = 64 in two 32-element atoms 16 KB apart
+        K = 64;
+        N = (mode == 7) ? 128 : 64;
+        for (int e = tid; e < N * K; e += blockDim.x) {
+            const int n = e / K, k = e % K;
+            uint32_t off;
+            if (mode == 6) off = (k >> 5) * 8192 + sw128(n, (k & 31) >> 2) + (k & 3) * 4;
+            else off = (k >> 5) * 16384 + sw128(n, (k & 31) >> 2) + (k & 3) * 4;
+            *reinterpret_cast<float*>(sbt + off) = B[e];
+        }
+    } else {
     for (int e = tid; e < M * K; e += blockDim.x) {
         const int m = e / K, k = e % K;
         uint32_t off;
@@ -55,14 +69,24 @@ __global__ void umma_check_kernel(int mode, const float* A, const float* B, cons
         else off = kmaj(n, k, 16384);
         *reinterpret_cast<__nv_bfloat16*>(sbt + off) = __float2bfloat16_rn(B[n * K + k]);
     }
+    }
     if (tid == 0) { mbar_init(&bar, 1); fence_mbar_init(); }
-    if (warp == 0) tmem_alloc(&tslot, 128);
+    if (warp == 0) tmem_alloc(&tslot, 256);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tslot;
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    if (mode == 6 || mode == 7) {   // A (fp32) into TMEM columns 128..191
+        for (int part = 0; part < 2; ++part) {
+            float v[32];
+            for (int e = 0; e < 32; ++e) v[e] = A[tid * K + part * 32 + e];
+            tmem_st32(trow + 128 + part * 32, v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+    }
     if (mode == 5) {
         for (int part = 0; part < N / 32; ++part) {
             float v[32];
@@ -83,6 +107,8 @@ __global__ void umma_check_kernel(int mode, const float* A, const float* B, cons
             case 3: mma_ak_bmn(tmem, a, 16384, b, 8192, idesc_bf16(128, 64, false, true), 8, 8, 0); break;
             case 4: mma_ak_bmn(tmem, a, 16384, b, 16384, idesc_bf16(128, 128, false, true), 8, 4, 0); break;
             case 5: mma_ak_bk(tmem, a, 16384, b, 0, idesc_bf16(128, 64, false, false), 8, 1); break;
+            case 6: mma_tf32_ta_bk(tmem, tmem + 128, b, 8192, idesc_tf32(128, 64, false, false), 8, 0); break;
+            case 7: mma_tf32_ta_bk(tmem, tmem + 128, b, 16384, idesc_tf32(128, 128, false, false), 8, 0); break;
         }
         mma_commit(&bar);
     }
@@ -99,7 +125,7 @@ __global__ void umma_check_kernel(int mode, const float* A, const float* B, cons
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 128);
+    if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 }  // namespace

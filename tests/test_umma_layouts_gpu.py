@@ -34,6 +34,8 @@ def lib(tmp_path_factory):
     (3, 128, 64, 128, False),   # S W^T      (B MN-major)
     (4, 128, 128, 128, True),   # (D X)^T K  (B MN-major, K rows re-read for hi|lo)
     (5, 128, 64, 128, True),    # X^T P^T accumulated onto an initial D
+    (6, 128, 64, 64, False),    # tf32: X (TMEM) P^T, P K-major fp32
+    (7, 128, 128, 64, False),   # tf32: X (TMEM) (D K), (D K)^T K-major fp32, N = 128
 ])
 def test_mma_layout(lib, mode, M, N, K, wrapB):
     g = torch.Generator().manual_seed(mode)
@@ -48,9 +50,15 @@ def test_mma_layout(lib, mode, M, N, K, wrapB):
     rc = lib.umma_layout_check(mode, Ad.data_ptr(), Bd.data_ptr(), D0d.data_ptr(), D.data_ptr(),
                                status.data_ptr())
     assert rc == 0 and int(status.item()) == 0
-    Ab = A.bfloat16().double()
-    Bb = B.bfloat16().double()
-    want = Ab @ Bb.T + (D0.double() if mode == 5 else 0)
+    if mode in (6, 7):
+        # tf32 keeps 10 explicit mantissa bits of each operand
+        want = A.double() @ B.double().T
+        tol = 2e-3 * (A.abs() @ B.abs().T).double().max().item()
+    else:
+        Ab = A.bfloat16().double()
+        Bb = B.bfloat16().double()
+        want = Ab @ Bb.T + (D0.double() if mode == 5 else 0)
+        tol = 1e-3 * max(1.0, want.abs().max().item())
     got = D.double().cpu()
     err = (got - want).abs().max().item()
-    assert err < 1e-3 * max(1.0, want.abs().max().item()), f"mode {mode}: max err {err}"
+    assert err < tol, f"mode {mode}: max err {err}"
