@@ -93,33 +93,48 @@ def profiled_traffic(workload: str):
 
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi during a region."""
+    """Samples SM clocks and throttle reasons with nvidia-smi.  Started before
+    the timed region; ``summary(t0, t1)`` keeps the samples taken between the
+    host times t0 and t1 (at least the first one after t0)."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, interval_ms: int = 50):
         self.gpu = gpu_index
+        self.interval = interval_ms
         self.proc = None
-        self.lines = []
+        self.samples = []   # (host time, fields)
 
-    def __enter__(self):
+    def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.interval)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            t_end = time.time() + 5.0
+            while not self.samples and time.time() < t_end and self.proc.poll() is None:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
 
-    def __exit__(self, *exc):
+    def wait_after(self, t: float, timeout: float = 2.0):
+        t_end = time.time() + timeout
+        while self.proc is not None and time.time() < t_end:
+            if any(ts >= t for ts, _ in self.samples):
+                return
+            time.sleep(0.01)
+
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -128,13 +143,14 @@ class ClockSampler:
                 self.proc.kill()
             self.thread.join(timeout=2)
 
-    def summary(self):
-        sm, mx, reasons = [], None, set()
+    def summary(self, t0: float, t1: float):
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
+        inside = [p for ts, p in self.samples if t0 <= ts <= t1]
+        if not inside:
+            after = [p for ts, p in self.samples if ts >= t0]
+            inside = after[:1]
+        sm, mx, reasons = [], None, set()
+        for parts in inside:
             try:
                 sm.append(float(parts[1]))
                 mx = float(parts[2])
@@ -148,6 +164,12 @@ class ClockSampler:
         sm.sort()
         return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def weak_scaling_value(tokens_per_rank: int, world: int, ms_per_step_max: float) -> float:
+    """Whole-job throughput: every rank processes its own batch; time is the
+    slowest rank's."""
+    return world * tokens_per_rank / (ms_per_step_max / 1e3)
 
 
 def dist_setup(n_gpus: int):
@@ -170,6 +192,7 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's time (all ranks must call)."""
     if world == 1:
         return x
     import torch.distributed as dist
@@ -178,11 +201,16 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
-def cpu_baseline(cfg, x, target_s: float = 15.0):
+def rank_seed(cfg, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling over independent chains)."""
+    return cfg.seed + 1000 * rank
+
+
+def cpu_baseline(cfg, x, target_s: float = 10.0):
     """Times the float64 oracle (as it stands) on the host cores on a bounded
-    sample of the workload's chains; returns the baseline record."""
+    sample of the workload's (b, h) chains -- the whole workload, repeated,
+    when it takes less than ``target_s`` -- and returns the baseline record."""
     import oracle
-    import numpy as np
     threads = oracle.num_threads()
     B, H = cfg.B, cfg.H
 
@@ -203,13 +231,18 @@ def cpu_baseline(cfg, x, target_s: float = 15.0):
 
     probe = run([0])
     n = max(1, min(B * H, int(target_s / max(probe, 1e-6)) * threads))
-    n = min(n, B * H)
     chains = list(range(n))
-    el = run(chains)
-    tokens = n * cfg.T / H  # a token carries all H heads
+    el, reps = 0.0, 0
+    while True:
+        el += run(chains)
+        reps += 1
+        if el >= target_s or n < B * H:
+            break
+    tokens = reps * n * cfg.T / H  # a token carries all H heads
     return {"value": tokens / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n} of {B * H} (b,h) chains x {cfg.T} tokens of {cfg.name}, float64 C "
-                      f"recurrence, OpenMP over chains; {el:.1f} s",
+            "sample": f"{n} of {B * H} (b,h) chains x {cfg.T} tokens of {cfg.name}"
+                      f"{'' if reps == 1 else f', {reps} passes'}; float64 C recurrence, OpenMP "
+                      f"over chains; {el:.1f} s",
             "seconds": el}
 
 
@@ -219,9 +252,9 @@ def run_reference(args, cfg):
     if rank != 0:
         return
     x = make_chunk_inputs(cfg)
-    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    per_step = max(1.0, min(10.0, 60.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        cpu_baseline(cfg, x, target_s=per_step / 4)
+        cpu_baseline(cfg, x, target_s=0.2)
     vals, secs, rec = [], 0.0, None
     for _ in range(args.steps):
         rec = cpu_baseline(cfg, x, target_s=per_step)
@@ -253,8 +286,8 @@ def config_record(cfg):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="layer1p3b_bf16", choices=sorted(CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -273,7 +306,7 @@ def main():
     cdr.library()  # fails loudly if the CUDA library is missing
 
     # Weak scaling: every rank owns a full batch of independent chains.
-    x = make_chunk_inputs(cfg, seed=cfg.seed + 1000 * rank)
+    x = make_chunk_inputs(cfg, seed=rank_seed(cfg, rank))
     names = ("q", "k", "v", "log_alpha", "beta", "d", "S0")
     host = {k: x[k].pin_memory() for k in names if x[k] is not None}
     dv_ = {k: host[k].to(dev, non_blocking=True) for k in host}
@@ -293,20 +326,24 @@ def main():
 
     # ---- device-timed region: inputs resident in HBM -------------------------------
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local).start()
     barrier(world)
     torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clocks:
-        ev0.record(stream)
-        for _ in range(args.steps):
-            step()
-        ev1.record(stream)
-        torch.cuda.synchronize(dev)
+    th0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    th1 = time.time()
+    clocks.wait_after(th0)
+    clocks.stop()
     barrier(world)
     ms = ev0.elapsed_time(ev1)
     ms = max_over_ranks(ms, world, dev)
     ms_step = ms / args.steps
     tokens_all = world * cfg.B * cfg.T
-    value = tokens_all / (ms_step / 1e3)
+    value = weak_scaling_value(cfg.B * cfg.T, world, ms_step)
     if cdr.get_last_error(dev) != 0:
         raise RuntimeError("device-side error during the timed region")
 
@@ -359,7 +396,7 @@ def main():
                      "tensor_frac_of_bf16_peak": tflops / peaks["bf16_tflops"]},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
-        "clocks": clocks.summary(),
+        "clocks": clocks.summary(th0, th1),
         "gpu_launches": args.steps,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

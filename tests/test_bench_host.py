@@ -1,0 +1,81 @@
+"""Host logic of bench.py on CPU: the multi-rank path (gloo, world size 2), the
+weak-scaling arithmetic, the roofline counts and the CPU reference arm."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from comba_workloads import CONFIGS, make_chunk_inputs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # rank r reports a step time of 1 + r ms: every rank must see the max
+        t = bench.max_over_ranks(1.0 + rank, world, "cpu")
+        cfg = CONFIGS["tiny_fp32"]
+        x = make_chunk_inputs(cfg, seed=bench.rank_seed(cfg, rank))
+        digest = float(x["q"].double().sum())
+        gathered = [None] * world
+        dist.all_gather_object(gathered, digest)
+        q.put((rank, t, gathered))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_max_time_and_distinct_batches():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + (os.getpid() % 1000)
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, t, gathered in res:
+        assert t == 2.0                    # max over ranks, on every rank
+        assert gathered[0] != gathered[1]  # each rank owns its own batch
+
+
+def test_weak_scaling_value():
+    assert bench.weak_scaling_value(32768, 1, 1.0) == pytest.approx(32768e3)
+    assert bench.weak_scaling_value(32768, 8, 2.0) == pytest.approx(8 * 32768 / 2e-3)
+
+
+def test_algorithmic_counts_headline_shape():
+    flops, bytes_ = bench.algorithmic_counts(CONFIGS["layer1p3b_bf16"])
+    ht = 8 * 4096 * 16
+    assert flops == ht * 139264
+    assert bytes_ == ht * 1032 + 8 * 16 * 128 * 128 * 4 * 2
+
+
+def test_reference_arm_prints_one_line():
+    env = dict(os.environ, PYTHONPATH=ROOT)
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny_fp32", "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, env=env, timeout=600, check=True)
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["value"] > 0 and j["unit"] == "tokens/s"
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    env = dict(os.environ, PYTHONPATH=ROOT, RANK="1", WORLD_SIZE="2")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny_fp32", "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, env=env, timeout=600, check=True)
+    assert out.stdout.strip() == ""
