@@ -33,7 +33,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from comba_workloads import CONFIGS, make_chunk_inputs  # noqa: E402
+from comba_workloads import (CONFIGS, DECODE, decode_step_inputs, make_chunk_inputs,  # noqa: E402
+                             make_decode_state)
 
 METRIC = "Comba chunk-fwd tokens/s and TFLOP/s on 1 B200, % of roofline"
 L2_BYTES = 126 * 2 ** 20
@@ -283,17 +284,112 @@ def config_record(cfg):
                   % (cfg.B * cfg.T * cfg.H * (2 * cfg.dk + 2 * cfg.dv) * (2 if cfg.dtype == "bf16" else 4) / 2 ** 20)}
 
 
+def decode_counts(cfg):
+    """Algorithmic bytes and FLOPs of one decode step over all (b, h): the fp32
+    state read and written once, q, k, v, out in bf16, two fp32 gates."""
+    heads = cfg.B * cfg.H
+    bytes_ = heads * (2 * cfg.dv * cfg.dk * 4 + (2 * cfg.dk + 2 * cfg.dv) * 2 + 8)
+    flops = heads * 8 * cfg.dv * cfg.dk
+    return flops, bytes_
+
+
+def run_decode(args):
+    """One step = one comba_recurrent_step for every (b, h) of the decode
+    workload, state resident in HBM (537 MB, larger than L2)."""
+    import chunk_delta_rule_b200 as cdr
+    cfg = DECODE
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cdr.library()
+    st = make_decode_state(cfg)
+    d = st["d"].to(dev)
+    S = st["S"].to(dev)
+    n_in = 8   # distinct tokens, cycled
+    host = [decode_step_inputs(st["gen"], st["decay_scale"], cfg) for _ in range(n_in)]
+    host = [{k: v.pin_memory() for k, v in x.items()} for x in host]
+    dev_in = [{k: v.to(dev) for k, v in x.items()} for x in host]
+    out = torch.empty((cfg.B, cfg.H, cfg.dv), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        x = dev_in[i % n_in]
+        cdr.recurrent_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], d, S, out=out,
+                           stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(0).start()
+    th0 = time.time()
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    th1 = time.time()
+    clocks.wait_after(th0)
+    clocks.stop()
+    ms_step = ev0.elapsed_time(ev1) / args.steps
+    # end to end: this step's token inputs from pinned host memory, out back to host
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    stage = {k: torch.empty_like(v) for k, v in dev_in[0].items()}
+
+    def e2e_step(i):
+        for k, v in host[i % n_in].items():
+            stage[k].copy_(v, non_blocking=True)
+        cdr.recurrent_step(stage["q"], stage["k"], stage["v"], stage["log_alpha"], stage["beta"],
+                           d, S, out=out, stream=stream)
+        out_h.copy_(out, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_e2e = ev0.elapsed_time(ev1) / args.steps
+    flops, bytes_ = decode_counts(cfg)
+    peaks = load_peaks()
+    gbs = bytes_ / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": "Comba decode-step tokens/s (one token per batch row, all heads), % of HBM roofline",
+        "value": cfg.B / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "dk": cfg.dk, "dv": cfg.dv,
+                   "l2": "state 537 MB larger than L2; no flush"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "algorithmic_bytes_per_launch": bytes_},
+        "e2e": {"value": cfg.B / (ms_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in host[0].values()),
+                "d2h_bytes_per_step": out_h.numel() * 2, "ms_per_step": ms_e2e},
+        "clocks": clocks.summary(th0, th1),
+        "gpu_launches": args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="layer1p3b_bf16", choices=sorted(CONFIGS))
+    ap.add_argument("--workload", default="layer1p3b_bf16", choices=sorted(CONFIGS) + [DECODE.name])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload == DECODE.name:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the decode workload has no reference arm; the headline workload does"}))
+            return
+        run_decode(args)
+        return
     cfg = CONFIGS[args.workload]
     if args.impl == "reference":
         run_reference(args, cfg)

@@ -7,23 +7,28 @@
 // inverse for the intermediates W and U, section "硬件高效的分块并行计算"):
 //
 //   1. gates (prefetched one chunk ahead): g by warp-shuffle scan, e^{g_r},
-//      e^{g_L - g_r}, c_r = beta_r e^{g_{r-1}}
-//   2. Gram MMA      G = [K; Q] K^T                                  (bf16 -> TMEM)
-//   3. P_rs = e^{g_r-g_s}(Q K^T - d K K^T)_rs (s <= r) as an fp32 operand;
-//      A_rs = beta_r e^{g_{r-1}-g_s}(K K^T)_rs (s < r)
-//   4. Tinv = (I + A)^{-1}: 16 x 16 diagonal blocks by forward substitution,
-//      off-diagonal blocks by distance with warp-level tf32 MMAs
-//   5. Tc = Tinv diag(c), Eb = (Tinv - I) diag(beta) (bf16); Qh = diag(e^g)(Q - d K)
-//      over Q; (D K)^T with D = diag(e^{g_L - g}) (fp32 operand, K-major)
-//   6. X^T <- beta V^T (TMEM store); MMAs W^T = K^T Tc^T, X^T += V^T Eb^T
+//      e^{-g_r}, e^{g_L - g_r}, c_r = beta_r e^{g_{r-1}}
+//   2. Gram MMA G = [K; Q] K^T (bf16 -> TMEM), issued during the previous chunk
+//   3. K K^T staged in the P operand; A_rs = beta_r e^{g_{r-1}-g_s}(K K^T)_rs (s < r);
+//      then, concurrently: P_rs = e^{g_r-g_s}(Q K^T - d K K^T)_rs (s <= r) in
+//      place (fp32 operand), Qh = diag(e^g)(Q - d K) over Q and (D K)^T with
+//      D = diag(e^{g_L - g}) (fp32, K-major) on half the warps; the 16 x 16
+//      diagonal blocks of Tinv = (I + A)^{-1} by substitution on the others
+//   4. off-diagonal blocks of Tinv by distance, warp-level tf32 MMAs per 8-column slab
+//   5. Tc = Tinv diag(c); Eb = (Tinv - I) diag(beta) + diag(hi(beta)) (bf16),
+//      diag(lo(beta)) (bf16), so that beta = hi + lo to 16 bits
+//   6. MMAs W^T = K^T Tc^T,  X^T = V^T Eb^T + V^T diag(lo)^T  (= U~^T)
 //   7. -W^T -> bf16 operand
 //   8. MMAs X^T += S (-W)^T, O^T = S Qh^T (bf16, S from its bf16 copy);
 //      then, reading X^T straight from TMEM as a tf32 operand,
-//      S += X^T (D K) and O^T += X^T P^T
+//      S += X^T (D K) and O^T += X^T P^T; then the next chunk's Gram MMA
 //   9. S -> bf16 operand, S master *= e^{g_L} of the next chunk; O^T -> TMA store
 //
-// The leading beta V term of U~ = beta V + (Tinv - I) beta V and the state
-// master stay fp32 throughout.  A ragged last chunk is zero-filled by TMA and
+// The leading beta V term of U~ = beta V + (Tinv - I) beta V is carried to
+// 16 bits (hi + lo bf16 diagonals against the exact bf16 V), and the state
+// master stays fp32 throughout.  Within a chunk e^{g_r - g_s} is formed as
+// e^{g_r} e^{-g_s} when the chunk's total log-decay is above -80 (both factors
+// stay normal fp32 numbers); otherwise each entry takes exp2 of the difference.  A ragged last chunk is zero-filled by TMA and
 // its gates padded with log_alpha = 0, beta = 0, which leaves the state and
 // the valid outputs exact.
 #pragma once
@@ -51,11 +56,12 @@ constexpr uint32_t SM_KQ1 = 32768;    // stage 1
 constexpr uint32_t SM_V = 65536;      // V: 2 dv-atoms x 64 tokens x 128 B
 constexpr uint32_t SM_S = 81920;      // S bf16: 2 K-atoms x 128 rows
 constexpr uint32_t SM_W = 114688;     // -W bf16, MN-major: 128 rows (j) x 64 tokens
-constexpr uint32_t SM_P = 131072;     // P fp32, K-major: 2 atoms (32 s) x 64 rows
+constexpr uint32_t SM_P = 131072;     // P fp32, K-major: 2 atoms (32 s) x 64 rows (K K^T first)
 constexpr uint32_t SM_DK = 147456;    // (D K)^T fp32, K-major: 2 atoms (32 r) x 128 rows (j); out staging
-constexpr uint32_t SM_F1 = 180224;    // fp32 64x64: K K^T, then A; then Tc (bf16) | Eb (bf16)
+constexpr uint32_t SM_F1 = 180224;    // fp32 64x64: A; then Tc (bf16) | Eb (bf16)
 constexpr uint32_t SM_F2 = 196608;    // fp32 64x64: Tinv (upper blocks: scratch)
-constexpr uint32_t SM_MISC = 212992;  // gates, barriers
+constexpr uint32_t SM_BLO = 212992;   // bf16 64x64 K-major: diag(lo(beta)), zero elsewhere
+constexpr uint32_t SM_MISC = 221184;  // gates, barriers
 constexpr uint32_t SM_END = SM_MISC + 2048;
 constexpr uint32_t kSmemBytes = SM_END + 1024;
 
@@ -77,85 +83,113 @@ constexpr float kLog2e = 1.4426950408889634f;
 // fp32 64 x 64 scratch with an XOR swizzle on the column.
 __device__ __forceinline__ int fidx(int r, int s) { return r * 64 + (s ^ (r & 31)); }
 
-// C[16 x 16] += A-block(FA at ra, ca) * B-block(FB at rb, cb), one warp, tf32.
-__device__ __forceinline__ void blk_mma(float (&c)[2][4], const float* FA, int ra, int ca,
-                                        const float* FB, int rb, int cb, int lane) {
+// c[16 x 8] += A-block(FA at ra, ca: 16 x 16) * B-slab(FB at rb, cb: 16 x 8), one warp, tf32.
+__device__ __forceinline__ void slab_mma(float (&c)[4], const float* FA, int ra, int ca,
+                                         const float* FB, int rb, int cb, int lane) {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int kk = 0; kk < 2; ++kk) {
-        uint32_t a[4];
+        uint32_t a[4], bb[2];
         a[0] = tc::f32_to_tf32(FA[fidx(ra + g, ca + 8 * kk + t)]);
         a[1] = tc::f32_to_tf32(FA[fidx(ra + g + 8, ca + 8 * kk + t)]);
         a[2] = tc::f32_to_tf32(FA[fidx(ra + g, ca + 8 * kk + t + 4)]);
         a[3] = tc::f32_to_tf32(FA[fidx(ra + g + 8, ca + 8 * kk + t + 4)]);
-#pragma unroll
-        for (int nn = 0; nn < 2; ++nn) {
-            uint32_t b[2];
-            b[0] = tc::f32_to_tf32(FB[fidx(rb + 8 * kk + t, cb + 8 * nn + g)]);
-            b[1] = tc::f32_to_tf32(FB[fidx(rb + 8 * kk + t + 4, cb + 8 * nn + g)]);
-            tc::mma_sync_tf32(c[nn], a, b);
-        }
+        bb[0] = tc::f32_to_tf32(FB[fidx(rb + 8 * kk + t, cb + g)]);
+        bb[1] = tc::f32_to_tf32(FB[fidx(rb + 8 * kk + t + 4, cb + g)]);
+        tc::mma_sync_tf32(c, a, bb);
     }
 }
 
-__device__ __forceinline__ void blk_store(float* F, int r0, int c0, const float (&c)[2][4],
-                                          float scale, int lane) {
+__device__ __forceinline__ void slab_store(float* F, int r0, int c0, const float (&c)[4],
+                                           float scale, int lane) {
     const int g = lane >> 2, t = lane & 3;
+    F[fidx(r0 + g, c0 + 2 * t)] = scale * c[0];
+    F[fidx(r0 + g, c0 + 2 * t + 1)] = scale * c[1];
+    F[fidx(r0 + g + 8, c0 + 2 * t)] = scale * c[2];
+    F[fidx(r0 + g + 8, c0 + 2 * t + 1)] = scale * c[3];
+}
+
+// Diagonal 16 x 16 block `blk` of (I + A)^{-1} (A strictly lower, fp32 in F1)
+// into F2: one warp, lane j < 16 owns column j, right-looking substitution.
+// Inside block `blk`, fidx(16 blk + r, 16 blk + s) = (16 blk + r) 64 + 32 (blk >> 1)
+// + (s ^ r), so every A offset below is a compile-time constant.
+__device__ __forceinline__ void diag_block_inverse(const float* __restrict__ F1, float* F2,
+                                                   int blk, int lane) {
+    const int o = 16 * blk;
+    const int base = o * 64 + 32 * (blk >> 1);
+    const float* Ab = F1 + base;
+    const int j = lane & 15;
+    float x[16];
 #pragma unroll
-    for (int nn = 0; nn < 2; ++nn) {
-        F[fidx(r0 + g, c0 + 8 * nn + 2 * t)] = scale * c[nn][0];
-        F[fidx(r0 + g, c0 + 8 * nn + 2 * t + 1)] = scale * c[nn][1];
-        F[fidx(r0 + g + 8, c0 + 8 * nn + 2 * t)] = scale * c[nn][2];
-        F[fidx(r0 + g + 8, c0 + 8 * nn + 2 * t + 1)] = scale * c[nn][3];
+    for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
+#pragma unroll
+    for (int s = 0; s < 15; ++s) {
+        const float xs = x[s];
+#pragma unroll
+        for (int r = s + 1; r < 16; ++r) x[r] = fmaf(-Ab[r * 64 + (s ^ r)], xs, x[r]);
+    }
+    if (lane < 16) {
+        float* Tb = F2 + base;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tb[r * 64 + (j ^ r)] = x[r];
     }
 }
 
-// (I + A)^{-1} for strictly lower A (64 x 64 fp32 in F1) into F2 (lower triangle
-// with the unit diagonal; the upper 16 x 16 blocks of F2 are used as scratch).
-__device__ __forceinline__ void unit_lower_inverse(const float* __restrict__ F1, float* F2,
-                                                   int tid) {
+// Off-diagonal blocks of (I + A)^{-1} by distance, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj,
+// one warp per 16 x 8 slab (warp 2j + slab); M_ij is staged in the upper block (j, i).
+__device__ __forceinline__ void offdiag_inverse(const float* __restrict__ F1, float* F2,
+                                                int tid) {
     const int warp = tid >> 5, lane = tid & 31;
-    if (warp < 4) {
-        // Diagonal block `warp`, column j per lane, right-looking substitution.
-        const int o = 16 * warp;
-        const int j = lane & 15;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
-#pragma unroll
-        for (int s = 0; s < 15; ++s) {
-            const float xs = x[s];
-#pragma unroll
-            for (int r = s + 1; r < 16; ++r) x[r] = fmaf(-F1[fidx(o + r, o + s)], xs, x[r]);
-        }
-        if (lane < 16) {
-#pragma unroll
-            for (int r = 0; r < 16; ++r) F2[fidx(o + r, o + j)] = x[r];
-        }
-    }
-    __syncthreads();
-    // Off-diagonal blocks by distance: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj
-    // (warp j computes block (j + dist, j); M_ij is staged in upper block (j, i)).
 #pragma unroll
     for (int dist = 1; dist <= 3; ++dist) {
-        if (warp < 4 - dist) {
-            const int j = warp, i = warp + dist;
-            float m[2][4] = {};
-            for (int kb = j; kb < i; ++kb) blk_mma(m, F1, 16 * i, 16 * kb, F2, 16 * kb, 16 * j, lane);
-            blk_store(F2, 16 * j, 16 * i, m, 1.f, lane);
+        if (warp < 2 * (4 - dist)) {
+            const int j = warp >> 1, nt = warp & 1, i = j + dist;
+            float m[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int kb = j; kb < i; ++kb)
+                slab_mma(m, F1, 16 * i, 16 * kb, F2, 16 * kb, 16 * j + 8 * nt, lane);
+            slab_store(F2, 16 * j, 16 * i + 8 * nt, m, 1.f, lane);
             __syncwarp();
-            float r2[2][4] = {};
-            blk_mma(r2, F2, 16 * i, 16 * i, F2, 16 * j, 16 * i, lane);
-            blk_store(F2, 16 * i, 16 * j, r2, -1.f, lane);
+            float r2[4] = {0.f, 0.f, 0.f, 0.f};
+            slab_mma(r2, F2, 16 * i, 16 * i, F2, 16 * j, 16 * i + 8 * nt, lane);
+            slab_store(F2, 16 * i, 16 * j + 8 * nt, r2, -1.f, lane);
         }
         __syncthreads();
     }
 }
 
+// Exact-exponential fallbacks for a chunk whose total log-decay is at or
+// below -80 (e^{-g} would leave the normal fp32 range): each entry takes exp2
+// of its own exponent difference.  Kept out of line: they are rarely taken.
+__device__ __noinline__ void a_row_exact(float* F1, uint32_t gram_taddr, int r, int s0, float br,
+                                         float gpr, const float* g2_s) {
+    float gv[32];
+    tc::tmem_ld32(gram_taddr, gv);
+    tc::tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const int s = s0 + e;
+        F1[fidx(r, s)] = (s < r) ? br * exp2f(gpr - g2_s[s]) * gv[e] : 0.f;
+    }
+}
+
+__device__ __noinline__ void p_row_exact(uint8_t* prow, uint32_t gram_taddr, int r, int s0,
+                                         float dh, const float* g2_s) {
+    float gv[32];
+    tc::tmem_ld32(gram_taddr, gv);
+    tc::tmem_ld_wait();
+    const float gr = g2_s[r];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const int s = s0 + e;
+        float* pp = reinterpret_cast<float*>(prow + tc::sw128(r, e >> 2)) + (e & 3);
+        *pp = (s <= r) ? exp2f(gr - g2_s[s]) * fmaf(-dh, *pp, gv[e]) : 0.f;
+    }
+}
+
 // All threads wait on `bar`; a timeout is latched and makes every thread see
 // `false` after the barrier.
-__device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
-                                         volatile int* abort_flag) {
+__device__ __noinline__ bool cta_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
+                                      volatile int* abort_flag) {
     if (!tc::mbar_wait(bar, parity, timeout_ns)) {
         *abort_flag = 1;
         latch_status(-4 /* COMBA_ETIMEOUT */);
@@ -171,6 +205,18 @@ __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
     w.z = tc::pack_bf16(v[4], v[5]);
     w.w = tc::pack_bf16(v[6], v[7]);
     return w;
+}
+
+// Gram MMA of chunk n by one thread: waits for the chunk's q/k tiles, then
+// G = [K; Q] K^T into TMEM, committed to bars[5].
+__device__ __noinline__ bool issue_gram_mma(uint64_t* bars, uint32_t sb, uint32_t tmem, int n,
+                                            uint64_t timeout_ns) {
+    if (!tc::mbar_wait(&bars[n & 1], (n >> 1) & 1, timeout_ns)) return false;
+    const uint32_t kq_a = sb + ((n & 1) ? SM_KQ1 : SM_KQ0);
+    tc::tc_fence_after();
+    tc::mma_ak_bk(tmem + TM_G, kq_a, KQ_ATOM, kq_a, KQ_ATOM, ID_G, 8, 0);
+    tc::mma_commit(&bars[5]);
+    return true;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -190,9 +236,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     float* c_s = g2_s + 192;                                // beta_r e^{g_{r-1}}
     float* eg_s = g2_s + 256;                               // e^{g_r}
     float* ed_s = g2_s + 320;                               // e^{g_L - g_r}
-    float* red_s = g2_s + 384;                              // [0..1] scan carries, [2..3] sums
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 1600);  // kq0, kq1, v, mma, mma1
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
+    float* ieg_s = g2_s + 384;                              // e^{-g_r} (when the chunk allows)
+    float* red_s = g2_s + 448;                              // [0..1] scan carries, [2..3] next-chunk sums
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 1856);  // kq0, kq1, v, mma, mma1, gram
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     float* F1 = reinterpret_cast<float*>(sm + SM_F1);
     float* F2 = reinterpret_cast<float*>(sm + SM_F2);
@@ -206,7 +253,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t trow = (uint32_t)((warp & 3) * 32) << 16;
 
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i) tc::mbar_init(&bars[i], 1);
+        for (int i = 0; i < 6; ++i) tc::mbar_init(&bars[i], 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
         tc::prefetch_tmap(&tm_q);
@@ -215,6 +262,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tc::prefetch_tmap(&tm_o);
     }
     if (warp == 0) tc::tmem_alloc(tmem_slot, TM_COLS);
+    for (int i = tid; i < 8192 / 16; i += kThreads)   // diag(lo(beta)): zero off the diagonal
+        reinterpret_cast<uint4*>(sm + SM_BLO)[i] = make_uint4(0u, 0u, 0u, 0u);
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
@@ -237,33 +286,31 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tc::tma_load_4d(sm + SM_V, &tm_v, &bars[2], 0, h, t0, b);
         tc::tma_load_4d(sm + SM_V + V_ATOM, &tm_v, &bars[2], 64, h, t0, b);
     };
+    // Gram MMA of chunk n (thread 0): waits for its q/k tiles, commits to bars[5].
+    auto issue_gram = [&](int n) -> bool { return issue_gram_mma(bars, sb, tmem, n, timeout_ns); };
     auto gate = [&](const float* p, int t) -> float {
         return (t < T) ? p[((size_t)b * T + t) * H + h] : 0.f;
-    };
-    // Sum over the 64 gates held by threads 0..63 (warps 0 and 1); all threads call.
-    auto sum64 = [&](float x, int slot) -> float {
-        if (tid < 64) {
-            x = warp_sum(x);
-            if (lane == 0) red_s[2 + warp] = x;
-        }
-        __syncthreads();
-        const float r = red_s[2] + red_s[3];
-        (void)slot;
-        return r;
     };
 
     if (tid == 0) {
         load_kq(0);
         if (nchunks > 1) load_kq(1);
         load_v(0);
+        if (!issue_gram(0)) {
+            *abort_flag = 1;
+            latch_status(-4);
+        }
     }
-    // Gates of chunk 0 and, one chunk ahead, of chunk 1 (threads 0..63).
+    // Gates of chunk 0 (threads 0..63), and their total for the initial decay.
     float la_c = 0.f, bt_c = 0.f, la_n = 0.f, bt_n = 0.f;
     if (tid < 64) {
         la_c = gate(log_alpha, tid);
         bt_c = gate(beta, tid);
+        const float w = warp_sum(la_c);
+        if (lane == 0) red_s[2 + warp] = w;
     }
-    const float eL0 = __expf(sum64(la_c, 0));
+    __syncthreads();
+    const float eL0 = __expf(red_s[2] + red_s[3]);
 
     // Initial state: fp32 master (decayed for chunk 0) into TMEM, bf16 copy.
     {
@@ -293,7 +340,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tc::tc_fence_after();
 
     uint32_t mma_phase = 0, mma1_phase = 0;
-    bool ok = true;
+    bool ok = *abort_flag == 0;
     COMBA_PHASE_BEGIN();
     for (int n = 0; n < nchunks && ok; ++n) {
         const int t0 = n * kC;
@@ -315,86 +362,119 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (lane >= off) x += y;
             }
             if (lane == 31) red_s[warp] = x;
-            g2_s[tid] = x;     // inclusive within the warp for now
+            g2_s[tid] = x;
         }
         if (tid == 0) tc::bulk_wait_read0();   // previous out tile has left SM_DK
         __syncthreads();
+        const float gL = red_s[0] + red_s[1];
+        const bool fast = gL > -80.f;           // e^{-g} stays a normal fp32 number
         if (tid < 64) {
             const float g = g2_s[tid] + (tid >= 32 ? red_s[0] : 0.f);
-            const float gL = red_s[0] + red_s[1];
             const float gp = g - la_c;
             bt_s[tid] = bt_c;
             c_s[tid] = bt_c * __expf(gp);
             eg_s[tid] = __expf(g);
+            ieg_s[tid] = fast ? __expf(-g) : 0.f;
             ed_s[tid] = __expf(gL - g);
             gp2_s[tid] = gp * kLog2e;
-            __syncwarp();
             g2_s[tid] = g * kLog2e;
         }
         COMBA_PHASE(0);
 
-        // ---- 2. Gram MMA ------------------------------------------------------------
+        // ---- 2. Gram of this chunk (issued earlier) -----------------------------------
         if (!cta_wait(&bars[st], (n >> 1) & 1, timeout_ns, abort_flag)) { ok = false; break; }
-        if (tid == 0) {
-            tc::tc_fence_after();
-            tc::mma_ak_bk(tmem + TM_G, kq_a, KQ_ATOM, kq_a, KQ_ATOM, ID_G, 8, 0);
-            tc::mma_commit(&bars[3]);
-        }
-        if (!cta_wait(&bars[3], mma_phase, timeout_ns, abort_flag)) { ok = false; break; }
-        mma_phase ^= 1;
+        if (!cta_wait(&bars[5], n & 1, timeout_ns, abort_flag)) { ok = false; break; }
         tc::tc_fence_after();
         COMBA_PHASE(1);
 
-        // ---- 3. P (fp32 operand) and A ----------------------------------------------
+        // ---- 3. K K^T -> P buffer, A -> F1; then P/Qh/(DK)^T || diagonal inverse -------
         {
             float gv[32];
             tc::tmem_ld32(tl + TM_G + half * 32, gv);
             tc::tmem_ld_wait();
             const int s0 = half * 32;
             if (row < 64) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) F1[fidx(row, s0 + e)] = gv[e];
-            }
-            __syncthreads();
-            if (row >= 64) {
-                const int r = row - 64;
-                const float gr = g2_s[r];
+                const int r = row;
                 uint8_t* prow = sm + SM_P + half * F32_ATOM;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float p[4];
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<float4*>(prow + tc::sw128(r, c)) =
+                        make_float4(gv[4 * c], gv[4 * c + 1], gv[4 * c + 2], gv[4 * c + 3]);
+                if (fast) {
+                    const float cr = c_s[r];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int s = s0 + c * 4 + e;
-                        p[e] = (s <= r) ? exp2f(gr - g2_s[s]) * (gv[c * 4 + e] - dh * F1[fidx(r, s)]) : 0.f;
+                    for (int e = 0; e < 32; ++e) {
+                        const int s = s0 + e;
+                        F1[fidx(r, s)] = (s < r) ? cr * ieg_s[s] * gv[e] : 0.f;
                     }
-                    *reinterpret_cast<float4*>(prow + tc::sw128(r, c)) = make_float4(p[0], p[1], p[2], p[3]);
+                } else {
+                    a_row_exact(F1, tl + TM_G + half * 32, r, s0, bt_s[r], gp2_s[r], g2_s);
                 }
-            } else {
-                const float br = bt_s[row], gpr = gp2_s[row];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int s = s0 + e;
-                    gv[e] = (s < row) ? br * exp2f(gpr - g2_s[s]) * gv[e] : 0.f;
+                if (!last && tid < 64) {   // total log-decay of the next chunk
+                    const float w = warp_sum(la_n);
+                    if (lane == 0) red_s[2 + warp] = w;
                 }
             }
             __syncthreads();
-            if (row < 64) {
+            COMBA_PHASE(9);
+            if (row >= 64) {
+                // P in place over K K^T (row r, columns s0 .. s0 + 31)
+                const int r = row - 64;
+                uint8_t* prow = sm + SM_P + half * F32_ATOM;
+                const float er = eg_s[r];
+                if (fast) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) F1[fidx(row, s0 + e)] = gv[e];
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 kk = *reinterpret_cast<const float4*>(prow + tc::sw128(r, c));
+                        const float4 ig = *reinterpret_cast<const float4*>(ieg_s + s0 + 4 * c);
+                        const int s = s0 + 4 * c;
+                        float4 p;
+                        p.x = (s + 0 <= r) ? er * ig.x * fmaf(-dh, kk.x, gv[4 * c + 0]) : 0.f;
+                        p.y = (s + 1 <= r) ? er * ig.y * fmaf(-dh, kk.y, gv[4 * c + 1]) : 0.f;
+                        p.z = (s + 2 <= r) ? er * ig.z * fmaf(-dh, kk.z, gv[4 * c + 2]) : 0.f;
+                        p.w = (s + 3 <= r) ? er * ig.w * fmaf(-dh, kk.w, gv[4 * c + 3]) : 0.f;
+                        *reinterpret_cast<float4*>(prow + tc::sw128(r, c)) = p;
+                    }
+                } else {
+                    p_row_exact(prow, tl + TM_G + half * 32, r, s0, dh, g2_s);
+                }
+                // Qh (over Q) and (D K)^T for row r, key columns 64 half .. 64 half + 63
+                const float edr = ed_s[r];
+                uint8_t* dka = sm + SM_DK + (r >> 5) * DKT_ATOM + (r & 3) * 4;
+                const uint32_t rc = (r & 31) >> 2;
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t off = half * KQ_ATOM + tc::sw128(r, c);
+                    const uint4 kw = *reinterpret_cast<const uint4*>(kq + off);
+                    uint4 qw = *reinterpret_cast<const uint4*>(kq + 8192 + off);
+                    const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kw);
+                    __nv_bfloat162* q2 = reinterpret_cast<__nv_bfloat162*>(&qw);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 kf = __bfloat1622float2(k2[e]);
+                        const float2 qf = __bfloat1622float2(q2[e]);
+                        q2[e] = __floats2bfloat162_rn(er * fmaf(-dh, kf.x, qf.x), er * fmaf(-dh, kf.y, qf.y));
+                        const int j = 64 * half + 8 * c + 2 * e;
+                        *reinterpret_cast<float*>(dka + tc::sw128(j, rc)) = edr * kf.x;
+                        *reinterpret_cast<float*>(dka + tc::sw128(j + 1, rc)) = edr * kf.y;
+                    }
+                    *reinterpret_cast<uint4*>(kq + 8192 + off) = qw;
+                }
+            } else {
+                // warps 0, 1, 4, 5 -> diagonal blocks 0, 1, 2, 3
+                diag_block_inverse(F1, F2, (warp & 1) + 2 * half, lane);
             }
             __syncthreads();
         }
         COMBA_PHASE(2);
 
-        // ---- 4. inverse -------------------------------------------------------------------
-        unit_lower_inverse(F1, F2, tid);
+        // ---- 4. off-diagonal blocks of the inverse -----------------------------------
+        offdiag_inverse(F1, F2, tid);
         COMBA_PHASE(3);
 
-        // ---- 5. Tc, Eb (bf16, over F1), Qh (over Q), D K (fp32) ----------------------------
+        // ---- 5. Tc, Eb (+ diag hi(beta)) over F1; diag lo(beta) ---------------------------
         {
             const int r = tid & 63, qq = tid >> 6;   // row, quarter of the columns
-            // Tc, Eb: columns 16 qq .. 16 qq + 15 -> chunks 2 qq, 2 qq + 1
 #pragma unroll
             for (int c2 = 0; c2 < 2; ++c2) {
                 const int c = 2 * qq + c2;
@@ -404,65 +484,27 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const int s = c * 8 + e;
                     const float t = (s <= r) ? F2[fidx(r, s)] : 0.f;
                     tcv[e] = t * c_s[s];
-                    ebv[e] = (s < r) ? t * bt_s[s] : 0.f;
+                    ebv[e] = (s < r) ? t * bt_s[s] : ((s == r) ? bt_s[s] : 0.f);
                 }
                 *reinterpret_cast<uint4*>(sm + SM_F1 + tc::sw128(r, c)) = pack8_bf16(tcv);
                 *reinterpret_cast<uint4*>(sm + SM_F1 + 8192 + tc::sw128(r, c)) = pack8_bf16(ebv);
             }
-            // Qh and D K for key columns 32 qq .. 32 qq + 31 (K atom qq / 2, chunks 4 (qq % 2) ..)
-            const float er = eg_s[r], edr = ed_s[r];
-            const uint32_t atom = (qq >> 1) * KQ_ATOM;
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                const int c = (qq & 1) * 4 + c4;
-                const uint32_t off = atom + tc::sw128(r, c);
-                const uint4 kw = *reinterpret_cast<const uint4*>(kq + off);
-                uint4 qw = *reinterpret_cast<const uint4*>(kq + 8192 + off);
-                const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kw);
-                __nv_bfloat162* q2 = reinterpret_cast<__nv_bfloat162*>(&qw);
-                float dk[8];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 kf = __bfloat1622float2(k2[e]);
-                    const float2 qf = __bfloat1622float2(q2[e]);
-                    q2[e] = __floats2bfloat162_rn(er * (qf.x - dh * kf.x), er * (qf.y - dh * kf.y));
-                    dk[2 * e] = edr * kf.x;
-                    dk[2 * e + 1] = edr * kf.y;
-                }
-                *reinterpret_cast<uint4*>(kq + 8192 + off) = qw;
-                // (D K)^T, K-major fp32: row j = 32 qq + 8 c4 + e, token r in atom r / 32
-                uint8_t* dka = sm + SM_DK + (r >> 5) * DKT_ATOM + (r & 3) * 4;
-                const uint32_t rc = (r & 31) >> 2;
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    *reinterpret_cast<float*>(dka + tc::sw128(32 * qq + 8 * c4 + e, rc)) = dk[e];
+            if (tid < 64) {
+                const float bh = __bfloat162float(__float2bfloat16_rn(bt_s[tid]));
+                *reinterpret_cast<__nv_bfloat16*>(sm + SM_BLO + tc::sw128(tid, tid >> 3) + (tid & 7) * 2) =
+                    __float2bfloat16_rn(bt_s[tid] - bh);
             }
         }
         tc::fence_proxy_async_smem();
         COMBA_PHASE(4);
 
-        // ---- 6. X^T <- beta V^T; W^T = K^T Tc^T; X^T += V^T Eb^T ---------------------------
+        // ---- 6. W^T = K^T Tc^T;  X^T = V^T Eb^T + V^T diag(lo)^T ---------------------------
         if (!cta_wait(&bars[2], n & 1, timeout_ns, abort_flag)) { ok = false; break; }
-        {
-            const uint8_t* vt = sm + SM_V + (row >> 6) * V_ATOM;
-            const int vc = (row & 63) >> 3, ve = row & 7;
-            float bv[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int r = half * 32 + e;
-                const float vv = __bfloat162float(
-                    *reinterpret_cast<const __nv_bfloat16*>(vt + tc::sw128(r, vc) + ve * 2));
-                bv[e] = bt_s[r] * vv;
-            }
-            tc::tmem_st32(tl + TM_X + half * 32, bv);
-            tc::tmem_st_wait();
-        }
-        tc::tc_fence_before();
-        __syncthreads();
         if (tid == 0) {
             tc::tc_fence_after();
             tc::mma_amn_bk(tmem + TM_G, kq_a, KQ_ATOM, sb + SM_F1, ID_WN, 4, 0);
-            tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_F1 + 8192, ID_WN, 4, 1);
+            tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_F1 + 8192, ID_WN, 4, 0);
+            tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
             tc::mma_commit(&bars[3]);
         }
         if (!cta_wait(&bars[3], mma_phase, timeout_ns, abort_flag)) { ok = false; break; }
@@ -490,23 +532,24 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         __syncthreads();
         COMBA_PHASE(6);
 
-        // ---- 8. X^T += S (-W)^T, O^T = S Qh^T; then S += X^T (D K), O^T += X^T P^T ---------
+        // ---- 8. X^T += S (-W)^T, O^T = S Qh^T; S += X^T (D K), O^T += X^T P^T; next Gram ------
         if (tid == 0) {
             tc::tc_fence_after();
             tc::mma_ak_bmn(tmem + TM_X, sb + SM_S, OP_ATOM, sb + SM_W, 8192, ID_SW, 8, 8, 1);
-            tc::mma_ak_bk(tmem + TM_O, sb + SM_S, OP_ATOM, kq_a + 8192, KQ_ATOM, ID_SQ, 8, 0);
             tc::mma_commit(&bars[4]);
-            const bool done1 = tc::mbar_wait(&bars[4], mma1_phase, timeout_ns);
-            if (done1) {
+            tc::mma_ak_bk(tmem + TM_O, sb + SM_S, OP_ATOM, kq_a + 8192, KQ_ATOM, ID_SQ, 8, 0);
+            bool good = tc::mbar_wait(&bars[4], mma1_phase, timeout_ns);
+            COMBA_PHASE(10);
+            if (good) {
                 tc::tc_fence_after();
-                if (n + 2 < nchunks) {
-                    tc::fence_proxy_async_smem();
-                    load_kq(n + 2);
-                }
                 tc::mma_tf32_ta_bk(tmem + TM_S, tmem + TM_X, sb + SM_DK, DKT_ATOM, ID_SU, 8, 1);
                 tc::mma_tf32_ta_bk(tmem + TM_O, tmem + TM_X, sb + SM_P, F32_ATOM, ID_XP, 8, 1);
                 tc::mma_commit(&bars[3]);
-            } else {
+                COMBA_PHASE(11);
+                if (!last) good = issue_gram(n + 1);          // TM_G is free again
+                COMBA_PHASE(12);
+            }
+            if (!good) {
                 *abort_flag = 1;
                 latch_status(-4);
             }
@@ -515,11 +558,15 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (!cta_wait(&bars[3], mma_phase, timeout_ns, abort_flag)) { ok = false; break; }
         mma_phase ^= 1;
         tc::tc_fence_after();
+        if (tid == 0 && n + 2 < nchunks) {   // stage st is free: its Qh was read by the MMAs above
+            tc::fence_proxy_async_smem();
+            load_kq(n + 2);
+        }
         COMBA_PHASE(7);
 
         // ---- 9. S -> bf16 operand, decay for the next chunk; output tile -------------------
         {
-            const float eLn = last ? 1.f : __expf(sum64(la_n, 1));
+            const float eLn = last ? 1.f : __expf(red_s[2] + red_s[3]);
             float* sfrow = (last && S_final)
                                ? S_final + ((size_t)blockIdx.x * kD + row) * kD + half * 64
                                : nullptr;
@@ -568,6 +615,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         COMBA_PHASE(8);
     }
 
+    COMBA_PHASE_END();
     if (tid == 0) tc::bulk_wait0();
     if (!ok) tc::mbar_wait(&bars[3], mma_phase, timeout_ns);
     tc::tc_fence_before();

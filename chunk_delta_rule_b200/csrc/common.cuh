@@ -14,22 +14,30 @@ __device__ int g_status = 0;
 __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0, code); }
 
 // Optional phase tracing (compile with -DCOMBA_TRACE_PHASES): thread 0 of CTA 0
-// accumulates clock64() deltas between consecutive COMBA_PHASE marks.  Off by
+// accumulates clock64() deltas between consecutive COMBA_PHASE marks in
+// registers and adds them to a device array at COMBA_PHASE_END.  Off by
 // default; the marks then compile to nothing.
 #ifdef COMBA_TRACE_PHASES
 __device__ unsigned long long g_phase_cycles[16];
-#define COMBA_PHASE_BEGIN() long long comba_phase_t = clock64()
-#define COMBA_PHASE(i)                                                              \
-    do {                                                                            \
-        if (blockIdx.x == 0 && threadIdx.x == 0) {                                  \
-            const long long comba_phase_now = clock64();                            \
-            g_phase_cycles[(i)] += (unsigned long long)(comba_phase_now - comba_phase_t); \
-            comba_phase_t = comba_phase_now;                                        \
-        }                                                                           \
+#define COMBA_PHASE_BEGIN()                                   \
+    long long comba_phase_t = clock64();                      \
+    unsigned long long comba_phase_acc[16] = {}
+#define COMBA_PHASE(i)                                                        \
+    do {                                                                      \
+        const long long comba_phase_now = clock64();                          \
+        comba_phase_acc[(i)] += (unsigned long long)(comba_phase_now - comba_phase_t); \
+        comba_phase_t = comba_phase_now;                                      \
+    } while (0)
+#define COMBA_PHASE_END()                                                     \
+    do {                                                                      \
+        if (blockIdx.x == 0 && threadIdx.x == 0)                              \
+            for (int comba_i = 0; comba_i < 16; ++comba_i)                    \
+                g_phase_cycles[comba_i] += comba_phase_acc[comba_i];          \
     } while (0)
 #else
 #define COMBA_PHASE_BEGIN() do {} while (0)
 #define COMBA_PHASE(i) do {} while (0)
+#define COMBA_PHASE_END() do {} while (0)
 #endif
 
 __device__ __forceinline__ float to_f32(float x) { return x; }

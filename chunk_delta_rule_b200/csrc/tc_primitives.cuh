@@ -248,6 +248,7 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 __device__ __forceinline__ void mma_ak_bk(uint32_t d, uint32_t a, uint32_t a_atom, uint32_t b,
                                           uint32_t b_atom, uint32_t idesc, int ksteps,
                                           uint32_t acc0) {
+#pragma unroll
     for (int ks = 0; ks < ksteps; ++ks) {
         const uint64_t ad = sdesc_sw128(a + (ks >> 2) * a_atom + (ks & 3) * 32, 16, 1024);
         const uint64_t bd = sdesc_sw128(b + (ks >> 2) * b_atom + (ks & 3) * 32, 16, 1024);
@@ -259,6 +260,7 @@ __device__ __forceinline__ void mma_ak_bk(uint32_t d, uint32_t a, uint32_t a_ato
 // index), B K-major (N rows, K within one 64-element atom).
 __device__ __forceinline__ void mma_amn_bk(uint32_t d, uint32_t a, uint32_t a_lbo, uint32_t b,
                                            uint32_t idesc, int ksteps, uint32_t acc0) {
+#pragma unroll
     for (int ks = 0; ks < ksteps; ++ks) {
         const uint64_t ad = sdesc_sw128(a + ks * 2048, a_lbo, 1024);
         const uint64_t bd = sdesc_sw128(b + ks * 32, 16, 1024);
@@ -272,6 +274,7 @@ __device__ __forceinline__ void mma_amn_bk(uint32_t d, uint32_t a, uint32_t a_lb
 __device__ __forceinline__ void mma_ak_bmn(uint32_t d, uint32_t a, uint32_t a_atom, uint32_t b,
                                            uint32_t b_lbo, uint32_t idesc, int ksteps, int kwrap,
                                            uint32_t acc0) {
+#pragma unroll
     for (int ks = 0; ks < ksteps; ++ks) {
         const uint64_t ad = sdesc_sw128(a + (ks >> 2) * a_atom + (ks & 3) * 32, 16, 1024);
         const uint64_t bd = sdesc_sw128(b + (ks % kwrap) * 2048, b_lbo, 1024);
@@ -284,6 +287,7 @@ __device__ __forceinline__ void mma_ak_bmn(uint32_t d, uint32_t a, uint32_t a_at
 __device__ __forceinline__ void mma_tf32_ta_bk(uint32_t d, uint32_t a_tmem, uint32_t b,
                                                uint32_t b_atom, uint32_t idesc, int ksteps,
                                                uint32_t acc0) {
+#pragma unroll
     for (int ks = 0; ks < ksteps; ++ks) {
         const uint64_t bd = sdesc_sw128(b + (ks >> 2) * b_atom + (ks & 3) * 32, 16, 1024);
         mma_tf32_ta(d, a_tmem + ks * 8, bd, idesc, (ks > 0) ? 1u : acc0);
