@@ -80,44 +80,45 @@ constexpr uint32_t ID_XP = tc::idesc_tf32(128, 64, false, false);   // X^T P^T
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// fp32 64 x 64 scratch with an XOR swizzle on the column.
+// fp32 64 x 64 scratch with an XOR swizzle on the column; byte address in a buffer.
 __device__ __forceinline__ int fidx(int r, int s) { return r * 64 + (s ^ (r & 31)); }
+__device__ __forceinline__ uint32_t faddr(uint32_t base, int r, int s) {
+    return base + 4u * (uint32_t)fidx(r, s);
+}
 
 // c[16 x 8] += A-block(FA at ra, ca: 16 x 16) * B-slab(FB at rb, cb: 16 x 8), one warp, tf32.
-__device__ __forceinline__ void slab_mma(float (&c)[4], const float* FA, int ra, int ca,
-                                         const float* FB, int rb, int cb, int lane) {
+__device__ __forceinline__ void slab_mma(float (&c)[4], uint32_t FA, int ra, int ca, uint32_t FB,
+                                         int rb, int cb, int lane) {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int kk = 0; kk < 2; ++kk) {
         uint32_t a[4], bb[2];
-        a[0] = tc::f32_to_tf32(FA[fidx(ra + g, ca + 8 * kk + t)]);
-        a[1] = tc::f32_to_tf32(FA[fidx(ra + g + 8, ca + 8 * kk + t)]);
-        a[2] = tc::f32_to_tf32(FA[fidx(ra + g, ca + 8 * kk + t + 4)]);
-        a[3] = tc::f32_to_tf32(FA[fidx(ra + g + 8, ca + 8 * kk + t + 4)]);
-        bb[0] = tc::f32_to_tf32(FB[fidx(rb + 8 * kk + t, cb + g)]);
-        bb[1] = tc::f32_to_tf32(FB[fidx(rb + 8 * kk + t + 4, cb + g)]);
+        a[0] = tc::f32_to_tf32(tc::lds_f32(faddr(FA, ra + g, ca + 8 * kk + t)));
+        a[1] = tc::f32_to_tf32(tc::lds_f32(faddr(FA, ra + g + 8, ca + 8 * kk + t)));
+        a[2] = tc::f32_to_tf32(tc::lds_f32(faddr(FA, ra + g, ca + 8 * kk + t + 4)));
+        a[3] = tc::f32_to_tf32(tc::lds_f32(faddr(FA, ra + g + 8, ca + 8 * kk + t + 4)));
+        bb[0] = tc::f32_to_tf32(tc::lds_f32(faddr(FB, rb + 8 * kk + t, cb + g)));
+        bb[1] = tc::f32_to_tf32(tc::lds_f32(faddr(FB, rb + 8 * kk + t + 4, cb + g)));
         tc::mma_sync_tf32(c, a, bb);
     }
 }
 
-__device__ __forceinline__ void slab_store(float* F, int r0, int c0, const float (&c)[4],
+__device__ __forceinline__ void slab_store(uint32_t F, int r0, int c0, const float (&c)[4],
                                            float scale, int lane) {
     const int g = lane >> 2, t = lane & 3;
-    F[fidx(r0 + g, c0 + 2 * t)] = scale * c[0];
-    F[fidx(r0 + g, c0 + 2 * t + 1)] = scale * c[1];
-    F[fidx(r0 + g + 8, c0 + 2 * t)] = scale * c[2];
-    F[fidx(r0 + g + 8, c0 + 2 * t + 1)] = scale * c[3];
+    tc::sts_f32(faddr(F, r0 + g, c0 + 2 * t), scale * c[0]);
+    tc::sts_f32(faddr(F, r0 + g, c0 + 2 * t + 1), scale * c[1]);
+    tc::sts_f32(faddr(F, r0 + g + 8, c0 + 2 * t), scale * c[2]);
+    tc::sts_f32(faddr(F, r0 + g + 8, c0 + 2 * t + 1), scale * c[3]);
 }
 
-// Diagonal 16 x 16 block `blk` of (I + A)^{-1} (A strictly lower, fp32 in F1)
+// Diagonal 16 x 16 block `blk` of (I + A)^{-1} (A strictly lower, fp32 at F1)
 // into F2: one warp, lane j < 16 owns column j, right-looking substitution.
 // Inside block `blk`, fidx(16 blk + r, 16 blk + s) = (16 blk + r) 64 + 32 (blk >> 1)
 // + (s ^ r), so every A offset below is a compile-time constant.
-__device__ __forceinline__ void diag_block_inverse(const float* __restrict__ F1, float* F2,
-                                                   int blk, int lane) {
-    const int o = 16 * blk;
-    const int base = o * 64 + 32 * (blk >> 1);
-    const float* Ab = F1 + base;
+__device__ __forceinline__ void diag_block_inverse(uint32_t F1, uint32_t F2, int blk, int lane) {
+    const uint32_t base = 4u * (uint32_t)(16 * blk * 64 + 32 * (blk >> 1));
+    const uint32_t Ab = F1 + base;
     const int j = lane & 15;
     float x[16];
 #pragma unroll
@@ -126,19 +127,19 @@ __device__ __forceinline__ void diag_block_inverse(const float* __restrict__ F1,
     for (int s = 0; s < 15; ++s) {
         const float xs = x[s];
 #pragma unroll
-        for (int r = s + 1; r < 16; ++r) x[r] = fmaf(-Ab[r * 64 + (s ^ r)], xs, x[r]);
+        for (int r = s + 1; r < 16; ++r)
+            x[r] = fmaf(-tc::lds_f32(Ab + 4u * (uint32_t)(r * 64 + (s ^ r))), xs, x[r]);
     }
     if (lane < 16) {
-        float* Tb = F2 + base;
+        const uint32_t Tb = F2 + base;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Tb[r * 64 + (j ^ r)] = x[r];
+        for (int r = 0; r < 16; ++r) tc::sts_f32(Tb + 4u * (uint32_t)(r * 64 + (j ^ r)), x[r]);
     }
 }
 
 // Off-diagonal blocks of (I + A)^{-1} by distance, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj,
 // one warp per 16 x 8 slab (warp 2j + slab); M_ij is staged in the upper block (j, i).
-__device__ __forceinline__ void offdiag_inverse(const float* __restrict__ F1, float* F2,
-                                                int tid) {
+__device__ __forceinline__ void offdiag_inverse(uint32_t F1, uint32_t F2, int tid) {
     const int warp = tid >> 5, lane = tid & 31;
 #pragma unroll
     for (int dist = 1; dist <= 3; ++dist) {
@@ -160,29 +161,31 @@ __device__ __forceinline__ void offdiag_inverse(const float* __restrict__ F1, fl
 // Exact-exponential fallbacks for a chunk whose total log-decay is at or
 // below -80 (e^{-g} would leave the normal fp32 range): each entry takes exp2
 // of its own exponent difference.  Kept out of line: they are rarely taken.
-__device__ __noinline__ void a_row_exact(float* F1, uint32_t gram_taddr, int r, int s0, float br,
-                                         float gpr, const float* g2_s) {
+__device__ __noinline__ void a_row_exact(uint32_t F1, uint32_t gram_taddr, int r, int s0, float br,
+                                         float gpr, uint32_t G2) {
     float gv[32];
     tc::tmem_ld32(gram_taddr, gv);
     tc::tmem_ld_wait();
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
         const int s = s0 + e;
-        F1[fidx(r, s)] = (s < r) ? br * exp2f(gpr - g2_s[s]) * gv[e] : 0.f;
+        const float v = br * exp2f(gpr - tc::lds_f32(G2 + 4u * s)) * gv[e];
+        tc::sts_f32(faddr(F1, r, s), (s < r) ? v : 0.f);
     }
 }
 
-__device__ __noinline__ void p_row_exact(uint8_t* prow, uint32_t gram_taddr, int r, int s0,
-                                         float dh, const float* g2_s) {
+__device__ __noinline__ void p_row_exact(uint32_t prow, uint32_t gram_taddr, int r, int s0,
+                                         float dh, uint32_t G2) {
     float gv[32];
     tc::tmem_ld32(gram_taddr, gv);
     tc::tmem_ld_wait();
-    const float gr = g2_s[r];
+    const float gr = tc::lds_f32(G2 + 4u * r);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
         const int s = s0 + e;
-        float* pp = reinterpret_cast<float*>(prow + tc::sw128(r, e >> 2)) + (e & 3);
-        *pp = (s <= r) ? exp2f(gr - g2_s[s]) * fmaf(-dh, *pp, gv[e]) : 0.f;
+        const uint32_t pa = prow + tc::sw128(r, e >> 2) + 4u * (e & 3);
+        const float v = exp2f(gr - tc::lds_f32(G2 + 4u * s)) * fmaf(-dh, tc::lds_f32(pa), gv[e]);
+        tc::sts_f32(pa, (s <= r) ? v : 0.f);
     }
 }
 
@@ -225,24 +228,24 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const float* __restrict__ log_alpha, const float* __restrict__ beta,
                     const float* __restrict__ dvec, const float* S0, float* S_final, int T, int H,
                     unsigned long long timeout_ns) {
-    extern __shared__ uint8_t smem_raw[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
     uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     const uint32_t sb = tc::smem_u32(sm);
 
-    float* g2_s = reinterpret_cast<float*>(sm + SM_MISC);  // g_r log2(e)
-    float* gp2_s = g2_s + 64;                               // g_{r-1} log2(e)
-    float* bt_s = g2_s + 128;                               // beta_r
-    float* c_s = g2_s + 192;                                // beta_r e^{g_{r-1}}
-    float* eg_s = g2_s + 256;                               // e^{g_r}
-    float* ed_s = g2_s + 320;                               // e^{g_L - g_r}
-    float* ieg_s = g2_s + 384;                              // e^{-g_r} (when the chunk allows)
-    float* red_s = g2_s + 448;                              // [0..1] scan carries, [2..3] next-chunk sums
+    // gate tables (64 fp32 each), by shared address
+    const uint32_t G2 = sb + SM_MISC;        // g_r log2(e)
+    const uint32_t GP2 = G2 + 256;           // g_{r-1} log2(e)
+    const uint32_t BT = G2 + 512;            // beta_r
+    const uint32_t CS = G2 + 768;            // beta_r e^{g_{r-1}}
+    const uint32_t EG = G2 + 1024;           // e^{g_r}
+    const uint32_t ED = G2 + 1280;           // e^{g_L - g_r}
+    const uint32_t IEG = G2 + 1536;          // e^{-g_r} (when the chunk allows)
+    const uint32_t RED = G2 + 1792;          // [0..1] scan carries, [2..3] next-chunk sums
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 1856);  // kq0, kq1, v, mma, mma1, gram
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    float* F1 = reinterpret_cast<float*>(sm + SM_F1);
-    float* F2 = reinterpret_cast<float*>(sm + SM_F2);
+    const uint32_t F1 = sb + SM_F1, F2 = sb + SM_F2;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int row = tid & 127;          // TMEM lane
@@ -263,7 +266,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
     if (warp == 0) tc::tmem_alloc(tmem_slot, TM_COLS);
     for (int i = tid; i < 8192 / 16; i += kThreads)   // diag(lo(beta)): zero off the diagonal
-        reinterpret_cast<uint4*>(sm + SM_BLO)[i] = make_uint4(0u, 0u, 0u, 0u);
+        tc::sts_u32x4(sb + SM_BLO + 16u * i, make_uint4(0u, 0u, 0u, 0u));
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
@@ -286,7 +289,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tc::tma_load_4d(sm + SM_V, &tm_v, &bars[2], 0, h, t0, b);
         tc::tma_load_4d(sm + SM_V + V_ATOM, &tm_v, &bars[2], 64, h, t0, b);
     };
-    // Gram MMA of chunk n (thread 0): waits for its q/k tiles, commits to bars[5].
     auto issue_gram = [&](int n) -> bool { return issue_gram_mma(bars, sb, tmem, n, timeout_ns); };
     auto gate = [&](const float* p, int t) -> float {
         return (t < T) ? p[((size_t)b * T + t) * H + h] : 0.f;
@@ -307,14 +309,15 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         la_c = gate(log_alpha, tid);
         bt_c = gate(beta, tid);
         const float w = warp_sum(la_c);
-        if (lane == 0) red_s[2 + warp] = w;
+        if (lane == 0) tc::sts_f32(RED + 8u + 4u * warp, w);
     }
     __syncthreads();
-    const float eL0 = __expf(red_s[2] + red_s[3]);
+    const float eL0 = __expf(tc::lds_f32(RED + 8u) + tc::lds_f32(RED + 12u));
 
     // Initial state: fp32 master (decayed for chunk 0) into TMEM, bf16 copy.
     {
         const float* s0row = S0 ? S0 + ((size_t)blockIdx.x * kD + row) * kD + half * 64 : nullptr;
+        const uint32_t sbase = sb + SM_S + half * OP_ATOM;
 #pragma unroll 1
         for (int part = 0; part < 2; ++part) {
             float v[32];
@@ -324,10 +327,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                         : make_float4(0.f, 0.f, 0.f, 0.f);
                 v[e] = t4.x; v[e + 1] = t4.y; v[e + 2] = t4.z; v[e + 3] = t4.w;
             }
-            uint8_t* base = sm + SM_S + half * OP_ATOM;
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4)
-                *reinterpret_cast<uint4*>(base + tc::sw128(row, part * 4 + c4)) = pack8_bf16(v + c4 * 8);
+                tc::sts_u32x4(sbase + tc::sw128(row, part * 4 + c4), pack8_bf16(v + c4 * 8));
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= eL0;
             tc::tmem_st32(tl + TM_S + half * 64 + part * 32, v);
@@ -345,7 +347,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     for (int n = 0; n < nchunks && ok; ++n) {
         const int t0 = n * kC;
         const int st = n & 1;
-        uint8_t* kq = sm + (st ? SM_KQ1 : SM_KQ0);
         const uint32_t kq_a = sb + (st ? SM_KQ1 : SM_KQ0);
         const bool last = (n + 1 == nchunks);
 
@@ -361,23 +362,24 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const float y = __shfl_up_sync(0xffffffffu, x, off);
                 if (lane >= off) x += y;
             }
-            if (lane == 31) red_s[warp] = x;
-            g2_s[tid] = x;
+            if (lane == 31) tc::sts_f32(RED + 4u * warp, x);
+            tc::sts_f32(G2 + 4u * tid, x);
         }
         if (tid == 0) tc::bulk_wait_read0();   // previous out tile has left SM_DK
         __syncthreads();
-        const float gL = red_s[0] + red_s[1];
+        const float carry = tc::lds_f32(RED);
+        const float gL = carry + tc::lds_f32(RED + 4u);
         const bool fast = gL > -80.f;           // e^{-g} stays a normal fp32 number
         if (tid < 64) {
-            const float g = g2_s[tid] + (tid >= 32 ? red_s[0] : 0.f);
+            const float g = tc::lds_f32(G2 + 4u * tid) + (tid >= 32 ? carry : 0.f);
             const float gp = g - la_c;
-            bt_s[tid] = bt_c;
-            c_s[tid] = bt_c * __expf(gp);
-            eg_s[tid] = __expf(g);
-            ieg_s[tid] = fast ? __expf(-g) : 0.f;
-            ed_s[tid] = __expf(gL - g);
-            gp2_s[tid] = gp * kLog2e;
-            g2_s[tid] = g * kLog2e;
+            tc::sts_f32(BT + 4u * tid, bt_c);
+            tc::sts_f32(CS + 4u * tid, bt_c * __expf(gp));
+            tc::sts_f32(EG + 4u * tid, __expf(g));
+            tc::sts_f32(IEG + 4u * tid, fast ? __expf(-g) : 0.f);
+            tc::sts_f32(ED + 4u * tid, __expf(gL - g));
+            tc::sts_f32(GP2 + 4u * tid, gp * kLog2e);
+            tc::sts_f32(G2 + 4u * tid, g * kLog2e);
         }
         COMBA_PHASE(0);
 
@@ -393,26 +395,32 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::tmem_ld32(tl + TM_G + half * 32, gv);
             tc::tmem_ld_wait();
             const int s0 = half * 32;
+            const uint32_t prow = sb + SM_P + half * F32_ATOM;
             if (row < 64) {
                 const int r = row;
-                uint8_t* prow = sm + SM_P + half * F32_ATOM;
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<float4*>(prow + tc::sw128(r, c)) =
-                        make_float4(gv[4 * c], gv[4 * c + 1], gv[4 * c + 2], gv[4 * c + 3]);
+                    tc::sts_f32x4(prow + tc::sw128(r, c),
+                                  make_float4(gv[4 * c], gv[4 * c + 1], gv[4 * c + 2], gv[4 * c + 3]));
                 if (fast) {
-                    const float cr = c_s[r];
+                    const float cr = tc::lds_f32(CS + 4u * r);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int s = s0 + e;
-                        F1[fidx(r, s)] = (s < r) ? cr * ieg_s[s] * gv[e] : 0.f;
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 ig = tc::lds_f32x4(IEG + 4u * (s0 + 4 * c));
+                        const float iv[4] = {ig.x, ig.y, ig.z, ig.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int s = s0 + 4 * c + e;
+                            tc::sts_f32(faddr(F1, r, s), (s < r) ? cr * iv[e] * gv[4 * c + e] : 0.f);
+                        }
                     }
                 } else {
-                    a_row_exact(F1, tl + TM_G + half * 32, r, s0, bt_s[r], gp2_s[r], g2_s);
+                    a_row_exact(F1, tl + TM_G + half * 32, r, s0, tc::lds_f32(BT + 4u * r),
+                                tc::lds_f32(GP2 + 4u * r), G2);
                 }
                 if (!last && tid < 64) {   // total log-decay of the next chunk
                     const float w = warp_sum(la_n);
-                    if (lane == 0) red_s[2 + warp] = w;
+                    if (lane == 0) tc::sts_f32(RED + 8u + 4u * warp, w);
                 }
             }
             __syncthreads();
@@ -420,33 +428,33 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (row >= 64) {
                 // P in place over K K^T (row r, columns s0 .. s0 + 31)
                 const int r = row - 64;
-                uint8_t* prow = sm + SM_P + half * F32_ATOM;
-                const float er = eg_s[r];
+                const float er = tc::lds_f32(EG + 4u * r);
                 if (fast) {
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        const float4 kk = *reinterpret_cast<const float4*>(prow + tc::sw128(r, c));
-                        const float4 ig = *reinterpret_cast<const float4*>(ieg_s + s0 + 4 * c);
+                        const uint32_t pa = prow + tc::sw128(r, c);
+                        const float4 kk = tc::lds_f32x4(pa);
+                        const float4 ig = tc::lds_f32x4(IEG + 4u * (s0 + 4 * c));
                         const int s = s0 + 4 * c;
                         float4 p;
                         p.x = (s + 0 <= r) ? er * ig.x * fmaf(-dh, kk.x, gv[4 * c + 0]) : 0.f;
                         p.y = (s + 1 <= r) ? er * ig.y * fmaf(-dh, kk.y, gv[4 * c + 1]) : 0.f;
                         p.z = (s + 2 <= r) ? er * ig.z * fmaf(-dh, kk.z, gv[4 * c + 2]) : 0.f;
                         p.w = (s + 3 <= r) ? er * ig.w * fmaf(-dh, kk.w, gv[4 * c + 3]) : 0.f;
-                        *reinterpret_cast<float4*>(prow + tc::sw128(r, c)) = p;
+                        tc::sts_f32x4(pa, p);
                     }
                 } else {
-                    p_row_exact(prow, tl + TM_G + half * 32, r, s0, dh, g2_s);
+                    p_row_exact(prow, tl + TM_G + half * 32, r, s0, dh, G2);
                 }
                 // Qh (over Q) and (D K)^T for row r, key columns 64 half .. 64 half + 63
-                const float edr = ed_s[r];
-                uint8_t* dka = sm + SM_DK + (r >> 5) * DKT_ATOM + (r & 3) * 4;
+                const float edr = tc::lds_f32(ED + 4u * r);
+                const uint32_t dka = sb + SM_DK + (r >> 5) * DKT_ATOM + (r & 3) * 4;
                 const uint32_t rc = (r & 31) >> 2;
-#pragma unroll 1
+#pragma unroll 2
                 for (int c = 0; c < 8; ++c) {
-                    const uint32_t off = half * KQ_ATOM + tc::sw128(r, c);
-                    const uint4 kw = *reinterpret_cast<const uint4*>(kq + off);
-                    uint4 qw = *reinterpret_cast<const uint4*>(kq + 8192 + off);
+                    const uint32_t off = kq_a + half * KQ_ATOM + tc::sw128(r, c);
+                    const uint4 kw = tc::lds_u32x4(off);
+                    uint4 qw = tc::lds_u32x4(off + 8192);
                     const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kw);
                     __nv_bfloat162* q2 = reinterpret_cast<__nv_bfloat162*>(&qw);
 #pragma unroll
@@ -455,10 +463,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         const float2 qf = __bfloat1622float2(q2[e]);
                         q2[e] = __floats2bfloat162_rn(er * fmaf(-dh, kf.x, qf.x), er * fmaf(-dh, kf.y, qf.y));
                         const int j = 64 * half + 8 * c + 2 * e;
-                        *reinterpret_cast<float*>(dka + tc::sw128(j, rc)) = edr * kf.x;
-                        *reinterpret_cast<float*>(dka + tc::sw128(j + 1, rc)) = edr * kf.y;
+                        tc::sts_f32(dka + tc::sw128(j, rc), edr * kf.x);
+                        tc::sts_f32(dka + tc::sw128(j + 1, rc), edr * kf.y);
                     }
-                    *reinterpret_cast<uint4*>(kq + 8192 + off) = qw;
+                    tc::sts_u32x4(off + 8192, qw);
                 }
             } else {
                 // warps 0, 1, 4, 5 -> diagonal blocks 0, 1, 2, 3
@@ -482,17 +490,20 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int s = c * 8 + e;
-                    const float t = (s <= r) ? F2[fidx(r, s)] : 0.f;
-                    tcv[e] = t * c_s[s];
-                    ebv[e] = (s < r) ? t * bt_s[s] : ((s == r) ? bt_s[s] : 0.f);
+                    const float t = tc::lds_f32(faddr(F2, r, s));
+                    const float cv = tc::lds_f32(CS + 4u * s), bv = tc::lds_f32(BT + 4u * s);
+                    tcv[e] = (s <= r) ? t * cv : 0.f;
+                    ebv[e] = (s < r) ? t * bv : ((s == r) ? bv : 0.f);
                 }
-                *reinterpret_cast<uint4*>(sm + SM_F1 + tc::sw128(r, c)) = pack8_bf16(tcv);
-                *reinterpret_cast<uint4*>(sm + SM_F1 + 8192 + tc::sw128(r, c)) = pack8_bf16(ebv);
+                tc::sts_u32x4(F1 + tc::sw128(r, c), pack8_bf16(tcv));
+                tc::sts_u32x4(F1 + 8192 + tc::sw128(r, c), pack8_bf16(ebv));
             }
             if (tid < 64) {
-                const float bh = __bfloat162float(__float2bfloat16_rn(bt_s[tid]));
-                *reinterpret_cast<__nv_bfloat16*>(sm + SM_BLO + tc::sw128(tid, tid >> 3) + (tid & 7) * 2) =
-                    __float2bfloat16_rn(bt_s[tid] - bh);
+                const float bv = tc::lds_f32(BT + 4u * tid);
+                const float bh = __bfloat162float(__float2bfloat16_rn(bv));
+                const __nv_bfloat16 lo = __float2bfloat16_rn(bv - bh);
+                tc::sts_u16(sb + SM_BLO + tc::sw128(tid, tid >> 3) + (tid & 7) * 2,
+                            *reinterpret_cast<const unsigned short*>(&lo));
             }
         }
         tc::fence_proxy_async_smem();
@@ -502,8 +513,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (!cta_wait(&bars[2], n & 1, timeout_ns, abort_flag)) { ok = false; break; }
         if (tid == 0) {
             tc::tc_fence_after();
-            tc::mma_amn_bk(tmem + TM_G, kq_a, KQ_ATOM, sb + SM_F1, ID_WN, 4, 0);
-            tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_F1 + 8192, ID_WN, 4, 0);
+            tc::mma_amn_bk(tmem + TM_G, kq_a, KQ_ATOM, F1, ID_WN, 4, 0);
+            tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, F1 + 8192, ID_WN, 4, 0);
             tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
             tc::mma_commit(&bars[3]);
         }
@@ -525,7 +536,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int e = 0; e < 32; ++e) w[e] = -w[e];
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4)
-                *reinterpret_cast<uint4*>(sm + SM_W + tc::sw128(row, half * 4 + c4)) = pack8_bf16(w + c4 * 8);
+                tc::sts_u32x4(sb + SM_W + tc::sw128(row, half * 4 + c4), pack8_bf16(w + c4 * 8));
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
@@ -566,11 +577,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
         // ---- 9. S -> bf16 operand, decay for the next chunk; output tile -------------------
         {
-            const float eLn = last ? 1.f : __expf(red_s[2] + red_s[3]);
+            const float eLn = last ? 1.f : __expf(tc::lds_f32(RED + 8u) + tc::lds_f32(RED + 12u));
             float* sfrow = (last && S_final)
                                ? S_final + ((size_t)blockIdx.x * kD + row) * kD + half * 64
                                : nullptr;
-            uint8_t* base = sm + SM_S + half * OP_ATOM;
+            const uint32_t sbase = sb + SM_S + half * OP_ATOM;
 #pragma unroll 1
             for (int part = 0; part < 2; ++part) {
                 float v[32];
@@ -578,7 +589,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::tmem_ld_wait();
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4)
-                    *reinterpret_cast<uint4*>(base + tc::sw128(row, part * 4 + c4)) = pack8_bf16(v + c4 * 8);
+                    tc::sts_u32x4(sbase + tc::sw128(row, part * 4 + c4), pack8_bf16(v + c4 * 8));
                 if (sfrow) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 4)
@@ -591,15 +602,16 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
             // O^T row i (value index) -> out tile [token][i], two 64-wide boxes
-            uint8_t* ot = sm + SM_DK + (row >> 6) * 8192;
-            const int oc = (row & 63) >> 3, oe = row & 7;
+            const uint32_t ot = sb + SM_DK + (row >> 6) * 8192 + (row & 7) * 2;
+            const int oc = (row & 63) >> 3;
             float o[32];
             tc::tmem_ld32(tl + TM_O + half * 32, o);
             tc::tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                *reinterpret_cast<__nv_bfloat16*>(ot + tc::sw128(half * 32 + e, oc) + oe * 2) =
-                    __float2bfloat16_rn(o[e]);
+            for (int e = 0; e < 32; ++e) {
+                const __nv_bfloat16 ob = __float2bfloat16_rn(o[e]);
+                tc::sts_u16(ot + tc::sw128(half * 32 + e, oc), *reinterpret_cast<const unsigned short*>(&ob));
+            }
             tc::tmem_st_wait();
         }
         tc::fence_proxy_async_smem();

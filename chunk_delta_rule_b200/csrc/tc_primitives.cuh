@@ -137,6 +137,19 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 (A: lane = row, two bf16 per column,
+// the lower K index in the low half)
+__device__ __forceinline__ void mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "setp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
+        "}\n"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]^T, tf32 (A: lane = row, one fp32 per column)
 __device__ __forceinline__ void mma_tf32_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
                                             uint32_t idesc, uint32_t accumulate) {
@@ -294,6 +307,29 @@ __device__ __forceinline__ void mma_tf32_ta_bk(uint32_t d, uint32_t a_tmem, uint
     }
 }
 
+// bf16, A from TMEM (K = 16 per MMA = 8 packed columns), B K-major (N rows, K
+// atoms `b_atom` apart).
+__device__ __forceinline__ void mma_bf16_ta_bk(uint32_t d, uint32_t a_tmem, uint32_t b,
+                                               uint32_t b_atom, uint32_t idesc, int ksteps,
+                                               uint32_t acc0) {
+#pragma unroll
+    for (int ks = 0; ks < ksteps; ++ks) {
+        const uint64_t bd = sdesc_sw128(b + (ks >> 2) * b_atom + (ks & 3) * 32, 16, 1024);
+        mma_bf16_ta(d, a_tmem + ks * 8, bd, idesc, (ks > 0) ? 1u : acc0);
+    }
+}
+
+// bf16, A from TMEM, B MN-major (N in atoms `b_lbo` apart; one 128 B row per K index).
+__device__ __forceinline__ void mma_bf16_ta_bmn(uint32_t d, uint32_t a_tmem, uint32_t b,
+                                                uint32_t b_lbo, uint32_t idesc, int ksteps,
+                                                uint32_t acc0) {
+#pragma unroll
+    for (int ks = 0; ks < ksteps; ++ks) {
+        const uint64_t bd = sdesc_sw128(b + ks * 2048, b_lbo, 1024);
+        mma_bf16_ta(d, a_tmem + ks * 8, bd, idesc, (ks > 0) ? 1u : acc0);
+    }
+}
+
 // ---------------------------------------------------------------- warp MMA (legacy)
 __device__ __forceinline__ uint32_t f32_to_tf32(float x) {
     uint32_t r;
@@ -313,6 +349,42 @@ __device__ __forceinline__ void mma_sync_tf32(float (&d)[4], const uint32_t (&a)
 
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------- shared memory
+// Explicit shared-space accesses by 32-bit shared address.  Loads are issued
+// unconditionally (callers select the value), which keeps element loops free
+// of divergent branches.
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ float4 lds_f32x4(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint4 lds_u32x4(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+__device__ __forceinline__ void sts_f32x4(uint32_t a, float4 v) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};"
+                 ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
+}
+__device__ __forceinline__ void sts_u32x4(uint32_t a, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                 ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ void sts_u16(uint32_t a, unsigned short v) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(v) : "memory");
 }
 
 // ---------------------------------------------------------------- swizzle

@@ -38,7 +38,18 @@ __global__ void umma_check_kernel(int mode, const float* A, const float* B, cons
     int M = 128, N = 64, K = 128;
     if (mode == 1 || mode == 2) K = 64;
     if (mode == 4) N = 128;
-    if (mode == 6 || mode == 7) {
+    if (mode == 8 || mode == 9) {
+        // bf16 with A in TMEM (two bf16 per column); B bf16 in smem:
+        // 8: K-major, N = 64, K = 128 in two atoms 16 KB apart
+        // 9: MN-major, N = 64 (one atom), K = 128 rows
+        K = 128;
+        N = 64;
+        for (int e = tid; e < N * K; e += blockDim.x) {
+            const int n = e / K, k = e % K;
+            const uint32_t off = (mode == 8) ? kmaj(n, k, 16384) : mnmaj(n, k, 8192);
+            *reinterpret_cast<__nv_bfloat16*>(sbt + off) = __float2bfloat16_rn(B[e]);
+        }
+    } else if (mode == 6 || mode == 7) {
         // tf32 with A in TMEM (fp32, lane = row, column = k); B fp32 in smem:
         // 6: K-major, N = 64, K = 64 in two 32-element atoms 8 KB apart
         // 7: K-major, N = 128, K = 64 in two 32-element atoms 16 KB apart
@@ -78,6 +89,19 @@ __global__ void umma_check_kernel(int mode, const float* A, const float* B, cons
     tc_fence_after();
     const uint32_t tmem = tslot;
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    if (mode == 8 || mode == 9) {   // A (bf16 pairs) into TMEM columns 128..191
+        for (int part = 0; part < 2; ++part) {
+            float v[32];
+            for (int e = 0; e < 32; ++e) {
+                const int k = part * 64 + 2 * e;
+                const uint32_t w = pack_bf16(A[tid * K + k], A[tid * K + k + 1]);
+                v[e] = __uint_as_float(w);
+            }
+            tmem_st32(trow + 128 + part * 32, v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+    }
     if (mode == 6 || mode == 7) {   // A (fp32) into TMEM columns 128..191
         for (int part = 0; part < 2; ++part) {
             float v[32];
@@ -108,6 +132,8 @@ __global__ void umma_check_kernel(int mode, const float* A, const float* B, cons
             case 4: mma_ak_bmn(tmem, a, 16384, b, 16384, idesc_bf16(128, 128, false, true), 8, 4, 0); break;
             case 5: mma_ak_bk(tmem, a, 16384, b, 0, idesc_bf16(128, 64, false, false), 8, 1); break;
             case 6: mma_tf32_ta_bk(tmem, tmem + 128, b, 8192, idesc_tf32(128, 64, false, false), 8, 0); break;
+            case 8: mma_bf16_ta_bk(tmem, tmem + 128, b, 16384, idesc_bf16(128, 64, false, false), 8, 0); break;
+            case 9: mma_bf16_ta_bmn(tmem, tmem + 128, b, 8192, idesc_bf16(128, 64, false, true), 8, 0); break;
             case 7: mma_tf32_ta_bk(tmem, tmem + 128, b, 16384, idesc_tf32(128, 128, false, false), 8, 0); break;
         }
         mma_commit(&bar);

@@ -36,6 +36,8 @@ def lib(tmp_path_factory):
     (5, 128, 64, 128, True),    # X^T P^T accumulated onto an initial D
     (6, 128, 64, 64, False),    # tf32: X (TMEM) P^T, P K-major fp32
     (7, 128, 128, 64, False),   # tf32: X (TMEM) (D K), (D K)^T K-major fp32, N = 128
+    (8, 128, 64, 128, False),   # bf16: S (TMEM, packed pairs) Qh^T, Qh K-major
+    (9, 128, 64, 128, False),   # bf16: S (TMEM, packed pairs) (-W)^T, W MN-major
 ])
 def test_mma_layout(lib, mode, M, N, K, wrapB):
     g = torch.Generator().manual_seed(mode)
