@@ -1,7 +1,9 @@
 // Tensor-core chunk-wise Comba forward for bf16 inputs, dk = dv = 128, chunk 64.
 //
-// One CTA (8 warps) owns one (b, h) chain and walks its chunks in order.
-// Thread t owns TMEM lane t % 128 and half of that lane's columns.  Per chunk
+// One CTA owns one (b, h) chain and walks its chunks in order, split into two
+// warp groups that run one chunk apart: a prep group (8 warps) builds chunk
+// n+1's operands while a state group (4 warps) runs chunk n's state-dependent
+// MMAs and epilogue; they hand buffers over through mbarriers.  Per chunk
 // (chunk-start state S, local tokens r, s, g_r = sum_{i<=r} log_alpha_i, g_0 = 0;
 // the write-up's "block-recurrent, intra-block parallel" form with a single
 // inverse for the intermediates W and U, section "硬件高效的分块并行计算"):
@@ -41,28 +43,36 @@ namespace tck {
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;        // warps 0-3: state group; warps 4-11: prep group
+constexpr int kStateThreads = 128;
+constexpr int kPrepThreads = 256;
+constexpr int BAR_PREP = 1;          // named barrier ids
+constexpr int BAR_STATE = 2;
 
 // TMEM columns (fp32, 128 lanes)
-constexpr uint32_t TM_G = 0;     // Gram (lanes 0-63 K K^T, 64-127 Q K^T), then W^T
-constexpr uint32_t TM_X = 64;    // X^T (lane = value index i, column = token r)
-constexpr uint32_t TM_O = 128;   // O^T accumulator
-constexpr uint32_t TM_S = 256;   // fp32 state master (lane i, column j)
+constexpr uint32_t TM_G = 0;     // Gram of even chunks (lanes 0-63 K K^T, 64-127 Q K^T), then W^T
+constexpr uint32_t TM_G1 = 320;  // the same for odd chunks
+constexpr uint32_t TM_X0 = 64;   // X^T of even chunks (lane = value index i, column = token r)
+constexpr uint32_t TM_X1 = 128;  // X^T of odd chunks
+constexpr uint32_t TM_O = 192;   // O^T accumulator
+constexpr uint32_t TM_SB = 256;  // bf16 copy of S, two per column (MMA A operand)
+constexpr uint32_t TM_S = 384;   // fp32 state master (lane i, column j)
 constexpr uint32_t TM_COLS = 512;
 
 // Shared memory (bytes from a 1024-aligned base).
 constexpr uint32_t SM_KQ0 = 0;        // [K;Q] stage 0: 2 K-atoms x 128 rows x 128 B (bf16)
 constexpr uint32_t SM_KQ1 = 32768;    // stage 1
 constexpr uint32_t SM_V = 65536;      // V: 2 dv-atoms x 64 tokens x 128 B
-constexpr uint32_t SM_S = 81920;      // S bf16: 2 K-atoms x 128 rows
-constexpr uint32_t SM_W = 114688;     // -W bf16, MN-major: 128 rows (j) x 64 tokens
-constexpr uint32_t SM_P = 131072;     // P fp32, K-major: 2 atoms (32 s) x 64 rows (K K^T first)
-constexpr uint32_t SM_DK = 147456;    // (D K)^T fp32, K-major: 2 atoms (32 r) x 128 rows (j); out staging
-constexpr uint32_t SM_F1 = 180224;    // fp32 64x64: A; then Tc (bf16) | Eb (bf16)
-constexpr uint32_t SM_F2 = 196608;    // fp32 64x64: Tinv (upper blocks: scratch)
-constexpr uint32_t SM_BLO = 212992;   // bf16 64x64 K-major: diag(lo(beta)), zero elsewhere
+constexpr uint32_t SM_W = 81920;      // -W bf16, MN-major: 128 rows (j) x 64 tokens
+constexpr uint32_t SM_P = 98304;      // P fp32, K-major: 2 atoms (32 s) x 64 rows
+constexpr uint32_t SM_DK = 114688;    // (D K)^T fp32, K-major: 2 atoms (32 r) x 128 rows (j)
+constexpr uint32_t SM_KK = 147456;    // fp32 64x64 (fidx): K K^T, then P before its copy to SM_P
+constexpr uint32_t SM_F1 = 163840;    // fp32 64x64: A; then Tc (bf16) | Eb (bf16)
+constexpr uint32_t SM_F2 = 180224;    // fp32 64x64: Tinv (upper blocks: scratch)
+constexpr uint32_t SM_BLO = 196608;   // bf16 64x64 K-major: diag(lo(beta)), zero elsewhere
+constexpr uint32_t SM_OUT = 204800;   // out tile staging: 2 boxes x 64 tokens x 128 B
 constexpr uint32_t SM_MISC = 221184;  // gates, barriers
-constexpr uint32_t SM_END = SM_MISC + 2048;
+constexpr uint32_t SM_END = SM_MISC + 4096;
 constexpr uint32_t kSmemBytes = SM_END + 1024;
 
 constexpr uint32_t KQ_ATOM = 16384;
@@ -84,32 +94,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 __device__ __forceinline__ int fidx(int r, int s) { return r * 64 + (s ^ (r & 31)); }
 __device__ __forceinline__ uint32_t faddr(uint32_t base, int r, int s) {
     return base + 4u * (uint32_t)fidx(r, s);
-}
-
-// c[16 x 8] += A-block(FA at ra, ca: 16 x 16) * B-slab(FB at rb, cb: 16 x 8), one warp, tf32.
-__device__ __forceinline__ void slab_mma(float (&c)[4], uint32_t FA, int ra, int ca, uint32_t FB,
-                                         int rb, int cb, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-        uint32_t a[4], bb[2];
-        a[0] = tc::f32_to_tf32(tc::lds_f32(faddr(FA, ra + g, ca + 8 * kk + t)));
-        a[1] = tc::f32_to_tf32(tc::lds_f32(faddr(FA, ra + g + 8, ca + 8 * kk + t)));
-        a[2] = tc::f32_to_tf32(tc::lds_f32(faddr(FA, ra + g, ca + 8 * kk + t + 4)));
-        a[3] = tc::f32_to_tf32(tc::lds_f32(faddr(FA, ra + g + 8, ca + 8 * kk + t + 4)));
-        bb[0] = tc::f32_to_tf32(tc::lds_f32(faddr(FB, rb + 8 * kk + t, cb + g)));
-        bb[1] = tc::f32_to_tf32(tc::lds_f32(faddr(FB, rb + 8 * kk + t + 4, cb + g)));
-        tc::mma_sync_tf32(c, a, bb);
-    }
-}
-
-__device__ __forceinline__ void slab_store(uint32_t F, int r0, int c0, const float (&c)[4],
-                                           float scale, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-    tc::sts_f32(faddr(F, r0 + g, c0 + 2 * t), scale * c[0]);
-    tc::sts_f32(faddr(F, r0 + g, c0 + 2 * t + 1), scale * c[1]);
-    tc::sts_f32(faddr(F, r0 + g + 8, c0 + 2 * t), scale * c[2]);
-    tc::sts_f32(faddr(F, r0 + g + 8, c0 + 2 * t + 1), scale * c[3]);
 }
 
 // Diagonal 16 x 16 block `blk` of (I + A)^{-1} (A strictly lower, fp32 at F1)
@@ -137,24 +121,177 @@ __device__ __forceinline__ void diag_block_inverse(uint32_t F1, uint32_t F2, int
     }
 }
 
-// Off-diagonal blocks of (I + A)^{-1} by distance, T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj,
-// one warp per 16 x 8 slab (warp 2j + slab); M_ij is staged in the upper block (j, i).
-__device__ __forceinline__ void offdiag_inverse(uint32_t F1, uint32_t F2, int tid) {
-    const int warp = tid >> 5, lane = tid & 31;
+__device__ __forceinline__ uint4 pack8_bf16(const float* v) {
+    uint4 w;
+    w.x = tc::pack_bf16(v[0], v[1]);
+    w.y = tc::pack_bf16(v[2], v[3]);
+    w.z = tc::pack_bf16(v[4], v[5]);
+    w.w = tc::pack_bf16(v[6], v[7]);
+    return w;
+}
+
+// c[16 x 16] += X(16 x 16 at FX, rx, cx) * Y(16 x 16 at FY, ry, cy), one warp, tf32.
+__device__ __forceinline__ void blk16_mma(float (&c)[2][4], uint32_t FX, int rx, int cx, uint32_t FY,
+                                          int ry, int cy, int lane) {
+    const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int dist = 1; dist <= 3; ++dist) {
-        if (warp < 2 * (4 - dist)) {
-            const int j = warp >> 1, nt = warp & 1, i = j + dist;
-            float m[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int kb = j; kb < i; ++kb)
-                slab_mma(m, F1, 16 * i, 16 * kb, F2, 16 * kb, 16 * j + 8 * nt, lane);
-            slab_store(F2, 16 * j, 16 * i + 8 * nt, m, 1.f, lane);
-            __syncwarp();
-            float r2[4] = {0.f, 0.f, 0.f, 0.f};
-            slab_mma(r2, F2, 16 * i, 16 * i, F2, 16 * j, 16 * i + 8 * nt, lane);
-            slab_store(F2, 16 * i, 16 * j + 8 * nt, r2, -1.f, lane);
+    for (int kk = 0; kk < 2; ++kk) {
+        uint32_t a[4];
+        a[0] = tc::f32_to_tf32(tc::lds_f32(faddr(FX, rx + g, cx + 8 * kk + t)));
+        a[1] = tc::f32_to_tf32(tc::lds_f32(faddr(FX, rx + g + 8, cx + 8 * kk + t)));
+        a[2] = tc::f32_to_tf32(tc::lds_f32(faddr(FX, rx + g, cx + 8 * kk + t + 4)));
+        a[3] = tc::f32_to_tf32(tc::lds_f32(faddr(FX, rx + g + 8, cx + 8 * kk + t + 4)));
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            uint32_t bb[2];
+            bb[0] = tc::f32_to_tf32(tc::lds_f32(faddr(FY, ry + 8 * kk + t, cy + 8 * nt + g)));
+            bb[1] = tc::f32_to_tf32(tc::lds_f32(faddr(FY, ry + 8 * kk + t + 4, cy + 8 * nt + g)));
+            tc::mma_sync_tf32(c[nt], a, bb);
         }
-        __syncthreads();
+    }
+}
+
+// The 16 x 16 block at (r0, c0) of F in the accumulator layout of blk16_mma.
+__device__ __forceinline__ void blk16_load(float (&c)[2][4], uint32_t F, int r0, int c0, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        c[nt][0] = tc::lds_f32(faddr(F, r0 + g, c0 + 8 * nt + 2 * t));
+        c[nt][1] = tc::lds_f32(faddr(F, r0 + g, c0 + 8 * nt + 2 * t + 1));
+        c[nt][2] = tc::lds_f32(faddr(F, r0 + g + 8, c0 + 8 * nt + 2 * t));
+        c[nt][3] = tc::lds_f32(faddr(F, r0 + g + 8, c0 + 8 * nt + 2 * t + 1));
+    }
+}
+
+__device__ __forceinline__ void blk16_store(uint32_t F, int r0, int c0, const float (&c)[2][4],
+                                            float scale, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        tc::sts_f32(faddr(F, r0 + g, c0 + 8 * nt + 2 * t), scale * c[nt][0]);
+        tc::sts_f32(faddr(F, r0 + g, c0 + 8 * nt + 2 * t + 1), scale * c[nt][1]);
+        tc::sts_f32(faddr(F, r0 + g + 8, c0 + 8 * nt + 2 * t), scale * c[nt][2]);
+        tc::sts_f32(faddr(F, r0 + g + 8, c0 + 8 * nt + 2 * t + 1), scale * c[nt][3]);
+    }
+}
+
+// Writes Tc = T diag(c) and Eb = (T - I) diag(beta) + diag(beta) (bf16, K-major
+// 64 x 64 at F1 and F1 + 8192) for the 16 x 16 block (i, j) whose T values sit
+// in accumulator layout in `t`.
+__device__ __forceinline__ void tceb_store_frag(uint32_t F1, int i, int j, const float (&t)[2][4],
+                                                uint32_t CS, uint32_t BT, int lane) {
+    const int g = lane >> 2, tt = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int s = 16 * j + 8 * nt + 2 * tt;
+        const float c0 = tc::lds_f32(CS + 4u * s), c1 = tc::lds_f32(CS + 4u * (s + 1));
+        const float b0 = tc::lds_f32(BT + 4u * s), b1 = tc::lds_f32(BT + 4u * (s + 1));
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int r = 16 * i + g + 8 * hh;
+            const uint32_t off = tc::sw128(r, 2 * j + nt) + 4u * tt;
+            const float t0 = t[nt][2 * hh], t1 = t[nt][2 * hh + 1];
+            asm volatile("st.shared.b32 [%0], %1;" ::"r"(F1 + off), "r"(tc::pack_bf16(t0 * c0, t1 * c1)) : "memory");
+            asm volatile("st.shared.b32 [%0], %1;" ::"r"(F1 + 8192 + off), "r"(tc::pack_bf16(t0 * b0, t1 * b1)) : "memory");
+        }
+    }
+}
+
+// Tc / Eb of diagonal block `blk` (T_ii in F2) and zeros for the upper block
+// row of that block: 32 threads, row 16 blk + (lane & 15), half of the columns.
+__device__ __forceinline__ void tceb_diag_and_upper(uint32_t F1, uint32_t F2, int blk, int lane,
+                                                    uint32_t CS, uint32_t BT) {
+    const int rr = lane & 15, r = 16 * blk + rr;
+    const int hc = lane >> 4;                     // which 8-element chunk of the block
+    const int c = 2 * blk + hc;
+    float tcv[8], ebv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const int s = 8 * c + e;
+        const float t = tc::lds_f32(faddr(F2, r, s));
+        const float cv = tc::lds_f32(CS + 4u * s), bv = tc::lds_f32(BT + 4u * s);
+        tcv[e] = (s <= r) ? t * cv : 0.f;
+        ebv[e] = (s < r) ? t * bv : ((s == r) ? bv : 0.f);
+    }
+    tc::sts_u32x4(F1 + tc::sw128(r, c), pack8_bf16(tcv));
+    tc::sts_u32x4(F1 + 8192 + tc::sw128(r, c), pack8_bf16(ebv));
+    // upper blocks of this block row: chunks 2 blk + 2 .. 7
+    for (int cz = 2 * blk + 2 + hc; cz < 8; cz += 2) {
+        tc::sts_u32x4(F1 + tc::sw128(r, cz), make_uint4(0u, 0u, 0u, 0u));
+        tc::sts_u32x4(F1 + 8192 + tc::sw128(r, cz), make_uint4(0u, 0u, 0u, 0u));
+    }
+}
+
+// Off-diagonal blocks of T = (I + A)^{-1} from its diagonal blocks T_ii (in F2),
+// written out directly as the Tc / Eb operands.
+// With N = T_D A_off (N_ij = T_ii A_ij, strictly block-lower, N^4 = 0),
+// I + A = (I + A_D)(I + N), so T = (I - N + N^2 - N^3) T_D.  In blocks:
+//   M_{i+1,i} = -N_{i+1,i}
+//   M_20 = -N_20 + N_21 N_10,   M_31 = -N_31 + N_32 N_21
+//   M_30 = -N_30 + N_31 N_10 - N_32 M_20
+//   T_ij = M_ij T_jj
+// Four levels of single 16 x 16 products, one warp per block.  N_ij is kept in
+// the unused upper block (j, i) of F2, M_20, M_31, M_30 in the lower blocks.
+// A (in F1) is dead after level 1, so from level 2 on the idle warps turn the
+// diagonal blocks into Tc / Eb (and zero the upper blocks) in F1, and level 4
+// writes the lower blocks there.
+__device__ __forceinline__ void offdiag_inverse(uint32_t F1, uint32_t F2, int pt, uint32_t CS,
+                                                uint32_t BT) {
+    const int warp = pt >> 5, lane = pt & 31;
+    // level 1: N_ij = T_ii A_ij for the six lower blocks
+    if (warp < 6) {
+        const int i = (warp < 3) ? warp + 1 : ((warp == 5) ? 3 : warp - 1);
+        const int j = (warp < 3) ? warp : ((warp == 5) ? 0 : warp - 3);
+        float c[2][4] = {};
+        blk16_mma(c, F2, 16 * i, 16 * i, F1, 16 * i, 16 * j, lane);
+        blk16_store(F2, 16 * j, 16 * i, c, 1.f, lane);
+    }
+    tc::named_barrier(BAR_PREP, kPrepThreads);
+    // level 2: M_20, M_31 and Q_30 = -N_30 + N_31 N_10; warps 4..7: Tc/Eb of diagonal blocks
+    if (warp < 3) {
+        const int xa = warp == 1 ? 2 : 1, xb = warp == 1 ? 3 : (warp == 0 ? 2 : 3);   // N_{xb, xa}
+        const int ya = warp == 1 ? 1 : 0, yb = warp == 1 ? 2 : 1;                     // N_{yb, ya}
+        const int si = warp == 0 ? 2 : 3, sj = warp == 1 ? 1 : 0;                      // N_{si, sj}
+        float c[2][4] = {}, ns[2][4];
+        blk16_mma(c, F2, 16 * xa, 16 * xb, F2, 16 * ya, 16 * yb, lane);
+        blk16_load(ns, F2, 16 * sj, 16 * si, lane);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c[nt][e] -= ns[nt][e];
+        blk16_store(F2, 16 * si, 16 * sj, c, 1.f, lane);
+    } else if (warp >= 4) {
+        tceb_diag_and_upper(F1, F2, warp - 4, lane, CS, BT);
+    }
+    tc::named_barrier(BAR_PREP, kPrepThreads);
+    // level 3: M_30 = Q_30 - N_32 M_20
+    if (warp == 0) {
+        float c[2][4] = {}, q[2][4];
+        blk16_mma(c, F2, 32, 48, F2, 32, 0, lane);
+        blk16_load(q, F2, 48, 0, lane);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c[nt][e] = q[nt][e] - c[nt][e];
+        blk16_store(F2, 48, 0, c, 1.f, lane);
+    }
+    tc::named_barrier(BAR_PREP, kPrepThreads);
+    // level 4: T_ij = M_ij T_jj -> Tc / Eb
+    if (warp < 6) {
+        float c[2][4] = {};
+        if (warp < 3) {          // T_{j+1,j} = -N_{j+1,j} T_jj
+            const int j = warp, i = warp + 1;
+            blk16_mma(c, F2, 16 * j, 16 * i, F2, 16 * j, 16 * j, lane);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) c[nt][e] = -c[nt][e];
+            tceb_store_frag(F1, i, j, c, CS, BT, lane);
+        } else {                 // T_20, T_31, T_30
+            const int i = warp == 3 ? 2 : 3, j = warp == 4 ? 1 : 0;
+            blk16_mma(c, F2, 16 * i, 16 * j, F2, 16 * j, 16 * j, lane);
+            tceb_store_frag(F1, i, j, c, CS, BT, lane);
+        }
     }
 }
 
@@ -174,8 +311,8 @@ __device__ __noinline__ void a_row_exact(uint32_t F1, uint32_t gram_taddr, int r
     }
 }
 
-__device__ __noinline__ void p_row_exact(uint32_t prow, uint32_t gram_taddr, int r, int s0,
-                                         float dh, uint32_t G2) {
+__device__ __noinline__ void p_row_exact(uint32_t KK, uint32_t gram_taddr, int r, int s0, float dh,
+                                         uint32_t G2) {
     float gv[32];
     tc::tmem_ld32(gram_taddr, gv);
     tc::tmem_ld_wait();
@@ -183,43 +320,16 @@ __device__ __noinline__ void p_row_exact(uint32_t prow, uint32_t gram_taddr, int
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
         const int s = s0 + e;
-        const uint32_t pa = prow + tc::sw128(r, e >> 2) + 4u * (e & 3);
+        const uint32_t pa = faddr(KK, r, s);
         const float v = exp2f(gr - tc::lds_f32(G2 + 4u * s)) * fmaf(-dh, tc::lds_f32(pa), gv[e]);
         tc::sts_f32(pa, (s <= r) ? v : 0.f);
     }
 }
 
-// All threads wait on `bar`; a timeout is latched and makes every thread see
-// `false` after the barrier.
-__device__ __noinline__ bool cta_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
-                                      volatile int* abort_flag) {
-    if (!tc::mbar_wait(bar, parity, timeout_ns)) {
-        *abort_flag = 1;
-        latch_status(-4 /* COMBA_ETIMEOUT */);
-    }
-    __syncthreads();
-    return *abort_flag == 0;
-}
 
-__device__ __forceinline__ uint4 pack8_bf16(const float* v) {
-    uint4 w;
-    w.x = tc::pack_bf16(v[0], v[1]);
-    w.y = tc::pack_bf16(v[2], v[3]);
-    w.z = tc::pack_bf16(v[4], v[5]);
-    w.w = tc::pack_bf16(v[6], v[7]);
-    return w;
-}
-
-// Gram MMA of chunk n by one thread: waits for the chunk's q/k tiles, then
-// G = [K; Q] K^T into TMEM, committed to bars[5].
-__device__ __noinline__ bool issue_gram_mma(uint64_t* bars, uint32_t sb, uint32_t tmem, int n,
-                                            uint64_t timeout_ns) {
-    if (!tc::mbar_wait(&bars[n & 1], (n >> 1) & 1, timeout_ns)) return false;
-    const uint32_t kq_a = sb + ((n & 1) ? SM_KQ1 : SM_KQ0);
-    tc::tc_fence_after();
-    tc::mma_ak_bk(tmem + TM_G, kq_a, KQ_ATOM, kq_a, KQ_ATOM, ID_G, 8, 0);
-    tc::mma_commit(&bars[5]);
-    return true;
+__device__ __forceinline__ void fail(volatile int* gabort) {
+    *gabort = 1;
+    latch_status(-4 /* COMBA_ETIMEOUT */);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -233,7 +343,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     const uint32_t sb = tc::smem_u32(sm);
 
-    // gate tables (64 fp32 each), by shared address
+    // prep-private gate tables (64 fp32 each), by shared address
     const uint32_t G2 = sb + SM_MISC;        // g_r log2(e)
     const uint32_t GP2 = G2 + 256;           // g_{r-1} log2(e)
     const uint32_t BT = G2 + 512;            // beta_r
@@ -241,23 +351,27 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t EG = G2 + 1024;           // e^{g_r}
     const uint32_t ED = G2 + 1280;           // e^{g_L - g_r}
     const uint32_t IEG = G2 + 1536;          // e^{-g_r} (when the chunk allows)
-    const uint32_t RED = G2 + 1792;          // [0..1] scan carries, [2..3] next-chunk sums
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 1856);  // kq0, kq1, v, mma, mma1, gram
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    const uint32_t F1 = sb + SM_F1, F2 = sb + SM_F2;
+    const uint32_t RED = G2 + 1792;          // [0..1] scan carries
+    const uint32_t SRED = G2 + 1936;         // state group: [0..1] scan carries
+    const uint32_t SED = G2 + 2048;          // state group: e^{g_L - g_r} of the next chunk
+    // barriers: q/k stages, v, gram, wn, prep ready, mma1, mma2, state ready
+    enum { B_KQ0 = 0, B_KQ1 = 1, B_V = 2, B_GRAM = 3, B_WN = 4, B_PREP = 5, B_MMA1 = 6, B_MMA2 = 7,
+           B_SREADY = 8 };
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 1856);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+    volatile int* gabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const uint32_t F1 = sb + SM_F1, F2 = sb + SM_F2, KKS = sb + SM_KK;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int row = tid & 127;          // TMEM lane
-    const int half = tid >> 7;          // column half of that lane
     const int b = blockIdx.x / H, h = blockIdx.x % H;
     const float dh = dvec[h];
     const int nchunks = (T + kC - 1) / kC;
     const uint32_t trow = (uint32_t)((warp & 3) * 32) << 16;
 
     if (tid == 0) {
-        for (int i = 0; i < 6; ++i) tc::mbar_init(&bars[i], 1);
-        *abort_flag = 0;
+        for (int i = 0; i < 9; ++i)
+            tc::mbar_init(&bars[i], i == B_PREP ? kPrepThreads : (i == B_SREADY ? kStateThreads : 1));
+        *gabort = 0;
         tc::fence_mbar_init();
         tc::prefetch_tmap(&tm_q);
         tc::prefetch_tmap(&tm_k);
@@ -284,124 +398,305 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tc::tma_load_4d(dst + KQ_ATOM + 8192, &tm_q, bar, 64, h, t0, b);
     };
     auto load_v = [&](int n) {
-        tc::mbar_arrive_expect_tx(&bars[2], 16384);
+        tc::mbar_arrive_expect_tx(&bars[B_V], 16384);
         const int t0 = n * kC;
-        tc::tma_load_4d(sm + SM_V, &tm_v, &bars[2], 0, h, t0, b);
-        tc::tma_load_4d(sm + SM_V + V_ATOM, &tm_v, &bars[2], 64, h, t0, b);
+        tc::tma_load_4d(sm + SM_V, &tm_v, &bars[B_V], 0, h, t0, b);
+        tc::tma_load_4d(sm + SM_V + V_ATOM, &tm_v, &bars[B_V], 64, h, t0, b);
     };
-    auto issue_gram = [&](int n) -> bool { return issue_gram_mma(bars, sb, tmem, n, timeout_ns); };
     auto gate = [&](const float* p, int t) -> float {
         return (t < T) ? p[((size_t)b * T + t) * H + h] : 0.f;
     };
 
-    if (tid == 0) {
-        load_kq(0);
-        if (nchunks > 1) load_kq(1);
-        load_v(0);
-        if (!issue_gram(0)) {
-            *abort_flag = 1;
-            latch_status(-4);
-        }
-    }
-    // Gates of chunk 0 (threads 0..63), and their total for the initial decay.
-    float la_c = 0.f, bt_c = 0.f, la_n = 0.f, bt_n = 0.f;
-    if (tid < 64) {
-        la_c = gate(log_alpha, tid);
-        bt_c = gate(beta, tid);
-        const float w = warp_sum(la_c);
-        if (lane == 0) tc::sts_f32(RED + 8u + 4u * warp, w);
-    }
-    __syncthreads();
-    const float eL0 = __expf(tc::lds_f32(RED + 8u) + tc::lds_f32(RED + 12u));
-
-    // Initial state: fp32 master (decayed for chunk 0) into TMEM, bf16 copy.
-    {
-        const float* s0row = S0 ? S0 + ((size_t)blockIdx.x * kD + row) * kD + half * 64 : nullptr;
-        const uint32_t sbase = sb + SM_S + half * OP_ATOM;
-#pragma unroll 1
-        for (int part = 0; part < 2; ++part) {
-            float v[32];
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-                const float4 t4 = s0row ? *reinterpret_cast<const float4*>(s0row + part * 32 + e)
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-                v[e] = t4.x; v[e + 1] = t4.y; v[e + 2] = t4.z; v[e + 3] = t4.w;
-            }
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4)
-                tc::sts_u32x4(sbase + tc::sw128(row, part * 4 + c4), pack8_bf16(v + c4 * 8));
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] *= eL0;
-            tc::tmem_st32(tl + TM_S + half * 64 + part * 32, v);
-        }
-        tc::tmem_st_wait();
-    }
-    tc::fence_proxy_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-
-    uint32_t mma_phase = 0, mma1_phase = 0;
-    bool ok = *abort_flag == 0;
     COMBA_PHASE_BEGIN();
-    for (int n = 0; n < nchunks && ok; ++n) {
-        const int t0 = n * kC;
-        const int st = n & 1;
-        const uint32_t kq_a = sb + (st ? SM_KQ1 : SM_KQ0);
-        const bool last = (n + 1 == nchunks);
-
-        // ---- 1. gates ------------------------------------------------------------
-        if (tid < 64) {
-            if (!last) {   // prefetch the next chunk's gates
-                la_n = gate(log_alpha, t0 + kC + tid);
-                bt_n = gate(beta, t0 + kC + tid);
-            }
-            float x = la_c;
+    if (warp < 4) {
+        // =============================== state group ===============================
+        // Per chunk n: MMA1(n) X^T += S (-W)^T, O^T = S Qh^T; MMA2(n) S += X^T (D K),
+        // O^T += X^T P^T; then S -> bf16 copy, S *= e^{g_L(n+1)}, O^T -> out, and the
+        // (D K)^T operand of chunk n+1 (from the group's own scan of its log-decays).
+        const int row = tid;
+        const bool issuer = (tid == 0);
+        // Scan of one chunk's log-decays held by threads 0..63: writes e^{g_L - g_r}
+        // to SED and returns e^{g_L} to every thread of the group.
+        auto state_gates = [&](float la) -> float {
+            float x = la;
+            if (tid < 64) {
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, off);
-                if (lane >= off) x += y;
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                if (lane == 31) tc::sts_f32(SRED + 4u * warp, x);
             }
-            if (lane == 31) tc::sts_f32(RED + 4u * warp, x);
-            tc::sts_f32(G2 + 4u * tid, x);
-        }
-        if (tid == 0) tc::bulk_wait_read0();   // previous out tile has left SM_DK
-        __syncthreads();
-        const float carry = tc::lds_f32(RED);
-        const float gL = carry + tc::lds_f32(RED + 4u);
-        const bool fast = gL > -80.f;           // e^{-g} stays a normal fp32 number
-        if (tid < 64) {
-            const float g = tc::lds_f32(G2 + 4u * tid) + (tid >= 32 ? carry : 0.f);
-            const float gp = g - la_c;
-            tc::sts_f32(BT + 4u * tid, bt_c);
-            tc::sts_f32(CS + 4u * tid, bt_c * __expf(gp));
-            tc::sts_f32(EG + 4u * tid, __expf(g));
-            tc::sts_f32(IEG + 4u * tid, fast ? __expf(-g) : 0.f);
-            tc::sts_f32(ED + 4u * tid, __expf(gL - g));
-            tc::sts_f32(GP2 + 4u * tid, gp * kLog2e);
-            tc::sts_f32(G2 + 4u * tid, g * kLog2e);
-        }
-        COMBA_PHASE(0);
-
-        // ---- 2. Gram of this chunk (issued earlier) -----------------------------------
-        if (!cta_wait(&bars[st], (n >> 1) & 1, timeout_ns, abort_flag)) { ok = false; break; }
-        if (!cta_wait(&bars[5], n & 1, timeout_ns, abort_flag)) { ok = false; break; }
-        tc::tc_fence_after();
-        COMBA_PHASE(1);
-
-        // ---- 3. K K^T -> P buffer, A -> F1; then P/Qh/(DK)^T || diagonal inverse -------
+            tc::named_barrier(BAR_STATE, kStateThreads);
+            const float c0 = tc::lds_f32(SRED), gL = c0 + tc::lds_f32(SRED + 4u);
+            if (tid < 64) {
+                const float g = x + (tid >= 32 ? c0 : 0.f);
+                tc::sts_f32(SED + 4u * tid, __expf(gL - g));
+            }
+            return __expf(gL);
+        };
+        // (D K)^T of chunk c (K-major fp32 operand of the state update).
+        auto state_dk = [&](int c) -> bool {
+            const bool okc = tc::mbar_wait(&bars[c & 1], (c >> 1) & 1, timeout_ns);
+            const uint32_t kqc = sb + ((c & 1) ? SM_KQ1 : SM_KQ0);
+            const int r = tid & 63, jh = tid >> 6;
+            const float edr = tc::lds_f32(SED + 4u * r);
+            const uint32_t dka = sb + SM_DK + (r >> 5) * DKT_ATOM + (r & 3) * 4;
+            const uint32_t rc = (r & 31) >> 2;
+#pragma unroll 2
+            for (int c8 = 0; c8 < 8; ++c8) {
+                const uint4 kw = tc::lds_u32x4(kqc + jh * KQ_ATOM + tc::sw128(r, c8));
+                const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kw);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 kf = __bfloat1622float2(k2[e]);
+                    const int j = 64 * jh + 8 * c8 + 2 * e;
+                    tc::sts_f32(dka + tc::sw128(j, rc), edr * kf.x);
+                    tc::sts_f32(dka + tc::sw128(j + 1, rc), edr * kf.y);
+                }
+            }
+            tc::fence_proxy_async_smem();
+            return okc;
+        };
+        bool ok = true;
+        // decay and (D K)^T of chunk 0, initial state
         {
-            float gv[32];
-            tc::tmem_ld32(tl + TM_G + half * 32, gv);
-            tc::tmem_ld_wait();
-            const int s0 = half * 32;
-            const uint32_t prow = sb + SM_P + half * F32_ATOM;
-            if (row < 64) {
-                const int r = row;
+            const float la0 = (tid < 64) ? gate(log_alpha, tid) : 0.f;
+            const float eL0 = state_gates(la0);
+            tc::named_barrier(BAR_STATE, kStateThreads);
+            ok = state_dk(0);
+            const float* s0row = S0 ? S0 + ((size_t)blockIdx.x * kD + row) * kD : nullptr;
+#pragma unroll 1
+            for (int pair = 0; pair < 2; ++pair) {
+                float v0[32], v1[32], pk[32];
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    tc::sts_f32x4(prow + tc::sw128(r, c),
-                                  make_float4(gv[4 * c], gv[4 * c + 1], gv[4 * c + 2], gv[4 * c + 3]));
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 a4 = s0row ? *reinterpret_cast<const float4*>(s0row + 64 * pair + e)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4 b4 = s0row ? *reinterpret_cast<const float4*>(s0row + 64 * pair + 32 + e)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v0[e] = a4.x; v0[e + 1] = a4.y; v0[e + 2] = a4.z; v0[e + 3] = a4.w;
+                    v1[e] = b4.x; v1[e + 1] = b4.y; v1[e + 2] = b4.z; v1[e + 3] = b4.w;
+                }
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    pk[c] = __uint_as_float(tc::pack_bf16(v0[2 * c], v0[2 * c + 1]));
+                    pk[16 + c] = __uint_as_float(tc::pack_bf16(v1[2 * c], v1[2 * c + 1]));
+                }
+                tc::tmem_st32(tl + TM_SB + 32 * pair, pk);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) { v0[e] *= eL0; v1[e] *= eL0; }
+                tc::tmem_st32(tl + TM_S + 64 * pair, v0);
+                tc::tmem_st32(tl + TM_S + 64 * pair + 32, v1);
+            }
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            if (!ok) fail(gabort);
+            ok = tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok);
+            tc::mbar_arrive(&bars[B_SREADY]);
+        }
+        float la_n = 0.f;
+        for (int n = 0; n < nchunks && ok; ++n) {
+            const int t0 = n * kC;
+            const int stg = n & 1;
+            const uint32_t kq_a = sb + (stg ? SM_KQ1 : SM_KQ0);
+            const uint32_t txn = tmem + (stg ? TM_X1 : TM_X0);
+            const bool last = (n + 1 == nchunks);
+            if (tid < 64 && !last) la_n = gate(log_alpha, t0 + kC + tid);   // next chunk's decay
+            ok = (*gabort == 0);
+            if (issuer) {
+                ok = ok && tc::mbar_wait(&bars[B_SREADY], n & 1, timeout_ns) &&
+                     tc::mbar_wait(&bars[B_PREP], n & 1, timeout_ns);
+                COMBA_PHASE(0);
+                if (ok) {
+                    tc::tc_fence_after();
+                    tc::mma_bf16_ta_bmn(txn, tmem + TM_SB, sb + SM_W, 8192, ID_SW, 8, 1);
+                    tc::mma_commit(&bars[B_MMA1]);
+                    tc::mma_bf16_ta_bk(tmem + TM_O, tmem + TM_SB, kq_a + 8192, KQ_ATOM, ID_SQ, 8, 0);
+                    ok = tc::mbar_wait(&bars[B_MMA1], n & 1, timeout_ns);
+                    COMBA_PHASE(1);
+                    if (ok) {
+                        tc::tc_fence_after();
+                        tc::mma_tf32_ta_bk(tmem + TM_S, txn, sb + SM_DK, DKT_ATOM, ID_SU, 8, 1);
+                        tc::mma_tf32_ta_bk(tmem + TM_O, txn, sb + SM_P, F32_ATOM, ID_XP, 8, 1);
+                        tc::mma_commit(&bars[B_MMA2]);
+                    }
+                }
+                if (!ok) fail(gabort);
+            }
+            ok = ok && tc::mbar_wait(&bars[B_MMA2], n & 1, timeout_ns);
+            if (!ok) fail(gabort);
+            if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
+            tc::tc_fence_after();
+            COMBA_PHASE(2);
+            if (issuer && n + 2 < nchunks) {   // stage stg is free: its Qh was read by MMA1
+                tc::fence_proxy_async_smem();
+                load_kq(n + 2);
+            }
+            // O^T row (value index) -> bf16 pairs of tokens, read before S is released;
+            // the first half of S is loaded in the same batch
+            uint32_t ob[32];
+            float v0[32], v1[32];
+            {
+                float o0[32], o1[32];
+                tc::tmem_ld32(tl + TM_O, o0);
+                tc::tmem_ld32(tl + TM_O + 32, o1);
+                tc::tmem_ld32(tl + TM_S, v0);
+                tc::tmem_ld32(tl + TM_S + 32, v1);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    ob[c] = tc::pack_bf16(o0[2 * c], o0[2 * c + 1]);
+                    ob[16 + c] = tc::pack_bf16(o1[2 * c], o1[2 * c + 1]);
+                }
+            }
+            const float eLn = last ? 1.f : state_gates(la_n);
+            float* sfrow = (last && S_final) ? S_final + ((size_t)blockIdx.x * kD + row) * kD : nullptr;
+#pragma unroll 1
+            for (int pair = 0; pair < 2; ++pair) {
+                if (pair == 1) {
+                    tc::tmem_ld32(tl + TM_S + 64, v0);
+                    tc::tmem_ld32(tl + TM_S + 96, v1);
+                    tc::tmem_ld_wait();
+                }
+                float pk[32];
+                if (sfrow) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        *reinterpret_cast<float4*>(sfrow + 64 * pair + e) =
+                            make_float4(v0[e], v0[e + 1], v0[e + 2], v0[e + 3]);
+                        *reinterpret_cast<float4*>(sfrow + 64 * pair + 32 + e) =
+                            make_float4(v1[e], v1[e + 1], v1[e + 2], v1[e + 3]);
+                    }
+                } else if (!last) {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        pk[c] = __uint_as_float(tc::pack_bf16(v0[2 * c], v0[2 * c + 1]));
+                        pk[16 + c] = __uint_as_float(tc::pack_bf16(v1[2 * c], v1[2 * c + 1]));
+                    }
+                    tc::tmem_st32(tl + TM_SB + 32 * pair, pk);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) { v0[e] *= eLn; v1[e] *= eLn; }
+                    tc::tmem_st32(tl + TM_S + 64 * pair, v0);
+                    tc::tmem_st32(tl + TM_S + 64 * pair + 32, v1);
+                }
+            }
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            if (!last) tc::mbar_arrive(&bars[B_SREADY]);
+            COMBA_PHASE(3);
+            // out tile [token][value index] in two 64-wide 128B-swizzled boxes
+            if (issuer) tc::bulk_wait_read0();
+            tc::named_barrier(BAR_STATE, kStateThreads);
+            {
+                const uint32_t ot = sb + SM_OUT + (row >> 6) * 8192 + (row & 7) * 2;
+                const int oc = (row & 63) >> 3;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    tc::sts_u16(ot + tc::sw128(2 * c, oc), (unsigned short)(ob[c] & 0xffffu));
+                    tc::sts_u16(ot + tc::sw128(2 * c + 1, oc), (unsigned short)(ob[c] >> 16));
+                }
+            }
+            tc::fence_proxy_async_smem();
+            tc::named_barrier(BAR_STATE, kStateThreads);
+            if (issuer) {
+                tc::tma_store_4d(&tm_o, sm + SM_OUT, 0, h, t0, b);
+                tc::tma_store_4d(&tm_o, sm + SM_OUT + 8192, 64, h, t0, b);
+                tc::bulk_commit();
+            }
+            COMBA_PHASE(4);
+            // (D K)^T of the next chunk (MMA2 of this chunk has read the buffer)
+            if (!last) {
+                const bool okd = state_dk(n + 1);
+                if (!okd) fail(gabort);
+                if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, okd && *gabort == 0)) break;
+            }
+            COMBA_PHASE(5);
+        }
+        if (issuer) tc::bulk_wait0();
+    } else {
+        // =============================== prep group ================================
+        // Per chunk m (running one chunk ahead of the state group): gates, Gram, P, A,
+        // the inverse, Tc/Eb, Qh, W^T and U~^T (= X^T before MMA1), then, once the
+        // state group has released them, P, (D K)^T and -W.
+        const int pt = tid - kStateThreads;
+        const int prow = pt & 127, phalf = pt >> 7, pw = pt >> 5;
+        const bool issuer = (pt == 0);
+        bool gram_issued = false;   // Gram of the current chunk already issued (early)
+        float la_c = 0.f, bt_c = 0.f, la_n = 0.f, bt_n = 0.f;
+        if (pt < 64) {
+            la_c = gate(log_alpha, pt);
+            bt_c = gate(beta, pt);
+        }
+        if (issuer) {
+            load_kq(0);
+            if (nchunks > 1) load_kq(1);
+            load_v(0);
+        }
+        for (int m = 0; m < nchunks; ++m) {
+            const int t0 = m * kC;
+            const int stg = m & 1;
+            const uint32_t kq_a = sb + (stg ? SM_KQ1 : SM_KQ0);
+            const uint32_t txm = tmem + (stg ? TM_X1 : TM_X0);
+            const uint32_t tgm = stg ? TM_G1 : TM_G;    // Gram, then W^T, of this chunk
+            const bool last = (m + 1 == nchunks);
+            bool ok = (*gabort == 0);
+            // ---- Gram ([K;Q] K^T), unless it was issued during the previous chunk --------
+            if (issuer && !gram_issued) {
+                ok = ok && tc::mbar_wait(&bars[stg], (m >> 1) & 1, timeout_ns);
+                if (ok) {
+                    tc::tc_fence_after();
+                    tc::mma_ak_bk(tmem + tgm, kq_a, KQ_ATOM, kq_a, KQ_ATOM, ID_G, 8, 0);
+                    tc::mma_commit(&bars[B_GRAM]);
+                } else {
+                    fail(gabort);
+                }
+            }
+            gram_issued = false;
+            // ---- gates --------------------------------------------------------------------
+            if (pt < 64) {
+                if (!last) {
+                    la_n = gate(log_alpha, t0 + kC + pt);
+                    bt_n = gate(beta, t0 + kC + pt);
+                }
+                float x = la_c;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                if (lane == 31) tc::sts_f32(RED + 4u * pw, x);
+                tc::sts_f32(G2 + 4u * pt, x);
+            }
+            tc::named_barrier(BAR_PREP, kPrepThreads);
+            const float carry = tc::lds_f32(RED);
+            const float gL = carry + tc::lds_f32(RED + 4u);
+            const bool fast = gL > -80.f;
+            if (pt < 64) {
+                const float g = tc::lds_f32(G2 + 4u * pt) + (pt >= 32 ? carry : 0.f);
+                const float gp = g - la_c;
+                tc::sts_f32(BT + 4u * pt, bt_c);
+                tc::sts_f32(CS + 4u * pt, bt_c * __expf(gp));
+                tc::sts_f32(EG + 4u * pt, __expf(g));
+                tc::sts_f32(IEG + 4u * pt, fast ? __expf(-g) : 0.f);
+                tc::sts_f32(GP2 + 4u * pt, gp * kLog2e);
+                tc::sts_f32(G2 + 4u * pt, g * kLog2e);
+            }
+            ok = ok && tc::mbar_wait(&bars[B_GRAM], m & 1, timeout_ns) &&
+                 tc::mbar_wait(&bars[stg], (m >> 1) & 1, timeout_ns);
+            if (!ok) fail(gabort);
+            if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
+            tc::tc_fence_after();
+            COMBA_PHASE(8);
+            // ---- K K^T -> staging, A -> F1 --------------------------------------------
+            const int s0 = phalf * 32;
+            float gv[32];
+            tc::tmem_ld32(tl + tgm + phalf * 32, gv);
+            tc::tmem_ld_wait();
+            if (prow < 64) {
+                const int r = prow;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) tc::sts_f32(faddr(KKS, r, s0 + e), gv[e]);
                 if (fast) {
                     const float cr = tc::lds_f32(CS + 4u * r);
 #pragma unroll
@@ -415,44 +710,34 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         }
                     }
                 } else {
-                    a_row_exact(F1, tl + TM_G + half * 32, r, s0, tc::lds_f32(BT + 4u * r),
+                    a_row_exact(F1, tl + tgm + phalf * 32, r, s0, tc::lds_f32(BT + 4u * r),
                                 tc::lds_f32(GP2 + 4u * r), G2);
                 }
-                if (!last && tid < 64) {   // total log-decay of the next chunk
-                    const float w = warp_sum(la_n);
-                    if (lane == 0) tc::sts_f32(RED + 8u + 4u * warp, w);
-                }
             }
-            __syncthreads();
-            COMBA_PHASE(9);
-            if (row >= 64) {
-                // P in place over K K^T (row r, columns s0 .. s0 + 31)
-                const int r = row - 64;
+            tc::named_barrier(BAR_PREP, kPrepThreads);
+            // ---- P (in the staging buffer) and Qh  ||  diagonal inverse blocks ----------
+            if (prow >= 64) {
+                const int r = prow - 64;
                 const float er = tc::lds_f32(EG + 4u * r);
                 if (fast) {
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        const uint32_t pa = prow + tc::sw128(r, c);
-                        const float4 kk = tc::lds_f32x4(pa);
                         const float4 ig = tc::lds_f32x4(IEG + 4u * (s0 + 4 * c));
-                        const int s = s0 + 4 * c;
-                        float4 p;
-                        p.x = (s + 0 <= r) ? er * ig.x * fmaf(-dh, kk.x, gv[4 * c + 0]) : 0.f;
-                        p.y = (s + 1 <= r) ? er * ig.y * fmaf(-dh, kk.y, gv[4 * c + 1]) : 0.f;
-                        p.z = (s + 2 <= r) ? er * ig.z * fmaf(-dh, kk.z, gv[4 * c + 2]) : 0.f;
-                        p.w = (s + 3 <= r) ? er * ig.w * fmaf(-dh, kk.w, gv[4 * c + 3]) : 0.f;
-                        tc::sts_f32x4(pa, p);
+                        const float iv[4] = {ig.x, ig.y, ig.z, ig.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int s = s0 + 4 * c + e;
+                            const uint32_t pa = faddr(KKS, r, s);
+                            const float pv = er * iv[e] * fmaf(-dh, tc::lds_f32(pa), gv[4 * c + e]);
+                            tc::sts_f32(pa, (s <= r) ? pv : 0.f);
+                        }
                     }
                 } else {
-                    p_row_exact(prow, tl + TM_G + half * 32, r, s0, dh, G2);
+                    p_row_exact(KKS, tl + tgm + phalf * 32, r, s0, dh, G2);
                 }
-                // Qh (over Q) and (D K)^T for row r, key columns 64 half .. 64 half + 63
-                const float edr = tc::lds_f32(ED + 4u * r);
-                const uint32_t dka = sb + SM_DK + (r >> 5) * DKT_ATOM + (r & 3) * 4;
-                const uint32_t rc = (r & 31) >> 2;
 #pragma unroll 2
                 for (int c = 0; c < 8; ++c) {
-                    const uint32_t off = kq_a + half * KQ_ATOM + tc::sw128(r, c);
+                    const uint32_t off = kq_a + phalf * KQ_ATOM + tc::sw128(r, c);
                     const uint4 kw = tc::lds_u32x4(off);
                     uint4 qw = tc::lds_u32x4(off + 8192);
                     const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kw);
@@ -462,174 +747,97 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         const float2 kf = __bfloat1622float2(k2[e]);
                         const float2 qf = __bfloat1622float2(q2[e]);
                         q2[e] = __floats2bfloat162_rn(er * fmaf(-dh, kf.x, qf.x), er * fmaf(-dh, kf.y, qf.y));
-                        const int j = 64 * half + 8 * c + 2 * e;
-                        tc::sts_f32(dka + tc::sw128(j, rc), edr * kf.x);
-                        tc::sts_f32(dka + tc::sw128(j + 1, rc), edr * kf.y);
                     }
                     tc::sts_u32x4(off + 8192, qw);
                 }
             } else {
-                // warps 0, 1, 4, 5 -> diagonal blocks 0, 1, 2, 3
-                diag_block_inverse(F1, F2, (warp & 1) + 2 * half, lane);
+                diag_block_inverse(F1, F2, (pw & 1) + 2 * phalf, lane);
             }
-            __syncthreads();
-        }
-        COMBA_PHASE(2);
-
-        // ---- 4. off-diagonal blocks of the inverse -----------------------------------
-        offdiag_inverse(F1, F2, tid);
-        COMBA_PHASE(3);
-
-        // ---- 5. Tc, Eb (+ diag hi(beta)) over F1; diag lo(beta) ---------------------------
-        {
-            const int r = tid & 63, qq = tid >> 6;   // row, quarter of the columns
-#pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                const int c = 2 * qq + c2;
-                float tcv[8], ebv[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int s = c * 8 + e;
-                    const float t = tc::lds_f32(faddr(F2, r, s));
-                    const float cv = tc::lds_f32(CS + 4u * s), bv = tc::lds_f32(BT + 4u * s);
-                    tcv[e] = (s <= r) ? t * cv : 0.f;
-                    ebv[e] = (s < r) ? t * bv : ((s == r) ? bv : 0.f);
-                }
-                tc::sts_u32x4(F1 + tc::sw128(r, c), pack8_bf16(tcv));
-                tc::sts_u32x4(F1 + 8192 + tc::sw128(r, c), pack8_bf16(ebv));
-            }
-            if (tid < 64) {
-                const float bv = tc::lds_f32(BT + 4u * tid);
+            tc::named_barrier(BAR_PREP, kPrepThreads);
+            COMBA_PHASE(9);
+            // ---- off-diagonal blocks of the inverse, written out as Tc / Eb ----------------
+            offdiag_inverse(F1, F2, pt, CS, BT);
+            COMBA_PHASE(10);
+            if (pt < 64) {   // diag(lo(beta))
+                const float bv = tc::lds_f32(BT + 4u * pt);
                 const float bh = __bfloat162float(__float2bfloat16_rn(bv));
                 const __nv_bfloat16 lo = __float2bfloat16_rn(bv - bh);
-                tc::sts_u16(sb + SM_BLO + tc::sw128(tid, tid >> 3) + (tid & 7) * 2,
+                tc::sts_u16(sb + SM_BLO + tc::sw128(pt, pt >> 3) + (pt & 7) * 2,
                             *reinterpret_cast<const unsigned short*>(&lo));
             }
-        }
-        tc::fence_proxy_async_smem();
-        COMBA_PHASE(4);
-
-        // ---- 6. W^T = K^T Tc^T;  X^T = V^T Eb^T + V^T diag(lo)^T ---------------------------
-        if (!cta_wait(&bars[2], n & 1, timeout_ns, abort_flag)) { ok = false; break; }
-        if (tid == 0) {
-            tc::tc_fence_after();
-            tc::mma_amn_bk(tmem + TM_G, kq_a, KQ_ATOM, F1, ID_WN, 4, 0);
-            tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, F1 + 8192, ID_WN, 4, 0);
-            tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
-            tc::mma_commit(&bars[3]);
-        }
-        if (!cta_wait(&bars[3], mma_phase, timeout_ns, abort_flag)) { ok = false; break; }
-        mma_phase ^= 1;
-        tc::tc_fence_after();
-        if (tid == 0 && !last) {
             tc::fence_proxy_async_smem();
-            load_v(n + 1);
-        }
-        COMBA_PHASE(5);
-
-        // ---- 7. -W operand (MN-major: row j holds -W[0..63][j]) ------------------------------
-        {
-            float w[32];
-            tc::tmem_ld32(tl + TM_G + half * 32, w);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) w[e] = -w[e];
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4)
-                tc::sts_u32x4(sb + SM_W + tc::sw128(row, half * 4 + c4), pack8_bf16(w + c4 * 8));
-        }
-        tc::fence_proxy_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-        COMBA_PHASE(6);
-
-        // ---- 8. X^T += S (-W)^T, O^T = S Qh^T; S += X^T (D K), O^T += X^T P^T; next Gram ------
-        if (tid == 0) {
-            tc::tc_fence_after();
-            tc::mma_ak_bmn(tmem + TM_X, sb + SM_S, OP_ATOM, sb + SM_W, 8192, ID_SW, 8, 8, 1);
-            tc::mma_commit(&bars[4]);
-            tc::mma_ak_bk(tmem + TM_O, sb + SM_S, OP_ATOM, kq_a + 8192, KQ_ATOM, ID_SQ, 8, 0);
-            bool good = tc::mbar_wait(&bars[4], mma1_phase, timeout_ns);
-            COMBA_PHASE(10);
-            if (good) {
-                tc::tc_fence_after();
-                tc::mma_tf32_ta_bk(tmem + TM_S, tmem + TM_X, sb + SM_DK, DKT_ATOM, ID_SU, 8, 1);
-                tc::mma_tf32_ta_bk(tmem + TM_O, tmem + TM_X, sb + SM_P, F32_ATOM, ID_XP, 8, 1);
-                tc::mma_commit(&bars[3]);
-                COMBA_PHASE(11);
-                if (!last) good = issue_gram(n + 1);          // TM_G is free again
-                COMBA_PHASE(12);
-            }
-            if (!good) {
-                *abort_flag = 1;
-                latch_status(-4);
-            }
-        }
-        mma1_phase ^= 1;
-        if (!cta_wait(&bars[3], mma_phase, timeout_ns, abort_flag)) { ok = false; break; }
-        mma_phase ^= 1;
-        tc::tc_fence_after();
-        if (tid == 0 && n + 2 < nchunks) {   // stage st is free: its Qh was read by the MMAs above
-            tc::fence_proxy_async_smem();
-            load_kq(n + 2);
-        }
-        COMBA_PHASE(7);
-
-        // ---- 9. S -> bf16 operand, decay for the next chunk; output tile -------------------
-        {
-            const float eLn = last ? 1.f : __expf(tc::lds_f32(RED + 8u) + tc::lds_f32(RED + 12u));
-            float* sfrow = (last && S_final)
-                               ? S_final + ((size_t)blockIdx.x * kD + row) * kD + half * 64
-                               : nullptr;
-            const uint32_t sbase = sb + SM_S + half * OP_ATOM;
-#pragma unroll 1
-            for (int part = 0; part < 2; ++part) {
-                float v[32];
-                tc::tmem_ld32(tl + TM_S + half * 64 + part * 32, v);
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4)
-                    tc::sts_u32x4(sbase + tc::sw128(row, part * 4 + c4), pack8_bf16(v + c4 * 8));
-                if (sfrow) {
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4*>(sfrow + part * 32 + e) =
-                            make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                } else if (!last) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] *= eLn;
-                    tc::tmem_st32(tl + TM_S + half * 64 + part * 32, v);
+            tc::named_barrier(BAR_PREP, kPrepThreads);
+            COMBA_PHASE(11);
+            // ---- W^T = K^T Tc^T;  X^T = U~^T = V^T Eb^T + V^T diag(lo)^T --------------------
+            if (issuer) {
+                ok = ok && tc::mbar_wait(&bars[B_V], m & 1, timeout_ns);
+                if (ok) {
+                    tc::tc_fence_after();
+                    tc::mma_amn_bk(tmem + tgm, kq_a, KQ_ATOM, F1, ID_WN, 4, 0);
+                    tc::mma_amn_bk(txm, sb + SM_V, V_ATOM, F1 + 8192, ID_WN, 4, 0);
+                    tc::mma_amn_bk(txm, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
+                    tc::mma_commit(&bars[B_WN]);
+                    // next chunk's Gram into the other buffer, if its q/k tiles are in
+                    const int m1 = m + 1;
+                    if (!last && tc::mbar_try_wait(&bars[m1 & 1], (m1 >> 1) & 1)) {
+                        const uint32_t kq1 = sb + ((m1 & 1) ? SM_KQ1 : SM_KQ0);
+                        tc::tc_fence_after();
+                        tc::mma_ak_bk(tmem + ((m1 & 1) ? TM_G1 : TM_G), kq1, KQ_ATOM, kq1, KQ_ATOM,
+                                      ID_G, 8, 0);
+                        tc::mma_commit(&bars[B_GRAM]);
+                        gram_issued = true;
+                    }
+                } else {
+                    fail(gabort);
                 }
             }
-            // O^T row i (value index) -> out tile [token][i], two 64-wide boxes
-            const uint32_t ot = sb + SM_DK + (row >> 6) * 8192 + (row & 7) * 2;
-            const int oc = (row & 63) >> 3;
-            float o[32];
-            tc::tmem_ld32(tl + TM_O + half * 32, o);
-            tc::tmem_ld_wait();
+            // ---- once MMA2 of the previous chunk is done: P -> operand ------------------------
+            ok = ok && (m == 0 || tc::mbar_wait(&bars[B_MMA2], (m - 1) & 1, timeout_ns));
+            if (!ok) fail(gabort);
+            if (prow >= 64) {
+                const int r = prow - 64;
+                const uint32_t prw = sb + SM_P + phalf * F32_ATOM;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const __nv_bfloat16 ob = __float2bfloat16_rn(o[e]);
-                tc::sts_u16(ot + tc::sw128(half * 32 + e, oc), *reinterpret_cast<const unsigned short*>(&ob));
+                for (int c = 0; c < 8; ++c) {
+                    float4 p;
+                    p.x = tc::lds_f32(faddr(KKS, r, s0 + 4 * c + 0));
+                    p.y = tc::lds_f32(faddr(KKS, r, s0 + 4 * c + 1));
+                    p.z = tc::lds_f32(faddr(KKS, r, s0 + 4 * c + 2));
+                    p.w = tc::lds_f32(faddr(KKS, r, s0 + 4 * c + 3));
+                    tc::sts_f32x4(prw + tc::sw128(r, c), p);
+                }
             }
-            tc::tmem_st_wait();
+            COMBA_PHASE(12);
+            // ---- once W^T is in and MMA1 of the previous chunk is done: -W operand ------------
+            ok = ok && tc::mbar_wait(&bars[B_WN], m & 1, timeout_ns) &&
+                 (m == 0 || tc::mbar_wait(&bars[B_MMA1], (m - 1) & 1, timeout_ns));
+            if (!ok) fail(gabort);
+            tc::tc_fence_after();
+            if (issuer && ok && !last) {   // V was read by the W/X MMAs above
+                tc::fence_proxy_async_smem();
+                load_v(m + 1);
+            }
+            {
+                float w[32];
+                tc::tmem_ld32(tl + tgm + phalf * 32, w);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) w[e] = -w[e];
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4)
+                    tc::sts_u32x4(sb + SM_W + tc::sw128(prow, phalf * 4 + c4), pack8_bf16(w + c4 * 8));
+            }
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
+            if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
+            tc::mbar_arrive(&bars[B_PREP]);
+            la_c = la_n;
+            bt_c = bt_n;
+            COMBA_PHASE(13);
         }
-        tc::fence_proxy_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc::tma_store_4d(&tm_o, sm + SM_DK, 0, h, t0, b);
-            tc::tma_store_4d(&tm_o, sm + SM_DK + 8192, 64, h, t0, b);
-            tc::bulk_commit();
-        }
-        la_c = la_n;
-        bt_c = bt_n;
-        COMBA_PHASE(8);
     }
-
     COMBA_PHASE_END();
-    if (tid == 0) tc::bulk_wait0();
-    if (!ok) tc::mbar_wait(&bars[3], mma_phase, timeout_ns);
+
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, TM_COLS);

@@ -13,9 +13,10 @@ __device__ int g_status = 0;
 
 __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0, code); }
 
-// Optional phase tracing (compile with -DCOMBA_TRACE_PHASES): thread 0 of CTA 0
-// accumulates clock64() deltas between consecutive COMBA_PHASE marks in
-// registers and adds them to a device array at COMBA_PHASE_END.  Off by
+// Optional phase tracing (compile with -DCOMBA_TRACE_PHASES): threads 0 and 128
+// of CTA 0 accumulate clock64() deltas between consecutive COMBA_PHASE marks in
+// registers (each thread its own slots) and add them to a device array at
+// COMBA_PHASE_END.  Off by
 // default; the marks then compile to nothing.
 #ifdef COMBA_TRACE_PHASES
 __device__ unsigned long long g_phase_cycles[16];
@@ -30,7 +31,7 @@ __device__ unsigned long long g_phase_cycles[16];
     } while (0)
 #define COMBA_PHASE_END()                                                     \
     do {                                                                      \
-        if (blockIdx.x == 0 && threadIdx.x == 0)                              \
+        if (blockIdx.x == 0 && (threadIdx.x == 0 || threadIdx.x == 128))      \
             for (int comba_i = 0; comba_i < 16; ++comba_i)                    \
                 g_phase_cycles[comba_i] += comba_phase_acc[comba_i];          \
     } while (0)

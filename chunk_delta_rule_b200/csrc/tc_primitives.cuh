@@ -90,13 +90,28 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps (issuing nothing) until
+// the phase completes or about `hint_ns` pass.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        "selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns) : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: false if the phase has not completed after `timeout_ns`.
+// Waiting threads sleep in the barrier instead of spinning, so they leave
+// issue slots to the other warps of the SM.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
-        for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
         if (globaltimer_ns() - t0 > timeout_ns) return false;
     }
 }
@@ -349,6 +364,26 @@ __device__ __forceinline__ void mma_sync_tf32(float (&d)[4], const uint32_t (&a)
 
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier that also ORs a per-thread failure flag across the
+// participating threads: returns true only if no thread reported failure, so
+// every thread of the group takes the same decision.
+__device__ __forceinline__ bool named_barrier_all_ok(int id, int nthreads, bool ok) {
+    uint32_t any_fail;
+    asm volatile(
+        "{\n"
+        ".reg .pred pf, pa;\n"
+        "setp.eq.u32 pf, %1, 0;\n"
+        "bar.red.or.pred pa, %2, %3, pf;\n"
+        "selp.u32 %0, 1, 0, pa;\n"
+        "}\n"
+        : "=r"(any_fail) : "r"((uint32_t)ok), "r"(id), "r"(nthreads) : "memory");
+    return any_fail == 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // ---------------------------------------------------------------- shared memory
