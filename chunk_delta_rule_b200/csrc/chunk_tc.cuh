@@ -64,9 +64,9 @@ constexpr uint32_t SM_KQ0 = 0;        // [K;Q] stage 0: 2 K-atoms x 128 rows x 1
 constexpr uint32_t SM_KQ1 = 32768;    // stage 1
 constexpr uint32_t SM_V = 65536;      // V: 2 dv-atoms x 64 tokens x 128 B
 constexpr uint32_t SM_W = 81920;      // -W bf16, MN-major: 128 rows (j) x 64 tokens
-constexpr uint32_t SM_P = 98304;      // P fp32, K-major: 2 atoms (32 s) x 64 rows
-constexpr uint32_t SM_DK = 114688;    // (D K)^T fp32, K-major: 2 atoms (32 r) x 128 rows (j)
-constexpr uint32_t SM_KK = 147456;    // fp32 64x64 (fidx): K K^T, then P before its copy to SM_P
+constexpr uint32_t SM_P0 = 98304;     // P fp32, K-major: 2 atoms (32 s) x 64 rows; even chunks
+constexpr uint32_t SM_P1 = 114688;    // odd chunks (K K^T is staged here first, P formed in place)
+constexpr uint32_t SM_DK = 131072;    // (D K)^T fp32, K-major: 2 atoms (32 r) x 128 rows (j)
 constexpr uint32_t SM_F1 = 163840;    // fp32 64x64: A; then Tc (bf16) | Eb (bf16)
 constexpr uint32_t SM_F2 = 180224;    // fp32 64x64: Tinv (upper blocks: scratch)
 constexpr uint32_t SM_BLO = 196608;   // bf16 64x64 K-major: diag(lo(beta)), zero elsewhere
@@ -311,8 +311,8 @@ __device__ __noinline__ void a_row_exact(uint32_t F1, uint32_t gram_taddr, int r
     }
 }
 
-__device__ __noinline__ void p_row_exact(uint32_t KK, uint32_t gram_taddr, int r, int s0, float dh,
-                                         uint32_t G2) {
+__device__ __noinline__ void p_row_exact(uint32_t prow, uint32_t gram_taddr, int r, int s0,
+                                         float dh, uint32_t G2) {
     float gv[32];
     tc::tmem_ld32(gram_taddr, gv);
     tc::tmem_ld_wait();
@@ -320,12 +320,11 @@ __device__ __noinline__ void p_row_exact(uint32_t KK, uint32_t gram_taddr, int r
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
         const int s = s0 + e;
-        const uint32_t pa = faddr(KK, r, s);
+        const uint32_t pa = prow + tc::sw128(r, e >> 2) + 4u * (e & 3);
         const float v = exp2f(gr - tc::lds_f32(G2 + 4u * s)) * fmaf(-dh, tc::lds_f32(pa), gv[e]);
         tc::sts_f32(pa, (s <= r) ? v : 0.f);
     }
 }
-
 
 __device__ __forceinline__ void fail(volatile int* gabort) {
     *gabort = 1;
@@ -354,13 +353,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t RED = G2 + 1792;          // [0..1] scan carries
     const uint32_t SRED = G2 + 1936;         // state group: [0..1] scan carries
     const uint32_t SED = G2 + 2048;          // state group: e^{g_L - g_r} of the next chunk
-    // barriers: q/k stages, v, gram, wn, prep ready, mma1, mma2, state ready
+    // barriers: q/k stages, v, gram, wn, prep ready, mma1 (X), mma2, state ready,
+    // mma1 (O), and per P buffer: the MMA2 that read it is done
     enum { B_KQ0 = 0, B_KQ1 = 1, B_V = 2, B_GRAM = 3, B_WN = 4, B_PREP = 5, B_MMA1 = 6, B_MMA2 = 7,
-           B_SREADY = 8 };
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 1856);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+           B_SREADY = 8, B_MMA1B = 9, B_PBUF0 = 10, B_PBUF1 = 11, NBARS = 12 };
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 2560);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
     volatile int* gabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    const uint32_t F1 = sb + SM_F1, F2 = sb + SM_F2, KKS = sb + SM_KK;
+    const uint32_t F1 = sb + SM_F1, F2 = sb + SM_F2;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.x / H, h = blockIdx.x % H;
@@ -369,7 +369,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t trow = (uint32_t)((warp & 3) * 32) << 16;
 
     if (tid == 0) {
-        for (int i = 0; i < 9; ++i)
+        for (int i = 0; i < NBARS; ++i)
             tc::mbar_init(&bars[i], i == B_PREP ? kPrepThreads : (i == B_SREADY ? kStateThreads : 1));
         *gabort = 0;
         tc::fence_mbar_init();
@@ -513,13 +513,21 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     tc::mma_bf16_ta_bmn(txn, tmem + TM_SB, sb + SM_W, 8192, ID_SW, 8, 1);
                     tc::mma_commit(&bars[B_MMA1]);
                     tc::mma_bf16_ta_bk(tmem + TM_O, tmem + TM_SB, kq_a + 8192, KQ_ATOM, ID_SQ, 8, 0);
+                    tc::mma_commit(&bars[B_MMA1B]);
                     ok = tc::mbar_wait(&bars[B_MMA1], n & 1, timeout_ns);
                     COMBA_PHASE(1);
                     if (ok) {
                         tc::tc_fence_after();
                         tc::mma_tf32_ta_bk(tmem + TM_S, txn, sb + SM_DK, DKT_ATOM, ID_SU, 8, 1);
-                        tc::mma_tf32_ta_bk(tmem + TM_O, txn, sb + SM_P, F32_ATOM, ID_XP, 8, 1);
+                        tc::mma_tf32_ta_bk(tmem + TM_O, txn, sb + (stg ? SM_P1 : SM_P0), F32_ATOM, ID_XP, 8, 1);
                         tc::mma_commit(&bars[B_MMA2]);
+                        tc::mma_commit(&bars[stg ? B_PBUF1 : B_PBUF0]);
+                        // stage stg is free once S Qh^T has read Qh (K: read by Gram, W^T, D K)
+                        ok = tc::mbar_wait(&bars[B_MMA1B], n & 1, timeout_ns);
+                        if (ok && n + 2 < nchunks) {
+                            tc::fence_proxy_async_smem();
+                            load_kq(n + 2);
+                        }
                     }
                 }
                 if (!ok) fail(gabort);
@@ -529,20 +537,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
             tc::tc_fence_after();
             COMBA_PHASE(2);
-            if (issuer && n + 2 < nchunks) {   // stage stg is free: its Qh was read by MMA1
-                tc::fence_proxy_async_smem();
-                load_kq(n + 2);
-            }
             // O^T row (value index) -> bf16 pairs of tokens, read before S is released;
             // the first half of S is loaded in the same batch
             uint32_t ob[32];
-            float v0[32], v1[32];
             {
                 float o0[32], o1[32];
                 tc::tmem_ld32(tl + TM_O, o0);
                 tc::tmem_ld32(tl + TM_O + 32, o1);
-                tc::tmem_ld32(tl + TM_S, v0);
-                tc::tmem_ld32(tl + TM_S + 32, v1);
                 tc::tmem_ld_wait();
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
@@ -554,11 +555,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             float* sfrow = (last && S_final) ? S_final + ((size_t)blockIdx.x * kD + row) * kD : nullptr;
 #pragma unroll 1
             for (int pair = 0; pair < 2; ++pair) {
-                if (pair == 1) {
-                    tc::tmem_ld32(tl + TM_S + 64, v0);
-                    tc::tmem_ld32(tl + TM_S + 96, v1);
-                    tc::tmem_ld_wait();
-                }
+                float v0[32], v1[32];
+                tc::tmem_ld32(tl + TM_S + 64 * pair, v0);
+                tc::tmem_ld32(tl + TM_S + 64 * pair + 32, v1);
+                tc::tmem_ld_wait();
                 float pk[32];
                 if (sfrow) {
 #pragma unroll
@@ -585,7 +585,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::tc_fence_before();
             if (!last) tc::mbar_arrive(&bars[B_SREADY]);
             COMBA_PHASE(3);
-            // out tile [token][value index] in two 64-wide 128B-swizzled boxes
+            // out tile [token][value index] in two 64-wide 128B-swizzled boxes, TMA store
             if (issuer) tc::bulk_wait_read0();
             tc::named_barrier(BAR_STATE, kStateThreads);
             {
@@ -688,15 +688,23 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
             tc::tc_fence_after();
             COMBA_PHASE(8);
-            // ---- K K^T -> staging, A -> F1 --------------------------------------------
+            // ---- K K^T -> P buffer of this chunk (once MMA2 of chunk m-2 has read it), A -> F1
+            if (m >= 2) {
+                const bool okp = tc::mbar_wait(&bars[stg ? B_PBUF1 : B_PBUF0], ((m - 2) >> 1) & 1, timeout_ns);
+                if (!okp) fail(gabort);
+                if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, okp && *gabort == 0)) break;
+            }
             const int s0 = phalf * 32;
+            const uint32_t prow_base = sb + (stg ? SM_P1 : SM_P0) + phalf * F32_ATOM;
             float gv[32];
             tc::tmem_ld32(tl + tgm + phalf * 32, gv);
             tc::tmem_ld_wait();
             if (prow < 64) {
                 const int r = prow;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) tc::sts_f32(faddr(KKS, r, s0 + e), gv[e]);
+                for (int c = 0; c < 8; ++c)
+                    tc::sts_f32x4(prow_base + tc::sw128(r, c),
+                                  make_float4(gv[4 * c], gv[4 * c + 1], gv[4 * c + 2], gv[4 * c + 3]));
                 if (fast) {
                     const float cr = tc::lds_f32(CS + 4u * r);
 #pragma unroll
@@ -715,25 +723,26 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
             tc::named_barrier(BAR_PREP, kPrepThreads);
-            // ---- P (in the staging buffer) and Qh  ||  diagonal inverse blocks ----------
+            // ---- P (in place over K K^T) and Qh  ||  diagonal inverse blocks -------------
             if (prow >= 64) {
                 const int r = prow - 64;
                 const float er = tc::lds_f32(EG + 4u * r);
                 if (fast) {
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
+                        const uint32_t pa = prow_base + tc::sw128(r, c);
+                        const float4 kk = tc::lds_f32x4(pa);
                         const float4 ig = tc::lds_f32x4(IEG + 4u * (s0 + 4 * c));
-                        const float iv[4] = {ig.x, ig.y, ig.z, ig.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int s = s0 + 4 * c + e;
-                            const uint32_t pa = faddr(KKS, r, s);
-                            const float pv = er * iv[e] * fmaf(-dh, tc::lds_f32(pa), gv[4 * c + e]);
-                            tc::sts_f32(pa, (s <= r) ? pv : 0.f);
-                        }
+                        const int s = s0 + 4 * c;
+                        float4 p;
+                        p.x = (s + 0 <= r) ? er * ig.x * fmaf(-dh, kk.x, gv[4 * c + 0]) : 0.f;
+                        p.y = (s + 1 <= r) ? er * ig.y * fmaf(-dh, kk.y, gv[4 * c + 1]) : 0.f;
+                        p.z = (s + 2 <= r) ? er * ig.z * fmaf(-dh, kk.z, gv[4 * c + 2]) : 0.f;
+                        p.w = (s + 3 <= r) ? er * ig.w * fmaf(-dh, kk.w, gv[4 * c + 3]) : 0.f;
+                        tc::sts_f32x4(pa, p);
                     }
                 } else {
-                    p_row_exact(KKS, tl + tgm + phalf * 32, r, s0, dh, G2);
+                    p_row_exact(prow_base, tl + tgm + phalf * 32, r, s0, dh, G2);
                 }
 #pragma unroll 2
                 for (int c = 0; c < 8; ++c) {
@@ -789,22 +798,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 } else {
                     fail(gabort);
-                }
-            }
-            // ---- once MMA2 of the previous chunk is done: P -> operand ------------------------
-            ok = ok && (m == 0 || tc::mbar_wait(&bars[B_MMA2], (m - 1) & 1, timeout_ns));
-            if (!ok) fail(gabort);
-            if (prow >= 64) {
-                const int r = prow - 64;
-                const uint32_t prw = sb + SM_P + phalf * F32_ATOM;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float4 p;
-                    p.x = tc::lds_f32(faddr(KKS, r, s0 + 4 * c + 0));
-                    p.y = tc::lds_f32(faddr(KKS, r, s0 + 4 * c + 1));
-                    p.z = tc::lds_f32(faddr(KKS, r, s0 + 4 * c + 2));
-                    p.w = tc::lds_f32(faddr(KKS, r, s0 + 4 * c + 3));
-                    tc::sts_f32x4(prw + tc::sw128(r, c), p);
                 }
             }
             COMBA_PHASE(12);
