@@ -353,10 +353,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t RED = G2 + 1792;          // [0..1] scan carries
     const uint32_t SRED = G2 + 1936;         // state group: [0..1] scan carries
     const uint32_t SED = G2 + 2048;          // state group: e^{g_L - g_r} of the next chunk
-    // barriers: q/k stages, v, gram, wn, prep ready, mma1 (X), mma2, state ready,
-    // mma1 (O), and per P buffer: the MMA2 that read it is done
+    // barriers: q/k stages, v, gram, wn, prep ready, mma1 (X), mma2, mma1 (O), and
+    // per P buffer: the MMA2 that read it is done.  Each is arrived on once per
+    // phase (by a commit, a TMA transaction count or one elected thread after its
+    // group's named barrier): many arrivals on one barrier serialise in the
+    // shared-memory pipe and hold up the group's next shared-memory accesses.
     enum { B_KQ0 = 0, B_KQ1 = 1, B_V = 2, B_GRAM = 3, B_WN = 4, B_PREP = 5, B_MMA1 = 6, B_MMA2 = 7,
-           B_SREADY = 8, B_MMA1B = 9, B_PBUF0 = 10, B_PBUF1 = 11, NBARS = 12 };
+           B_MMA1B = 8, B_PBUF0 = 9, B_PBUF1 = 10, NBARS = 11 };
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 2560);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
     volatile int* gabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -370,7 +373,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     if (tid == 0) {
         for (int i = 0; i < NBARS; ++i)
-            tc::mbar_init(&bars[i], i == B_PREP ? kPrepThreads : (i == B_SREADY ? kStateThreads : 1));
+            tc::mbar_init(&bars[i], 1);
         *gabort = 0;
         tc::fence_mbar_init();
         tc::prefetch_tmap(&tm_q);
@@ -492,8 +495,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::tmem_st_wait();
             tc::tc_fence_before();
             if (!ok) fail(gabort);
+            // the issuer's first MMAs follow this barrier: the S copies are in TMEM
             ok = tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok);
-            tc::mbar_arrive(&bars[B_SREADY]);
         }
         float la_n = 0.f;
         for (int n = 0; n < nchunks && ok; ++n) {
@@ -504,9 +507,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const bool last = (n + 1 == nchunks);
             if (tid < 64 && !last) la_n = gate(log_alpha, t0 + kC + tid);   // next chunk's decay
             ok = (*gabort == 0);
-            if (issuer) {
-                ok = ok && tc::mbar_wait(&bars[B_SREADY], n & 1, timeout_ns) &&
-                     tc::mbar_wait(&bars[B_PREP], n & 1, timeout_ns);
+            if (warp == 0) {   // MMA issue: the whole warp, one elected lane
+                ok = ok && tc::mbar_wait(&bars[B_PREP], n & 1, timeout_ns);
                 COMBA_PHASE(0);
                 if (ok) {
                     tc::tc_fence_after();
@@ -524,7 +526,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         tc::mma_commit(&bars[stg ? B_PBUF1 : B_PBUF0]);
                         // stage stg is free once S Qh^T has read Qh (K: read by Gram, W^T, D K)
                         ok = tc::mbar_wait(&bars[B_MMA1B], n & 1, timeout_ns);
-                        if (ok && n + 2 < nchunks) {
+                        if (ok && n + 2 < nchunks && lane == 0) {
                             tc::fence_proxy_async_smem();
                             load_kq(n + 2);
                         }
@@ -583,9 +585,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             tc::tmem_st_wait();
             tc::tc_fence_before();
-            if (!last) tc::mbar_arrive(&bars[B_SREADY]);
             COMBA_PHASE(3);
-            // out tile [token][value index] in two 64-wide 128B-swizzled boxes, TMA store
+            // out tile [token][value index] in two 64-wide 128B-swizzled boxes, TMA store.
+            // This barrier also hands the new S copies to the issuer's next MMAs.
             if (issuer) tc::bulk_wait_read0();
             tc::named_barrier(BAR_STATE, kStateThreads);
             {
@@ -612,6 +614,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, okd && *gabort == 0)) break;
             }
             COMBA_PHASE(5);
+            COMBA_ITER_NEXT();
         }
         if (issuer) tc::bulk_wait0();
     } else {
@@ -642,7 +645,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const bool last = (m + 1 == nchunks);
             bool ok = (*gabort == 0);
             // ---- Gram ([K;Q] K^T), unless it was issued during the previous chunk --------
-            if (issuer && !gram_issued) {
+            if (pw == 0 && !gram_issued) {
                 ok = ok && tc::mbar_wait(&bars[stg], (m >> 1) & 1, timeout_ns);
                 if (ok) {
                     tc::tc_fence_after();
@@ -669,6 +672,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::sts_f32(G2 + 4u * pt, x);
             }
             tc::named_barrier(BAR_PREP, kPrepThreads);
+            COMBA_PHASE(22);
             const float carry = tc::lds_f32(RED);
             const float gL = carry + tc::lds_f32(RED + 4u);
             const bool fast = gL > -80.f;
@@ -682,12 +686,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::sts_f32(GP2 + 4u * pt, gp * kLog2e);
                 tc::sts_f32(G2 + 4u * pt, g * kLog2e);
             }
+            COMBA_PHASE(23);
             ok = ok && tc::mbar_wait(&bars[B_GRAM], m & 1, timeout_ns) &&
                  tc::mbar_wait(&bars[stg], (m >> 1) & 1, timeout_ns);
+            COMBA_PHASE(24);
             if (!ok) fail(gabort);
             if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
             tc::tc_fence_after();
-            COMBA_PHASE(8);
+            COMBA_PHASE(16);
             // ---- K K^T -> P buffer of this chunk (once MMA2 of chunk m-2 has read it), A -> F1
             if (m >= 2) {
                 const bool okp = tc::mbar_wait(&bars[stg ? B_PBUF1 : B_PBUF0], ((m - 2) >> 1) & 1, timeout_ns);
@@ -722,6 +728,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                 tc::lds_f32(GP2 + 4u * r), G2);
                 }
             }
+            COMBA_PHASE(31);
             tc::named_barrier(BAR_PREP, kPrepThreads);
             // ---- P (in place over K K^T) and Qh  ||  diagonal inverse blocks -------------
             if (prow >= 64) {
@@ -762,11 +769,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             } else {
                 diag_block_inverse(F1, F2, (pw & 1) + 2 * phalf, lane);
             }
+            COMBA_PHASE(30);
             tc::named_barrier(BAR_PREP, kPrepThreads);
-            COMBA_PHASE(9);
+            COMBA_PHASE(17);
             // ---- off-diagonal blocks of the inverse, written out as Tc / Eb ----------------
             offdiag_inverse(F1, F2, pt, CS, BT);
-            COMBA_PHASE(10);
+            COMBA_PHASE(18);
             if (pt < 64) {   // diag(lo(beta))
                 const float bv = tc::lds_f32(BT + 4u * pt);
                 const float bh = __bfloat162float(__float2bfloat16_rn(bv));
@@ -776,16 +784,18 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             tc::fence_proxy_async_smem();
             tc::named_barrier(BAR_PREP, kPrepThreads);
-            COMBA_PHASE(11);
+            COMBA_PHASE(19);
             // ---- W^T = K^T Tc^T;  X^T = U~^T = V^T Eb^T + V^T diag(lo)^T --------------------
-            if (issuer) {
+            if (pw == 0) {   // MMA issue: the whole warp, one elected lane
                 ok = ok && tc::mbar_wait(&bars[B_V], m & 1, timeout_ns);
+                COMBA_PHASE(25);
                 if (ok) {
                     tc::tc_fence_after();
                     tc::mma_amn_bk(tmem + tgm, kq_a, KQ_ATOM, F1, ID_WN, 4, 0);
                     tc::mma_amn_bk(txm, sb + SM_V, V_ATOM, F1 + 8192, ID_WN, 4, 0);
                     tc::mma_amn_bk(txm, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
                     tc::mma_commit(&bars[B_WN]);
+                    COMBA_PHASE(26);
                     // next chunk's Gram into the other buffer, if its q/k tiles are in
                     const int m1 = m + 1;
                     if (!last && tc::mbar_try_wait(&bars[m1 & 1], (m1 >> 1) & 1)) {
@@ -800,10 +810,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     fail(gabort);
                 }
             }
-            COMBA_PHASE(12);
+            COMBA_PHASE(20);
             // ---- once W^T is in and MMA1 of the previous chunk is done: -W operand ------------
-            ok = ok && tc::mbar_wait(&bars[B_WN], m & 1, timeout_ns) &&
-                 (m == 0 || tc::mbar_wait(&bars[B_MMA1], (m - 1) & 1, timeout_ns));
+            ok = ok && tc::mbar_wait(&bars[B_WN], m & 1, timeout_ns);
+            COMBA_PHASE(27);
+            ok = ok && (m == 0 || tc::mbar_wait(&bars[B_MMA1], (m - 1) & 1, timeout_ns));
+            COMBA_PHASE(28);
             if (!ok) fail(gabort);
             tc::tc_fence_after();
             if (issuer && ok && !last) {   // V was read by the W/X MMAs above
@@ -822,11 +834,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             tc::fence_proxy_async_smem();
             tc::tc_fence_before();
+            COMBA_PHASE(29);
             if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
-            tc::mbar_arrive(&bars[B_PREP]);
+            if (issuer) tc::mbar_arrive(&bars[B_PREP]);
             la_c = la_n;
             bt_c = bt_n;
-            COMBA_PHASE(13);
+            COMBA_PHASE(21);
+            COMBA_ITER_NEXT();
         }
     }
     COMBA_PHASE_END();

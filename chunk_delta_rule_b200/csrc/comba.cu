@@ -203,11 +203,19 @@ extern "C" int comba_version(void) { return 100; }
 
 #ifdef COMBA_TRACE_PHASES
 // Tracing builds only: copies and clears the per-phase cycle counters.
-extern "C" int comba_trace_read_phases(unsigned long long* host16) {
+extern "C" int comba_trace_read_phases(unsigned long long* host_slots) {
     if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;
-    if (cudaMemcpyFromSymbol(host16, comba::g_phase_cycles, 16 * sizeof(unsigned long long)) != cudaSuccess)
+    if (cudaMemcpyFromSymbol(host_slots, comba::g_phase_cycles,
+                             COMBA_TRACE_SLOTS * sizeof(unsigned long long)) != cudaSuccess)
         return COMBA_ECUDA;
-    static const unsigned long long zeros[16] = {};
+    static const unsigned long long zeros[COMBA_TRACE_SLOTS] = {};
     return cudaMemcpyToSymbol(comba::g_phase_cycles, zeros, sizeof(zeros)) == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
+}
+
+// Tracing builds only: absolute mark timestamps of one loop iteration, two threads.
+extern "C" int comba_trace_read_ts(long long* host_2slots) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;
+    return cudaMemcpyFromSymbol(host_2slots, comba::g_phase_ts, 2 * COMBA_TRACE_SLOTS * sizeof(long long)) ==
+                   cudaSuccess ? COMBA_OK : COMBA_ECUDA;
 }
 #endif

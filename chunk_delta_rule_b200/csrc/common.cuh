@@ -13,31 +13,47 @@ __device__ int g_status = 0;
 
 __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0, code); }
 
-// Optional phase tracing (compile with -DCOMBA_TRACE_PHASES): threads 0 and 128
-// of CTA 0 accumulate clock64() deltas between consecutive COMBA_PHASE marks in
-// registers (each thread its own slots) and add them to a device array at
-// COMBA_PHASE_END.  Off by
-// default; the marks then compile to nothing.
+// Optional phase tracing (compile with -DCOMBA_TRACE_PHASES): thread 0 and thread
+// COMBA_TRACE_TID2 (default 128) of CTA 0 accumulate clock64() deltas between
+// consecutive COMBA_PHASE marks in registers (each thread its own slots) and add
+// them to a device array at COMBA_PHASE_END.  Off by default; the marks then
+// compile to nothing.
+#define COMBA_TRACE_SLOTS 32
 #ifdef COMBA_TRACE_PHASES
-__device__ unsigned long long g_phase_cycles[16];
+#ifndef COMBA_TRACE_TID2
+#define COMBA_TRACE_TID2 128
+#endif
+#ifndef COMBA_TRACE_ITER
+#define COMBA_TRACE_ITER 10
+#endif
+__device__ unsigned long long g_phase_cycles[COMBA_TRACE_SLOTS];
+// absolute clock64() of each mark: thread 0 in loop iteration COMBA_TRACE_ITER,
+// thread TID2 in the next one (the prep group runs one chunk ahead): [thread 0 | TID2]
+__device__ long long g_phase_ts[2 * COMBA_TRACE_SLOTS];
 #define COMBA_PHASE_BEGIN()                                   \
     long long comba_phase_t = clock64();                      \
-    unsigned long long comba_phase_acc[16] = {}
+    int comba_iter = 0;                                       \
+    unsigned long long comba_phase_acc[COMBA_TRACE_SLOTS] = {}
 #define COMBA_PHASE(i)                                                        \
     do {                                                                      \
         const long long comba_phase_now = clock64();                          \
         comba_phase_acc[(i)] += (unsigned long long)(comba_phase_now - comba_phase_t); \
         comba_phase_t = comba_phase_now;                                      \
+        if (comba_iter == COMBA_TRACE_ITER + (threadIdx.x == 0 ? 0 : 1) && blockIdx.x == 0 && \
+            (threadIdx.x == 0 || threadIdx.x == COMBA_TRACE_TID2))            \
+            g_phase_ts[(threadIdx.x == 0 ? 0 : COMBA_TRACE_SLOTS) + (i)] = comba_phase_now; \
     } while (0)
+#define COMBA_ITER_NEXT() (++comba_iter)
 #define COMBA_PHASE_END()                                                     \
     do {                                                                      \
-        if (blockIdx.x == 0 && (threadIdx.x == 0 || threadIdx.x == 128))      \
-            for (int comba_i = 0; comba_i < 16; ++comba_i)                    \
+        if (blockIdx.x == 0 && (threadIdx.x == 0 || threadIdx.x == COMBA_TRACE_TID2)) \
+            for (int comba_i = 0; comba_i < COMBA_TRACE_SLOTS; ++comba_i)     \
                 g_phase_cycles[comba_i] += comba_phase_acc[comba_i];          \
     } while (0)
 #else
 #define COMBA_PHASE_BEGIN() do {} while (0)
 #define COMBA_PHASE(i) do {} while (0)
+#define COMBA_ITER_NEXT() do {} while (0)
 #define COMBA_PHASE_END() do {} while (0)
 #endif
 

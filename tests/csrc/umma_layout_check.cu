@@ -121,7 +121,7 @@ __global__ void umma_check_kernel(int mode, const float* A, const float* B, cons
         tc_fence_before();
     }
     __syncthreads();
-    if (tid == 0) {
+    if (warp == 0) {   // one converged warp issues (one elected lane)
         tc_fence_after();
         const uint32_t a = sb, b = sb + 32768;
         switch (mode) {
