@@ -91,18 +91,33 @@ constexpr uint32_t ID_XP = tc::idesc_tf32(128, 64, false, false);   // X^T P^T
 constexpr float kLog2e = 1.4426950408889634f;
 
 // fp32 64 x 64 scratch with an XOR swizzle on the column; byte address in a buffer.
-__device__ __forceinline__ int fidx(int r, int s) { return r * 64 + (s ^ (r & 31)); }
+// h(r) maps the low five row bits onto the five bank bits so that a warp's accesses
+// are conflict-free for one row per lane and for the 8 x 4 / 4 x 8 row-column
+// patterns of the m16n8k8 A and B fragments: r bits 0-1 -> bank bits 3-4, r bit 2
+// -> bank bit 2, r bits 3-4 -> bank bits 0-1.
+__device__ __forceinline__ int fswz(int r) { return ((r & 3) << 3) | (r & 4) | ((r >> 3) & 3); }
+__device__ __forceinline__ int fidx(int r, int s) { return r * 64 + (s ^ fswz(r)); }
 __device__ __forceinline__ uint32_t faddr(uint32_t base, int r, int s) {
     return base + 4u * (uint32_t)fidx(r, s);
 }
 
+// Inside diagonal block blk (parity P = blk & 1), fidx(16 blk + r, 16 blk + s) =
+// 16 blk 64 + 32 (blk >> 1) + r 64 + ((s ^ fswz_blk(r)) ^ 18 P), with fswz_blk(r) the
+// row swizzle of an even block: the parity flips bits 1 and 4 of the column.
+__device__ __forceinline__ constexpr int fswz_blk(int r) { return ((r & 3) << 3) | (r & 4) | (r >> 3); }
+
 // Diagonal 16 x 16 block `blk` of (I + A)^{-1} (A strictly lower, fp32 at F1)
 // into F2: one warp, lane j < 16 owns column j, right-looking substitution.
-// Inside block `blk`, fidx(16 blk + r, 16 blk + s) = (16 blk + r) 64 + 32 (blk >> 1)
-// + (s ^ r), so every A offset below is a compile-time constant.
+// The loads use four base pointers, one per value of column bits 1 and 4, so
+// that every offset is a compile-time constant for either parity (one copy of
+// the code for all four blocks).
 __device__ __forceinline__ void diag_block_inverse(uint32_t F1, uint32_t F2, int blk, int lane) {
+    const int P = blk & 1;
     const uint32_t base = 4u * (uint32_t)(16 * blk * 64 + 32 * (blk >> 1));
     const uint32_t Ab = F1 + base;
+    const int d1 = 2 * P, d4 = 16 * P;
+    const uint32_t bb[4] = {Ab + 4u * (uint32_t)(d1 + d4), Ab + 4u * (uint32_t)(-d1 + d4),
+                            Ab + 4u * (uint32_t)(d1 - d4), Ab + 4u * (uint32_t)(-d1 - d4)};
     const int j = lane & 15;
     float x[16];
 #pragma unroll
@@ -111,13 +126,17 @@ __device__ __forceinline__ void diag_block_inverse(uint32_t F1, uint32_t F2, int
     for (int s = 0; s < 15; ++s) {
         const float xs = x[s];
 #pragma unroll
-        for (int r = s + 1; r < 16; ++r)
-            x[r] = fmaf(-tc::lds_f32(Ab + 4u * (uint32_t)(r * 64 + (s ^ r))), xs, x[r]);
+        for (int r = s + 1; r < 16; ++r) {
+            const int c = s ^ fswz_blk(r);
+            const int sel = ((c >> 1) & 1) | (((c >> 4) & 1) << 1);
+            x[r] = fmaf(-tc::lds_f32(bb[sel] + 4u * (uint32_t)(r * 64 + c)), xs, x[r]);
+        }
     }
     if (lane < 16) {
         const uint32_t Tb = F2 + base;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) tc::sts_f32(Tb + 4u * (uint32_t)(r * 64 + (j ^ r)), x[r]);
+        for (int r = 0; r < 16; ++r)
+            tc::sts_f32(Tb + 4u * (uint32_t)(r * 64 + ((j ^ fswz_blk(r)) ^ (18 * P))), x[r]);
     }
 }
 
@@ -646,6 +665,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             bool ok = (*gabort == 0);
             // ---- Gram ([K;Q] K^T), unless it was issued during the previous chunk --------
             if (pw == 0 && !gram_issued) {
+                COMBA_COUNT(14);
                 ok = ok && tc::mbar_wait(&bars[stg], (m >> 1) & 1, timeout_ns);
                 if (ok) {
                     tc::tc_fence_after();
@@ -656,6 +676,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
             gram_issued = false;
+            COMBA_PHASE(12);
             // ---- gates --------------------------------------------------------------------
             if (pt < 64) {
                 if (!last) {
@@ -671,6 +692,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (lane == 31) tc::sts_f32(RED + 4u * pw, x);
                 tc::sts_f32(G2 + 4u * pt, x);
             }
+            COMBA_PHASE(13);
             tc::named_barrier(BAR_PREP, kPrepThreads);
             COMBA_PHASE(22);
             const float carry = tc::lds_f32(RED);

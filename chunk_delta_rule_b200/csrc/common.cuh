@@ -44,6 +44,7 @@ __device__ long long g_phase_ts[2 * COMBA_TRACE_SLOTS];
             g_phase_ts[(threadIdx.x == 0 ? 0 : COMBA_TRACE_SLOTS) + (i)] = comba_phase_now; \
     } while (0)
 #define COMBA_ITER_NEXT() (++comba_iter)
+#define COMBA_COUNT(i) (++comba_phase_acc[(i)])
 #define COMBA_PHASE_END()                                                     \
     do {                                                                      \
         if (blockIdx.x == 0 && (threadIdx.x == 0 || threadIdx.x == COMBA_TRACE_TID2)) \
@@ -54,6 +55,7 @@ __device__ long long g_phase_ts[2 * COMBA_TRACE_SLOTS];
 #define COMBA_PHASE_BEGIN() do {} while (0)
 #define COMBA_PHASE(i) do {} while (0)
 #define COMBA_ITER_NEXT() do {} while (0)
+#define COMBA_COUNT(i) do {} while (0)
 #define COMBA_PHASE_END() do {} while (0)
 #endif
 

@@ -278,33 +278,44 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 }
 
 // ---------------------------------------------------------------- MMA issue
-// Every helper issues `ksteps` MMAs of K = 16 (bf16) from one thread; the
-// first accumulates into D only if `acc0` is set, the rest always do.
-// Shapes are taken from `idesc`.  Byte arguments are shared-memory addresses.
+// Every helper issues `ksteps` MMAs (K = 16 for bf16, K = 8 for tf32) from one
+// converged warp; the first accumulates into D only if `acc0` is set, the rest
+// always do.  Shapes are taken from `idesc`.  Byte arguments are shared-memory
+// addresses.  Each descriptor is built once: the start address sits in its low
+// 14 bits (address / 16, below 2^14 for any shared-memory address), so a
+// k-step's operand offset is added to the descriptor directly.  The loops are
+// unrolled by COMBA_MMA_UNROLL (default: fully); rolled loops issue measurably
+// slower.
+#ifndef COMBA_MMA_UNROLL
+#define COMBA_MMA_UNROLL 8
+#endif
+constexpr int kMmaUnroll = COMBA_MMA_UNROLL;
+
+__device__ __forceinline__ uint32_t katom_off(int ks, uint32_t atom) {   // K-major k-step offset
+    return (uint32_t)(ks >> 2) * atom + (uint32_t)(ks & 3) * 32u;
+}
 
 // A K-major (128 rows, 64-element K atoms `a_atom` bytes apart),
 // B K-major (N rows, K atoms `b_atom` bytes apart; 0 re-reads atom 0).
 __device__ __forceinline__ void mma_ak_bk(uint32_t d, uint32_t a, uint32_t a_atom, uint32_t b,
                                           uint32_t b_atom, uint32_t idesc, int ksteps,
                                           uint32_t acc0) {
-#pragma unroll
-    for (int ks = 0; ks < ksteps; ++ks) {
-        const uint64_t ad = sdesc_sw128(a + (ks >> 2) * a_atom + (ks & 3) * 32, 16, 1024);
-        const uint64_t bd = sdesc_sw128(b + (ks >> 2) * b_atom + (ks & 3) * 32, 16, 1024);
-        mma_bf16(d, ad, bd, idesc, (ks > 0) ? 1u : acc0);
-    }
+    const uint64_t ad0 = sdesc_sw128(a, 16, 1024), bd0 = sdesc_sw128(b, 16, 1024);
+#pragma unroll kMmaUnroll
+    for (int ks = 0; ks < ksteps; ++ks)
+        mma_bf16(d, ad0 + (katom_off(ks, a_atom) >> 4), bd0 + (katom_off(ks, b_atom) >> 4), idesc,
+                 (ks > 0) ? 1u : acc0);
 }
 
 // A MN-major (M in 64-element atoms `a_lbo` bytes apart; one 128 B row per K
 // index), B K-major (N rows, K within one 64-element atom).
 __device__ __forceinline__ void mma_amn_bk(uint32_t d, uint32_t a, uint32_t a_lbo, uint32_t b,
                                            uint32_t idesc, int ksteps, uint32_t acc0) {
-#pragma unroll
-    for (int ks = 0; ks < ksteps; ++ks) {
-        const uint64_t ad = sdesc_sw128(a + ks * 2048, a_lbo, 1024);
-        const uint64_t bd = sdesc_sw128(b + ks * 32, 16, 1024);
-        mma_bf16(d, ad, bd, idesc, (ks > 0) ? 1u : acc0);
-    }
+    const uint64_t ad0 = sdesc_sw128(a, a_lbo, 1024), bd0 = sdesc_sw128(b, 16, 1024);
+#pragma unroll kMmaUnroll
+    for (int ks = 0; ks < ksteps; ++ks)
+        mma_bf16(d, ad0 + (uint32_t)(ks * (2048 >> 4)), bd0 + (uint32_t)(ks * (32 >> 4)), idesc,
+                 (ks > 0) ? 1u : acc0);
 }
 
 // A K-major (128 rows, K atoms `a_atom` apart), B MN-major (N in atoms
@@ -313,12 +324,11 @@ __device__ __forceinline__ void mma_amn_bk(uint32_t d, uint32_t a, uint32_t a_lb
 __device__ __forceinline__ void mma_ak_bmn(uint32_t d, uint32_t a, uint32_t a_atom, uint32_t b,
                                            uint32_t b_lbo, uint32_t idesc, int ksteps, int kwrap,
                                            uint32_t acc0) {
-#pragma unroll
-    for (int ks = 0; ks < ksteps; ++ks) {
-        const uint64_t ad = sdesc_sw128(a + (ks >> 2) * a_atom + (ks & 3) * 32, 16, 1024);
-        const uint64_t bd = sdesc_sw128(b + (ks % kwrap) * 2048, b_lbo, 1024);
-        mma_bf16(d, ad, bd, idesc, (ks > 0) ? 1u : acc0);
-    }
+    const uint64_t ad0 = sdesc_sw128(a, 16, 1024), bd0 = sdesc_sw128(b, b_lbo, 1024);
+#pragma unroll kMmaUnroll
+    for (int ks = 0; ks < ksteps; ++ks)
+        mma_bf16(d, ad0 + (katom_off(ks, a_atom) >> 4), bd0 + (uint32_t)((ks % kwrap) * (2048 >> 4)),
+                 idesc, (ks > 0) ? 1u : acc0);
 }
 
 // tf32, A from TMEM (K = 8 columns per MMA), B K-major fp32 (N rows; 32-element
@@ -326,11 +336,10 @@ __device__ __forceinline__ void mma_ak_bmn(uint32_t d, uint32_t a, uint32_t a_at
 __device__ __forceinline__ void mma_tf32_ta_bk(uint32_t d, uint32_t a_tmem, uint32_t b,
                                                uint32_t b_atom, uint32_t idesc, int ksteps,
                                                uint32_t acc0) {
-#pragma unroll
-    for (int ks = 0; ks < ksteps; ++ks) {
-        const uint64_t bd = sdesc_sw128(b + (ks >> 2) * b_atom + (ks & 3) * 32, 16, 1024);
-        mma_tf32_ta(d, a_tmem + ks * 8, bd, idesc, (ks > 0) ? 1u : acc0);
-    }
+    const uint64_t bd0 = sdesc_sw128(b, 16, 1024);
+#pragma unroll kMmaUnroll
+    for (int ks = 0; ks < ksteps; ++ks)
+        mma_tf32_ta(d, a_tmem + ks * 8, bd0 + (katom_off(ks, b_atom) >> 4), idesc, (ks > 0) ? 1u : acc0);
 }
 
 // bf16, A from TMEM (K = 16 per MMA = 8 packed columns), B K-major (N rows, K
@@ -338,22 +347,20 @@ __device__ __forceinline__ void mma_tf32_ta_bk(uint32_t d, uint32_t a_tmem, uint
 __device__ __forceinline__ void mma_bf16_ta_bk(uint32_t d, uint32_t a_tmem, uint32_t b,
                                                uint32_t b_atom, uint32_t idesc, int ksteps,
                                                uint32_t acc0) {
-#pragma unroll
-    for (int ks = 0; ks < ksteps; ++ks) {
-        const uint64_t bd = sdesc_sw128(b + (ks >> 2) * b_atom + (ks & 3) * 32, 16, 1024);
-        mma_bf16_ta(d, a_tmem + ks * 8, bd, idesc, (ks > 0) ? 1u : acc0);
-    }
+    const uint64_t bd0 = sdesc_sw128(b, 16, 1024);
+#pragma unroll kMmaUnroll
+    for (int ks = 0; ks < ksteps; ++ks)
+        mma_bf16_ta(d, a_tmem + ks * 8, bd0 + (katom_off(ks, b_atom) >> 4), idesc, (ks > 0) ? 1u : acc0);
 }
 
 // bf16, A from TMEM, B MN-major (N in atoms `b_lbo` apart; one 128 B row per K index).
 __device__ __forceinline__ void mma_bf16_ta_bmn(uint32_t d, uint32_t a_tmem, uint32_t b,
                                                 uint32_t b_lbo, uint32_t idesc, int ksteps,
                                                 uint32_t acc0) {
-#pragma unroll
-    for (int ks = 0; ks < ksteps; ++ks) {
-        const uint64_t bd = sdesc_sw128(b + ks * 2048, b_lbo, 1024);
-        mma_bf16_ta(d, a_tmem + ks * 8, bd, idesc, (ks > 0) ? 1u : acc0);
-    }
+    const uint64_t bd0 = sdesc_sw128(b, b_lbo, 1024);
+#pragma unroll kMmaUnroll
+    for (int ks = 0; ks < ksteps; ++ks)
+        mma_bf16_ta(d, a_tmem + ks * 8, bd0 + (uint32_t)(ks * (2048 >> 4)), idesc, (ks > 0) ? 1u : acc0);
 }
 
 // ---------------------------------------------------------------- warp MMA (legacy)
