@@ -70,12 +70,13 @@ constexpr uint32_t SM_DK = 131072;    // (D K)^T fp32, K-major: 2 atoms (32 r) x
 constexpr uint32_t SM_F1 = 163840;    // fp32 64x64: A; then Tc (bf16) | Eb (bf16)
 constexpr uint32_t SM_F2 = 180224;    // fp32 64x64: Tinv (upper blocks: scratch)
 constexpr uint32_t SM_BLO = 196608;   // bf16 64x64 K-major: diag(lo(beta)), zero elsewhere
-constexpr uint32_t SM_OUT = 204800;   // out tile staging: 2 boxes x 64 tokens x 128 B
+constexpr uint32_t SM_QH = 204800;    // Qh bf16, K-major like Q: 2 atoms (64 j) x 64 tokens
 constexpr uint32_t SM_MISC = 221184;  // gates, barriers
 constexpr uint32_t SM_END = SM_MISC + 4096;
 constexpr uint32_t kSmemBytes = SM_END + 1024;
 
 constexpr uint32_t KQ_ATOM = 16384;
+constexpr uint32_t QH_ATOM = 8192;
 constexpr uint32_t V_ATOM = 8192;
 constexpr uint32_t OP_ATOM = 16384;
 constexpr uint32_t F32_ATOM = 8192;   // 64 rows x 128 B
@@ -361,24 +362,24 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     const uint32_t sb = tc::smem_u32(sm);
 
-    // prep-private gate tables (64 fp32 each), by shared address
+    // gate tables (64 fp32 each), by shared address; the prep group's and the state group's
     const uint32_t G2 = sb + SM_MISC;        // g_r log2(e)
     const uint32_t GP2 = G2 + 256;           // g_{r-1} log2(e)
     const uint32_t BT = G2 + 512;            // beta_r
     const uint32_t CS = G2 + 768;            // beta_r e^{g_{r-1}}
     const uint32_t EG = G2 + 1024;           // e^{g_r}
-    const uint32_t ED = G2 + 1280;           // e^{g_L - g_r}
     const uint32_t IEG = G2 + 1536;          // e^{-g_r} (when the chunk allows)
     const uint32_t RED = G2 + 1792;          // [0..1] scan carries
     const uint32_t SRED = G2 + 1936;         // state group: [0..1] scan carries
     const uint32_t SED = G2 + 2048;          // state group: e^{g_L - g_r} of the next chunk
-    // barriers: q/k stages, v, gram, wn, prep ready, mma1 (X), mma2, mma1 (O), and
-    // per P buffer: the MMA2 that read it is done.  Each is arrived on once per
-    // phase (by a commit, a TMA transaction count or one elected thread after its
-    // group's named barrier): many arrivals on one barrier serialise in the
-    // shared-memory pipe and hold up the group's next shared-memory accesses.
-    enum { B_KQ0 = 0, B_KQ1 = 1, B_V = 2, B_GRAM = 3, B_WN = 4, B_PREP = 5, B_MMA1 = 6, B_MMA2 = 7,
-           B_MMA1B = 8, B_PBUF0 = 9, B_PBUF1 = 10, NBARS = 11 };
+    const uint32_t SEG = G2 + 2304;          // state group: e^{g_r} of the next chunk
+    // barriers: q/k stages, v, gram, wn (W^T, U~^T in TMEM), mma1 (X), mma2, the P
+    // buffers (MMA2 and the out store have read them) and the Gram/W^T TMEM buffer
+    // (the state group has read W^T).  Each is arrived on once per phase (by a
+    // commit, a TMA transaction count or one thread after its group's named
+    // barrier): many arrivals on one barrier serialise in the shared-memory pipe.
+    enum { B_KQ0 = 0, B_KQ1 = 1, B_V = 2, B_GRAM = 3, B_WN = 4, B_MMA1 = 5, B_MMA2 = 6, B_PBUF0 = 7,
+           B_PBUF1 = 8, B_GFREE = 9, NBARS = 10 };
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 2560);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
     volatile int* gabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -425,20 +426,30 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tc::tma_load_4d(sm + SM_V, &tm_v, &bars[B_V], 0, h, t0, b);
         tc::tma_load_4d(sm + SM_V + V_ATOM, &tm_v, &bars[B_V], 64, h, t0, b);
     };
+    // One token's gate value.  The load is issued where it is written (volatile) and
+    // consumed a phase later, so its latency stays hidden; a plain load may be sunk
+    // by the compiler to its use, past the waits in between.
     auto gate = [&](const float* p, int t) -> float {
-        return (t < T) ? p[((size_t)b * T + t) * H + h] : 0.f;
+        float v = 0.f;
+        if (t < T) {
+            const float* a = p + ((size_t)b * T + t) * H + h;
+            asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(a));
+        }
+        return v;
     };
 
     COMBA_PHASE_BEGIN();
     if (warp < 4) {
         // =============================== state group ===============================
-        // Per chunk n: MMA1(n) X^T += S (-W)^T, O^T = S Qh^T; MMA2(n) S += X^T (D K),
-        // O^T += X^T P^T; then S -> bf16 copy, S *= e^{g_L(n+1)}, O^T -> out, and the
-        // (D K)^T operand of chunk n+1 (from the group's own scan of its log-decays).
+        // Per chunk n: -W operand from W^T (TMEM, the prep group's MMA); MMA1(n)
+        // X^T += S (-W)^T, O^T = S Qh^T; MMA2(n) S += X^T (D K), O^T += X^T P^T; then
+        // S -> bf16 copy, S *= e^{g_L(n+1)}, O^T -> out (staged in this chunk's P
+        // buffer), and the (D K)^T and Qh operands of chunk n+1 from the group's own
+        // scan of its log-decays.
         const int row = tid;
         const bool issuer = (tid == 0);
         // Scan of one chunk's log-decays held by threads 0..63: writes e^{g_L - g_r}
-        // to SED and returns e^{g_L} to every thread of the group.
+        // to SED and e^{g_r} to SEG, and returns e^{g_L} to every thread of the group.
         auto state_gates = [&](float la) -> float {
             float x = la;
             if (tid < 64) {
@@ -454,39 +465,47 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (tid < 64) {
                 const float g = x + (tid >= 32 ? c0 : 0.f);
                 tc::sts_f32(SED + 4u * tid, __expf(gL - g));
+                tc::sts_f32(SEG + 4u * tid, __expf(g));
             }
             return __expf(gL);
         };
-        // (D K)^T of chunk c (K-major fp32 operand of the state update).
-        auto state_dk = [&](int c) -> bool {
+        // (D K)^T (K-major fp32 operand of the state update) and Qh = diag(e^g)(Q - d K)
+        // (bf16, K-major like Q) of chunk c, from its q/k tiles.
+        auto state_dk_qh = [&](int c) -> bool {
             const bool okc = tc::mbar_wait(&bars[c & 1], (c >> 1) & 1, timeout_ns);
             const uint32_t kqc = sb + ((c & 1) ? SM_KQ1 : SM_KQ0);
             const int r = tid & 63, jh = tid >> 6;
-            const float edr = tc::lds_f32(SED + 4u * r);
+            const float edr = tc::lds_f32(SED + 4u * r), egr = tc::lds_f32(SEG + 4u * r);
             const uint32_t dka = sb + SM_DK + (r >> 5) * DKT_ATOM + (r & 3) * 4;
             const uint32_t rc = (r & 31) >> 2;
 #pragma unroll 2
             for (int c8 = 0; c8 < 8; ++c8) {
-                const uint4 kw = tc::lds_u32x4(kqc + jh * KQ_ATOM + tc::sw128(r, c8));
+                const uint32_t off = kqc + jh * KQ_ATOM + tc::sw128(r, c8);
+                const uint4 kw = tc::lds_u32x4(off);
+                uint4 qw = tc::lds_u32x4(off + 8192);
                 const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kw);
+                __nv_bfloat162* q2 = reinterpret_cast<__nv_bfloat162*>(&qw);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 kf = __bfloat1622float2(k2[e]);
+                    const float2 qf = __bfloat1622float2(q2[e]);
                     const int j = 64 * jh + 8 * c8 + 2 * e;
                     tc::sts_f32(dka + tc::sw128(j, rc), edr * kf.x);
                     tc::sts_f32(dka + tc::sw128(j + 1, rc), edr * kf.y);
+                    q2[e] = __floats2bfloat162_rn(egr * fmaf(-dh, kf.x, qf.x), egr * fmaf(-dh, kf.y, qf.y));
                 }
+                tc::sts_u32x4(sb + SM_QH + jh * QH_ATOM + tc::sw128(r, c8), qw);
             }
             tc::fence_proxy_async_smem();
             return okc;
         };
         bool ok = true;
-        // decay and (D K)^T of chunk 0, initial state
+        // decay, (D K)^T and Qh of chunk 0, initial state
         {
             const float la0 = (tid < 64) ? gate(log_alpha, tid) : 0.f;
             const float eL0 = state_gates(la0);
             tc::named_barrier(BAR_STATE, kStateThreads);
-            ok = state_dk(0);
+            ok = state_dk_qh(0);
             const float* s0row = S0 ? S0 + ((size_t)blockIdx.x * kD + row) * kD : nullptr;
 #pragma unroll 1
             for (int pair = 0; pair < 2; ++pair) {
@@ -514,42 +533,58 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::tmem_st_wait();
             tc::tc_fence_before();
             if (!ok) fail(gabort);
-            // the issuer's first MMAs follow this barrier: the S copies are in TMEM
             ok = tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok);
         }
         float la_n = 0.f;
         for (int n = 0; n < nchunks && ok; ++n) {
             const int t0 = n * kC;
             const int stg = n & 1;
-            const uint32_t kq_a = sb + (stg ? SM_KQ1 : SM_KQ0);
             const uint32_t txn = tmem + (stg ? TM_X1 : TM_X0);
+            const uint32_t tgn = stg ? TM_G1 : TM_G;
+            const uint32_t pbuf = stg ? SM_P1 : SM_P0;
             const bool last = (n + 1 == nchunks);
             if (tid < 64 && !last) la_n = gate(log_alpha, t0 + kC + tid);   // next chunk's decay
-            ok = (*gabort == 0);
+            // ---- -W operand from W^T (lane = j, column = token) once the prep's MMAs are done
+            ok = (*gabort == 0) && tc::mbar_wait(&bars[B_WN], n & 1, timeout_ns);
+            COMBA_PHASE(0);
+            tc::tc_fence_after();
+            {
+                float w0[32], w1[32];
+                tc::tmem_ld32(tl + tgn, w0);
+                tc::tmem_ld32(tl + tgn + 32, w1);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) { w0[e] = -w0[e]; w1[e] = -w1[e]; }
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    tc::sts_u32x4(sb + SM_W + tc::sw128(row, c4), pack8_bf16(w0 + c4 * 8));
+                    tc::sts_u32x4(sb + SM_W + tc::sw128(row, 4 + c4), pack8_bf16(w1 + c4 * 8));
+                }
+            }
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
+            if (!ok) fail(gabort);
+            if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
+            if (issuer) {
+                tc::mbar_arrive(&bars[B_GFREE]);   // W^T read: the prep may reuse this TMEM buffer
+                // V and this chunk's q/k stage have been read (W/X MMAs, Gram, (D K)^T, Qh)
+                tc::fence_proxy_async_smem();
+                if (n + 1 < nchunks) load_v(n + 1);
+                if (n + 2 < nchunks) load_kq(n + 2);
+            }
+            COMBA_PHASE(1);
             if (warp == 0) {   // MMA issue: the whole warp, one elected lane
-                ok = ok && tc::mbar_wait(&bars[B_PREP], n & 1, timeout_ns);
-                COMBA_PHASE(0);
+                __syncwarp();   // reconverge after the single-thread block above
+                tc::tc_fence_after();
+                tc::mma_bf16_ta_bmn(txn, tmem + TM_SB, sb + SM_W, 8192, ID_SW, 8, 1);
+                tc::mma_commit(&bars[B_MMA1]);
+                tc::mma_bf16_ta_bk(tmem + TM_O, tmem + TM_SB, sb + SM_QH, QH_ATOM, ID_SQ, 8, 0);
+                ok = tc::mbar_wait(&bars[B_MMA1], n & 1, timeout_ns);
                 if (ok) {
                     tc::tc_fence_after();
-                    tc::mma_bf16_ta_bmn(txn, tmem + TM_SB, sb + SM_W, 8192, ID_SW, 8, 1);
-                    tc::mma_commit(&bars[B_MMA1]);
-                    tc::mma_bf16_ta_bk(tmem + TM_O, tmem + TM_SB, kq_a + 8192, KQ_ATOM, ID_SQ, 8, 0);
-                    tc::mma_commit(&bars[B_MMA1B]);
-                    ok = tc::mbar_wait(&bars[B_MMA1], n & 1, timeout_ns);
-                    COMBA_PHASE(1);
-                    if (ok) {
-                        tc::tc_fence_after();
-                        tc::mma_tf32_ta_bk(tmem + TM_S, txn, sb + SM_DK, DKT_ATOM, ID_SU, 8, 1);
-                        tc::mma_tf32_ta_bk(tmem + TM_O, txn, sb + (stg ? SM_P1 : SM_P0), F32_ATOM, ID_XP, 8, 1);
-                        tc::mma_commit(&bars[B_MMA2]);
-                        tc::mma_commit(&bars[stg ? B_PBUF1 : B_PBUF0]);
-                        // stage stg is free once S Qh^T has read Qh (K: read by Gram, W^T, D K)
-                        ok = tc::mbar_wait(&bars[B_MMA1B], n & 1, timeout_ns);
-                        if (ok && n + 2 < nchunks && lane == 0) {
-                            tc::fence_proxy_async_smem();
-                            load_kq(n + 2);
-                        }
-                    }
+                    tc::mma_tf32_ta_bk(tmem + TM_S, txn, sb + SM_DK, DKT_ATOM, ID_SU, 8, 1);
+                    tc::mma_tf32_ta_bk(tmem + TM_O, txn, sb + pbuf, F32_ATOM, ID_XP, 8, 1);
+                    tc::mma_commit(&bars[B_MMA2]);
                 }
                 if (!ok) fail(gabort);
             }
@@ -558,8 +593,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
             tc::tc_fence_after();
             COMBA_PHASE(2);
-            // O^T row (value index) -> bf16 pairs of tokens, read before S is released;
-            // the first half of S is loaded in the same batch
+            // O^T row (value index) -> bf16 pairs of tokens
             uint32_t ob[32];
             {
                 float o0[32], o1[32];
@@ -605,12 +639,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::tmem_st_wait();
             tc::tc_fence_before();
             COMBA_PHASE(3);
-            // out tile [token][value index] in two 64-wide 128B-swizzled boxes, TMA store.
-            // This barrier also hands the new S copies to the issuer's next MMAs.
-            if (issuer) tc::bulk_wait_read0();
-            tc::named_barrier(BAR_STATE, kStateThreads);
+            // out tile [token][value index] in two 64-wide 128B-swizzled boxes, staged in
+            // this chunk's P buffer (MMA2 has read it), TMA store; once the store has
+            // read it the buffer goes back to the prep group.  The barrier below also
+            // hands the new S copies to the next MMA1.
             {
-                const uint32_t ot = sb + SM_OUT + (row >> 6) * 8192 + (row & 7) * 2;
+                const uint32_t ot = sb + pbuf + (row >> 6) * 8192 + (row & 7) * 2;
                 const int oc = (row & 63) >> 3;
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
@@ -621,14 +655,15 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::fence_proxy_async_smem();
             tc::named_barrier(BAR_STATE, kStateThreads);
             if (issuer) {
-                tc::tma_store_4d(&tm_o, sm + SM_OUT, 0, h, t0, b);
-                tc::tma_store_4d(&tm_o, sm + SM_OUT + 8192, 64, h, t0, b);
+                tc::tma_store_4d(&tm_o, sm + pbuf, 0, h, t0, b);
+                tc::tma_store_4d(&tm_o, sm + pbuf + 8192, 64, h, t0, b);
                 tc::bulk_commit();
+                tc::bulk_wait_read0();
+                tc::mbar_arrive(&bars[stg ? B_PBUF1 : B_PBUF0]);
             }
             COMBA_PHASE(4);
-            // (D K)^T of the next chunk (MMA2 of this chunk has read the buffer)
             if (!last) {
-                const bool okd = state_dk(n + 1);
+                const bool okd = state_dk_qh(n + 1);
                 if (!okd) fail(gabort);
                 if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, okd && *gabort == 0)) break;
             }
@@ -639,8 +674,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     } else {
         // =============================== prep group ================================
         // Per chunk m (running one chunk ahead of the state group): gates, Gram, P, A,
-        // the inverse, Tc/Eb, Qh, W^T and U~^T (= X^T before MMA1), then, once the
-        // state group has released them, P, (D K)^T and -W.
+        // the inverse, Tc/Eb, then the MMAs W^T = K^T Tc^T and U~^T (= X^T before MMA1),
+        // and the next chunk's Gram.
         const int pt = tid - kStateThreads;
         const int prow = pt & 127, phalf = pt >> 7, pw = pt >> 5;
         const bool issuer = (pt == 0);
@@ -665,6 +700,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             bool ok = (*gabort == 0);
             // ---- Gram ([K;Q] K^T), unless it was issued during the previous chunk --------
             if (pw == 0 && !gram_issued) {
+                __syncwarp();
                 COMBA_COUNT(14);
                 ok = ok && tc::mbar_wait(&bars[stg], (m >> 1) & 1, timeout_ns);
                 if (ok) {
@@ -709,14 +745,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::sts_f32(G2 + 4u * pt, g * kLog2e);
             }
             COMBA_PHASE(23);
+            // Gram of this chunk in; the previous chunk's W/X MMAs have read F1 and BLO
             ok = ok && tc::mbar_wait(&bars[B_GRAM], m & 1, timeout_ns) &&
-                 tc::mbar_wait(&bars[stg], (m >> 1) & 1, timeout_ns);
+                 tc::mbar_wait(&bars[stg], (m >> 1) & 1, timeout_ns) &&
+                 (m == 0 || tc::mbar_wait(&bars[B_WN], (m - 1) & 1, timeout_ns));
             COMBA_PHASE(24);
             if (!ok) fail(gabort);
             if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
             tc::tc_fence_after();
             COMBA_PHASE(16);
-            // ---- K K^T -> P buffer of this chunk (once MMA2 of chunk m-2 has read it), A -> F1
+            // ---- K K^T -> P buffer of this chunk (once MMA2 and the out store of chunk
+            // m-2 have read it), A -> F1
             if (m >= 2) {
                 const bool okp = tc::mbar_wait(&bars[stg ? B_PBUF1 : B_PBUF0], ((m - 2) >> 1) & 1, timeout_ns);
                 if (!okp) fail(gabort);
@@ -750,9 +789,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                 tc::lds_f32(GP2 + 4u * r), G2);
                 }
             }
+            tc::tc_fence_before();
             COMBA_PHASE(31);
             tc::named_barrier(BAR_PREP, kPrepThreads);
-            // ---- P (in place over K K^T) and Qh  ||  diagonal inverse blocks -------------
+            // ---- P (in place over K K^T)  ||  diagonal inverse blocks ---------------------
             if (prow >= 64) {
                 const int r = prow - 64;
                 const float er = tc::lds_f32(EG + 4u * r);
@@ -772,21 +812,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 } else {
                     p_row_exact(prow_base, tl + tgm + phalf * 32, r, s0, dh, G2);
-                }
-#pragma unroll 2
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t off = kq_a + phalf * KQ_ATOM + tc::sw128(r, c);
-                    const uint4 kw = tc::lds_u32x4(off);
-                    uint4 qw = tc::lds_u32x4(off + 8192);
-                    const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kw);
-                    __nv_bfloat162* q2 = reinterpret_cast<__nv_bfloat162*>(&qw);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 kf = __bfloat1622float2(k2[e]);
-                        const float2 qf = __bfloat1622float2(q2[e]);
-                        q2[e] = __floats2bfloat162_rn(er * fmaf(-dh, kf.x, qf.x), er * fmaf(-dh, kf.y, qf.y));
-                    }
-                    tc::sts_u32x4(off + 8192, qw);
                 }
             } else {
                 diag_block_inverse(F1, F2, (pw & 1) + 2 * phalf, lane);
@@ -808,8 +833,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::named_barrier(BAR_PREP, kPrepThreads);
             COMBA_PHASE(19);
             // ---- W^T = K^T Tc^T;  X^T = U~^T = V^T Eb^T + V^T diag(lo)^T --------------------
+            // (into TMEM; the state group turns W^T into its -W operand), then the next
+            // chunk's Gram into the other TMEM buffer once the state group has read the
+            // W^T that buffer held
             if (pw == 0) {   // MMA issue: the whole warp, one elected lane
-                ok = ok && tc::mbar_wait(&bars[B_V], m & 1, timeout_ns);
+                __syncwarp();   // reconverge after the per-thread code above
+                ok = ok && tc::mbar_wait(&bars[B_V], m & 1, timeout_ns) &&
+                     (m == 0 || tc::mbar_wait(&bars[B_GFREE], (m - 1) & 1, timeout_ns));
                 COMBA_PHASE(25);
                 if (ok) {
                     tc::tc_fence_after();
@@ -818,7 +848,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     tc::mma_amn_bk(txm, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
                     tc::mma_commit(&bars[B_WN]);
                     COMBA_PHASE(26);
-                    // next chunk's Gram into the other buffer, if its q/k tiles are in
                     const int m1 = m + 1;
                     if (!last && tc::mbar_try_wait(&bars[m1 & 1], (m1 >> 1) & 1)) {
                         const uint32_t kq1 = sb + ((m1 & 1) ? SM_KQ1 : SM_KQ0);
@@ -833,32 +862,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
             COMBA_PHASE(20);
-            // ---- once W^T is in and MMA1 of the previous chunk is done: -W operand ------------
-            ok = ok && tc::mbar_wait(&bars[B_WN], m & 1, timeout_ns);
-            COMBA_PHASE(27);
-            ok = ok && (m == 0 || tc::mbar_wait(&bars[B_MMA1], (m - 1) & 1, timeout_ns));
-            COMBA_PHASE(28);
-            if (!ok) fail(gabort);
-            tc::tc_fence_after();
-            if (issuer && ok && !last) {   // V was read by the W/X MMAs above
-                tc::fence_proxy_async_smem();
-                load_v(m + 1);
-            }
-            {
-                float w[32];
-                tc::tmem_ld32(tl + tgm + phalf * 32, w);
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) w[e] = -w[e];
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4)
-                    tc::sts_u32x4(sb + SM_W + tc::sw128(prow, phalf * 4 + c4), pack8_bf16(w + c4 * 8));
-            }
-            tc::fence_proxy_async_smem();
-            tc::tc_fence_before();
-            COMBA_PHASE(29);
-            if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
-            if (issuer) tc::mbar_arrive(&bars[B_PREP]);
             la_c = la_n;
             bt_c = bt_n;
             COMBA_PHASE(21);

@@ -34,8 +34,12 @@ __device__ long long g_phase_ts[2 * COMBA_TRACE_SLOTS];
     long long comba_phase_t = clock64();                      \
     int comba_iter = 0;                                       \
     unsigned long long comba_phase_acc[COMBA_TRACE_SLOTS] = {}
+#ifndef COMBA_TRACE_MASK
+#define COMBA_TRACE_MASK 0xffffffffu
+#endif
 #define COMBA_PHASE(i)                                                        \
     do {                                                                      \
+        if (!((COMBA_TRACE_MASK >> (i)) & 1u)) break;                         \
         const long long comba_phase_now = clock64();                          \
         comba_phase_acc[(i)] += (unsigned long long)(comba_phase_now - comba_phase_t); \
         comba_phase_t = comba_phase_now;                                      \

@@ -184,6 +184,9 @@ __device__ __forceinline__ void mma_tf32_ta(uint32_t d_tmem, uint32_t a_tmem, ui
 // Like the MMA helpers above, it is called by all 32 lanes of one converged warp
 // and issued by the lane elect.sync picks (the same lane every time for a full
 // mask), so the operands stay warp-uniform and no per-lane serialisation is needed.
+// Callers reconverge the warp (__syncwarp) before an issue block that follows
+// divergent code: without it the compiler may leave the warp split across the
+// block, which was measured to slow the whole kernel by half.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile(
         "{\n"
