@@ -52,8 +52,8 @@ constexpr int BAR_STATE = 2;
 // TMEM columns (fp32, 128 lanes)
 constexpr uint32_t TM_G = 0;     // Gram of even chunks (lanes 0-63 K K^T, 64-127 Q K^T), then W^T
 constexpr uint32_t TM_G1 = 320;  // the same for odd chunks
-constexpr uint32_t TM_X0 = 64;   // X^T of even chunks (lane = value index i, column = token r)
-constexpr uint32_t TM_X1 = 128;  // X^T of odd chunks
+constexpr uint32_t TM_X = 64;    // X^T (lane = value index i, column = token r), fp32
+constexpr uint32_t TM_XH = 128;  // (X diag(e^{g_L - g}))^T as bf16 hi (32 columns) and lo (32)
 constexpr uint32_t TM_O = 192;   // O^T accumulator
 constexpr uint32_t TM_SB = 256;  // bf16 copy of S, two per column (MMA A operand)
 constexpr uint32_t TM_S = 384;   // fp32 state master (lane i, column j)
@@ -66,12 +66,11 @@ constexpr uint32_t SM_V = 65536;      // V: 2 dv-atoms x 64 tokens x 128 B
 constexpr uint32_t SM_W = 81920;      // -W bf16, MN-major: 128 rows (j) x 64 tokens
 constexpr uint32_t SM_P0 = 98304;     // P fp32, K-major: 2 atoms (32 s) x 64 rows; even chunks
 constexpr uint32_t SM_P1 = 114688;    // odd chunks (K K^T is staged here first, P formed in place)
-constexpr uint32_t SM_DK = 131072;    // (D K)^T fp32, K-major: 2 atoms (32 r) x 128 rows (j)
-constexpr uint32_t SM_F1 = 163840;    // fp32 64x64: A; then Tc (bf16) | Eb (bf16)
-constexpr uint32_t SM_F2 = 180224;    // fp32 64x64: Tinv (upper blocks: scratch)
-constexpr uint32_t SM_BLO = 196608;   // bf16 64x64 K-major: diag(lo(beta)), zero elsewhere
-constexpr uint32_t SM_QH = 204800;    // Qh bf16, K-major like Q: 2 atoms (64 j) x 64 tokens
-constexpr uint32_t SM_MISC = 221184;  // gates, barriers
+constexpr uint32_t SM_F1 = 131072;    // fp32 64x64: A; then Tc (bf16) | Eb (bf16)
+constexpr uint32_t SM_F2 = 147456;    // fp32 64x64: Tinv (upper blocks: scratch)
+constexpr uint32_t SM_BLO = 163840;   // bf16 64x64 K-major: diag(lo(beta)), zero elsewhere
+constexpr uint32_t SM_QH = 172032;    // Qh bf16, K-major like Q: 2 atoms (64 j) x 64 tokens
+constexpr uint32_t SM_MISC = 188416;  // gates, barriers
 constexpr uint32_t SM_END = SM_MISC + 4096;
 constexpr uint32_t kSmemBytes = SM_END + 1024;
 
@@ -80,13 +79,12 @@ constexpr uint32_t QH_ATOM = 8192;
 constexpr uint32_t V_ATOM = 8192;
 constexpr uint32_t OP_ATOM = 16384;
 constexpr uint32_t F32_ATOM = 8192;   // 64 rows x 128 B
-constexpr uint32_t DKT_ATOM = 16384;  // 128 rows x 128 B
 
 constexpr uint32_t ID_G = tc::idesc_bf16(128, 64, false, false);    // [K;Q] K^T
 constexpr uint32_t ID_WN = tc::idesc_bf16(128, 64, true, false);    // K^T Tc^T, V^T Eb^T
 constexpr uint32_t ID_SW = tc::idesc_bf16(128, 64, false, true);    // S (-W)^T (W MN-major)
 constexpr uint32_t ID_SQ = tc::idesc_bf16(128, 64, false, false);   // S Qh^T
-constexpr uint32_t ID_SU = tc::idesc_tf32(128, 128, false, false);  // X^T (D K), (D K)^T K-major
+constexpr uint32_t ID_SK = tc::idesc_bf16(128, 128, false, true);   // X'^T K (K MN-major)
 constexpr uint32_t ID_XP = tc::idesc_tf32(128, 64, false, false);   // X^T P^T
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -469,15 +467,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             return __expf(gL);
         };
-        // (D K)^T (K-major fp32 operand of the state update) and Qh = diag(e^g)(Q - d K)
-        // (bf16, K-major like Q) of chunk c, from its q/k tiles.
-        auto state_dk_qh = [&](int c) -> bool {
+        // Qh = diag(e^g)(Q - d K) of chunk c (bf16, K-major like Q), from its q/k tiles.
+        auto state_qh = [&](int c) -> bool {
             const bool okc = tc::mbar_wait(&bars[c & 1], (c >> 1) & 1, timeout_ns);
             const uint32_t kqc = sb + ((c & 1) ? SM_KQ1 : SM_KQ0);
             const int r = tid & 63, jh = tid >> 6;
-            const float edr = tc::lds_f32(SED + 4u * r), egr = tc::lds_f32(SEG + 4u * r);
-            const uint32_t dka = sb + SM_DK + (r >> 5) * DKT_ATOM + (r & 3) * 4;
-            const uint32_t rc = (r & 31) >> 2;
+            const float egr = tc::lds_f32(SEG + 4u * r);
 #pragma unroll 2
             for (int c8 = 0; c8 < 8; ++c8) {
                 const uint32_t off = kqc + jh * KQ_ATOM + tc::sw128(r, c8);
@@ -489,9 +484,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int e = 0; e < 4; ++e) {
                     const float2 kf = __bfloat1622float2(k2[e]);
                     const float2 qf = __bfloat1622float2(q2[e]);
-                    const int j = 64 * jh + 8 * c8 + 2 * e;
-                    tc::sts_f32(dka + tc::sw128(j, rc), edr * kf.x);
-                    tc::sts_f32(dka + tc::sw128(j + 1, rc), edr * kf.y);
                     q2[e] = __floats2bfloat162_rn(egr * fmaf(-dh, kf.x, qf.x), egr * fmaf(-dh, kf.y, qf.y));
                 }
                 tc::sts_u32x4(sb + SM_QH + jh * QH_ATOM + tc::sw128(r, c8), qw);
@@ -500,12 +492,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             return okc;
         };
         bool ok = true;
-        // decay, (D K)^T and Qh of chunk 0, initial state
+        // decays and Qh of chunk 0, initial state
         {
             const float la0 = (tid < 64) ? gate(log_alpha, tid) : 0.f;
             const float eL0 = state_gates(la0);
             tc::named_barrier(BAR_STATE, kStateThreads);
-            ok = state_dk_qh(0);
+            ok = state_qh(0);
             const float* s0row = S0 ? S0 + ((size_t)blockIdx.x * kD + row) * kD : nullptr;
 #pragma unroll 1
             for (int pair = 0; pair < 2; ++pair) {
@@ -539,8 +531,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int n = 0; n < nchunks && ok; ++n) {
             const int t0 = n * kC;
             const int stg = n & 1;
-            const uint32_t txn = tmem + (stg ? TM_X1 : TM_X0);
             const uint32_t tgn = stg ? TM_G1 : TM_G;
+            const uint32_t kqn = sb + (stg ? SM_KQ1 : SM_KQ0);
             const uint32_t pbuf = stg ? SM_P1 : SM_P0;
             const bool last = (n + 1 == nchunks);
             if (tid < 64 && !last) la_n = gate(log_alpha, t0 + kC + tid);   // next chunk's decay
@@ -567,31 +559,62 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
             if (issuer) {
                 tc::mbar_arrive(&bars[B_GFREE]);   // W^T read: the prep may reuse this TMEM buffer
-                // V and this chunk's q/k stage have been read (W/X MMAs, Gram, (D K)^T, Qh)
-                tc::fence_proxy_async_smem();
+                tc::fence_proxy_async_smem();      // V has been read by the W/X MMAs
                 if (n + 1 < nchunks) load_v(n + 1);
-                if (n + 2 < nchunks) load_kq(n + 2);
             }
             COMBA_PHASE(1);
             if (warp == 0) {   // MMA issue: the whole warp, one elected lane
                 __syncwarp();   // reconverge after the single-thread block above
                 tc::tc_fence_after();
-                tc::mma_bf16_ta_bmn(txn, tmem + TM_SB, sb + SM_W, 8192, ID_SW, 8, 1);
+                tc::mma_bf16_ta_bmn(tmem + TM_X, tmem + TM_SB, sb + SM_W, 8192, ID_SW, 8, 1);
                 tc::mma_commit(&bars[B_MMA1]);
                 tc::mma_bf16_ta_bk(tmem + TM_O, tmem + TM_SB, sb + SM_QH, QH_ATOM, ID_SQ, 8, 0);
-                ok = tc::mbar_wait(&bars[B_MMA1], n & 1, timeout_ns);
-                if (ok) {
-                    tc::tc_fence_after();
-                    tc::mma_tf32_ta_bk(tmem + TM_S, txn, sb + SM_DK, DKT_ATOM, ID_SU, 8, 1);
-                    tc::mma_tf32_ta_bk(tmem + TM_O, txn, sb + pbuf, F32_ATOM, ID_XP, 8, 1);
-                    tc::mma_commit(&bars[B_MMA2]);
+            }
+            // ---- X' = X diag(e^{g_L - g}) as bf16 hi + lo (operand of the state update)
+            ok = ok && tc::mbar_wait(&bars[B_MMA1], n & 1, timeout_ns);
+            tc::tc_fence_after();
+            COMBA_PHASE(6);
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float xv[32], hv[16], lv[16];
+                tc::tmem_ld32(tl + TM_X + 32 * half, xv);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float4 d4 = tc::lds_f32x4(SED + 4u * (32 * half + 4 * c));
+                    const float a0 = xv[4 * c] * d4.x, a1 = xv[4 * c + 1] * d4.y;
+                    const float a2 = xv[4 * c + 2] * d4.z, a3 = xv[4 * c + 3] * d4.w;
+                    const uint32_t h01 = tc::pack_bf16(a0, a1), h23 = tc::pack_bf16(a2, a3);
+                    hv[2 * c] = __uint_as_float(h01);
+                    hv[2 * c + 1] = __uint_as_float(h23);
+                    lv[2 * c] = __uint_as_float(tc::pack_bf16(a0 - __uint_as_float(h01 << 16),
+                                                              a1 - __uint_as_float(h01 & 0xffff0000u)));
+                    lv[2 * c + 1] = __uint_as_float(tc::pack_bf16(a2 - __uint_as_float(h23 << 16),
+                                                                  a3 - __uint_as_float(h23 & 0xffff0000u)));
                 }
-                if (!ok) fail(gabort);
+                tc::tmem_st16(tl + TM_XH + 16 * half, hv);
+                tc::tmem_st16(tl + TM_XH + 32 + 16 * half, lv);
+            }
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            if (!ok) fail(gabort);
+            if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
+            if (warp == 0) {
+                __syncwarp();
+                tc::tc_fence_after();
+                tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH, kqn, KQ_ATOM, ID_SK, 4, 1);
+                tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH + 32, kqn, KQ_ATOM, ID_SK, 4, 1);
+                tc::mma_tf32_ta_bk(tmem + TM_O, tmem + TM_X, sb + pbuf, F32_ATOM, ID_XP, 8, 1);
+                tc::mma_commit(&bars[B_MMA2]);
             }
             ok = ok && tc::mbar_wait(&bars[B_MMA2], n & 1, timeout_ns);
             if (!ok) fail(gabort);
             if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
             tc::tc_fence_after();
+            if (issuer && n + 2 < nchunks) {   // this chunk's q/k stage is read (MMAs, Qh)
+                tc::fence_proxy_async_smem();
+                load_kq(n + 2);
+            }
             COMBA_PHASE(2);
             // O^T row (value index) -> bf16 pairs of tokens
             uint32_t ob[32];
@@ -663,7 +686,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             COMBA_PHASE(4);
             if (!last) {
-                const bool okd = state_dk_qh(n + 1);
+                const bool okd = state_qh(n + 1);
                 if (!okd) fail(gabort);
                 if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, okd && *gabort == 0)) break;
             }
@@ -694,7 +717,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const int t0 = m * kC;
             const int stg = m & 1;
             const uint32_t kq_a = sb + (stg ? SM_KQ1 : SM_KQ0);
-            const uint32_t txm = tmem + (stg ? TM_X1 : TM_X0);
             const uint32_t tgm = stg ? TM_G1 : TM_G;    // Gram, then W^T, of this chunk
             const bool last = (m + 1 == nchunks);
             bool ok = (*gabort == 0);
@@ -838,14 +860,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // W^T that buffer held
             if (pw == 0) {   // MMA issue: the whole warp, one elected lane
                 __syncwarp();   // reconverge after the per-thread code above
+                // V in; W^T of chunk m-1 read (this chunk's next-Gram buffer); X^T of
+                // chunk m-1 read by its MMA2
                 ok = ok && tc::mbar_wait(&bars[B_V], m & 1, timeout_ns) &&
-                     (m == 0 || tc::mbar_wait(&bars[B_GFREE], (m - 1) & 1, timeout_ns));
+                     (m == 0 || (tc::mbar_wait(&bars[B_GFREE], (m - 1) & 1, timeout_ns) &&
+                                 tc::mbar_wait(&bars[B_MMA2], (m - 1) & 1, timeout_ns)));
                 COMBA_PHASE(25);
                 if (ok) {
                     tc::tc_fence_after();
                     tc::mma_amn_bk(tmem + tgm, kq_a, KQ_ATOM, F1, ID_WN, 4, 0);
-                    tc::mma_amn_bk(txm, sb + SM_V, V_ATOM, F1 + 8192, ID_WN, 4, 0);
-                    tc::mma_amn_bk(txm, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
+                    tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, F1 + 8192, ID_WN, 4, 0);
+                    tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
                     tc::mma_commit(&bars[B_WN]);
                     COMBA_PHASE(26);
                     const int m1 = m + 1;
