@@ -46,8 +46,11 @@ constexpr int kD = 128;
 constexpr int kThreads = 384;        // warps 0-3: state group; warps 4-11: prep group
 constexpr int kStateThreads = 128;
 constexpr int kPrepThreads = 256;
-constexpr int BAR_PREP = 1;          // named barrier ids
-constexpr int BAR_STATE = 2;
+constexpr int BAR_PREP = 1;          // named barrier ids: the prep group
+constexpr int BAR_STATE = 2;         // the state group
+constexpr int BAR_KK = 3;            // K K^T staged (3 warps arrive) -> P warps (3 warps wait)
+constexpr int BAR_GATES = 4;         // the two gate warps
+constexpr int kKKThreads = 192;
 
 // TMEM columns (fp32, 128 lanes)
 constexpr uint32_t TM_G = 0;     // Gram of even chunks (lanes 0-63 K K^T, 64-127 Q K^T), then W^T
@@ -60,18 +63,19 @@ constexpr uint32_t TM_S = 384;   // fp32 state master (lane i, column j)
 constexpr uint32_t TM_COLS = 512;
 
 // Shared memory (bytes from a 1024-aligned base).
-constexpr uint32_t SM_KQ0 = 0;        // [K;Q] stage 0: 2 K-atoms x 128 rows x 128 B (bf16)
-constexpr uint32_t SM_KQ1 = 32768;    // stage 1
-constexpr uint32_t SM_V = 65536;      // V: 2 dv-atoms x 64 tokens x 128 B
-constexpr uint32_t SM_W = 81920;      // -W bf16, MN-major: 128 rows (j) x 64 tokens
-constexpr uint32_t SM_P0 = 98304;     // P fp32, K-major: 2 atoms (32 s) x 64 rows; even chunks
-constexpr uint32_t SM_P1 = 114688;    // odd chunks (K K^T is staged here first, P formed in place)
-constexpr uint32_t SM_F1 = 131072;    // fp32 64x64: A; then Tc (bf16) | Eb (bf16)
-constexpr uint32_t SM_F2 = 147456;    // fp32 64x64: Tinv (upper blocks: scratch)
-constexpr uint32_t SM_BLO = 163840;   // bf16 64x64 K-major: diag(lo(beta)), zero elsewhere
-constexpr uint32_t SM_QH = 172032;    // Qh bf16, K-major like Q: 2 atoms (64 j) x 64 tokens
-constexpr uint32_t SM_MISC = 188416;  // gates, barriers
-constexpr uint32_t SM_END = SM_MISC + 4096;
+constexpr int kKQStages = 3;          // q/k tiles in flight: chunk c in stage c % 3
+constexpr uint32_t SM_KQ0 = 0;        // [K;Q] stages: 2 K-atoms x 128 rows x 128 B (bf16) each
+constexpr uint32_t KQ_STAGE = 32768;
+constexpr uint32_t SM_V = 98304;      // V: 2 dv-atoms x 64 tokens x 128 B
+constexpr uint32_t SM_W = 114688;     // -W bf16, MN-major: 128 rows (j) x 64 tokens
+constexpr uint32_t SM_P0 = 131072;    // P fp32, K-major: 2 atoms (32 s) x 64 rows; even chunks
+constexpr uint32_t SM_P1 = 147456;    // odd chunks (K K^T is staged here first, P formed in place)
+constexpr uint32_t SM_F1 = 163840;    // fp32 64x64: A; then Tc (bf16) | Eb (bf16)
+constexpr uint32_t SM_F2 = 180224;    // fp32 64x64: Tinv (upper blocks: scratch)
+constexpr uint32_t SM_BLO = 196608;   // bf16 64x64 K-major: diag(lo(beta)), zero elsewhere
+constexpr uint32_t SM_QH = 204800;    // Qh bf16, K-major like Q: 2 atoms (64 j) x 64 tokens
+constexpr uint32_t SM_MISC = 221184;  // gate tables, barriers
+constexpr uint32_t SM_END = SM_MISC + 8192;
 constexpr uint32_t kSmemBytes = SM_END + 1024;
 
 constexpr uint32_t KQ_ATOM = 16384;
@@ -100,24 +104,16 @@ __device__ __forceinline__ uint32_t faddr(uint32_t base, int r, int s) {
     return base + 4u * (uint32_t)fidx(r, s);
 }
 
-// Inside diagonal block blk (parity P = blk & 1), fidx(16 blk + r, 16 blk + s) =
-// 16 blk 64 + 32 (blk >> 1) + r 64 + ((s ^ fswz_blk(r)) ^ 18 P), with fswz_blk(r) the
-// row swizzle of an even block: the parity flips bits 1 and 4 of the column.
-__device__ __forceinline__ constexpr int fswz_blk(int r) { return ((r & 3) << 3) | (r & 4) | (r >> 3); }
-
-// Diagonal 16 x 16 block `blk` of (I + A)^{-1} (A strictly lower, fp32 at F1)
-// into F2: one warp, lane j < 16 owns column j, right-looking substitution.
-// The loads use four base pointers, one per value of column bits 1 and 4, so
-// that every offset is a compile-time constant for either parity (one copy of
-// the code for all four blocks).
-__device__ __forceinline__ void diag_block_inverse(uint32_t F1, uint32_t F2, int blk, int lane) {
-    const int P = blk & 1;
-    const uint32_t base = 4u * (uint32_t)(16 * blk * 64 + 32 * (blk >> 1));
-    const uint32_t Ab = F1 + base;
-    const int d1 = 2 * P, d4 = 16 * P;
-    const uint32_t bb[4] = {Ab + 4u * (uint32_t)(d1 + d4), Ab + 4u * (uint32_t)(-d1 + d4),
-                            Ab + 4u * (uint32_t)(d1 - d4), Ab + 4u * (uint32_t)(-d1 - d4)};
-    const int j = lane & 15;
+// Diagonal blocks 2p and 2p+1 of Tinv = (I + A)^{-1} from A rows held in registers:
+// one warp, lane l holds row 32p + l of A over columns 32p .. 32p + 31 in a[].
+// Lanes 0-15 invert block 2p, lanes 16-31 block 2p + 1; lane l owns column l & 15
+// of its block (right-looking substitution, the A entries taken from the lane that
+// holds the row by shuffle), and writes it to F2.
+__device__ __forceinline__ void diag_pair_inverse(const float (&a)[32], uint32_t F2, int p, int lane) {
+    const int hb = lane >> 4, j = lane & 15, src = lane & 16;
+    float al[16];
+#pragma unroll
+    for (int s = 0; s < 16; ++s) al[s] = hb ? a[16 + s] : a[s];
     float x[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
@@ -125,18 +121,12 @@ __device__ __forceinline__ void diag_block_inverse(uint32_t F1, uint32_t F2, int
     for (int s = 0; s < 15; ++s) {
         const float xs = x[s];
 #pragma unroll
-        for (int r = s + 1; r < 16; ++r) {
-            const int c = s ^ fswz_blk(r);
-            const int sel = ((c >> 1) & 1) | (((c >> 4) & 1) << 1);
-            x[r] = fmaf(-tc::lds_f32(bb[sel] + 4u * (uint32_t)(r * 64 + c)), xs, x[r]);
-        }
+        for (int r = s + 1; r < 16; ++r)
+            x[r] = fmaf(-__shfl_sync(0xffffffffu, al[s], src | r), xs, x[r]);
     }
-    if (lane < 16) {
-        const uint32_t Tb = F2 + base;
+    const int blk = 2 * p + hb;
 #pragma unroll
-        for (int r = 0; r < 16; ++r)
-            tc::sts_f32(Tb + 4u * (uint32_t)(r * 64 + ((j ^ fswz_blk(r)) ^ (18 * P))), x[r]);
-    }
+    for (int r = 0; r < 16; ++r) tc::sts_f32(faddr(F2, 16 * blk + r, 16 * blk + j), x[r]);
 }
 
 __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
@@ -313,37 +303,6 @@ __device__ __forceinline__ void offdiag_inverse(uint32_t F1, uint32_t F2, int pt
     }
 }
 
-// Exact-exponential fallbacks for a chunk whose total log-decay is at or
-// below -80 (e^{-g} would leave the normal fp32 range): each entry takes exp2
-// of its own exponent difference.  Kept out of line: they are rarely taken.
-__device__ __noinline__ void a_row_exact(uint32_t F1, uint32_t gram_taddr, int r, int s0, float br,
-                                         float gpr, uint32_t G2) {
-    float gv[32];
-    tc::tmem_ld32(gram_taddr, gv);
-    tc::tmem_ld_wait();
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-        const int s = s0 + e;
-        const float v = br * exp2f(gpr - tc::lds_f32(G2 + 4u * s)) * gv[e];
-        tc::sts_f32(faddr(F1, r, s), (s < r) ? v : 0.f);
-    }
-}
-
-__device__ __noinline__ void p_row_exact(uint32_t prow, uint32_t gram_taddr, int r, int s0,
-                                         float dh, uint32_t G2) {
-    float gv[32];
-    tc::tmem_ld32(gram_taddr, gv);
-    tc::tmem_ld_wait();
-    const float gr = tc::lds_f32(G2 + 4u * r);
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-        const int s = s0 + e;
-        const uint32_t pa = prow + tc::sw128(r, e >> 2) + 4u * (e & 3);
-        const float v = exp2f(gr - tc::lds_f32(G2 + 4u * s)) * fmaf(-dh, tc::lds_f32(pa), gv[e]);
-        tc::sts_f32(pa, (s <= r) ? v : 0.f);
-    }
-}
-
 __device__ __forceinline__ void fail(volatile int* gabort) {
     *gabort = 1;
     latch_status(-4 /* COMBA_ETIMEOUT */);
@@ -355,30 +314,31 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const float* __restrict__ log_alpha, const float* __restrict__ beta,
                     const float* __restrict__ dvec, const float* S0, float* S_final, int T, int H,
                     unsigned long long timeout_ns) {
+    COMBA_CTA_MARK(0);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
     uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     const uint32_t sb = tc::smem_u32(sm);
 
-    // gate tables (64 fp32 each), by shared address; the prep group's and the state group's
-    const uint32_t G2 = sb + SM_MISC;        // g_r log2(e)
-    const uint32_t GP2 = G2 + 256;           // g_{r-1} log2(e)
-    const uint32_t BT = G2 + 512;            // beta_r
-    const uint32_t CS = G2 + 768;            // beta_r e^{g_{r-1}}
-    const uint32_t EG = G2 + 1024;           // e^{g_r}
-    const uint32_t IEG = G2 + 1536;          // e^{-g_r} (when the chunk allows)
-    const uint32_t RED = G2 + 1792;          // [0..1] scan carries
-    const uint32_t SRED = G2 + 1936;         // state group: [0..1] scan carries
-    const uint32_t SED = G2 + 2048;          // state group: e^{g_L - g_r} of the next chunk
-    const uint32_t SEG = G2 + 2304;          // state group: e^{g_r} of the next chunk
-    // barriers: q/k stages, v, gram, wn (W^T, U~^T in TMEM), mma1 (X), mma2, the P
-    // buffers (MMA2 and the out store have read them) and the Gram/W^T TMEM buffer
-    // (the state group has read W^T).  Each is arrived on once per phase (by a
-    // commit, a TMA transaction count or one thread after its group's named
-    // barrier): many arrivals on one barrier serialise in the shared-memory pipe.
-    enum { B_KQ0 = 0, B_KQ1 = 1, B_V = 2, B_GRAM = 3, B_WN = 4, B_MMA1 = 5, B_MMA2 = 6, B_PBUF0 = 7,
-           B_PBUF1 = 8, B_GFREE = 9, NBARS = 10 };
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 2560);
+    // Prep gate tables, two sets (chunk c uses set c & 1; the next chunk's set is
+    // built while the current one is in use), 64 fp32 each, by shared address:
+    //   +0 g_r log2(e), +256 g_{r-1} log2(e), +512 beta_r, +768 beta_r e^{g_{r-1}},
+    //   +1024 e^{g_r}, +1280 e^{-g_r} (when the chunk allows), +1536 the chunk's
+    //   "fast" flag (total log-decay above -80)
+    auto tset = [&](int c) -> uint32_t { return sb + SM_MISC + 2048u * (uint32_t)(c & 1); };
+    const uint32_t RED = sb + SM_MISC + 4096;   // gate warps: [0..1] scan carries
+    const uint32_t SRED = RED + 16;             // state group: [0..1] scan carries
+    // state group, per chunk parity: e^{g_L - g_r} (SED) and e^{g_r} (SEG) of a chunk
+    auto sed = [&](int c) -> uint32_t { return sb + SM_MISC + 4352u + 512u * (uint32_t)(c & 1); };
+    auto seg = [&](int c) -> uint32_t { return sed(c) + 256u; };
+    // barriers: q/k stages, v, gram per TMEM buffer, wn (W^T, U~^T in TMEM), mma1 (X),
+    // mma2, the P buffers (MMA2 and the out store have read them) and the Gram/W^T
+    // TMEM buffers (the state group has read W^T).  Each is arrived on once per
+    // phase (by a commit, a TMA transaction count or one thread after its group's
+    // named barrier): many arrivals on one barrier serialise in the shared-memory pipe.
+    enum { B_KQ0 = 0, B_V = 3, B_GRAM0 = 4, B_GRAM1 = 5, B_WN = 6, B_MMA1 = 7, B_MMA2 = 8,
+           B_PBUF0 = 9, B_PBUF1 = 10, B_GFREE = 11, B_MMA1B = 12, NBARS = 13 };
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 6144);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
     volatile int* gabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
     const uint32_t F1 = sb + SM_F1, F2 = sb + SM_F2;
@@ -408,9 +368,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t tmem = *tmem_slot;
     const uint32_t tl = tmem + trow;    // this thread's TMEM lane, column 0
 
+    auto kq_stage = [&](int n) -> uint32_t { return SM_KQ0 + KQ_STAGE * (uint32_t)(n % kKQStages); };
+    auto kq_bar = [&](int n) -> uint64_t* { return &bars[B_KQ0 + n % kKQStages]; };
+    auto kq_par = [&](int n) -> uint32_t { return (uint32_t)(n / kKQStages) & 1u; };
     auto load_kq = [&](int n) {
-        uint8_t* dst = sm + ((n & 1) ? SM_KQ1 : SM_KQ0);
-        uint64_t* bar = &bars[n & 1];
+        uint8_t* dst = sm + kq_stage(n);
+        uint64_t* bar = kq_bar(n);
         tc::mbar_arrive_expect_tx(bar, 32768);
         const int t0 = n * kC;
         tc::tma_load_4d(dst, &tm_k, bar, 0, h, t0, b);
@@ -446,9 +409,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // scan of its log-decays.
         const int row = tid;
         const bool issuer = (tid == 0);
-        // Scan of one chunk's log-decays held by threads 0..63: writes e^{g_L - g_r}
-        // to SED and e^{g_r} to SEG, and returns e^{g_L} to every thread of the group.
-        auto state_gates = [&](float la) -> float {
+        // Scan of chunk c's log-decays held by threads 0..63: writes e^{g_L - g_r} to
+        // sed(c) and e^{g_r} to seg(c), and returns e^{g_L} to every thread of the group.
+        auto state_gates = [&](float la, int c) -> float {
             float x = la;
             if (tid < 64) {
 #pragma unroll
@@ -462,17 +425,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const float c0 = tc::lds_f32(SRED), gL = c0 + tc::lds_f32(SRED + 4u);
             if (tid < 64) {
                 const float g = x + (tid >= 32 ? c0 : 0.f);
-                tc::sts_f32(SED + 4u * tid, __expf(gL - g));
-                tc::sts_f32(SEG + 4u * tid, __expf(g));
+                tc::sts_f32(sed(c) + 4u * tid, __expf(gL - g));
+                tc::sts_f32(seg(c) + 4u * tid, __expf(g));
             }
             return __expf(gL);
         };
         // Qh = diag(e^g)(Q - d K) of chunk c (bf16, K-major like Q), from its q/k tiles.
         auto state_qh = [&](int c) -> bool {
-            const bool okc = tc::mbar_wait(&bars[c & 1], (c >> 1) & 1, timeout_ns);
-            const uint32_t kqc = sb + ((c & 1) ? SM_KQ1 : SM_KQ0);
+            const bool okc = tc::mbar_wait(kq_bar(c), kq_par(c), timeout_ns);
+            const uint32_t kqc = sb + kq_stage(c);
             const int r = tid & 63, jh = tid >> 6;
-            const float egr = tc::lds_f32(SEG + 4u * r);
+            const float egr = tc::lds_f32(seg(c) + 4u * r);
 #pragma unroll 2
             for (int c8 = 0; c8 < 8; ++c8) {
                 const uint32_t off = kqc + jh * KQ_ATOM + tc::sw128(r, c8);
@@ -495,7 +458,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // decays and Qh of chunk 0, initial state
         {
             const float la0 = (tid < 64) ? gate(log_alpha, tid) : 0.f;
-            const float eL0 = state_gates(la0);
+            const float eL0 = state_gates(la0, 0);
             tc::named_barrier(BAR_STATE, kStateThreads);
             ok = state_qh(0);
             const float* s0row = S0 ? S0 + ((size_t)blockIdx.x * kD + row) * kD : nullptr;
@@ -527,17 +490,20 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!ok) fail(gabort);
             ok = tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok);
         }
-        float la_n = 0.f;
+        // next chunk's log-decay (threads 0..63), loaded a chunk ahead of its scan
+        float la_n = (tid < 64 && nchunks > 1) ? gate(log_alpha, kC + tid) : 0.f;
         for (int n = 0; n < nchunks && ok; ++n) {
             const int t0 = n * kC;
             const int stg = n & 1;
             const uint32_t tgn = stg ? TM_G1 : TM_G;
-            const uint32_t kqn = sb + (stg ? SM_KQ1 : SM_KQ0);
+            const uint32_t kqn = sb + kq_stage(n);
             const uint32_t pbuf = stg ? SM_P1 : SM_P0;
             const bool last = (n + 1 == nchunks);
-            if (tid < 64 && !last) la_n = gate(log_alpha, t0 + kC + tid);   // next chunk's decay
-            // ---- -W operand from W^T (lane = j, column = token) once the prep's MMAs are done
+            // ---- -W operand from W^T (lane = j, column = token) once the prep's MMAs are
+            // done and the previous chunk's out store has read its staging (same buffer)
             ok = (*gabort == 0) && tc::mbar_wait(&bars[B_WN], n & 1, timeout_ns);
+            if (issuer) tc::bulk_wait_read0();
+            tc::named_barrier(BAR_STATE, kStateThreads);
             COMBA_PHASE(0);
             tc::tc_fence_after();
             {
@@ -569,11 +535,16 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::mma_bf16_ta_bmn(tmem + TM_X, tmem + TM_SB, sb + SM_W, 8192, ID_SW, 8, 1);
                 tc::mma_commit(&bars[B_MMA1]);
                 tc::mma_bf16_ta_bk(tmem + TM_O, tmem + TM_SB, sb + SM_QH, QH_ATOM, ID_SQ, 8, 0);
+                tc::mma_commit(&bars[B_MMA1B]);
             }
+            // ---- while MMA1 runs: the next chunk's decays
+            const float eLn = last ? 1.f : state_gates(la_n, n + 1);
+            if (tid < 64 && n + 2 < nchunks) la_n = gate(log_alpha, t0 + 2 * kC + tid);
             // ---- X' = X diag(e^{g_L - g}) as bf16 hi + lo (operand of the state update)
             ok = ok && tc::mbar_wait(&bars[B_MMA1], n & 1, timeout_ns);
             tc::tc_fence_after();
             COMBA_PHASE(6);
+            const uint32_t sedn = sed(n);
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
                 float xv[32], hv[16], lv[16];
@@ -581,7 +552,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::tmem_ld_wait();
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const float4 d4 = tc::lds_f32x4(SED + 4u * (32 * half + 4 * c));
+                    const float4 d4 = tc::lds_f32x4(sedn + 4u * (32 * half + 4 * c));
                     const float a0 = xv[4 * c] * d4.x, a1 = xv[4 * c + 1] * d4.y;
                     const float a2 = xv[4 * c + 2] * d4.z, a3 = xv[4 * c + 3] * d4.w;
                     const uint32_t h01 = tc::pack_bf16(a0, a1), h23 = tc::pack_bf16(a2, a3);
@@ -607,15 +578,26 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::mma_tf32_ta_bk(tmem + TM_O, tmem + TM_X, sb + pbuf, F32_ATOM, ID_XP, 8, 1);
                 tc::mma_commit(&bars[B_MMA2]);
             }
+            COMBA_PHASE(2);
+            // ---- while MMA2 runs: Qh of the next chunk (MMA1 has read this chunk's)
+            if (!last) {
+                ok = ok && tc::mbar_wait(&bars[B_MMA1B], n & 1, timeout_ns);
+                ok = state_qh(n + 1) && ok;
+            }
+            COMBA_PHASE(3);
             ok = ok && tc::mbar_wait(&bars[B_MMA2], n & 1, timeout_ns);
             if (!ok) fail(gabort);
             if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
             tc::tc_fence_after();
-            if (issuer && n + 2 < nchunks) {   // this chunk's q/k stage is read (MMAs, Qh)
-                tc::fence_proxy_async_smem();
-                load_kq(n + 2);
+            if (issuer) {   // P of this chunk and its q/k stage are read
+                tc::mbar_arrive(&bars[stg ? B_PBUF1 : B_PBUF0]);
+                if (n + kKQStages < nchunks) {
+                    tc::fence_proxy_async_smem();
+                    load_kq(n + kKQStages);
+                }
             }
-            COMBA_PHASE(2);
+            __syncwarp();
+            COMBA_PHASE(4);
             // O^T row (value index) -> bf16 pairs of tokens
             uint32_t ob[32];
             {
@@ -629,7 +611,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ob[16 + c] = tc::pack_bf16(o1[2 * c], o1[2 * c + 1]);
                 }
             }
-            const float eLn = last ? 1.f : state_gates(la_n);
             float* sfrow = (last && S_final) ? S_final + ((size_t)blockIdx.x * kD + row) * kD : nullptr;
 #pragma unroll 1
             for (int pair = 0; pair < 2; ++pair) {
@@ -661,13 +642,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             tc::tmem_st_wait();
             tc::tc_fence_before();
-            COMBA_PHASE(3);
+            COMBA_PHASE(5);
             // out tile [token][value index] in two 64-wide 128B-swizzled boxes, staged in
-            // this chunk's P buffer (MMA2 has read it), TMA store; once the store has
-            // read it the buffer goes back to the prep group.  The barrier below also
-            // hands the new S copies to the next MMA1.
+            // the -W buffer (MMA1 has read it), TMA store.  The barrier below also hands
+            // the new S copies to the next MMA1.
             {
-                const uint32_t ot = sb + pbuf + (row >> 6) * 8192 + (row & 7) * 2;
+                const uint32_t ot = sb + SM_W + (row >> 6) * 8192 + (row & 7) * 2;
                 const int oc = (row & 63) >> 3;
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
@@ -678,217 +658,236 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::fence_proxy_async_smem();
             tc::named_barrier(BAR_STATE, kStateThreads);
             if (issuer) {
-                tc::tma_store_4d(&tm_o, sm + pbuf, 0, h, t0, b);
-                tc::tma_store_4d(&tm_o, sm + pbuf + 8192, 64, h, t0, b);
+                tc::tma_store_4d(&tm_o, sm + SM_W, 0, h, t0, b);
+                tc::tma_store_4d(&tm_o, sm + SM_W + 8192, 64, h, t0, b);
                 tc::bulk_commit();
-                tc::bulk_wait_read0();
-                tc::mbar_arrive(&bars[stg ? B_PBUF1 : B_PBUF0]);
             }
-            COMBA_PHASE(4);
-            if (!last) {
-                const bool okd = state_qh(n + 1);
-                if (!okd) fail(gabort);
-                if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, okd && *gabort == 0)) break;
-            }
-            COMBA_PHASE(5);
             COMBA_ITER_NEXT();
         }
         if (issuer) tc::bulk_wait0();
     } else {
         // =============================== prep group ================================
-        // Per chunk m (running one chunk ahead of the state group): gates, Gram, P, A,
-        // the inverse, Tc/Eb, then the MMAs W^T = K^T Tc^T and U~^T (= X^T before MMA1),
-        // and the next chunk's Gram.
+        // Chunk m's operands for the state group: the inverse's blocks, Tc / Eb, P,
+        // then the MMAs W^T = K^T Tc^T and U~^T (= X^T before MMA1).  Warp pw reads
+        // TMEM lanes 32 (pw & 3) .. + 31 of the Gram, columns 32 (pw >> 2) .. + 31:
+        //   pw 0, 1, 5: K K^T rows (0-31, 32-63, 32-63) x columns (0-31, 0-31, 32-63):
+        //               A in registers, K K^T staged for P; pw 0 and 5 then invert the
+        //               diagonal blocks (0, 1) and (2, 3) from their registers
+        //   pw 2, 3, 7: Q K^T of the same row/column blocks: P, once K K^T is staged
+        //   pw 6:       P rows 0-31 x columns 32-63 are zero (s > r); issues the next
+        //               chunk's Gram
+        //   pw 1, 4:    the next chunk's gate tables;  pw 4 issues this chunk's W/X MMAs
+        // then all eight warps: the off-diagonal blocks, Tc / Eb, diag(lo(beta)).
         const int pt = tid - kStateThreads;
-        const int prow = pt & 127, phalf = pt >> 7, pw = pt >> 5;
+        const int pw = pt >> 5, q = pw & 3, ch = pw >> 2;
         const bool issuer = (pt == 0);
-        bool gram_issued = false;   // Gram of the current chunk already issued (early)
-        float la_c = 0.f, bt_c = 0.f, la_n = 0.f, bt_n = 0.f;
-        if (pt < 64) {
-            la_c = gate(log_alpha, pt);
-            bt_c = gate(beta, pt);
-        }
+        const int gtok = (pw == 1) ? lane : 32 + lane;   // gate warps: token of this thread
+        float la_x = 0.f, bt_x = 0.f;                     // gate warps: next chunk's values
+        // gate tables of chunk c into tset(c) from this thread's token values (gate warps)
+        auto make_tables = [&](int c, float la, float bt) {
+            float x = la;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, off);
+                if (lane >= off) x += y;
+            }
+            if (lane == 31) tc::sts_f32(RED + (pw == 1 ? 0u : 4u), x);
+            tc::named_barrier(BAR_GATES, 64);
+            const float c0 = tc::lds_f32(RED), gL = c0 + tc::lds_f32(RED + 4u);
+            const bool fst = gL > -80.f;
+            const float g = x + (pw == 4 ? c0 : 0.f), gp = g - la;
+            const uint32_t ts = tset(c);
+            tc::sts_f32(ts + 4u * gtok, g * kLog2e);
+            tc::sts_f32(ts + 256 + 4u * gtok, gp * kLog2e);
+            tc::sts_f32(ts + 512 + 4u * gtok, bt);
+            tc::sts_f32(ts + 768 + 4u * gtok, bt * __expf(gp));
+            tc::sts_f32(ts + 1024 + 4u * gtok, __expf(g));
+            tc::sts_f32(ts + 1280 + 4u * gtok, fst ? __expf(-g) : 0.f);
+            if (gtok == 0) asm volatile("st.shared.u32 [%0], %1;" ::"r"(ts + 1536), "r"(fst ? 1u : 0u) : "memory");
+            tc::named_barrier(BAR_GATES, 64);   // RED is reused by the next call
+        };
+        // Gram ([K;Q] K^T) of chunk c into its TMEM buffer (warp pw 6, one elected lane)
+        auto issue_gram = [&](int c) -> bool {
+            __syncwarp();
+            bool okg = tc::mbar_wait(kq_bar(c), kq_par(c), timeout_ns) &&
+                       (c < 2 || tc::mbar_wait(&bars[B_GFREE], (c - 2) & 1, timeout_ns));
+            if (okg) {
+                const uint32_t kq = sb + kq_stage(c);
+                tc::tc_fence_after();
+                tc::mma_ak_bk(tmem + ((c & 1) ? TM_G1 : TM_G), kq, KQ_ATOM, kq, KQ_ATOM, ID_G, 8, 0);
+                tc::mma_commit(&bars[(c & 1) ? B_GRAM1 : B_GRAM0]);
+            }
+            return okg;
+        };
+        bool ok = true;
         if (issuer) {
-            load_kq(0);
-            if (nchunks > 1) load_kq(1);
+            for (int c = 0; c < kKQStages && c < nchunks; ++c) load_kq(c);
             load_v(0);
         }
-        for (int m = 0; m < nchunks; ++m) {
-            const int t0 = m * kC;
-            const int stg = m & 1;
-            const uint32_t kq_a = sb + (stg ? SM_KQ1 : SM_KQ0);
-            const uint32_t tgm = stg ? TM_G1 : TM_G;    // Gram, then W^T, of this chunk
+        if (pw == 1 || pw == 4) {
+            make_tables(0, gate(log_alpha, gtok), gate(beta, gtok));
+            if (nchunks > 1) {
+                la_x = gate(log_alpha, kC + gtok);
+                bt_x = gate(beta, kC + gtok);
+            }
+        }
+        if (pw == 6) ok = issue_gram(0);
+        if (!ok) fail(gabort);
+        ok = tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok);
+        for (int m = 0; m < nchunks && ok; ++m) {
             const bool last = (m + 1 == nchunks);
-            bool ok = (*gabort == 0);
-            // ---- Gram ([K;Q] K^T), unless it was issued during the previous chunk --------
-            if (pw == 0 && !gram_issued) {
-                __syncwarp();
-                COMBA_COUNT(14);
-                ok = ok && tc::mbar_wait(&bars[stg], (m >> 1) & 1, timeout_ns);
-                if (ok) {
-                    tc::tc_fence_after();
-                    tc::mma_ak_bk(tmem + tgm, kq_a, KQ_ATOM, kq_a, KQ_ATOM, ID_G, 8, 0);
-                    tc::mma_commit(&bars[B_GRAM]);
-                } else {
-                    fail(gabort);
-                }
-            }
-            gram_issued = false;
-            COMBA_PHASE(12);
-            // ---- gates --------------------------------------------------------------------
-            if (pt < 64) {
-                if (!last) {
-                    la_n = gate(log_alpha, t0 + kC + pt);
-                    bt_n = gate(beta, t0 + kC + pt);
-                }
-                float x = la_c;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, x, off);
-                    if (lane >= off) x += y;
-                }
-                if (lane == 31) tc::sts_f32(RED + 4u * pw, x);
-                tc::sts_f32(G2 + 4u * pt, x);
-            }
-            COMBA_PHASE(13);
-            tc::named_barrier(BAR_PREP, kPrepThreads);
-            COMBA_PHASE(22);
-            const float carry = tc::lds_f32(RED);
-            const float gL = carry + tc::lds_f32(RED + 4u);
-            const bool fast = gL > -80.f;
-            if (pt < 64) {
-                const float g = tc::lds_f32(G2 + 4u * pt) + (pt >= 32 ? carry : 0.f);
-                const float gp = g - la_c;
-                tc::sts_f32(BT + 4u * pt, bt_c);
-                tc::sts_f32(CS + 4u * pt, bt_c * __expf(gp));
-                tc::sts_f32(EG + 4u * pt, __expf(g));
-                tc::sts_f32(IEG + 4u * pt, fast ? __expf(-g) : 0.f);
-                tc::sts_f32(GP2 + 4u * pt, gp * kLog2e);
-                tc::sts_f32(G2 + 4u * pt, g * kLog2e);
-            }
-            COMBA_PHASE(23);
-            // Gram of this chunk in; the previous chunk's W/X MMAs have read F1 and BLO
-            ok = ok && tc::mbar_wait(&bars[B_GRAM], m & 1, timeout_ns) &&
-                 tc::mbar_wait(&bars[stg], (m >> 1) & 1, timeout_ns) &&
-                 (m == 0 || tc::mbar_wait(&bars[B_WN], (m - 1) & 1, timeout_ns));
-            COMBA_PHASE(24);
-            if (!ok) fail(gabort);
-            if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
-            tc::tc_fence_after();
-            COMBA_PHASE(16);
-            // ---- K K^T -> P buffer of this chunk (once MMA2 and the out store of chunk
-            // m-2 have read it), A -> F1
-            if (m >= 2) {
-                const bool okp = tc::mbar_wait(&bars[stg ? B_PBUF1 : B_PBUF0], ((m - 2) >> 1) & 1, timeout_ns);
-                if (!okp) fail(gabort);
-                if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, okp && *gabort == 0)) break;
-            }
-            const int s0 = phalf * 32;
-            const uint32_t prow_base = sb + (stg ? SM_P1 : SM_P0) + phalf * F32_ATOM;
-            float gv[32];
-            tc::tmem_ld32(tl + tgm + phalf * 32, gv);
-            tc::tmem_ld_wait();
-            if (prow < 64) {
-                const int r = prow;
+            const uint32_t ts = tset(m);
+            const uint32_t tgm = (m & 1) ? TM_G1 : TM_G;
+            const uint32_t pbm = sb + ((m & 1) ? SM_P1 : SM_P0);
+            const bool fast = tc::lds_u32(ts + 1536) != 0u;
+            ok = (*gabort == 0);
+            // ================= phase 1: A, K K^T, P, diagonal inverse blocks =================
+            if (pw == 0 || pw == 1 || pw == 5) {
+                const int r = 32 * q + lane;          // row (token) of this thread
+                ok = ok && tc::mbar_wait(&bars[(m & 1) ? B_GRAM1 : B_GRAM0], (m >> 1) & 1, timeout_ns) &&
+                     (m < 2 || tc::mbar_wait(&bars[(m & 1) ? B_PBUF1 : B_PBUF0], ((m - 2) >> 1) & 1, timeout_ns));
+                tc::tc_fence_after();
+                COMBA_PHASE(7);
+                float a[32];
+                tc::tmem_ld32(tl + tgm + 32 * ch, a);
+                tc::tmem_ld_wait();
+                COMBA_PHASE(8);
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
-                    tc::sts_f32x4(prow_base + tc::sw128(r, c),
-                                  make_float4(gv[4 * c], gv[4 * c + 1], gv[4 * c + 2], gv[4 * c + 3]));
+                    tc::sts_f32x4(pbm + ch * F32_ATOM + tc::sw128(r, c),
+                                  make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]));
+                tc::fence_proxy_async_smem();
+                tc::tc_fence_before();
+                tc::named_barrier_arrive(BAR_KK, kKKThreads);
+                // A_rs = beta_r e^{g_{r-1} - g_s} (K K^T)_rs for s < r, in registers
                 if (fast) {
-                    const float cr = tc::lds_f32(CS + 4u * r);
+                    const float cr = tc::lds_f32(ts + 768 + 4u * r);
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        const float4 ig = tc::lds_f32x4(IEG + 4u * (s0 + 4 * c));
+                        const float4 ig = tc::lds_f32x4(ts + 1280 + 4u * (32 * ch + 4 * c));
                         const float iv[4] = {ig.x, ig.y, ig.z, ig.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int s = s0 + 4 * c + e;
-                            tc::sts_f32(faddr(F1, r, s), (s < r) ? cr * iv[e] * gv[4 * c + e] : 0.f);
-                        }
+                        for (int e = 0; e < 4; ++e)
+                            a[4 * c + e] = (32 * ch + 4 * c + e < r) ? cr * iv[e] * a[4 * c + e] : 0.f;
                     }
                 } else {
-                    a_row_exact(F1, tl + tgm + phalf * 32, r, s0, tc::lds_f32(BT + 4u * r),
-                                tc::lds_f32(GP2 + 4u * r), G2);
+                    const float br = tc::lds_f32(ts + 512 + 4u * r), gpr = tc::lds_f32(ts + 256 + 4u * r);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int s = 32 * ch + e;
+                        a[e] = (s < r) ? br * exp2f(gpr - tc::lds_f32(ts + 4u * s)) * a[e] : 0.f;
+                    }
                 }
-            }
-            tc::tc_fence_before();
-            COMBA_PHASE(31);
-            tc::named_barrier(BAR_PREP, kPrepThreads);
-            // ---- P (in place over K K^T)  ||  diagonal inverse blocks ---------------------
-            if (prow >= 64) {
-                const int r = prow - 64;
-                const float er = tc::lds_f32(EG + 4u * r);
+                COMBA_PHASE(9);
+                if (pw != 1) diag_pair_inverse(a, F2, pw == 5 ? 1 : 0, lane);
+                COMBA_PHASE(10);
+                // A into F1 for the off-diagonal blocks (its lower blocks A_10, A_2x,
+                // A_3x only), once the previous chunk's W/X MMAs have read F1
+                ok = ok && (m == 0 || tc::mbar_wait(&bars[B_WN], (m - 1) & 1, timeout_ns));
+                COMBA_PHASE(11);
+                if (pw == 1) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) tc::sts_f32(faddr(F1, r, e), a[e]);
+                } else if (lane >= 16) {   // rows 16-31 x cols 0-15 (pw 0), 48-63 x 32-47 (pw 5)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) tc::sts_f32(faddr(F1, r, 32 * ch + e), a[e]);
+                }
+            } else if (pw == 2 || pw == 3 || pw == 7) {
+                const int r = 32 * (q - 2) + lane;    // row (token) of this thread
+                ok = ok && tc::mbar_wait(&bars[(m & 1) ? B_GRAM1 : B_GRAM0], (m >> 1) & 1, timeout_ns);
+                tc::tc_fence_after();
+                float gv[32];
+                tc::tmem_ld32(tl + tgm + 32 * ch, gv);
+                tc::tmem_ld_wait();
+                tc::tc_fence_before();
+                tc::named_barrier(BAR_KK, kKKThreads);
+                // P_rs = e^{g_r - g_s} (Q K^T - d K K^T)_rs for s <= r, in place over K K^T
+                const uint32_t prow = pbm + ch * F32_ATOM;
                 if (fast) {
+                    const float er = tc::lds_f32(ts + 1024 + 4u * r);
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        const uint32_t pa = prow_base + tc::sw128(r, c);
+                        const uint32_t pa = prow + tc::sw128(r, c);
                         const float4 kk = tc::lds_f32x4(pa);
-                        const float4 ig = tc::lds_f32x4(IEG + 4u * (s0 + 4 * c));
-                        const int s = s0 + 4 * c;
-                        float4 p;
-                        p.x = (s + 0 <= r) ? er * ig.x * fmaf(-dh, kk.x, gv[4 * c + 0]) : 0.f;
-                        p.y = (s + 1 <= r) ? er * ig.y * fmaf(-dh, kk.y, gv[4 * c + 1]) : 0.f;
-                        p.z = (s + 2 <= r) ? er * ig.z * fmaf(-dh, kk.z, gv[4 * c + 2]) : 0.f;
-                        p.w = (s + 3 <= r) ? er * ig.w * fmaf(-dh, kk.w, gv[4 * c + 3]) : 0.f;
-                        tc::sts_f32x4(pa, p);
+                        const float4 ig = tc::lds_f32x4(ts + 1280 + 4u * (32 * ch + 4 * c));
+                        const int s = 32 * ch + 4 * c;
+                        float4 pv;
+                        pv.x = (s + 0 <= r) ? er * ig.x * fmaf(-dh, kk.x, gv[4 * c + 0]) : 0.f;
+                        pv.y = (s + 1 <= r) ? er * ig.y * fmaf(-dh, kk.y, gv[4 * c + 1]) : 0.f;
+                        pv.z = (s + 2 <= r) ? er * ig.z * fmaf(-dh, kk.z, gv[4 * c + 2]) : 0.f;
+                        pv.w = (s + 3 <= r) ? er * ig.w * fmaf(-dh, kk.w, gv[4 * c + 3]) : 0.f;
+                        tc::sts_f32x4(pa, pv);
                     }
                 } else {
-                    p_row_exact(prow_base, tl + tgm + phalf * 32, r, s0, dh, G2);
+                    const float gr = tc::lds_f32(ts + 4u * r);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t pa = prow + tc::sw128(r, c);
+                        const float4 kk = tc::lds_f32x4(pa);
+                        const float kv[4] = {kk.x, kk.y, kk.z, kk.w};
+                        float pv[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int s = 32 * ch + 4 * c + e;
+                            pv[e] = (s <= r) ? exp2f(gr - tc::lds_f32(ts + 4u * s)) * fmaf(-dh, kv[e], gv[4 * c + e])
+                                             : 0.f;
+                        }
+                        tc::sts_f32x4(pa, make_float4(pv[0], pv[1], pv[2], pv[3]));
+                    }
                 }
-            } else {
-                diag_block_inverse(F1, F2, (pw & 1) + 2 * phalf, lane);
+                tc::fence_proxy_async_smem();
+            } else if (pw == 6) {
+                ok = ok && (m < 2 || tc::mbar_wait(&bars[(m & 1) ? B_PBUF1 : B_PBUF0], ((m - 2) >> 1) & 1, timeout_ns));
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    tc::sts_u32x4(pbm + F32_ATOM + tc::sw128(lane, c), make_uint4(0u, 0u, 0u, 0u));
+                tc::fence_proxy_async_smem();
+                // next chunk's Gram, into the TMEM buffer whose W^T (chunk m - 1) the state read
+                if (!last) ok = issue_gram(m + 1) && ok;
             }
-            COMBA_PHASE(30);
-            tc::named_barrier(BAR_PREP, kPrepThreads);
+            COMBA_PHASE(16);
+            // ================= phase 2: next chunk's gate tables (gate warps) =================
+            if ((pw == 1 || pw == 4) && !last) {
+                make_tables(m + 1, la_x, bt_x);
+                if (m + 2 < nchunks) {
+                    la_x = gate(log_alpha, (m + 2) * kC + gtok);
+                    bt_x = gate(beta, (m + 2) * kC + gtok);
+                }
+            }
+            if (!ok) fail(gabort);
             COMBA_PHASE(17);
-            // ---- off-diagonal blocks of the inverse, written out as Tc / Eb ----------------
-            offdiag_inverse(F1, F2, pt, CS, BT);
+            if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
             COMBA_PHASE(18);
-            if (pt < 64) {   // diag(lo(beta))
-                const float bv = tc::lds_f32(BT + 4u * pt);
+            // ================= phase 3: off-diagonal blocks of the inverse -> Tc / Eb ==========
+            offdiag_inverse(F1, F2, pt, ts + 768, ts + 512);
+            COMBA_PHASE(19);
+            if (pt < 64) {   // diag(lo(beta)) (the previous W/X MMAs are done: see F1 above)
+                const float bv = tc::lds_f32(ts + 512 + 4u * pt);
                 const float bh = __bfloat162float(__float2bfloat16_rn(bv));
                 const __nv_bfloat16 lo = __float2bfloat16_rn(bv - bh);
                 tc::sts_u16(sb + SM_BLO + tc::sw128(pt, pt >> 3) + (pt & 7) * 2,
                             *reinterpret_cast<const unsigned short*>(&lo));
             }
             tc::fence_proxy_async_smem();
-            tc::named_barrier(BAR_PREP, kPrepThreads);
-            COMBA_PHASE(19);
-            // ---- W^T = K^T Tc^T;  X^T = U~^T = V^T Eb^T + V^T diag(lo)^T --------------------
-            // (into TMEM; the state group turns W^T into its -W operand), then the next
-            // chunk's Gram into the other TMEM buffer once the state group has read the
-            // W^T that buffer held
-            if (pw == 0) {   // MMA issue: the whole warp, one elected lane
-                __syncwarp();   // reconverge after the per-thread code above
-                // V in; W^T of chunk m-1 read (this chunk's next-Gram buffer); X^T of
-                // chunk m-1 read by its MMA2
-                ok = ok && tc::mbar_wait(&bars[B_V], m & 1, timeout_ns) &&
-                     (m == 0 || (tc::mbar_wait(&bars[B_GFREE], (m - 1) & 1, timeout_ns) &&
-                                 tc::mbar_wait(&bars[B_MMA2], (m - 1) & 1, timeout_ns)));
-                COMBA_PHASE(25);
-                if (ok) {
+            if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
+            COMBA_PHASE(20);
+            // ================= phase 4: W^T = K^T Tc^T; X^T = U~^T = V^T Eb^T + V^T diag(lo)^T =====
+            // (warp pw 4; X^T of chunk m - 1 must have been read by its MMA2)
+            if (pw == 4) {
+                __syncwarp();
+                bool okw = tc::mbar_wait(&bars[B_V], m & 1, timeout_ns) &&
+                           (m == 0 || tc::mbar_wait(&bars[B_MMA2], (m - 1) & 1, timeout_ns));
+                if (okw) {
+                    const uint32_t kq = sb + kq_stage(m);
                     tc::tc_fence_after();
-                    tc::mma_amn_bk(tmem + tgm, kq_a, KQ_ATOM, F1, ID_WN, 4, 0);
+                    tc::mma_amn_bk(tmem + tgm, kq, KQ_ATOM, F1, ID_WN, 4, 0);
                     tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, F1 + 8192, ID_WN, 4, 0);
                     tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
                     tc::mma_commit(&bars[B_WN]);
-                    COMBA_PHASE(26);
-                    const int m1 = m + 1;
-                    if (!last && tc::mbar_try_wait(&bars[m1 & 1], (m1 >> 1) & 1)) {
-                        const uint32_t kq1 = sb + ((m1 & 1) ? SM_KQ1 : SM_KQ0);
-                        tc::tc_fence_after();
-                        tc::mma_ak_bk(tmem + ((m1 & 1) ? TM_G1 : TM_G), kq1, KQ_ATOM, kq1, KQ_ATOM,
-                                      ID_G, 8, 0);
-                        tc::mma_commit(&bars[B_GRAM]);
-                        gram_issued = true;
-                    }
                 } else {
                     fail(gabort);
                 }
             }
-            COMBA_PHASE(20);
-            la_c = la_n;
-            bt_c = bt_n;
             COMBA_PHASE(21);
             COMBA_ITER_NEXT();
         }
@@ -897,6 +896,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     tc::tc_fence_before();
     __syncthreads();
+    COMBA_CTA_MARK(1);
     if (warp == 0) tc::tmem_dealloc(tmem, TM_COLS);
 }
 

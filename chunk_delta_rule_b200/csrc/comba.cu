@@ -212,6 +212,18 @@ extern "C" int comba_trace_read_phases(unsigned long long* host_slots) {
     return cudaMemcpyToSymbol(comba::g_phase_cycles, zeros, sizeof(zeros)) == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
 }
 
+// Tracing builds only: per-CTA start / end global-timer stamps (2 per CTA, 1024 CTAs).
+extern "C" int comba_trace_read_cta(unsigned long long* host_2048) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;
+    return cudaMemcpyFromSymbol(host_2048, comba::g_cta_ns, 2048 * sizeof(unsigned long long)) ==
+                   cudaSuccess ? COMBA_OK : COMBA_ECUDA;
+}
+extern "C" int comba_trace_read_cta_clk(long long* host_3072) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;
+    return cudaMemcpyFromSymbol(host_3072, comba::g_cta_clk, 3072 * sizeof(long long)) ==
+                   cudaSuccess ? COMBA_OK : COMBA_ECUDA;
+}
+
 // Tracing builds only: absolute mark timestamps of one loop iteration, two threads.
 extern "C" int comba_trace_read_ts(long long* host_2slots) {
     if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;

@@ -26,6 +26,9 @@ __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0,
 #ifndef COMBA_TRACE_ITER
 #define COMBA_TRACE_ITER 10
 #endif
+#ifndef COMBA_TRACE_CTA
+#define COMBA_TRACE_CTA 0
+#endif
 __device__ unsigned long long g_phase_cycles[COMBA_TRACE_SLOTS];
 // absolute clock64() of each mark: thread 0 in loop iteration COMBA_TRACE_ITER,
 // thread TID2 in the next one (the prep group runs one chunk ahead): [thread 0 | TID2]
@@ -43,15 +46,32 @@ __device__ long long g_phase_ts[2 * COMBA_TRACE_SLOTS];
         const long long comba_phase_now = clock64();                          \
         comba_phase_acc[(i)] += (unsigned long long)(comba_phase_now - comba_phase_t); \
         comba_phase_t = comba_phase_now;                                      \
-        if (comba_iter == COMBA_TRACE_ITER + (threadIdx.x == 0 ? 0 : 1) && blockIdx.x == 0 && \
+        if (comba_iter == COMBA_TRACE_ITER + (threadIdx.x == 0 ? 0 : 1) && blockIdx.x == COMBA_TRACE_CTA && \
             (threadIdx.x == 0 || threadIdx.x == COMBA_TRACE_TID2))            \
             g_phase_ts[(threadIdx.x == 0 ? 0 : COMBA_TRACE_SLOTS) + (i)] = comba_phase_now; \
     } while (0)
 #define COMBA_ITER_NEXT() (++comba_iter)
+// per-CTA start / end (global timer, ns) of up to 1024 CTAs, and SM clock cycles
+__device__ unsigned long long g_cta_ns[2 * 1024];
+__device__ long long g_cta_clk[3 * 1024];
+#define COMBA_CTA_MARK(k)                                                          \
+    do {                                                                           \
+        if (threadIdx.x == 0 && blockIdx.x < 1024) {                               \
+            unsigned long long comba_t;                                            \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(comba_t));            \
+            g_cta_ns[2 * blockIdx.x + (k)] = comba_t;                              \
+            g_cta_clk[2 * blockIdx.x + (k)] = clock64();                           \
+            if ((k) == 0) {                                                        \
+                unsigned comba_sm;                                                 \
+                asm volatile("mov.u32 %0, %%smid;" : "=r"(comba_sm));              \
+                g_cta_clk[2048 + blockIdx.x] = comba_sm;                           \
+            }                                                                      \
+        }                                                                          \
+    } while (0)
 #define COMBA_COUNT(i) (++comba_phase_acc[(i)])
 #define COMBA_PHASE_END()                                                     \
     do {                                                                      \
-        if (blockIdx.x == 0 && (threadIdx.x == 0 || threadIdx.x == COMBA_TRACE_TID2)) \
+        if (blockIdx.x == COMBA_TRACE_CTA && (threadIdx.x == 0 || threadIdx.x == COMBA_TRACE_TID2)) \
             for (int comba_i = 0; comba_i < COMBA_TRACE_SLOTS; ++comba_i)     \
                 g_phase_cycles[comba_i] += comba_phase_acc[comba_i];          \
     } while (0)
@@ -59,6 +79,7 @@ __device__ long long g_phase_ts[2 * COMBA_TRACE_SLOTS];
 #define COMBA_PHASE_BEGIN() do {} while (0)
 #define COMBA_PHASE(i) do {} while (0)
 #define COMBA_ITER_NEXT() do {} while (0)
+#define COMBA_CTA_MARK(k) do {} while (0)
 #define COMBA_COUNT(i) do {} while (0)
 #define COMBA_PHASE_END() do {} while (0)
 #endif

@@ -401,6 +401,11 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Producer side of a named barrier: counts this warp's threads without waiting.
+__device__ __forceinline__ void named_barrier_arrive(int id, int nthreads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Named barrier that also ORs a per-thread failure flag across the
 // participating threads: returns true only if no thread reported failure, so
 // every thread of the group takes the same decision.
@@ -425,6 +430,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 // Explicit shared-space accesses by 32-bit shared address.  Loads are issued
 // unconditionally (callers select the value), which keeps element loops free
 // of divergent branches.
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ float lds_f32(uint32_t a) {
     float v;
     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
