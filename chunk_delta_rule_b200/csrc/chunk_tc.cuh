@@ -43,9 +43,11 @@ namespace tck {
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr int kThreads = 384;        // warps 0-3: state group; warps 4-11: prep group
+constexpr int kThreads = 384;        // warps 0-3: state group; warp 4: MMA issue; warps 5-11: prep
 constexpr int kStateThreads = 128;
-constexpr int kPrepThreads = 256;
+constexpr int kCtlWarp = 4;
+constexpr int kPrepThreads = 224;
+constexpr int kPrepBase = 160;       // first thread of the prep group
 constexpr int BAR_PREP = 1;          // named barrier ids: the prep group
 constexpr int BAR_STATE = 2;         // the state group
 constexpr int BAR_KK = 3;            // K K^T staged (3 warps arrive) -> P warps (3 warps wait)
@@ -238,9 +240,9 @@ __device__ __forceinline__ void tceb_diag_and_upper(uint32_t F1, uint32_t F2, in
 //   M_20 = -N_20 + N_21 N_10,   M_31 = -N_31 + N_32 N_21
 //   M_30 = -N_30 + N_31 N_10 - N_32 M_20
 //   T_ij = M_ij T_jj
-// Four levels of single 16 x 16 products, one warp per block.  N_ij is kept in
-// the unused upper block (j, i) of F2, M_20, M_31, M_30 in the lower blocks.
-// A (in F1) is dead after level 1, so from level 2 on the idle warps turn the
+// Four levels of single 16 x 16 products, one warp per block (seven warps).  N_ij
+// is kept in the unused upper block (j, i) of F2, M_20, M_31, M_30 in the lower
+// blocks.  A (in F1) is dead after level 1, so at level 2 warps 3-6 turn the
 // diagonal blocks into Tc / Eb (and zero the upper blocks) in F1, and level 4
 // writes the lower blocks there.
 __device__ __forceinline__ void offdiag_inverse(uint32_t F1, uint32_t F2, int pt, uint32_t CS,
@@ -255,7 +257,7 @@ __device__ __forceinline__ void offdiag_inverse(uint32_t F1, uint32_t F2, int pt
         blk16_store(F2, 16 * j, 16 * i, c, 1.f, lane);
     }
     tc::named_barrier(BAR_PREP, kPrepThreads);
-    // level 2: M_20, M_31 and Q_30 = -N_30 + N_31 N_10; warps 4..7: Tc/Eb of diagonal blocks
+    // level 2: M_20, M_31 and Q_30 = -N_30 + N_31 N_10; warps 3..6: Tc/Eb of diagonal blocks
     if (warp < 3) {
         const int xa = warp == 1 ? 2 : 1, xb = warp == 1 ? 3 : (warp == 0 ? 2 : 3);   // N_{xb, xa}
         const int ya = warp == 1 ? 1 : 0, yb = warp == 1 ? 2 : 1;                     // N_{yb, ya}
@@ -268,8 +270,8 @@ __device__ __forceinline__ void offdiag_inverse(uint32_t F1, uint32_t F2, int pt
 #pragma unroll
             for (int e = 0; e < 4; ++e) c[nt][e] -= ns[nt][e];
         blk16_store(F2, 16 * si, 16 * sj, c, 1.f, lane);
-    } else if (warp >= 4) {
-        tceb_diag_and_upper(F1, F2, warp - 4, lane, CS, BT);
+    } else if (warp >= 3) {
+        tceb_diag_and_upper(F1, F2, warp - 3, lane, CS, BT);
     }
     tc::named_barrier(BAR_PREP, kPrepThreads);
     // level 3: M_30 = Q_30 - N_32 M_20
@@ -332,12 +334,15 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     auto sed = [&](int c) -> uint32_t { return sb + SM_MISC + 4352u + 512u * (uint32_t)(c & 1); };
     auto seg = [&](int c) -> uint32_t { return sed(c) + 256u; };
     // barriers: q/k stages, v, gram per TMEM buffer, wn (W^T, U~^T in TMEM), mma1 (X),
-    // mma2, the P buffers (MMA2 and the out store have read them) and the Gram/W^T
-    // TMEM buffers (the state group has read W^T).  Each is arrived on once per
+    // mma2, the P buffers (MMA2 has read them), mma1 (O).  Each is arrived on once per
     // phase (by a commit, a TMA transaction count or one thread after its group's
     // named barrier): many arrivals on one barrier serialise in the shared-memory pipe.
+    // The MMA-issue warp waits on three hand-overs: the prep group's Tc / Eb / diag(lo)
+    // of a chunk (WNREADY), the state group's -W operand and S copies (WREADY) and its
+    // bf16 X' (SPLIT).
     enum { B_KQ0 = 0, B_V = 3, B_GRAM0 = 4, B_GRAM1 = 5, B_WN = 6, B_MMA1 = 7, B_MMA2 = 8,
-           B_PBUF0 = 9, B_PBUF1 = 10, B_GFREE = 11, B_MMA1B = 12, NBARS = 13 };
+           B_PBUF0 = 9, B_PBUF1 = 10, B_MMA1B = 11, B_WNREADY = 12, B_WREADY = 13, B_SPLIT = 14,
+           NBARS = 15 };
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 6144);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
     volatile int* gabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -496,8 +501,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const int t0 = n * kC;
             const int stg = n & 1;
             const uint32_t tgn = stg ? TM_G1 : TM_G;
-            const uint32_t kqn = sb + kq_stage(n);
-            const uint32_t pbuf = stg ? SM_P1 : SM_P0;
             const bool last = (n + 1 == nchunks);
             // ---- -W operand from W^T (lane = j, column = token) once the prep's MMAs are
             // done and the previous chunk's out store has read its staging (same buffer)
@@ -524,19 +527,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!ok) fail(gabort);
             if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
             if (issuer) {
-                tc::mbar_arrive(&bars[B_GFREE]);   // W^T read: the prep may reuse this TMEM buffer
+                tc::mbar_arrive(&bars[B_WREADY]);  // -W and the S copies are in: MMA1
                 tc::fence_proxy_async_smem();      // V has been read by the W/X MMAs
                 if (n + 1 < nchunks) load_v(n + 1);
             }
+            __syncwarp();
             COMBA_PHASE(1);
-            if (warp == 0) {   // MMA issue: the whole warp, one elected lane
-                __syncwarp();   // reconverge after the single-thread block above
-                tc::tc_fence_after();
-                tc::mma_bf16_ta_bmn(tmem + TM_X, tmem + TM_SB, sb + SM_W, 8192, ID_SW, 8, 1);
-                tc::mma_commit(&bars[B_MMA1]);
-                tc::mma_bf16_ta_bk(tmem + TM_O, tmem + TM_SB, sb + SM_QH, QH_ATOM, ID_SQ, 8, 0);
-                tc::mma_commit(&bars[B_MMA1B]);
-            }
             // ---- while MMA1 runs: the next chunk's decays
             const float eLn = last ? 1.f : state_gates(la_n, n + 1);
             if (tid < 64 && n + 2 < nchunks) la_n = gate(log_alpha, t0 + 2 * kC + tid);
@@ -570,14 +566,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::tc_fence_before();
             if (!ok) fail(gabort);
             if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
-            if (warp == 0) {
-                __syncwarp();
-                tc::tc_fence_after();
-                tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH, kqn, KQ_ATOM, ID_SK, 4, 1);
-                tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH + 32, kqn, KQ_ATOM, ID_SK, 4, 1);
-                tc::mma_tf32_ta_bk(tmem + TM_O, tmem + TM_X, sb + pbuf, F32_ATOM, ID_XP, 8, 1);
-                tc::mma_commit(&bars[B_MMA2]);
-            }
+            if (issuer) tc::mbar_arrive(&bars[B_SPLIT]);   // X' is in: MMA2
+            __syncwarp();
             COMBA_PHASE(2);
             // ---- while MMA2 runs: Qh of the next chunk (MMA1 has read this chunk's)
             if (!last) {
@@ -589,12 +579,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!ok) fail(gabort);
             if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
             tc::tc_fence_after();
-            if (issuer) {   // P of this chunk and its q/k stage are read
-                tc::mbar_arrive(&bars[stg ? B_PBUF1 : B_PBUF0]);
-                if (n + kKQStages < nchunks) {
-                    tc::fence_proxy_async_smem();
-                    load_kq(n + kKQStages);
-                }
+            if (issuer && n + kKQStages < nchunks) {   // this chunk's q/k stage is read
+                tc::fence_proxy_async_smem();
+                load_kq(n + kKQStages);
             }
             __syncwarp();
             COMBA_PHASE(4);
@@ -665,52 +652,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             COMBA_ITER_NEXT();
         }
         if (issuer) tc::bulk_wait0();
-    } else {
-        // =============================== prep group ================================
-        // Chunk m's operands for the state group: the inverse's blocks, Tc / Eb, P,
-        // then the MMAs W^T = K^T Tc^T and U~^T (= X^T before MMA1).  Warp pw reads
-        // TMEM lanes 32 (pw & 3) .. + 31 of the Gram, columns 32 (pw >> 2) .. + 31:
-        //   pw 0, 1, 5: K K^T rows (0-31, 32-63, 32-63) x columns (0-31, 0-31, 32-63):
-        //               A in registers, K K^T staged for P; pw 0 and 5 then invert the
-        //               diagonal blocks (0, 1) and (2, 3) from their registers
-        //   pw 2, 3, 7: Q K^T of the same row/column blocks: P, once K K^T is staged
-        //   pw 6:       P rows 0-31 x columns 32-63 are zero (s > r); issues the next
-        //               chunk's Gram
-        //   pw 1, 4:    the next chunk's gate tables;  pw 4 issues this chunk's W/X MMAs
-        // then all eight warps: the off-diagonal blocks, Tc / Eb, diag(lo(beta)).
-        const int pt = tid - kStateThreads;
-        const int pw = pt >> 5, q = pw & 3, ch = pw >> 2;
-        const bool issuer = (pt == 0);
-        const int gtok = (pw == 1) ? lane : 32 + lane;   // gate warps: token of this thread
-        float la_x = 0.f, bt_x = 0.f;                     // gate warps: next chunk's values
-        // gate tables of chunk c into tset(c) from this thread's token values (gate warps)
-        auto make_tables = [&](int c, float la, float bt) {
-            float x = la;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, off);
-                if (lane >= off) x += y;
-            }
-            if (lane == 31) tc::sts_f32(RED + (pw == 1 ? 0u : 4u), x);
-            tc::named_barrier(BAR_GATES, 64);
-            const float c0 = tc::lds_f32(RED), gL = c0 + tc::lds_f32(RED + 4u);
-            const bool fst = gL > -80.f;
-            const float g = x + (pw == 4 ? c0 : 0.f), gp = g - la;
-            const uint32_t ts = tset(c);
-            tc::sts_f32(ts + 4u * gtok, g * kLog2e);
-            tc::sts_f32(ts + 256 + 4u * gtok, gp * kLog2e);
-            tc::sts_f32(ts + 512 + 4u * gtok, bt);
-            tc::sts_f32(ts + 768 + 4u * gtok, bt * __expf(gp));
-            tc::sts_f32(ts + 1024 + 4u * gtok, __expf(g));
-            tc::sts_f32(ts + 1280 + 4u * gtok, fst ? __expf(-g) : 0.f);
-            if (gtok == 0) asm volatile("st.shared.u32 [%0], %1;" ::"r"(ts + 1536), "r"(fst ? 1u : 0u) : "memory");
-            tc::named_barrier(BAR_GATES, 64);   // RED is reused by the next call
-        };
-        // Gram ([K;Q] K^T) of chunk c into its TMEM buffer (warp pw 6, one elected lane)
+    } else if (warp == kCtlWarp) {
+        // ============================ MMA-issue warp ===============================
+        // All tensor-core MMAs, in one order per chunk n: W^T / U~^T of chunk n (once
+        // the prep group hands over its Tc / Eb), MMA1(n) (once the state group hands
+        // over -W and the S copies), MMA2(n) (once it hands over X'), then the Gram of
+        // chunk n+2 into the TMEM buffer whose W^T the state group has just read.  Each
+        // wait depends only on MMAs issued before it, so the order cannot deadlock.
+        bool ok = true;
         auto issue_gram = [&](int c) -> bool {
+            const bool okg = tc::mbar_wait(kq_bar(c), kq_par(c), timeout_ns);
             __syncwarp();
-            bool okg = tc::mbar_wait(kq_bar(c), kq_par(c), timeout_ns) &&
-                       (c < 2 || tc::mbar_wait(&bars[B_GFREE], (c - 2) & 1, timeout_ns));
             if (okg) {
                 const uint32_t kq = sb + kq_stage(c);
                 tc::tc_fence_after();
@@ -719,20 +671,105 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             return okg;
         };
+        ok = issue_gram(0) && (nchunks < 2 || issue_gram(1));
+        for (int n = 0; n < nchunks && ok; ++n) {
+            const int stg = n & 1;
+            const uint32_t kqn = sb + kq_stage(n);
+            const uint32_t tgn = stg ? TM_G1 : TM_G;
+            // ---- W^T = K^T Tc^T;  X^T = U~^T = V^T Eb^T + V^T diag(lo)^T  (X^T of chunk n-1
+            // read by its MMA2)
+            ok = tc::mbar_wait(&bars[B_WNREADY], n & 1, timeout_ns) &&
+                 tc::mbar_wait(&bars[B_V], n & 1, timeout_ns) &&
+                 (n == 0 || tc::mbar_wait(&bars[B_MMA2], (n - 1) & 1, timeout_ns));
+            __syncwarp();
+            if (!ok) break;
+            tc::tc_fence_after();
+            tc::mma_amn_bk(tmem + tgn, kqn, KQ_ATOM, F1, ID_WN, 4, 0);
+            tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, F1 + 8192, ID_WN, 4, 0);
+            tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
+            tc::mma_commit(&bars[B_WN]);
+            // ---- MMA1(n): X^T += S (-W)^T;  O^T = S Qh^T
+            ok = tc::mbar_wait(&bars[B_WREADY], n & 1, timeout_ns);
+            __syncwarp();
+            if (!ok) break;
+            tc::tc_fence_after();
+            tc::mma_bf16_ta_bmn(tmem + TM_X, tmem + TM_SB, sb + SM_W, 8192, ID_SW, 8, 1);
+            tc::mma_commit(&bars[B_MMA1]);
+            tc::mma_bf16_ta_bk(tmem + TM_O, tmem + TM_SB, sb + SM_QH, QH_ATOM, ID_SQ, 8, 0);
+            tc::mma_commit(&bars[B_MMA1B]);
+            // ---- MMA2(n): S += X'^T K (bf16 hi + lo);  O^T += X^T P^T
+            ok = tc::mbar_wait(&bars[B_SPLIT], n & 1, timeout_ns);
+            __syncwarp();
+            if (!ok) break;
+            tc::tc_fence_after();
+            tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH, kqn, KQ_ATOM, ID_SK, 4, 1);
+            tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH + 32, kqn, KQ_ATOM, ID_SK, 4, 1);
+            tc::mma_tf32_ta_bk(tmem + TM_O, tmem + TM_X, sb + (stg ? SM_P1 : SM_P0), F32_ATOM, ID_XP, 8, 1);
+            tc::mma_commit(&bars[B_MMA2]);
+            tc::mma_commit(&bars[stg ? B_PBUF1 : B_PBUF0]);
+            // ---- Gram of chunk n+2 (its TMEM buffer held W^T of chunk n, read above)
+            if (n + 2 < nchunks) ok = issue_gram(n + 2);
+        }
+        if (!ok) fail(gabort);
+    } else {
+        // =============================== prep group ================================
+        // Chunk m's operands for the MMA warp: the inverse's blocks, Tc / Eb, P and
+        // diag(lo(beta)).  Seven warps; warp pw reads TMEM lanes 32 (warp & 3) .. + 31 of
+        // the Gram (K K^T in lanes 0-63, Q K^T in lanes 64-127):
+        //   pw 3, 0, 4: K K^T rows 0-31 x cols 0-31, rows 32-63 x cols 0-31, rows 32-63 x
+        //               cols 32-63: A in registers, K K^T staged for P; pw 3 and 4 then
+        //               invert the diagonal blocks (0, 1) and (2, 3) from their registers
+        //   pw 1, 2, 6: Q K^T of the same row/column blocks: P, once K K^T is staged
+        //   pw 5:       P rows 0-31 x cols 32-63 are zero (s > r)
+        //   pw 5, 0:    the next chunk's gate tables (tokens 0-31, 32-63)
+        // then all seven warps: the off-diagonal blocks, Tc / Eb, diag(lo(beta)).
+        const int pt = tid - kPrepBase;
+        const int pw = pt >> 5, q = warp & 3;
+        const bool kk_warp = (pw == 0 || pw == 3 || pw == 4);
+        const bool p_warp = (pw == 1 || pw == 2 || pw == 6);
+        const int ch = (pw == 4 || pw == 6) ? 1 : 0;        // Gram column half
+        const bool gate_warp = (pw == 5 || pw == 0);
+        const bool issuer = (pt == 0);
+        const int gtok = (pw == 5) ? lane : 32 + lane;     // gate warps: token of this thread
+        float la_x = 0.f, bt_x = 0.f;                       // gate warps: next chunk's values
+        // gate tables of chunk c into tset(c) from this thread's token values (gate warps)
+        auto make_tables = [&](int c, float la, float bt) {
+            float x = la;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, off);
+                if (lane >= off) x += y;
+            }
+            if (lane == 31) tc::sts_f32(RED + (pw == 5 ? 0u : 4u), x);
+            __syncwarp();
+            tc::named_barrier(BAR_GATES, 64);
+            const float c0 = tc::lds_f32(RED), gL = c0 + tc::lds_f32(RED + 4u);
+            const bool fst = gL > -80.f;
+            const float g = x + (pw == 0 ? c0 : 0.f), gp = g - la;
+            const uint32_t ts = tset(c);
+            tc::sts_f32(ts + 4u * gtok, g * kLog2e);
+            tc::sts_f32(ts + 256 + 4u * gtok, gp * kLog2e);
+            tc::sts_f32(ts + 512 + 4u * gtok, bt);
+            tc::sts_f32(ts + 768 + 4u * gtok, bt * __expf(gp));
+            tc::sts_f32(ts + 1024 + 4u * gtok, __expf(g));
+            tc::sts_f32(ts + 1280 + 4u * gtok, fst ? __expf(-g) : 0.f);
+            if (gtok == 0) asm volatile("st.shared.u32 [%0], %1;" ::"r"(ts + 1536), "r"(fst ? 1u : 0u) : "memory");
+            __syncwarp();
+            tc::named_barrier(BAR_GATES, 64);   // RED is reused by the next call
+        };
         bool ok = true;
         if (issuer) {
             for (int c = 0; c < kKQStages && c < nchunks; ++c) load_kq(c);
             load_v(0);
         }
-        if (pw == 1 || pw == 4) {
+        __syncwarp();
+        if (gate_warp) {
             make_tables(0, gate(log_alpha, gtok), gate(beta, gtok));
             if (nchunks > 1) {
                 la_x = gate(log_alpha, kC + gtok);
                 bt_x = gate(beta, kC + gtok);
             }
         }
-        if (pw == 6) ok = issue_gram(0);
-        if (!ok) fail(gabort);
         ok = tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok);
         for (int m = 0; m < nchunks && ok; ++m) {
             const bool last = (m + 1 == nchunks);
@@ -742,10 +779,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const bool fast = tc::lds_u32(ts + 1536) != 0u;
             ok = (*gabort == 0);
             // ================= phase 1: A, K K^T, P, diagonal inverse blocks =================
-            if (pw == 0 || pw == 1 || pw == 5) {
+            if (kk_warp) {
                 const int r = 32 * q + lane;          // row (token) of this thread
                 ok = ok && tc::mbar_wait(&bars[(m & 1) ? B_GRAM1 : B_GRAM0], (m >> 1) & 1, timeout_ns) &&
                      (m < 2 || tc::mbar_wait(&bars[(m & 1) ? B_PBUF1 : B_PBUF0], ((m - 2) >> 1) & 1, timeout_ns));
+                __syncwarp();
                 tc::tc_fence_after();
                 COMBA_PHASE(7);
                 float a[32];
@@ -756,7 +794,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int c = 0; c < 8; ++c)
                     tc::sts_f32x4(pbm + ch * F32_ATOM + tc::sw128(r, c),
                                   make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]));
-                tc::fence_proxy_async_smem();
                 tc::tc_fence_before();
                 tc::named_barrier_arrive(BAR_KK, kKKThreads);
                 // A_rs = beta_r e^{g_{r-1} - g_s} (K K^T)_rs for s < r, in registers
@@ -779,22 +816,24 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 }
                 COMBA_PHASE(9);
-                if (pw != 1) diag_pair_inverse(a, F2, pw == 5 ? 1 : 0, lane);
+                if (pw != 0) diag_pair_inverse(a, F2, pw == 4 ? 1 : 0, lane);
                 COMBA_PHASE(10);
                 // A into F1 for the off-diagonal blocks (its lower blocks A_10, A_2x,
                 // A_3x only), once the previous chunk's W/X MMAs have read F1
                 ok = ok && (m == 0 || tc::mbar_wait(&bars[B_WN], (m - 1) & 1, timeout_ns));
+                __syncwarp();
                 COMBA_PHASE(11);
-                if (pw == 1) {
+                if (pw == 0) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) tc::sts_f32(faddr(F1, r, e), a[e]);
-                } else if (lane >= 16) {   // rows 16-31 x cols 0-15 (pw 0), 48-63 x 32-47 (pw 5)
+                } else if (lane >= 16) {   // rows 16-31 x cols 0-15 (pw 3), 48-63 x 32-47 (pw 4)
 #pragma unroll
                     for (int e = 0; e < 16; ++e) tc::sts_f32(faddr(F1, r, 32 * ch + e), a[e]);
                 }
-            } else if (pw == 2 || pw == 3 || pw == 7) {
+            } else if (p_warp) {
                 const int r = 32 * (q - 2) + lane;    // row (token) of this thread
                 ok = ok && tc::mbar_wait(&bars[(m & 1) ? B_GRAM1 : B_GRAM0], (m >> 1) & 1, timeout_ns);
+                __syncwarp();
                 tc::tc_fence_after();
                 float gv[32];
                 tc::tmem_ld32(tl + tgm + 32 * ch, gv);
@@ -836,18 +875,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 }
                 tc::fence_proxy_async_smem();
-            } else if (pw == 6) {
+            } else {   // pw 5
                 ok = ok && (m < 2 || tc::mbar_wait(&bars[(m & 1) ? B_PBUF1 : B_PBUF0], ((m - 2) >> 1) & 1, timeout_ns));
+                __syncwarp();
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
                     tc::sts_u32x4(pbm + F32_ATOM + tc::sw128(lane, c), make_uint4(0u, 0u, 0u, 0u));
                 tc::fence_proxy_async_smem();
-                // next chunk's Gram, into the TMEM buffer whose W^T (chunk m - 1) the state read
-                if (!last) ok = issue_gram(m + 1) && ok;
             }
             COMBA_PHASE(16);
             // ================= phase 2: next chunk's gate tables (gate warps) =================
-            if ((pw == 1 || pw == 4) && !last) {
+            if (gate_warp && !last) {
                 make_tables(m + 1, la_x, bt_x);
                 if (m + 2 < nchunks) {
                     la_x = gate(log_alpha, (m + 2) * kC + gtok);
@@ -870,25 +908,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             tc::fence_proxy_async_smem();
             if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
+            if (issuer) tc::mbar_arrive(&bars[B_WNREADY]);   // Tc, Eb, diag(lo) of chunk m are in
+            __syncwarp();
             COMBA_PHASE(20);
-            // ================= phase 4: W^T = K^T Tc^T; X^T = U~^T = V^T Eb^T + V^T diag(lo)^T =====
-            // (warp pw 4; X^T of chunk m - 1 must have been read by its MMA2)
-            if (pw == 4) {
-                __syncwarp();
-                bool okw = tc::mbar_wait(&bars[B_V], m & 1, timeout_ns) &&
-                           (m == 0 || tc::mbar_wait(&bars[B_MMA2], (m - 1) & 1, timeout_ns));
-                if (okw) {
-                    const uint32_t kq = sb + kq_stage(m);
-                    tc::tc_fence_after();
-                    tc::mma_amn_bk(tmem + tgm, kq, KQ_ATOM, F1, ID_WN, 4, 0);
-                    tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, F1 + 8192, ID_WN, 4, 0);
-                    tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
-                    tc::mma_commit(&bars[B_WN]);
-                } else {
-                    fail(gabort);
-                }
-            }
-            COMBA_PHASE(21);
             COMBA_ITER_NEXT();
         }
     }

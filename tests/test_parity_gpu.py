@@ -52,6 +52,25 @@ def test_small_shapes_against_oracle(B, H, T, dk, dv, chunk, dt):
     assert_close("S_final", S, rS, tol)
 
 
+@pytest.mark.parametrize("dt", ["bf16", "fp32"])
+def test_strong_decay_mixes_exact_and_factored_chunks(dt):
+    # log a ~ U(-2, -0.5): a chunk's total log-decay spreads around -80 (about -89 to
+    # -75 for this seed, half of the chunks on either side), so chunks take both the
+    # factored e^{g_r} e^{-g_s} form and the exact per-entry exponent, and in-chunk
+    # decays reach the limits of fp32.
+    base = CONFIGS["layer340m_bf16"] if dt == "bf16" else CONFIGS["tiny_fp32"]
+    cfg = base.replace(B=2, H=2, T=320, dk=128, dv=128, chunk=64, decay="uniform",
+                       decay_lo=-2.0, decay_hi=-0.5, s0_std=0.5)
+    x = make_chunk_inputs(cfg, seed=4242)
+    g = x["log_alpha"].double().reshape(2, 5, 64, 2).sum(2)
+    assert bool((g > -80).any()) and bool((g <= -80).any())
+    o, S = gpu_chunk(x, 64)
+    ro, rS = oracle.recurrence(**x)
+    tol = TOL_BF16 if dt == "bf16" else TOL_F32
+    assert_close("out", o, ro, tol)
+    assert_close("S_final", S, rS, tol)
+
+
 @pytest.mark.parametrize("name,chains", [
     ("layer340m_bf16", [(0, 0), (3, 5), (7, 7)]),
     ("layer1p3b_bf16", [(0, 0), (4, 9), (7, 15)]),
