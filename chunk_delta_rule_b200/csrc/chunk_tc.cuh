@@ -305,6 +305,48 @@ __device__ __forceinline__ void offdiag_inverse(uint32_t F1, uint32_t F2, int pt
     }
 }
 
+// Gram [K;Q] K^T of one chunk's q/k stage into a TMEM buffer, committed to `bar`
+// (the MMA-issue warp; one out-of-line copy for its three call sites).
+__device__ __noinline__ void gram_mma(uint32_t d, uint32_t kq, uint64_t* bar) {
+    tc::tc_fence_after();
+    tc::mma_ak_bk(d, kq, KQ_ATOM, kq, KQ_ATOM, ID_G, 8, 0);
+    tc::mma_commit(bar);
+}
+
+// Exact-exponential forms for a chunk whose total log-decay is at or below -80
+// (e^{-g} would leave the normal fp32 range): each entry takes exp2 of its own
+// exponent difference.  Out of line, they are never on the common path.
+//   a_rows_exact: A_rs = beta_r 2^{g'_{r-1} - g'_s} (K K^T)_rs (s < r) for row r over
+//   columns 32 ch .. + 31, from the Gram in TMEM, into F1 (g' = g log2 e)
+__device__ __noinline__ void a_rows_exact(uint32_t F1, uint32_t gram_taddr, int r, int ch, uint32_t ts) {
+    float gv[32];
+    tc::tmem_ld32(gram_taddr, gv);
+    tc::tmem_ld_wait();
+    const float br = tc::lds_f32(ts + 512 + 4u * r), gpr = tc::lds_f32(ts + 256 + 4u * r);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const int s = 32 * ch + e;
+        const float v = br * exp2f(gpr - tc::lds_f32(ts + 4u * s)) * gv[e];
+        tc::sts_f32(faddr(F1, r, s), (s < r) ? v : 0.f);
+    }
+}
+//   p_row_exact: P_rs = 2^{g'_r - g'_s} (Q K^T - d K K^T)_rs (s <= r) for row r over
+//   columns 32 ch .. + 31, in place over the staged K K^T row
+__device__ __noinline__ void p_row_exact(uint32_t prow, uint32_t gram_taddr, int r, int ch, float dh,
+                                         uint32_t ts) {
+    float gv[32];
+    tc::tmem_ld32(gram_taddr, gv);
+    tc::tmem_ld_wait();
+    const float gr = tc::lds_f32(ts + 4u * r);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const int s = 32 * ch + e;
+        const uint32_t pa = prow + tc::sw128(r, e >> 2) + 4u * (e & 3);
+        const float v = exp2f(gr - tc::lds_f32(ts + 4u * s)) * fmaf(-dh, tc::lds_f32(pa), gv[e]);
+        tc::sts_f32(pa, (s <= r) ? v : 0.f);
+    }
+}
+
 __device__ __forceinline__ void fail(volatile int* gabort) {
     *gabort = 1;
     latch_status(-4 /* COMBA_ETIMEOUT */);
@@ -663,12 +705,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         auto issue_gram = [&](int c) -> bool {
             const bool okg = tc::mbar_wait(kq_bar(c), kq_par(c), timeout_ns);
             __syncwarp();
-            if (okg) {
-                const uint32_t kq = sb + kq_stage(c);
-                tc::tc_fence_after();
-                tc::mma_ak_bk(tmem + ((c & 1) ? TM_G1 : TM_G), kq, KQ_ATOM, kq, KQ_ATOM, ID_G, 8, 0);
-                tc::mma_commit(&bars[(c & 1) ? B_GRAM1 : B_GRAM0]);
-            }
+            if (okg)
+                gram_mma(tmem + ((c & 1) ? TM_G1 : TM_G), sb + kq_stage(c), &bars[(c & 1) ? B_GRAM1 : B_GRAM0]);
             return okg;
         };
         ok = issue_gram(0) && (nchunks < 2 || issue_gram(1));
@@ -807,13 +845,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         for (int e = 0; e < 4; ++e)
                             a[4 * c + e] = (32 * ch + 4 * c + e < r) ? cr * iv[e] * a[4 * c + e] : 0.f;
                     }
-                } else {
-                    const float br = tc::lds_f32(ts + 512 + 4u * r), gpr = tc::lds_f32(ts + 256 + 4u * r);
+                } else {   // rows straight into F1 (once free), then back into registers
+                    ok = ok && (m == 0 || tc::mbar_wait(&bars[B_WN], (m - 1) & 1, timeout_ns));
+                    __syncwarp();
+                    a_rows_exact(F1, tl + tgm + 32 * ch, r, ch, ts);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int s = 32 * ch + e;
-                        a[e] = (s < r) ? br * exp2f(gpr - tc::lds_f32(ts + 4u * s)) * a[e] : 0.f;
-                    }
+                    for (int e = 0; e < 32; ++e) a[e] = tc::lds_f32(faddr(F1, r, 32 * ch + e));
                 }
                 COMBA_PHASE(9);
                 if (pw != 0) diag_pair_inverse(a, F2, pw == 4 ? 1 : 0, lane);
@@ -858,21 +895,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         tc::sts_f32x4(pa, pv);
                     }
                 } else {
-                    const float gr = tc::lds_f32(ts + 4u * r);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint32_t pa = prow + tc::sw128(r, c);
-                        const float4 kk = tc::lds_f32x4(pa);
-                        const float kv[4] = {kk.x, kk.y, kk.z, kk.w};
-                        float pv[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int s = 32 * ch + 4 * c + e;
-                            pv[e] = (s <= r) ? exp2f(gr - tc::lds_f32(ts + 4u * s)) * fmaf(-dh, kv[e], gv[4 * c + e])
-                                             : 0.f;
-                        }
-                        tc::sts_f32x4(pa, make_float4(pv[0], pv[1], pv[2], pv[3]));
-                    }
+                    p_row_exact(prow, tl + tgm + 32 * ch, r, ch, dh, ts);
                 }
                 tc::fence_proxy_async_smem();
             } else {   // pw 5

@@ -301,10 +301,12 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 // addresses.  Each descriptor is built once: the start address sits in its low
 // 14 bits (address / 16, below 2^14 for any shared-memory address), so a
 // k-step's operand offset is added to the descriptor directly.  The loops are
-// unrolled by COMBA_MMA_UNROLL (default: fully); rolled loops issue measurably
-// slower.
+// unrolled by COMBA_MMA_UNROLL (default: rolled).  Issue runs at the tensor pipe's
+// pace either way once a warp is dedicated to it, and the rolled loops keep that
+// warp's code small (instruction fetch stalls were the largest stall reason with
+// every loop unrolled).
 #ifndef COMBA_MMA_UNROLL
-#define COMBA_MMA_UNROLL 8
+#define COMBA_MMA_UNROLL 1
 #endif
 constexpr int kMmaUnroll = COMBA_MMA_UNROLL;
 
