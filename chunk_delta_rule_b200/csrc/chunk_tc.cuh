@@ -1,38 +1,31 @@
 // Tensor-core chunk-wise Comba forward for bf16 inputs, dk = dv = 128, chunk 64.
 //
-// One CTA owns one (b, h) chain and walks its chunks in order, split into two
-// warp groups that run one chunk apart: a prep group (8 warps) builds chunk
-// n+1's operands while a state group (4 warps) runs chunk n's state-dependent
-// MMAs and epilogue; they hand buffers over through mbarriers.  Per chunk
-// (chunk-start state S, local tokens r, s, g_r = sum_{i<=r} log_alpha_i, g_0 = 0;
-// the write-up's "block-recurrent, intra-block parallel" form with a single
-// inverse for the intermediates W and U, section "硬件高效的分块并行计算"):
+// One CTA owns one (b, h) chain and walks its chunks in order, in the write-up's
+// "block-recurrent, intra-block parallel" form with a single inverse for the
+// intermediates W and U (section "硬件高效的分块并行计算").  Per chunk (chunk-start
+// state S, local tokens r, s, g_r = sum_{i<=r} log_alpha_i):
 //
-//   1. gates (prefetched one chunk ahead): g by warp-shuffle scan, e^{g_r},
-//      e^{-g_r}, e^{g_L - g_r}, c_r = beta_r e^{g_{r-1}}
-//   2. Gram MMA G = [K; Q] K^T (bf16 -> TMEM), issued during the previous chunk
-//   3. K K^T staged in the P operand; A_rs = beta_r e^{g_{r-1}-g_s}(K K^T)_rs (s < r);
-//      then, concurrently: P_rs = e^{g_r-g_s}(Q K^T - d K K^T)_rs (s <= r) in
-//      place (fp32 operand), Qh = diag(e^g)(Q - d K) over Q and (D K)^T with
-//      D = diag(e^{g_L - g}) (fp32, K-major) on half the warps; the 16 x 16
-//      diagonal blocks of Tinv = (I + A)^{-1} by substitution on the others
-//   4. off-diagonal blocks of Tinv by distance, warp-level tf32 MMAs per 8-column slab
-//   5. Tc = Tinv diag(c); Eb = (Tinv - I) diag(beta) + diag(hi(beta)) (bf16),
-//      diag(lo(beta)) (bf16), so that beta = hi + lo to 16 bits
-//   6. MMAs W^T = K^T Tc^T,  X^T = V^T Eb^T + V^T diag(lo)^T  (= U~^T)
-//   7. -W^T -> bf16 operand
-//   8. MMAs X^T += S (-W)^T, O^T = S Qh^T (bf16, S from its bf16 copy);
-//      then, reading X^T straight from TMEM as a tf32 operand,
-//      S += X^T (D K) and O^T += X^T P^T; then the next chunk's Gram MMA
-//   9. S -> bf16 operand, S master *= e^{g_L} of the next chunk; O^T -> TMA store
+//   A_rs = beta_r e^{g_{r-1} - g_s} (k_r . k_s)  (s < r),   Tinv = (I + A)^{-1}
+//   W = Tinv diag(beta e^{g_{r-1}}) K,   U~ = Tinv diag(beta) V,   X = U~ - W S^T
+//   P_rs = e^{g_r - g_s} (q_r - d k_r) . k_s  (s <= r)
+//   O = diag(e^g)(Q - d K) S^T + P X,    S <- e^{g_L} S + (X diag(e^{g_L - g}))^T K
 //
-// The leading beta V term of U~ = beta V + (Tinv - I) beta V is carried to
-// 16 bits (hi + lo bf16 diagonals against the exact bf16 V), and the state
-// master stays fp32 throughout.  Within a chunk e^{g_r - g_s} is formed as
-// e^{g_r} e^{-g_s} when the chunk's total log-decay is above -80 (both factors
-// stay normal fp32 numbers); otherwise each entry takes exp2 of the difference.  A ragged last chunk is zero-filled by TMA and
-// its gates padded with log_alpha = 0, beta = 0, which leaves the state and
-// the valid outputs exact.
+// Three warp-specialised roles run different chunks at once and hand buffers
+// over through mbarriers:
+//   prep group (7 warps): gate tables (one chunk ahead), A and P from the Gram
+//     products, the 16 x 16 diagonal inverse blocks from registers, the
+//     off-diagonal blocks with warp MMAs, Tc = Tinv diag(c) and Eb (bf16);
+//   MMA-issue warp: every tcgen05 MMA (Gram, W^T / U~^T, X and O against the state,
+//     the state update and the intra-chunk output), in a fixed order per chunk;
+//   state group (4 warps, TMEM lane = value index): -W and Qh operands, X' = X
+//     diag(e^{g_L - g}) as bf16 hi + lo, the O readout, the bf16 copy and decay of
+//     the fp32 state master in TMEM, and the out tile's TMA store.
+// The leading beta V term of U~ is carried to 16 bits (hi + lo bf16 diagonals
+// against the exact bf16 V).  Within a chunk e^{g_r - g_s} is formed as
+// e^{g_r} e^{-g_s} when the chunk's total log-decay is above -80 (both factors stay
+// normal fp32 numbers); otherwise each entry takes exp2 of the difference.  A ragged
+// last chunk is zero-filled by TMA and its gates padded with log_alpha = 0,
+// beta = 0, which leaves the state and the valid outputs exact.
 #pragma once
 
 #include "common.cuh"
