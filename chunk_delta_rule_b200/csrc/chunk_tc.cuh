@@ -103,9 +103,9 @@ __device__ __forceinline__ uint32_t faddr(uint32_t base, int r, int s) {
 // one warp, lane l holds row 32p + l of A over columns 32p .. 32p + 31 in a[].
 // Lanes 0-15 invert block 2p, lanes 16-31 block 2p + 1; lane l owns column l & 15
 // of its block (right-looking substitution, the A entries taken from the lane that
-// holds the row by shuffle), and writes it to F2.
+// holds the row by a shuffle within each 16-lane half), and writes it to F2.
 __device__ __forceinline__ void diag_pair_inverse(const float (&a)[32], uint32_t F2, int p, int lane) {
-    const int hb = lane >> 4, j = lane & 15, src = lane & 16;
+    const int hb = lane >> 4, j = lane & 15;
     float al[16];
 #pragma unroll
     for (int s = 0; s < 16; ++s) al[s] = hb ? a[16 + s] : a[s];
@@ -117,7 +117,7 @@ __device__ __forceinline__ void diag_pair_inverse(const float (&a)[32], uint32_t
         const float xs = x[s];
 #pragma unroll
         for (int r = s + 1; r < 16; ++r)
-            x[r] = fmaf(-__shfl_sync(0xffffffffu, al[s], src | r), xs, x[r]);
+            x[r] = fmaf(-__shfl_sync(0xffffffffu, al[s], r, 16), xs, x[r]);
     }
     const int blk = 2 * p + hb;
 #pragma unroll
@@ -233,68 +233,89 @@ __device__ __forceinline__ void tceb_diag_and_upper(uint32_t F1, uint32_t F2, in
 //   M_20 = -N_20 + N_21 N_10,   M_31 = -N_31 + N_32 N_21
 //   M_30 = -N_30 + N_31 N_10 - N_32 M_20
 //   T_ij = M_ij T_jj
-// Four levels of single 16 x 16 products, one warp per block (seven warps).  N_ij
-// is kept in the unused upper block (j, i) of F2, M_20, M_31, M_30 in the lower
-// blocks.  A (in F1) is dead after level 1, so at level 2 warps 3-6 turn the
-// diagonal blocks into Tc / Eb (and zero the upper blocks) in F1, and level 4
-// writes the lower blocks there.
+// Four levels of single 16 x 16 products, one warp per block.  N_ij is kept in
+// the unused upper block (j, i) of F2, M_20, M_31, M_30 in the lower blocks.
+// A (in F1) is dead after level 1, so at level 2 warps 3-6 turn the diagonal
+// blocks into Tc / Eb (and zero the upper blocks) in F1, and level 4 writes the
+// lower blocks there.
+//
+// Every product step has the form  c = s_i B_init + s_p X Y,  stored to a block of
+// F2 or written out as Tc / Eb, so the levels run as one loop over a per-(level,
+// warp) task table: one copy of the product code instead of one per step (the
+// kernel is sensitive to its instruction footprint).  Table fields, in 16-row
+// block units: kind (0 idle, 1 product, 2 Tc/Eb of diagonal block xr), X (xr, xc)
+// in F2, Y in F1 if yf else F2 at (yr, yc), init (0 none, 1 subtract, 2 add) from
+// F2 (ir, ic), product sign (+1 / -1), output (0: F2 block (or, oc); 1: Tc / Eb
+// block (or, oc)).
+__constant__ signed char kOffTask[4][7][16] = {
+    {   // level 1: N_ij = T_ii A_ij -> F2 (j, i)
+        {1, 1, 1, 1, 1, 0, 0, 0, 0, 1, 0, 0, 1},
+        {1, 2, 2, 1, 2, 1, 0, 0, 0, 1, 0, 1, 2},
+        {1, 3, 3, 1, 3, 2, 0, 0, 0, 1, 0, 2, 3},
+        {1, 2, 2, 1, 2, 0, 0, 0, 0, 1, 0, 0, 2},
+        {1, 3, 3, 1, 3, 1, 0, 0, 0, 1, 0, 1, 3},
+        {1, 3, 3, 1, 3, 0, 0, 0, 0, 1, 0, 0, 3},
+        {0},
+    },
+    {   // level 2: M_20 = N_21 N_10 - N_20, M_31 = N_32 N_21 - N_31, Q_30 = N_31 N_10 - N_30;
+        //          Tc / Eb of the diagonal blocks
+        {1, 1, 2, 0, 0, 1, 1, 0, 2, 1, 0, 2, 0},
+        {1, 2, 3, 0, 1, 2, 1, 1, 3, 1, 0, 3, 1},
+        {1, 1, 3, 0, 0, 1, 1, 0, 3, 1, 0, 3, 0},
+        {2, 0},
+        {2, 1},
+        {2, 2},
+        {2, 3},
+    },
+    {   // level 3: M_30 = Q_30 - N_32 M_20
+        {1, 2, 3, 0, 2, 0, 2, 3, 0, -1, 0, 3, 0},
+        {0}, {0}, {0}, {0}, {0}, {0},
+    },
+    {   // level 4: T_{j+1,j} = -N_{j+1,j} T_jj, T_20 = M_20 T_00, T_31 = M_31 T_11, T_30 = M_30 T_00
+        {1, 0, 1, 0, 0, 0, 0, 0, 0, -1, 1, 1, 0},
+        {1, 1, 2, 0, 1, 1, 0, 0, 0, -1, 1, 2, 1},
+        {1, 2, 3, 0, 2, 2, 0, 0, 0, -1, 1, 3, 2},
+        {1, 2, 0, 0, 0, 0, 0, 0, 0, 1, 1, 2, 0},
+        {1, 3, 1, 0, 1, 1, 0, 0, 0, 1, 1, 3, 1},
+        {1, 3, 0, 0, 0, 0, 0, 0, 0, 1, 1, 3, 0},
+        {0},
+    },
+};
+
 __device__ __forceinline__ void offdiag_inverse(uint32_t F1, uint32_t F2, int pt, uint32_t CS,
                                                 uint32_t BT) {
     const int warp = pt >> 5, lane = pt & 31;
-    // level 1: N_ij = T_ii A_ij for the six lower blocks
-    if (warp < 6) {
-        const int i = (warp < 3) ? warp + 1 : ((warp == 5) ? 3 : warp - 1);
-        const int j = (warp < 3) ? warp : ((warp == 5) ? 0 : warp - 3);
-        float c[2][4] = {};
-        blk16_mma(c, F2, 16 * i, 16 * i, F1, 16 * i, 16 * j, lane);
-        blk16_store(F2, 16 * j, 16 * i, c, 1.f, lane);
-    }
-    tc::named_barrier(BAR_PREP, kPrepThreads);
-    // level 2: M_20, M_31 and Q_30 = -N_30 + N_31 N_10; warps 3..6: Tc/Eb of diagonal blocks
-    if (warp < 3) {
-        const int xa = warp == 1 ? 2 : 1, xb = warp == 1 ? 3 : (warp == 0 ? 2 : 3);   // N_{xb, xa}
-        const int ya = warp == 1 ? 1 : 0, yb = warp == 1 ? 2 : 1;                     // N_{yb, ya}
-        const int si = warp == 0 ? 2 : 3, sj = warp == 1 ? 1 : 0;                      // N_{si, sj}
-        float c[2][4] = {}, ns[2][4];
-        blk16_mma(c, F2, 16 * xa, 16 * xb, F2, 16 * ya, 16 * yb, lane);
-        blk16_load(ns, F2, 16 * sj, 16 * si, lane);
+#pragma unroll 1
+    for (int lv = 0; lv < 4; ++lv) {
+        const signed char* t = kOffTask[lv][warp];
+        const int kind = t[0];
+        if (kind == 1) {
+            float c[2][4], pr[2][4] = {};
+            if (t[6] != 0) {
+                blk16_load(c, F2, 16 * t[7], 16 * t[8], lane);
+                const float si = (t[6] == 1) ? -1.f : 1.f;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+                for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) c[nt][e] -= ns[nt][e];
-        blk16_store(F2, 16 * si, 16 * sj, c, 1.f, lane);
-    } else if (warp >= 3) {
-        tceb_diag_and_upper(F1, F2, warp - 3, lane, CS, BT);
-    }
-    tc::named_barrier(BAR_PREP, kPrepThreads);
-    // level 3: M_30 = Q_30 - N_32 M_20
-    if (warp == 0) {
-        float c[2][4] = {}, q[2][4];
-        blk16_mma(c, F2, 32, 48, F2, 32, 0, lane);
-        blk16_load(q, F2, 48, 0, lane);
+                    for (int e = 0; e < 4; ++e) c[nt][e] *= si;
+            } else {
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+                for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) c[nt][e] = q[nt][e] - c[nt][e];
-        blk16_store(F2, 48, 0, c, 1.f, lane);
-    }
-    tc::named_barrier(BAR_PREP, kPrepThreads);
-    // level 4: T_ij = M_ij T_jj -> Tc / Eb
-    if (warp < 6) {
-        float c[2][4] = {};
-        if (warp < 3) {          // T_{j+1,j} = -N_{j+1,j} T_jj
-            const int j = warp, i = warp + 1;
-            blk16_mma(c, F2, 16 * j, 16 * i, F2, 16 * j, 16 * j, lane);
+                    for (int e = 0; e < 4; ++e) c[nt][e] = 0.f;
+            }
+            blk16_mma(pr, F2, 16 * t[1], 16 * t[2], t[3] ? F1 : F2, 16 * t[4], 16 * t[5], lane);
+            const float sp = (float)t[9];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) c[nt][e] = -c[nt][e];
-            tceb_store_frag(F1, i, j, c, CS, BT, lane);
-        } else {                 // T_20, T_31, T_30
-            const int i = warp == 3 ? 2 : 3, j = warp == 4 ? 1 : 0;
-            blk16_mma(c, F2, 16 * i, 16 * j, F2, 16 * j, 16 * j, lane);
-            tceb_store_frag(F1, i, j, c, CS, BT, lane);
+                for (int e = 0; e < 4; ++e) c[nt][e] = fmaf(sp, pr[nt][e], c[nt][e]);
+            if (t[10] == 0) blk16_store(F2, 16 * t[11], 16 * t[12], c, 1.f, lane);
+            else tceb_store_frag(F1, t[11], t[12], c, CS, BT, lane);
+        } else if (kind == 2) {
+            tceb_diag_and_upper(F1, F2, t[1], lane, CS, BT);
         }
+        if (lv < 3) tc::named_barrier(BAR_PREP, kPrepThreads);
     }
 }
 
