@@ -55,9 +55,12 @@ def library():
             chunk_sig = [vp] * 9 + [i] * 6 + [vp]
             lib.comba_chunk_fwd.argtypes = chunk_sig
             lib.comba_chunk_fwd_f32.argtypes = chunk_sig
+            lib.comba_chunk_fwd_ws.argtypes = [vp] * 9 + [i] * 6 + [vp, ctypes.c_size_t, vp]
+            lib.comba_chunk_fwd_workspace_size.argtypes = [i] * 6
+            lib.comba_chunk_fwd_workspace_size.restype = ctypes.c_size_t
             lib.comba_recurrent_step.argtypes = [vp] * 8 + [i] * 4 + [vp]
-            for fn in (lib.comba_chunk_fwd, lib.comba_chunk_fwd_f32, lib.comba_recurrent_step,
-                       lib.comba_get_last_error, lib.comba_version):
+            for fn in (lib.comba_chunk_fwd, lib.comba_chunk_fwd_f32, lib.comba_chunk_fwd_ws,
+                       lib.comba_recurrent_step, lib.comba_get_last_error, lib.comba_version):
                 fn.restype = ctypes.c_int
             lib.comba_get_last_error.argtypes = []
             lib.comba_version.argtypes = []
@@ -100,11 +103,13 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
               beta: torch.Tensor, d: torch.Tensor, S0: Optional[torch.Tensor] = None,
               chunk: int = 64, out: Optional[torch.Tensor] = None,
               S_final: Optional[torch.Tensor] = None, return_state: bool = True,
-              stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+              stream=None, segment: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunk-wise forward.  q, k [B,T,H,dk], v [B,T,H,dv] (bf16 or fp32, same
     dtype); log_alpha, beta [B,T,H] fp32; d [H] fp32; S0 [B,H,dv,dk] fp32 or None.
     Returns (out [B,T,H,dv] in q's dtype, S_final [B,H,dv,dk] fp32 or None).
-    ``S_final`` may be passed as ``S0`` itself for an in-place state carry."""
+    ``S_final`` may be passed as ``S0`` itself for an in-place state carry.
+    ``segment=False`` keeps every chain in one CTA even when the library would cut
+    long sequences of few chains into segments (comba_chunk_fwd_ws)."""
     if q.dim() != 4:
         raise ValueError("q must be [B, T, H, dk]")
     B, T, H, dk = q.shape
@@ -129,12 +134,21 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
     if S_final is not None:
         _check(S_final, "S_final", torch.float32, (B, H, dv, dk))
     lib = library()
-    fn = lib.comba_chunk_fwd if dt == torch.bfloat16 else lib.comba_chunk_fwd_f32
     with torch.cuda.device(dev):
-        st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(d), _ptr(S0),
-                _ptr(out), _ptr(S_final), B, T, H, dk, dv, int(chunk), _stream_handle(dev, stream))
+        args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(d), _ptr(S0),
+                _ptr(out), _ptr(S_final), B, T, H, dk, dv, int(chunk))
+        if dt == torch.bfloat16:
+            # too few (b, h) chains for the GPU: the library runs them segmented in a
+            # workspace from PyTorch's allocator (empty otherwise)
+            nbytes = lib.comba_chunk_fwd_workspace_size(B, T, H, dk, dv, int(chunk)) if segment else 0
+            ws = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
+            st = lib.comba_chunk_fwd_ws(*args, _ptr(ws), nbytes, _stream_handle(dev, stream))
+            name = "comba_chunk_fwd_ws"
+        else:
+            st = lib.comba_chunk_fwd_f32(*args, _stream_handle(dev, stream))
+            name = "comba_chunk_fwd_f32"
     if st != 0:
-        raise CombaError(st, "comba_chunk_fwd" + ("" if dt == torch.bfloat16 else "_f32"))
+        raise CombaError(st, name)
     return out, S_final
 
 

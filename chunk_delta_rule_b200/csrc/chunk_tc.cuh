@@ -371,7 +371,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     const float* __restrict__ log_alpha, const float* __restrict__ beta,
                     const float* __restrict__ dvec, const float* S0, float* S_final, int T, int H,
-                    unsigned long long timeout_ns) {
+                    int b_split, int no_out, unsigned long long timeout_ns) {
     COMBA_CTA_MARK(0);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
@@ -405,7 +405,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t F1 = sb + SM_F1, F2 = sb + SM_F2;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int b = blockIdx.x / H, h = blockIdx.x % H;
+    // CTAs of batch index >= b_split solve the same chain of batch (index - b_split)
+    // with V = 0 (a stacked launch that also yields each chain's state transition);
+    // S0 and S_final are indexed by the CTA.  no_out: the outputs are not written.
+    const int bcta = blockIdx.x / H, h = blockIdx.x % H;
+    const bool vzero = bcta >= b_split;
+    const int b = vzero ? bcta - b_split : bcta;
+    const bool want_out = (no_out == 0);
     const float dh = dvec[h];
     const int nchunks = (T + kC - 1) / kC;
     const uint32_t trow = (uint32_t)((warp & 3) * 32) << 16;
@@ -585,7 +591,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (issuer) {
                 tc::mbar_arrive(&bars[B_WREADY]);  // -W and the S copies are in: MMA1
                 tc::fence_proxy_async_smem();      // V has been read by the W/X MMAs
-                if (n + 1 < nchunks) load_v(n + 1);
+                if (n + 1 < nchunks && !vzero) load_v(n + 1);
             }
             __syncwarp();
             COMBA_PHASE(1);
@@ -626,7 +632,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             __syncwarp();
             COMBA_PHASE(2);
             // ---- while MMA2 runs: Qh of the next chunk (MMA1 has read this chunk's)
-            if (!last) {
+            if (!last && want_out) {
                 ok = ok && tc::mbar_wait(&bars[B_MMA1B], n & 1, timeout_ns);
                 ok = state_qh(n + 1) && ok;
             }
@@ -643,7 +649,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             COMBA_PHASE(4);
             // O^T row (value index) -> bf16 pairs of tokens
             uint32_t ob[32];
-            {
+            if (want_out) {
                 float o0[32], o1[32];
                 tc::tmem_ld32(tl + TM_O, o0);
                 tc::tmem_ld32(tl + TM_O + 32, o1);
@@ -686,6 +692,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::tmem_st_wait();
             tc::tc_fence_before();
             COMBA_PHASE(5);
+            if (want_out) {
             // out tile [token][value index] in two 64-wide 128B-swizzled boxes, staged in
             // the -W buffer (MMA1 has read it), TMA store.  The barrier below also hands
             // the new S copies to the next MMA1.
@@ -704,6 +711,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::tma_store_4d(&tm_o, sm + SM_W, 0, h, t0, b);
                 tc::tma_store_4d(&tm_o, sm + SM_W + 8192, 64, h, t0, b);
                 tc::bulk_commit();
+            }
             }
             COMBA_ITER_NEXT();
         }
@@ -731,23 +739,25 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // ---- W^T = K^T Tc^T;  X^T = U~^T = V^T Eb^T + V^T diag(lo)^T  (X^T of chunk n-1
             // read by its MMA2)
             ok = tc::mbar_wait(&bars[B_WNREADY], n & 1, timeout_ns) &&
-                 tc::mbar_wait(&bars[B_V], n & 1, timeout_ns) &&
+                 (vzero || tc::mbar_wait(&bars[B_V], n & 1, timeout_ns)) &&
                  (n == 0 || tc::mbar_wait(&bars[B_MMA2], (n - 1) & 1, timeout_ns));
             __syncwarp();
             if (!ok) break;
             tc::tc_fence_after();
             tc::mma_amn_bk(tmem + tgn, kqn, KQ_ATOM, F1, ID_WN, 4, 0);
-            tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, F1 + 8192, ID_WN, 4, 0);
-            tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
+            if (!vzero) {
+                tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, F1 + 8192, ID_WN, 4, 0);
+                tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
+            }
             tc::mma_commit(&bars[B_WN]);
             // ---- MMA1(n): X^T += S (-W)^T;  O^T = S Qh^T
             ok = tc::mbar_wait(&bars[B_WREADY], n & 1, timeout_ns);
             __syncwarp();
             if (!ok) break;
             tc::tc_fence_after();
-            tc::mma_bf16_ta_bmn(tmem + TM_X, tmem + TM_SB, sb + SM_W, 8192, ID_SW, 8, 1);
+            tc::mma_bf16_ta_bmn(tmem + TM_X, tmem + TM_SB, sb + SM_W, 8192, ID_SW, 8, vzero ? 0u : 1u);
             tc::mma_commit(&bars[B_MMA1]);
-            tc::mma_bf16_ta_bk(tmem + TM_O, tmem + TM_SB, sb + SM_QH, QH_ATOM, ID_SQ, 8, 0);
+            if (want_out) tc::mma_bf16_ta_bk(tmem + TM_O, tmem + TM_SB, sb + SM_QH, QH_ATOM, ID_SQ, 8, 0);
             tc::mma_commit(&bars[B_MMA1B]);
             // ---- MMA2(n): S += X'^T K (bf16 hi + lo);  O^T += X^T P^T
             ok = tc::mbar_wait(&bars[B_SPLIT], n & 1, timeout_ns);
@@ -756,7 +766,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::tc_fence_after();
             tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH, kqn, KQ_ATOM, ID_SK, 4, 1);
             tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH + 32, kqn, KQ_ATOM, ID_SK, 4, 1);
-            tc::mma_tf32_ta_bk(tmem + TM_O, tmem + TM_X, sb + (stg ? SM_P1 : SM_P0), F32_ATOM, ID_XP, 8, 1);
+            if (want_out) tc::mma_tf32_ta_bk(tmem + TM_O, tmem + TM_X, sb + (stg ? SM_P1 : SM_P0), F32_ATOM, ID_XP, 8, 1);
             tc::mma_commit(&bars[B_MMA2]);
             tc::mma_commit(&bars[stg ? B_PBUF1 : B_PBUF0]);
             // ---- Gram of chunk n+2 (its TMEM buffer held W^T of chunk n, read above)
@@ -812,7 +822,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         bool ok = true;
         if (issuer) {
             for (int c = 0; c < kKQStages && c < nchunks; ++c) load_kq(c);
-            load_v(0);
+            if (!vzero) load_v(0);
         }
         __syncwarp();
         if (gate_warp) {
@@ -999,10 +1009,14 @@ inline bool make_tmap_bthd(CUtensorMap* map, const void* ptr, int B, int T, int 
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
 
+// One CTA per (b, h) of Bc stacked batches over data with B batches (Bc defaults to B):
+// stacked batches b >= B repeat data batch b - B with V = 0.  out == nullptr: no
+// outputs are written.
 inline int launch_chunk_tc(const void* q, const void* k, const void* v, const float* log_alpha,
                            const float* beta, const float* d, const float* S0, void* out,
                            float* S_final, int B, int T, int H, cudaStream_t stream,
-                           unsigned long long timeout_ns = kWaitTimeoutNs) {
+                           int Bc = -1, unsigned long long timeout_ns = kWaitTimeoutNs) {
+    if (Bc < 0) Bc = B;
     static bool attr_set[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -3;
@@ -1014,10 +1028,10 @@ inline int launch_chunk_tc(const void* q, const void* k, const void* v, const fl
     }
     CUtensorMap tq, tk, tv, to;
     if (!make_tmap_bthd(&tq, q, B, T, H) || !make_tmap_bthd(&tk, k, B, T, H) ||
-        !make_tmap_bthd(&tv, v, B, T, H) || !make_tmap_bthd(&to, out, B, T, H))
+        !make_tmap_bthd(&tv, v, B, T, H) || !make_tmap_bthd(&to, out ? out : q, B, T, H))
         return -3;
-    tck::chunk_fwd_tc_kernel<<<(unsigned)(B * H), tck::kThreads, tck::kSmemBytes, stream>>>(
-        tq, tk, tv, to, log_alpha, beta, d, S0, S_final, T, H, timeout_ns);
+    tck::chunk_fwd_tc_kernel<<<(unsigned)(Bc * H), tck::kThreads, tck::kSmemBytes, stream>>>(
+        tq, tk, tv, to, log_alpha, beta, d, S0, S_final, T, H, B, out ? 0 : 1, timeout_ns);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 

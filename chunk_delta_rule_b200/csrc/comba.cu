@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "chunk_simt.cuh"
 #include "chunk_tc.cuh"
+#include "chunk_segments.cuh"
 #include "recurrent_step.cuh"
 
 namespace {
@@ -124,6 +125,40 @@ extern "C" int comba_chunk_fwd(const void* q, const void* k, const void* v,
     if (T == 0) return empty_sequence(a, s);
     if (comba::tc_supported(dk, dv, chunk)) return comba::launch_chunk_tc(a.q, a.k, a.v, a.log_alpha, a.beta, a.d, a.S0, a.out, a.S_final, B, T, H, s);
     return launch_simt<__nv_bfloat16>(a, s);
+}
+
+extern "C" size_t comba_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk) {
+    if (B <= 0 || H <= 0 || T <= 0 || !comba::tc_supported(dk, dv, chunk)) return 0;
+    const int P = comba::seg::segment_count(B, T, H, comba::seg::sm_count());
+    return comba::seg::workspace_floats(B, H, P) * sizeof(float);
+}
+
+extern "C" int comba_chunk_fwd_ws(const void* q, const void* k, const void* v,
+                                  const float* log_alpha, const float* beta, const float* d,
+                                  const float* S0, void* out, float* S_final, int B, int T, int H,
+                                  int dk, int dv, int chunk, void* workspace, size_t workspace_bytes,
+                                  comba_stream_t stream) {
+    const ChunkArgs a{q, k, v, log_alpha, beta, d, S0, out, S_final, B, T, H, dk, dv, chunk, 2};
+    if (int st = validate_chunk(a)) return st;
+    if (B == 0 || H == 0) return COMBA_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) return empty_sequence(a, s);
+    if (!comba::tc_supported(dk, dv, chunk)) return launch_simt<__nv_bfloat16>(a, s);
+    const int P = comba::seg::segment_count(B, T, H, comba::seg::sm_count());
+    const size_t need = comba::seg::workspace_floats(B, H, P) * sizeof(float);
+    if (P > 1 && workspace && workspace_bytes >= need) {
+        if (!aligned(workspace, 16)) return COMBA_EINVAL;
+        const size_t bth = (size_t)B * T * H;
+        const void* bufs[] = {q, k, v, log_alpha, beta, d, S0, out, S_final};
+        const size_t nb[] = {bth * dk * 2, bth * dk * 2, bth * dv * 2, bth * 4, bth * 4, (size_t)H * 4,
+                             (size_t)B * H * dv * dk * 4, bth * dv * 2, (size_t)B * H * dv * dk * 4};
+        for (int i = 0; i < 9; ++i)
+            if (overlap(workspace, need, bufs[i], nb[i])) return COMBA_EINVAL;
+        return comba::seg::launch_segmented(q, k, v, log_alpha, beta, d, S0, out, S_final, B, T, H, P,
+                                            static_cast<float*>(workspace), s) == 0 ? COMBA_OK : COMBA_ECUDA;
+    }
+    return comba::launch_chunk_tc(a.q, a.k, a.v, a.log_alpha, a.beta, a.d, a.S0, a.out, a.S_final, B, T, H, s) == 0
+               ? COMBA_OK : COMBA_ECUDA;
 }
 
 extern "C" int comba_chunk_fwd_f32(const float* q, const float* k, const float* v,

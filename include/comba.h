@@ -40,6 +40,8 @@
 #ifndef COMBA_H_
 #define COMBA_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -74,6 +76,33 @@ int comba_chunk_fwd(const void* q, const void* k, const void* v,
                     const float* S0, void* out, float* S_final,
                     int B, int T, int H, int dk, int dv, int chunk,
                     comba_stream_t stream);
+
+/*
+ * Workspace the segmented form of comba_chunk_fwd_ws needs for this shape on the
+ * current device, in bytes; 0 when the shape runs unsegmented (enough (b, h)
+ * chains to fill the GPU, a T that is not a multiple of 64, or a shape outside the
+ * tensor-core kernel).  The answer depends on the device's SM count.
+ */
+size_t comba_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk);
+
+/*
+ * comba_chunk_fwd with a caller-owned device workspace (16-byte aligned, not
+ * overlapping any argument).  With at least comba_chunk_fwd_workspace_size()
+ * bytes, a shape with too few (b, h) chains for the GPU is run segmented: each
+ * chain's sequence is cut into P pieces that run as independent chains, joined by
+ * their affine state transitions (the end state from S is S M + R, with R the
+ * piece's end state from S = 0 and M its end state from S = I with V = 0), then
+ * rerun from the composed start states for the outputs.  The result is the same
+ * computation regrouped (write-up, section "硬件高效的分块并行计算": recurrent across
+ * blocks, parallel inside), equal up to rounding.  With less workspace (or NULL)
+ * it behaves exactly as comba_chunk_fwd.  The workspace is in use until the work
+ * enqueued on `stream` completes.
+ */
+int comba_chunk_fwd_ws(const void* q, const void* k, const void* v,
+                       const float* log_alpha, const float* beta, const float* d,
+                       const float* S0, void* out, float* S_final,
+                       int B, int T, int H, int dk, int dv, int chunk,
+                       void* workspace, size_t workspace_bytes, comba_stream_t stream);
 
 /*
  * Chunk-wise forward with fp32 q, k, v and out (same math, same layouts, same

@@ -71,6 +71,38 @@ def test_strong_decay_mixes_exact_and_factored_chunks(dt):
     assert_close("S_final", S, rS, tol)
 
 
+@pytest.mark.parametrize("with_s0,in_place", [(False, False), (True, False), (True, True)])
+def test_segmented_long_sequence_matches_oracle_and_unsegmented(with_s0, in_place):
+    # Two chains of 4096 tokens leave most of the GPU idle, so the library cuts each
+    # chain into segments joined by their state transitions (comba_chunk_fwd_ws).
+    cfg = CONFIGS["layer340m_bf16"].replace(B=1, H=2, T=4096, s0_std=0.05 if with_s0 else 0.0)
+    x = make_chunk_inputs(cfg, seed=777)
+    if not with_s0:
+        x["S0"] = None
+    lib = cdr.library()
+    assert lib.comba_chunk_fwd_workspace_size(1, 4096, 2, 128, 128, 64) > 0
+    xd = to_dev(x)
+    args = {k: xd[k] for k in ("q", "k", "v", "log_alpha", "beta", "d")}
+    S0 = xd["S0"]
+    o_plain, S_plain = cdr.chunk_fwd(**args, S0=S0, chunk=64, segment=False)
+    if in_place:
+        Sc = S0.clone()
+        o_seg, S_seg = cdr.chunk_fwd(**args, S0=Sc, S_final=Sc, chunk=64)
+    else:
+        o_seg, S_seg = cdr.chunk_fwd(**args, S0=S0, chunk=64)
+    torch.cuda.synchronize()
+    assert cdr.library().comba_get_last_error() == 0
+    ro, rS = oracle.recurrence(**x)
+    np64 = lambda t: t.double().cpu().numpy()
+    assert_close("out (segmented)", np64(o_seg), ro, TOL_BF16)
+    assert_close("S_final (segmented)", np64(S_seg), rS, TOL_BF16)
+    assert_close("out (unsegmented)", np64(o_plain), ro, TOL_BF16)
+    # the two groupings of the same computation agree to well inside the bf16 bound
+    d_o = (o_seg.float() - o_plain.float()).norm() / o_plain.float().norm()
+    d_S = (S_seg - S_plain).norm() / S_plain.norm()
+    assert float(d_o) < 2e-3 and float(d_S) < 2e-3
+
+
 @pytest.mark.parametrize("name,chains", [
     ("layer340m_bf16", [(0, 0), (3, 5), (7, 7)]),
     ("layer1p3b_bf16", [(0, 0), (4, 9), (7, 15)]),
