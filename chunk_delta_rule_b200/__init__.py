@@ -56,10 +56,12 @@ def library():
             lib.comba_chunk_fwd.argtypes = chunk_sig
             lib.comba_chunk_fwd_f32.argtypes = chunk_sig
             lib.comba_chunk_fwd_ws.argtypes = [vp] * 9 + [i] * 6 + [vp, ctypes.c_size_t, vp]
+            lib.comba_chunk_fwd_noalloc.argtypes = chunk_sig
             lib.comba_chunk_fwd_workspace_size.argtypes = [i] * 6
             lib.comba_chunk_fwd_workspace_size.restype = ctypes.c_size_t
             lib.comba_recurrent_step.argtypes = [vp] * 8 + [i] * 4 + [vp]
             for fn in (lib.comba_chunk_fwd, lib.comba_chunk_fwd_f32, lib.comba_chunk_fwd_ws,
+                       lib.comba_chunk_fwd_noalloc,
                        lib.comba_recurrent_step, lib.comba_get_last_error, lib.comba_version):
                 fn.restype = ctypes.c_int
             lib.comba_get_last_error.argtypes = []
@@ -150,6 +152,31 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
     if st != 0:
         raise CombaError(st, name)
     return out, S_final
+
+
+def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                      beta: torch.Tensor, d: torch.Tensor, S0: Optional[torch.Tensor],
+                      out: torch.Tensor, S_final: Optional[torch.Tensor], chunk: int = 64,
+                      stream=None) -> None:
+    """comba_chunk_fwd_noalloc on caller-allocated bf16 tensors (same layouts as
+    chunk_fwd): the segmented form's scratch is the library's static device array."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _check(t, name, torch.bfloat16, (B, T, H, dk if name in ("q", "k") else dv))
+    _check(log_alpha, "log_alpha", torch.float32, (B, T, H))
+    _check(beta, "beta", torch.float32, (B, T, H))
+    _check(d, "d", torch.float32, (H,))
+    for t, name in ((S0, "S0"), (S_final, "S_final")):
+        if t is not None:
+            _check(t, name, torch.float32, (B, H, dv, dk))
+    dev = q.device
+    with torch.cuda.device(dev):
+        st = library().comba_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                               _ptr(d), _ptr(S0), _ptr(out), _ptr(S_final), B, T, H, dk,
+                                               dv, int(chunk), _stream_handle(dev, stream))
+    if st != 0:
+        raise CombaError(st, "comba_chunk_fwd_noalloc")
 
 
 def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,

@@ -161,6 +161,22 @@ extern "C" int comba_chunk_fwd_ws(const void* q, const void* k, const void* v,
                ? COMBA_OK : COMBA_ECUDA;
 }
 
+// Scratch of comba_chunk_fwd_noalloc: the segmented form's workspace for up to
+// kNoallocChains segment-chains (B * P * H), in the module's static device memory.
+constexpr size_t kNoallocChains = 128;
+constexpr size_t kNoallocFloats = 6 * kNoallocChains * comba::seg::kStateFloats;
+static __device__ __align__(256) float g_noalloc_ws[kNoallocFloats];
+
+extern "C" int comba_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                       const float* log_alpha, const float* beta, const float* d,
+                                       const float* S0, void* out, float* S_final, int B, int T,
+                                       int H, int dk, int dv, int chunk, comba_stream_t stream) {
+    void* ws = nullptr;
+    if (cudaGetSymbolAddress(&ws, g_noalloc_ws) != cudaSuccess) return COMBA_ECUDA;
+    return comba_chunk_fwd_ws(q, k, v, log_alpha, beta, d, S0, out, S_final, B, T, H, dk, dv, chunk, ws,
+                              sizeof(g_noalloc_ws), stream);
+}
+
 extern "C" int comba_chunk_fwd_f32(const float* q, const float* k, const float* v,
                                    const float* log_alpha, const float* beta, const float* d,
                                    const float* S0, float* out, float* S_final, int B, int T,

@@ -105,6 +105,20 @@ int comba_chunk_fwd_ws(const void* q, const void* k, const void* v,
                        void* workspace, size_t workspace_bytes, comba_stream_t stream);
 
 /*
+ * comba_chunk_fwd_ws with the workspace taken from a scratch array in the
+ * library's static device memory (48 MiB, room for B * P * H <= 128 segment-chains;
+ * larger shapes run unsegmented): neither the library nor the caller allocates
+ * anything for the call.  No counterpart in the write-up; an entry point for
+ * callers that cannot provide device memory.  The scratch is one per device for the
+ * whole process, so calls must not run concurrently (use one stream, or order them).
+ */
+int comba_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                            const float* log_alpha, const float* beta, const float* d,
+                            const float* S0, void* out, float* S_final,
+                            int B, int T, int H, int dk, int dv, int chunk,
+                            comba_stream_t stream);
+
+/*
  * Chunk-wise forward with fp32 q, k, v and out (same math, same layouts, same
  * size rules as comba_chunk_fwd); every product is an fp32 FMA, no reduced-
  * precision tensor-core arithmetic.
