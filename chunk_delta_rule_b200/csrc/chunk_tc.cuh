@@ -13,8 +13,9 @@
 // Three warp-specialised roles run different chunks at once and hand buffers
 // over through mbarriers:
 //   prep group (7 warps): gate tables (one chunk ahead), A and P from the Gram
-//     products, the 16 x 16 diagonal inverse blocks from registers, the
-//     off-diagonal blocks with warp MMAs, Tc = Tinv diag(c) and Eb (bf16);
+//     products, the 16 x 16 diagonal inverse blocks by substitution, then Tinv
+//     by block forward substitution in 8-column strips on warp MMAs, written out
+//     as Tc = Tinv diag(c) and Eb = Tinv diag(beta) (bf16);
 //   MMA-issue warp: every tcgen05 MMA (Gram, W^T / U~^T, X and O against the state,
 //     the state update and the intra-chunk output), in a fixed order per chunk;
 //   state group (4 warps, TMEM lane = value index): -W and Qh operands, X' = X
@@ -65,8 +66,8 @@ constexpr uint32_t SM_V = 98304;      // V: 2 dv-atoms x 64 tokens x 128 B
 constexpr uint32_t SM_W = 114688;     // -W bf16, MN-major: 128 rows (j) x 64 tokens
 constexpr uint32_t SM_P0 = 131072;    // P fp32, K-major: 2 atoms (32 s) x 64 rows; even chunks
 constexpr uint32_t SM_P1 = 147456;    // odd chunks (K K^T is staged here first, P formed in place)
-constexpr uint32_t SM_F1 = 163840;    // fp32 64x64: A; then Tc (bf16) | Eb (bf16)
-constexpr uint32_t SM_F2 = 180224;    // fp32 64x64: Tinv (upper blocks: scratch)
+constexpr uint32_t SM_F1 = 163840;    // Tc (bf16) | Eb (bf16), K-major, operands of the W / U~ MMAs
+constexpr uint32_t SM_F2 = 180224;    // fp32 16x16 blocks: -A and the diagonal blocks of Tinv
 constexpr uint32_t SM_BLO = 196608;   // bf16 64x64 K-major: diag(lo(beta)), zero elsewhere
 constexpr uint32_t SM_QH = 204800;    // Qh bf16, K-major like Q: 2 atoms (64 j) x 64 tokens
 constexpr uint32_t SM_MISC = 221184;  // gate tables, barriers
@@ -88,42 +89,6 @@ constexpr uint32_t ID_XP = tc::idesc_tf32(128, 64, false, false);   // X^T P^T
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// fp32 64 x 64 scratch with an XOR swizzle on the column; byte address in a buffer.
-// h(r) maps the low five row bits onto the five bank bits so that a warp's accesses
-// are conflict-free for one row per lane and for the 8 x 4 / 4 x 8 row-column
-// patterns of the m16n8k8 A and B fragments: r bits 0-1 -> bank bits 3-4, r bit 2
-// -> bank bit 2, r bits 3-4 -> bank bits 0-1.
-__device__ __forceinline__ int fswz(int r) { return ((r & 3) << 3) | (r & 4) | ((r >> 3) & 3); }
-__device__ __forceinline__ int fidx(int r, int s) { return r * 64 + (s ^ fswz(r)); }
-__device__ __forceinline__ uint32_t faddr(uint32_t base, int r, int s) {
-    return base + 4u * (uint32_t)fidx(r, s);
-}
-
-// Diagonal blocks 2p and 2p+1 of Tinv = (I + A)^{-1} from A rows held in registers:
-// one warp, lane l holds row 32p + l of A over columns 32p .. 32p + 31 in a[].
-// Lanes 0-15 invert block 2p, lanes 16-31 block 2p + 1; lane l owns column l & 15
-// of its block (right-looking substitution, the A entries taken from the lane that
-// holds the row by a shuffle within each 16-lane half), and writes it to F2.
-__device__ __forceinline__ void diag_pair_inverse(const float (&a)[32], uint32_t F2, int p, int lane) {
-    const int hb = lane >> 4, j = lane & 15;
-    float al[16];
-#pragma unroll
-    for (int s = 0; s < 16; ++s) al[s] = hb ? a[16 + s] : a[s];
-    float x[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
-#pragma unroll
-    for (int s = 0; s < 15; ++s) {
-        const float xs = x[s];
-#pragma unroll
-        for (int r = s + 1; r < 16; ++r)
-            x[r] = fmaf(-__shfl_sync(0xffffffffu, al[s], r, 16), xs, x[r]);
-    }
-    const int blk = 2 * p + hb;
-#pragma unroll
-    for (int r = 0; r < 16; ++r) tc::sts_f32(faddr(F2, 16 * blk + r, 16 * blk + j), x[r]);
-}
-
 __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
     uint4 w;
     w.x = tc::pack_bf16(v[0], v[1]);
@@ -133,189 +98,151 @@ __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
     return w;
 }
 
-// c[16 x 16] += X(16 x 16 at FX, rx, cx) * Y(16 x 16 at FY, ry, cy), one warp, tf32.
-__device__ __forceinline__ void blk16_mma(float (&c)[2][4], uint32_t FX, int rx, int cx, uint32_t FY,
-                                          int ry, int cy, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-        uint32_t a[4];
-        a[0] = tc::f32_to_tf32(tc::lds_f32(faddr(FX, rx + g, cx + 8 * kk + t)));
-        a[1] = tc::f32_to_tf32(tc::lds_f32(faddr(FX, rx + g + 8, cx + 8 * kk + t)));
-        a[2] = tc::f32_to_tf32(tc::lds_f32(faddr(FX, rx + g, cx + 8 * kk + t + 4)));
-        a[3] = tc::f32_to_tf32(tc::lds_f32(faddr(FX, rx + g + 8, cx + 8 * kk + t + 4)));
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            uint32_t bb[2];
-            bb[0] = tc::f32_to_tf32(tc::lds_f32(faddr(FY, ry + 8 * kk + t, cy + 8 * nt + g)));
-            bb[1] = tc::f32_to_tf32(tc::lds_f32(faddr(FY, ry + 8 * kk + t + 4, cy + 8 * nt + g)));
-            tc::mma_sync_tf32(c[nt], a, bb);
-        }
-    }
-}
+// ---- the inverse Tinv = (I + A)^{-1} of one chunk (prep group) ----
+// Scratch F2 (fp32) is a 4 x 4 grid of 16 x 16 blocks, block (R, C) at float
+// offset 256 (4 R + C).  Its lower blocks hold -A (off-diagonal blocks rounded to
+// tf32, the precision of the warp MMAs that read them; diagonal blocks exact), and
+// four of the unused upper slots hold the diagonal inverse blocks T_ii.  Inside a
+// block, element (r, c) sits at 16 r + (c ^ bsw(r)), bsw(r) = 8 (bit 1 of r) +
+// 4 (bit 2 of r): conflict-free for a row of four floats per lane (16-byte
+// accesses, eight rows per phase), for the m16n8k8 A fragment (rows g, g + 8,
+// columns t, t + 4), the B fragment (rows t, t + 4, column g) and accumulator pairs
+// (rows g, g + 8, columns 2t, 2t + 1).
+__device__ __forceinline__ int bsw(int r) { return ((r & 2) << 2) | (r & 4); }
+__device__ __forceinline__ int boff(int r, int c) { return 16 * r + (c ^ bsw(r)); }
+__device__ __forceinline__ int blk_off(int R, int C) { return 256 * (4 * R + C); }
+__device__ __forceinline__ int td_off(int i) { return 256 * (i < 3 ? i + 1 : 6); }   // T_ii slots
+__device__ __forceinline__ float tf32_round(float x) { return __uint_as_float(tc::f32_to_tf32(x)); }
 
-// The 16 x 16 block at (r0, c0) of F in the accumulator layout of blk16_mma.
-__device__ __forceinline__ void blk16_load(float (&c)[2][4], uint32_t F, int r0, int c0, int lane) {
-    const int g = lane >> 2, t = lane & 3;
+// -A of row r over columns 32 ch .. 32 ch + 31 (a[], zero for s >= r) into its
+// blocks of F2; an upper block of the pair is skipped.
+__device__ __forceinline__ void store_neg_a(float* F2p, int r, int ch, const float (&a)[32]) {
+    const int R = r >> 4, rr = r & 15;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        c[nt][0] = tc::lds_f32(faddr(F, r0 + g, c0 + 8 * nt + 2 * t));
-        c[nt][1] = tc::lds_f32(faddr(F, r0 + g, c0 + 8 * nt + 2 * t + 1));
-        c[nt][2] = tc::lds_f32(faddr(F, r0 + g + 8, c0 + 8 * nt + 2 * t));
-        c[nt][3] = tc::lds_f32(faddr(F, r0 + g + 8, c0 + 8 * nt + 2 * t + 1));
-    }
-}
-
-__device__ __forceinline__ void blk16_store(uint32_t F, int r0, int c0, const float (&c)[2][4],
-                                            float scale, int lane) {
-    const int g = lane >> 2, t = lane & 3;
+    for (int cb = 0; cb < 2; ++cb) {
+        const int C = 2 * ch + cb;
+        if (C > R) continue;
+        float* row = F2p + blk_off(R, C) + 16 * rr;
+        const bool off = (C < R);
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        tc::sts_f32(faddr(F, r0 + g, c0 + 8 * nt + 2 * t), scale * c[nt][0]);
-        tc::sts_f32(faddr(F, r0 + g, c0 + 8 * nt + 2 * t + 1), scale * c[nt][1]);
-        tc::sts_f32(faddr(F, r0 + g + 8, c0 + 8 * nt + 2 * t), scale * c[nt][2]);
-        tc::sts_f32(faddr(F, r0 + g + 8, c0 + 8 * nt + 2 * t + 1), scale * c[nt][3]);
-    }
-}
-
-// Writes Tc = T diag(c) and Eb = (T - I) diag(beta) + diag(beta) (bf16, K-major
-// 64 x 64 at F1 and F1 + 8192) for the 16 x 16 block (i, j) whose T values sit
-// in accumulator layout in `t`.
-__device__ __forceinline__ void tceb_store_frag(uint32_t F1, int i, int j, const float (&t)[2][4],
-                                                uint32_t CS, uint32_t BT, int lane) {
-    const int g = lane >> 2, tt = lane & 3;
+        for (int c4 = 0; c4 < 4; ++c4) {
+            float v[4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        const int s = 16 * j + 8 * nt + 2 * tt;
-        const float c0 = tc::lds_f32(CS + 4u * s), c1 = tc::lds_f32(CS + 4u * (s + 1));
-        const float b0 = tc::lds_f32(BT + 4u * s), b1 = tc::lds_f32(BT + 4u * (s + 1));
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int r = 16 * i + g + 8 * hh;
-            const uint32_t off = tc::sw128(r, 2 * j + nt) + 4u * tt;
-            const float t0 = t[nt][2 * hh], t1 = t[nt][2 * hh + 1];
-            asm volatile("st.shared.b32 [%0], %1;" ::"r"(F1 + off), "r"(tc::pack_bf16(t0 * c0, t1 * c1)) : "memory");
-            asm volatile("st.shared.b32 [%0], %1;" ::"r"(F1 + 8192 + off), "r"(tc::pack_bf16(t0 * b0, t1 * b1)) : "memory");
-        }
-    }
-}
-
-// Tc / Eb of diagonal block `blk` (T_ii in F2) and zeros for the upper block
-// row of that block: 32 threads, row 16 blk + (lane & 15), half of the columns.
-__device__ __forceinline__ void tceb_diag_and_upper(uint32_t F1, uint32_t F2, int blk, int lane,
-                                                    uint32_t CS, uint32_t BT) {
-    const int rr = lane & 15, r = 16 * blk + rr;
-    const int hc = lane >> 4;                     // which 8-element chunk of the block
-    const int c = 2 * blk + hc;
-    float tcv[8], ebv[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const int s = 8 * c + e;
-        const float t = tc::lds_f32(faddr(F2, r, s));
-        const float cv = tc::lds_f32(CS + 4u * s), bv = tc::lds_f32(BT + 4u * s);
-        tcv[e] = (s <= r) ? t * cv : 0.f;
-        ebv[e] = (s < r) ? t * bv : ((s == r) ? bv : 0.f);
-    }
-    tc::sts_u32x4(F1 + tc::sw128(r, c), pack8_bf16(tcv));
-    tc::sts_u32x4(F1 + 8192 + tc::sw128(r, c), pack8_bf16(ebv));
-    // upper blocks of this block row: chunks 2 blk + 2 .. 7
-    for (int cz = 2 * blk + 2 + hc; cz < 8; cz += 2) {
-        tc::sts_u32x4(F1 + tc::sw128(r, cz), make_uint4(0u, 0u, 0u, 0u));
-        tc::sts_u32x4(F1 + 8192 + tc::sw128(r, cz), make_uint4(0u, 0u, 0u, 0u));
-    }
-}
-
-// Off-diagonal blocks of T = (I + A)^{-1} from its diagonal blocks T_ii (in F2),
-// written out directly as the Tc / Eb operands.
-// With N = T_D A_off (N_ij = T_ii A_ij, strictly block-lower, N^4 = 0),
-// I + A = (I + A_D)(I + N), so T = (I - N + N^2 - N^3) T_D.  In blocks:
-//   M_{i+1,i} = -N_{i+1,i}
-//   M_20 = -N_20 + N_21 N_10,   M_31 = -N_31 + N_32 N_21
-//   M_30 = -N_30 + N_31 N_10 - N_32 M_20
-//   T_ij = M_ij T_jj
-// Four levels of single 16 x 16 products, one warp per block.  N_ij is kept in
-// the unused upper block (j, i) of F2, M_20, M_31, M_30 in the lower blocks.
-// A (in F1) is dead after level 1, so at level 2 warps 3-6 turn the diagonal
-// blocks into Tc / Eb (and zero the upper blocks) in F1, and level 4 writes the
-// lower blocks there.
-//
-// Every product step has the form  c = s_i B_init + s_p X Y,  stored to a block of
-// F2 or written out as Tc / Eb, so the levels run as one loop over a per-(level,
-// warp) task table: one copy of the product code instead of one per step (the
-// kernel is sensitive to its instruction footprint).  Table fields, in 16-row
-// block units: kind (0 idle, 1 product, 2 Tc/Eb of diagonal block xr), X (xr, xc)
-// in F2, Y in F1 if yf else F2 at (yr, yc), init (0 none, 1 subtract, 2 add) from
-// F2 (ir, ic), product sign (+1 / -1), output (0: F2 block (or, oc); 1: Tc / Eb
-// block (or, oc)).
-__constant__ signed char kOffTask[4][7][16] = {
-    {   // level 1: N_ij = T_ii A_ij -> F2 (j, i)
-        {1, 1, 1, 1, 1, 0, 0, 0, 0, 1, 0, 0, 1},
-        {1, 2, 2, 1, 2, 1, 0, 0, 0, 1, 0, 1, 2},
-        {1, 3, 3, 1, 3, 2, 0, 0, 0, 1, 0, 2, 3},
-        {1, 2, 2, 1, 2, 0, 0, 0, 0, 1, 0, 0, 2},
-        {1, 3, 3, 1, 3, 1, 0, 0, 0, 1, 0, 1, 3},
-        {1, 3, 3, 1, 3, 0, 0, 0, 0, 1, 0, 0, 3},
-        {0},
-    },
-    {   // level 2: M_20 = N_21 N_10 - N_20, M_31 = N_32 N_21 - N_31, Q_30 = N_31 N_10 - N_30;
-        //          Tc / Eb of the diagonal blocks
-        {1, 1, 2, 0, 0, 1, 1, 0, 2, 1, 0, 2, 0},
-        {1, 2, 3, 0, 1, 2, 1, 1, 3, 1, 0, 3, 1},
-        {1, 1, 3, 0, 0, 1, 1, 0, 3, 1, 0, 3, 0},
-        {2, 0},
-        {2, 1},
-        {2, 2},
-        {2, 3},
-    },
-    {   // level 3: M_30 = Q_30 - N_32 M_20
-        {1, 2, 3, 0, 2, 0, 2, 3, 0, -1, 0, 3, 0},
-        {0}, {0}, {0}, {0}, {0}, {0},
-    },
-    {   // level 4: T_{j+1,j} = -N_{j+1,j} T_jj, T_20 = M_20 T_00, T_31 = M_31 T_11, T_30 = M_30 T_00
-        {1, 0, 1, 0, 0, 0, 0, 0, 0, -1, 1, 1, 0},
-        {1, 1, 2, 0, 1, 1, 0, 0, 0, -1, 1, 2, 1},
-        {1, 2, 3, 0, 2, 2, 0, 0, 0, -1, 1, 3, 2},
-        {1, 2, 0, 0, 0, 0, 0, 0, 0, 1, 1, 2, 0},
-        {1, 3, 1, 0, 1, 1, 0, 0, 0, 1, 1, 3, 1},
-        {1, 3, 0, 0, 0, 0, 0, 0, 0, 1, 1, 3, 0},
-        {0},
-    },
-};
-
-__device__ __forceinline__ void offdiag_inverse(uint32_t F1, uint32_t F2, int pt, uint32_t CS,
-                                                uint32_t BT) {
-    const int warp = pt >> 5, lane = pt & 31;
-#pragma unroll 1
-    for (int lv = 0; lv < 4; ++lv) {
-        const signed char* t = kOffTask[lv][warp];
-        const int kind = t[0];
-        if (kind == 1) {
-            float c[2][4], pr[2][4] = {};
-            if (t[6] != 0) {
-                blk16_load(c, F2, 16 * t[7], 16 * t[8], lane);
-                const float si = (t[6] == 1) ? -1.f : 1.f;
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) c[nt][e] *= si;
-            } else {
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) c[nt][e] = 0.f;
+            for (int e = 0; e < 4; ++e) {
+                const float x = -a[16 * cb + 4 * c4 + e];
+                v[e] = off ? tf32_round(x) : x;
             }
-            blk16_mma(pr, F2, 16 * t[1], 16 * t[2], t[3] ? F1 : F2, 16 * t[4], 16 * t[5], lane);
-            const float sp = (float)t[9];
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) c[nt][e] = fmaf(sp, pr[nt][e], c[nt][e]);
-            if (t[10] == 0) blk16_store(F2, 16 * t[11], 16 * t[12], c, 1.f, lane);
-            else tceb_store_frag(F1, t[11], t[12], c, CS, BT, lane);
-        } else if (kind == 2) {
-            tceb_diag_and_upper(F1, F2, t[1], lane, CS, BT);
+            *reinterpret_cast<float4*>(row + ((4 * c4) ^ bsw(rr))) = make_float4(v[0], v[1], v[2], v[3]);
         }
-        if (lv < 3) tc::named_barrier(BAR_PREP, kPrepThreads);
+    }
+}
+
+// Diagonal block T_bb = (I + A_bb)^{-1}, column j of it per lane (16 lanes per
+// block): x_r = [r = j] + sum_{s<r} (-A)_rs x_s for r = 0 .. 15 (left-looking
+// substitution; row r of -A_bb read as 16-byte broadcasts), into the T_bb slot.
+// Entries above the diagonal come out exactly zero.
+__device__ __forceinline__ void diag_block_inverse(float* F2p, int b, int j) {
+    const float* Ab = F2p + blk_off(b, b);
+    float x[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        float acc = (r == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int c4 = 0; 4 * c4 < r; ++c4) {
+            const float4 v = *reinterpret_cast<const float4*>(Ab + 16 * r + ((4 * c4) ^ bsw(r)));
+            const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (4 * c4 + e < r) acc = fmaf(vv[e], x[4 * c4 + e], acc);
+        }
+        x[r] = acc;
+    }
+    float* Tb = F2p + td_off(b);
+#pragma unroll
+    for (int r = 0; r < 16; ++r) Tb[boff(r, j)] = x[r];
+}
+
+// A 16 x 8 accumulator tile C (c0 = C[g][2t], c1 = C[g][2t+1], c2 = C[g+8][2t],
+// c3 = C[g+8][2t+1]) as the B operand of a K = 16 product: tf32 b = {C[t][g],
+// C[t+4][g], C[8+t][g], C[12+t][g]} (two m16n8k8 steps), by shuffles.
+__device__ __forceinline__ void acc_to_bfrag(const float (&c)[4], uint32_t (&b)[4], int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const int s0 = 4 * t + (g >> 1), s1 = s0 + 16;
+    const bool odd = (g & 1) != 0;
+    const float v00 = __shfl_sync(0xffffffffu, c[0], s0), v01 = __shfl_sync(0xffffffffu, c[1], s0);
+    const float v10 = __shfl_sync(0xffffffffu, c[0], s1), v11 = __shfl_sync(0xffffffffu, c[1], s1);
+    const float v20 = __shfl_sync(0xffffffffu, c[2], s0), v21 = __shfl_sync(0xffffffffu, c[3], s0);
+    const float v30 = __shfl_sync(0xffffffffu, c[2], s1), v31 = __shfl_sync(0xffffffffu, c[3], s1);
+    b[0] = tc::f32_to_tf32(odd ? v01 : v00);
+    b[1] = tc::f32_to_tf32(odd ? v11 : v10);
+    b[2] = tc::f32_to_tf32(odd ? v21 : v20);
+    b[3] = tc::f32_to_tf32(odd ? v31 : v30);
+}
+
+// One strip w (columns 8 w .. 8 w + 7, inside block column j = w / 2) of Tinv by
+// block forward substitution down the strip, from (I + A) Tinv = I:
+//   T_j = the strip of T_jj,   T_i = T_ii (-A_ij T_j - ... - A_i,i-1 T_i-1)  (i > j),
+// each product on m16n8k8 tf32 warp MMAs (the strip's blocks so far kept as B
+// fragments).  Writes the strip's 64 rows of Tc = Tinv diag(c) and
+// Eb = Tinv diag(beta) (bf16, K-major 128B-swizzled at F1 and F1 + 8192), zero
+// above block row j.  CS / BT: shared addresses of c and beta.
+__device__ __forceinline__ void strip_inverse(const float* F2p, uint32_t F1, int w, int lane, uint32_t CS,
+                                              uint32_t BT) {
+    const int j = w >> 1, co = 8 * (w & 1);
+    const int g = lane >> 2, t = lane & 3;
+    const int oa0 = boff(g, t), oa1 = boff(g, t + 4), oa2 = boff(g, 8 + t), oa3 = boff(g, 12 + t);
+    const int ob0 = boff(t, co + g), ob1 = boff(t + 4, co + g);
+    const int s0 = 8 * w + 2 * t;
+    const float c0 = tc::lds_f32(CS + 4u * s0), c1 = tc::lds_f32(CS + 4u * (s0 + 1));
+    const float e0 = tc::lds_f32(BT + 4u * s0), e1 = tc::lds_f32(BT + 4u * (s0 + 1));
+    // rows 16 i + g (+ 8) of this strip: 128B-swizzled chunk w of each row
+    const uint32_t orow = F1 + (uint32_t)g * 128u + ((uint32_t)(w ^ g) << 4) + 4u * (uint32_t)t;
+    auto out = [&](int i, float x0, float x1, float x2, float x3) {
+        const uint32_t o = orow + 2048u * (uint32_t)i;
+        tc::sts_u32(o, tc::pack_bf16(x0 * c0, x1 * c1));
+        tc::sts_u32(o + 8192, tc::pack_bf16(x0 * e0, x1 * e1));
+        tc::sts_u32(o + 1024, tc::pack_bf16(x2 * c0, x3 * c1));
+        tc::sts_u32(o + 1024 + 8192, tc::pack_bf16(x2 * e0, x3 * e1));
+    };
+    const float* Tj = F2p + td_off(j);
+    uint32_t tb[3][4];
+    {
+        const float2 u = *reinterpret_cast<const float2*>(Tj + boff(g, co + 2 * t));
+        const float2 v = *reinterpret_cast<const float2*>(Tj + boff(g, co + 2 * t) + 128);
+        const uint32_t q0 = tc::f32_to_tf32(Tj[ob0]), q1 = tc::f32_to_tf32(Tj[ob1]);
+        const uint32_t q2 = tc::f32_to_tf32(Tj[ob0 + 128]), q3 = tc::f32_to_tf32(Tj[ob1 + 128]);
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            tb[k][0] = q0; tb[k][1] = q1; tb[k][2] = q2; tb[k][3] = q3;
+        }
+#pragma unroll
+        for (int i = 0; i < 3; ++i)
+            if (i < j) out(i, 0.f, 0.f, 0.f, 0.f);
+        out(j, u.x, u.y, v.x, v.y);
+    }
+#pragma unroll
+    for (int i = 1; i < 4; ++i) {
+        if (i <= j) continue;
+        float p[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < i; ++k) {
+            if (k < j) continue;
+            const float* Ab = F2p + blk_off(i, k);
+            tc::mma_sync_tf32(p, __float_as_uint(Ab[oa0]), __float_as_uint(Ab[oa0 + 128]),
+                              __float_as_uint(Ab[oa1]), __float_as_uint(Ab[oa1 + 128]), tb[k][0], tb[k][1]);
+            tc::mma_sync_tf32(p, __float_as_uint(Ab[oa2]), __float_as_uint(Ab[oa2 + 128]),
+                              __float_as_uint(Ab[oa3]), __float_as_uint(Ab[oa3 + 128]), tb[k][2], tb[k][3]);
+        }
+        uint32_t pb[4];
+        acc_to_bfrag(p, pb, lane);
+        const float* Ti = F2p + td_off(i);
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        tc::mma_sync_tf32(x, tc::f32_to_tf32(Ti[oa0]), tc::f32_to_tf32(Ti[oa0 + 128]), tc::f32_to_tf32(Ti[oa1]),
+                          tc::f32_to_tf32(Ti[oa1 + 128]), pb[0], pb[1]);
+        tc::mma_sync_tf32(x, tc::f32_to_tf32(Ti[oa2]), tc::f32_to_tf32(Ti[oa2 + 128]), tc::f32_to_tf32(Ti[oa3]),
+                          tc::f32_to_tf32(Ti[oa3 + 128]), pb[2], pb[3]);
+        out(i, x[0], x[1], x[2], x[3]);
+        if (i < 3) acc_to_bfrag(x, tb[i], lane);
     }
 }
 
@@ -331,18 +258,20 @@ __device__ __noinline__ void gram_mma(uint32_t d, uint32_t kq, uint64_t* bar) {
 // (e^{-g} would leave the normal fp32 range): each entry takes exp2 of its own
 // exponent difference.  Out of line, they are never on the common path.
 //   a_rows_exact: A_rs = beta_r 2^{g'_{r-1} - g'_s} (K K^T)_rs (s < r) for row r over
-//   columns 32 ch .. + 31, from the Gram in TMEM, into F1 (g' = g log2 e)
-__device__ __noinline__ void a_rows_exact(uint32_t F1, uint32_t gram_taddr, int r, int ch, uint32_t ts) {
-    float gv[32];
-    tc::tmem_ld32(gram_taddr, gv);
+//   columns 32 ch .. + 31, from the Gram in TMEM, stored as -A into F2's blocks
+//   (g' = g log2 e)
+__device__ __noinline__ void a_rows_exact(float* F2p, uint32_t gram_taddr, int r, int ch, uint32_t ts) {
+    float a[32];
+    tc::tmem_ld32(gram_taddr, a);
     tc::tmem_ld_wait();
     const float br = tc::lds_f32(ts + 512 + 4u * r), gpr = tc::lds_f32(ts + 256 + 4u * r);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
         const int s = 32 * ch + e;
-        const float v = br * exp2f(gpr - tc::lds_f32(ts + 4u * s)) * gv[e];
-        tc::sts_f32(faddr(F1, r, s), (s < r) ? v : 0.f);
+        const float v = br * exp2f(gpr - tc::lds_f32(ts + 4u * s)) * a[e];
+        a[e] = (s < r) ? v : 0.f;
     }
+    store_neg_a(F2p, r, ch, a);
 }
 //   p_row_exact: P_rs = 2^{g'_r - g'_s} (Q K^T - d K K^T)_rs (s <= r) for row r over
 //   columns 32 ch .. + 31, in place over the staged K K^T row
@@ -402,7 +331,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 6144);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
     volatile int* gabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    const uint32_t F1 = sb + SM_F1, F2 = sb + SM_F2;
+    const uint32_t F1 = sb + SM_F1;
+    float* F2p = reinterpret_cast<float*>(sm + SM_F2);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // CTAs of batch index >= b_split solve the same chain of batch (index - b_split)
@@ -743,6 +673,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                  (n == 0 || tc::mbar_wait(&bars[B_MMA2], (n - 1) & 1, timeout_ns));
             __syncwarp();
             if (!ok) break;
+            COMBA_PHASE(21);
             tc::tc_fence_after();
             tc::mma_amn_bk(tmem + tgn, kqn, KQ_ATOM, F1, ID_WN, 4, 0);
             if (!vzero) {
@@ -754,6 +685,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ok = tc::mbar_wait(&bars[B_WREADY], n & 1, timeout_ns);
             __syncwarp();
             if (!ok) break;
+            COMBA_PHASE(22);
             tc::tc_fence_after();
             tc::mma_bf16_ta_bmn(tmem + TM_X, tmem + TM_SB, sb + SM_W, 8192, ID_SW, 8, vzero ? 0u : 1u);
             tc::mma_commit(&bars[B_MMA1]);
@@ -763,6 +695,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ok = tc::mbar_wait(&bars[B_SPLIT], n & 1, timeout_ns);
             __syncwarp();
             if (!ok) break;
+            COMBA_PHASE(23);
             tc::tc_fence_after();
             tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH, kqn, KQ_ATOM, ID_SK, 4, 1);
             tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH + 32, kqn, KQ_ATOM, ID_SK, 4, 1);
@@ -771,6 +704,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::mma_commit(&bars[stg ? B_PBUF1 : B_PBUF0]);
             // ---- Gram of chunk n+2 (its TMEM buffer held W^T of chunk n, read above)
             if (n + 2 < nchunks) ok = issue_gram(n + 2);
+            COMBA_PHASE(24);
+            COMBA_ITER_NEXT();
         }
         if (!ok) fail(gabort);
     } else {
@@ -779,12 +714,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // diag(lo(beta)).  Seven warps; warp pw reads TMEM lanes 32 (warp & 3) .. + 31 of
         // the Gram (K K^T in lanes 0-63, Q K^T in lanes 64-127):
         //   pw 3, 0, 4: K K^T rows 0-31 x cols 0-31, rows 32-63 x cols 0-31, rows 32-63 x
-        //               cols 32-63: A in registers, K K^T staged for P; pw 3 and 4 then
-        //               invert the diagonal blocks (0, 1) and (2, 3) from their registers
+        //               cols 32-63: K K^T staged for P, -A into F2; pw 3 and 4 then
+        //               invert the diagonal blocks (0, 1) and (2, 3) of their rows
         //   pw 1, 2, 6: Q K^T of the same row/column blocks: P, once K K^T is staged
         //   pw 5:       P rows 0-31 x cols 32-63 are zero (s > r)
         //   pw 5, 0:    the next chunk's gate tables (tokens 0-31, 32-63)
-        // then all seven warps: the off-diagonal blocks, Tc / Eb, diag(lo(beta)).
+        // then one 8-column strip of Tinv per warp (pw 6: strips 6 and 7), written out
+        // as Tc / Eb, and diag(lo(beta)) (pw 4, 5).
         const int pt = tid - kPrepBase;
         const int pw = pt >> 5, q = warp & 3;
         const bool kk_warp = (pw == 0 || pw == 3 || pw == 4);
@@ -858,7 +794,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                   make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]));
                 tc::tc_fence_before();
                 tc::named_barrier_arrive(BAR_KK, kKKThreads);
-                // A_rs = beta_r e^{g_{r-1} - g_s} (K K^T)_rs for s < r, in registers
+                // A_rs = beta_r e^{g_{r-1} - g_s} (K K^T)_rs for s < r -> -A into F2
                 if (fast) {
                     const float cr = tc::lds_f32(ts + 768 + 4u * r);
 #pragma unroll
@@ -869,28 +805,16 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         for (int e = 0; e < 4; ++e)
                             a[4 * c + e] = (32 * ch + 4 * c + e < r) ? cr * iv[e] * a[4 * c + e] : 0.f;
                     }
-                } else {   // rows straight into F1 (once free), then back into registers
-                    ok = ok && (m == 0 || tc::mbar_wait(&bars[B_WN], (m - 1) & 1, timeout_ns));
-                    __syncwarp();
-                    a_rows_exact(F1, tl + tgm + 32 * ch, r, ch, ts);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) a[e] = tc::lds_f32(faddr(F1, r, 32 * ch + e));
+                    store_neg_a(F2p, r, ch, a);
+                } else {
+                    a_rows_exact(F2p, tl + tgm + 32 * ch, r, ch, ts);
                 }
                 COMBA_PHASE(9);
-                if (pw != 0) diag_pair_inverse(a, F2, pw == 4 ? 1 : 0, lane);
-                COMBA_PHASE(10);
-                // A into F1 for the off-diagonal blocks (its lower blocks A_10, A_2x,
-                // A_3x only), once the previous chunk's W/X MMAs have read F1
-                ok = ok && (m == 0 || tc::mbar_wait(&bars[B_WN], (m - 1) & 1, timeout_ns));
-                __syncwarp();
-                COMBA_PHASE(11);
-                if (pw == 0) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) tc::sts_f32(faddr(F1, r, e), a[e]);
-                } else if (lane >= 16) {   // rows 16-31 x cols 0-15 (pw 3), 48-63 x 32-47 (pw 4)
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) tc::sts_f32(faddr(F1, r, 32 * ch + e), a[e]);
+                if (pw != 0) {   // diagonal blocks 0, 1 (pw 3) and 2, 3 (pw 4) from this warp's rows
+                    __syncwarp();
+                    diag_block_inverse(F2p, (pw == 4 ? 2 : 0) + (lane >> 4), lane & 15);
                 }
+                COMBA_PHASE(10);
             } else if (p_warp) {
                 const int r = 32 * (q - 2) + lane;    // row (token) of this thread
                 ok = ok && tc::mbar_wait(&bars[(m & 1) ? B_GRAM1 : B_GRAM0], (m >> 1) & 1, timeout_ns);
@@ -943,17 +867,26 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             COMBA_PHASE(17);
             if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
             COMBA_PHASE(18);
-            // ================= phase 3: off-diagonal blocks of the inverse -> Tc / Eb ==========
-            offdiag_inverse(F1, F2, pt, ts + 768, ts + 512);
+            // ================= phase 3: the inverse's strips -> Tc / Eb ==========
+            // F1 and diag(lo) are free once the previous chunk's W / U~ MMAs are done
+            ok = ok && (m == 0 || tc::mbar_wait(&bars[B_WN], (m - 1) & 1, timeout_ns));
+            __syncwarp();
+            COMBA_PHASE(11);
+            if (ok) {
+                strip_inverse(F2p, F1, pw, lane, ts + 768, ts + 512);
+                if (pw == 6) strip_inverse(F2p, F1, 7, lane, ts + 768, ts + 512);
+            }
             COMBA_PHASE(19);
-            if (pt < 64) {   // diag(lo(beta)) (the previous W/X MMAs are done: see F1 above)
-                const float bv = tc::lds_f32(ts + 512 + 4u * pt);
+            if (pt >= 128 && pt < 192) {   // diag(lo(beta))
+                const int e = pt - 128;
+                const float bv = tc::lds_f32(ts + 512 + 4u * e);
                 const float bh = __bfloat162float(__float2bfloat16_rn(bv));
                 const __nv_bfloat16 lo = __float2bfloat16_rn(bv - bh);
-                tc::sts_u16(sb + SM_BLO + tc::sw128(pt, pt >> 3) + (pt & 7) * 2,
+                tc::sts_u16(sb + SM_BLO + tc::sw128(e, e >> 3) + (e & 7) * 2,
                             *reinterpret_cast<const unsigned short*>(&lo));
             }
             tc::fence_proxy_async_smem();
+            if (!ok) fail(gabort);
             if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
             if (issuer) tc::mbar_arrive(&bars[B_WNREADY]);   // Tc, Eb, diag(lo) of chunk m are in
             __syncwarp();

@@ -389,14 +389,16 @@ __device__ __forceinline__ uint32_t f32_to_tf32(float x) {
     return r;
 }
 
-// d[16x8] += a[16x8] * b[8x8], tf32 inputs, fp32 accumulation, one warp.
-__device__ __forceinline__ void mma_sync_tf32(float (&d)[4], const uint32_t (&a)[4],
-                                              const uint32_t (&b)[2]) {
-    asm volatile(
+// d[16x8] += a[16x8] * b[8x8], tf32 inputs, fp32 accumulation, one warp.  Not
+// volatile: a pure register operation the compiler may schedule among the loads
+// that feed it.
+__device__ __forceinline__ void mma_sync_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm(
         "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
@@ -465,6 +467,9 @@ __device__ __forceinline__ void sts_f32x4(uint32_t a, float4 v) {
 __device__ __forceinline__ void sts_u32x4(uint32_t a, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
                  ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 __device__ __forceinline__ void sts_u16(uint32_t a, unsigned short v) {
     asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(v) : "memory");
