@@ -62,8 +62,9 @@ constexpr uint32_t TM_COLS = 512;
 constexpr int kKQStages = 3;          // q/k tiles in flight: chunk c in stage c % 3
 constexpr uint32_t SM_KQ0 = 0;        // [K;Q] stages: 2 K-atoms x 128 rows x 128 B (bf16) each
 constexpr uint32_t KQ_STAGE = 32768;
-constexpr uint32_t SM_V = 98304;      // V: 2 dv-atoms x 64 tokens x 128 B
-constexpr uint32_t SM_W = 114688;     // -W bf16, MN-major: 128 rows (j) x 64 tokens
+constexpr uint32_t SM_V = 98304;      // V: 2 dv-atoms x 64 tokens x 128 B; once the W / U~ MMAs
+                                      // have read it, -W bf16, MN-major: 128 rows (j) x 64 tokens
+constexpr uint32_t SM_W = 114688;     // out tile staging (two 64-wide boxes)
 constexpr uint32_t SM_P0 = 131072;    // P fp32, K-major: 2 atoms (32 s) x 64 rows; even chunks
 constexpr uint32_t SM_P1 = 147456;    // odd chunks (K K^T is staged here first, P formed in place)
 constexpr uint32_t SM_F1 = 163840;    // Tc (bf16) | Eb (bf16), K-major, operands of the W / U~ MMAs
@@ -399,11 +400,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     COMBA_PHASE_BEGIN();
     if (warp < 4) {
         // =============================== state group ===============================
-        // Per chunk n: -W operand from W^T (TMEM, the prep group's MMA); MMA1(n)
-        // X^T += S (-W)^T, O^T = S Qh^T; MMA2(n) S += X^T (D K), O^T += X^T P^T; then
-        // S -> bf16 copy, S *= e^{g_L(n+1)}, O^T -> out (staged in this chunk's P
-        // buffer), and the (D K)^T and Qh operands of chunk n+1 from the group's own
-        // scan of its log-decays.
+        // Per chunk n: the -W operand from W^T (TMEM, the prep group's MMA) into the V
+        // buffer; MMA1(n) X^T += S (-W)^T, O^T = S Qh^T; X' = X diag(e^{g_L - g}) as bf16
+        // hi + lo; MMA2(n) S += X'^T K, O^T += X^T P^T; then S -> bf16 copy,
+        // S *= e^{g_L(n+1)}, O^T -> out (staged, TMA store), and the Qh operand of
+        // chunk n+1 from the group's own scan of its log-decays.
         const int row = tid;
         const bool issuer = (tid == 0);
         // Scan of chunk c's log-decays held by threads 0..63: writes e^{g_L - g_r} to
@@ -495,9 +496,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const uint32_t tgn = stg ? TM_G1 : TM_G;
             const bool last = (n + 1 == nchunks);
             // ---- -W operand from W^T (lane = j, column = token) once the prep's MMAs are
-            // done and the previous chunk's out store has read its staging (same buffer)
+            // done, into the V buffer (those MMAs have read V)
             ok = (*gabort == 0) && tc::mbar_wait(&bars[B_WN], n & 1, timeout_ns);
-            if (issuer) tc::bulk_wait_read0();
             tc::named_barrier(BAR_STATE, kStateThreads);
             COMBA_PHASE(0);
             tc::tc_fence_after();
@@ -510,19 +510,15 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int e = 0; e < 32; ++e) { w0[e] = -w0[e]; w1[e] = -w1[e]; }
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
-                    tc::sts_u32x4(sb + SM_W + tc::sw128(row, c4), pack8_bf16(w0 + c4 * 8));
-                    tc::sts_u32x4(sb + SM_W + tc::sw128(row, 4 + c4), pack8_bf16(w1 + c4 * 8));
+                    tc::sts_u32x4(sb + SM_V + tc::sw128(row, c4), pack8_bf16(w0 + c4 * 8));
+                    tc::sts_u32x4(sb + SM_V + tc::sw128(row, 4 + c4), pack8_bf16(w1 + c4 * 8));
                 }
             }
             tc::fence_proxy_async_smem();
             tc::tc_fence_before();
             if (!ok) fail(gabort);
             if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
-            if (issuer) {
-                tc::mbar_arrive(&bars[B_WREADY]);  // -W and the S copies are in: MMA1
-                tc::fence_proxy_async_smem();      // V has been read by the W/X MMAs
-                if (n + 1 < nchunks && !vzero) load_v(n + 1);
-            }
+            if (issuer) tc::mbar_arrive(&bars[B_WREADY]);  // -W and the S copies are in: MMA1
             __syncwarp();
             COMBA_PHASE(1);
             // ---- while MMA1 runs: the next chunk's decays
@@ -531,6 +527,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // ---- X' = X diag(e^{g_L - g}) as bf16 hi + lo (operand of the state update)
             ok = ok && tc::mbar_wait(&bars[B_MMA1], n & 1, timeout_ns);
             tc::tc_fence_after();
+            if (issuer && ok && n + 1 < nchunks && !vzero) load_v(n + 1);   // MMA1 has read -W
             COMBA_PHASE(6);
             const uint32_t sedn = sed(n);
 #pragma unroll 1
@@ -568,12 +565,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             COMBA_PHASE(3);
             ok = ok && tc::mbar_wait(&bars[B_MMA2], n & 1, timeout_ns);
+            if (issuer) tc::bulk_wait_read0();   // the previous out store has read its staging
             if (!ok) fail(gabort);
             if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
             tc::tc_fence_after();
             if (issuer && n + kKQStages < nchunks) {   // this chunk's q/k stage is read
                 tc::fence_proxy_async_smem();
                 load_kq(n + kKQStages);
+                COMBA_PHASE(26);
             }
             __syncwarp();
             COMBA_PHASE(4);
@@ -624,8 +623,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             COMBA_PHASE(5);
             if (want_out) {
             // out tile [token][value index] in two 64-wide 128B-swizzled boxes, staged in
-            // the -W buffer (MMA1 has read it), TMA store.  The barrier below also hands
-            // the new S copies to the next MMA1.
+            // its own buffer, TMA store.  The barrier below also hands the new S copies to
+            // the next MMA1.
             {
                 const uint32_t ot = sb + SM_W + (row >> 6) * 8192 + (row & 7) * 2;
                 const int oc = (row & 63) >> 3;
@@ -648,11 +647,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (issuer) tc::bulk_wait0();
     } else if (warp == kCtlWarp) {
         // ============================ MMA-issue warp ===============================
-        // All tensor-core MMAs, in one order per chunk n: W^T / U~^T of chunk n (once
-        // the prep group hands over its Tc / Eb), MMA1(n) (once the state group hands
-        // over -W and the S copies), MMA2(n) (once it hands over X'), then the Gram of
-        // chunk n+2 into the TMEM buffer whose W^T the state group has just read.  Each
-        // wait depends only on MMAs issued before it, so the order cannot deadlock.
+        // All tensor-core MMAs.  Per chunk n: MMA1(n) (once the state group hands over
+        // -W and the S copies), then O^T += X^T P^T (needs only X^T and P, so it runs
+        // while the state group splits X'), then the state update (once it hands over
+        // X').  Then W^T / U~^T of chunk n+1 (once the prep group hands over Tc / Eb)
+        // and the Gram of chunk n+2 (into the TMEM buffer whose W^T the state group
+        // has read), W^T / U~^T first unless the prep group is not done with chunk
+        // n+1 yet.  The tensor pipe runs MMAs in issue order; every wait depends only
+        // on MMAs issued before it, so no order of these can deadlock.
         bool ok = true;
         auto issue_gram = [&](int c) -> bool {
             const bool okg = tc::mbar_wait(kq_bar(c), kq_par(c), timeout_ns);
@@ -661,37 +663,44 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 gram_mma(tmem + ((c & 1) ? TM_G1 : TM_G), sb + kq_stage(c), &bars[(c & 1) ? B_GRAM1 : B_GRAM0]);
             return okg;
         };
-        ok = issue_gram(0) && (nchunks < 2 || issue_gram(1));
+        // W^T = K^T Tc^T;  X^T = U~^T = V^T Eb^T + V^T diag(lo)^T  of chunk c (X^T of chunk
+        // c-1 read by its O MMA, committed with its P buffer)
+        auto issue_wn = [&](int c) -> bool {
+            const bool okw = tc::mbar_wait(&bars[B_WNREADY], c & 1, timeout_ns) &&
+                             (vzero || tc::mbar_wait(&bars[B_V], c & 1, timeout_ns)) &&
+                             (c == 0 || tc::mbar_wait(&bars[((c - 1) & 1) ? B_PBUF1 : B_PBUF0],
+                                                      ((c - 1) >> 1) & 1, timeout_ns));
+            __syncwarp();
+            if (okw) {
+                COMBA_PHASE(21);
+                tc::tc_fence_after();
+                const uint32_t kqc = sb + kq_stage(c);
+                tc::mma_amn_bk(tmem + ((c & 1) ? TM_G1 : TM_G), kqc, KQ_ATOM, F1, ID_WN, 4, 0);
+                if (!vzero) {
+                    tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, F1 + 8192, ID_WN, 4, 0);
+                    tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
+                }
+                tc::mma_commit(&bars[B_WN]);
+            }
+            return okw;
+        };
+        ok = issue_gram(0) && (nchunks < 2 || issue_gram(1)) && issue_wn(0);
         for (int n = 0; n < nchunks && ok; ++n) {
             const int stg = n & 1;
             const uint32_t kqn = sb + kq_stage(n);
-            const uint32_t tgn = stg ? TM_G1 : TM_G;
-            // ---- W^T = K^T Tc^T;  X^T = U~^T = V^T Eb^T + V^T diag(lo)^T  (X^T of chunk n-1
-            // read by its MMA2)
-            ok = tc::mbar_wait(&bars[B_WNREADY], n & 1, timeout_ns) &&
-                 (vzero || tc::mbar_wait(&bars[B_V], n & 1, timeout_ns)) &&
-                 (n == 0 || tc::mbar_wait(&bars[B_MMA2], (n - 1) & 1, timeout_ns));
-            __syncwarp();
-            if (!ok) break;
-            COMBA_PHASE(21);
-            tc::tc_fence_after();
-            tc::mma_amn_bk(tmem + tgn, kqn, KQ_ATOM, F1, ID_WN, 4, 0);
-            if (!vzero) {
-                tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, F1 + 8192, ID_WN, 4, 0);
-                tc::mma_amn_bk(tmem + TM_X, sb + SM_V, V_ATOM, sb + SM_BLO, ID_WN, 4, 1);
-            }
-            tc::mma_commit(&bars[B_WN]);
-            // ---- MMA1(n): X^T += S (-W)^T;  O^T = S Qh^T
+            // ---- MMA1(n): X^T += S (-W)^T;  O^T = S Qh^T;  then O^T += X^T P^T
             ok = tc::mbar_wait(&bars[B_WREADY], n & 1, timeout_ns);
             __syncwarp();
             if (!ok) break;
             COMBA_PHASE(22);
             tc::tc_fence_after();
-            tc::mma_bf16_ta_bmn(tmem + TM_X, tmem + TM_SB, sb + SM_W, 8192, ID_SW, 8, vzero ? 0u : 1u);
+            tc::mma_bf16_ta_bmn(tmem + TM_X, tmem + TM_SB, sb + SM_V, 8192, ID_SW, 8, vzero ? 0u : 1u);
             tc::mma_commit(&bars[B_MMA1]);
             if (want_out) tc::mma_bf16_ta_bk(tmem + TM_O, tmem + TM_SB, sb + SM_QH, QH_ATOM, ID_SQ, 8, 0);
             tc::mma_commit(&bars[B_MMA1B]);
-            // ---- MMA2(n): S += X'^T K (bf16 hi + lo);  O^T += X^T P^T
+            if (want_out) tc::mma_tf32_ta_bk(tmem + TM_O, tmem + TM_X, sb + (stg ? SM_P1 : SM_P0), F32_ATOM, ID_XP, 8, 1);
+            tc::mma_commit(&bars[stg ? B_PBUF1 : B_PBUF0]);
+            // ---- MMA2(n): S += X'^T K (bf16 hi + lo)
             ok = tc::mbar_wait(&bars[B_SPLIT], n & 1, timeout_ns);
             __syncwarp();
             if (!ok) break;
@@ -699,11 +708,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::tc_fence_after();
             tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH, kqn, KQ_ATOM, ID_SK, 4, 1);
             tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH + 32, kqn, KQ_ATOM, ID_SK, 4, 1);
-            if (want_out) tc::mma_tf32_ta_bk(tmem + TM_O, tmem + TM_X, sb + (stg ? SM_P1 : SM_P0), F32_ATOM, ID_XP, 8, 1);
             tc::mma_commit(&bars[B_MMA2]);
-            tc::mma_commit(&bars[stg ? B_PBUF1 : B_PBUF0]);
-            // ---- Gram of chunk n+2 (its TMEM buffer held W^T of chunk n, read above)
-            if (n + 2 < nchunks) ok = issue_gram(n + 2);
+            COMBA_PHASE(25);
+            // ---- W^T / U~^T of chunk n+1 and the Gram of chunk n+2
+            bool need_wn = n + 1 < nchunks, need_gram = n + 2 < nchunks;
+            if (need_wn && need_gram &&
+                !(tc::mbar_test(&bars[B_WNREADY], (n + 1) & 1) && (vzero || tc::mbar_test(&bars[B_V], (n + 1) & 1)))) {
+                ok = issue_gram(n + 2);
+                need_gram = false;
+            }
+            if (ok && need_wn) ok = issue_wn(n + 1);
+            if (ok && need_gram) ok = issue_gram(n + 2);
             COMBA_PHASE(24);
             COMBA_ITER_NEXT();
         }

@@ -275,10 +275,11 @@ extern "C" int comba_trace_read_cta_clk(long long* host_3072) {
                    cudaSuccess ? COMBA_OK : COMBA_ECUDA;
 }
 
-// Tracing builds only: absolute mark timestamps of one loop iteration, two threads.
-extern "C" int comba_trace_read_ts(long long* host_2slots) {
+// Tracing builds only: absolute mark timestamps of three threads over four loop iterations.
+extern "C" int comba_trace_read_ts(long long* host_ts) {
     if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;
-    return cudaMemcpyFromSymbol(host_2slots, comba::g_phase_ts, 2 * COMBA_TRACE_SLOTS * sizeof(long long)) ==
+    return cudaMemcpyFromSymbol(host_ts, comba::g_phase_ts,
+                                3 * COMBA_TRACE_TS_ITERS * COMBA_TRACE_SLOTS * sizeof(long long)) ==
                    cudaSuccess ? COMBA_OK : COMBA_ECUDA;
 }
 #endif

@@ -16,9 +16,12 @@ __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0,
 // Optional phase tracing (compile with -DCOMBA_TRACE_PHASES): thread 0 and thread
 // COMBA_TRACE_TID2 (default 128) of CTA 0 accumulate clock64() deltas between
 // consecutive COMBA_PHASE marks in registers (each thread its own slots) and add
-// them to a device array at COMBA_PHASE_END.  Off by default; the marks then
-// compile to nothing.
+// them to a device array at COMBA_PHASE_END; threads 0 (state group), 128 (MMA-issue
+// warp) and COMBA_TRACE_TID2 also record the absolute clock64() of every mark in
+// loop iterations COMBA_TRACE_ITER .. + 3.  Off by default; the marks then compile
+// to nothing.
 #define COMBA_TRACE_SLOTS 32
+#define COMBA_TRACE_TS_ITERS 4
 #ifdef COMBA_TRACE_PHASES
 #ifndef COMBA_TRACE_TID2
 #define COMBA_TRACE_TID2 128
@@ -30,9 +33,8 @@ __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0,
 #define COMBA_TRACE_CTA 0
 #endif
 __device__ unsigned long long g_phase_cycles[COMBA_TRACE_SLOTS];
-// absolute clock64() of each mark: thread 0 in loop iteration COMBA_TRACE_ITER,
-// thread TID2 in the next one (the prep group runs one chunk ahead): [thread 0 | TID2]
-__device__ long long g_phase_ts[2 * COMBA_TRACE_SLOTS];
+// [thread 0 | thread 128 | thread TID2][iteration ITER + k][mark]
+__device__ long long g_phase_ts[3 * COMBA_TRACE_TS_ITERS * COMBA_TRACE_SLOTS];
 #define COMBA_PHASE_BEGIN()                                   \
     long long comba_phase_t = clock64();                      \
     int comba_iter = 0;                                       \
@@ -46,9 +48,13 @@ __device__ long long g_phase_ts[2 * COMBA_TRACE_SLOTS];
         const long long comba_phase_now = clock64();                          \
         comba_phase_acc[(i)] += (unsigned long long)(comba_phase_now - comba_phase_t); \
         comba_phase_t = comba_phase_now;                                      \
-        if (comba_iter == COMBA_TRACE_ITER + (threadIdx.x == 0 ? 0 : 1) && blockIdx.x == COMBA_TRACE_CTA && \
-            (threadIdx.x == 0 || threadIdx.x == COMBA_TRACE_TID2))            \
-            g_phase_ts[(threadIdx.x == 0 ? 0 : COMBA_TRACE_SLOTS) + (i)] = comba_phase_now; \
+        const int comba_k = comba_iter - COMBA_TRACE_ITER;                    \
+        const int comba_w = threadIdx.x == 0 ? 0 : threadIdx.x == 128 ? 1     \
+                          : threadIdx.x == COMBA_TRACE_TID2 ? 2 : -1;         \
+        if (comba_k >= 0 && comba_k < COMBA_TRACE_TS_ITERS && comba_w >= 0 && \
+            blockIdx.x == COMBA_TRACE_CTA)                                    \
+            g_phase_ts[(comba_w * COMBA_TRACE_TS_ITERS + comba_k) * COMBA_TRACE_SLOTS + (i)] = \
+                comba_phase_now;                                              \
     } while (0)
 #define COMBA_ITER_NEXT() (++comba_iter)
 // per-CTA start / end (global timer, ns) of up to 1024 CTAs, and SM clock cycles
