@@ -20,16 +20,17 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["chunk_fwd", "recurrent_step", "get_last_error", "CombaError", "library",
-           "library_path", "EXPORTS", "status_string"]
+__all__ = ["chunk_fwd", "chunk_fwd_varlen", "chunk_fwd_noalloc", "recurrent_step",
+           "get_last_error", "CombaError", "library", "library_path", "EXPORTS", "status_string"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libcomba.so")
 _lib = None
 _lock = threading.Lock()
 
-EXPORTS = ("comba_chunk_fwd", "comba_chunk_fwd_f32", "comba_recurrent_step",
-           "comba_get_last_error", "comba_status_string", "comba_version")
+EXPORTS = ("comba_chunk_fwd", "comba_chunk_fwd_f32", "comba_chunk_fwd_varlen",
+           "comba_chunk_fwd_workspace_size", "comba_chunk_fwd_ws", "comba_chunk_fwd_noalloc",
+           "comba_recurrent_step", "comba_get_last_error", "comba_status_string", "comba_version")
 
 
 class CombaError(RuntimeError):
@@ -59,9 +60,10 @@ def library():
             lib.comba_chunk_fwd_noalloc.argtypes = chunk_sig
             lib.comba_chunk_fwd_workspace_size.argtypes = [i] * 6
             lib.comba_chunk_fwd_workspace_size.restype = ctypes.c_size_t
+            lib.comba_chunk_fwd_varlen.argtypes = [vp] * 10 + [i] * 7 + [vp]
             lib.comba_recurrent_step.argtypes = [vp] * 8 + [i] * 4 + [vp]
             for fn in (lib.comba_chunk_fwd, lib.comba_chunk_fwd_f32, lib.comba_chunk_fwd_ws,
-                       lib.comba_chunk_fwd_noalloc,
+                       lib.comba_chunk_fwd_noalloc, lib.comba_chunk_fwd_varlen,
                        lib.comba_recurrent_step, lib.comba_get_last_error, lib.comba_version):
                 fn.restype = ctypes.c_int
             lib.comba_get_last_error.argtypes = []
@@ -151,6 +153,51 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
             name = "comba_chunk_fwd_f32"
     if st != 0:
         raise CombaError(st, name)
+    return out, S_final
+
+
+def chunk_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                     beta: torch.Tensor, d: torch.Tensor, cu_seqlens: torch.Tensor,
+                     S0: Optional[torch.Tensor] = None, chunk: int = 64,
+                     out: Optional[torch.Tensor] = None, S_final: Optional[torch.Tensor] = None,
+                     return_state: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunk-wise forward over packed variable-length sequences (comba_chunk_fwd_varlen).
+    q, k [total_T, Hqk, dk] bf16; v [total_T, H, dv] bf16 with Hqk dividing H (value
+    head h reads q / k head h // (H // Hqk)); log_alpha, beta [total_T, H] fp32; d [H]
+    fp32; cu_seqlens [N+1] int32 on the device (sequence n = tokens cu_seqlens[n] ..
+    cu_seqlens[n+1]-1); S0 [N, H, dv, dk] fp32 or None.  Returns (out [total_T, H, dv]
+    bf16, S_final [N, H, dv, dk] fp32 or None)."""
+    if q.dim() != 3:
+        raise ValueError("q must be [total_T, Hqk, dk]")
+    total_T, Hqk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be [N + 1]")
+    N = cu_seqlens.numel() - 1
+    _check(q, "q", torch.bfloat16, (total_T, Hqk, dk))
+    _check(k, "k", torch.bfloat16, (total_T, Hqk, dk))
+    _check(v, "v", torch.bfloat16, (total_T, H, dv))
+    _check(log_alpha, "log_alpha", torch.float32, (total_T, H))
+    _check(beta, "beta", torch.float32, (total_T, H))
+    _check(d, "d", torch.float32, (H,))
+    _check(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,))
+    dev = q.device
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (N, H, dv, dk))
+    if out is None:
+        out = torch.empty((total_T, H, dv), dtype=torch.bfloat16, device=dev)
+    _check(out, "out", torch.bfloat16, (total_T, H, dv))
+    if S_final is None and return_state:
+        S_final = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _check(S_final, "S_final", torch.float32, (N, H, dv, dk))
+    with torch.cuda.device(dev):
+        st = library().comba_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                              _ptr(d), _ptr(S0), _ptr(out), _ptr(S_final),
+                                              _ptr(cu_seqlens), N, total_T, H, Hqk, dk, dv, int(chunk),
+                                              _stream_handle(dev, stream))
+    if st != 0:
+        raise CombaError(st, "comba_chunk_fwd_varlen")
     return out, S_final
 
 

@@ -62,7 +62,8 @@ chunk_fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                       const Tin* __restrict__ v, const float* __restrict__ log_alpha,
                       const float* __restrict__ beta, const float* __restrict__ dvec,
                       const float* S0, Tin* __restrict__ out, float* S_final,
-                      int T, int H, int dk, int dv, int C, int dvt) {
+                      int T, int H, int dk, int dv, int C, int dvt,
+                      const int* __restrict__ cu_seqlens, int Hqk) {
     extern __shared__ float sm[];
     const SimtSmem L_ = simt_smem_layout(dk, dvt, C);
     float* Ks = sm + L_.k;
@@ -82,6 +83,22 @@ chunk_fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     const int tid = threadIdx.x, nt = blockDim.x;
     const int i0 = blockIdx.x * dvt;
     const int h = blockIdx.y, b = blockIdx.z;
+    // The chain's tokens: rows b T .. b T + T - 1 of the token axis, or, for packed
+    // sequences, rows cu_seqlens[b] .. cu_seqlens[b+1]-1 (T = total tokens); its q / k
+    // head is h / (H / Hqk).
+    size_t row0 = (size_t)b * T;
+    int Tc = T;
+    if (cu_seqlens) {
+        const int s0 = cu_seqlens[b], s1 = cu_seqlens[b + 1];
+        if (s0 < 0 || s1 < s0 || s1 > T) {   // malformed bounds: the sequence is skipped
+            if (threadIdx.x == 0) latch_status(-1 /* COMBA_EINVAL */);
+            Tc = 0;
+        } else {
+            row0 = (size_t)s0;
+            Tc = s1 - s0;
+        }
+    }
+    const int hq = h / (H / Hqk);
     const int nv = min(dvt, dv - i0);
     const int ny = dk + nv;
     const float dh = dvec[h];
@@ -92,21 +109,21 @@ chunk_fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         Ss[i * ldk + j] = S0 ? S0[state_off + (size_t)(i0 + i) * dk + j] : 0.f;
     }
 
-    for (int c0 = 0; c0 < T; c0 += C) {
-        const int L = min(C, T - c0);
+    for (int c0 = 0; c0 < Tc; c0 += C) {
+        const int L = min(C, Tc - c0);
         __syncthreads();
         for (int idx = tid; idx < L * dk; idx += nt) {
             const int r = idx / dk, j = idx % dk;
-            const size_t off = (((size_t)b * T + c0 + r) * H + h) * dk + j;
+            const size_t off = ((row0 + c0 + r) * Hqk + hq) * dk + j;
             Ks[r * ldk + j] = to_f32(k[off]);
             Qs[r * ldk + j] = to_f32(q[off]);
         }
         for (int idx = tid; idx < L * nv; idx += nt) {
             const int r = idx / nv, i = idx % nv;
-            Vs[r * ldv + i] = to_f32(v[(((size_t)b * T + c0 + r) * H + h) * dv + i0 + i]);
+            Vs[r * ldv + i] = to_f32(v[((row0 + c0 + r) * H + h) * dv + i0 + i]);
         }
         if (tid < L) {
-            const size_t o = ((size_t)b * T + c0 + tid) * H + h;
+            const size_t o = (row0 + c0 + tid) * H + h;
             gs[tid] = log_alpha[o];
             bs[tid] = beta[o];
         }
@@ -166,7 +183,7 @@ chunk_fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                 acc = fmaf(Qs[r * ldk + j] - dh * Ks[r * ldk + j], Ss[i * ldk + j], acc);
             acc *= expf(gs[r]);
             for (int s = 0; s <= r; ++s) acc = fmaf(PP[r * ldc + s], Xs[s * ldx + i], acc);
-            out[(((size_t)b * T + c0 + r) * H + h) * dv + i0 + i] = from_f32<Tin>(acc);
+            out[((row0 + c0 + r) * H + h) * dv + i0 + i] = from_f32<Tin>(acc);
         }
         __syncthreads();
         // S <- e^{g_L} S + X^T diag(e^{g_L - g_s}) K

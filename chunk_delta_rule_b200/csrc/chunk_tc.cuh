@@ -296,12 +296,17 @@ __device__ __forceinline__ void fail(volatile int* gabort) {
     latch_status(-4 /* COMBA_ETIMEOUT */);
 }
 
+// kPacked: chains are packed variable-length sequences (cu_seqlens) whose q / k heads
+// may be shared by groups of value heads; the fixed-length instantiation compiles
+// without those paths.
+template <bool kPacked>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     const float* __restrict__ log_alpha, const float* __restrict__ beta,
                     const float* __restrict__ dvec, const float* S0, float* S_final, int T, int H,
-                    int b_split, int no_out, unsigned long long timeout_ns) {
+                    int b_split, int no_out, unsigned long long timeout_ns,
+                    const int* __restrict__ cu_seqlens, int qk_group, unsigned short* out_raw) {
     COMBA_CTA_MARK(0);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
@@ -344,7 +349,26 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int b = vzero ? bcta - b_split : bcta;
     const bool want_out = (no_out == 0);
     const float dh = dvec[h];
-    const int nchunks = (T + kC - 1) / kC;
+    // The chain's tokens along the tensor maps' token axis (extent T): rows 0 .. T-1 of
+    // batch b, or, for packed sequences (cu_seqlens), rows cu_seqlens[b] ..
+    // cu_seqlens[b+1]-1 of the single batch.  Its q / k head is h / qk_group.
+    int tok0 = 0, Tc = T, bm = b;
+    if constexpr (kPacked) {
+        const int s0 = cu_seqlens[b], s1 = cu_seqlens[b + 1];
+        bm = 0;
+        if (s0 < 0 || s1 < s0 || s1 > T) {   // malformed bounds: the sequence is skipped
+            if (tid == 0) latch_status(-1 /* COMBA_EINVAL */);
+            Tc = 0;
+        } else {
+            tok0 = s0;
+            Tc = s1 - s0;
+        }
+    }
+    const int hq = kPacked ? h / qk_group : h;
+    // a packed sequence's ragged last tile is written with plain stores (a TMA store
+    // would write into the next sequence's rows)
+    const bool clip_tail = kPacked && (Tc % kC != 0);
+    const int nchunks = (Tc + kC - 1) / kC;
     const uint32_t trow = (uint32_t)((warp & 3) * 32) << 16;
 
     if (tid == 0) {
@@ -373,32 +397,40 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         uint8_t* dst = sm + kq_stage(n);
         uint64_t* bar = kq_bar(n);
         tc::mbar_arrive_expect_tx(bar, 32768);
-        const int t0 = n * kC;
-        tc::tma_load_4d(dst, &tm_k, bar, 0, h, t0, b);
-        tc::tma_load_4d(dst + 8192, &tm_q, bar, 0, h, t0, b);
-        tc::tma_load_4d(dst + KQ_ATOM, &tm_k, bar, 64, h, t0, b);
-        tc::tma_load_4d(dst + KQ_ATOM + 8192, &tm_q, bar, 64, h, t0, b);
+        const int t0 = tok0 + n * kC;
+        tc::tma_load_4d(dst, &tm_k, bar, 0, hq, t0, bm);
+        tc::tma_load_4d(dst + 8192, &tm_q, bar, 0, hq, t0, bm);
+        tc::tma_load_4d(dst + KQ_ATOM, &tm_k, bar, 64, hq, t0, bm);
+        tc::tma_load_4d(dst + KQ_ATOM + 8192, &tm_q, bar, 64, hq, t0, bm);
     };
     auto load_v = [&](int n) {
         tc::mbar_arrive_expect_tx(&bars[B_V], 16384);
-        const int t0 = n * kC;
-        tc::tma_load_4d(sm + SM_V, &tm_v, &bars[B_V], 0, h, t0, b);
-        tc::tma_load_4d(sm + SM_V + V_ATOM, &tm_v, &bars[B_V], 64, h, t0, b);
+        const int t0 = tok0 + n * kC;
+        tc::tma_load_4d(sm + SM_V, &tm_v, &bars[B_V], 0, h, t0, bm);
+        tc::tma_load_4d(sm + SM_V + V_ATOM, &tm_v, &bars[B_V], 64, h, t0, bm);
     };
     // One token's gate value.  The load is issued where it is written (volatile) and
     // consumed a phase later, so its latency stays hidden; a plain load may be sunk
     // by the compiler to its use, past the waits in between.
     auto gate = [&](const float* p, int t) -> float {
         float v = 0.f;
-        if (t < T) {
-            const float* a = p + ((size_t)b * T + t) * H + h;
+        if (t < Tc) {
+            const float* a = p + ((size_t)bm * T + tok0 + t) * H + h;
             asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(a));
         }
         return v;
     };
 
     COMBA_PHASE_BEGIN();
-    if (warp < 4) {
+    if (kPacked && nchunks == 0) {
+        // an empty chain (a zero-length packed sequence): S_final = S0 (or zero)
+        if (warp < 4 && S_final) {
+            const size_t ro = ((size_t)blockIdx.x * kD + tid) * kD;
+            for (int e = 0; e < kD; e += 4)
+                *reinterpret_cast<float4*>(S_final + ro + e) =
+                    S0 ? *reinterpret_cast<const float4*>(S0 + ro + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    } else if (warp < 4) {
         // =============================== state group ===============================
         // Per chunk n: the -W operand from W^T (TMEM, the prep group's MMA) into the V
         // buffer; MMA1(n) X^T += S (-W)^T, O^T = S Qh^T; X' = X diag(e^{g_L - g}) as bf16
@@ -623,7 +655,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             COMBA_PHASE(5);
             if (want_out) {
             // out tile [token][value index] in two 64-wide 128B-swizzled boxes, staged in
-            // its own buffer, TMA store.  The barrier below also hands the new S copies to
+            // its own buffer, TMA store; a packed sequence's ragged last tile is copied
+            // out row by row instead.  The barrier below also hands the new S copies to
             // the next MMA1.
             {
                 const uint32_t ot = sb + SM_W + (row >> 6) * 8192 + (row & 7) * 2;
@@ -636,9 +669,16 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             tc::fence_proxy_async_smem();
             tc::named_barrier(BAR_STATE, kStateThreads);
-            if (issuer) {
-                tc::tma_store_4d(&tm_o, sm + SM_W, 0, h, t0, b);
-                tc::tma_store_4d(&tm_o, sm + SM_W + 8192, 64, h, t0, b);
+            if (clip_tail && last) {
+                const int rows = Tc - t0;   // 16-byte pieces: value indices 8c .. 8c+7 of row r
+                for (int e = row; e < rows * 16; e += kStateThreads) {
+                    const int r = e >> 4, c = e & 15;
+                    const uint4 w = tc::lds_u32x4(sb + SM_W + (c >> 3) * 8192 + tc::sw128(r, c & 7));
+                    *reinterpret_cast<uint4*>(out_raw + (((size_t)bm * T + tok0 + t0 + r) * H + h) * kD + 8 * c) = w;
+                }
+            } else if (issuer) {
+                tc::tma_store_4d(&tm_o, sm + SM_W, 0, h, tok0 + t0, bm);
+                tc::tma_store_4d(&tm_o, sm + SM_W + 8192, 64, h, tok0 + t0, bm);
                 tc::bulk_commit();
             }
             }
@@ -959,27 +999,38 @@ constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
 
 // One CTA per (b, h) of Bc stacked batches over data with B batches (Bc defaults to B):
 // stacked batches b >= B repeat data batch b - B with V = 0.  out == nullptr: no
-// outputs are written.
+// outputs are written.  Packed sequences: cu_seqlens (device, nseq + 1 entries) cuts
+// the token axis of a single batch (B = 1, T = total tokens) into nseq chains, one
+// CTA per (sequence, head).  Hqk: number of q / k heads (divides H; 0 means H).
 inline int launch_chunk_tc(const void* q, const void* k, const void* v, const float* log_alpha,
                            const float* beta, const float* d, const float* S0, void* out,
                            float* S_final, int B, int T, int H, cudaStream_t stream,
-                           int Bc = -1, unsigned long long timeout_ns = kWaitTimeoutNs) {
+                           int Bc = -1, unsigned long long timeout_ns = kWaitTimeoutNs,
+                           const int* cu_seqlens = nullptr, int nseq = 0, int Hqk = 0) {
     if (Bc < 0) Bc = B;
+    if (Hqk <= 0) Hqk = H;
+    if (H % Hqk != 0) return -1;
     static bool attr_set[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -3;
     if (!attr_set[dev]) {
-        if (cudaFuncSetAttribute(tck::chunk_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(tck::chunk_fwd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tck::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(tck::chunk_fwd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)tck::kSmemBytes) != cudaSuccess)
             return -3;
         attr_set[dev] = true;
     }
     CUtensorMap tq, tk, tv, to;
-    if (!make_tmap_bthd(&tq, q, B, T, H) || !make_tmap_bthd(&tk, k, B, T, H) ||
-        !make_tmap_bthd(&tv, v, B, T, H) || !make_tmap_bthd(&to, out ? out : q, B, T, H))
+    if (!make_tmap_bthd(&tq, q, B, T, Hqk) || !make_tmap_bthd(&tk, k, B, T, Hqk) ||
+        !make_tmap_bthd(&tv, v, B, T, H) || !make_tmap_bthd(&to, out ? out : v, B, T, H))
         return -3;
-    tck::chunk_fwd_tc_kernel<<<(unsigned)(Bc * H), tck::kThreads, tck::kSmemBytes, stream>>>(
-        tq, tk, tv, to, log_alpha, beta, d, S0, S_final, T, H, B, out ? 0 : 1, timeout_ns);
+    const int chains = cu_seqlens ? nseq : Bc;
+    const int b_split = cu_seqlens ? nseq : B;
+    auto kern = cu_seqlens ? tck::chunk_fwd_tc_kernel<true> : tck::chunk_fwd_tc_kernel<false>;
+    kern<<<(unsigned)(chains * H), tck::kThreads, tck::kSmemBytes, stream>>>(
+        tq, tk, tv, to, log_alpha, beta, d, S0, S_final, T, H, b_split, out ? 0 : 1, timeout_ns,
+        cu_seqlens, H / Hqk, static_cast<unsigned short*>(out));
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 

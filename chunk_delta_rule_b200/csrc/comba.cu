@@ -88,8 +88,16 @@ int empty_sequence(const ChunkArgs& a, cudaStream_t stream) {
     return e == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
 }
 
+// Packed sequences for launch_simt: cu_seqlens (device, nseq + 1 entries) over the
+// token axis of a single batch; Hqk q / k heads.
+struct Packing {
+    const int* cu_seqlens = nullptr;
+    int nseq = 0;
+    int Hqk = 0;
+};
+
 template <typename Tin>
-int launch_simt(const ChunkArgs& a, cudaStream_t stream) {
+int launch_simt(const ChunkArgs& a, cudaStream_t stream, Packing pk = Packing()) {
     static bool attr_set[kMaxDevices] = {};
     int dev;
     if (int st = current_device(&dev)) return st;
@@ -104,11 +112,11 @@ int launch_simt(const ChunkArgs& a, cudaStream_t stream) {
             return COMBA_ECUDA;
         attr_set[dev] = true;
     }
-    dim3 grid((a.dv + dvt - 1) / dvt, a.H, a.B);
+    dim3 grid((a.dv + dvt - 1) / dvt, a.H, pk.cu_seqlens ? pk.nseq : a.B);
     kern<<<grid, comba::kSimtThreads, smem, stream>>>(
         static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
         a.log_alpha, a.beta, a.d, a.S0, static_cast<Tin*>(a.out), a.S_final, a.T, a.H, a.dk,
-        a.dv, a.chunk, dvt);
+        a.dv, a.chunk, dvt, pk.cu_seqlens, pk.Hqk > 0 ? pk.Hqk : a.H);
     return cudaGetLastError() == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
 }
 
@@ -125,6 +133,46 @@ extern "C" int comba_chunk_fwd(const void* q, const void* k, const void* v,
     if (T == 0) return empty_sequence(a, s);
     if (comba::tc_supported(dk, dv, chunk)) return comba::launch_chunk_tc(a.q, a.k, a.v, a.log_alpha, a.beta, a.d, a.S0, a.out, a.S_final, B, T, H, s);
     return launch_simt<__nv_bfloat16>(a, s);
+}
+
+extern "C" int comba_chunk_fwd_varlen(const void* q, const void* k, const void* v,
+                                      const float* log_alpha, const float* beta, const float* d,
+                                      const float* S0, void* out, float* S_final,
+                                      const int* cu_seqlens, int N, int total_T, int H, int Hqk,
+                                      int dk, int dv, int chunk, comba_stream_t stream) {
+    if (N < 0 || total_T < 0 || H < 0) return COMBA_EINVAL;
+    if (dk < 16 || dk > 128 || dk % 16 || dv < 16 || dv > 128 || dv % 16) return COMBA_EINVAL;
+    if (chunk != 16 && chunk != 32 && chunk != 64) return COMBA_EINVAL;
+    if (N == 0 || H == 0) return COMBA_OK;
+    if (Hqk < 1 || H % Hqk != 0 || !d || !cu_seqlens) return COMBA_EINVAL;
+    if (total_T > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return COMBA_EINVAL;
+    const size_t th = (size_t)total_T * H;
+    if (th > (size_t)1 << 40) return COMBA_EINVAL;
+    const size_t nqk = (size_t)total_T * Hqk * dk * 2, nv = th * dv * 2, ng = th * sizeof(float);
+    const size_t nd = (size_t)H * sizeof(float), ns = (size_t)N * H * dv * dk * sizeof(float);
+    const size_t ncu = ((size_t)N + 1) * sizeof(int);
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(S0, 16) ||
+        !aligned(S_final, 16) || !aligned(log_alpha, 4) || !aligned(beta, 4) || !aligned(d, 4) ||
+        !aligned(cu_seqlens, 4))
+        return COMBA_EINVAL;
+    const void* ins[] = {q, k, v, log_alpha, beta, d, S0, cu_seqlens};
+    const size_t nin[] = {nqk, nqk, nv, ng, ng, nd, ns, ncu};
+    for (int i = 0; i < 8; ++i) {
+        if (overlap(out, nv, ins[i], nin[i])) return COMBA_EINVAL;
+        if (i == 6 && S_final == S0) continue;   // in-place state carry
+        if (overlap(S_final, ns, ins[i], nin[i])) return COMBA_EINVAL;
+    }
+    if (overlap(S_final, ns, out, nv)) return COMBA_EINVAL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // one batch of total_T tokens; the kernels read each chain's bounds from cu_seqlens
+    const ChunkArgs a{q, k, v, log_alpha, beta, d, S0, out, S_final, N, total_T, H, dk, dv, chunk, 2};
+    if (total_T == 0) return empty_sequence(a, s);   // every sequence is empty
+    if (comba::tc_supported(dk, dv, chunk))
+        return comba::launch_chunk_tc(q, k, v, log_alpha, beta, d, S0, out, S_final, 1, total_T, H, s, -1,
+                                      comba::kWaitTimeoutNs, cu_seqlens, N, Hqk);
+    ChunkArgs a1 = a;
+    a1.B = 1;
+    return launch_simt<__nv_bfloat16>(a1, s, Packing{cu_seqlens, N, Hqk});
 }
 
 extern "C" size_t comba_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk) {

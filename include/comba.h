@@ -78,6 +78,35 @@ int comba_chunk_fwd(const void* q, const void* k, const void* v,
                     comba_stream_t stream);
 
 /*
+ * Chunk-wise forward over packed variable-length sequences whose value heads
+ * share q / k heads in groups (the write-up's "mamba form" of the Comba family,
+ * which works like multi-value attention with one shared 128-dim query and key:
+ * end of section "硬件高效的分块并行计算").  Each (sequence, value head) is an
+ * independent chain with the recurrence of comba_chunk_fwd; packing sequences
+ * along one token axis is a layout of that computation (no counterpart in the
+ * write-up).
+ *
+ * Layouts (total_T packed tokens, N sequences):
+ *     q, k [total_T, Hqk, dk]   v, out [total_T, H, dv]   bf16
+ *     log_alpha, beta [total_T, H] fp32     d [H] fp32
+ *     S0, S_final [N, H, dv, dk] fp32 (per sequence and value head)
+ *     cu_seqlens  DEVICE int32 [N + 1]: sequence n covers tokens
+ *                 cu_seqlens[n] .. cu_seqlens[n+1]-1 (nondecreasing, from 0 to total_T)
+ * Value head h reads q / k head h / (H / Hqk); Hqk must divide H (Hqk == H is
+ * the plain per-head layout).  Each sequence is chunked from its own first token;
+ * a zero-length sequence gets S_final = S0 (or zeros).  Shapes as comba_chunk_fwd
+ * (dk == dv == 128 with chunk == 64 runs the tensor-core kernel).  A sequence
+ * whose bounds are malformed (negative, decreasing, or past total_T) is skipped
+ * and COMBA_EINVAL is latched in the device status word (comba_get_last_error);
+ * the host cannot check device-resident bounds.
+ */
+int comba_chunk_fwd_varlen(const void* q, const void* k, const void* v,
+                           const float* log_alpha, const float* beta, const float* d,
+                           const float* S0, void* out, float* S_final,
+                           const int* cu_seqlens, int N, int total_T, int H, int Hqk,
+                           int dk, int dv, int chunk, comba_stream_t stream);
+
+/*
  * Workspace the segmented form of comba_chunk_fwd_ws needs for this shape on the
  * current device, in bytes; 0 when the shape runs unsegmented (enough (b, h)
  * chains to fill the GPU, a T that is not a multiple of 64, or a shape outside the

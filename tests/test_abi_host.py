@@ -124,3 +124,37 @@ def test_binding_refuses_cpu_tensors():
     g = torch.zeros(1, 4, 1)
     with pytest.raises(ValueError):
         cdr.chunk_fwd(x, x, x, g, g, torch.zeros(1))
+
+
+def _varlen_args(**kw):
+    a = dict(q=BASE, k=BASE + GB, v=BASE + 2 * GB, log_alpha=BASE + 3 * GB, beta=BASE + 4 * GB,
+             d=BASE + 5 * GB, S0=BASE + 6 * GB, out=BASE + 7 * GB, S_final=BASE + 8 * GB,
+             cu=BASE + 9 * GB, N=3, total_T=200, H=4, Hqk=2, dk=128, dv=128, chunk=64)
+    a.update(kw)
+    return a
+
+
+def _call_varlen(lib, a):
+    p = lambda x: ctypes.c_void_p(x)
+    return lib.comba_chunk_fwd_varlen(p(a["q"]), p(a["k"]), p(a["v"]), p(a["log_alpha"]),
+                                      p(a["beta"]), p(a["d"]), p(a["S0"]), p(a["out"]),
+                                      p(a["S_final"]), p(a["cu"]), a["N"], a["total_T"], a["H"],
+                                      a["Hqk"], a["dk"], a["dv"], a["chunk"], ctypes.c_void_p(None))
+
+
+@pytest.mark.parametrize("bad", [
+    dict(N=-1), dict(total_T=-1), dict(H=-1), dict(Hqk=0), dict(Hqk=3), dict(Hqk=8),
+    dict(dk=24), dict(chunk=48), dict(cu=None), dict(d=None), dict(q=None), dict(out=None),
+    dict(cu=BASE + 9 * GB + 2),            # misaligned cu_seqlens
+    dict(q=BASE + 8),                      # misaligned q
+    dict(out=BASE + 9 * GB),               # out overlaps cu_seqlens
+    dict(S_final=BASE + 2 * GB + 64),      # S_final overlaps v
+    dict(S_final=BASE + 6 * GB + 16),      # partial overlap with S0
+])
+def test_varlen_rejects_bad_arguments(lib, bad):
+    assert _call_varlen(lib, _varlen_args(**bad)) == -1
+
+
+@pytest.mark.parametrize("empty", [dict(N=0), dict(H=0)])
+def test_varlen_empty_is_noop(lib, empty):
+    assert _call_varlen(lib, _varlen_args(**empty, q=None, k=None, v=None, cu=None)) == 0
