@@ -33,7 +33,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from comba_workloads import (CONFIGS, DECODE, decode_step_inputs, make_chunk_inputs,  # noqa: E402
+from comba_workloads import (CONFIGS, DECODE, VARLEN, make_varlen_inputs,  # noqa: E402
+                             decode_step_inputs, make_chunk_inputs,
                              make_decode_state)
 
 METRIC = "Comba chunk-fwd tokens/s and TFLOP/s on 1 B200, % of roofline"
@@ -373,13 +374,111 @@ def run_decode(args):
     print(json.dumps(line), flush=True)
 
 
+def varlen_counts(cfg, nseq):
+    """Algorithmic FLOPs and bytes of one packed varlen forward: the per-head-token
+    FLOPs of the chunk workloads over every value head; q and k once per q / k head,
+    v and out per value head, two fp32 gates, S0 read and S_final written once per
+    (sequence, value head)."""
+    C, dk, dv, H = cfg.chunk, cfg.dk, cfg.dv, cfg.H
+    flops = cfg.total_T * H * (C * (3 * dk + 2 * dv) + 6 * dk * dv)
+    bytes_ = cfg.total_T * ((2 * cfg.Hqk * dk + 2 * H * dv) * 2 + 8 * H) + nseq * H * dv * dk * 4 * 2
+    return flops, bytes_
+
+
+def run_varlen(args):
+    """One step = one comba_chunk_fwd_varlen over the packed workload (every
+    sequence, every value head), inputs resident in HBM."""
+    import chunk_delta_rule_b200 as cdr
+    cfg = VARLEN
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cdr.library()
+    x = make_varlen_inputs(cfg)
+    N = x["cu_seqlens"].numel() - 1
+    host = {k: v.pin_memory() for k, v in x.items()}
+    d_ = {k: v.to(dev) for k, v in host.items()}
+    out = torch.empty((cfg.total_T, cfg.H, cfg.dv), dtype=torch.bfloat16, device=dev)
+    S_final = torch.empty((N, cfg.H, cfg.dv, cfg.dk), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        cdr.chunk_fwd_varlen(d_["q"], d_["k"], d_["v"], d_["log_alpha"], d_["beta"], d_["d"],
+                             d_["cu_seqlens"], S0=d_["S0"], chunk=cfg.chunk, out=out,
+                             S_final=S_final, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert cdr.get_last_error(dev) == 0
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(0).start()
+    th0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    th1 = time.time()
+    clocks.wait_after(th0)
+    clocks.stop()
+    ms_step = ev0.elapsed_time(ev1) / args.steps
+    if cdr.get_last_error(dev) != 0:
+        raise RuntimeError("device-side error during the timed region")
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    S_h = torch.empty(S_final.shape, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        for k in host:
+            d_[k].copy_(host[k], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        S_h.copy_(S_final, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_e2e = ev0.elapsed_time(ev1) / args.steps
+    flops, bytes_ = varlen_counts(cfg, N)
+    peaks = load_peaks()
+    gbs = bytes_ / (ms_step / 1e3) / 1e9
+    lengths = (x["cu_seqlens"][1:] - x["cu_seqlens"][:-1]).tolist()
+    line = {
+        "metric": "Comba chunk-fwd tokens/s over packed variable-length sequences, % of HBM roofline",
+        "value": cfg.total_T / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "total_T": cfg.total_T, "sequences": N,
+                   "length_min": min(lengths), "length_max": max(lengths), "H": cfg.H, "Hqk": cfg.Hqk,
+                   "dk": cfg.dk, "dv": cfg.dv, "chunk": cfg.chunk,
+                   "l2": "inputs larger than L2 (q,k,v,out %.0f MiB vs 126 MiB L2); no flush"
+                         % (cfg.total_T * (2 * cfg.Hqk * cfg.dk + 2 * cfg.H * cfg.dv) * 2 / 2 ** 20)},
+        "tflops": flops / (ms_step / 1e3) / 1e12,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": peaks["source"] + " hbm_gbs (copy)",
+                     "algorithmic_bytes_per_launch": bytes_, "algorithmic_flops_per_launch": flops},
+        "e2e": {"value": cfg.total_T / (ms_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in host.values()),
+                "d2h_bytes_per_step": out_h.numel() * 2 + S_h.numel() * 4, "ms_per_step": ms_e2e},
+        "clocks": clocks.summary(th0, th1),
+        "gpu_launches": args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="layer1p3b_bf16", choices=sorted(CONFIGS) + [DECODE.name])
+    ap.add_argument("--workload", default="layer1p3b_bf16",
+                    choices=sorted(CONFIGS) + [DECODE.name, VARLEN.name])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -389,6 +488,12 @@ def main():
             print(json.dumps({"impl": "reference", "unavailable": "the decode workload has no reference arm; the headline workload does"}))
             return
         run_decode(args)
+        return
+    if args.workload == VARLEN.name:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the packed varlen workload has no reference arm; the headline workload does"}))
+            return
+        run_varlen(args)
         return
     cfg = CONFIGS[args.workload]
     if args.impl == "reference":

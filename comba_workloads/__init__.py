@@ -38,7 +38,7 @@ import torch
 __all__ = [
     "ChunkConfig", "DecodeConfig", "CONFIGS", "DECODE", "chunk_config",
     "make_chunk_inputs", "make_decode_state", "decode_step_inputs",
-    "head_token_count",
+    "head_token_count", "VarlenConfig", "VARLEN", "varlen_lengths", "make_varlen_inputs",
 ]
 
 
@@ -93,6 +93,69 @@ CONFIGS: Dict[str, ChunkConfig] = {
 
 DECODE = DecodeConfig("decode_b256_h32", B=256, H=32, dk=128, dv=128, steps=512,
                       s0_std=0.02, seed=4)
+
+
+@dataclasses.dataclass(frozen=True)
+class VarlenConfig:
+    """Packed variable-length sequences whose value heads share q / k heads."""
+    name: str
+    total_T: int          # packed tokens per step
+    H: int                # value heads
+    Hqk: int              # q / k heads (divides H)
+    dk: int
+    dv: int
+    chunk: int
+    len_median: float     # sequence lengths: log-normal, clipped to [len_min, len_max]
+    len_sigma: float
+    len_min: int
+    len_max: int
+    s0_std: float
+    seed: int
+
+
+# The 1.3B layer's tokens per step in the mamba form (16 value heads sharing one
+# 128-dim q / k head), as a mix of sequence lengths.
+VARLEN = VarlenConfig("varlen_mamba1p3b_bf16", total_T=32768, H=16, Hqk=1, dk=128, dv=128, chunk=64,
+                      len_median=1024.0, len_sigma=1.0, len_min=64, len_max=8192, s0_std=0.02, seed=5)
+
+
+def varlen_lengths(cfg: VarlenConfig):
+    """Seeded sequence lengths summing to cfg.total_T (the last one trimmed)."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(cfg.seed)
+    lengths, total = [], 0
+    while total < cfg.total_T:
+        z = float(torch.randn((), generator=gen))
+        n = int(round(cfg.len_median * math.exp(cfg.len_sigma * z)))
+        n = max(cfg.len_min, min(cfg.len_max, n))
+        n = min(n, cfg.total_T - total)
+        lengths.append(n)
+        total += n
+    return lengths
+
+
+def make_varlen_inputs(cfg: VarlenConfig) -> Dict[str, torch.Tensor]:
+    """Packed inputs of one varlen workload, CPU tensors: q, k [total_T, Hqk, dk] and
+    v [total_T, H, dv] bf16, log_alpha / beta [total_T, H] and d [H] fp32 (draws of the
+    chunk workloads), S0 [N, H, dv, dk] fp32, cu_seqlens [N+1] int32."""
+    lengths = varlen_lengths(cfg)
+    base = ChunkConfig(cfg.name, B=1, H=cfg.H, T=cfg.total_T, dk=cfg.dk, dv=cfg.dv, chunk=cfg.chunk,
+                       dtype="bf16", decay="mamba", s0_std=0.0, seed=cfg.seed)
+    xv = make_chunk_inputs(base)
+    xq = make_chunk_inputs(base.replace(H=cfg.Hqk), seed=cfg.seed + 1)
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(cfg.seed + 2)
+    N = len(lengths)
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + n)
+    return {
+        "q": xq["q"][0].contiguous(), "k": xq["k"][0].contiguous(), "v": xv["v"][0].contiguous(),
+        "log_alpha": xv["log_alpha"][0].contiguous(), "beta": xv["beta"][0].contiguous(),
+        "d": xv["d"],
+        "S0": (cfg.s0_std * _normal(gen, (N, cfg.H, cfg.dv, cfg.dk))).to(torch.float32).contiguous(),
+        "cu_seqlens": torch.tensor(cu, dtype=torch.int32),
+    }
 
 
 def chunk_config(name: str) -> ChunkConfig:

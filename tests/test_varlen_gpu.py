@@ -128,3 +128,27 @@ def test_malformed_bounds_skip_the_sequence_and_report():
     ro, _ = oracle_packed(y, 2, 2)
     assert_close("out", out[:100].double().cpu().numpy(), ro[:100], TOL_BF16)
     assert bool((out[100:] == 7.0).all())
+
+
+def test_bench_workload_sampled_chains():
+    # The benchmark's packed workload (25 sequences, 16 value heads on one q / k head),
+    # run whole; sampled (sequence, head) chains against the oracle one by one.
+    from comba_workloads import VARLEN, make_varlen_inputs
+    x = make_varlen_inputs(VARLEN)
+    dev = {k: v.cuda() for k, v in x.items()}
+    out, S = cdr.chunk_fwd_varlen(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
+                                  dev["d"], dev["cu_seqlens"], S0=dev["S0"], chunk=VARLEN.chunk)
+    torch.cuda.synchronize()
+    assert cdr.get_last_error() == 0
+    cu = x["cu_seqlens"].tolist()
+    lengths = np.diff(cu)
+    G = VARLEN.H // VARLEN.Hqk
+    for n, h in [(0, 0), (len(lengths) - 1, VARLEN.H - 1), (int(np.argmax(lengths)), 7),
+                 (int(np.argmin(lengths)), 3)]:
+        s0, s1 = cu[n], cu[n + 1]
+        o, Sn = oracle.recurrence(
+            q=x["q"][s0:s1, h // G][None, :, None], k=x["k"][s0:s1, h // G][None, :, None],
+            v=x["v"][s0:s1, h][None, :, None], log_alpha=x["log_alpha"][s0:s1, h][None, :, None],
+            beta=x["beta"][s0:s1, h][None, :, None], d=x["d"][h:h + 1], S0=x["S0"][n:n + 1, h:h + 1])
+        assert_close(f"out seq {n} head {h}", out[s0:s1, h].double().cpu().numpy(), o[0, :, 0], TOL_BF16)
+        assert_close(f"S_final seq {n} head {h}", S[n, h].double().cpu().numpy(), Sn[0, 0], TOL_BF16)
