@@ -849,6 +849,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                   make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]));
                 tc::tc_fence_before();
                 tc::named_barrier_arrive(BAR_KK, kKKThreads);
+                COMBA_PHASE(27);
                 // A_rs = beta_r e^{g_{r-1} - g_s} (K K^T)_rs for s < r -> -A into F2
                 if (fast) {
                     const float cr = tc::lds_f32(ts + 768 + 4u * r);
@@ -860,6 +861,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         for (int e = 0; e < 4; ++e)
                             a[4 * c + e] = (32 * ch + 4 * c + e < r) ? cr * iv[e] * a[4 * c + e] : 0.f;
                     }
+                    COMBA_PHASE(28);
                     store_neg_a(F2p, r, ch, a);
                 } else {
                     a_rows_exact(F2p, tl + tgm + 32 * ch, r, ch, ts);
