@@ -774,7 +774,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         //   pw 1, 2, 6: Q K^T of the same row/column blocks: P, once K K^T is staged
         //   pw 5:       P rows 0-31 x cols 32-63 are zero (s > r)
         //   pw 5, 0:    the next chunk's gate tables (tokens 0-31, 32-63)
-        // then one 8-column strip of Tinv per warp (pw 6: strips 6 and 7), written out
+        // then one 8-column strip of Tinv per warp (pw 4: strips 6 and 7), written out
         // as Tc / Eb, and diag(lo(beta)) (pw 4, 5).
         const int pt = tid - kPrepBase;
         const int pw = pt >> 5, q = warp & 3;
@@ -930,8 +930,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             __syncwarp();
             COMBA_PHASE(11);
             if (ok) {
-                strip_inverse(F2p, F1, pw, lane, ts + 768, ts + 512);
-                if (pw == 6) strip_inverse(F2p, F1, 7, lane, ts + 768, ts + 512);
+                // the two longest strips (0, 1) on warps of schedulers 0 and 1 (warp % 4),
+                // the others spread so that each scheduler carries a similar MMA load
+                const int strip = (pw == 3) ? 0 : (pw == 0) ? 1 : (pw <= 2) ? pw + 1 : (pw == 4) ? 6 : pw - 1;
+                strip_inverse(F2p, F1, strip, lane, ts + 768, ts + 512);
+                if (pw == 4) strip_inverse(F2p, F1, 7, lane, ts + 768, ts + 512);
             }
             COMBA_PHASE(19);
             if (pt >= 128 && pt < 192) {   // diag(lo(beta))
