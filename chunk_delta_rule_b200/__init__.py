@@ -30,7 +30,8 @@ _lock = threading.Lock()
 
 EXPORTS = ("comba_chunk_fwd", "comba_chunk_fwd_f32", "comba_chunk_fwd_varlen",
            "comba_chunk_fwd_workspace_size", "comba_chunk_fwd_ws", "comba_chunk_fwd_noalloc",
-           "comba_recurrent_step", "comba_get_last_error", "comba_status_string", "comba_version")
+           "comba_recurrent_step", "comba_recurrent_step_grouped", "comba_get_last_error",
+           "comba_status_string", "comba_version")
 
 
 class CombaError(RuntimeError):
@@ -62,8 +63,10 @@ def library():
             lib.comba_chunk_fwd_workspace_size.restype = ctypes.c_size_t
             lib.comba_chunk_fwd_varlen.argtypes = [vp] * 10 + [i] * 7 + [vp]
             lib.comba_recurrent_step.argtypes = [vp] * 8 + [i] * 4 + [vp]
+            lib.comba_recurrent_step_grouped.argtypes = [vp] * 8 + [i] * 5 + [vp]
             for fn in (lib.comba_chunk_fwd, lib.comba_chunk_fwd_f32, lib.comba_chunk_fwd_ws,
                        lib.comba_chunk_fwd_noalloc, lib.comba_chunk_fwd_varlen,
+                       lib.comba_recurrent_step_grouped,
                        lib.comba_recurrent_step, lib.comba_get_last_error, lib.comba_version):
                 fn.restype = ctypes.c_int
             lib.comba_get_last_error.argtypes = []
@@ -229,14 +232,16 @@ def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alp
 def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
                    beta: torch.Tensor, d: torch.Tensor, S: torch.Tensor,
                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """One decode token: q, k [B,H,dk] bf16, v [B,H,dv] bf16, log_alpha, beta [B,H]
-    fp32, d [H] fp32, S [B,H,dv,dk] fp32 updated in place.  Returns out [B,H,dv] bf16."""
-    if q.dim() != 3:
-        raise ValueError("q must be [B, H, dk]")
-    B, H, dk = q.shape
-    dv = v.shape[-1]
-    _check(q, "q", torch.bfloat16, (B, H, dk))
-    _check(k, "k", torch.bfloat16, (B, H, dk))
+    """One decode token: q, k [B,Hqk,dk] bf16, v [B,H,dv] bf16 with Hqk dividing H
+    (Hqk == H: one q / k head per value head; otherwise value head h reads q / k head
+    h // (H // Hqk)), log_alpha, beta [B,H] fp32, d [H] fp32, S [B,H,dv,dk] fp32
+    updated in place.  Returns out [B,H,dv] bf16."""
+    if q.dim() != 3 or v.dim() != 3:
+        raise ValueError("q must be [B, Hqk, dk] and v [B, H, dv]")
+    B, Hqk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
+    _check(q, "q", torch.bfloat16, (B, Hqk, dk))
+    _check(k, "k", torch.bfloat16, (B, Hqk, dk))
     _check(v, "v", torch.bfloat16, (B, H, dv))
     _check(log_alpha, "log_alpha", torch.float32, (B, H))
     _check(beta, "beta", torch.float32, (B, H))
@@ -247,11 +252,11 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha:
         out = torch.empty((B, H, dv), dtype=torch.bfloat16, device=dev)
     _check(out, "out", torch.bfloat16, (B, H, dv))
     with torch.cuda.device(dev):
-        st = library().comba_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
-                                            _ptr(beta), _ptr(d), _ptr(S), _ptr(out), B, H, dk,
-                                            dv, _stream_handle(dev, stream))
+        st = library().comba_recurrent_step_grouped(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                                    _ptr(beta), _ptr(d), _ptr(S), _ptr(out), B, H, Hqk,
+                                                    dk, dv, _stream_handle(dev, stream))
     if st != 0:
-        raise CombaError(st, "comba_recurrent_step")
+        raise CombaError(st, "comba_recurrent_step_grouped")
     return out
 
 

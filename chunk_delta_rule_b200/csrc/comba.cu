@@ -237,11 +237,12 @@ extern "C" int comba_chunk_fwd_f32(const float* q, const float* k, const float* 
     return launch_simt<float>(a, s);
 }
 
-extern "C" int comba_recurrent_step(const void* q, const void* k, const void* v,
-                                    const float* log_alpha, const float* beta, const float* d,
-                                    float* S, void* out, int B, int H, int dk, int dv,
-                                    comba_stream_t stream) {
+extern "C" int comba_recurrent_step_grouped(const void* q, const void* k, const void* v,
+                                            const float* log_alpha, const float* beta, const float* d,
+                                            float* S, void* out, int B, int H, int Hqk, int dk, int dv,
+                                            comba_stream_t stream) {
     if (B < 0 || H < 0) return COMBA_EINVAL;
+    if (H > 0 && (Hqk < 1 || H % Hqk != 0)) return COMBA_EINVAL;
     if (dk != 32 && dk != 64 && dk != 128) return COMBA_EINVAL;
     if (dv < 16 || dv > 128 || dv % 16) return COMBA_EINVAL;
     if (B == 0 || H == 0) return COMBA_OK;
@@ -251,7 +252,7 @@ extern "C" int comba_recurrent_step(const void* q, const void* k, const void* v,
         return COMBA_EINVAL;
     const size_t bh = (size_t)B * H;
     if (bh > (size_t)1 << 31) return COMBA_EINVAL;
-    const size_t nqk = bh * dk * 2, nv = bh * dv * 2, ng = bh * 4, ns = bh * dv * dk * 4;
+    const size_t nqk = (size_t)B * Hqk * dk * 2, nv = bh * dv * 2, ng = bh * 4, ns = bh * dv * dk * 4;
     const void* ins[] = {q, k, v, log_alpha, beta, d};
     const size_t nin[] = {nqk, nqk, nv, ng, ng, (size_t)H * 4};
     for (int i = 0; i < 6; ++i)
@@ -265,16 +266,23 @@ extern "C" int comba_recurrent_step(const void* q, const void* k, const void* v,
     const unsigned grid = (unsigned)bh;
     switch (dk) {
         case 32:
-            comba::recurrent_step_kernel<32><<<grid, comba::kStepThreads, 0, s>>>(qb, kb, vb, log_alpha, beta, d, S, ob, H, dv);
+            comba::recurrent_step_kernel<32><<<grid, comba::kStepThreads, 0, s>>>(qb, kb, vb, log_alpha, beta, d, S, ob, H, dv, Hqk);
             break;
         case 64:
-            comba::recurrent_step_kernel<64><<<grid, comba::kStepThreads, 0, s>>>(qb, kb, vb, log_alpha, beta, d, S, ob, H, dv);
+            comba::recurrent_step_kernel<64><<<grid, comba::kStepThreads, 0, s>>>(qb, kb, vb, log_alpha, beta, d, S, ob, H, dv, Hqk);
             break;
         default:
-            comba::recurrent_step_kernel<128><<<grid, comba::kStepThreads, 0, s>>>(qb, kb, vb, log_alpha, beta, d, S, ob, H, dv);
+            comba::recurrent_step_kernel<128><<<grid, comba::kStepThreads, 0, s>>>(qb, kb, vb, log_alpha, beta, d, S, ob, H, dv, Hqk);
             break;
     }
     return cudaGetLastError() == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
+}
+
+extern "C" int comba_recurrent_step(const void* q, const void* k, const void* v,
+                                    const float* log_alpha, const float* beta, const float* d,
+                                    float* S, void* out, int B, int H, int dk, int dv,
+                                    comba_stream_t stream) {
+    return comba_recurrent_step_grouped(q, k, v, log_alpha, beta, d, S, out, B, H, H, dk, dv, stream);
 }
 
 extern "C" int comba_get_last_error(void) {

@@ -54,11 +54,13 @@ __global__ void __launch_bounds__(kStepThreads)
 recurrent_step_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                       const __nv_bfloat16* __restrict__ v, const float* __restrict__ log_alpha,
                       const float* __restrict__ beta, const float* __restrict__ dvec,
-                      float* __restrict__ S, __nv_bfloat16* __restrict__ out, int H, int dv) {
+                      float* __restrict__ S, __nv_bfloat16* __restrict__ out, int H, int dv, int Hqk) {
     constexpr int PER = DK / 32;
     __shared__ float o_s[128];
     const int bh = blockIdx.x;
     const int h = bh % H;
+    // q / k of value head h: head h / (H / Hqk) of the batch row's Hqk heads
+    const size_t qk = ((size_t)(bh / H) * Hqk + h / (H / Hqk)) * DK;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     constexpr int nwarps = kStepThreads / 32;
 
@@ -68,8 +70,8 @@ recurrent_step_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
     float kr[PER], qt[PER];
 #pragma unroll
     for (int p = 0; p < PER; ++p) {
-        kr[p] = __bfloat162float(k[(size_t)bh * DK + lane * PER + p]);
-        qt[p] = __bfloat162float(q[(size_t)bh * DK + lane * PER + p]) - dh * kr[p];
+        kr[p] = __bfloat162float(k[qk + lane * PER + p]);
+        qt[p] = __bfloat162float(q[qk + lane * PER + p]) - dh * kr[p];
     }
     float* Sb = S + (size_t)bh * dv * DK + lane * PER;
     const __nv_bfloat16* vb = v + (size_t)bh * dv;

@@ -174,6 +174,17 @@ int comba_recurrent_step(const void* q, const void* k, const void* v,
                          comba_stream_t stream);
 
 /*
+ * The decode step of the mamba form (value heads sharing q / k heads in groups,
+ * as in comba_chunk_fwd_varlen): comba_recurrent_step with q, k [B, Hqk, dk];
+ * value head h reads q / k head h / (H / Hqk).  Hqk must divide H; Hqk == H is
+ * comba_recurrent_step itself.
+ */
+int comba_recurrent_step_grouped(const void* q, const void* k, const void* v,
+                                 const float* log_alpha, const float* beta, const float* d,
+                                 float* S, void* out, int B, int H, int Hqk, int dk, int dv,
+                                 comba_stream_t stream);
+
+/*
  * Reads and clears the current device's status word (synchronises the
  * device first).  Returns COMBA_OK, COMBA_ETIMEOUT, COMBA_EDEVICE, or
  * COMBA_ECUDA if the synchronisation or the read itself failed.

@@ -158,3 +158,20 @@ def test_varlen_rejects_bad_arguments(lib, bad):
 @pytest.mark.parametrize("empty", [dict(N=0), dict(H=0)])
 def test_varlen_empty_is_noop(lib, empty):
     assert _call_varlen(lib, _varlen_args(**empty, q=None, k=None, v=None, cu=None)) == 0
+
+
+def _call_step_grouped(lib, a, Hqk):
+    p = lambda x: ctypes.c_void_p(x)
+    return lib.comba_recurrent_step_grouped(p(a["q"]), p(a["k"]), p(a["v"]), p(a["log_alpha"]),
+                                            p(a["beta"]), p(a["d"]), p(a["S"]), p(a["out"]), a["B"],
+                                            a["H"], Hqk, a["dk"], a["dv"], ctypes.c_void_p(None))
+
+
+@pytest.mark.parametrize("Hqk", [0, -1, 3, 4])
+def test_grouped_step_rejects_bad_head_counts(lib, Hqk):
+    # H = 2: Hqk must be 1 or 2
+    assert _call_step_grouped(lib, _step_args(), Hqk) == -1
+
+
+def test_grouped_step_empty_is_noop(lib):
+    assert _call_step_grouped(lib, _step_args(B=0), 1) == 0

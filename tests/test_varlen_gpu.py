@@ -152,3 +152,57 @@ def test_bench_workload_sampled_chains():
             beta=x["beta"][s0:s1, h][None, :, None], d=x["d"][h:h + 1], S0=x["S0"][n:n + 1, h:h + 1])
         assert_close(f"out seq {n} head {h}", out[s0:s1, h].double().cpu().numpy(), o[0, :, 0], TOL_BF16)
         assert_close(f"S_final seq {n} head {h}", S[n, h].double().cpu().numpy(), Sn[0, 0], TOL_BF16)
+
+
+def test_mamba_form_prefill_then_grouped_decode():
+    # Packed prefill of 3 sequences (4 value heads on one q / k head), then 5 decode
+    # steps per sequence from its final state with the grouped step; the oracle runs
+    # each sequence's prefill and decode tokens as one chain.
+    lengths, H, Hqk, D, steps = [100, 37, 64], 4, 1, 128, 5
+    x = packed_inputs(lengths, H, Hqk, D, D, seed=2024)
+    _, S = run_varlen(x, 64)
+    g = torch.Generator().manual_seed(99)
+    N = len(lengths)
+    dec = []
+    for _ in range(steps):
+        qk = torch.nn.functional.normalize(torch.randn(2, N, Hqk, D, generator=g), dim=-1).bfloat16()
+        dec.append({"q": qk[0], "k": qk[1], "v": torch.randn(N, H, D, generator=g).bfloat16(),
+                    "log_alpha": -0.05 * torch.rand(N, H, generator=g),
+                    "beta": torch.rand(N, H, generator=g)})
+    d = x["d"].cuda()
+    outs = []
+    for t in range(steps):
+        xd = {k: v.cuda() for k, v in dec[t].items()}
+        outs.append(cdr.recurrent_step(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], d, S))
+    torch.cuda.synchronize()
+    assert cdr.get_last_error() == 0
+    cu = x["cu"].tolist()
+    heads = np.arange(H) // (H // Hqk)
+    for n in range(N):
+        s0, s1 = cu[n], cu[n + 1]
+        cat = lambda pre, key: torch.cat([pre[s0:s1]] + [dec[t][key][n:n + 1] for t in range(steps)])
+        qn, kn = cat(x["q"], "q")[:, heads], cat(x["k"], "k")[:, heads]
+        o, Sn = oracle.recurrence(q=qn[None], k=kn[None], v=cat(x["v"], "v")[None],
+                                  log_alpha=cat(x["log_alpha"], "log_alpha")[None],
+                                  beta=cat(x["beta"], "beta")[None], d=x["d"], S0=x["S0"][n:n + 1])
+        got = torch.stack([outs[t][n] for t in range(steps)]).double().cpu().numpy()
+        assert_close(f"decode out seq {n}", got, o[0, s1 - s0:], TOL_BF16)
+        assert_close(f"state seq {n}", S[n].double().cpu().numpy(), Sn[0], TOL_BF16)
+
+
+def test_grouped_decode_equals_the_step_on_expanded_heads():
+    g = torch.Generator().manual_seed(5)
+    B, H, Hqk, D = 3, 8, 2, 128
+    q = torch.nn.functional.normalize(torch.randn(B, Hqk, D, generator=g), dim=-1).bfloat16().cuda()
+    k = torch.nn.functional.normalize(torch.randn(B, Hqk, D, generator=g), dim=-1).bfloat16().cuda()
+    v = torch.randn(B, H, D, generator=g).bfloat16().cuda()
+    la = (-0.1 * torch.rand(B, H, generator=g)).cuda()
+    be = torch.rand(B, H, generator=g).cuda()
+    d = torch.rand(H, generator=g).cuda()
+    S0 = (0.05 * torch.randn(B, H, D, D, generator=g)).cuda()
+    S1, S2 = S0.clone(), S0.clone()
+    o1 = cdr.recurrent_step(q, k, v, la, be, d, S1)
+    rep = lambda t: t.repeat_interleave(H // Hqk, dim=1).contiguous()
+    o2 = cdr.recurrent_step(rep(q), rep(k), v, la, be, d, S2)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
