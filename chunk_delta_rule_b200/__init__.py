@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["chunk_fwd", "chunk_fwd_varlen", "chunk_fwd_noalloc", "recurrent_step",
+__all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_varlen", "chunk_fwd_noalloc", "recurrent_step",
            "get_last_error", "CombaError", "library", "library_path", "EXPORTS", "status_string"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -30,6 +30,7 @@ _lock = threading.Lock()
 
 EXPORTS = ("comba_chunk_fwd", "comba_chunk_fwd_f32", "comba_chunk_fwd_varlen",
            "comba_chunk_fwd_workspace_size", "comba_chunk_fwd_ws", "comba_chunk_fwd_noalloc",
+           "comba_chunk_fwd_host", "comba_chunk_fwd_host_workspace_size",
            "comba_recurrent_step", "comba_recurrent_step_grouped", "comba_get_last_error",
            "comba_status_string", "comba_version")
 
@@ -62,11 +63,14 @@ def library():
             lib.comba_chunk_fwd_workspace_size.argtypes = [i] * 6
             lib.comba_chunk_fwd_workspace_size.restype = ctypes.c_size_t
             lib.comba_chunk_fwd_varlen.argtypes = [vp] * 10 + [i] * 7 + [vp]
+            lib.comba_chunk_fwd_host.argtypes = [vp] * 9 + [i] * 6 + [vp, ctypes.c_size_t, i, vp]
+            lib.comba_chunk_fwd_host_workspace_size.argtypes = [i] * 5
+            lib.comba_chunk_fwd_host_workspace_size.restype = ctypes.c_size_t
             lib.comba_recurrent_step.argtypes = [vp] * 8 + [i] * 4 + [vp]
             lib.comba_recurrent_step_grouped.argtypes = [vp] * 8 + [i] * 5 + [vp]
             for fn in (lib.comba_chunk_fwd, lib.comba_chunk_fwd_f32, lib.comba_chunk_fwd_ws,
                        lib.comba_chunk_fwd_noalloc, lib.comba_chunk_fwd_varlen,
-                       lib.comba_recurrent_step_grouped,
+                       lib.comba_recurrent_step_grouped, lib.comba_chunk_fwd_host,
                        lib.comba_recurrent_step, lib.comba_get_last_error, lib.comba_version):
                 fn.restype = ctypes.c_int
             lib.comba_get_last_error.argtypes = []
@@ -156,6 +160,66 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
             name = "comba_chunk_fwd_f32"
     if st != 0:
         raise CombaError(st, name)
+    return out, S_final
+
+
+_host_ws = {}
+
+
+def chunk_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                   beta: torch.Tensor, d: torch.Tensor, S0: Optional[torch.Tensor] = None,
+                   chunk: int = 64, out: Optional[torch.Tensor] = None,
+                   S_final: Optional[torch.Tensor] = None, return_state: bool = True,
+                   slices: int = 8, device=None, stream=None,
+                   workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """comba_chunk_fwd_host: bf16 HOST tensors in (pin them for overlap), host
+    results out, the device work and both copy directions pipelined over `slices`
+    groups of batch rows.  Layouts as chunk_fwd.  The device workspace comes from
+    PyTorch's allocator (kept per device for later calls) unless given.  The call
+    returns once the work is enqueued: keep every host tensor alive, and do not
+    write the inputs or read the results, until ``stream`` (default: the current
+    stream of ``device``) has passed the call."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+
+    def host(t, name, dtype, shape):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+            raise ValueError(f"{name} must be a CPU tensor")
+        if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+
+    for t, name in ((q, "q"), (k, "k")):
+        host(t, name, torch.bfloat16, (B, T, H, dk))
+    host(v, "v", torch.bfloat16, (B, T, H, dv))
+    host(log_alpha, "log_alpha", torch.float32, (B, T, H))
+    host(beta, "beta", torch.float32, (B, T, H))
+    host(d, "d", torch.float32, (H,))
+    if S0 is not None:
+        host(S0, "S0", torch.float32, (B, H, dv, dk))
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=torch.bfloat16, pin_memory=True)
+    host(out, "out", torch.bfloat16, (B, T, H, dv))
+    if S_final is None and return_state:
+        S_final = torch.empty((B, H, dv, dk), dtype=torch.float32, pin_memory=True)
+    if S_final is not None:
+        host(S_final, "S_final", torch.float32, (B, H, dv, dk))
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    lib = library()
+    nbytes = lib.comba_chunk_fwd_host_workspace_size(B, T, H, dk, dv)
+    if workspace is None and nbytes:
+        ws = _host_ws.get(dev)
+        if ws is None or ws.numel() < nbytes:
+            ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+            _host_ws[dev] = ws
+        workspace = ws
+    with torch.cuda.device(dev):
+        st = lib.comba_chunk_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(d),
+                                      _ptr(S0), _ptr(out), _ptr(S_final), B, T, H, dk, dv, int(chunk),
+                                      _ptr(workspace), nbytes, int(slices), _stream_handle(dev, stream))
+    if st != 0:
+        raise CombaError(st, "comba_chunk_fwd_host")
     return out, S_final
 
 

@@ -11,6 +11,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cstring>
 
 #include "common.cuh"
 #include "chunk_simt.cuh"
@@ -235,6 +236,141 @@ extern "C" int comba_chunk_fwd_f32(const float* q, const float* k, const float* 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (T == 0) return empty_sequence(a, s);
     return launch_simt<float>(a, s);
+}
+
+// ---------------------------------------------------------------- host buffers
+namespace {
+
+size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+// Device regions of comba_chunk_fwd_host's workspace, in order.
+struct HostLayout {
+    size_t q, k, v, la, be, d, s0, out, sf, total;
+};
+
+HostLayout host_layout(int B, int T, int H, int dk, int dv) {
+    const size_t bth = (size_t)B * T * H, ns = (size_t)B * H * dv * dk * sizeof(float);
+    HostLayout L{};
+    size_t o = 0;
+    auto take = [&](size_t n) { const size_t at = o; o += round256(n); return at; };
+    L.q = take(bth * dk * 2);
+    L.k = take(bth * dk * 2);
+    L.v = take(bth * dv * 2);
+    L.la = take(bth * sizeof(float));
+    L.be = take(bth * sizeof(float));
+    L.d = take((size_t)H * sizeof(float));
+    L.s0 = take(ns);
+    L.out = take(bth * dv * 2);
+    L.sf = take(ns);
+    L.total = o;
+    return L;
+}
+
+// Copy streams of one device, created on first use and kept for the process.
+bool copy_streams(int dev, cudaStream_t* h2d, cudaStream_t* d2h) {
+    static cudaStream_t s[kMaxDevices][2] = {};
+    if (!s[dev][0]) {
+        if (cudaStreamCreateWithFlags(&s[dev][0], cudaStreamNonBlocking) != cudaSuccess) return false;
+        if (cudaStreamCreateWithFlags(&s[dev][1], cudaStreamNonBlocking) != cudaSuccess) return false;
+    }
+    *h2d = s[dev][0];
+    *d2h = s[dev][1];
+    return true;
+}
+
+}  // namespace
+
+extern "C" size_t comba_chunk_fwd_host_workspace_size(int B, int T, int H, int dk, int dv) {
+    if (B <= 0 || T <= 0 || H <= 0 || dk <= 0 || dv <= 0) return 0;
+    return host_layout(B, T, H, dk, dv).total;
+}
+
+extern "C" int comba_chunk_fwd_host(const void* q, const void* k, const void* v,
+                                    const float* log_alpha, const float* beta, const float* d,
+                                    const float* S0, void* out, float* S_final, int B, int T, int H,
+                                    int dk, int dv, int chunk, void* workspace, size_t workspace_bytes,
+                                    int slices, comba_stream_t stream) {
+    const ChunkArgs h{q, k, v, log_alpha, beta, d, S0, out, S_final, B, T, H, dk, dv, chunk, 2};
+    if (int st = validate_chunk(h)) return st;
+    if (B == 0 || H == 0) return COMBA_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t ns = (size_t)B * H * dv * dk * sizeof(float);
+    if (T == 0) {   // the final state is the initial one (or zero)
+        if (!S_final) return COMBA_OK;
+        if (S0) return cudaMemcpyAsync(S_final, S0, ns, cudaMemcpyHostToHost, s) == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return COMBA_ECUDA;
+        memset(S_final, 0, ns);
+        return COMBA_OK;
+    }
+    const HostLayout L = host_layout(B, T, H, dk, dv);
+    if (!workspace || workspace_bytes < L.total || !aligned(workspace, 256)) return COMBA_EINVAL;
+    if (slices < 1) return COMBA_EINVAL;
+    int dev;
+    if (int st = current_device(&dev)) return st;
+    cudaStream_t sh, sd;
+    if (!copy_streams(dev, &sh, &sd)) return COMBA_ECUDA;
+    char* w = static_cast<char*>(workspace);
+    const int P = slices < B ? slices : B;
+    // events: start, per slice in / out, done
+    cudaEvent_t ev[2 * 64 + 2];
+    const int nev = 2 * (P < 64 ? P : 64) + 2;
+    for (int i = 0; i < nev; ++i)
+        if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) {
+            for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
+            return COMBA_ECUDA;
+        }
+    int st = COMBA_OK;
+    auto ok = [&](cudaError_t e) { if (e != cudaSuccess && st == COMBA_OK) st = COMBA_ECUDA; };
+    // the copies start behind everything already on the caller's stream (an earlier
+    // call may still be reading this workspace)
+    ok(cudaEventRecord(ev[0], s));
+    ok(cudaStreamWaitEvent(sh, ev[0], 0));
+    ok(cudaMemcpyAsync(w + L.d, d, (size_t)H * sizeof(float), cudaMemcpyHostToDevice, sh));
+    const int Pn = nev / 2 - 1;   // slices actually used (at most 64)
+    const size_t th = (size_t)T * H;
+    for (int p = 0; p < Pn && st == COMBA_OK; ++p) {
+        const int b0 = (int)((long)B * p / Pn), b1 = (int)((long)B * (p + 1) / Pn), nb = b1 - b0;
+        if (nb == 0) continue;
+        auto h2d = [&](size_t at, const void* src, size_t per_b) {
+            ok(cudaMemcpyAsync(w + at + b0 * per_b, static_cast<const char*>(src) + b0 * per_b, nb * per_b,
+                               cudaMemcpyHostToDevice, sh));
+        };
+        h2d(L.q, q, th * dk * 2);
+        h2d(L.k, k, th * dk * 2);
+        h2d(L.v, v, th * dv * 2);
+        h2d(L.la, log_alpha, th * sizeof(float));
+        h2d(L.be, beta, th * sizeof(float));
+        const size_t sb = (size_t)H * dv * dk * sizeof(float);
+        if (S0) h2d(L.s0, S0, sb);
+        ok(cudaEventRecord(ev[1 + 2 * p], sh));
+        ok(cudaStreamWaitEvent(s, ev[1 + 2 * p], 0));
+        const ChunkArgs a{w + L.q + b0 * th * dk * 2, w + L.k + b0 * th * dk * 2, w + L.v + b0 * th * dv * 2,
+                          reinterpret_cast<const float*>(w + L.la + b0 * th * 4),
+                          reinterpret_cast<const float*>(w + L.be + b0 * th * 4),
+                          reinterpret_cast<const float*>(w + L.d),
+                          S0 ? reinterpret_cast<const float*>(w + L.s0 + b0 * sb) : nullptr,
+                          w + L.out + b0 * th * dv * 2,
+                          S_final ? reinterpret_cast<float*>(w + L.sf + b0 * sb) : nullptr,
+                          nb, T, H, dk, dv, chunk, 2};
+        int lst;
+        if (comba::tc_supported(dk, dv, chunk))
+            lst = comba::launch_chunk_tc(a.q, a.k, a.v, a.log_alpha, a.beta, a.d, a.S0, a.out, a.S_final, nb, T, H, s);
+        else
+            lst = launch_simt<__nv_bfloat16>(a, s);
+        if (lst != 0 && st == COMBA_OK) st = lst;
+        ok(cudaEventRecord(ev[2 + 2 * p], s));
+        ok(cudaStreamWaitEvent(sd, ev[2 + 2 * p], 0));
+        ok(cudaMemcpyAsync(static_cast<char*>(out) + b0 * th * dv * 2, w + L.out + b0 * th * dv * 2,
+                           nb * th * dv * 2, cudaMemcpyDeviceToHost, sd));
+        if (S_final)
+            ok(cudaMemcpyAsync(reinterpret_cast<char*>(S_final) + b0 * sb, w + L.sf + b0 * sb, nb * sb,
+                               cudaMemcpyDeviceToHost, sd));
+    }
+    // the caller's stream completes once the results are in host memory
+    ok(cudaEventRecord(ev[nev - 1], sd));
+    ok(cudaStreamWaitEvent(s, ev[nev - 1], 0));
+    for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
+    return st;
 }
 
 extern "C" int comba_recurrent_step_grouped(const void* q, const void* k, const void* v,

@@ -148,6 +148,34 @@ int comba_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
                             comba_stream_t stream);
 
 /*
+ * comba_chunk_fwd from and to HOST memory: the same computation, with the inputs
+ * copied to the device and the results back inside the call, pipelined over
+ * `slices` groups of batch rows so that the copies in, the kernel and the copies
+ * out of different groups overlap (no counterpart in the write-up).
+ *
+ * q, k, v, log_alpha, beta, d, S0, out, S_final: HOST pointers with the layouts,
+ * alignment and aliasing rules of comba_chunk_fwd (pinned memory lets the copies
+ * run asynchronously and overlap; pageable memory works but serialises).  They
+ * stay owned by the caller, who keeps them valid, the inputs unchanged and the
+ * outputs unread until `stream` has passed this call.
+ * workspace: DEVICE memory, 256-byte aligned, at least
+ * comba_chunk_fwd_host_workspace_size(B, T, H, dk, dv) bytes, owned by the caller
+ * and not to be used by anything else until `stream` has passed this call.  The
+ * copies run on two library-owned streams per device (created on first use and
+ * kept for the process) ordered after the work already on `stream`; `stream`
+ * itself completes only once out and S_final are in host memory.  slices >= 1
+ * (more slices than batch rows act as one per row; at most 64).  T == 0 with
+ * S0 == NULL zeroes S_final after synchronising `stream`.
+ */
+size_t comba_chunk_fwd_host_workspace_size(int B, int T, int H, int dk, int dv);
+int comba_chunk_fwd_host(const void* q, const void* k, const void* v,
+                         const float* log_alpha, const float* beta, const float* d,
+                         const float* S0, void* out, float* S_final,
+                         int B, int T, int H, int dk, int dv, int chunk,
+                         void* workspace, size_t workspace_bytes, int slices,
+                         comba_stream_t stream);
+
+/*
  * Chunk-wise forward with fp32 q, k, v and out (same math, same layouts, same
  * size rules as comba_chunk_fwd); every product is an fp32 FMA, no reduced-
  * precision tensor-core arithmetic.

@@ -175,3 +175,26 @@ def test_grouped_step_rejects_bad_head_counts(lib, Hqk):
 
 def test_grouped_step_empty_is_noop(lib):
     assert _call_step_grouped(lib, _step_args(B=0), 1) == 0
+
+
+def _call_host(lib, a, ws, ws_bytes, slices):
+    p = lambda x: ctypes.c_void_p(x)
+    return lib.comba_chunk_fwd_host(p(a["q"]), p(a["k"]), p(a["v"]), p(a["log_alpha"]), p(a["beta"]),
+                                    p(a["d"]), p(a["S0"]), p(a["out"]), p(a["S_final"]), a["B"], a["T"],
+                                    a["H"], a["dk"], a["dv"], a["chunk"], p(ws), ws_bytes, slices,
+                                    ctypes.c_void_p(None))
+
+
+def test_host_entry_workspace_size_and_rejections(lib):
+    a = _chunk_args()
+    need = lib.comba_chunk_fwd_host_workspace_size(a["B"], a["T"], a["H"], a["dk"], a["dv"])
+    bth = a["B"] * a["T"] * a["H"]
+    assert need >= bth * (2 * a["dk"] + 2 * a["dv"]) * 2 + 2 * bth * 4 + 2 * a["B"] * a["H"] * a["dk"] * a["dv"] * 4
+    assert lib.comba_chunk_fwd_host_workspace_size(0, 8, 2, 64, 64) == 0
+    ws = BASE + 20 * GB
+    assert _call_host(lib, a, ws, need - 1, 4) == -1          # workspace too small
+    assert _call_host(lib, a, ws + 128, need, 4) == -1        # workspace misaligned
+    assert _call_host(lib, a, None, need, 4) == -1            # no workspace
+    assert _call_host(lib, a, ws, need, 0) == -1              # no slices
+    assert _call_host(lib, _chunk_args(dk=24), ws, need, 4) == -1
+    assert _call_host(lib, _chunk_args(out=BASE + 16), ws, need, 4) == -1   # out overlaps q
