@@ -79,3 +79,19 @@ def test_reference_arm_other_ranks_exit_quietly():
                           "--workload", "tiny_fp32", "--steps", "1", "--warmup", "3"],
                          capture_output=True, text=True, env=env, timeout=600, check=True)
     assert out.stdout.strip() == ""
+
+
+def test_varlen_workload_is_seeded_and_covers_its_tokens():
+    from comba_workloads import VARLEN, make_varlen_inputs, varlen_lengths
+    a, b = varlen_lengths(VARLEN), varlen_lengths(VARLEN)
+    assert a == b and sum(a) == VARLEN.total_T
+    assert all(n >= 1 for n in a) and max(a) <= VARLEN.len_max
+    x = make_varlen_inputs(VARLEN)
+    cu = x["cu_seqlens"].tolist()
+    assert cu[0] == 0 and cu[-1] == VARLEN.total_T and len(cu) == len(a) + 1
+    assert tuple(x["q"].shape) == (VARLEN.total_T, VARLEN.Hqk, VARLEN.dk)
+    assert tuple(x["v"].shape) == (VARLEN.total_T, VARLEN.H, VARLEN.dv)
+    assert tuple(x["S0"].shape) == (len(a), VARLEN.H, VARLEN.dv, VARLEN.dk)
+    import bench
+    flops, bytes_ = bench.varlen_counts(VARLEN, len(a))
+    assert bytes_ < bench.algorithmic_counts(bench.CONFIGS["layer1p3b_bf16"])[1]   # shared q / k heads
