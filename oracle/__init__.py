@@ -17,6 +17,10 @@ hand-worked example, brute-force transition products and invariants):
                          for the GPU; it pins the chunk algebra the kernels use
                          to the recurrence.
 * ``decode_steps``    -- repeated single-token steps (the recurrence at T=1).
+* ``gate_inputs``     -- the inputs of the recurrence from raw projections: q, k
+                         L2-normalised per token and head, log_alpha and beta from
+                         raw gate projections (a reading: the pages fix neither the
+                         normalisation constant nor the gate parameterisation).
 
 The recurrence (Comba, "Improving Bilinear RNNs with Closed-loop Control";
 PaperWeekly write-up, sections "Comba架构：基于闭环控制理论" and
@@ -204,3 +208,28 @@ def decode_steps(steps, d, S, threads: int = 0):
         o, S = recurrence(q, k, v, la, be, d, S, threads=threads)
         outs.append(o[:, 0])
     return outs, S
+
+
+def gate_inputs(q_raw, k_raw, a_raw, b_raw, A_log, dt_bias, eps: float = 1e-6):
+    """The recurrence's q, k, log_alpha and beta from raw projections, float64:
+
+        q_t = q_raw_t / sqrt(|q_raw_t|^2 + eps)   (likewise k; per token and head)
+        log_alpha_t = -exp(A_log_h) * softplus(a_raw_t + dt_bias_h)
+        beta_t = sigmoid(b_raw_t)
+
+    q_raw, k_raw [B,T,H,dk]; a_raw, b_raw [B,T,H]; A_log, dt_bias [H].  The Comba
+    write-up fixes neither step.  The decay follows the diagonal-SSM discretisation
+    the pages describe on the MaRK page (Hydra: A = -exp(A_log), step softplus(input
+    + bias), log of the discrete eigenvalue = A * step), which is also how the
+    synthetic gates are drawn; beta is a sigmoid gate and q, k are L2-normalised
+    with a small eps (readings).  Returns (q, k, log_alpha, beta) as float64 arrays."""
+    q, k = _f64(q_raw), _f64(k_raw)
+    a, b = _f64(a_raw), _f64(b_raw)
+    A, dtb = _f64(A_log), _f64(dt_bias)
+    q = q / np.sqrt((q * q).sum(-1, keepdims=True) + eps)
+    k = k / np.sqrt((k * k).sum(-1, keepdims=True) + eps)
+    x = a + dtb
+    softplus = np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x)))   # log(1 + e^x), stable
+    log_alpha = -np.exp(A) * softplus
+    beta = 1.0 / (1.0 + np.exp(-b))
+    return q, k, log_alpha, beta

@@ -115,3 +115,42 @@ def test_state_stays_bounded_under_slow_decay():
         (x["beta"].double() * x["v"].double().norm(dim=-1)).sum())
     assert np.linalg.norm(S) <= bound
     assert np.linalg.norm(S) < 200.0
+
+
+def test_gate_inputs_closed_forms():
+    # hand values: softplus(0) = ln 2, sigmoid(0) = 1/2, exp(A_log = ln 3) = 3;
+    # a 3-4-0 row normalises to 0.6, 0.8 (eps negligible)
+    q = np.zeros((1, 2, 1, 3)); q[0, 0, 0] = [3.0, 4.0, 0.0]; q[0, 1, 0] = [0.0, 0.0, -2.0]
+    k = 2.0 * q
+    a = np.array([[[0.0], [25.0]]]); b = np.array([[[0.0], [np.log(3.0)]]])
+    qn, kn, la, be = oracle.gate_inputs(q, k, a, b, np.array([np.log(3.0)]), np.array([0.0]), eps=0.0)
+    np.testing.assert_allclose(qn[0, 0, 0], [0.6, 0.8, 0.0], rtol=1e-15)
+    np.testing.assert_allclose(kn[0, 1, 0], [0.0, 0.0, -1.0], rtol=1e-15)
+    np.testing.assert_allclose(la[0, 0, 0], -3.0 * np.log(2.0), rtol=1e-15)
+    np.testing.assert_allclose(la[0, 1, 0], -3.0 * 25.0, rtol=1e-10)     # softplus(25) = 25 + O(e^-25)
+    np.testing.assert_allclose(be[0, :, 0], [0.5, 0.75], rtol=1e-15)
+
+
+def test_gate_inputs_norms_and_softplus_tails():
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((2, 5, 3, 16)); k = rng.standard_normal((2, 5, 3, 16))
+    qn, kn, _, _ = oracle.gate_inputs(q, k, np.zeros((2, 5, 3)), np.zeros((2, 5, 3)),
+                                      np.zeros(3), np.zeros(3), eps=0.0)
+    np.testing.assert_allclose(np.linalg.norm(qn, axis=-1), 1.0, rtol=1e-14)
+    np.testing.assert_allclose(np.linalg.norm(kn, axis=-1), 1.0, rtol=1e-14)
+    # softplus stays log(1 + e^x) for large and very negative arguments
+    x = np.array([[[25.0], [-30.0]]])
+    _, _, la, _ = oracle.gate_inputs(np.ones((1, 2, 1, 2)), np.ones((1, 2, 1, 2)), x, np.zeros((1, 2, 1)),
+                                     np.zeros(1), np.zeros(1))
+    # log(1 + e^x) = x + e^-x - e^-2x / 2 + ... for x = 25, and e^x - e^2x / 2 + ... for x = -30
+    want = [25.0 + np.exp(-25.0) - np.exp(-50.0) / 2, np.exp(-30.0) - np.exp(-60.0) / 2]
+    np.testing.assert_allclose(-la[0, :, 0], want, rtol=1e-15)
+
+
+def test_gate_inputs_match_the_input_modules_decay_draws():
+    # the chunk workloads draw log a = -softplus(N(0,1)) * exp(U(-4,-1)) per head: the same
+    # form with A_log = that per-head log scale and dt_bias = 0
+    rng = np.random.default_rng(4)
+    z = rng.standard_normal((1, 7, 2)); A_log = np.array([-4.0, -1.5])
+    _, _, la, _ = oracle.gate_inputs(np.ones((1, 7, 2, 4)), np.ones((1, 7, 2, 4)), z, z, A_log, np.zeros(2))
+    np.testing.assert_allclose(la, -np.log1p(np.exp(z)) * np.exp(A_log), rtol=1e-14)
