@@ -20,7 +20,8 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["chunk_fwd", "chunk_fwd_host", "chunk_fwd_varlen", "chunk_fwd_noalloc", "recurrent_step",
+__all__ = ["chunk_fwd", "chunk_fwd_gated", "chunk_fwd_host", "chunk_fwd_varlen", "chunk_fwd_noalloc",
+           "recurrent_step",
            "get_last_error", "CombaError", "library", "library_path", "EXPORTS", "status_string"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -30,7 +31,7 @@ _lock = threading.Lock()
 
 EXPORTS = ("comba_chunk_fwd", "comba_chunk_fwd_f32", "comba_chunk_fwd_varlen",
            "comba_chunk_fwd_workspace_size", "comba_chunk_fwd_ws", "comba_chunk_fwd_noalloc",
-           "comba_chunk_fwd_host", "comba_chunk_fwd_host_workspace_size",
+           "comba_chunk_fwd_host", "comba_chunk_fwd_host_workspace_size", "comba_chunk_fwd_gated",
            "comba_recurrent_step", "comba_recurrent_step_grouped", "comba_get_last_error",
            "comba_status_string", "comba_version")
 
@@ -63,6 +64,7 @@ def library():
             lib.comba_chunk_fwd_workspace_size.argtypes = [i] * 6
             lib.comba_chunk_fwd_workspace_size.restype = ctypes.c_size_t
             lib.comba_chunk_fwd_varlen.argtypes = [vp] * 10 + [i] * 7 + [vp]
+            lib.comba_chunk_fwd_gated.argtypes = [vp] * 11 + [i] * 6 + [ctypes.c_float, vp]
             lib.comba_chunk_fwd_host.argtypes = [vp] * 9 + [i] * 6 + [vp, ctypes.c_size_t, i, vp]
             lib.comba_chunk_fwd_host_workspace_size.argtypes = [i] * 5
             lib.comba_chunk_fwd_host_workspace_size.restype = ctypes.c_size_t
@@ -71,6 +73,7 @@ def library():
             for fn in (lib.comba_chunk_fwd, lib.comba_chunk_fwd_f32, lib.comba_chunk_fwd_ws,
                        lib.comba_chunk_fwd_noalloc, lib.comba_chunk_fwd_varlen,
                        lib.comba_recurrent_step_grouped, lib.comba_chunk_fwd_host,
+                       lib.comba_chunk_fwd_gated,
                        lib.comba_recurrent_step, lib.comba_get_last_error, lib.comba_version):
                 fn.restype = ctypes.c_int
             lib.comba_get_last_error.argtypes = []
@@ -160,6 +163,50 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
             name = "comba_chunk_fwd_f32"
     if st != 0:
         raise CombaError(st, name)
+    return out, S_final
+
+
+def chunk_fwd_gated(q_raw: torch.Tensor, k_raw: torch.Tensor, v: torch.Tensor, a_raw: torch.Tensor,
+                    b_raw: torch.Tensor, A_log: torch.Tensor, dt_bias: Optional[torch.Tensor],
+                    d: torch.Tensor, S0: Optional[torch.Tensor] = None, chunk: int = 64,
+                    norm_eps: float = 1e-6, out: Optional[torch.Tensor] = None,
+                    S_final: Optional[torch.Tensor] = None, return_state: bool = True,
+                    stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """comba_chunk_fwd_gated: the chunk-wise forward from raw projections.  q_raw,
+    k_raw [B,T,H,dk] and v [B,T,H,dv] bf16; a_raw, b_raw [B,T,H] fp32 (raw gate
+    projections); A_log [H], dt_bias [H] or None, d [H] fp32; S0 [B,H,dv,dk] or None.
+    The kernel L2-normalises q, k (eps ``norm_eps``) and forms log_alpha =
+    -exp(A_log) softplus(a_raw + dt_bias), beta = sigmoid(b_raw)."""
+    if q_raw.dim() != 4:
+        raise ValueError("q_raw must be [B, T, H, dk]")
+    B, T, H, dk = q_raw.shape
+    dv = v.shape[-1]
+    _check(q_raw, "q_raw", torch.bfloat16, (B, T, H, dk))
+    _check(k_raw, "k_raw", torch.bfloat16, (B, T, H, dk))
+    _check(v, "v", torch.bfloat16, (B, T, H, dv))
+    _check(a_raw, "a_raw", torch.float32, (B, T, H))
+    _check(b_raw, "b_raw", torch.float32, (B, T, H))
+    _check(A_log, "A_log", torch.float32, (H,))
+    if dt_bias is not None:
+        _check(dt_bias, "dt_bias", torch.float32, (H,))
+    _check(d, "d", torch.float32, (H,))
+    dev = q_raw.device
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (B, H, dv, dk))
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    _check(out, "out", torch.bfloat16, (B, T, H, dv))
+    if S_final is None and return_state:
+        S_final = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _check(S_final, "S_final", torch.float32, (B, H, dv, dk))
+    with torch.cuda.device(dev):
+        st = library().comba_chunk_fwd_gated(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a_raw), _ptr(b_raw),
+                                             _ptr(A_log), _ptr(dt_bias), _ptr(d), _ptr(S0), _ptr(out),
+                                             _ptr(S_final), B, T, H, dk, dv, int(chunk), float(norm_eps),
+                                             _stream_handle(dev, stream))
+    if st != 0:
+        raise CombaError(st, "comba_chunk_fwd_gated")
     return out, S_final
 
 

@@ -63,7 +63,8 @@ chunk_fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                       const float* __restrict__ beta, const float* __restrict__ dvec,
                       const float* S0, Tin* __restrict__ out, float* S_final,
                       int T, int H, int dk, int dv, int C, int dvt,
-                      const int* __restrict__ cu_seqlens, int Hqk) {
+                      const int* __restrict__ cu_seqlens, int Hqk,
+                      const float* __restrict__ A_log, const float* __restrict__ dt_bias, float norm_eps) {
     extern __shared__ float sm[];
     const SimtSmem L_ = simt_smem_layout(dk, dvt, C);
     float* Ks = sm + L_.k;
@@ -99,6 +100,11 @@ chunk_fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         }
     }
     const int hq = h / (H / Hqk);
+    // gated inputs (A_log != null): q and k rows are L2-normalised here and log_alpha /
+    // beta hold raw gate projections a, b: log-decay -exp(A_log_h) softplus(a + dt_bias_h),
+    // beta sigmoid(b)
+    const float gA = A_log ? -expf(A_log[h]) : 0.f;
+    const float gdt = (A_log && dt_bias) ? dt_bias[h] : 0.f;
     const int nv = min(dvt, dv - i0);
     const int ny = dk + nv;
     const float dh = dvec[h];
@@ -124,10 +130,26 @@ chunk_fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         }
         if (tid < L) {
             const size_t o = (row0 + c0 + tid) * H + h;
-            gs[tid] = log_alpha[o];
-            bs[tid] = beta[o];
+            float la = log_alpha[o], bt = beta[o];
+            if (A_log) {
+                const float x = la + gdt;
+                la = gA * (fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))));
+                bt = 1.f / (1.f + expf(-bt));
+            }
+            gs[tid] = la;
+            bs[tid] = bt;
         }
         __syncthreads();
+        if (A_log) {   // L2-normalise the chunk's q and k rows in place
+            for (int idx = tid; idx < 2 * L; idx += nt) {
+                float* rowp = (idx < L ? Ks : Qs) + (idx % L) * ldk;
+                float ss = 0.f;
+                for (int j = 0; j < dk; ++j) ss = fmaf(rowp[j], rowp[j], ss);
+                const float rs = rsqrtf(ss + norm_eps);
+                for (int j = 0; j < dk; ++j) rowp[j] *= rs;
+            }
+            __syncthreads();
+        }
         if (tid == 0) {  // within-chunk cumulative log-decay
             float acc = 0.f;
             for (int r = 0; r < L; ++r) {

@@ -297,16 +297,19 @@ __device__ __forceinline__ void fail(volatile int* gabort) {
 }
 
 // kPacked: chains are packed variable-length sequences (cu_seqlens) whose q / k heads
-// may be shared by groups of value heads; the fixed-length instantiation compiles
-// without those paths.
-template <bool kPacked>
+// may be shared by groups of value heads.  kGated: the inputs are raw projections --
+// q and k rows are L2-normalised in the kernel and log_alpha / beta hold raw gate
+// projections a, b (log-decay -exp(A_log_h) softplus(a + dt_bias_h), beta sigmoid(b)).
+// The plain instantiation compiles without either path.
+template <bool kPacked, bool kGated>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     const float* __restrict__ log_alpha, const float* __restrict__ beta,
                     const float* __restrict__ dvec, const float* S0, float* S_final, int T, int H,
                     int b_split, int no_out, unsigned long long timeout_ns,
-                    const int* __restrict__ cu_seqlens, int qk_group, unsigned short* out_raw) {
+                    const int* __restrict__ cu_seqlens, int qk_group, unsigned short* out_raw,
+                    const float* __restrict__ A_log, const float* __restrict__ dt_bias, float norm_eps) {
     COMBA_CTA_MARK(0);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
@@ -333,7 +336,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // bf16 X' (SPLIT).
     enum { B_KQ0 = 0, B_V = 3, B_GRAM0 = 4, B_GRAM1 = 5, B_WN = 6, B_MMA1 = 7, B_MMA2 = 8,
            B_PBUF0 = 9, B_PBUF1 = 10, B_MMA1B = 11, B_WNREADY = 12, B_WREADY = 13, B_SPLIT = 14,
-           NBARS = 15 };
+           B_NORM0 = 15, NBARS = 18 };   // B_NORM0..2: a q/k stage normalised (gated inputs)
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 6144);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
     volatile int* gabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -349,6 +352,22 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int b = vzero ? bcta - b_split : bcta;
     const bool want_out = (no_out == 0);
     const float dh = dvec[h];
+    // gated inputs: a token's raw gate projections become its log-decay and beta where
+    // they are consumed; tokens past the end stay neutral (log-decay 0, beta 0)
+    const float gA = kGated ? -__expf(A_log[h]) : 0.f;
+    const float gdt = (kGated && dt_bias) ? dt_bias[h] : 0.f;
+    auto to_la = [&](float raw, bool valid) -> float {
+        if constexpr (kGated) {
+            const float x = raw + gdt;
+            return valid ? gA * (fmaxf(x, 0.f) + log1pf(__expf(-fabsf(x)))) : 0.f;
+        } else {
+            return raw;
+        }
+    };
+    auto to_bt = [&](float raw, bool valid) -> float {
+        if constexpr (kGated) return valid ? 1.f / (1.f + __expf(-raw)) : 0.f;
+        else return raw;
+    };
     // The chain's tokens along the tensor maps' token axis (extent T): rows 0 .. T-1 of
     // batch b, or, for packed sequences (cu_seqlens), rows cu_seqlens[b] ..
     // cu_seqlens[b+1]-1 of the single batch.  Its q / k head is h / qk_group.
@@ -442,7 +461,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // Scan of chunk c's log-decays held by threads 0..63: writes e^{g_L - g_r} to
         // sed(c) and e^{g_r} to seg(c), and returns e^{g_L} to every thread of the group.
         auto state_gates = [&](float la, int c) -> float {
-            float x = la;
+            float x = (tid < 64) ? to_la(la, c * kC + tid < Tc) : 0.f;
             if (tid < 64) {
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
@@ -484,13 +503,53 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::fence_proxy_async_smem();
             return okc;
         };
+        // gated inputs: the q and k rows of chunk c's tile L2-normalised in place (row r
+        // of K by thread r, of Q by thread 64 + r; two passes over the row), then the
+        // tile is handed to the tensor pipe
+        auto normalize_tile = [&](int c) -> bool {
+            const bool okc = tc::mbar_wait(kq_bar(c), kq_par(c), timeout_ns);
+            const uint32_t base = sb + kq_stage(c) + (tid >= 64 ? 8192u : 0u);
+            const int r = tid & 63;
+            float ss = 0.f;
+#pragma unroll 4
+            for (int i = 0; i < 16; ++i) {
+                const uint4 w = tc::lds_u32x4(base + (i >> 3) * KQ_ATOM + tc::sw128(r, i & 7));
+                const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(e2[e]);
+                    ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                }
+            }
+            const float rs = rsqrtf(ss + norm_eps);
+#pragma unroll 4
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t a = base + (i >> 3) * KQ_ATOM + tc::sw128(r, i & 7);
+                uint4 w = tc::lds_u32x4(a);
+                __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&w);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(e2[e]);
+                    e2[e] = __floats2bfloat162_rn(f.x * rs, f.y * rs);
+                }
+                tc::sts_u32x4(a, w);
+            }
+            tc::fence_proxy_async_smem();
+            tc::named_barrier(BAR_STATE, kStateThreads);
+            if (issuer) tc::mbar_arrive(&bars[B_NORM0 + c % kKQStages]);
+            return okc;
+        };
         bool ok = true;
         // decays and Qh of chunk 0, initial state
         {
             const float la0 = (tid < 64) ? gate(log_alpha, tid) : 0.f;
             const float eL0 = state_gates(la0, 0);
             tc::named_barrier(BAR_STATE, kStateThreads);
-            ok = state_qh(0);
+            if constexpr (kGated) {   // tiles of chunks 0 and 1 (later ones two chunks ahead)
+                ok = normalize_tile(0) && ok;
+                if (nchunks > 1) ok = normalize_tile(1) && ok;
+            }
+            ok = state_qh(0) && ok;
             const float* s0row = S0 ? S0 + ((size_t)blockIdx.x * kD + row) * kD : nullptr;
 #pragma unroll 1
             for (int pair = 0; pair < 2; ++pair) {
@@ -595,6 +654,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ok = ok && tc::mbar_wait(&bars[B_MMA1B], n & 1, timeout_ns);
                 ok = state_qh(n + 1) && ok;
             }
+            if constexpr (kGated) {   // the tile of chunk n+2 (its TMA was issued a chunk ago)
+                if (n + 2 < nchunks) ok = normalize_tile(n + 2) && ok;
+            }
             COMBA_PHASE(3);
             ok = ok && tc::mbar_wait(&bars[B_MMA2], n & 1, timeout_ns);
             if (issuer) tc::bulk_wait_read0();   // the previous out store has read its staging
@@ -697,7 +759,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // on MMAs issued before it, so no order of these can deadlock.
         bool ok = true;
         auto issue_gram = [&](int c) -> bool {
-            const bool okg = tc::mbar_wait(kq_bar(c), kq_par(c), timeout_ns);
+            // gated inputs: the state group normalises the stage first
+            const bool okg = tc::mbar_wait(kGated ? &bars[B_NORM0 + c % kKQStages] : kq_bar(c), kq_par(c),
+                                           timeout_ns);
             __syncwarp();
             if (okg)
                 gram_mma(tmem + ((c & 1) ? TM_G1 : TM_G), sb + kq_stage(c), &bars[(c & 1) ? B_GRAM1 : B_GRAM0]);
@@ -787,6 +851,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         float la_x = 0.f, bt_x = 0.f;                       // gate warps: next chunk's values
         // gate tables of chunk c into tset(c) from this thread's token values (gate warps)
         auto make_tables = [&](int c, float la, float bt) {
+            la = to_la(la, c * kC + gtok < Tc);
+            bt = to_bt(bt, c * kC + gtok < Tc);
             float x = la;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -1011,7 +1077,9 @@ inline int launch_chunk_tc(const void* q, const void* k, const void* v, const fl
                            const float* beta, const float* d, const float* S0, void* out,
                            float* S_final, int B, int T, int H, cudaStream_t stream,
                            int Bc = -1, unsigned long long timeout_ns = kWaitTimeoutNs,
-                           const int* cu_seqlens = nullptr, int nseq = 0, int Hqk = 0) {
+                           const int* cu_seqlens = nullptr, int nseq = 0, int Hqk = 0,
+                           const float* A_log = nullptr, const float* dt_bias = nullptr,
+                           float norm_eps = 0.f) {
     if (Bc < 0) Bc = B;
     if (Hqk <= 0) Hqk = H;
     if (H % Hqk != 0) return -1;
@@ -1019,9 +1087,11 @@ inline int launch_chunk_tc(const void* q, const void* k, const void* v, const fl
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -3;
     if (!attr_set[dev]) {
-        if (cudaFuncSetAttribute(tck::chunk_fwd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(tck::chunk_fwd_tc_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)tck::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(tck::chunk_fwd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(tck::chunk_fwd_tc_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tck::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(tck::chunk_fwd_tc_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)tck::kSmemBytes) != cudaSuccess)
             return -3;
         attr_set[dev] = true;
@@ -1032,10 +1102,12 @@ inline int launch_chunk_tc(const void* q, const void* k, const void* v, const fl
         return -3;
     const int chains = cu_seqlens ? nseq : Bc;
     const int b_split = cu_seqlens ? nseq : B;
-    auto kern = cu_seqlens ? tck::chunk_fwd_tc_kernel<true> : tck::chunk_fwd_tc_kernel<false>;
+    if (cu_seqlens && A_log) return -2;   // packed sequences with gated inputs: not built
+    auto kern = cu_seqlens ? tck::chunk_fwd_tc_kernel<true, false>
+                           : (A_log ? tck::chunk_fwd_tc_kernel<false, true> : tck::chunk_fwd_tc_kernel<false, false>);
     kern<<<(unsigned)(chains * H), tck::kThreads, tck::kSmemBytes, stream>>>(
         tq, tk, tv, to, log_alpha, beta, d, S0, S_final, T, H, b_split, out ? 0 : 1, timeout_ns,
-        cu_seqlens, H / Hqk, static_cast<unsigned short*>(out));
+        cu_seqlens, H / Hqk, static_cast<unsigned short*>(out), A_log, dt_bias, norm_eps);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 

@@ -95,6 +95,9 @@ struct Packing {
     const int* cu_seqlens = nullptr;
     int nseq = 0;
     int Hqk = 0;
+    const float* A_log = nullptr;     // gated inputs (see comba_chunk_fwd_gated)
+    const float* dt_bias = nullptr;
+    float norm_eps = 0.f;
 };
 
 template <typename Tin>
@@ -117,7 +120,7 @@ int launch_simt(const ChunkArgs& a, cudaStream_t stream, Packing pk = Packing())
     kern<<<grid, comba::kSimtThreads, smem, stream>>>(
         static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
         a.log_alpha, a.beta, a.d, a.S0, static_cast<Tin*>(a.out), a.S_final, a.T, a.H, a.dk,
-        a.dv, a.chunk, dvt, pk.cu_seqlens, pk.Hqk > 0 ? pk.Hqk : a.H);
+        a.dv, a.chunk, dvt, pk.cu_seqlens, pk.Hqk > 0 ? pk.Hqk : a.H, pk.A_log, pk.dt_bias, pk.norm_eps);
     return cudaGetLastError() == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
 }
 
@@ -174,6 +177,32 @@ extern "C" int comba_chunk_fwd_varlen(const void* q, const void* k, const void* 
     ChunkArgs a1 = a;
     a1.B = 1;
     return launch_simt<__nv_bfloat16>(a1, s, Packing{cu_seqlens, N, Hqk});
+}
+
+extern "C" int comba_chunk_fwd_gated(const void* q_raw, const void* k_raw, const void* v,
+                                     const float* a_raw, const float* b_raw, const float* A_log,
+                                     const float* dt_bias, const float* d, const float* S0, void* out,
+                                     float* S_final, int B, int T, int H, int dk, int dv, int chunk,
+                                     float norm_eps, comba_stream_t stream) {
+    const ChunkArgs a{q_raw, k_raw, v, a_raw, b_raw, d, S0, out, S_final, B, T, H, dk, dv, chunk, 2};
+    if (int st = validate_chunk(a)) return st;
+    if (!(norm_eps >= 0.f)) return COMBA_EINVAL;
+    if (B == 0 || H == 0) return COMBA_OK;
+    if (!A_log || !aligned(A_log, 4) || !aligned(dt_bias, 4)) return COMBA_EINVAL;
+    const size_t nv = (size_t)B * T * H * dv * 2, ns = (size_t)B * H * dv * dk * sizeof(float);
+    if (overlap(out, nv, A_log, (size_t)H * 4) || overlap(out, nv, dt_bias, (size_t)H * 4) ||
+        overlap(S_final, ns, A_log, (size_t)H * 4) || overlap(S_final, ns, dt_bias, (size_t)H * 4))
+        return COMBA_EINVAL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) return empty_sequence(a, s);
+    if (comba::tc_supported(dk, dv, chunk))
+        return comba::launch_chunk_tc(q_raw, k_raw, v, a_raw, b_raw, d, S0, out, S_final, B, T, H, s, -1,
+                                      comba::kWaitTimeoutNs, nullptr, 0, 0, A_log, dt_bias, norm_eps);
+    Packing pk;
+    pk.A_log = A_log;
+    pk.dt_bias = dt_bias;
+    pk.norm_eps = norm_eps;
+    return launch_simt<__nv_bfloat16>(a, s, pk);
 }
 
 extern "C" size_t comba_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk) {

@@ -39,6 +39,7 @@ __all__ = [
     "ChunkConfig", "DecodeConfig", "CONFIGS", "DECODE", "chunk_config",
     "make_chunk_inputs", "make_decode_state", "decode_step_inputs",
     "head_token_count", "VarlenConfig", "VARLEN", "varlen_lengths", "make_varlen_inputs",
+    "make_gated_inputs",
 ]
 
 
@@ -156,6 +157,31 @@ def make_varlen_inputs(cfg: VarlenConfig) -> Dict[str, torch.Tensor]:
         "S0": (cfg.s0_std * _normal(gen, (N, cfg.H, cfg.dv, cfg.dk))).to(torch.float32).contiguous(),
         "cu_seqlens": torch.tensor(cu, dtype=torch.int32),
     }
+
+
+def make_gated_inputs(cfg: ChunkConfig, seed: Optional[int] = None, dt_bias_std: float = 0.0) -> Dict[str, torch.Tensor]:
+    """Raw-projection inputs of a chunk workload, CPU tensors: q_raw, k_raw [B,T,H,dk]
+    bf16 drawn N(0,1) and scaled per row by exp(U(-1,1)) (not normalised); v bf16 as
+    the chunk workloads; a_raw, b_raw [B,T,H] ~ N(0,1); A_log [H] ~ U(-4,-1) (the
+    per-head log scale of the chunk workloads' decay draws); dt_bias [H] ~ N(0,
+    dt_bias_std^2); d [H] ~ U(0,1); S0 as cfg.s0_std."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(cfg.seed + 7919 if seed is None else seed)
+    B, T, H, dk, dv = cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv
+    scale_q = torch.exp(_uniform(gen, (B, T, H, 1), -1.0, 1.0))
+    scale_k = torch.exp(_uniform(gen, (B, T, H, 1), -1.0, 1.0))
+    q = (_normal(gen, (B, T, H, dk)) * scale_q).to(torch.bfloat16)
+    k = (_normal(gen, (B, T, H, dk)) * scale_k).to(torch.bfloat16)
+    v = _normal(gen, (B, T, H, dv)).to(torch.bfloat16)
+    a = _normal(gen, (B, T, H)).to(torch.float32)
+    b = _normal(gen, (B, T, H)).to(torch.float32)
+    A_log = _uniform(gen, (H,), -4.0, -1.0).to(torch.float32)
+    dt_bias = (dt_bias_std * _normal(gen, (H,))).to(torch.float32)
+    d = _uniform(gen, (H,), 0.0, 1.0).to(torch.float32)
+    S0 = (cfg.s0_std * _normal(gen, (B, H, dv, dk))).to(torch.float32) if cfg.s0_std > 0 else None
+    return {"q_raw": q.contiguous(), "k_raw": k.contiguous(), "v": v.contiguous(), "a_raw": a.contiguous(),
+            "b_raw": b.contiguous(), "A_log": A_log.contiguous(), "dt_bias": dt_bias.contiguous(),
+            "d": d.contiguous(), "S0": None if S0 is None else S0.contiguous()}
 
 
 def chunk_config(name: str) -> ChunkConfig:

@@ -107,6 +107,25 @@ int comba_chunk_fwd_varlen(const void* q, const void* k, const void* v,
                            int dk, int dv, int chunk, comba_stream_t stream);
 
 /*
+ * comba_chunk_fwd from raw projections ("gate-in-kernel"): the kernel forms the
+ * recurrence's inputs itself, per token and head,
+ *     q_t = q_raw_t / sqrt(|q_raw_t|^2 + norm_eps)      (likewise k_t)
+ *     log_alpha_t = -exp(A_log_h) * softplus(a_raw_t + dt_bias_h)
+ *     beta_t = 1 / (1 + exp(-b_raw_t))
+ * (the pages fix neither step: the decay follows the diagonal-SSM discretisation
+ * described on the MaRK page, the rest are readings).  Layouts as comba_chunk_fwd
+ * with q_raw, k_raw in place of q, k and a_raw, b_raw [B, T, H] fp32 in place of
+ * log_alpha, beta; A_log [H] fp32 (device, required); dt_bias [H] fp32 (device;
+ * NULL means zero); norm_eps >= 0.  In the tensor-core kernel the normalised q, k
+ * rows are rounded to bf16 before use, as normalised bf16 inputs would be.
+ */
+int comba_chunk_fwd_gated(const void* q_raw, const void* k_raw, const void* v,
+                          const float* a_raw, const float* b_raw, const float* A_log,
+                          const float* dt_bias, const float* d, const float* S0, void* out,
+                          float* S_final, int B, int T, int H, int dk, int dv, int chunk,
+                          float norm_eps, comba_stream_t stream);
+
+/*
  * Workspace the segmented form of comba_chunk_fwd_ws needs for this shape on the
  * current device, in bytes; 0 when the shape runs unsegmented (enough (b, h)
  * chains to fill the GPU, a T that is not a multiple of 64, or a shape outside the

@@ -198,3 +198,32 @@ def test_host_entry_workspace_size_and_rejections(lib):
     assert _call_host(lib, a, ws, need, 0) == -1              # no slices
     assert _call_host(lib, _chunk_args(dk=24), ws, need, 4) == -1
     assert _call_host(lib, _chunk_args(out=BASE + 16), ws, need, 4) == -1   # out overlaps q
+
+
+def _call_gated(lib, a, A_log, dt_bias, eps):
+    p = lambda x: ctypes.c_void_p(x)
+    return lib.comba_chunk_fwd_gated(p(a["q"]), p(a["k"]), p(a["v"]), p(a["log_alpha"]), p(a["beta"]),
+                                     p(A_log), p(dt_bias), p(a["d"]), p(a["S0"]), p(a["out"]),
+                                     p(a["S_final"]), a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                                     a["chunk"], ctypes.c_float(eps), ctypes.c_void_p(None))
+
+
+@pytest.mark.parametrize("A_log,dt_bias,eps", [
+    (None, BASE + 11 * GB, 1e-6),                     # A_log required
+    (BASE + 10 * GB + 2, BASE + 11 * GB, 1e-6),       # misaligned A_log
+    (BASE + 10 * GB, BASE + 11 * GB + 1, 1e-6),       # misaligned dt_bias
+    (BASE + 10 * GB, BASE + 11 * GB, -1.0),           # negative eps
+    (BASE + 10 * GB, BASE + 11 * GB, float("nan")),
+    (BASE + 7 * GB + 64, BASE + 11 * GB, 1e-6),       # A_log inside out
+])
+def test_gated_rejects_bad_arguments(lib, A_log, dt_bias, eps):
+    assert _call_gated(lib, _chunk_args(), A_log, dt_bias, eps) == -1
+
+
+def test_gated_rejects_the_chunk_entrys_bad_arguments(lib):
+    assert _call_gated(lib, _chunk_args(dk=24), BASE + 10 * GB, None, 1e-6) == -1
+    assert _call_gated(lib, _chunk_args(out=BASE + 16), BASE + 10 * GB, None, 1e-6) == -1
+
+
+def test_gated_empty_is_noop(lib):
+    assert _call_gated(lib, _chunk_args(B=0, q=None, k=None, v=None), BASE + 10 * GB, None, 1e-6) == 0
