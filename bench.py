@@ -33,7 +33,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from comba_workloads import (CONFIGS, DECODE, VARLEN, make_varlen_inputs,  # noqa: E402
+from comba_workloads import (CONFIGS, DECODE, VARLEN, make_gated_inputs, make_varlen_inputs,  # noqa: E402
                              decode_step_inputs, make_chunk_inputs,
                              make_decode_state)
 
@@ -475,6 +475,90 @@ def run_varlen(args):
     print(json.dumps(line), flush=True)
 
 
+GATED = "layer1p3b_gated_bf16"
+
+
+def run_gated(args):
+    """One step = one comba_chunk_fwd_gated over the 1.3B-layer workload given as raw
+    projections (q, k not normalised, raw gate projections): the same algorithmic
+    bytes as the plain workload, inputs resident in HBM."""
+    import chunk_delta_rule_b200 as cdr
+    cfg = CONFIGS["layer1p3b_bf16"]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cdr.library()
+    x = make_gated_inputs(cfg)
+    host = {k: v.pin_memory() for k, v in x.items() if v is not None}
+    d_ = {k: v.to(dev) for k, v in host.items()}
+    out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.dv), dtype=torch.bfloat16, device=dev)
+    S_final = torch.empty((cfg.B, cfg.H, cfg.dv, cfg.dk), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        cdr.chunk_fwd_gated(d_["q_raw"], d_["k_raw"], d_["v"], d_["a_raw"], d_["b_raw"], d_["A_log"],
+                            d_["dt_bias"], d_["d"], d_.get("S0"), chunk=cfg.chunk, out=out,
+                            S_final=S_final, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert cdr.get_last_error(dev) == 0
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(0).start()
+    th0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    th1 = time.time()
+    clocks.wait_after(th0)
+    clocks.stop()
+    ms_step = ev0.elapsed_time(ev1) / args.steps
+    if cdr.get_last_error(dev) != 0:
+        raise RuntimeError("device-side error during the timed region")
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    S_h = torch.empty(S_final.shape, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        for k in host:
+            d_[k].copy_(host[k], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        S_h.copy_(S_final, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_e2e = ev0.elapsed_time(ev1) / args.steps
+    flops, bytes_ = algorithmic_counts(cfg)
+    peaks = load_peaks()
+    gbs = bytes_ / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": "Comba chunk-fwd tokens/s from raw projections (normalisation and gates in the kernel), % of HBM roofline",
+        "value": cfg.B * cfg.T / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(config_record(cfg), workload=GATED),
+        "tflops": flops / (ms_step / 1e3) / 1e12,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": peaks["source"] + " hbm_gbs (copy)",
+                     "algorithmic_bytes_per_launch": bytes_, "algorithmic_flops_per_launch": flops},
+        "e2e": {"value": cfg.B * cfg.T / (ms_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in host.values()),
+                "d2h_bytes_per_step": out_h.numel() * 2 + S_h.numel() * 4, "ms_per_step": ms_e2e},
+        "clocks": clocks.summary(th0, th1),
+        "gpu_launches": args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -482,7 +566,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="layer1p3b_bf16",
-                    choices=sorted(CONFIGS) + [DECODE.name, VARLEN.name])
+                    choices=sorted(CONFIGS) + [DECODE.name, VARLEN.name, GATED])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -492,6 +576,12 @@ def main():
             print(json.dumps({"impl": "reference", "unavailable": "the decode workload has no reference arm; the headline workload does"}))
             return
         run_decode(args)
+        return
+    if args.workload == GATED:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the raw-projection workload has no reference arm; the headline workload does"}))
+            return
+        run_gated(args)
         return
     if args.workload == VARLEN.name:
         if args.impl == "reference":

@@ -56,3 +56,23 @@ def test_gated_zero_length_copies_state():
                                  empty(xd["b_raw"]), xd["A_log"], None, xd["d"], xd["S0"], chunk=64)
     torch.cuda.synchronize()
     assert torch.equal(S, xd["S0"])
+
+
+def test_gated_full_size_sampled_chains():
+    # the benchmark's raw-projection workload (1.3B layer), run whole; two (b, h) chains
+    # against the oracle
+    cfg = CONFIGS["layer1p3b_bf16"]
+    x = make_gated_inputs(cfg)
+    xd = {k: (None if v is None else v.cuda()) for k, v in x.items()}
+    out, S = cdr.chunk_fwd_gated(xd["q_raw"], xd["k_raw"], xd["v"], xd["a_raw"], xd["b_raw"], xd["A_log"],
+                                 xd["dt_bias"], xd["d"], xd["S0"], chunk=cfg.chunk, norm_eps=EPS)
+    torch.cuda.synchronize()
+    assert cdr.get_last_error() == 0
+    q, k, la, be = oracle.gate_inputs(x["q_raw"], x["k_raw"], x["a_raw"], x["b_raw"], x["A_log"],
+                                      x["dt_bias"], eps=EPS)
+    for b, h in [(0, 0), (7, 15)]:
+        sl = lambda a: a[b:b + 1, :, h:h + 1]
+        ro, rS = oracle.recurrence(sl(q), sl(k), sl(x["v"]), sl(la), sl(be), x["d"][h:h + 1],
+                                   x["S0"][b:b + 1, h:h + 1])
+        assert_close(f"out {b},{h}", out[b, :, h].double().cpu().numpy(), ro[0, :, 0], TOL_BF16)
+        assert_close(f"S_final {b},{h}", S[b, h].double().cpu().numpy(), rS[0, 0], TOL_BF16)
