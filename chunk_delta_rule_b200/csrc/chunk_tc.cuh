@@ -188,13 +188,17 @@ __device__ __forceinline__ void acc_to_bfrag(const float (&c)[4], uint32_t (&b)[
 // Eb = Tinv diag(beta) (bf16, K-major 128B-swizzled at F1 and F1 + 8192), zero
 // above block row j.  CS / BT: shared addresses of c and beta.
 __device__ __forceinline__ void strip_inverse(const float* F2p, uint32_t F1, int w, int lane, uint32_t CS,
-                                              uint32_t BT) {
+                                              uint32_t BT, uint32_t IK = 0) {
     const int j = w >> 1, co = 8 * (w & 1);
     const int g = lane >> 2, t = lane & 3;
     const int oa0 = boff(g, t), oa1 = boff(g, t + 4), oa2 = boff(g, 8 + t), oa3 = boff(g, 12 + t);
     const int ob0 = boff(t, co + g), ob1 = boff(t + 4, co + g);
     const int s0 = 8 * w + 2 * t;
-    const float c0 = tc::lds_f32(CS + 4u * s0), c1 = tc::lds_f32(CS + 4u * (s0 + 1));
+    float c0 = tc::lds_f32(CS + 4u * s0), c1 = tc::lds_f32(CS + 4u * (s0 + 1));
+    if (IK) {   // normalised k: W = Tinv diag(c / |k|) K
+        c0 *= tc::lds_f32(IK + 4u * s0);
+        c1 *= tc::lds_f32(IK + 4u * (s0 + 1));
+    }
     const float e0 = tc::lds_f32(BT + 4u * s0), e1 = tc::lds_f32(BT + 4u * (s0 + 1));
     // rows 16 i + g (+ 8) of this strip: 128B-swizzled chunk w of each row
     const uint32_t orow = F1 + (uint32_t)g * 128u + ((uint32_t)(w ^ g) << 4) + 4u * (uint32_t)t;
@@ -261,32 +265,47 @@ __device__ __noinline__ void gram_mma(uint32_t d, uint32_t kq, uint64_t* bar) {
 //   a_rows_exact: A_rs = beta_r 2^{g'_{r-1} - g'_s} (K K^T)_rs (s < r) for row r over
 //   columns 32 ch .. + 31, from the Gram in TMEM, stored as -A into F2's blocks
 //   (g' = g log2 e)
-__device__ __noinline__ void a_rows_exact(float* F2p, uint32_t gram_taddr, int r, int ch, uint32_t ts) {
+//   (ikt: shared address of 1 / |k| per token when q and k are normalised in the
+//   kernel, else 0)
+template <bool kNorm>
+__device__ __noinline__ void a_rows_exact(float* F2p, uint32_t gram_taddr, int r, int ch, uint32_t ts,
+                                          uint32_t ikt) {
     float a[32];
     tc::tmem_ld32(gram_taddr, a);
     tc::tmem_ld_wait();
-    const float br = tc::lds_f32(ts + 512 + 4u * r), gpr = tc::lds_f32(ts + 256 + 4u * r);
+    float br = tc::lds_f32(ts + 512 + 4u * r);
+    const float gpr = tc::lds_f32(ts + 256 + 4u * r);
+    if constexpr (kNorm) br *= tc::lds_f32(ikt + 4u * r);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
         const int s = 32 * ch + e;
-        const float v = br * exp2f(gpr - tc::lds_f32(ts + 4u * s)) * a[e];
+        float v = br * exp2f(gpr - tc::lds_f32(ts + 4u * s)) * a[e];
+        if constexpr (kNorm) v *= tc::lds_f32(ikt + 4u * s);
         a[e] = (s < r) ? v : 0.f;
     }
     store_neg_a(F2p, r, ch, a);
 }
 //   p_row_exact: P_rs = 2^{g'_r - g'_s} (Q K^T - d K K^T)_rs (s <= r) for row r over
 //   columns 32 ch .. + 31, in place over the staged K K^T row
+//   (ikt as above; iq: 1 / |q_r|, 1 when not normalised)
+template <bool kNorm>
 __device__ __noinline__ void p_row_exact(uint32_t prow, uint32_t gram_taddr, int r, int ch, float dh,
-                                         uint32_t ts) {
+                                         uint32_t ts, uint32_t ikt, float iq) {
     float gv[32];
     tc::tmem_ld32(gram_taddr, gv);
     tc::tmem_ld_wait();
     const float gr = tc::lds_f32(ts + 4u * r);
+    const float dk = kNorm ? dh * tc::lds_f32(ikt + 4u * r) : dh;
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
         const int s = 32 * ch + e;
         const uint32_t pa = prow + tc::sw128(r, e >> 2) + 4u * (e & 3);
-        const float v = exp2f(gr - tc::lds_f32(ts + 4u * s)) * fmaf(-dh, tc::lds_f32(pa), gv[e]);
+        float v;
+        if constexpr (kNorm)
+            v = exp2f(gr - tc::lds_f32(ts + 4u * s)) * tc::lds_f32(ikt + 4u * s) *
+                fmaf(-dk, tc::lds_f32(pa), iq * gv[e]);
+        else
+            v = exp2f(gr - tc::lds_f32(ts + 4u * s)) * fmaf(-dh, tc::lds_f32(pa), gv[e]);
         tc::sts_f32(pa, (s <= r) ? v : 0.f);
     }
 }
@@ -320,13 +339,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // built while the current one is in use), 64 fp32 each, by shared address:
     //   +0 g_r log2(e), +256 g_{r-1} log2(e), +512 beta_r, +768 beta_r e^{g_{r-1}},
     //   +1024 e^{g_r}, +1280 e^{-g_r} (when the chunk allows), +1536 the chunk's
-    //   "fast" flag (total log-decay above -80)
+    //   "fast" flag (total log-decay above -80), +1792 1 / |k_r| (normalised q, k only)
     auto tset = [&](int c) -> uint32_t { return sb + SM_MISC + 2048u * (uint32_t)(c & 1); };
     const uint32_t RED = sb + SM_MISC + 4096;   // gate warps: [0..1] scan carries
     const uint32_t SRED = RED + 16;             // state group: [0..1] scan carries
     // state group, per chunk parity: e^{g_L - g_r} (SED) and e^{g_r} (SEG) of a chunk
     auto sed = [&](int c) -> uint32_t { return sb + SM_MISC + 4352u + 512u * (uint32_t)(c & 1); };
     auto seg = [&](int c) -> uint32_t { return sed(c) + 256u; };
+    // gated inputs: the state group's 1 / |k_r| of a chunk (per parity), and its
+    // partial row sums of squares exchanged between the two threads of a row
+    auto sik = [&](int c) -> uint32_t { return sb + SM_MISC + 5376u + 256u * (uint32_t)(c & 1); };
+    const uint32_t XCH = sb + SM_MISC + 7168;
     // barriers: q/k stages, v, gram per TMEM buffer, wn (W^T, U~^T in TMEM), mma1 (X),
     // mma2, the P buffers (MMA2 has read them), mma1 (O).  Each is arrived on once per
     // phase (by a commit, a TMA transaction count or one thread after its group's
@@ -336,7 +359,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // bf16 X' (SPLIT).
     enum { B_KQ0 = 0, B_V = 3, B_GRAM0 = 4, B_GRAM1 = 5, B_WN = 6, B_MMA1 = 7, B_MMA2 = 8,
            B_PBUF0 = 9, B_PBUF1 = 10, B_MMA1B = 11, B_WNREADY = 12, B_WREADY = 13, B_SPLIT = 14,
-           B_NORM0 = 15, NBARS = 18 };   // B_NORM0..2: a q/k stage normalised (gated inputs)
+           NBARS = 15 };
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 6144);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
     volatile int* gabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -485,6 +508,34 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const uint32_t kqc = sb + kq_stage(c);
             const int r = tid & 63, jh = tid >> 6;
             const float egr = tc::lds_f32(seg(c) + 4u * r);
+            float fq = egr, fk = egr * dh;   // Qh row = fq q - fk k
+            if constexpr (kGated) {
+                // gated inputs: |q_r|, |k_r| from this thread's half-rows and the partner
+                // thread's (64 + r or r - 64) partial sums; 1 / |k_r| kept for the state update
+                float sk = 0.f, sq = 0.f;
+#pragma unroll 2
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const uint32_t off = kqc + jh * KQ_ATOM + tc::sw128(r, c8);
+                    const uint4 kw = tc::lds_u32x4(off), qw = tc::lds_u32x4(off + 8192);
+                    const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kw);
+                    const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qw);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 kf = __bfloat1622float2(k2[e]), qf = __bfloat1622float2(q2[e]);
+                        sk = fmaf(kf.x, kf.x, fmaf(kf.y, kf.y, sk));
+                        sq = fmaf(qf.x, qf.x, fmaf(qf.y, qf.y, sq));
+                    }
+                }
+                tc::sts_f32(XCH + 8u * (64u * jh + r), sk);
+                tc::sts_f32(XCH + 8u * (64u * jh + r) + 4u, sq);
+                tc::named_barrier(BAR_STATE, kStateThreads);
+                sk += tc::lds_f32(XCH + 8u * (64u * (1 - jh) + r));
+                sq += tc::lds_f32(XCH + 8u * (64u * (1 - jh) + r) + 4u);
+                const float ik = rsqrtf(sk + norm_eps), iq = rsqrtf(sq + norm_eps);
+                if (jh == 0) tc::sts_f32(sik(c) + 4u * r, ik);
+                fq = egr * iq;
+                fk = egr * dh * ik;
+            }
 #pragma unroll 2
             for (int c8 = 0; c8 < 8; ++c8) {
                 const uint32_t off = kqc + jh * KQ_ATOM + tc::sw128(r, c8);
@@ -496,47 +547,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int e = 0; e < 4; ++e) {
                     const float2 kf = __bfloat1622float2(k2[e]);
                     const float2 qf = __bfloat1622float2(q2[e]);
-                    q2[e] = __floats2bfloat162_rn(egr * fmaf(-dh, kf.x, qf.x), egr * fmaf(-dh, kf.y, qf.y));
+                    if constexpr (kGated)
+                        q2[e] = __floats2bfloat162_rn(fmaf(-fk, kf.x, fq * qf.x), fmaf(-fk, kf.y, fq * qf.y));
+                    else
+                        q2[e] = __floats2bfloat162_rn(egr * fmaf(-dh, kf.x, qf.x), egr * fmaf(-dh, kf.y, qf.y));
                 }
                 tc::sts_u32x4(sb + SM_QH + jh * QH_ATOM + tc::sw128(r, c8), qw);
             }
             tc::fence_proxy_async_smem();
-            return okc;
-        };
-        // gated inputs: the q and k rows of chunk c's tile L2-normalised in place (row r
-        // of K by thread r, of Q by thread 64 + r; two passes over the row), then the
-        // tile is handed to the tensor pipe
-        auto normalize_tile = [&](int c) -> bool {
-            const bool okc = tc::mbar_wait(kq_bar(c), kq_par(c), timeout_ns);
-            const uint32_t base = sb + kq_stage(c) + (tid >= 64 ? 8192u : 0u);
-            const int r = tid & 63;
-            float ss = 0.f;
-#pragma unroll 4
-            for (int i = 0; i < 16; ++i) {
-                const uint4 w = tc::lds_u32x4(base + (i >> 3) * KQ_ATOM + tc::sw128(r, i & 7));
-                const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&w);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(e2[e]);
-                    ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
-                }
-            }
-            const float rs = rsqrtf(ss + norm_eps);
-#pragma unroll 4
-            for (int i = 0; i < 16; ++i) {
-                const uint32_t a = base + (i >> 3) * KQ_ATOM + tc::sw128(r, i & 7);
-                uint4 w = tc::lds_u32x4(a);
-                __nv_bfloat162* e2 = reinterpret_cast<__nv_bfloat162*>(&w);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(e2[e]);
-                    e2[e] = __floats2bfloat162_rn(f.x * rs, f.y * rs);
-                }
-                tc::sts_u32x4(a, w);
-            }
-            tc::fence_proxy_async_smem();
-            tc::named_barrier(BAR_STATE, kStateThreads);
-            if (issuer) tc::mbar_arrive(&bars[B_NORM0 + c % kKQStages]);
             return okc;
         };
         bool ok = true;
@@ -545,10 +563,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const float la0 = (tid < 64) ? gate(log_alpha, tid) : 0.f;
             const float eL0 = state_gates(la0, 0);
             tc::named_barrier(BAR_STATE, kStateThreads);
-            if constexpr (kGated) {   // tiles of chunks 0 and 1 (later ones two chunks ahead)
-                ok = normalize_tile(0) && ok;
-                if (nchunks > 1) ok = normalize_tile(1) && ok;
-            }
             ok = state_qh(0) && ok;
             const float* s0row = S0 ? S0 + ((size_t)blockIdx.x * kD + row) * kD : nullptr;
 #pragma unroll 1
@@ -628,7 +642,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::tmem_ld_wait();
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const float4 d4 = tc::lds_f32x4(sedn + 4u * (32 * half + 4 * c));
+                    float4 d4 = tc::lds_f32x4(sedn + 4u * (32 * half + 4 * c));
+                    if constexpr (kGated) {   // the state update reads the normalised k: X' columns / |k_s|
+                        const float4 k4 = tc::lds_f32x4(sik(n) + 4u * (32 * half + 4 * c));
+                        d4.x *= k4.x; d4.y *= k4.y; d4.z *= k4.z; d4.w *= k4.w;
+                    }
                     const float a0 = xv[4 * c] * d4.x, a1 = xv[4 * c + 1] * d4.y;
                     const float a2 = xv[4 * c + 2] * d4.z, a3 = xv[4 * c + 3] * d4.w;
                     const uint32_t h01 = tc::pack_bf16(a0, a1), h23 = tc::pack_bf16(a2, a3);
@@ -653,9 +671,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!last && want_out) {
                 ok = ok && tc::mbar_wait(&bars[B_MMA1B], n & 1, timeout_ns);
                 ok = state_qh(n + 1) && ok;
-            }
-            if constexpr (kGated) {   // the tile of chunk n+2 (its TMA was issued a chunk ago)
-                if (n + 2 < nchunks) ok = normalize_tile(n + 2) && ok;
             }
             COMBA_PHASE(3);
             ok = ok && tc::mbar_wait(&bars[B_MMA2], n & 1, timeout_ns);
@@ -759,9 +774,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // on MMAs issued before it, so no order of these can deadlock.
         bool ok = true;
         auto issue_gram = [&](int c) -> bool {
-            // gated inputs: the state group normalises the stage first
-            const bool okg = tc::mbar_wait(kGated ? &bars[B_NORM0 + c % kKQStages] : kq_bar(c), kq_par(c),
-                                           timeout_ns);
+            const bool okg = tc::mbar_wait(kq_bar(c), kq_par(c), timeout_ns);
             __syncwarp();
             if (okg)
                 gram_mma(tmem + ((c & 1) ? TM_G1 : TM_G), sb + kq_stage(c), &bars[(c & 1) ? B_GRAM1 : B_GRAM0]);
@@ -913,15 +926,35 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int c = 0; c < 8; ++c)
                     tc::sts_f32x4(pbm + ch * F32_ATOM + tc::sw128(r, c),
                                   make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]));
-                tc::tc_fence_before();
-                tc::named_barrier_arrive(BAR_KK, kKKThreads);
+                if constexpr (kGated) {
+                    // normalised q, k: 1 / |k_r| from the Gram's diagonal (pw 3: rows 0-31,
+                    // pw 4: rows 32-63) for the whole prep group; pw 0 reads it after them
+                    if (pw != 0) {
+                        float dg = 0.f;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) dg = (e == lane) ? a[e] : dg;
+                        tc::sts_f32(ts + 1792 + 4u * r, rsqrtf(dg + norm_eps));
+                    }
+                    tc::tc_fence_before();
+                    if (pw != 0) tc::named_barrier_arrive(BAR_KK, kKKThreads);
+                    else tc::named_barrier(BAR_KK, kKKThreads);
+                    __syncwarp();
+                } else {
+                    tc::tc_fence_before();
+                    tc::named_barrier_arrive(BAR_KK, kKKThreads);
+                }
                 COMBA_PHASE(27);
                 // A_rs = beta_r e^{g_{r-1} - g_s} (K K^T)_rs for s < r -> -A into F2
                 if (fast) {
-                    const float cr = tc::lds_f32(ts + 768 + 4u * r);
+                    float cr = tc::lds_f32(ts + 768 + 4u * r);
+                    if constexpr (kGated) cr *= tc::lds_f32(ts + 1792 + 4u * r);
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        const float4 ig = tc::lds_f32x4(ts + 1280 + 4u * (32 * ch + 4 * c));
+                        float4 ig = tc::lds_f32x4(ts + 1280 + 4u * (32 * ch + 4 * c));
+                        if constexpr (kGated) {
+                            const float4 k4 = tc::lds_f32x4(ts + 1792 + 4u * (32 * ch + 4 * c));
+                            ig.x *= k4.x; ig.y *= k4.y; ig.z *= k4.z; ig.w *= k4.w;
+                        }
                         const float iv[4] = {ig.x, ig.y, ig.z, ig.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
@@ -930,7 +963,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     COMBA_PHASE(28);
                     store_neg_a(F2p, r, ch, a);
                 } else {
-                    a_rows_exact(F2p, tl + tgm + 32 * ch, r, ch, ts);
+                    a_rows_exact<kGated>(F2p, tl + tgm + 32 * ch, r, ch, ts, ts + 1792);
                 }
                 COMBA_PHASE(9);
                 if (pw != 0) {   // diagonal blocks 0, 1 (pw 3) and 2, 3 (pw 4) from this warp's rows
@@ -945,28 +978,58 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::tc_fence_after();
                 float gv[32];
                 tc::tmem_ld32(tl + tgm + 32 * ch, gv);
+                // normalised q, k: 1 / |q_r| from this chunk's q row (while the K K^T warps work)
+                float iq = 1.f;
+                if constexpr (kGated) {
+                    const uint32_t qrow = sb + kq_stage(m) + 8192;
+                    float sq = 0.f;
+#pragma unroll 4
+                    for (int i = 0; i < 16; ++i) {
+                        const uint4 w = tc::lds_u32x4(qrow + (i >> 3) * KQ_ATOM + tc::sw128(r, i & 7));
+                        const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(e2[e]);
+                            sq = fmaf(f.x, f.x, fmaf(f.y, f.y, sq));
+                        }
+                    }
+                    iq = rsqrtf(sq + norm_eps);
+                }
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
                 tc::named_barrier(BAR_KK, kKKThreads);
                 // P_rs = e^{g_r - g_s} (Q K^T - d K K^T)_rs for s <= r, in place over K K^T
+                // (normalised q, k: e^{g_r - g_s} / |k_s| (Q K^T / |q_r| - d K K^T / |k_r|)_rs)
                 const uint32_t prow = pbm + ch * F32_ATOM;
                 if (fast) {
                     const float er = tc::lds_f32(ts + 1024 + 4u * r);
+                    const float dk = kGated ? dh * tc::lds_f32(ts + 1792 + 4u * r) : dh;
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         const uint32_t pa = prow + tc::sw128(r, c);
                         const float4 kk = tc::lds_f32x4(pa);
-                        const float4 ig = tc::lds_f32x4(ts + 1280 + 4u * (32 * ch + 4 * c));
+                        float4 ig = tc::lds_f32x4(ts + 1280 + 4u * (32 * ch + 4 * c));
+                        if constexpr (kGated) {
+                            const float4 k4 = tc::lds_f32x4(ts + 1792 + 4u * (32 * ch + 4 * c));
+                            ig.x *= k4.x; ig.y *= k4.y; ig.z *= k4.z; ig.w *= k4.w;
+                        }
                         const int s = 32 * ch + 4 * c;
                         float4 pv;
-                        pv.x = (s + 0 <= r) ? er * ig.x * fmaf(-dh, kk.x, gv[4 * c + 0]) : 0.f;
-                        pv.y = (s + 1 <= r) ? er * ig.y * fmaf(-dh, kk.y, gv[4 * c + 1]) : 0.f;
-                        pv.z = (s + 2 <= r) ? er * ig.z * fmaf(-dh, kk.z, gv[4 * c + 2]) : 0.f;
-                        pv.w = (s + 3 <= r) ? er * ig.w * fmaf(-dh, kk.w, gv[4 * c + 3]) : 0.f;
+                        if constexpr (kGated) {
+                            pv.x = (s + 0 <= r) ? er * ig.x * fmaf(-dk, kk.x, iq * gv[4 * c + 0]) : 0.f;
+                            pv.y = (s + 1 <= r) ? er * ig.y * fmaf(-dk, kk.y, iq * gv[4 * c + 1]) : 0.f;
+                            pv.z = (s + 2 <= r) ? er * ig.z * fmaf(-dk, kk.z, iq * gv[4 * c + 2]) : 0.f;
+                            pv.w = (s + 3 <= r) ? er * ig.w * fmaf(-dk, kk.w, iq * gv[4 * c + 3]) : 0.f;
+                        } else {
+                            pv.x = (s + 0 <= r) ? er * ig.x * fmaf(-dh, kk.x, gv[4 * c + 0]) : 0.f;
+                            pv.y = (s + 1 <= r) ? er * ig.y * fmaf(-dh, kk.y, gv[4 * c + 1]) : 0.f;
+                            pv.z = (s + 2 <= r) ? er * ig.z * fmaf(-dh, kk.z, gv[4 * c + 2]) : 0.f;
+                            pv.w = (s + 3 <= r) ? er * ig.w * fmaf(-dh, kk.w, gv[4 * c + 3]) : 0.f;
+                        }
                         tc::sts_f32x4(pa, pv);
                     }
                 } else {
-                    p_row_exact(prow, tl + tgm + 32 * ch, r, ch, dh, ts);
+                    p_row_exact<kGated>(prow, tl + tgm + 32 * ch, r, ch, dh, ts, ts + 1792, iq);
                 }
                 tc::fence_proxy_async_smem();
             } else {   // pw 5
@@ -999,8 +1062,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // the two longest strips (0, 1) on warps of schedulers 0 and 1 (warp % 4),
                 // the others spread so that each scheduler carries a similar MMA load
                 const int strip = (pw == 3) ? 0 : (pw == 0) ? 1 : (pw <= 2) ? pw + 1 : (pw == 4) ? 6 : pw - 1;
-                strip_inverse(F2p, F1, strip, lane, ts + 768, ts + 512);
-                if (pw == 4) strip_inverse(F2p, F1, 7, lane, ts + 768, ts + 512);
+                strip_inverse(F2p, F1, strip, lane, ts + 768, ts + 512, kGated ? ts + 1792 : 0u);
+                if (pw == 4) strip_inverse(F2p, F1, 7, lane, ts + 768, ts + 512, kGated ? ts + 1792 : 0u);
             }
             COMBA_PHASE(19);
             if (pt >= 128 && pt < 192) {   // diag(lo(beta))
