@@ -17,6 +17,9 @@ hand-worked example, brute-force transition products and invariants):
                          for the GPU; it pins the chunk algebra the kernels use
                          to the recurrence.
 * ``decode_steps``    -- repeated single-token steps (the recurrence at T=1).
+* ``recurrence_bwd_np`` -- gradients of the recurrence (reverse mode through the
+                         token loop, float64), pinned by finite differences of
+                         ``recurrence``, torch.autograd and a closed form;
 * ``gate_inputs``     -- the inputs of the recurrence from raw projections: q, k
                          L2-normalised per token and head, log_alpha and beta from
                          raw gate projections (a reading: the pages fix neither the
@@ -233,3 +236,80 @@ def gate_inputs(q_raw, k_raw, a_raw, b_raw, A_log, dt_bias, eps: float = 1e-6):
     log_alpha = -np.exp(A) * softplus
     beta = 1.0 / (1.0 + np.exp(-b))
     return q, k, log_alpha, beta
+
+
+def recurrence_bwd_np(q, k, v, log_alpha, beta, d, S0=None, dout=None, dS_final=None,
+                      checkpoint: int = 64):
+    """Gradients of the token-by-token recurrence, float64 (reverse-mode through the
+    definition, one token at a time).  The loss is <dout, out> + <dS_final, S_final>
+    (either cotangent may be None = 0).  The pages give no backward formulas (the
+    write-up's section "硬件高效的分块并行计算" says only that the backward pass
+    reuses the cached inverse and chunk states); these are the adjoint of
+
+        S_t = alpha_t S_{t-1} - beta_t (S_{t-1} k_t) k_t^T + beta_t v_t k_t^T
+        o_t = S_t qt_t,   qt_t = q_t - d_h k_t,   alpha_t = exp(log_alpha_t).
+
+    Going backwards with G = dL/dS_t (the future's gradient plus dout_t qt_t^T),
+    p = S_{t-1} k_t and u = G k_t:
+
+        dqt_t = S_t^T dout_t            dq_t = dqt_t,  dd_h -= dqt_t . k_t
+        dlog_alpha_t = alpha_t <G, S_{t-1}>
+        dbeta_t = u . (v_t - p)         dv_t = beta_t u
+        dk_t = beta_t (G^T (v_t - p) - S_{t-1}^T u) - d_h dqt_t
+        dL/dS_{t-1} = alpha_t G - beta_t u k_t^T
+
+    States S_{t-1} are recomputed forward from checkpoints every ``checkpoint``
+    tokens.  Returns a dict of float64 arrays: dq, dk [B,T,H,dk], dv [B,T,H,dv],
+    dlog_alpha, dbeta [B,T,H], dd [H], dS0 [B,H,dv,dk]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    la, be, d = _f64(log_alpha), _f64(beta), _f64(d)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    S = np.zeros((B, H, dv, dk)) if S0 is None else _f64(S0).copy()
+    dO = np.zeros((B, T, H, dv)) if dout is None else _f64(dout)
+    G = np.zeros((B, H, dv, dk)) if dS_final is None else _f64(dS_final).copy()
+    qt = q - d[None, None, :, None] * k
+    al = np.exp(la)
+
+    def step(S, t):
+        kt = k[:, t]
+        Sk = np.einsum("bhij,bhj->bhi", S, kt)
+        return (al[:, t][..., None, None] * S
+                - be[:, t][..., None, None] * np.einsum("bhi,bhj->bhij", Sk, kt)
+                + be[:, t][..., None, None] * np.einsum("bhi,bhj->bhij", v[:, t], kt))
+
+    # forward: the state before each checkpoint block
+    starts = []
+    for t in range(T):
+        if t % checkpoint == 0:
+            starts.append(S.copy())
+        S = step(S, t)
+    gq = np.zeros_like(q)
+    gk = np.zeros_like(k)
+    gv = np.zeros_like(v)
+    gla = np.zeros_like(la)
+    gbe = np.zeros_like(be)
+    gd = np.zeros(H)
+    for blk in range(len(starts) - 1, -1, -1):
+        t0, t1 = blk * checkpoint, min(T, (blk + 1) * checkpoint)
+        states = [starts[blk]]                    # states[i] = S_{t0 + i - 1}
+        for t in range(t0, t1):
+            states.append(step(states[-1], t))
+        for t in range(t1 - 1, t0 - 1, -1):
+            Sp, St = states[t - t0], states[t - t0 + 1]
+            kt, vt = k[:, t], v[:, t]
+            G = G + np.einsum("bhi,bhj->bhij", dO[:, t], qt[:, t])
+            dqt = np.einsum("bhij,bhi->bhj", St, dO[:, t])
+            gq[:, t] = dqt
+            gd -= np.einsum("bhj,bhj->h", dqt, kt)
+            p = np.einsum("bhij,bhj->bhi", Sp, kt)
+            u = np.einsum("bhij,bhj->bhi", G, kt)
+            r = vt - p
+            bt = be[:, t][..., None]
+            gla[:, t] = al[:, t] * np.einsum("bhij,bhij->bh", G, Sp)
+            gbe[:, t] = np.einsum("bhi,bhi->bh", u, r)
+            gv[:, t] = bt * u
+            gk[:, t] = (bt * (np.einsum("bhij,bhi->bhj", G, r) - np.einsum("bhij,bhi->bhj", Sp, u))
+                        - d[None, :, None] * dqt)
+            G = al[:, t][..., None, None] * G - be[:, t][..., None, None] * np.einsum("bhi,bhj->bhij", u, kt)
+    return {"dq": gq, "dk": gk, "dv": gv, "dlog_alpha": gla, "dbeta": gbe, "dd": gd, "dS0": G}
