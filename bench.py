@@ -33,7 +33,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from comba_workloads import (CONFIGS, DECODE, VARLEN, make_gated_inputs, make_varlen_inputs,  # noqa: E402
+from comba_workloads import (CONFIGS, DECODE, VARLEN, make_cotangents, make_gated_inputs, make_varlen_inputs,  # noqa: E402
                              decode_step_inputs, make_chunk_inputs,
                              make_decode_state)
 
@@ -559,6 +559,118 @@ def run_gated(args):
     print(json.dumps(line), flush=True)
 
 
+BWD = "layer1p3b_bwd_bf16"
+BWD_CHUNK = 32   # tokens per chunk of the backward kernels
+
+
+def bwd_algorithmic_flops(cfg):
+    """Multiply-add work of one backward over the workload, 2 flops per FMA, per
+    32-token chunk of every (b, h) chain.  It counts the products and triangular
+    solves the chunk adjoint performs, including recomputing the forward's W, U~,
+    X and P.
+      prep     K K^T, Q~ K^T, the two-column-block solve, P W, dO^T (Gamma Q~ - P W)
+      states   W S^T, X^T diag K
+      dstates  dS K^T, Z W
+      grads    K S^T, K K^T, K dS'^T, Q~ K^T, two solves, P^T dO, dR X^T, dO X^T,
+               dO S, X dS', dZ K, dZ^T Q~, (dY + dY^T) K, dR S"""
+    L, dk, dv = BWD_CHUNK, cfg.dk, cfg.dv
+    tri = L * (L - 1)                      # flops of one column of a unit-triangular solve
+    prep = 3 * 2 * L * L * dk + tri * (dk + dv) + 2 * dv * dk * L
+    states = 2 * (2 * L * dk * dv)
+    dstates = 2 * (2 * L * dk * dv)
+    grads = (5 * 2 * L * dv * dk + 2 * 2 * L * L * dk + 2 * tri * dv + 3 * 2 * L * L * dv
+             + 3 * 2 * L * L * dk)
+    chunks = cfg.B * cfg.H * ((cfg.T + L - 1) // L)
+    return chunks * (prep + states + dstates + grads)
+
+
+def fp32_alu_peak_tflops(sm_mhz: float, sms: int = 148) -> float:
+    """fp32 FMA peak: 148 SMs x 128 fp32 lanes x 2 flops x the SM clock."""
+    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def run_bwd(args):
+    """One step = one comba_chunk_bwd over the 1.3B layer (bf16 q, k, v, dout; fp32
+    gates, S0 and dS_final), inputs and cotangents resident in HBM."""
+    import chunk_delta_rule_b200 as cdr
+    cfg = CONFIGS["layer1p3b_bf16"]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    lib = cdr.library()
+    x = make_chunk_inputs(cfg)
+    x.update(make_cotangents(cfg))
+    host = {k: v.pin_memory() for k, v in x.items() if v is not None}
+    d_ = {k: v.to(dev) for k, v in host.items()}
+    stream = torch.cuda.current_stream(dev)
+    need = int(lib.comba_chunk_bwd_workspace_size(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv))
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    res = {}
+
+    def step():
+        res.update(cdr.chunk_bwd(d_["q"], d_["k"], d_["v"], d_["log_alpha"], d_["beta"], d_["d"], d_["dout"],
+                                 S0=d_.get("S0"), dS_final=d_.get("dS_final"), workspace=ws, stream=stream))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert cdr.get_last_error(dev) == 0
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(0).start()
+    th0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    th1 = time.time()
+    clocks.wait_after(th0)
+    clocks.stop()
+    ms_step = ev0.elapsed_time(ev1) / args.steps
+    if cdr.get_last_error(dev) != 0:
+        raise RuntimeError("device-side error during the timed region")
+    outs_h = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in res.items() if v is not None}
+
+    def e2e_step():
+        for k in host:
+            d_[k].copy_(host[k], non_blocking=True)
+        step()
+        for k in outs_h:
+            outs_h[k].copy_(res[k], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_e2e = ev0.elapsed_time(ev1) / args.steps
+    flops = bwd_algorithmic_flops(cfg)
+    ck = clocks.summary(th0, th1)
+    sm_max = ck.get("sm_max_mhz") or 1965.0
+    peak = fp32_alu_peak_tflops(sm_max)
+    tf = flops / (ms_step / 1e3) / 1e12
+    line = {
+        "metric": "Comba chunk-bwd tokens/s (all input gradients) on 1 B200, % of fp32 ALU roofline",
+        "value": cfg.B * cfg.T / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(config_record(cfg), workload=BWD, chunk=BWD_CHUNK, inputs="bf16 q, k, v, dout"),
+        "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                     "traffic": None,
+                     "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x max SM clock",
+                     "algorithmic_flops_per_launch": flops, "scope": "whole backward (5 kernels)"},
+        "e2e": {"value": cfg.B * cfg.T / (ms_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in host.values()),
+                "d2h_bytes_per_step": sum(v.numel() * v.element_size() for v in outs_h.values()),
+                "ms_per_step": ms_e2e},
+        "clocks": ck,
+        "gpu_launches": 5 * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -566,7 +678,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="layer1p3b_bf16",
-                    choices=sorted(CONFIGS) + [DECODE.name, VARLEN.name, GATED])
+                    choices=sorted(CONFIGS) + [DECODE.name, VARLEN.name, GATED, BWD])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -576,6 +688,12 @@ def main():
             print(json.dumps({"impl": "reference", "unavailable": "the decode workload has no reference arm; the headline workload does"}))
             return
         run_decode(args)
+        return
+    if args.workload == BWD:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the backward workload has no reference arm; the headline workload does"}))
+            return
+        run_bwd(args)
         return
     if args.workload == GATED:
         if args.impl == "reference":

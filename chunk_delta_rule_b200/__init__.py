@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["chunk_fwd", "chunk_fwd_gated", "chunk_fwd_host", "chunk_fwd_varlen", "chunk_fwd_noalloc",
+__all__ = ["chunk_fwd", "chunk_bwd", "chunk_fwd_gated", "chunk_fwd_host", "chunk_fwd_varlen", "chunk_fwd_noalloc",
            "recurrent_step",
            "get_last_error", "CombaError", "library", "library_path", "EXPORTS", "status_string"]
 
@@ -32,6 +32,7 @@ _lock = threading.Lock()
 EXPORTS = ("comba_chunk_fwd", "comba_chunk_fwd_f32", "comba_chunk_fwd_varlen",
            "comba_chunk_fwd_workspace_size", "comba_chunk_fwd_ws", "comba_chunk_fwd_noalloc",
            "comba_chunk_fwd_host", "comba_chunk_fwd_host_workspace_size", "comba_chunk_fwd_gated",
+           "comba_chunk_bwd", "comba_chunk_bwd_workspace_size",
            "comba_recurrent_step", "comba_recurrent_step_grouped", "comba_get_last_error",
            "comba_status_string", "comba_version")
 
@@ -69,11 +70,14 @@ def library():
             lib.comba_chunk_fwd_host_workspace_size.argtypes = [i] * 5
             lib.comba_chunk_fwd_host_workspace_size.restype = ctypes.c_size_t
             lib.comba_recurrent_step.argtypes = [vp] * 8 + [i] * 4 + [vp]
+            lib.comba_chunk_bwd.argtypes = [vp] * 16 + [i] * 6 + [vp, ctypes.c_size_t, vp]
+            lib.comba_chunk_bwd_workspace_size.argtypes = [i] * 5
+            lib.comba_chunk_bwd_workspace_size.restype = ctypes.c_size_t
             lib.comba_recurrent_step_grouped.argtypes = [vp] * 8 + [i] * 5 + [vp]
             for fn in (lib.comba_chunk_fwd, lib.comba_chunk_fwd_f32, lib.comba_chunk_fwd_ws,
                        lib.comba_chunk_fwd_noalloc, lib.comba_chunk_fwd_varlen,
                        lib.comba_recurrent_step_grouped, lib.comba_chunk_fwd_host,
-                       lib.comba_chunk_fwd_gated,
+                       lib.comba_chunk_fwd_gated, lib.comba_chunk_bwd,
                        lib.comba_recurrent_step, lib.comba_get_last_error, lib.comba_version):
                 fn.restype = ctypes.c_int
             lib.comba_get_last_error.argtypes = []
@@ -208,6 +212,65 @@ def chunk_fwd_gated(q_raw: torch.Tensor, k_raw: torch.Tensor, v: torch.Tensor, a
     if st != 0:
         raise CombaError(st, "comba_chunk_fwd_gated")
     return out, S_final
+
+
+_bwd_ws = {}
+
+
+def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+              beta: torch.Tensor, d: torch.Tensor, dout: torch.Tensor, S0: Optional[torch.Tensor] = None,
+              dS_final: Optional[torch.Tensor] = None, need_dd: bool = True, need_dS0: bool = True,
+              workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """comba_chunk_bwd: gradients of <dout, out> + <dS_final, S_final> of the chunk
+    forward with respect to q, k, v, log_alpha, beta, d and S0.  q, k [B,T,H,dk], v,
+    dout [B,T,H,dv]: all bf16 or all fp32; log_alpha, beta [B,T,H], d [H], S0 and
+    dS_final [B,H,dv,dk] (or None): fp32.  Returns a dict of fp32 tensors dq, dk, dv,
+    dlog_alpha, dbeta, dd (or None) and dS0 (or None).  ``workspace``: a uint8 device
+    tensor of at least comba_chunk_bwd_workspace_size bytes; by default one is kept per
+    device and grown as needed (it must not be shared by calls in flight on different
+    streams)."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("q, k, v, dout must be bf16 or fp32")
+    dt = q.dtype
+    _check(q, "q", dt, (B, T, H, dk))
+    _check(k, "k", dt, (B, T, H, dk))
+    _check(v, "v", dt, (B, T, H, dv))
+    _check(dout, "dout", dt, (B, T, H, dv))
+    _check(log_alpha, "log_alpha", torch.float32, (B, T, H))
+    _check(beta, "beta", torch.float32, (B, T, H))
+    _check(d, "d", torch.float32, (H,))
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (B, H, dv, dk))
+    if dS_final is not None:
+        _check(dS_final, "dS_final", torch.float32, (B, H, dv, dk))
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = {"dq": torch.empty((B, T, H, dk), **f32), "dk": torch.empty((B, T, H, dk), **f32),
+         "dv": torch.empty((B, T, H, dv), **f32), "dlog_alpha": torch.empty((B, T, H), **f32),
+         "dbeta": torch.empty((B, T, H), **f32),
+         "dd": torch.empty((H,), **f32) if need_dd else None,
+         "dS0": torch.empty((B, H, dv, dk), **f32) if need_dS0 else None}
+    lib = library()
+    need = int(lib.comba_chunk_bwd_workspace_size(B, T, H, dk, dv))
+    if workspace is None:
+        key = dev.index if dev.index is not None else torch.cuda.current_device()
+        workspace = _bwd_ws.get(key)
+        if workspace is None or workspace.numel() < need:
+            workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+            _bwd_ws[key] = workspace
+    with torch.cuda.device(dev):
+        st = lib.comba_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(d), _ptr(S0),
+                                 _ptr(dout), _ptr(dS_final), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                                 _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]), _ptr(g["dd"]), _ptr(g["dS0"]),
+                                 B, T, H, dk, dv, 0 if dt == torch.bfloat16 else 1, _ptr(workspace),
+                                 workspace.numel(), _stream_handle(dev, stream))
+    if st != 0:
+        raise CombaError(st, "comba_chunk_bwd")
+    return g
 
 
 _host_ws = {}

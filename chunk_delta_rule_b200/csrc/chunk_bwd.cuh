@@ -1,0 +1,577 @@
+// Chunk-wise Comba backward: gradients of the chunk forward with respect to q, k, v,
+// log_alpha, beta, d and S0, given the cotangents of out and S_final.  fp32 FMA
+// arithmetic throughout.
+//
+// The write-up (section "硬件高效的分块并行计算") says only that the backward pass
+// reuses the chunk-level states and the single inverse per chunk.  The algebra
+// below is the adjoint of the chunk form the forward kernels use.  It uses
+// chunk-local positions r, s, g_r = sum_{i<=r} log_alpha_i, g'_r = g_{r-1}
+// (g'_0 = 0) and Gamma = diag(e^{g_r}), and gives every chunk
+//   AF_rs = e^{g'_r - g_s} (k_r.k_s) (s < r),   A = diag(beta) AF,   T = (I + A)^{-1}
+//   W = T diag(beta e^{g'}) K,   U~ = T diag(beta) V,   X = U~ - W S^T
+//   P_rs = e^{g_r - g_s} (q~_r.k_s) (s <= r),    q~ = q - d k
+//   O = Gamma Q~ S^T + P X,      S' = e^{g_L} S + X^T diag(e^{g_L - g}) K.
+// Going backwards, with dS' the gradient at the chunk's end state:
+//   dS  = dS' (e^{g_L} I - K^T diag(e^{g_L - g}) W) + dO^T (Gamma Q~ - P W)
+//   dX  = P^T dO + diag(e^{g_L - g}) K dS'^T,     dR = T^T dX
+//   dA  = -(dR X^T) strictly lower,               dP = (dO X^T) lower incl. diagonal
+//   dq~ = Gamma dO S + (dP o E) K                  (E_rs = e^{g_r - g_s})
+//   dk  = (dP o E)^T Q~ - diag(beta e^{g'}) dR S + (dY + dY^T) K
+//         + diag(e^{g_L - g}) X dS' - d dq~,        dY = dA o (beta_r e^{g'_r - g_s})
+//   dv  = diag(beta) dR,    dbeta_r = dR_r.(v_r - e^{g'_r} S k_r) + sum_s dA_rs AF_rs
+// and the decay gradients collect every exponent's sensitivity into dg_r, then
+// dlog_alpha_i = sum_{r >= i} dg_r inside the chunk.
+//
+// Four kernels, all over a fixed 32-token chunk (a tiling choice: the gradients are
+// the same function of the inputs for any chunk length):
+//   bwd_prep     (chunk, chain) in parallel: W, U~ and C = dO^T (Gamma Q~ - P W)
+//   bwd_states   one CTA per chain, chunks in order: chunk-start states S_c
+//   bwd_dstates  one CTA per chain, chunks in reverse: end-state gradients dS'_c, dS0
+//   bwd_grads    (chunk, chain) in parallel: dq, dk, dv, dlog_alpha, dbeta and a
+//                per-chunk partial of dd
+// plus bwd_dd_sum, which adds the dd partials per head in a fixed order.
+#pragma once
+
+#include "common.cuh"
+
+namespace comba {
+namespace bwd {
+
+constexpr int kL = 32;           // tokens per backward chunk (one warp's lanes)
+constexpr int kLDL = kL + 1;     // padded row stride of the L x L tiles
+constexpr int kThreads = 256;
+
+// Per-chain workspace, chunk-major: W [L, dk], U~ [L, dv], C [dv, dk], S_c [dv, dk],
+// dS'_c [dv, dk] per chunk, then one dd partial per chunk.
+struct Workspace {
+    float *W, *U, *C, *S, *dS, *ddp;
+};
+
+__host__ __device__ inline size_t workspace_floats(long chains, int nch, int dk, int dv) {
+    return (size_t)chains * nch * ((size_t)kL * (dk + dv) + 3 * (size_t)dk * dv + 1);
+}
+
+__host__ __device__ inline Workspace carve(float* base, long chains, int nch, int dk, int dv) {
+    const size_t n = (size_t)chains * nch;
+    Workspace w;
+    w.W = base;
+    w.U = w.W + n * kL * dk;
+    w.C = w.U + n * kL * dv;
+    w.S = w.C + n * (size_t)dv * dk;
+    w.dS = w.S + n * (size_t)dv * dk;
+    w.ddp = w.dS + n * (size_t)dv * dk;
+    return w;
+}
+
+// C(m, n) = sum_k a(m, k) b(k, n) for m < M, n < N, handed to epi(m, n, c).  Thread t
+// owns rows mt + i (M / TM) and columns nt + j (N / TN), (mt, nt) = (t / (N / TN),
+// t % (N / TN)): neighbouring threads take neighbouring columns, so row-major
+// operands read with stride 1 and transposed ones with an odd padded stride hit
+// distinct banks, and an operand indexed by the row alone is a broadcast.  The
+// ownership depends only on <M, N, TM, TN>, so calls with the same tiling may
+// accumulate into one buffer without a barrier between them.
+template <int M, int N, int K, int TM, int TN, typename FA, typename FB, typename Epi>
+__device__ __forceinline__ void bgemm(const FA& a, const FB& b, const Epi& epi) {
+    static_assert(M % TM == 0 && N % TN == 0, "tile must divide the product");
+    constexpr int MS = M / TM, NS = N / TN, TILES = MS * NS;
+    for (int t = threadIdx.x; t < TILES; t += kThreads) {
+        const int mt = t / NS, nt = t % NS;
+        float acc[TM][TN];
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+#pragma unroll
+            for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+        for (int k = 0; k < K; ++k) {
+            float av[TM], bv[TN];
+#pragma unroll
+            for (int i = 0; i < TM; ++i) av[i] = a(mt + i * MS, k);
+#pragma unroll
+            for (int j = 0; j < TN; ++j) bv[j] = b(k, nt + j * NS);
+#pragma unroll
+            for (int i = 0; i < TM; ++i)
+#pragma unroll
+                for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+#pragma unroll
+            for (int j = 0; j < TN; ++j) epi(mt + i * MS, nt + j * NS, acc[i][j]);
+    }
+}
+
+// Chunk-local decay prefix of chunk c (warp 0): g_r = sum_{i<=r} log_alpha_i over
+// the chunk's tokens (0 past the end of the sequence), g'_r = g_{r-1}.
+__device__ __forceinline__ void chunk_decays(const float* __restrict__ log_alpha, const float* __restrict__ beta,
+                                             size_t row0, int H, int Lc, float* g, float* gp, float* bt) {
+    if (threadIdx.x < 32) {
+        const int r = threadIdx.x;
+        const float la = (r < Lc) ? log_alpha[row0 + (size_t)r * H] : 0.f;
+        float x = la;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, o);
+            if (r >= o) x += y;
+        }
+        const float prev = __shfl_up_sync(0xffffffffu, x, 1);
+        g[r] = x;
+        gp[r] = (r == 0) ? 0.f : prev;
+        bt[r] = (r < Lc) ? beta[row0 + (size_t)r * H] : 0.f;
+    }
+}
+
+// rows [L, D] of a [B, T, H, D] tensor into shared memory (stride ld), zero past Lc
+template <int D, typename Tin>
+__device__ __forceinline__ void load_rows(float* dst, int ld, const Tin* __restrict__ src, size_t row0, int H,
+                                          int Lc) {
+    for (int e = threadIdx.x; e < kL * D; e += kThreads) {
+        const int r = e / D, c = e % D;
+        dst[r * ld + c] = (r < Lc) ? to_f32(src[(row0 + (size_t)r * H) * D + c]) : 0.f;
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// bwd_prep: W, U~ and C = dO^T (Gamma Q~ - P W) of one chunk.
+template <typename Tin, int DK, int DV>
+struct PrepSmem {
+    static constexpr int LDK = DK + 1, LDV = DV + 1;
+    static constexpr size_t K = 0, Q = K + kL * LDK, V = Q + kL * LDK, O = V + kL * LDV, A = O + kL * LDV,
+                            P = A + kL * kLDL, G = P + kL * kLDL, GP = G + kL, BT = GP + kL, CW = BT + kL,
+                            total = CW + kL;
+};
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(kThreads)
+bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+                const float* __restrict__ log_alpha, const float* __restrict__ beta, const float* __restrict__ d,
+                const Tin* __restrict__ dout, Workspace ws, int T, int H, int nch) {
+    using SM = PrepSmem<Tin, DK, DV>;
+    constexpr int LDK = SM::LDK, LDV = SM::LDV;
+    extern __shared__ float sm[];
+    float *Ks = sm + SM::K, *Qs = sm + SM::Q, *Vs = sm + SM::V, *Os = sm + SM::O;
+    float *Am = sm + SM::A, *Pm = sm + SM::P, *g = sm + SM::G, *gp = sm + SM::GP, *bt = sm + SM::BT,
+          *cw = sm + SM::CW;
+    const int c = blockIdx.x, bh = blockIdx.y, b = bh / H, h = bh % H;
+    const int t0 = c * kL, Lc = min(kL, T - t0);
+    const size_t row0 = ((size_t)b * T + t0) * H + h;
+    const float dh = d[h];
+    load_rows<DK>(Ks, LDK, k, row0, H, Lc);
+    load_rows<DK>(Qs, LDK, q, row0, H, Lc);
+    load_rows<DV>(Vs, LDV, v, row0, H, Lc);
+    load_rows<DV>(Os, LDV, dout, row0, H, Lc);
+    chunk_decays(log_alpha, beta, row0, H, Lc, g, gp, bt);
+    __syncthreads();
+    for (int e = threadIdx.x; e < kL * DK; e += kThreads) {   // q~ = q - d k
+        const int r = e / DK, j = e % DK;
+        Qs[r * LDK + j] = fmaf(-dh, Ks[r * LDK + j], Qs[r * LDK + j]);
+    }
+    if (threadIdx.x < kL) cw[threadIdx.x] = bt[threadIdx.x] * expf(gp[threadIdx.x]);
+    // A = diag(beta) AF (strictly lower) and P, both from the raw k rows
+    bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Ks[m * LDK + x]; },
+                            [&](int x, int n) { return Ks[n * LDK + x]; },
+                            [&](int m, int n, float s) {
+                                Am[m * kLDL + n] = (n < m) ? bt[m] * expf(gp[m] - g[n]) * s : 0.f;
+                            });
+    __syncthreads();   // q~ complete
+    bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Qs[m * LDK + x]; },
+                            [&](int x, int n) { return Ks[n * LDK + x]; },
+                            [&](int m, int n, float s) { Pm[m * kLDL + n] = (n <= m) ? expf(g[m] - g[n]) * s : 0.f; });
+    __syncthreads();
+    // [W | U~] = (I + A)^{-1} [diag(beta e^{g'}) K | diag(beta) V]: one column per
+    // thread, forward substitution down the column, in place over K and V
+    for (int col = threadIdx.x; col < DK + DV; col += kThreads) {
+        float* base = (col < DK) ? Ks + col : Vs + (col - DK);
+        const int ld = (col < DK) ? LDK : LDV;
+        float x[kL];
+#pragma unroll
+        for (int r = 0; r < kL; ++r) {
+            float acc = ((col < DK) ? cw[r] : bt[r]) * base[r * ld];
+#pragma unroll
+            for (int s = 0; s < r; ++s) acc = fmaf(-Am[r * kLDL + s], x[s], acc);
+            x[r] = acc;
+        }
+#pragma unroll
+        for (int r = 0; r < kL; ++r) base[r * ld] = x[r];
+    }
+    __syncthreads();
+    // Gamma Q~ - P W, in place over Q~
+    bgemm<kL, DK, kL, 2, 4>([&](int m, int x) { return Pm[m * kLDL + x]; },
+                            [&](int x, int n) { return Ks[x * LDK + n]; },
+                            [&](int m, int n, float s) { Qs[m * LDK + n] = fmaf(expf(g[m]), Qs[m * LDK + n], -s); });
+    __syncthreads();
+    const size_t ci = (size_t)bh * nch + c;
+    float* Cg = ws.C + ci * DV * DK;
+    bgemm<DV, DK, kL, 8, 8>([&](int i, int r) { return Os[r * LDV + i]; },
+                            [&](int r, int j) { return Qs[r * LDK + j]; },
+                            [&](int i, int j, float s) { Cg[(size_t)i * DK + j] = s; });
+    float* Wg = ws.W + ci * kL * DK;
+    float* Ug = ws.U + ci * kL * DV;
+    for (int e = threadIdx.x; e < kL * DK; e += kThreads) Wg[e] = Ks[(e / DK) * LDK + e % DK];
+    for (int e = threadIdx.x; e < kL * DV; e += kThreads) Ug[e] = Vs[(e / DV) * LDV + e % DV];
+}
+
+// ---------------------------------------------------------------------------------
+// bwd_states: S_c for every chunk of one chain (S_0 = S0), from W and U~:
+//   X = U~ - W S^T,   S <- e^{g_L} S + X^T diag(e^{g_L - g}) K.
+template <int DK, int DV>
+struct StatesSmem {
+    static constexpr int LDK = DK + 1, LDV = DV + 1;
+    static constexpr size_t S = 0, W = S + DV * LDK, U = W + kL * LDK, K = U + kL * LDV, G = K + kL * LDK,
+                            GP = G + kL, BT = GP + kL, DEC = BT + kL, total = DEC + kL;
+};
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(kThreads)
+bwd_states_kernel(const Tin* __restrict__ k, const float* __restrict__ log_alpha, const float* __restrict__ beta,
+                  const float* __restrict__ S0, Workspace ws, int T, int H, int nch) {
+    using SM = StatesSmem<DK, DV>;
+    constexpr int LDK = SM::LDK, LDV = SM::LDV;
+    extern __shared__ float sm[];
+    float *S = sm + SM::S, *Ws = sm + SM::W, *Us = sm + SM::U, *Ks = sm + SM::K;
+    float *g = sm + SM::G, *gp = sm + SM::GP, *bt = sm + SM::BT, *dec = sm + SM::DEC;
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const float* s0 = S0 ? S0 + (size_t)bh * DV * DK : nullptr;
+    for (int e = threadIdx.x; e < DV * DK; e += kThreads) S[(e / DK) * LDK + e % DK] = s0 ? s0[e] : 0.f;
+    for (int c = 0; c < nch; ++c) {
+        const int t0 = c * kL, Lc = min(kL, T - t0);
+        const size_t row0 = ((size_t)b * T + t0) * H + h, ci = (size_t)bh * nch + c;
+        const float* Wg = ws.W + ci * kL * DK;
+        const float* Ug = ws.U + ci * kL * DV;
+        for (int e = threadIdx.x; e < kL * DK; e += kThreads) Ws[(e / DK) * LDK + e % DK] = Wg[e];
+        for (int e = threadIdx.x; e < kL * DV; e += kThreads) Us[(e / DV) * LDV + e % DV] = Ug[e];
+        load_rows<DK>(Ks, LDK, k, row0, H, Lc);
+        chunk_decays(log_alpha, beta, row0, H, Lc, g, gp, bt);
+        __syncthreads();   // S of this chunk (previous iteration) and its tiles are in place
+        float* Sg = ws.S + ci * DV * DK;
+        for (int e = threadIdx.x; e < DV * DK; e += kThreads) Sg[e] = S[(e / DK) * LDK + e % DK];
+        if (threadIdx.x < kL) dec[threadIdx.x] = expf(g[kL - 1] - g[threadIdx.x]);
+        bgemm<kL, DV, DK, 2, 4>([&](int r, int j) { return Ws[r * LDK + j]; },
+                                [&](int j, int i) { return S[i * LDK + j]; },
+                                [&](int r, int i, float s) { Us[r * LDV + i] -= s; });
+        __syncthreads();
+        const float eL = expf(g[kL - 1]);
+        bgemm<DV, DK, kL, 8, 8>([&](int i, int r) { return Us[r * LDV + i] * dec[r]; },
+                                [&](int r, int j) { return Ks[r * LDK + j]; },
+                                [&](int i, int j, float s) { S[i * LDK + j] = fmaf(eL, S[i * LDK + j], s); });
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// bwd_dstates: end-state gradients dS'_c of every chunk of one chain, last chunk
+// first (dS'_{last} = dS_final), and dS0:
+//   dS <- e^{g_L} dS - (dS K^T diag(e^{g_L - g})) W + C.
+template <int DK, int DV>
+struct DStatesSmem {
+    static constexpr int LDK = DK + 1;
+    static constexpr size_t S = 0, W = S + DV * LDK, K = W + kL * LDK, Z = K + kL * LDK, G = Z + DV * kLDL,
+                            GP = G + kL, BT = GP + kL, DEC = BT + kL, total = DEC + kL;
+};
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(kThreads)
+bwd_dstates_kernel(const Tin* __restrict__ k, const float* __restrict__ log_alpha, const float* __restrict__ beta,
+                   const float* __restrict__ dS_final, float* __restrict__ dS0, Workspace ws, int T, int H,
+                   int nch) {
+    using SM = DStatesSmem<DK, DV>;
+    constexpr int LDK = SM::LDK;
+    extern __shared__ float sm[];
+    float *dS = sm + SM::S, *Ws = sm + SM::W, *Ks = sm + SM::K, *Z = sm + SM::Z;
+    float *g = sm + SM::G, *gp = sm + SM::GP, *bt = sm + SM::BT, *dec = sm + SM::DEC;
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const float* df = dS_final ? dS_final + (size_t)bh * DV * DK : nullptr;
+    for (int e = threadIdx.x; e < DV * DK; e += kThreads) dS[(e / DK) * LDK + e % DK] = df ? df[e] : 0.f;
+    for (int c = nch - 1; c >= 0; --c) {
+        const int t0 = c * kL, Lc = min(kL, T - t0);
+        const size_t row0 = ((size_t)b * T + t0) * H + h, ci = (size_t)bh * nch + c;
+        const float* Wg = ws.W + ci * kL * DK;
+        for (int e = threadIdx.x; e < kL * DK; e += kThreads) Ws[(e / DK) * LDK + e % DK] = Wg[e];
+        load_rows<DK>(Ks, LDK, k, row0, H, Lc);
+        chunk_decays(log_alpha, beta, row0, H, Lc, g, gp, bt);
+        __syncthreads();
+        float* dSg = ws.dS + ci * DV * DK;
+        for (int e = threadIdx.x; e < DV * DK; e += kThreads) dSg[e] = dS[(e / DK) * LDK + e % DK];
+        if (threadIdx.x < kL) dec[threadIdx.x] = expf(g[kL - 1] - g[threadIdx.x]);
+        __syncthreads();
+        bgemm<DV, kL, DK, 4, 1>([&](int i, int j) { return dS[i * LDK + j]; },
+                                [&](int j, int r) { return Ks[r * LDK + j]; },
+                                [&](int i, int r, float s) { Z[i * kLDL + r] = dec[r] * s; });
+        __syncthreads();
+        const float eL = expf(g[kL - 1]);
+        const float* Cg = ws.C + ci * DV * DK;
+        bgemm<DV, DK, kL, 8, 8>([&](int i, int r) { return Z[i * kLDL + r]; },
+                                [&](int r, int j) { return Ws[r * LDK + j]; },
+                                [&](int i, int j, float s) {
+                                    dS[i * LDK + j] = fmaf(eL, dS[i * LDK + j], Cg[(size_t)i * DK + j] - s);
+                                });
+        __syncthreads();
+    }
+    if (dS0)
+        for (int e = threadIdx.x; e < DV * DK; e += kThreads)
+            dS0[(size_t)bh * DV * DK + e] = dS[(e / DK) * LDK + e % DK];
+}
+
+// ---------------------------------------------------------------------------------
+// bwd_grads: every input gradient of one chunk, from S_c and dS'_c.
+template <int DK, int DV>
+struct GradSmem {
+    static constexpr int DM = (DK > DV ? DK : DV), LD = DM + 1;
+    static constexpr int NV = 24;   // per-row vectors
+    // [L, LD] tiles: K, Q~, dO, V, KS^T (then F), X, dX (then dR), Gamma dO S (then dq~), dk
+    static constexpr size_t K = 0, Q = K + kL * LD, O = Q + kL * LD, V = O + kL * LD, R = V + kL * LD,
+                            X = R + kL * LD, D = X + kL * LD, G = D + kL * LD, TK = G + kL * LD,
+                            AF = TK + kL * LD, P = AF + kL * kLDL, DP = P + kL * kLDL, DA = DP + kL * kLDL,
+                            VEC = DA + kL * kLDL, RED = VEC + NV * kL, total = RED + kThreads / 32;
+};
+
+enum { V_G, V_GP, V_BT, V_EG, V_EGP, V_DEC, V_T1, V_T2, V_ROWA, V_COLA, V_ROWP, V_COLP, V_QG, V_F, V_DQK, V_DG };
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(kThreads)
+bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+                 const float* __restrict__ log_alpha, const float* __restrict__ beta, const float* __restrict__ d,
+                 const Tin* __restrict__ dout, float* __restrict__ dq, float* __restrict__ dk,
+                 float* __restrict__ dv, float* __restrict__ dlog_alpha, float* __restrict__ dbeta, Workspace ws,
+                 int T, int H, int nch) {
+    using SM = GradSmem<DK, DV>;
+    constexpr int LD = SM::LD;
+    extern __shared__ float sm[];
+    float *Ks = sm + SM::K, *Qs = sm + SM::Q, *Os = sm + SM::O, *Vs = sm + SM::V, *Rs = sm + SM::R;
+    float *Xs = sm + SM::X, *Ds = sm + SM::D, *Gs = sm + SM::G, *TKs = sm + SM::TK;
+    float *AF = sm + SM::AF, *Pm = sm + SM::P, *dPm = sm + SM::DP, *dAm = sm + SM::DA;
+    float* vec = sm + SM::VEC;
+    float* red = sm + SM::RED;
+    auto V_ = [&](int which) { return vec + which * kL; };
+    float *g = V_(V_G), *gp = V_(V_GP), *bt = V_(V_BT), *eg = V_(V_EG), *egp = V_(V_EGP), *dec = V_(V_DEC);
+    const int c = blockIdx.x, bh = blockIdx.y, b = bh / H, h = bh % H, tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int t0 = c * kL, Lc = min(kL, T - t0);
+    const size_t row0 = ((size_t)b * T + t0) * H + h, ci = (size_t)bh * nch + c;
+    const float dh = d[h];
+    const float* S = ws.S + ci * DV * DK;      // chunk-start state
+    const float* dSp = ws.dS + ci * DV * DK;   // gradient at the chunk's end state
+
+    // 1. tiles and decays
+    load_rows<DK>(Ks, LD, k, row0, H, Lc);
+    load_rows<DK>(Qs, LD, q, row0, H, Lc);
+    load_rows<DV>(Os, LD, dout, row0, H, Lc);
+    load_rows<DV>(Vs, LD, v, row0, H, Lc);
+    chunk_decays(log_alpha, beta, row0, H, Lc, g, gp, bt);
+    __syncthreads();
+    for (int e = tid; e < kL * DK; e += kThreads) {
+        const int r = e / DK, j = e % DK;
+        Qs[r * LD + j] = fmaf(-dh, Ks[r * LD + j], Qs[r * LD + j]);
+    }
+    if (tid < kL) {
+        eg[tid] = expf(g[tid]);
+        egp[tid] = expf(gp[tid]);
+        dec[tid] = expf(g[kL - 1] - g[tid]);
+    }
+    // 2. K S^T, AF, dX = diag(e^{g_L - g}) K dS'^T (P^T dO added below)
+    bgemm<DV, kL, DK, 4, 1>([&](int i, int j) { return S[(size_t)i * DK + j]; },
+                            [&](int j, int r) { return Ks[r * LD + j]; },
+                            [&](int i, int r, float s) { Rs[r * LD + i] = s; });
+    bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Ks[m * LD + x]; },
+                            [&](int x, int n) { return Ks[n * LD + x]; },
+                            [&](int m, int n, float s) { AF[m * kLDL + n] = (n < m) ? expf(gp[m] - g[n]) * s : 0.f; });
+    __syncthreads();   // q~, decays
+    bgemm<DV, kL, DK, 4, 1>([&](int i, int j) { return dSp[(size_t)i * DK + j]; },
+                            [&](int j, int r) { return Ks[r * LD + j]; },
+                            [&](int i, int r, float s) { Ds[r * LD + i] = dec[r] * s; });
+    bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Qs[m * LD + x]; },
+                            [&](int x, int n) { return Ks[n * LD + x]; },
+                            [&](int m, int n, float s) { Pm[m * kLDL + n] = (n <= m) ? expf(g[m] - g[n]) * s : 0.f; });
+    __syncthreads();
+    // 3. X = T diag(beta) (V - diag(e^{g'}) K S^T) by forward substitution (one column
+    //    per thread); dX += P^T dO
+    for (int col = tid; col < DV; col += kThreads) {
+        float x[kL];
+#pragma unroll
+        for (int r = 0; r < kL; ++r) {
+            float acc = bt[r] * fmaf(-egp[r], Rs[r * LD + col], Vs[r * LD + col]);
+#pragma unroll
+            for (int s = 0; s < r; ++s) acc = fmaf(-bt[r] * AF[r * kLDL + s], x[s], acc);
+            x[r] = acc;
+        }
+#pragma unroll
+        for (int r = 0; r < kL; ++r) Xs[r * LD + col] = x[r];
+    }
+    bgemm<kL, DV, kL, 2, 4>([&](int r, int s) { return Pm[s * kLDL + r]; },
+                            [&](int s, int i) { return Os[s * LD + i]; },
+                            [&](int r, int i, float s) { Ds[r * LD + i] += s; });
+    __syncthreads();
+    // 4. dR = T^T dX by back substitution, in place
+    for (int col = tid; col < DV; col += kThreads) {
+        float x[kL];
+#pragma unroll
+        for (int r = kL - 1; r >= 0; --r) {
+            float acc = Ds[r * LD + col];
+#pragma unroll
+            for (int s = r + 1; s < kL; ++s) acc = fmaf(-bt[s] * AF[s * kLDL + r], x[s], acc);
+            x[r] = acc;
+        }
+#pragma unroll
+        for (int r = 0; r < kL; ++r) Ds[r * LD + col] = x[r];
+    }
+    __syncthreads();
+    // 5. dA, dP; row dots dR.(V - e^{g'} K S^T) and dR.(K S^T); Gamma dO S
+    bgemm<kL, kL, DV, 4, 1>([&](int r, int i) { return Ds[r * LD + i]; },
+                            [&](int i, int s) { return Xs[s * LD + i]; },
+                            [&](int r, int s, float x) { dAm[r * kLDL + s] = (s < r) ? -x : 0.f; });
+    bgemm<kL, kL, DV, 4, 1>([&](int r, int i) { return Os[r * LD + i]; },
+                            [&](int i, int s) { return Xs[s * LD + i]; },
+                            [&](int r, int s, float x) { dPm[r * kLDL + s] = (s <= r) ? x : 0.f; });
+    for (int r = warp; r < kL; r += kThreads / 32) {
+        float t1 = 0.f, t2 = 0.f;
+        for (int i = lane; i < DV; i += 32) {
+            const float dr = Ds[r * LD + i], ks = Rs[r * LD + i];
+            t1 = fmaf(dr, fmaf(-egp[r], ks, Vs[r * LD + i]), t1);
+            t2 = fmaf(dr, ks, t2);
+        }
+        t1 = warp_sum(t1);
+        t2 = warp_sum(t2);
+        if (lane == 0) {
+            V_(V_T1)[r] = t1;
+            V_(V_T2)[r] = t2;
+        }
+    }
+    bgemm<kL, DK, DV, 2, 4>([&](int r, int i) { return Os[r * LD + i]; },
+                            [&](int i, int j) { return S[(size_t)i * DK + j]; },
+                            [&](int r, int j, float s) { Gs[r * LD + j] = eg[r] * s; });
+    __syncthreads();
+    // 6. F = diag(e^{g_L - g}) X dS' (over K S^T); sums of dA o AF and dP o P by row
+    //    and column; q~_r . (Gamma dO S)_r
+    bgemm<kL, DK, DV, 2, 4>([&](int s, int i) { return Xs[s * LD + i]; },
+                            [&](int i, int j) { return dSp[(size_t)i * DK + j]; },
+                            [&](int s, int j, float x) { Rs[s * LD + j] = dec[s] * x; });
+    if (tid < kL) {
+        const int r = tid;
+        float ra = 0.f, rp = 0.f;
+        for (int s = 0; s < kL; ++s) {
+            ra = fmaf(dAm[r * kLDL + s], AF[r * kLDL + s], ra);
+            rp = fmaf(dPm[r * kLDL + s], Pm[r * kLDL + s], rp);
+        }
+        V_(V_ROWA)[r] = ra;
+        V_(V_ROWP)[r] = rp;
+    } else if (tid < 2 * kL) {
+        const int s = tid - kL;
+        float ca = 0.f, cp = 0.f;
+        for (int r = 0; r < kL; ++r) {
+            ca = fmaf(dAm[r * kLDL + s] * bt[r], AF[r * kLDL + s], ca);
+            cp = fmaf(dPm[r * kLDL + s], Pm[r * kLDL + s], cp);
+        }
+        V_(V_COLA)[s] = ca;
+        V_(V_COLP)[s] = cp;
+    }
+    for (int r = warp; r < kL; r += kThreads / 32) {
+        float x = 0.f;
+        for (int j = lane; j < DK; j += 32) x = fmaf(Qs[r * LD + j], Gs[r * LD + j], x);
+        x = warp_sum(x);
+        if (lane == 0) V_(V_QG)[r] = x;
+    }
+    __syncthreads();
+    // 7. dP -> dZ = dP o E, dA -> dY = dA o (beta_r e^{g'_r - g_s}); f_s = F_s . k_s
+    for (int e = tid; e < kL * kL; e += kThreads) {
+        const int r = e / kL, s = e % kL;
+        dPm[r * kLDL + s] = (s <= r) ? dPm[r * kLDL + s] * expf(g[r] - g[s]) : 0.f;
+        dAm[r * kLDL + s] = (s < r) ? dAm[r * kLDL + s] * bt[r] * expf(gp[r] - g[s]) : 0.f;
+    }
+    for (int r = warp; r < kL; r += kThreads / 32) {
+        float x = 0.f;
+        for (int j = lane; j < DK; j += 32) x = fmaf(Rs[r * LD + j], Ks[r * LD + j], x);
+        x = warp_sum(x);
+        if (lane == 0) V_(V_F)[r] = x;
+    }
+    __syncthreads();
+    // 8. dq~ = Gamma dO S + dZ K;  dk (without F and -d dq~) =
+    //    dZ^T Q~ + (dY + dY^T) K - diag(beta e^{g'}) dR S
+    bgemm<kL, DK, kL, 2, 4>([&](int r, int s) { return dPm[r * kLDL + s]; },
+                            [&](int s, int j) { return Ks[s * LD + j]; },
+                            [&](int r, int j, float x) { Gs[r * LD + j] += x; });
+    bgemm<kL, DK, kL, 2, 4>([&](int r, int s) { return dPm[s * kLDL + r]; },
+                            [&](int s, int j) { return Qs[s * LD + j]; },
+                            [&](int r, int j, float x) { TKs[r * LD + j] = x; });
+    bgemm<kL, DK, kL, 2, 4>([&](int r, int s) { return dAm[r * kLDL + s] + dAm[s * kLDL + r]; },
+                            [&](int s, int j) { return Ks[s * LD + j]; },
+                            [&](int r, int j, float x) { TKs[r * LD + j] += x; });
+    bgemm<kL, DK, DV, 2, 4>([&](int r, int i) { return Ds[r * LD + i]; },
+                            [&](int i, int j) { return S[(size_t)i * DK + j]; },
+                            [&](int r, int j, float x) { TKs[r * LD + j] = fmaf(-bt[r] * egp[r], x, TKs[r * LD + j]); });
+    __syncthreads();
+    // 9. outputs: dq, dk, dv; decay gradients; dd partial
+    for (int e = tid; e < Lc * DK; e += kThreads) {
+        const int r = e / DK, j = e % DK;
+        const size_t o = (row0 + (size_t)r * H) * DK + j;
+        const float dqt = Gs[r * LD + j];
+        dq[o] = dqt;
+        dk[o] = fmaf(-dh, dqt, TKs[r * LD + j] + Rs[r * LD + j]);
+    }
+    for (int e = tid; e < Lc * DV; e += kThreads) {
+        const int r = e / DV, i = e % DV;
+        dv[(row0 + (size_t)r * H) * DV + i] = bt[r] * Ds[r * LD + i];
+    }
+    // <dS', S> and sum_r dq~_r . k_r (block sums in a fixed order)
+    float ss = 0.f;
+    for (int e = tid; e < DV * DK; e += kThreads) ss = fmaf(dSp[e], S[e], ss);
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    for (int r = warp; r < kL; r += kThreads / 32) {
+        float x = 0.f;
+        for (int j = lane; j < DK; j += 32) x = fmaf(Gs[r * LD + j], Ks[r * LD + j], x);
+        x = warp_sum(x);
+        if (lane == 0) V_(V_DQK)[r] = x;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int r = lane;
+        float sdS = 0.f;
+#pragma unroll
+        for (int w = 0; w < kThreads / 32; ++w) sdS += red[w];
+        const float f = V_(V_F)[r];
+        const float fsum = warp_sum(f);
+        const float dgL = fsum + expf(g[kL - 1]) * sdS;
+        const float rowa = V_(V_ROWA)[r];
+        // sensitivity to g'_r = g_{r-1}, moved onto g_{r-1}
+        const float dgp = bt[r] * (rowa - egp[r] * V_(V_T2)[r]);
+        const float dgp_next = __shfl_down_sync(0xffffffffu, dgp, 1);
+        float dg = V_(V_ROWP)[r] - V_(V_COLP)[r] + V_(V_QG)[r] - V_(V_COLA)[r] - f;
+        if (r < kL - 1) dg += dgp_next;
+        if (r == kL - 1) dg += dgL;
+        // dlog_alpha_i = sum_{r >= i} dg_r
+        float x = dg;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_down_sync(0xffffffffu, x, o);
+            if (r + o < kL) x += y;
+        }
+        if (r < Lc) {
+            dlog_alpha[row0 + (size_t)r * H] = x;
+            dbeta[row0 + (size_t)r * H] = V_(V_T1)[r] + rowa;
+        }
+        const float ddp = warp_sum(-V_(V_DQK)[r]);
+        if (r == 0) ws.ddp[ci] = ddp;
+    }
+}
+
+// dd[h] = sum over b and chunks of the per-chunk partials, in a fixed order.
+__global__ void __launch_bounds__(kThreads)
+bwd_dd_sum_kernel(const float* __restrict__ ddp, float* __restrict__ dd, int B, int H, int nch) {
+    __shared__ float red[kThreads / 32];
+    const int h = blockIdx.x;
+    float x = 0.f;
+    for (long e = threadIdx.x; e < (long)B * nch; e += kThreads) {
+        const long b = e / nch, c = e % nch;
+        x += ddp[((size_t)b * H + h) * nch + c];
+    }
+    x = warp_sum(x);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = x;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float s = 0.f;
+        for (int w = 0; w < kThreads / 32; ++w) s += red[w];
+        dd[h] = s;
+    }
+}
+
+}  // namespace bwd
+}  // namespace comba

@@ -17,6 +17,7 @@
 #include "chunk_simt.cuh"
 #include "chunk_tc.cuh"
 #include "chunk_segments.cuh"
+#include "chunk_bwd.cuh"
 #include "recurrent_step.cuh"
 
 namespace {
@@ -448,6 +449,127 @@ extern "C" int comba_recurrent_step(const void* q, const void* k, const void* v,
                                     float* S, void* out, int B, int H, int dk, int dv,
                                     comba_stream_t stream) {
     return comba_recurrent_step_grouped(q, k, v, log_alpha, beta, d, S, out, B, H, H, dk, dv, stream);
+}
+
+namespace {
+
+struct BwdArgs {
+    const void *q, *k, *v, *dout;
+    const float *log_alpha, *beta, *d, *S0, *dS_final;
+    float *dq, *dk, *dv, *dlog_alpha, *dbeta, *dd, *dS0;
+    int B, T, H, DK, DV;
+};
+
+template <typename Tin, int DK, int DV>
+int launch_bwd(const BwdArgs& a, float* wsp, cudaStream_t s) {
+    namespace bw = comba::bwd;
+    const long chains = (long)a.B * a.H;
+    const int nch = (a.T + bw::kL - 1) / bw::kL;
+    const bw::Workspace ws = bw::carve(wsp, chains, nch, DK, DV);
+    const auto* q = static_cast<const Tin*>(a.q);
+    const auto* k = static_cast<const Tin*>(a.k);
+    const auto* v = static_cast<const Tin*>(a.v);
+    const auto* o = static_cast<const Tin*>(a.dout);
+    const size_t sp = bw::PrepSmem<Tin, DK, DV>::total * sizeof(float);
+    const size_t ss = bw::StatesSmem<DK, DV>::total * sizeof(float);
+    const size_t sd = bw::DStatesSmem<DK, DV>::total * sizeof(float);
+    const size_t sg = bw::GradSmem<DK, DV>::total * sizeof(float);
+    if (cudaFuncSetAttribute(bw::bwd_prep_kernel<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sp) != cudaSuccess ||
+        cudaFuncSetAttribute(bw::bwd_states_kernel<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)ss) != cudaSuccess ||
+        cudaFuncSetAttribute(bw::bwd_dstates_kernel<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sd) != cudaSuccess ||
+        cudaFuncSetAttribute(bw::bwd_grads_kernel<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sg) != cudaSuccess)
+        return COMBA_ECUDA;
+    if (chains > 0 && nch > 0) {
+        const dim3 grid((unsigned)nch, (unsigned)chains);
+        bw::bwd_prep_kernel<Tin, DK, DV><<<grid, bw::kThreads, sp, s>>>(q, k, v, a.log_alpha, a.beta, a.d, o, ws,
+                                                                         a.T, a.H, nch);
+        bw::bwd_states_kernel<Tin, DK, DV><<<(unsigned)chains, bw::kThreads, ss, s>>>(k, a.log_alpha, a.beta, a.S0,
+                                                                                       ws, a.T, a.H, nch);
+    }
+    if (chains > 0)
+        bw::bwd_dstates_kernel<Tin, DK, DV><<<(unsigned)chains, bw::kThreads, sd, s>>>(
+            k, a.log_alpha, a.beta, a.dS_final, a.dS0, ws, a.T, a.H, nch);
+    if (chains > 0 && nch > 0) {
+        const dim3 grid((unsigned)nch, (unsigned)chains);
+        bw::bwd_grads_kernel<Tin, DK, DV><<<grid, bw::kThreads, sg, s>>>(q, k, v, a.log_alpha, a.beta, a.d, o, a.dq,
+                                                                          a.dk, a.dv, a.dlog_alpha, a.dbeta, ws,
+                                                                          a.T, a.H, nch);
+    }
+    if (a.dd && a.H > 0)
+        bw::bwd_dd_sum_kernel<<<(unsigned)a.H, bw::kThreads, 0, s>>>(ws.ddp, a.dd, a.B, a.H, nch);
+    return cudaGetLastError() == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
+}
+
+template <typename Tin, int DK>
+int launch_bwd_dv(const BwdArgs& a, float* ws, cudaStream_t s) {
+    switch (a.DV) {
+        case 32: return launch_bwd<Tin, DK, 32>(a, ws, s);
+        case 64: return launch_bwd<Tin, DK, 64>(a, ws, s);
+        default: return launch_bwd<Tin, DK, 128>(a, ws, s);
+    }
+}
+
+template <typename Tin>
+int launch_bwd_dk(const BwdArgs& a, float* ws, cudaStream_t s) {
+    switch (a.DK) {
+        case 32: return launch_bwd_dv<Tin, 32>(a, ws, s);
+        case 64: return launch_bwd_dv<Tin, 64>(a, ws, s);
+        default: return launch_bwd_dv<Tin, 128>(a, ws, s);
+    }
+}
+
+bool bwd_dim(int x) { return x == 32 || x == 64 || x == 128; }
+
+}  // namespace
+
+extern "C" size_t comba_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv) {
+    if (B < 0 || T < 0 || H < 0 || !bwd_dim(dk) || !bwd_dim(dv)) return 0;
+    const int nch = (T + comba::bwd::kL - 1) / comba::bwd::kL;
+    return comba::bwd::workspace_floats((long)B * H, nch, dk, dv) * sizeof(float);
+}
+
+extern "C" int comba_chunk_bwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                               const float* beta, const float* d, const float* S0, const void* dout,
+                               const float* dS_final, float* dq, float* dk, float* dv, float* dlog_alpha,
+                               float* dbeta, float* dd, float* dS0, int B, int T, int H, int dk_, int dv_,
+                               int dtype, void* workspace, size_t workspace_bytes, comba_stream_t stream) {
+    if (B < 0 || T < 0 || H < 0 || !bwd_dim(dk_) || !bwd_dim(dv_)) return COMBA_EINVAL;
+    if (dtype != COMBA_BF16 && dtype != COMBA_F32) return COMBA_EINVAL;
+    const size_t elt = (dtype == COMBA_BF16) ? 2 : 4;
+    const long chains = (long)B * H;
+    if (chains > 65535) return COMBA_EUNSUPPORTED;
+    const size_t bth = (size_t)B * T * H;
+    if (bth > (size_t)1 << 40) return COMBA_EINVAL;
+    if (chains == 0 && !(dd && H > 0)) return COMBA_OK;
+    const size_t need = comba_chunk_bwd_workspace_size(B, T, H, dk_, dv_);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16))) return COMBA_EINVAL;
+    if (bth > 0 && (!q || !k || !v || !dout || !log_alpha || !beta || !dq || !dk || !dv || !dlog_alpha || !dbeta))
+        return COMBA_EINVAL;
+    if (chains > 0 && !d) return COMBA_EINVAL;
+    const void* ins[] = {q, k, v, dout, log_alpha, beta, d, S0, dS_final};
+    const size_t nqk = bth * dk_ * elt, nv = bth * dv_ * elt, ng = bth * 4, nh = (size_t)H * 4;
+    const size_t ns = (size_t)chains * dv_ * dk_ * 4;
+    const size_t nin[] = {nqk, nqk, nv, nv, ng, ng, nh, ns, ns};
+    const void* outs[] = {dq, dk, dv, dlog_alpha, dbeta, dd, dS0, workspace};
+    const size_t nout[] = {bth * dk_ * 4, bth * dk_ * 4, bth * dv_ * 4, ng, ng, nh, ns, need};
+    for (int i = 0; i < 9; ++i)
+        if (!aligned(ins[i], elt < 4 && i < 4 ? 2 : 4)) return COMBA_EINVAL;
+    for (int i = 0; i < 8; ++i) {
+        if (!aligned(outs[i], 4)) return COMBA_EINVAL;
+        for (int j = 0; j < 9; ++j)
+            if (overlap(outs[i], nout[i], ins[j], nin[j])) return COMBA_EINVAL;
+        for (int j = i + 1; j < 8; ++j)
+            if (overlap(outs[i], nout[i], outs[j], nout[j])) return COMBA_EINVAL;
+    }
+    const BwdArgs a{q, k, v, dout, log_alpha, beta, d, S0, dS_final, dq, dk, dv, dlog_alpha, dbeta, dd, dS0,
+                    B, T, H, dk_, dv_};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float* ws = static_cast<float*>(workspace);
+    return dtype == COMBA_BF16 ? launch_bwd_dk<__nv_bfloat16>(a, ws, s) : launch_bwd_dk<float>(a, ws, s);
 }
 
 extern "C" int comba_get_last_error(void) {

@@ -39,7 +39,7 @@ __all__ = [
     "ChunkConfig", "DecodeConfig", "CONFIGS", "DECODE", "chunk_config",
     "make_chunk_inputs", "make_decode_state", "decode_step_inputs",
     "head_token_count", "VarlenConfig", "VARLEN", "varlen_lengths", "make_varlen_inputs",
-    "make_gated_inputs",
+    "make_gated_inputs", "make_cotangents",
 ]
 
 
@@ -245,6 +245,20 @@ def make_chunk_inputs(cfg: ChunkConfig, seed: Optional[int] = None) -> Dict[str,
         "d": d.to(torch.float32).contiguous(),
         "S0": None if S0 is None else S0.contiguous(),
     }
+
+
+def make_cotangents(cfg: ChunkConfig, seed: Optional[int] = None, dS_std: float = 1.0) -> Dict[str, torch.Tensor]:
+    """Cotangents for the backward: dout [B,T,H,dv] ~ N(0,1) in the workload's storage
+    dtype and dS_final [B,H,dv,dk] ~ N(0, dS_std^2) fp32 (None when dS_std == 0), as
+    CPU tensors."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed((cfg.seed if seed is None else seed) + 7919)
+    B, T, H, dk, dv = cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv
+    dout = _normal(gen, (B, T, H, dv)).to(cfg.torch_dtype).contiguous()
+    dS = None
+    if dS_std > 0:
+        dS = (dS_std * _normal(gen, (B, H, dv, dk))).to(torch.float32).contiguous()
+    return {"dout": dout, "dS_final": dS}
 
 
 def make_decode_state(cfg: DecodeConfig = DECODE, B: Optional[int] = None,

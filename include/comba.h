@@ -58,6 +58,12 @@ enum comba_status {
     COMBA_EDEVICE = -5        /* device side: inconsistent internal state detected */
 };
 
+/* Element type of q, k, v and the output cotangent in comba_chunk_bwd. */
+enum comba_dtype {
+    COMBA_BF16 = 0,           /* __nv_bfloat16 */
+    COMBA_F32 = 1             /* float */
+};
+
 /*
  * Chunk-wise forward, bf16 inputs and output, fp32 gates/state/accumulation.
  *
@@ -230,6 +236,47 @@ int comba_recurrent_step_grouped(const void* q, const void* k, const void* v,
                                  const float* log_alpha, const float* beta, const float* d,
                                  float* S, void* out, int B, int H, int Hqk, int dk, int dv,
                                  comba_stream_t stream);
+
+/*
+ * Backward of the chunk-wise forward: the gradients of
+ *     L = <dout, out> + <dS_final, S_final>
+ * with respect to q, k, v, log_alpha, beta, d and S0, for the recurrence and
+ * output above.  The write-up (section "硬件高效的分块并行计算") states only that
+ * the backward pass reuses the chunk-level states and the per-chunk inverse; this
+ * entry point computes the adjoint of the chunk form in four stages.
+ *  1. Per chunk in parallel: W, U~ and dO^T (Gamma Q~ - P W).
+ *  2. The chunk-start states, chunks in order.
+ *  3. The end-state gradients, chunks in reverse.
+ *  4. Per chunk in parallel: the input gradients.
+ * It recomputes the states rather than reading saved ones.  Chunks are 32 tokens
+ * (a tiling choice: the result is the same function of the inputs for any chunk
+ * length).  fp32 arithmetic throughout.
+ *
+ * q, k [B, T, H, dk], v and dout [B, T, H, dv]: element type `dtype` (COMBA_BF16 or
+ * COMBA_F32), the same values the forward read.  log_alpha, beta [B, T, H], d [H],
+ * S0 [B, H, dv, dk]: fp32 (S0 NULL = zero initial state).  dS_final [B, H, dv,
+ * dk] fp32 or NULL (= 0).
+ * Outputs, fp32:
+ *  - dq, dk [B, T, H, dk] and dv [B, T, H, dv];
+ *  - dlog_alpha, dbeta [B, T, H];
+ *  - dd [H] (NULL skips it; a sum over batch and time in a fixed order);
+ *  - dS0 [B, H, dv, dk] (NULL skips it).
+ * dk, dv in {32, 64, 128}; any T >= 0 (T == 0: dS0 = dS_final, dd = 0); B * H <= 65535.
+ * workspace: DEVICE memory, 16-byte aligned, at least
+ * comba_chunk_bwd_workspace_size(B, T, H, dk, dv) bytes (per chunk: W, U~ and three
+ * dv x dk fp32 matrices), owned by the caller and in use until `stream` has passed
+ * the call.  Alignment is the element size.  No output may overlap an input,
+ * another output or the workspace.  Returns COMBA_EINVAL for a bad size, pointer,
+ * alignment, overlap or workspace; COMBA_EUNSUPPORTED for B * H > 65535.
+ */
+size_t comba_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv);
+int comba_chunk_bwd(const void* q, const void* k, const void* v,
+                    const float* log_alpha, const float* beta, const float* d,
+                    const float* S0, const void* dout, const float* dS_final,
+                    float* dq, float* dk, float* dv, float* dlog_alpha, float* dbeta,
+                    float* dd, float* dS0,
+                    int B, int T, int H, int dk_dim, int dv_dim, int dtype,
+                    void* workspace, size_t workspace_bytes, comba_stream_t stream);
 
 /*
  * Reads and clears the current device's status word (synchronises the

@@ -227,3 +227,51 @@ def test_gated_rejects_the_chunk_entrys_bad_arguments(lib):
 
 def test_gated_empty_is_noop(lib):
     assert _call_gated(lib, _chunk_args(B=0, q=None, k=None, v=None), BASE + 10 * GB, None, 1e-6) == 0
+
+
+def _bwd_args(**kw):
+    a = dict(q=BASE, k=BASE + GB, v=BASE + 2 * GB, log_alpha=BASE + 3 * GB, beta=BASE + 4 * GB,
+             d=BASE + 5 * GB, S0=BASE + 6 * GB, dout=BASE + 7 * GB, dS_final=BASE + 8 * GB,
+             dq=BASE + 9 * GB, dk=BASE + 10 * GB, dv=BASE + 11 * GB, dlog_alpha=BASE + 12 * GB,
+             dbeta=BASE + 13 * GB, dd=BASE + 14 * GB, dS0=BASE + 15 * GB,
+             B=2, T=100, H=4, dk_dim=64, dv_dim=64, dtype=0, ws=BASE + 20 * GB, ws_bytes=None)
+    a.update(kw)
+    return a
+
+
+def _call_bwd(lib, a):
+    p = lambda x: ctypes.c_void_p(x)
+    need = lib.comba_chunk_bwd_workspace_size(a["B"], a["T"], a["H"], a["dk_dim"], a["dv_dim"])
+    nb = need if a["ws_bytes"] is None else a["ws_bytes"]
+    return lib.comba_chunk_bwd(*(p(a[n]) for n in ("q", "k", "v", "log_alpha", "beta", "d", "S0", "dout",
+                                                    "dS_final", "dq", "dk", "dv", "dlog_alpha", "dbeta",
+                                                    "dd", "dS0")),
+                               a["B"], a["T"], a["H"], a["dk_dim"], a["dv_dim"], a["dtype"], p(a["ws"]), nb,
+                               ctypes.c_void_p(None))
+
+
+def test_bwd_workspace_size(lib):
+    # per chunk of 32 tokens: W [32, dk], U~ [32, dv], three dv x dk matrices, one dd partial
+    n = 2 * 4 * 4          # B * H chains x ceil(100 / 32) chunks
+    assert lib.comba_chunk_bwd_workspace_size(2, 100, 4, 64, 64) == n * (32 * 128 + 3 * 64 * 64 + 1) * 4
+    assert lib.comba_chunk_bwd_workspace_size(2, 100, 4, 48, 64) == 0     # unsupported dk
+    assert lib.comba_chunk_bwd_workspace_size(0, 100, 4, 64, 64) == 0
+
+
+@pytest.mark.parametrize("bad", [
+    dict(dk_dim=48), dict(dv_dim=16), dict(dtype=2), dict(B=-1), dict(T=-3),
+    dict(q=None), dict(dout=None), dict(dq=None), dict(dbeta=None), dict(d=None),
+    dict(ws=None), dict(ws_bytes=1024), dict(ws=BASE + 20 * GB + 8),
+    dict(dq=BASE + 16),                    # dq overlaps q
+    dict(dk=BASE + 9 * GB + 64),           # dk overlaps dq
+    dict(dS0=BASE + 20 * GB + 4096),       # dS0 inside the workspace
+    dict(log_alpha=BASE + 3 * GB + 2),     # fp32 array misaligned
+    dict(q=BASE + 1),                      # bf16 array misaligned
+])
+def test_bwd_rejects_bad_arguments(lib, bad):
+    assert _call_bwd(lib, _bwd_args(**bad)) == -1
+
+
+def test_bwd_too_many_chains_and_empty_batch(lib):
+    assert _call_bwd(lib, _bwd_args(B=65536, H=1, T=1)) == -2
+    assert _call_bwd(lib, _bwd_args(B=0, dd=None, q=None, k=None, v=None, ws=None)) == 0
