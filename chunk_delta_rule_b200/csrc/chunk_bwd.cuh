@@ -25,8 +25,9 @@
 // Four kernels, all over a fixed 32-token chunk (a tiling choice: the gradients are
 // the same function of the inputs for any chunk length):
 //   bwd_prep     (chunk, chain) in parallel: W, U~ and C = dO^T (Gamma Q~ - P W)
-//   bwd_states   one CTA per chain, chunks in order: chunk-start states S_c
-//   bwd_dstates  one CTA per chain, chunks in reverse: end-state gradients dS'_c, dS0
+//   bwd_states   one CTA per 32 state rows of a chain, chunks in order: chunk-start
+//                states S_c
+//   bwd_dstates  likewise, chunks in reverse: end-state gradients dS'_c, dS0
 //   bwd_grads    (chunk, chain) in parallel: dq, dk, dv, dlog_alpha, dbeta and a
 //                per-chunk partial of dd
 // plus bwd_dd_sum, which adds the dd partials per head in a fixed order.
@@ -100,6 +101,78 @@ __device__ __forceinline__ void bgemm(const FA& a, const FB& b, const Epi& epi) 
     }
 }
 
+// The same product with the k x n operand in global memory, staged through shared
+// memory in slabs of 32 k-rows (`stage`: 32 x (N + 1) floats).  kTrans = false: the
+// operand is G[k][n] (row-major K x N); kTrans = true: it is G[n][k] (row-major
+// N x K).  One tile per thread (TILES <= kThreads), so the accumulators stay in
+// registers across slabs; every thread of the block must make the call (it
+// synchronises the block before each slab).
+template <int M, int N, int K, int TM, int TN, bool kTrans, typename FA, typename Epi>
+__device__ __forceinline__ void bgemm_staged(const FA& a, const float* __restrict__ G, float* stage,
+                                             const Epi& epi) {
+    static_assert(M % TM == 0 && N % TN == 0 && K % 32 == 0 && N % 4 == 0, "tile must divide the product");
+    constexpr int MS = M / TM, NS = N / TN, LS = kTrans ? N + 1 : N;
+    static_assert(MS * NS <= kThreads, "one tile per thread");
+    const int t = threadIdx.x, mt = t / NS, nt = t % NS;
+    const bool act = t < MS * NS;
+    float acc[TM][TN];
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
+    for (int k0 = 0; k0 < K; k0 += 32) {
+        __syncthreads();   // the previous slab (or the caller's last use of stage) is done
+        constexpr int NV = 8 * N, PER = (NV + kThreads - 1) / kThreads;   // float4s per slab
+        float4 v[PER];
+#pragma unroll
+        for (int it = 0; it < PER; ++it) {
+            const int e = t + it * kThreads;
+            if (NV % kThreads == 0 || e < NV) {
+                if constexpr (kTrans)   // row n of G, k0 + 4 (e % 8) .. + 3
+                    v[it] = *reinterpret_cast<const float4*>(G + (size_t)(e / 8) * K + k0 + 4 * (e % 8));
+                else
+                    v[it] = *reinterpret_cast<const float4*>(G + (size_t)k0 * N + 4 * e);
+            }
+        }
+#pragma unroll
+        for (int it = 0; it < PER; ++it) {
+            const int e = t + it * kThreads;
+            if (NV % kThreads == 0 || e < NV) {
+                if constexpr (kTrans) {   // odd stride in stage: the four k rows hit distinct banks
+                    const int n = e / 8, k = 4 * (e % 8);
+                    stage[(k + 0) * LS + n] = v[it].x;
+                    stage[(k + 1) * LS + n] = v[it].y;
+                    stage[(k + 2) * LS + n] = v[it].z;
+                    stage[(k + 3) * LS + n] = v[it].w;
+                } else {
+                    *reinterpret_cast<float4*>(stage + 4 * e) = v[it];
+                }
+            }
+        }
+        __syncthreads();
+        if (act) {
+#pragma unroll 4
+            for (int k = 0; k < 32; ++k) {
+                float av[TM], bv[TN];
+#pragma unroll
+                for (int i = 0; i < TM; ++i) av[i] = a(mt + i * MS, k0 + k);
+#pragma unroll
+                for (int j = 0; j < TN; ++j) bv[j] = stage[k * LS + nt + j * NS];
+#pragma unroll
+                for (int i = 0; i < TM; ++i)
+#pragma unroll
+                    for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+            }
+        }
+    }
+    if (act) {
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+#pragma unroll
+            for (int j = 0; j < TN; ++j) epi(mt + i * MS, nt + j * NS, acc[i][j]);
+    }
+}
+
 // Chunk-local decay prefix of chunk c (warp 0): g_r = sum_{i<=r} log_alpha_i over
 // the chunk's tokens (0 past the end of the sequence), g'_r = g_{r-1}.
 __device__ __forceinline__ void chunk_decays(const float* __restrict__ log_alpha, const float* __restrict__ beta,
@@ -120,13 +193,70 @@ __device__ __forceinline__ void chunk_decays(const float* __restrict__ log_alpha
     }
 }
 
+// The shared-memory fills below issue all of a thread's 16-byte global loads before
+// its first store, so their latencies overlap instead of adding up.
+__device__ __forceinline__ void unpack16(const uint4& w, float (&f)[4]) {
+    f[0] = __uint_as_float(w.x); f[1] = __uint_as_float(w.y);
+    f[2] = __uint_as_float(w.z); f[3] = __uint_as_float(w.w);
+}
+__device__ __forceinline__ void unpack16(const uint4& w, float (&f)[8]) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 x = __bfloat1622float2(h[e]);
+        f[2 * e] = x.x;
+        f[2 * e + 1] = x.y;
+    }
+}
+
 // rows [L, D] of a [B, T, H, D] tensor into shared memory (stride ld), zero past Lc
+// (rows 16-byte aligned)
 template <int D, typename Tin>
 __device__ __forceinline__ void load_rows(float* dst, int ld, const Tin* __restrict__ src, size_t row0, int H,
                                           int Lc) {
-    for (int e = threadIdx.x; e < kL * D; e += kThreads) {
-        const int r = e / D, c = e % D;
-        dst[r * ld + c] = (r < Lc) ? to_f32(src[(row0 + (size_t)r * H) * D + c]) : 0.f;
+    constexpr int VE = 16 / (int)sizeof(Tin), VPR = D / VE, NV = kL * VPR;
+    constexpr int PER = (NV + kThreads - 1) / kThreads;
+    uint4 w[PER];
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+        const int e = threadIdx.x + it * kThreads, r = e / VPR;
+        w[it] = make_uint4(0u, 0u, 0u, 0u);
+        if ((NV % kThreads == 0 || e < NV) && r < Lc)
+            w[it] = *reinterpret_cast<const uint4*>(src + (row0 + (size_t)r * H) * D + (e % VPR) * VE);
+    }
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+        const int e = threadIdx.x + it * kThreads;
+        if (NV % kThreads == 0 || e < NV) {
+            float f[VE];
+            unpack16(w[it], f);
+            float* o = dst + (e / VPR) * ld + (e % VPR) * VE;
+#pragma unroll
+            for (int x = 0; x < VE; ++x) o[x] = f[x];
+        }
+    }
+}
+
+// an R x C fp32 tile (global rows ldg floats apart, 16-byte aligned) into shared
+// memory (stride lds); src == nullptr fills zeros
+template <int R, int C>
+__device__ __forceinline__ void tile_to_smem(float* dst, int lds, const float* __restrict__ src, size_t ldg) {
+    constexpr int VPR = C / 4, NV = R * VPR, PER = (NV + kThreads - 1) / kThreads;
+    float4 v[PER];
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+        const int e = threadIdx.x + it * kThreads;
+        v[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (src && (NV % kThreads == 0 || e < NV))
+            v[it] = *reinterpret_cast<const float4*>(src + (size_t)(e / VPR) * ldg + 4 * (e % VPR));
+    }
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+        const int e = threadIdx.x + it * kThreads;
+        if (NV % kThreads == 0 || e < NV) {
+            float* o = dst + (e / VPR) * lds + 4 * (e % VPR);
+            o[0] = v[it].x; o[1] = v[it].y; o[2] = v[it].z; o[3] = v[it].w;
+        }
     }
 }
 
@@ -213,10 +343,14 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
 // ---------------------------------------------------------------------------------
 // bwd_states: S_c for every chunk of one chain (S_0 = S0), from W and U~:
 //   X = U~ - W S^T,   S <- e^{g_L} S + X^T diag(e^{g_L - g}) K.
+// Row i of the new state needs only row i of S and column i of X, so each CTA keeps
+// a slice of kRows state rows (blockIdx.x = chain * (dv / kRows) + slice).
+constexpr int kRows = 32;
+
 template <int DK, int DV>
 struct StatesSmem {
-    static constexpr int LDK = DK + 1, LDV = DV + 1;
-    static constexpr size_t S = 0, W = S + DV * LDK, U = W + kL * LDK, K = U + kL * LDV, G = K + kL * LDK,
+    static constexpr int LDK = DK + 1, LDU = kRows + 1;
+    static constexpr size_t S = 0, W = S + kRows * LDK, U = W + kL * LDK, K = U + kL * LDU, G = K + kL * LDK,
                             GP = G + kL, BT = GP + kL, DEC = BT + kL, total = DEC + kL;
 };
 
@@ -225,34 +359,32 @@ __global__ void __launch_bounds__(kThreads)
 bwd_states_kernel(const Tin* __restrict__ k, const float* __restrict__ log_alpha, const float* __restrict__ beta,
                   const float* __restrict__ S0, Workspace ws, int T, int H, int nch) {
     using SM = StatesSmem<DK, DV>;
-    constexpr int LDK = SM::LDK, LDV = SM::LDV;
+    constexpr int LDK = SM::LDK, LDU = SM::LDU, SPLIT = DV / kRows;
     extern __shared__ float sm[];
     float *S = sm + SM::S, *Ws = sm + SM::W, *Us = sm + SM::U, *Ks = sm + SM::K;
     float *g = sm + SM::G, *gp = sm + SM::GP, *bt = sm + SM::BT, *dec = sm + SM::DEC;
-    const int bh = blockIdx.x, b = bh / H, h = bh % H;
-    const float* s0 = S0 ? S0 + (size_t)bh * DV * DK : nullptr;
-    for (int e = threadIdx.x; e < DV * DK; e += kThreads) S[(e / DK) * LDK + e % DK] = s0 ? s0[e] : 0.f;
+    const int bh = blockIdx.x / SPLIT, i0 = (blockIdx.x % SPLIT) * kRows, b = bh / H, h = bh % H;
+    const float* s0 = S0 ? S0 + (size_t)bh * DV * DK + (size_t)i0 * DK : nullptr;
+    tile_to_smem<kRows, DK>(S, LDK, s0, DK);
     for (int c = 0; c < nch; ++c) {
         const int t0 = c * kL, Lc = min(kL, T - t0);
         const size_t row0 = ((size_t)b * T + t0) * H + h, ci = (size_t)bh * nch + c;
-        const float* Wg = ws.W + ci * kL * DK;
-        const float* Ug = ws.U + ci * kL * DV;
-        for (int e = threadIdx.x; e < kL * DK; e += kThreads) Ws[(e / DK) * LDK + e % DK] = Wg[e];
-        for (int e = threadIdx.x; e < kL * DV; e += kThreads) Us[(e / DV) * LDV + e % DV] = Ug[e];
+        tile_to_smem<kL, DK>(Ws, LDK, ws.W + ci * kL * DK, DK);
+        tile_to_smem<kL, kRows>(Us, LDU, ws.U + ci * kL * DV + i0, DV);
         load_rows<DK>(Ks, LDK, k, row0, H, Lc);
         chunk_decays(log_alpha, beta, row0, H, Lc, g, gp, bt);
         __syncthreads();   // S of this chunk (previous iteration) and its tiles are in place
-        float* Sg = ws.S + ci * DV * DK;
-        for (int e = threadIdx.x; e < DV * DK; e += kThreads) Sg[e] = S[(e / DK) * LDK + e % DK];
+        float* Sg = ws.S + ci * DV * DK + (size_t)i0 * DK;
+        for (int e = threadIdx.x; e < kRows * DK; e += kThreads) Sg[e] = S[(e / DK) * LDK + e % DK];
         if (threadIdx.x < kL) dec[threadIdx.x] = expf(g[kL - 1] - g[threadIdx.x]);
-        bgemm<kL, DV, DK, 2, 4>([&](int r, int j) { return Ws[r * LDK + j]; },
-                                [&](int j, int i) { return S[i * LDK + j]; },
-                                [&](int r, int i, float s) { Us[r * LDV + i] -= s; });
+        bgemm<kL, kRows, DK, 2, 2>([&](int r, int j) { return Ws[r * LDK + j]; },
+                                   [&](int j, int i) { return S[i * LDK + j]; },
+                                   [&](int r, int i, float x) { Us[r * LDU + i] -= x; });
         __syncthreads();
         const float eL = expf(g[kL - 1]);
-        bgemm<DV, DK, kL, 8, 8>([&](int i, int r) { return Us[r * LDV + i] * dec[r]; },
-                                [&](int r, int j) { return Ks[r * LDK + j]; },
-                                [&](int i, int j, float s) { S[i * LDK + j] = fmaf(eL, S[i * LDK + j], s); });
+        bgemm<kRows, DK, kL, 4, 4>([&](int i, int r) { return Us[r * LDU + i] * dec[r]; },
+                                   [&](int r, int j) { return Ks[r * LDK + j]; },
+                                   [&](int i, int j, float x) { S[i * LDK + j] = fmaf(eL, S[i * LDK + j], x); });
         __syncthreads();
     }
 }
@@ -260,12 +392,13 @@ bwd_states_kernel(const Tin* __restrict__ k, const float* __restrict__ log_alpha
 // ---------------------------------------------------------------------------------
 // bwd_dstates: end-state gradients dS'_c of every chunk of one chain, last chunk
 // first (dS'_{last} = dS_final), and dS0:
-//   dS <- e^{g_L} dS - (dS K^T diag(e^{g_L - g})) W + C.
+//   dS <- e^{g_L} dS - (dS K^T diag(e^{g_L - g})) W + C,
+// row-separable like the state pass: each CTA keeps kRows rows of dS.
 template <int DK, int DV>
 struct DStatesSmem {
     static constexpr int LDK = DK + 1;
-    static constexpr size_t S = 0, W = S + DV * LDK, K = W + kL * LDK, Z = K + kL * LDK, G = Z + DV * kLDL,
-                            GP = G + kL, BT = GP + kL, DEC = BT + kL, total = DEC + kL;
+    static constexpr size_t S = 0, W = S + kRows * LDK, K = W + kL * LDK, Z = K + kL * LDK, G = Z + kRows * kLDL,
+                            GP = G + kL, BT = GP + kL, DEC = BT + kL, C = DEC + kL, total = C + kRows * LDK;
 };
 
 template <typename Tin, int DK, int DV>
@@ -274,41 +407,41 @@ bwd_dstates_kernel(const Tin* __restrict__ k, const float* __restrict__ log_alph
                    const float* __restrict__ dS_final, float* __restrict__ dS0, Workspace ws, int T, int H,
                    int nch) {
     using SM = DStatesSmem<DK, DV>;
-    constexpr int LDK = SM::LDK;
+    constexpr int LDK = SM::LDK, SPLIT = DV / kRows;
     extern __shared__ float sm[];
-    float *dS = sm + SM::S, *Ws = sm + SM::W, *Ks = sm + SM::K, *Z = sm + SM::Z;
+    float *dS = sm + SM::S, *Ws = sm + SM::W, *Ks = sm + SM::K, *Z = sm + SM::Z, *Cs = sm + SM::C;
     float *g = sm + SM::G, *gp = sm + SM::GP, *bt = sm + SM::BT, *dec = sm + SM::DEC;
-    const int bh = blockIdx.x, b = bh / H, h = bh % H;
-    const float* df = dS_final ? dS_final + (size_t)bh * DV * DK : nullptr;
-    for (int e = threadIdx.x; e < DV * DK; e += kThreads) dS[(e / DK) * LDK + e % DK] = df ? df[e] : 0.f;
+    const int bh = blockIdx.x / SPLIT, i0 = (blockIdx.x % SPLIT) * kRows, b = bh / H, h = bh % H;
+    const size_t soff = (size_t)bh * DV * DK + (size_t)i0 * DK;
+    const float* df = dS_final ? dS_final + soff : nullptr;
+    tile_to_smem<kRows, DK>(dS, LDK, df, DK);
     for (int c = nch - 1; c >= 0; --c) {
         const int t0 = c * kL, Lc = min(kL, T - t0);
         const size_t row0 = ((size_t)b * T + t0) * H + h, ci = (size_t)bh * nch + c;
-        const float* Wg = ws.W + ci * kL * DK;
-        for (int e = threadIdx.x; e < kL * DK; e += kThreads) Ws[(e / DK) * LDK + e % DK] = Wg[e];
+        tile_to_smem<kL, DK>(Ws, LDK, ws.W + ci * kL * DK, DK);
+        tile_to_smem<kRows, DK>(Cs, LDK, ws.C + ci * DV * DK + (size_t)i0 * DK, DK);
         load_rows<DK>(Ks, LDK, k, row0, H, Lc);
         chunk_decays(log_alpha, beta, row0, H, Lc, g, gp, bt);
         __syncthreads();
-        float* dSg = ws.dS + ci * DV * DK;
-        for (int e = threadIdx.x; e < DV * DK; e += kThreads) dSg[e] = dS[(e / DK) * LDK + e % DK];
+        float* dSg = ws.dS + ci * DV * DK + (size_t)i0 * DK;
+        for (int e = threadIdx.x; e < kRows * DK; e += kThreads) dSg[e] = dS[(e / DK) * LDK + e % DK];
         if (threadIdx.x < kL) dec[threadIdx.x] = expf(g[kL - 1] - g[threadIdx.x]);
         __syncthreads();
-        bgemm<DV, kL, DK, 4, 1>([&](int i, int j) { return dS[i * LDK + j]; },
-                                [&](int j, int r) { return Ks[r * LDK + j]; },
-                                [&](int i, int r, float s) { Z[i * kLDL + r] = dec[r] * s; });
+        bgemm<kRows, kL, DK, 2, 2>([&](int i, int j) { return dS[i * LDK + j]; },
+                                   [&](int j, int r) { return Ks[r * LDK + j]; },
+                                   [&](int i, int r, float x) { Z[i * kLDL + r] = dec[r] * x; });
         __syncthreads();
         const float eL = expf(g[kL - 1]);
-        const float* Cg = ws.C + ci * DV * DK;
-        bgemm<DV, DK, kL, 8, 8>([&](int i, int r) { return Z[i * kLDL + r]; },
-                                [&](int r, int j) { return Ws[r * LDK + j]; },
-                                [&](int i, int j, float s) {
-                                    dS[i * LDK + j] = fmaf(eL, dS[i * LDK + j], Cg[(size_t)i * DK + j] - s);
-                                });
+        bgemm<kRows, DK, kL, 4, 4>([&](int i, int r) { return Z[i * kLDL + r]; },
+                                   [&](int r, int j) { return Ws[r * LDK + j]; },
+                                   [&](int i, int j, float x) {
+                                       dS[i * LDK + j] = fmaf(eL, dS[i * LDK + j], Cs[i * LDK + j] - x);
+                                   });
         __syncthreads();
     }
+    __syncthreads();   // with no chunks, the fill above is the last writer of dS
     if (dS0)
-        for (int e = threadIdx.x; e < DV * DK; e += kThreads)
-            dS0[(size_t)bh * DV * DK + e] = dS[(e / DK) * LDK + e % DK];
+        for (int e = threadIdx.x; e < kRows * DK; e += kThreads) dS0[soff + e] = dS[(e / DK) * LDK + e % DK];
 }
 
 // ---------------------------------------------------------------------------------
@@ -321,7 +454,8 @@ struct GradSmem {
     static constexpr size_t K = 0, Q = K + kL * LD, O = Q + kL * LD, V = O + kL * LD, R = V + kL * LD,
                             X = R + kL * LD, D = X + kL * LD, G = D + kL * LD, TK = G + kL * LD,
                             AF = TK + kL * LD, P = AF + kL * kLDL, DP = P + kL * kLDL, DA = DP + kL * kLDL,
-                            VEC = DA + kL * kLDL, RED = VEC + NV * kL, total = RED + kThreads / 32;
+                            VEC = DA + kL * kLDL, RED = VEC + NV * kL, STG = RED + kThreads / 32,
+                            total = STG + kL * LD;   // STG: staging of S / dS' slabs
 };
 
 enum { V_G, V_GP, V_BT, V_EG, V_EGP, V_DEC, V_T1, V_T2, V_ROWA, V_COLA, V_ROWP, V_COLP, V_QG, V_F, V_DQK, V_DG };
@@ -341,6 +475,7 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     float *AF = sm + SM::AF, *Pm = sm + SM::P, *dPm = sm + SM::DP, *dAm = sm + SM::DA;
     float* vec = sm + SM::VEC;
     float* red = sm + SM::RED;
+    float* stage = sm + SM::STG;
     auto V_ = [&](int which) { return vec + which * kL; };
     float *g = V_(V_G), *gp = V_(V_GP), *bt = V_(V_BT), *eg = V_(V_EG), *egp = V_(V_EGP), *dec = V_(V_DEC);
     const int c = blockIdx.x, bh = blockIdx.y, b = bh / H, h = bh % H, tid = threadIdx.x;
@@ -368,16 +503,14 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         dec[tid] = expf(g[kL - 1] - g[tid]);
     }
     // 2. K S^T, AF, dX = diag(e^{g_L - g}) K dS'^T (P^T dO added below)
-    bgemm<DV, kL, DK, 4, 1>([&](int i, int j) { return S[(size_t)i * DK + j]; },
-                            [&](int j, int r) { return Ks[r * LD + j]; },
-                            [&](int i, int r, float s) { Rs[r * LD + i] = s; });
+    bgemm_staged<kL, DV, DK, 4, 4, true>([&](int r, int j) { return Ks[r * LD + j]; }, S, stage,
+                                         [&](int r, int i, float x) { Rs[r * LD + i] = x; });
     bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Ks[m * LD + x]; },
                             [&](int x, int n) { return Ks[n * LD + x]; },
                             [&](int m, int n, float s) { AF[m * kLDL + n] = (n < m) ? expf(gp[m] - g[n]) * s : 0.f; });
     __syncthreads();   // q~, decays
-    bgemm<DV, kL, DK, 4, 1>([&](int i, int j) { return dSp[(size_t)i * DK + j]; },
-                            [&](int j, int r) { return Ks[r * LD + j]; },
-                            [&](int i, int r, float s) { Ds[r * LD + i] = dec[r] * s; });
+    bgemm_staged<kL, DV, DK, 4, 4, true>([&](int r, int j) { return Ks[r * LD + j]; }, dSp, stage,
+                                         [&](int r, int i, float x) { Ds[r * LD + i] = dec[r] * x; });
     bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Qs[m * LD + x]; },
                             [&](int x, int n) { return Ks[n * LD + x]; },
                             [&](int m, int n, float s) { Pm[m * kLDL + n] = (n <= m) ? expf(g[m] - g[n]) * s : 0.f; });
@@ -435,15 +568,13 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
             V_(V_T2)[r] = t2;
         }
     }
-    bgemm<kL, DK, DV, 2, 4>([&](int r, int i) { return Os[r * LD + i]; },
-                            [&](int i, int j) { return S[(size_t)i * DK + j]; },
-                            [&](int r, int j, float s) { Gs[r * LD + j] = eg[r] * s; });
+    bgemm_staged<kL, DK, DV, 4, 4, false>([&](int r, int i) { return Os[r * LD + i]; }, S, stage,
+                                          [&](int r, int j, float x) { Gs[r * LD + j] = eg[r] * x; });
     __syncthreads();
     // 6. F = diag(e^{g_L - g}) X dS' (over K S^T); sums of dA o AF and dP o P by row
     //    and column; q~_r . (Gamma dO S)_r
-    bgemm<kL, DK, DV, 2, 4>([&](int s, int i) { return Xs[s * LD + i]; },
-                            [&](int i, int j) { return dSp[(size_t)i * DK + j]; },
-                            [&](int s, int j, float x) { Rs[s * LD + j] = dec[s] * x; });
+    bgemm_staged<kL, DK, DV, 4, 4, false>([&](int s, int i) { return Xs[s * LD + i]; }, dSp, stage,
+                                          [&](int s, int j, float x) { Rs[s * LD + j] = dec[s] * x; });
     if (tid < kL) {
         const int r = tid;
         float ra = 0.f, rp = 0.f;
@@ -488,15 +619,16 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     bgemm<kL, DK, kL, 2, 4>([&](int r, int s) { return dPm[r * kLDL + s]; },
                             [&](int s, int j) { return Ks[s * LD + j]; },
                             [&](int r, int j, float x) { Gs[r * LD + j] += x; });
-    bgemm<kL, DK, kL, 2, 4>([&](int r, int s) { return dPm[s * kLDL + r]; },
+    // (the three dk terms share one tiling, so each element stays with one thread)
+    bgemm<kL, DK, kL, 4, 4>([&](int r, int s) { return dPm[s * kLDL + r]; },
                             [&](int s, int j) { return Qs[s * LD + j]; },
                             [&](int r, int j, float x) { TKs[r * LD + j] = x; });
-    bgemm<kL, DK, kL, 2, 4>([&](int r, int s) { return dAm[r * kLDL + s] + dAm[s * kLDL + r]; },
+    bgemm<kL, DK, kL, 4, 4>([&](int r, int s) { return dAm[r * kLDL + s] + dAm[s * kLDL + r]; },
                             [&](int s, int j) { return Ks[s * LD + j]; },
                             [&](int r, int j, float x) { TKs[r * LD + j] += x; });
-    bgemm<kL, DK, DV, 2, 4>([&](int r, int i) { return Ds[r * LD + i]; },
-                            [&](int i, int j) { return S[(size_t)i * DK + j]; },
-                            [&](int r, int j, float x) { TKs[r * LD + j] = fmaf(-bt[r] * egp[r], x, TKs[r * LD + j]); });
+    bgemm_staged<kL, DK, DV, 4, 4, false>(
+        [&](int r, int i) { return Ds[r * LD + i]; }, S, stage,
+        [&](int r, int j, float x) { TKs[r * LD + j] = fmaf(-bt[r] * egp[r], x, TKs[r * LD + j]); });
     __syncthreads();
     // 9. outputs: dq, dk, dv; decay gradients; dd partial
     for (int e = tid; e < Lc * DK; e += kThreads) {
@@ -512,7 +644,15 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     }
     // <dS', S> and sum_r dq~_r . k_r (block sums in a fixed order)
     float ss = 0.f;
-    for (int e = tid; e < DV * DK; e += kThreads) ss = fmaf(dSp[e], S[e], ss);
+    {
+        constexpr int PER = DV * DK / 4 / kThreads;   // float4s of each matrix per thread
+#pragma unroll 4
+        for (int it = 0; it < PER; ++it) {
+            const float4 x = *reinterpret_cast<const float4*>(dSp + 4 * (tid + it * kThreads));
+            const float4 y = *reinterpret_cast<const float4*>(S + 4 * (tid + it * kThreads));
+            ss = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, ss))));
+        }
+    }
     ss = warp_sum(ss);
     if (lane == 0) red[warp] = ss;
     for (int r = warp; r < kL; r += kThreads / 32) {

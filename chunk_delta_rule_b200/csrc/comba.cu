@@ -487,11 +487,11 @@ int launch_bwd(const BwdArgs& a, float* wsp, cudaStream_t s) {
         const dim3 grid((unsigned)nch, (unsigned)chains);
         bw::bwd_prep_kernel<Tin, DK, DV><<<grid, bw::kThreads, sp, s>>>(q, k, v, a.log_alpha, a.beta, a.d, o, ws,
                                                                          a.T, a.H, nch);
-        bw::bwd_states_kernel<Tin, DK, DV><<<(unsigned)chains, bw::kThreads, ss, s>>>(k, a.log_alpha, a.beta, a.S0,
+        bw::bwd_states_kernel<Tin, DK, DV><<<(unsigned)(chains * (DV / bw::kRows)), bw::kThreads, ss, s>>>(k, a.log_alpha, a.beta, a.S0,
                                                                                        ws, a.T, a.H, nch);
     }
     if (chains > 0)
-        bw::bwd_dstates_kernel<Tin, DK, DV><<<(unsigned)chains, bw::kThreads, sd, s>>>(
+        bw::bwd_dstates_kernel<Tin, DK, DV><<<(unsigned)(chains * (DV / bw::kRows)), bw::kThreads, sd, s>>>(
             k, a.log_alpha, a.beta, a.dS_final, a.dS0, ws, a.T, a.H, nch);
     if (chains > 0 && nch > 0) {
         const dim3 grid((unsigned)nch, (unsigned)chains);
@@ -556,8 +556,9 @@ extern "C" int comba_chunk_bwd(const void* q, const void* k, const void* v, cons
     const size_t nin[] = {nqk, nqk, nv, nv, ng, ng, nh, ns, ns};
     const void* outs[] = {dq, dk, dv, dlog_alpha, dbeta, dd, dS0, workspace};
     const size_t nout[] = {bth * dk_ * 4, bth * dk_ * 4, bth * dv_ * 4, ng, ng, nh, ns, need};
+    // rows of q, k, v, dout and the state matrices are read with 16-byte vector loads
     for (int i = 0; i < 9; ++i)
-        if (!aligned(ins[i], elt < 4 && i < 4 ? 2 : 4)) return COMBA_EINVAL;
+        if (!aligned(ins[i], (i < 4 || i >= 7) ? 16 : 4)) return COMBA_EINVAL;
     for (int i = 0; i < 8; ++i) {
         if (!aligned(outs[i], 4)) return COMBA_EINVAL;
         for (int j = 0; j < 9; ++j)

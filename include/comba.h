@@ -265,7 +265,8 @@ int comba_recurrent_step_grouped(const void* q, const void* k, const void* v,
  * workspace: DEVICE memory, 16-byte aligned, at least
  * comba_chunk_bwd_workspace_size(B, T, H, dk, dv) bytes (per chunk: W, U~ and three
  * dv x dk fp32 matrices), owned by the caller and in use until `stream` has passed
- * the call.  Alignment is the element size.  No output may overlap an input,
+ * the call.  q, k, v, dout, S0 and dS_final 16-byte aligned; everything else
+ * 4-byte aligned.  No output may overlap an input,
  * another output or the workspace.  Returns COMBA_EINVAL for a bad size, pointer,
  * alignment, overlap or workspace; COMBA_EUNSUPPORTED for B * H > 65535.
  */

@@ -267,6 +267,8 @@ def test_bwd_workspace_size(lib):
     dict(dS0=BASE + 20 * GB + 4096),       # dS0 inside the workspace
     dict(log_alpha=BASE + 3 * GB + 2),     # fp32 array misaligned
     dict(q=BASE + 1),                      # bf16 array misaligned
+    dict(dout=BASE + 7 * GB + 8),          # rows need 16-byte alignment
+    dict(S0=BASE + 6 * GB + 4),
 ])
 def test_bwd_rejects_bad_arguments(lib, bad):
     assert _call_bwd(lib, _bwd_args(**bad)) == -1
