@@ -20,6 +20,8 @@ hand-worked example, brute-force transition products and invariants):
 * ``recurrence_bwd_np`` -- gradients of the recurrence (reverse mode through the
                          token loop, float64), pinned by finite differences of
                          ``recurrence``, torch.autograd and a closed form;
+* ``chunked_bwd_np``  -- the same gradients through the chunk form (the adjoint
+                         the backward kernels use), pinned to ``recurrence_bwd_np``;
 * ``gate_inputs``     -- the inputs of the recurrence from raw projections: q, k
                          L2-normalised per token and head, log_alpha and beta from
                          raw gate projections (a reading: the pages fix neither the
@@ -313,3 +315,102 @@ def recurrence_bwd_np(q, k, v, log_alpha, beta, d, S0=None, dout=None, dS_final=
                         - d[None, :, None] * dqt)
             G = al[:, t][..., None, None] * G - be[:, t][..., None, None] * np.einsum("bhi,bhj->bhij", u, kt)
     return {"dq": gq, "dk": gk, "dv": gv, "dlog_alpha": gla, "dbeta": gbe, "dd": gd, "dS0": G}
+
+
+def chunked_bwd_np(q, k, v, log_alpha, beta, d, S0=None, dout=None, dS_final=None, chunk: int = 32):
+    """The gradients of ``recurrence_bwd_np`` through the chunk form of ``chunked_np``
+    (float64, one (b, h) chain at a time; small cases).  It is not the oracle for
+    the GPU; it pins the chunk adjoint the backward kernels use to the token-level
+    gradients.  Per chunk (notation of ``chunked_np``; A = diag(beta) AF,
+    Gamma = diag(exp g), E_rs = exp(g_r - g_s), Dc = diag(exp(g_L - g))), with dS'
+    the gradient at the chunk's end state:
+
+        dS   = exp(g_L) dS' - (dS' K^T Dc) W + dO^T (Gamma Q~ - P W)   (reverse pass)
+        dX   = P^T dO + Dc K dS'^T,   dR = Tinv^T dX
+        dA   = -(dR X^T) (s < r),     dP = (dO X^T) (s <= r)
+        dQ~  = Gamma dO S + (dP o E) K
+        dK   = (dP o E)^T Q~ - diag(beta exp g') dR S + (dY + dY^T) K + Dc X dS' - d dQ~,
+               dY = dA o (beta_r exp(g'_r - g_s))
+        dV   = diag(beta) dR,  dbeta_r = dR_r . (v_r - exp(g'_r) S k_r) + sum_s dA_rs AF_rs
+        dg   = every exponent's sensitivity, dlog_alpha_i = sum_{r >= i} dg_r (in the chunk)
+
+    Returns the dict of ``recurrence_bwd_np``."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    la, be, d = _f64(log_alpha), _f64(beta), _f64(d)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    S0 = np.zeros((B, H, dv, dk)) if S0 is None else _f64(S0)
+    dO = np.zeros((B, T, H, dv)) if dout is None else _f64(dout)
+    dSf = np.zeros((B, H, dv, dk)) if dS_final is None else _f64(dS_final)
+    g_out = {"dq": np.zeros_like(q), "dk": np.zeros_like(k), "dv": np.zeros_like(v),
+             "dlog_alpha": np.zeros_like(la), "dbeta": np.zeros_like(be), "dd": np.zeros(H),
+             "dS0": np.zeros((B, H, dv, dk))}
+    for b in range(B):
+        for h in range(H):
+            Kc, Qc, Vc, Oc = k[b, :, h], q[b, :, h], v[b, :, h], dO[b, :, h]
+            dh = d[h]
+            chunks = []
+            for t0 in range(0, T, chunk):      # state-independent pieces of every chunk
+                t1 = min(T, t0 + chunk)
+                L = t1 - t0
+                K, Q, V, bt = Kc[t0:t1], Qc[t0:t1], Vc[t0:t1], be[b, t0:t1, h]
+                g = np.cumsum(la[b, t0:t1, h])
+                gp = np.concatenate([[0.0], g[:-1]])
+                strict = np.tril(np.ones((L, L), dtype=bool), k=-1)
+                incl = np.tril(np.ones((L, L), dtype=bool))
+                F = np.where(strict, np.exp(np.where(strict, gp[:, None] - g[None, :], 0.0)), 0.0)
+                E = np.where(incl, np.exp(np.where(incl, g[:, None] - g[None, :], 0.0)), 0.0)
+                Qt = Q - dh * K
+                AF = F * (K @ K.T)
+                A = bt[:, None] * AF
+                Tinv = np.linalg.inv(np.eye(L) + A)
+                W = Tinv @ ((bt * np.exp(gp))[:, None] * K)
+                Ut = Tinv @ (bt[:, None] * V)
+                P = E * (Qt @ K.T)
+                dec = np.exp(g[-1] - g)
+                C = Oc[t0:t1].T @ (np.exp(g)[:, None] * Qt - P @ W)
+                chunks.append(dict(t0=t0, t1=t1, K=K, V=V, Qt=Qt, bt=bt, g=g, gp=gp, F=F, E=E, AF=AF, A=A,
+                                   Tinv=Tinv, W=W, Ut=Ut, P=P, dec=dec, C=C))
+            S = S0[b, h].copy()                    # chunk-start states, in order
+            starts = []
+            for c in chunks:
+                starts.append(S.copy())
+                X = c["Ut"] - c["W"] @ S.T
+                S = np.exp(c["g"][-1]) * S + X.T @ (c["dec"][:, None] * c["K"])
+            dS = dSf[b, h].copy()                  # end-state gradients, in reverse
+            ends = [None] * len(chunks)
+            for i in range(len(chunks) - 1, -1, -1):
+                c = chunks[i]
+                ends[i] = dS.copy()
+                dS = np.exp(c["g"][-1]) * dS - ((dS @ c["K"].T) * c["dec"][None, :]) @ c["W"] + c["C"]
+            g_out["dS0"][b, h] = dS
+            for c, S, dSp in zip(chunks, starts, ends):
+                t0, t1 = c["t0"], c["t1"]
+                K, V, Qt, bt, g, gp = c["K"], c["V"], c["Qt"], c["bt"], c["g"], c["gp"]
+                A, AF, F, E, Tinv, P, dec = c["A"], c["AF"], c["F"], c["E"], c["Tinv"], c["P"], c["dec"]
+                O = Oc[t0:t1]
+                KS = K @ S.T
+                Rv = V - np.exp(gp)[:, None] * KS
+                X = Tinv @ (bt[:, None] * Rv)
+                dX = P.T @ O + dec[:, None] * (K @ dSp.T)
+                dR = Tinv.T @ dX
+                dA = -np.tril(dR @ X.T, -1)
+                dP = np.tril(O @ X.T)
+                dZ = dP * E
+                dY = dA * bt[:, None] * F
+                GdOS = np.exp(g)[:, None] * (O @ S)
+                dQt = GdOS + dZ @ K
+                Fm = dec[:, None] * (X @ dSp)
+                dK = dZ.T @ Qt - (bt * np.exp(gp))[:, None] * (dR @ S) + (dY + dY.T) @ K + Fm - dh * dQt
+                g_out["dq"][b, t0:t1, h] = dQt
+                g_out["dk"][b, t0:t1, h] = dK
+                g_out["dv"][b, t0:t1, h] = bt[:, None] * dR
+                g_out["dbeta"][b, t0:t1, h] = (dR * Rv).sum(1) + (dA * AF).sum(1)
+                f = (Fm * K).sum(1)
+                dg = (dP * P).sum(1) - (dP * P).sum(0) + (Qt * GdOS).sum(1) - (dA * A).sum(0) - f
+                dgp = -bt * (dR * (np.exp(gp)[:, None] * KS)).sum(1) + (dA * A).sum(1)
+                dg[:-1] += dgp[1:]                 # the sensitivity to g_{r-1} moves onto g_{r-1}
+                dg[-1] += f.sum() + np.exp(g[-1]) * (dSp * S).sum()
+                g_out["dlog_alpha"][b, t0:t1, h] = np.cumsum(dg[::-1])[::-1]
+                g_out["dd"][h] -= (dQt * K).sum()
+    return g_out

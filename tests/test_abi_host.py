@@ -124,6 +124,10 @@ def test_binding_refuses_cpu_tensors():
     g = torch.zeros(1, 4, 1)
     with pytest.raises(ValueError):
         cdr.chunk_fwd(x, x, x, g, g, torch.zeros(1))
+    with pytest.raises(ValueError):
+        cdr.chunk_bwd(x, x, x, g, g, torch.zeros(1), x)
+    with pytest.raises(ValueError):   # q, k, v, dout must be bf16 or fp32
+        cdr.chunk_bwd(x.double(), x, x, g, g, torch.zeros(1), x)
 
 
 def _varlen_args(**kw):

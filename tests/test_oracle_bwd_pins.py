@@ -155,3 +155,25 @@ def test_planted_backward_mistake_is_caught(kind):
     fn = _mutant(kind)
     caught = [n for n, (check, tol) in BATTERY.items() if not check(fn) <= tol]
     assert caught, f"no pin catches the '{kind}' mistake"
+
+
+@pytest.mark.parametrize("T,chunk,dk,dv", [(37, 8, 5, 4), (64, 16, 8, 6), (50, 64, 4, 4), (1, 4, 3, 3),
+                                           (17, 1, 3, 2), (70, 32, 6, 5)])
+def test_chunked_backward_matches_token_backward(T, chunk, dk, dv):
+    """The chunk adjoint (the form the backward kernels compute) against the token
+    gradients, ragged last chunks and chunk length 1 included."""
+    x, cot = _case(40 + T, B=2, T=T, H=2, dk=dk, dv=dv)
+    ref = oracle.recurrence_bwd_np(**x, **cot)
+    g = oracle.chunked_bwd_np(**x, **cot, chunk=chunk)
+    for n in GRADS:
+        err = np.abs(g[n] - ref[n]).max() / max(np.abs(ref[n]).max(), 1e-30)
+        assert err <= 1e-12, (n, err)
+
+
+def test_chunked_backward_without_state_inputs():
+    x, cot = _case(77, B=1, T=40, H=1, dk=4, dv=3)
+    x["S0"] = None
+    ref = oracle.recurrence_bwd_np(**x, dout=cot["dout"], dS_final=None)
+    g = oracle.chunked_bwd_np(**x, dout=cot["dout"], dS_final=None, chunk=32)
+    for n in GRADS:
+        assert np.allclose(g[n], ref[n], rtol=1e-12, atol=1e-12), n
