@@ -589,6 +589,33 @@ def fp32_alu_peak_tflops(sm_mhz: float, sms: int = 148) -> float:
     return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
+def cpu_baseline_bwd(cfg, x, cot, target_s: float = 10.0):
+    """Times the float64 oracle's gradients (``oracle.recurrence_bwd_np``, as it
+    stands) on a bounded sample of the workload's (b, h) chains, stacked as heads of
+    one batch row; returns the baseline record in tokens/s of the whole workload."""
+    import oracle
+    B, H = cfg.B, cfg.H
+
+    def run(chains):
+        sl = [(c // H, c % H) for c in chains]
+        pick = lambda t: torch.stack([t[b, :, h] for b, h in sl], dim=1)[None]
+        pick_s = lambda t: None if t is None else torch.stack([t[b, h] for b, h in sl])[None]
+        t0 = time.perf_counter()
+        oracle.recurrence_bwd_np(pick(x["q"]), pick(x["k"]), pick(x["v"]), pick(x["log_alpha"]),
+                                 pick(x["beta"]), torch.stack([x["d"][h] for _, h in sl]), pick_s(x["S0"]),
+                                 pick(cot["dout"]), pick_s(cot["dS_final"]))
+        return time.perf_counter() - t0
+
+    probe = run([0])
+    n = max(1, min(B * H, int(target_s / max(probe, 1e-6))))
+    el = run(list(range(n))) if n > 1 else probe
+    tokens = n * cfg.T / H   # a token carries all H heads
+    return {"value": tokens / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} of {B * H} (b,h) chains x {cfg.T} tokens of {cfg.name}; float64 NumPy "
+                      f"reverse-mode token loop (states recomputed from checkpoints), one thread; {el:.1f} s",
+            "seconds": el}
+
+
 def run_bwd(args):
     """One step = one comba_chunk_bwd over the 1.3B layer (bf16 q, k, v, dout; fp32
     gates, S0 and dS_final), inputs and cotangents resident in HBM."""
@@ -668,6 +695,8 @@ def run_bwd(args):
         "clocks": ck,
         "gpu_launches": 5 * args.steps,
     }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = {k: v for k, v in cpu_baseline_bwd(cfg, x, x).items() if k != "seconds"}
     print(json.dumps(line), flush=True)
 
 

@@ -95,3 +95,23 @@ def test_varlen_workload_is_seeded_and_covers_its_tokens():
     import bench
     flops, bytes_ = bench.varlen_counts(VARLEN, len(a))
     assert bytes_ < bench.algorithmic_counts(bench.CONFIGS["layer1p3b_bf16"])[1]   # shared q / k heads
+
+
+def test_backward_flop_count_and_alu_peak():
+    # per 32-token chunk of one chain at dk = dv = 128: prep 2,088,960, states and
+    # dstates 2,097,152 each, grads 7,593,984 flops; 16,384 chunks in the 1.3B layer
+    per_chunk = 2_088_960 + 2 * 2_097_152 + 7_593_984
+    assert bench.bwd_algorithmic_flops(CONFIGS["layer1p3b_bf16"]) == 8 * 16 * 128 * per_chunk
+    # a ragged last chunk counts as a whole chunk (the kernels pad it)
+    cfg = CONFIGS["layer1p3b_bf16"].replace(B=1, H=1, T=33)
+    assert bench.bwd_algorithmic_flops(cfg) == 2 * per_chunk
+    assert abs(bench.fp32_alu_peak_tflops(1965.0) - 74.44992) < 1e-9
+
+
+def test_backward_cpu_baseline_record():
+    from comba_workloads import make_cotangents
+    cfg = CONFIGS["layer340m_bf16"].replace(B=2, H=2, T=40, dk=16, dv=16, s0_std=0.1)
+    x = make_chunk_inputs(cfg, seed=3)
+    rec = bench.cpu_baseline_bwd(cfg, x, make_cotangents(cfg, seed=4), target_s=0.05)
+    assert rec["kind"] == "oracle" and rec["unit"] == "tokens/s" and rec["cores"] == 1
+    assert rec["value"] > 0 and "chains" in rec["sample"]
