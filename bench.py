@@ -618,14 +618,17 @@ def cpu_baseline_bwd(cfg, x, cot, target_s: float = 10.0):
 
 def run_bwd(args):
     """One step = one comba_chunk_bwd over the 1.3B layer (bf16 q, k, v, dout; fp32
-    gates, S0 and dS_final), inputs and cotangents resident in HBM."""
+    gates, S0 and dS_final), inputs and cotangents resident in HBM.  Under torchrun
+    every rank runs its own batch of independent chains (weak scaling, no collective
+    in the data path); times are the max over ranks."""
     import chunk_delta_rule_b200 as cdr
     cfg = CONFIGS["layer1p3b_bf16"]
-    dev = torch.device("cuda", 0)
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     lib = cdr.library()
-    x = make_chunk_inputs(cfg)
-    x.update(make_cotangents(cfg))
+    x = make_chunk_inputs(cfg, seed=rank_seed(cfg, rank))
+    x.update(make_cotangents(cfg, seed=rank_seed(cfg, rank)))
     host = {k: v.pin_memory() for k, v in x.items() if v is not None}
     d_ = {k: v.to(dev) for k, v in host.items()}
     stream = torch.cuda.current_stream(dev)
@@ -642,7 +645,9 @@ def run_bwd(args):
     torch.cuda.synchronize(dev)
     assert cdr.get_last_error(dev) == 0
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(0).start()
+    clocks = ClockSampler(local).start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
     th0 = time.time()
     ev0.record(stream)
     for _ in range(args.steps):
@@ -652,7 +657,8 @@ def run_bwd(args):
     th1 = time.time()
     clocks.wait_after(th0)
     clocks.stop()
-    ms_step = ev0.elapsed_time(ev1) / args.steps
+    barrier(world)
+    ms_step = max_over_ranks(ev0.elapsed_time(ev1), world, dev) / args.steps
     if cdr.get_last_error(dev) != 0:
         raise RuntimeError("device-side error during the timed region")
     outs_h = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in res.items() if v is not None}
@@ -667,12 +673,14 @@ def run_bwd(args):
     for _ in range(3):
         e2e_step()
     torch.cuda.synchronize(dev)
+    barrier(world)
     ev0.record(stream)
     for _ in range(args.steps):
         e2e_step()
     ev1.record(stream)
     torch.cuda.synchronize(dev)
-    ms_e2e = ev0.elapsed_time(ev1) / args.steps
+    barrier(world)
+    ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), world, dev) / args.steps
     flops = bwd_algorithmic_flops(cfg)
     ck = clocks.summary(th0, th1)
     sm_max = ck.get("sm_max_mhz") or 1965.0
@@ -680,7 +688,8 @@ def run_bwd(args):
     tf = flops / (ms_step / 1e3) / 1e12
     line = {
         "metric": "Comba chunk-bwd tokens/s (all input gradients) on 1 B200, % of fp32 ALU roofline",
-        "value": cfg.B * cfg.T / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "value": weak_scaling_value(cfg.B * cfg.T, world, ms_step), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": dict(config_record(cfg), workload=BWD, chunk=BWD_CHUNK, inputs="bf16 q, k, v, dout"),
@@ -688,16 +697,20 @@ def run_bwd(args):
                      "traffic": None,
                      "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x max SM clock",
                      "algorithmic_flops_per_launch": flops, "scope": "whole backward (5 kernels)"},
-        "e2e": {"value": cfg.B * cfg.T / (ms_e2e / 1e3), "unit": "tokens/s",
+        "e2e": {"value": weak_scaling_value(cfg.B * cfg.T, world, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in host.values()),
                 "d2h_bytes_per_step": sum(v.numel() * v.element_size() for v in outs_h.values()),
                 "ms_per_step": ms_e2e},
         "clocks": ck,
         "gpu_launches": 5 * args.steps,
     }
-    if not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline_bwd(cfg, x, x).items() if k != "seconds"}
-    print(json.dumps(line), flush=True)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
 
 
 def main():
