@@ -1,4 +1,4 @@
-"""Comba chunk-wise forward and decode step on B200 (sm_100a).
+"""Comba chunk-wise forward, its backward and the decode step on B200 (sm_100a).
 
 Thin ctypes binding over the C ABI in ``include/comba.h``: it checks tensor
 placement, dtypes and contiguity, allocates outputs with PyTorch when the

@@ -1,4 +1,5 @@
-// C ABI of the Comba chunk-wise forward and decode step (declared in comba.h).
+// C ABI of the Comba chunk-wise forward, its backward and the decode step (declared
+// in comba.h).
 //
 // The host side validates every argument before anything is enqueued, picks
 // the kernel for the shape, launches on the caller's stream and returns a

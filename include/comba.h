@@ -1,5 +1,6 @@
 /*
- * comba.h -- C ABI of the B200 (sm_100a) Comba chunk-wise forward and decode step.
+ * comba.h -- C ABI of the B200 (sm_100a) Comba chunk-wise forward, its backward
+ * and the decode step.
  *
  * The method: Comba, "Improving Bilinear RNNs with Closed-loop Control"
  * (PaperWeekly write-up and arXiv abstract 2506.02475).  Comba's recurrent
