@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["chunk_fwd", "chunk_bwd", "chunk_fwd_gated", "chunk_fwd_host", "chunk_fwd_varlen", "chunk_fwd_noalloc",
+__all__ = ["chunk_fwd", "chunk_bwd", "state_compose", "chunk_fwd_gated", "chunk_fwd_host", "chunk_fwd_varlen", "chunk_fwd_noalloc",
            "recurrent_step",
            "get_last_error", "CombaError", "library", "library_path", "EXPORTS", "status_string"]
 
@@ -32,7 +32,7 @@ _lock = threading.Lock()
 EXPORTS = ("comba_chunk_fwd", "comba_chunk_fwd_f32", "comba_chunk_fwd_varlen",
            "comba_chunk_fwd_workspace_size", "comba_chunk_fwd_ws", "comba_chunk_fwd_noalloc",
            "comba_chunk_fwd_host", "comba_chunk_fwd_host_workspace_size", "comba_chunk_fwd_gated",
-           "comba_chunk_bwd", "comba_chunk_bwd_workspace_size",
+           "comba_chunk_bwd", "comba_chunk_bwd_workspace_size", "comba_state_compose",
            "comba_recurrent_step", "comba_recurrent_step_grouped", "comba_get_last_error",
            "comba_status_string", "comba_version")
 
@@ -72,12 +72,13 @@ def library():
             lib.comba_recurrent_step.argtypes = [vp] * 8 + [i] * 4 + [vp]
             lib.comba_chunk_bwd.argtypes = [vp] * 16 + [i] * 6 + [vp, ctypes.c_size_t, vp]
             lib.comba_chunk_bwd_workspace_size.argtypes = [i] * 5
+            lib.comba_state_compose.argtypes = [vp] * 3 + [i] * 3 + [vp]
             lib.comba_chunk_bwd_workspace_size.restype = ctypes.c_size_t
             lib.comba_recurrent_step_grouped.argtypes = [vp] * 8 + [i] * 5 + [vp]
             for fn in (lib.comba_chunk_fwd, lib.comba_chunk_fwd_f32, lib.comba_chunk_fwd_ws,
                        lib.comba_chunk_fwd_noalloc, lib.comba_chunk_fwd_varlen,
                        lib.comba_recurrent_step_grouped, lib.comba_chunk_fwd_host,
-                       lib.comba_chunk_fwd_gated, lib.comba_chunk_bwd,
+                       lib.comba_chunk_fwd_gated, lib.comba_chunk_bwd, lib.comba_state_compose,
                        lib.comba_recurrent_step, lib.comba_get_last_error, lib.comba_version):
                 fn.restype = ctypes.c_int
             lib.comba_get_last_error.argtypes = []
@@ -212,6 +213,29 @@ def chunk_fwd_gated(q_raw: torch.Tensor, k_raw: torch.Tensor, v: torch.Tensor, a
     if st != 0:
         raise CombaError(st, "comba_chunk_fwd_gated")
     return out, S_final
+
+
+def state_compose(R: torch.Tensor, M: torch.Tensor, S0: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """comba_state_compose: start states of P consecutive sequence pieces from their
+    affine state transitions (a piece maps S to S M + R).  R, M [B, P, H, 128, 128]
+    fp32; S0 [B, H, 128, 128] or None.  Returns S_start [B, P, H, 128, 128] with
+    S_start[:, 0] = S0 and S_start[:, p] = S_start[:, p-1] M[:, p-1] + R[:, p-1]."""
+    if R.dim() != 5:
+        raise ValueError("R must be [B, P, H, 128, 128]")
+    B, P, H = R.shape[:3]
+    _check(R, "R", torch.float32, (B, P, H, 128, 128))
+    _check(M, "M", torch.float32, (B, P, H, 128, 128))
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (B, H, 128, 128))
+    dev = R.device
+    RM = torch.stack([R, M])   # the entry point's layout: all R, then all M
+    S_start = torch.empty((B, P, H, 128, 128), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        st = library().comba_state_compose(_ptr(RM), _ptr(S0), _ptr(S_start), B, H, P,
+                                           _stream_handle(dev, stream))
+    if st != 0:
+        raise CombaError(st, "comba_state_compose")
+    return S_start
 
 
 _bwd_ws = {}

@@ -574,6 +574,26 @@ extern "C" int comba_chunk_bwd(const void* q, const void* k, const void* v, cons
     return dtype == COMBA_BF16 ? launch_bwd_dk<__nv_bfloat16>(a, ws, s) : launch_bwd_dk<float>(a, ws, s);
 }
 
+extern "C" int comba_state_compose(const float* RM, const float* S0, float* S_start, int B, int H, int P,
+                                   comba_stream_t stream) {
+    if (B < 0 || H < 0 || P < 1) return COMBA_EINVAL;
+    if (B == 0 || H == 0) return COMBA_OK;
+    if (!RM || !S_start) return COMBA_EINVAL;
+    if (!aligned(RM, 16) || !aligned(S0, 16) || !aligned(S_start, 16)) return COMBA_EINVAL;
+    const size_t st = comba::seg::kStateFloats * sizeof(float);
+    const size_t bph = (size_t)B * P * H;
+    if (bph > (size_t)1 << 31) return COMBA_EINVAL;
+    if (overlap(S_start, bph * st, RM, 2 * bph * st) || overlap(S_start, bph * st, S0, (size_t)B * H * st))
+        return COMBA_EINVAL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaFuncSetAttribute(comba::seg::seg_compose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)comba::seg::kComposeSmem) != cudaSuccess)
+        return COMBA_ECUDA;
+    comba::seg::seg_compose_kernel<<<(unsigned)(B * H), comba::seg::kComposeThreads, comba::seg::kComposeSmem, s>>>(
+        RM, S0, S_start, B, H, P);
+    return cudaGetLastError() == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
+}
+
 extern "C" int comba_get_last_error(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;
     int h = 0;

@@ -281,6 +281,25 @@ int comba_chunk_bwd(const void* q, const void* k, const void* v,
                     void* workspace, size_t workspace_bytes, comba_stream_t stream);
 
 /*
+ * Start states of P consecutive sequence pieces from their affine state
+ * transitions: over a piece, the state pass maps a start state S to S M + R (R: the
+ * end state from S = 0; M: the end state from S = I with V = 0).  This is the
+ * write-up's "recurrent across blocks" form applied to pieces, as in
+ * comba_chunk_fwd_ws; here the transitions come from the caller, e.g. gathered
+ * from the ranks of a context-parallel group.
+ *
+ *     S_start[b, 0, h] = S0[b, h]  (0 when S0 == NULL)
+ *     S_start[b, p, h] = S_start[b, p-1, h] M[b, p-1, h] + R[b, p-1, h]
+ *
+ * RM: fp32, the R of all pieces [B, P, H, 128, 128] followed by the M of all
+ * pieces [B, P, H, 128, 128] (the last piece's R and M are not read).  S0 [B, H,
+ * 128, 128] or NULL; S_start [B, P, H, 128, 128].  dk = dv = 128.  All 16-byte
+ * aligned; S_start must not overlap RM or S0.  fp32 FMA arithmetic.
+ */
+int comba_state_compose(const float* RM, const float* S0, float* S_start, int B, int H, int P,
+                        comba_stream_t stream);
+
+/*
  * Reads and clears the current device's status word (synchronises the
  * device first).  Returns COMBA_OK, COMBA_ETIMEOUT, COMBA_EDEVICE, or
  * COMBA_ECUDA if the synchronisation or the read itself failed.

@@ -281,3 +281,18 @@ def test_bwd_rejects_bad_arguments(lib, bad):
 def test_bwd_too_many_chains_and_empty_batch(lib):
     assert _call_bwd(lib, _bwd_args(B=65536, H=1, T=1)) == -2
     assert _call_bwd(lib, _bwd_args(B=0, dd=None, q=None, k=None, v=None, ws=None)) == 0
+
+
+def test_state_compose_rejects_bad_arguments(lib):
+    p = lambda x: ctypes.c_void_p(x)
+    call = lambda RM, S0, Sst, B=2, H=4, P=3: lib.comba_state_compose(p(RM), p(S0), p(Sst), B, H, P,
+                                                                       ctypes.c_void_p(None))
+    RM, S0, Sst = BASE, BASE + GB, BASE + 2 * GB
+    assert call(RM, S0, Sst, P=0) == -1
+    assert call(RM, S0, Sst, B=-1) == -1
+    assert call(None, S0, Sst) == -1
+    assert call(RM, S0, None) == -1
+    assert call(RM + 8, S0, Sst) == -1                  # misaligned
+    assert call(RM, S0, RM + 4096) == -1                # S_start inside RM
+    assert call(RM, S0, S0 + 64) == -1                  # S_start overlaps S0
+    assert call(None, None, None, B=0) == 0             # empty
