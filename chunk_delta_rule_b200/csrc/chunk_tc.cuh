@@ -329,7 +329,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     int b_split, int no_out, unsigned long long timeout_ns,
                     const int* __restrict__ cu_seqlens, int qk_group, unsigned short* out_raw,
                     const float* __restrict__ A_log, const float* __restrict__ dt_bias, float norm_eps) {
-    COMBA_CTA_MARK(0);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
     uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -463,7 +462,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         return v;
     };
 
-    COMBA_PHASE_BEGIN();
     if (kPacked && nchunks == 0) {
         // an empty chain (a zero-length packed sequence): S_final = S0 (or zero)
         if (warp < 4 && S_final) {
@@ -604,7 +602,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // done, into the V buffer (those MMAs have read V)
             ok = (*gabort == 0) && tc::mbar_wait(&bars[B_WN], n & 1, timeout_ns);
             tc::named_barrier(BAR_STATE, kStateThreads);
-            COMBA_PHASE(0);
             tc::tc_fence_after();
             {
                 float w0[32], w1[32];
@@ -625,7 +622,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
             if (issuer) tc::mbar_arrive(&bars[B_WREADY]);  // -W and the S copies are in: MMA1
             __syncwarp();
-            COMBA_PHASE(1);
             // ---- while MMA1 runs: the next chunk's decays
             const float eLn = last ? 1.f : state_gates(la_n, n + 1);
             if (tid < 64 && n + 2 < nchunks) la_n = gate(log_alpha, t0 + 2 * kC + tid);
@@ -633,7 +629,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ok = ok && tc::mbar_wait(&bars[B_MMA1], n & 1, timeout_ns);
             tc::tc_fence_after();
             if (issuer && ok && n + 1 < nchunks && !vzero) load_v(n + 1);   // MMA1 has read -W
-            COMBA_PHASE(6);
             const uint32_t sedn = sed(n);
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
@@ -666,13 +661,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!tc::named_barrier_all_ok(BAR_STATE, kStateThreads, ok && *gabort == 0)) break;
             if (issuer) tc::mbar_arrive(&bars[B_SPLIT]);   // X' is in: MMA2
             __syncwarp();
-            COMBA_PHASE(2);
             // ---- while MMA2 runs: Qh of the next chunk (MMA1 has read this chunk's)
             if (!last && want_out) {
                 ok = ok && tc::mbar_wait(&bars[B_MMA1B], n & 1, timeout_ns);
                 ok = state_qh(n + 1) && ok;
             }
-            COMBA_PHASE(3);
             ok = ok && tc::mbar_wait(&bars[B_MMA2], n & 1, timeout_ns);
             if (issuer) tc::bulk_wait_read0();   // the previous out store has read its staging
             if (!ok) fail(gabort);
@@ -681,10 +674,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (issuer && n + kKQStages < nchunks) {   // this chunk's q/k stage is read
                 tc::fence_proxy_async_smem();
                 load_kq(n + kKQStages);
-                COMBA_PHASE(26);
             }
             __syncwarp();
-            COMBA_PHASE(4);
             // O^T row (value index) -> bf16 pairs of tokens
             uint32_t ob[32];
             if (want_out) {
@@ -729,7 +720,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             tc::tmem_st_wait();
             tc::tc_fence_before();
-            COMBA_PHASE(5);
             if (want_out) {
             // out tile [token][value index] in two 64-wide 128B-swizzled boxes, staged in
             // its own buffer, TMA store; a packed sequence's ragged last tile is copied
@@ -759,7 +749,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::bulk_commit();
             }
             }
-            COMBA_ITER_NEXT();
         }
         if (issuer) tc::bulk_wait0();
     } else if (warp == kCtlWarp) {
@@ -789,7 +778,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                                       ((c - 1) >> 1) & 1, timeout_ns));
             __syncwarp();
             if (okw) {
-                COMBA_PHASE(21);
                 tc::tc_fence_after();
                 const uint32_t kqc = sb + kq_stage(c);
                 tc::mma_amn_bk(tmem + ((c & 1) ? TM_G1 : TM_G), kqc, KQ_ATOM, F1, ID_WN, 4, 0);
@@ -809,7 +797,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ok = tc::mbar_wait(&bars[B_WREADY], n & 1, timeout_ns);
             __syncwarp();
             if (!ok) break;
-            COMBA_PHASE(22);
             tc::tc_fence_after();
             tc::mma_bf16_ta_bmn(tmem + TM_X, tmem + TM_SB, sb + SM_V, 8192, ID_SW, 8, vzero ? 0u : 1u);
             tc::mma_commit(&bars[B_MMA1]);
@@ -821,12 +808,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ok = tc::mbar_wait(&bars[B_SPLIT], n & 1, timeout_ns);
             __syncwarp();
             if (!ok) break;
-            COMBA_PHASE(23);
             tc::tc_fence_after();
             tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH, kqn, KQ_ATOM, ID_SK, 4, 1);
             tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH + 32, kqn, KQ_ATOM, ID_SK, 4, 1);
             tc::mma_commit(&bars[B_MMA2]);
-            COMBA_PHASE(25);
             // ---- W^T / U~^T of chunk n+1 and the Gram of chunk n+2
             bool need_wn = n + 1 < nchunks, need_gram = n + 2 < nchunks;
             if (need_wn && need_gram &&
@@ -836,8 +821,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             if (ok && need_wn) ok = issue_wn(n + 1);
             if (ok && need_gram) ok = issue_gram(n + 2);
-            COMBA_PHASE(24);
-            COMBA_ITER_NEXT();
         }
         if (!ok) fail(gabort);
     } else {
@@ -917,11 +900,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                      (m < 2 || tc::mbar_wait(&bars[(m & 1) ? B_PBUF1 : B_PBUF0], ((m - 2) >> 1) & 1, timeout_ns));
                 __syncwarp();
                 tc::tc_fence_after();
-                COMBA_PHASE(7);
                 float a[32];
                 tc::tmem_ld32(tl + tgm + 32 * ch, a);
                 tc::tmem_ld_wait();
-                COMBA_PHASE(8);
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
                     tc::sts_f32x4(pbm + ch * F32_ATOM + tc::sw128(r, c),
@@ -943,7 +924,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     tc::tc_fence_before();
                     tc::named_barrier_arrive(BAR_KK, kKKThreads);
                 }
-                COMBA_PHASE(27);
                 // A_rs = beta_r e^{g_{r-1} - g_s} (K K^T)_rs for s < r -> -A into F2
                 if (fast) {
                     float cr = tc::lds_f32(ts + 768 + 4u * r);
@@ -960,17 +940,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         for (int e = 0; e < 4; ++e)
                             a[4 * c + e] = (32 * ch + 4 * c + e < r) ? cr * iv[e] * a[4 * c + e] : 0.f;
                     }
-                    COMBA_PHASE(28);
                     store_neg_a(F2p, r, ch, a);
                 } else {
                     a_rows_exact<kGated>(F2p, tl + tgm + 32 * ch, r, ch, ts, ts + 1792);
                 }
-                COMBA_PHASE(9);
                 if (pw != 0) {   // diagonal blocks 0, 1 (pw 3) and 2, 3 (pw 4) from this warp's rows
                     __syncwarp();
                     diag_block_inverse(F2p, (pw == 4 ? 2 : 0) + (lane >> 4), lane & 15);
                 }
-                COMBA_PHASE(10);
             } else if (p_warp) {
                 const int r = 32 * (q - 2) + lane;    // row (token) of this thread
                 ok = ok && tc::mbar_wait(&bars[(m & 1) ? B_GRAM1 : B_GRAM0], (m >> 1) & 1, timeout_ns);
@@ -1040,7 +1017,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     tc::sts_u32x4(pbm + F32_ATOM + tc::sw128(lane, c), make_uint4(0u, 0u, 0u, 0u));
                 tc::fence_proxy_async_smem();
             }
-            COMBA_PHASE(16);
             // ================= phase 2: next chunk's gate tables (gate warps) =================
             if (gate_warp && !last) {
                 make_tables(m + 1, la_x, bt_x);
@@ -1050,14 +1026,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
             if (!ok) fail(gabort);
-            COMBA_PHASE(17);
             if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
-            COMBA_PHASE(18);
             // ================= phase 3: the inverse's strips -> Tc / Eb ==========
             // F1 and diag(lo) are free once the previous chunk's W / U~ MMAs are done
             ok = ok && (m == 0 || tc::mbar_wait(&bars[B_WN], (m - 1) & 1, timeout_ns));
             __syncwarp();
-            COMBA_PHASE(11);
             if (ok) {
                 // the two longest strips (0, 1) on warps of schedulers 0 and 1 (warp % 4),
                 // the others spread so that each scheduler carries a similar MMA load
@@ -1065,7 +1038,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 strip_inverse(F2p, F1, strip, lane, ts + 768, ts + 512, kGated ? ts + 1792 : 0u);
                 if (pw == 4) strip_inverse(F2p, F1, 7, lane, ts + 768, ts + 512, kGated ? ts + 1792 : 0u);
             }
-            COMBA_PHASE(19);
             if (pt >= 128 && pt < 192) {   // diag(lo(beta))
                 const int e = pt - 128;
                 const float bv = tc::lds_f32(ts + 512 + 4u * e);
@@ -1079,15 +1051,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!tc::named_barrier_all_ok(BAR_PREP, kPrepThreads, ok && *gabort == 0)) break;
             if (issuer) tc::mbar_arrive(&bars[B_WNREADY]);   // Tc, Eb, diag(lo) of chunk m are in
             __syncwarp();
-            COMBA_PHASE(20);
-            COMBA_ITER_NEXT();
         }
     }
-    COMBA_PHASE_END();
 
     tc::tc_fence_before();
     __syncthreads();
-    COMBA_CTA_MARK(1);
     if (warp == 0) tc::tmem_dealloc(tmem, TM_COLS);
 }
 

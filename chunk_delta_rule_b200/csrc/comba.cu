@@ -616,35 +616,3 @@ extern "C" const char* comba_status_string(int status) {
 }
 
 extern "C" int comba_version(void) { return 100; }
-
-#ifdef COMBA_TRACE_PHASES
-// Tracing builds only: copies and clears the per-phase cycle counters.
-extern "C" int comba_trace_read_phases(unsigned long long* host_slots) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;
-    if (cudaMemcpyFromSymbol(host_slots, comba::g_phase_cycles,
-                             COMBA_TRACE_SLOTS * sizeof(unsigned long long)) != cudaSuccess)
-        return COMBA_ECUDA;
-    static const unsigned long long zeros[COMBA_TRACE_SLOTS] = {};
-    return cudaMemcpyToSymbol(comba::g_phase_cycles, zeros, sizeof(zeros)) == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
-}
-
-// Tracing builds only: per-CTA start / end global-timer stamps (2 per CTA, 1024 CTAs).
-extern "C" int comba_trace_read_cta(unsigned long long* host_2048) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;
-    return cudaMemcpyFromSymbol(host_2048, comba::g_cta_ns, 2048 * sizeof(unsigned long long)) ==
-                   cudaSuccess ? COMBA_OK : COMBA_ECUDA;
-}
-extern "C" int comba_trace_read_cta_clk(long long* host_3072) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;
-    return cudaMemcpyFromSymbol(host_3072, comba::g_cta_clk, 3072 * sizeof(long long)) ==
-                   cudaSuccess ? COMBA_OK : COMBA_ECUDA;
-}
-
-// Tracing builds only: absolute mark timestamps of three threads over four loop iterations.
-extern "C" int comba_trace_read_ts(long long* host_ts) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;
-    return cudaMemcpyFromSymbol(host_ts, comba::g_phase_ts,
-                                3 * COMBA_TRACE_TS_ITERS * COMBA_TRACE_SLOTS * sizeof(long long)) ==
-                   cudaSuccess ? COMBA_OK : COMBA_ECUDA;
-}
-#endif
