@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["chunk_fwd", "chunk_bwd", "state_compose", "chunk_fwd_gated", "chunk_fwd_host", "chunk_fwd_varlen", "chunk_fwd_noalloc",
+__all__ = ["chunk_fwd", "chunk_bwd", "state_compose", "chunk_fwd_transition", "chunk_fwd_gated", "chunk_fwd_host", "chunk_fwd_varlen", "chunk_fwd_noalloc",
            "recurrent_step",
            "get_last_error", "CombaError", "library", "library_path", "EXPORTS", "status_string"]
 
@@ -33,8 +33,9 @@ EXPORTS = ("comba_chunk_fwd", "comba_chunk_fwd_f32", "comba_chunk_fwd_varlen",
            "comba_chunk_fwd_workspace_size", "comba_chunk_fwd_ws", "comba_chunk_fwd_noalloc",
            "comba_chunk_fwd_host", "comba_chunk_fwd_host_workspace_size", "comba_chunk_fwd_gated",
            "comba_chunk_bwd", "comba_chunk_bwd_workspace_size", "comba_state_compose",
+           "comba_chunk_fwd_transition", "comba_chunk_fwd_stall_test",
            "comba_recurrent_step", "comba_recurrent_step_grouped", "comba_get_last_error",
-           "comba_status_string", "comba_version")
+           "comba_get_last_error_stream", "comba_status_string", "comba_version")
 
 
 class CombaError(RuntimeError):
@@ -73,15 +74,20 @@ def library():
             lib.comba_chunk_bwd.argtypes = [vp] * 16 + [i] * 6 + [vp, ctypes.c_size_t, vp]
             lib.comba_chunk_bwd_workspace_size.argtypes = [i] * 5
             lib.comba_state_compose.argtypes = [vp] * 3 + [i] * 3 + [vp]
+            lib.comba_chunk_fwd_transition.argtypes = [vp] * 7 + [i] * 6 + [vp]
+            lib.comba_chunk_fwd_stall_test.argtypes = [vp] * 9 + [i] * 6 + [ctypes.c_ulonglong, i, vp]
             lib.comba_chunk_bwd_workspace_size.restype = ctypes.c_size_t
             lib.comba_recurrent_step_grouped.argtypes = [vp] * 8 + [i] * 5 + [vp]
             for fn in (lib.comba_chunk_fwd, lib.comba_chunk_fwd_f32, lib.comba_chunk_fwd_ws,
                        lib.comba_chunk_fwd_noalloc, lib.comba_chunk_fwd_varlen,
                        lib.comba_recurrent_step_grouped, lib.comba_chunk_fwd_host,
                        lib.comba_chunk_fwd_gated, lib.comba_chunk_bwd, lib.comba_state_compose,
-                       lib.comba_recurrent_step, lib.comba_get_last_error, lib.comba_version):
+                       lib.comba_chunk_fwd_transition, lib.comba_chunk_fwd_stall_test,
+                       lib.comba_recurrent_step, lib.comba_get_last_error,
+                       lib.comba_get_last_error_stream, lib.comba_version):
                 fn.restype = ctypes.c_int
             lib.comba_get_last_error.argtypes = []
+            lib.comba_get_last_error_stream.argtypes = [vp]
             lib.comba_version.argtypes = []
             lib.comba_status_string.argtypes = [ctypes.c_int]
             lib.comba_status_string.restype = ctypes.c_char_p
@@ -116,6 +122,25 @@ def _stream_handle(device: torch.device, stream) -> ctypes.c_void_p:
     if isinstance(stream, torch.cuda.Stream):
         return ctypes.c_void_p(stream.cuda_stream)
     return ctypes.c_void_p(int(stream))
+
+
+def _keep_for_stream(t: Optional[torch.Tensor], device: torch.device, stream) -> None:
+    """A device buffer from PyTorch's caching allocator that a call enqueues work on
+    ``stream`` with: when that is not the device's current stream, the allocator is
+    told, so the memory is not handed out again before the stream has passed the
+    work (the allocator otherwise tracks only the stream it was allocated on)."""
+    if t is None or stream is None:
+        return
+    cur = torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream):
+        if stream.cuda_stream == cur.cuda_stream:
+            return
+        t.record_stream(stream)
+    else:
+        handle = int(stream)
+        if handle == cur.cuda_stream:
+            return
+        t.record_stream(torch.cuda.ExternalStream(handle, device=device))
 
 
 def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
@@ -162,6 +187,7 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
             nbytes = lib.comba_chunk_fwd_workspace_size(B, T, H, dk, dv, int(chunk)) if segment else 0
             ws = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
             st = lib.comba_chunk_fwd_ws(*args, _ptr(ws), nbytes, _stream_handle(dev, stream))
+            _keep_for_stream(ws, dev, stream)
             name = "comba_chunk_fwd_ws"
         else:
             st = lib.comba_chunk_fwd_f32(*args, _stream_handle(dev, stream))
@@ -233,9 +259,40 @@ def state_compose(R: torch.Tensor, M: torch.Tensor, S0: Optional[torch.Tensor] =
     with torch.cuda.device(dev):
         st = library().comba_state_compose(_ptr(RM), _ptr(S0), _ptr(S_start), B, H, P,
                                            _stream_handle(dev, stream))
+        _keep_for_stream(RM, dev, stream)
     if st != 0:
         raise CombaError(st, "comba_state_compose")
     return S_start
+
+
+def chunk_fwd_transition(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                         beta: torch.Tensor, d: torch.Tensor, chunk: int = 64,
+                         RM: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """comba_chunk_fwd_transition: the affine state transition of these tokens, (R, M)
+    with the state pass mapping S to S M + R.  q, k, v [B,T,H,128] bf16; log_alpha,
+    beta [B,T,H] fp32; d [H] fp32.  Returns R, M [B, H, 128, 128] fp32 (views of one
+    [2, B, H, 128, 128] buffer, ``RM`` if given)."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", torch.bfloat16, (B, T, H, dk))
+    _check(k, "k", torch.bfloat16, (B, T, H, dk))
+    _check(v, "v", torch.bfloat16, (B, T, H, dv))
+    _check(log_alpha, "log_alpha", torch.float32, (B, T, H))
+    _check(beta, "beta", torch.float32, (B, T, H))
+    _check(d, "d", torch.float32, (H,))
+    dev = q.device
+    if RM is None:
+        RM = torch.empty((2, B, H, dv, dk), dtype=torch.float32, device=dev)
+    _check(RM, "RM", torch.float32, (2, B, H, dv, dk))
+    with torch.cuda.device(dev):
+        st = library().comba_chunk_fwd_transition(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                                  _ptr(d), _ptr(RM), B, T, H, dk, dv, int(chunk),
+                                                  _stream_handle(dev, stream))
+    if st != 0:
+        raise CombaError(st, "comba_chunk_fwd_transition")
+    return RM[0], RM[1]
 
 
 _bwd_ws = {}
@@ -292,6 +349,7 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torc
                                  _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]), _ptr(g["dd"]), _ptr(g["dS0"]),
                                  B, T, H, dk, dv, 0 if dt == torch.bfloat16 else 1, _ptr(workspace),
                                  workspace.numel(), _stream_handle(dev, stream))
+        _keep_for_stream(workspace, dev, stream)   # also covers a cached buffer replaced later
     if st != 0:
         raise CombaError(st, "comba_chunk_bwd")
     return g
@@ -352,6 +410,7 @@ def chunk_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha:
         st = lib.comba_chunk_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(d),
                                       _ptr(S0), _ptr(out), _ptr(S_final), B, T, H, dk, dv, int(chunk),
                                       _ptr(workspace), nbytes, int(slices), _stream_handle(dev, stream))
+        _keep_for_stream(workspace, dev, stream)
     if st != 0:
         raise CombaError(st, "comba_chunk_fwd_host")
     return out, S_final
@@ -408,6 +467,8 @@ def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alp
                       stream=None) -> None:
     """comba_chunk_fwd_noalloc on caller-allocated bf16 tensors (same layouts as
     chunk_fwd): the segmented form's scratch is the library's static device array."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     for t, name in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
@@ -458,8 +519,12 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha:
     return out
 
 
-def get_last_error(device=None) -> int:
-    """Reads and clears the device-side status word (synchronises the device)."""
+def get_last_error(device=None, stream=None) -> int:
+    """Reads and clears the device-side status word.  Without ``stream`` the whole
+    device is synchronised first (comba_get_last_error); with one, only that stream
+    (comba_get_last_error_stream: the word is shared by all streams of the device)."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     with torch.cuda.device(dev):
-        return int(library().comba_get_last_error())
+        if stream is None:
+            return int(library().comba_get_last_error())
+        return int(library().comba_get_last_error_stream(_stream_handle(dev, stream)))

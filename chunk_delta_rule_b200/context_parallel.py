@@ -13,8 +13,11 @@ single-GPU path.  Each rank:
   3. composes the start states of all pieces with the library's compose kernel
      (S_start(0) = S0, S_start(p+1) = S_start(p) M_p + R_p) and keeps its own;
   4. reruns the chunk kernel over its piece from that state, for its outputs.
-Every step of the computation runs in the library's kernels; torch.distributed
-carries the exchange (NCCL between GPUs).  dk = dv = 128.
+Step 1 is one launch of the chunk kernel over the piece's chains twice stacked,
+with no outputs (comba_chunk_fwd_transition), so a rank runs the kernel's state
+pass twice and writes its outputs once.  Every step of the computation runs in
+the library's kernels; torch.distributed carries the exchange (NCCL between
+GPUs).  dk = dv = 128.
 """
 from __future__ import annotations
 
@@ -27,7 +30,12 @@ __all__ = ["chunk_fwd_context_parallel"]
 
 
 class _LibraryOps:
-    """The two library calls the context-parallel forward is built from."""
+    """The three library calls the context-parallel forward is built from."""
+
+    @staticmethod
+    def transition(q, k, v, log_alpha, beta, d, chunk):
+        from . import chunk_fwd_transition
+        return chunk_fwd_transition(q, k, v, log_alpha, beta, d, chunk=chunk)
 
     @staticmethod
     def fwd(q, k, v, log_alpha, beta, d, S0, chunk):
@@ -51,8 +59,8 @@ def chunk_fwd_context_parallel(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor
     (read on rank 0's behalf by every rank; pass the same tensor everywhere).
     Returns (out for this piece, this piece's end state); on the last rank the end
     state is the chains' final state.  Every rank must make the call (collective).
-    ``ops`` replaces the library calls (fwd, compose); it exists for the host tests
-    of the exchange."""
+    ``ops`` replaces the library calls (transition, fwd, compose); it exists for the
+    host tests of the exchange."""
     ops = ops or _LibraryOps()
     B, Tr, H, dk = q.shape
     dv = v.shape[-1]
@@ -60,11 +68,8 @@ def chunk_fwd_context_parallel(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor
         raise ValueError("context-parallel forward: dk = dv = 128")
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
-    dev = q.device
     # 1. this piece's transition
-    _, R = ops.fwd(q, k, v, log_alpha, beta, d, None, chunk)
-    eye = torch.eye(dv, dk, dtype=torch.float32, device=dev).expand(B, H, dv, dk).contiguous()
-    _, M = ops.fwd(q, k, torch.zeros_like(v), log_alpha, beta, d, eye, chunk)
+    R, M = ops.transition(q, k, v, log_alpha, beta, d, chunk)
     # 2. the exchange
     Rs = [torch.empty_like(R) for _ in range(world)]
     Ms = [torch.empty_like(M) for _ in range(world)]

@@ -114,6 +114,7 @@ inline int sm_count() {
     static int cached[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lock(init_mutex());
     if (!cached[dev]) {
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
@@ -141,12 +142,14 @@ inline int launch_segmented(const void* q, const void* k, const void* v, const f
     static bool attr_set[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -3;
+    std::unique_lock<std::mutex> lock(init_mutex());
     if (!attr_set[dev]) {
         if (cudaFuncSetAttribute(seg_compose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kComposeSmem) != cudaSuccess)
             return -3;
         attr_set[dev] = true;
     }
+    lock.unlock();
     seg_compose_kernel<<<B * H, kComposeThreads, kComposeSmem, stream>>>(RM, S0, Sst, B, H, P);
     if (cudaGetLastError() != cudaSuccess) return -3;
     if (int st = launch_chunk_tc(q, k, v, log_alpha, beta, d, Sst, out, Sfin, Bs, Ts, H, stream))

@@ -328,7 +328,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const float* __restrict__ dvec, const float* S0, float* S_final, int T, int H,
                     int b_split, int no_out, unsigned long long timeout_ns,
                     const int* __restrict__ cu_seqlens, int qk_group, unsigned short* out_raw,
-                    const float* __restrict__ A_log, const float* __restrict__ dt_bias, float norm_eps) {
+                    const float* __restrict__ A_log, const float* __restrict__ dt_bias, float norm_eps,
+                    int stall) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = tc::smem_u32(smem_raw);
     uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -358,7 +359,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // bf16 X' (SPLIT).
     enum { B_KQ0 = 0, B_V = 3, B_GRAM0 = 4, B_GRAM1 = 5, B_WN = 6, B_MMA1 = 7, B_MMA2 = 8,
            B_PBUF0 = 9, B_PBUF1 = 10, B_MMA1B = 11, B_WNREADY = 12, B_WREADY = 13, B_SPLIT = 14,
-           NBARS = 15 };
+           B_DRAIN = 15, NBARS = 16 };
+    // Waits that drain in-flight copies and MMAs before the CTA exits (after a wait has
+    // given up, say) get at least this long.
+    const unsigned long long drain_ns = timeout_ns > 100000000ull ? timeout_ns : 100000000ull;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM_MISC + 6144);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
     volatile int* gabort = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -556,6 +560,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             return okc;
         };
         bool ok = true;
+        // the last q/k and V chunks loaded into this CTA's shared memory (the prep group
+        // issues chunks 0 .. 2 and V of chunk 0 first)
+        int kq_last = (nchunks < kKQStages ? nchunks : kKQStages) - 1;
+        int v_last = vzero ? -1 : 0;
         // decays and Qh of chunk 0, initial state
         {
             const float la0 = (tid < 64) ? gate(log_alpha, tid) : 0.f;
@@ -628,7 +636,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // ---- X' = X diag(e^{g_L - g}) as bf16 hi + lo (operand of the state update)
             ok = ok && tc::mbar_wait(&bars[B_MMA1], n & 1, timeout_ns);
             tc::tc_fence_after();
-            if (issuer && ok && n + 1 < nchunks && !vzero) load_v(n + 1);   // MMA1 has read -W
+            if (issuer && ok && n + 1 < nchunks && !vzero) {   // MMA1 has read -W
+                load_v(n + 1);
+                v_last = n + 1;
+            }
             const uint32_t sedn = sed(n);
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
@@ -674,6 +685,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (issuer && n + kKQStages < nchunks) {   // this chunk's q/k stage is read
                 tc::fence_proxy_async_smem();
                 load_kq(n + kKQStages);
+                kq_last = n + kKQStages;
             }
             __syncwarp();
             // O^T row (value index) -> bf16 pairs of tokens
@@ -750,7 +762,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             }
         }
-        if (issuer) tc::bulk_wait0();
+        if (issuer) {
+            tc::bulk_wait0();
+            // every q/k and V copy issued into this CTA's shared memory (the prep group's
+            // first ones included) has landed before the CTA exits, also after a wait gave up
+            for (int c = kq_last - kKQStages + 1; c <= kq_last; ++c)
+                if (c >= 0) tc::mbar_wait(kq_bar(c), kq_par(c), drain_ns);
+            if (v_last >= 0) tc::mbar_wait(&bars[B_V], v_last & 1, drain_ns);
+        }
     } else if (warp == kCtlWarp) {
         // ============================ MMA-issue warp ===============================
         // All tensor-core MMAs.  Per chunk n: MMA1(n) (once the state group hands over
@@ -762,9 +781,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // n+1 yet.  The tensor pipe runs MMAs in issue order; every wait depends only
         // on MMAs issued before it, so no order of these can deadlock.
         bool ok = true;
+        // waits are made warp-uniform before any issue (the issuing helpers use the full mask)
         auto issue_gram = [&](int c) -> bool {
-            const bool okg = tc::mbar_wait(kq_bar(c), kq_par(c), timeout_ns);
-            __syncwarp();
+            const bool okg = __all_sync(0xffffffffu, tc::mbar_wait(kq_bar(c), kq_par(c), timeout_ns)) != 0;
             if (okg)
                 gram_mma(tmem + ((c & 1) ? TM_G1 : TM_G), sb + kq_stage(c), &bars[(c & 1) ? B_GRAM1 : B_GRAM0]);
             return okg;
@@ -772,11 +791,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // W^T = K^T Tc^T;  X^T = U~^T = V^T Eb^T + V^T diag(lo)^T  of chunk c (X^T of chunk
         // c-1 read by its O MMA, committed with its P buffer)
         auto issue_wn = [&](int c) -> bool {
-            const bool okw = tc::mbar_wait(&bars[B_WNREADY], c & 1, timeout_ns) &&
+            bool okw = tc::mbar_wait(&bars[B_WNREADY], c & 1, timeout_ns) &&
                              (vzero || tc::mbar_wait(&bars[B_V], c & 1, timeout_ns)) &&
                              (c == 0 || tc::mbar_wait(&bars[((c - 1) & 1) ? B_PBUF1 : B_PBUF0],
                                                       ((c - 1) >> 1) & 1, timeout_ns));
-            __syncwarp();
+            okw = __all_sync(0xffffffffu, okw) != 0;
             if (okw) {
                 tc::tc_fence_after();
                 const uint32_t kqc = sb + kq_stage(c);
@@ -790,12 +809,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             return okw;
         };
         ok = issue_gram(0) && (nchunks < 2 || issue_gram(1)) && issue_wn(0);
+        // stall: a wait on a phase that nothing completes before the drain below (the
+        // failure-path test), so it runs out after timeout_ns
+        if (ok && stall) ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars[B_DRAIN], 0, timeout_ns)) != 0;
         for (int n = 0; n < nchunks && ok; ++n) {
             const int stg = n & 1;
             const uint32_t kqn = sb + kq_stage(n);
             // ---- MMA1(n): X^T += S (-W)^T;  O^T = S Qh^T;  then O^T += X^T P^T
-            ok = tc::mbar_wait(&bars[B_WREADY], n & 1, timeout_ns);
-            __syncwarp();
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars[B_WREADY], n & 1, timeout_ns)) != 0;
             if (!ok) break;
             tc::tc_fence_after();
             tc::mma_bf16_ta_bmn(tmem + TM_X, tmem + TM_SB, sb + SM_V, 8192, ID_SW, 8, vzero ? 0u : 1u);
@@ -805,8 +826,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (want_out) tc::mma_tf32_ta_bk(tmem + TM_O, tmem + TM_X, sb + (stg ? SM_P1 : SM_P0), F32_ATOM, ID_XP, 8, 1);
             tc::mma_commit(&bars[stg ? B_PBUF1 : B_PBUF0]);
             // ---- MMA2(n): S += X'^T K (bf16 hi + lo)
-            ok = tc::mbar_wait(&bars[B_SPLIT], n & 1, timeout_ns);
-            __syncwarp();
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars[B_SPLIT], n & 1, timeout_ns)) != 0;
             if (!ok) break;
             tc::tc_fence_after();
             tc::mma_bf16_ta_bmn(tmem + TM_S, tmem + TM_XH, kqn, KQ_ATOM, ID_SK, 4, 1);
@@ -815,7 +835,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // ---- W^T / U~^T of chunk n+1 and the Gram of chunk n+2
             bool need_wn = n + 1 < nchunks, need_gram = n + 2 < nchunks;
             if (need_wn && need_gram &&
-                !(tc::mbar_test(&bars[B_WNREADY], (n + 1) & 1) && (vzero || tc::mbar_test(&bars[B_V], (n + 1) & 1)))) {
+                !__all_sync(0xffffffffu, tc::mbar_test(&bars[B_WNREADY], (n + 1) & 1) &&
+                                         (vzero || tc::mbar_test(&bars[B_V], (n + 1) & 1)))) {
                 ok = issue_gram(n + 2);
                 need_gram = false;
             }
@@ -823,6 +844,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (ok && need_gram) ok = issue_gram(n + 2);
         }
         if (!ok) fail(gabort);
+        // every MMA issued has completed before the CTA releases TMEM and exits
+        __syncwarp();
+        tc::mma_commit(&bars[B_DRAIN]);
+        tc::mbar_wait(&bars[B_DRAIN], 0, drain_ns);
+        __syncwarp();
     } else {
         // =============================== prep group ================================
         // Chunk m's operands for the MMA warp: the inverse's blocks, Tc / Eb, P and
@@ -1031,7 +1057,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // F1 and diag(lo) are free once the previous chunk's W / U~ MMAs are done
             ok = ok && (m == 0 || tc::mbar_wait(&bars[B_WN], (m - 1) & 1, timeout_ns));
             __syncwarp();
-            if (ok) {
+            if (__all_sync(0xffffffffu, ok)) {   // warp-uniform: the strips use full-warp shuffles and MMAs
                 // the two longest strips (0, 1) on warps of schedulers 0 and 1 (warp % 4),
                 // the others spread so that each scheduler carries a similar MMA load
                 const int strip = (pw == 3) ? 0 : (pw == 0) ? 1 : (pw <= 2) ? pw + 1 : (pw == 4) ? 6 : pw - 1;
@@ -1070,17 +1096,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 inline EncodeTiledFn encode_tiled_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    // resolved once (a function-local static is initialised once even under concurrent calls)
+    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+            return reinterpret_cast<EncodeTiledFn>(p);
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -1110,13 +1135,14 @@ inline int launch_chunk_tc(const void* q, const void* k, const void* v, const fl
                            int Bc = -1, unsigned long long timeout_ns = kWaitTimeoutNs,
                            const int* cu_seqlens = nullptr, int nseq = 0, int Hqk = 0,
                            const float* A_log = nullptr, const float* dt_bias = nullptr,
-                           float norm_eps = 0.f) {
+                           float norm_eps = 0.f, bool stall = false) {
     if (Bc < 0) Bc = B;
     if (Hqk <= 0) Hqk = H;
     if (H % Hqk != 0) return -1;
     static bool attr_set[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -3;
+    std::unique_lock<std::mutex> lock(init_mutex());
     if (!attr_set[dev]) {
         if (cudaFuncSetAttribute(tck::chunk_fwd_tc_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)tck::kSmemBytes) != cudaSuccess ||
@@ -1127,6 +1153,7 @@ inline int launch_chunk_tc(const void* q, const void* k, const void* v, const fl
             return -3;
         attr_set[dev] = true;
     }
+    lock.unlock();
     CUtensorMap tq, tk, tv, to;
     if (!make_tmap_bthd(&tq, q, B, T, Hqk) || !make_tmap_bthd(&tk, k, B, T, Hqk) ||
         !make_tmap_bthd(&tv, v, B, T, H) || !make_tmap_bthd(&to, out ? out : v, B, T, H))
@@ -1138,7 +1165,7 @@ inline int launch_chunk_tc(const void* q, const void* k, const void* v, const fl
                            : (A_log ? tck::chunk_fwd_tc_kernel<false, true> : tck::chunk_fwd_tc_kernel<false, false>);
     kern<<<(unsigned)(chains * H), tck::kThreads, tck::kSmemBytes, stream>>>(
         tq, tk, tv, to, log_alpha, beta, d, S0, S_final, T, H, b_split, out ? 0 : 1, timeout_ns,
-        cu_seqlens, H / Hqk, static_cast<unsigned short*>(out), A_log, dt_bias, norm_eps);
+        cu_seqlens, H / Hqk, static_cast<unsigned short*>(out), A_log, dt_bias, norm_eps, stall ? 1 : 0);
     return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 

@@ -107,6 +107,7 @@ int launch_simt(const ChunkArgs& a, cudaStream_t stream, Packing pk = Packing())
     static bool attr_set[kMaxDevices] = {};
     int dev;
     if (int st = current_device(&dev)) return st;
+    std::unique_lock<std::mutex> lock(comba::init_mutex());
     const int dvt = (a.dv % 32 == 0) ? 32 : 16;
     const SimtSmem m = comba::simt_smem_layout(a.dk, dvt, a.chunk);
     const size_t smem = m.total * sizeof(float);
@@ -118,6 +119,7 @@ int launch_simt(const ChunkArgs& a, cudaStream_t stream, Packing pk = Packing())
             return COMBA_ECUDA;
         attr_set[dev] = true;
     }
+    lock.unlock();
     dim3 grid((a.dv + dvt - 1) / dvt, a.H, pk.cu_seqlens ? pk.nseq : a.B);
     kern<<<grid, comba::kSimtThreads, smem, stream>>>(
         static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
@@ -139,6 +141,22 @@ extern "C" int comba_chunk_fwd(const void* q, const void* k, const void* v,
     if (T == 0) return empty_sequence(a, s);
     if (comba::tc_supported(dk, dv, chunk)) return comba::launch_chunk_tc(a.q, a.k, a.v, a.log_alpha, a.beta, a.d, a.S0, a.out, a.S_final, B, T, H, s);
     return launch_simt<__nv_bfloat16>(a, s);
+}
+
+extern "C" int comba_chunk_fwd_stall_test(const void* q, const void* k, const void* v,
+                                       const float* log_alpha, const float* beta, const float* d,
+                                       const float* S0, void* out, float* S_final, int B, int T, int H,
+                                       int dk, int dv, int chunk, unsigned long long timeout_ns,
+                                       int stall, comba_stream_t stream) {
+    const ChunkArgs a{q, k, v, log_alpha, beta, d, S0, out, S_final, B, T, H, dk, dv, chunk, 2};
+    if (int st = validate_chunk(a)) return st;
+    if (!comba::tc_supported(dk, dv, chunk)) return COMBA_EUNSUPPORTED;
+    if (B == 0 || H == 0) return COMBA_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) return empty_sequence(a, s);
+    return comba::launch_chunk_tc(q, k, v, log_alpha, beta, d, S0, out, S_final, B, T, H, s, -1, timeout_ns,
+                                  nullptr, 0, 0, nullptr, nullptr, 0.f, stall != 0) == 0
+               ? COMBA_OK : COMBA_ECUDA;
 }
 
 extern "C" int comba_chunk_fwd_varlen(const void* q, const void* k, const void* v,
@@ -257,6 +275,37 @@ extern "C" int comba_chunk_fwd_noalloc(const void* q, const void* k, const void*
                               sizeof(g_noalloc_ws), stream);
 }
 
+extern "C" int comba_chunk_fwd_transition(const void* q, const void* k, const void* v,
+                                          const float* log_alpha, const float* beta, const float* d,
+                                          float* RM, int B, int T, int H, int dk, int dv, int chunk,
+                                          comba_stream_t stream) {
+    // the input rules of comba_chunk_fwd; RM (two states per chain) must not overlap an input
+    if (B < 0 || T < 0 || H < 0) return COMBA_EINVAL;
+    if (B == 0 || H == 0) return COMBA_OK;
+    if (!comba::tc_supported(dk, dv, chunk)) return COMBA_EUNSUPPORTED;
+    if (!RM || !aligned(RM, 16) || !d || !aligned(d, 4)) return COMBA_EINVAL;
+    const size_t bph = (size_t)B * H, bth = (size_t)B * T * H;
+    if (bth > (size_t)1 << 40 || 2 * bph > (size_t)1 << 31) return COMBA_EINVAL;
+    const size_t nrm = 2 * bph * comba::seg::kStateFloats * sizeof(float);
+    if (T > 0) {
+        if (!q || !k || !v || !log_alpha || !beta) return COMBA_EINVAL;
+        if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(log_alpha, 4) || !aligned(beta, 4))
+            return COMBA_EINVAL;
+    }
+    const void* ins[] = {q, k, v, log_alpha, beta, d};
+    const size_t nin[] = {bth * dk * 2, bth * dk * 2, bth * dv * 2, bth * 4, bth * 4, (size_t)H * 4};
+    for (int i = 0; i < 6; ++i)
+        if (overlap(RM, nrm, ins[i], nin[i])) return COMBA_EINVAL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // RM starts as the stacked start states [0 | I]; the launch carries each in place to
+    // its end state (CTAs of the second half see V = 0)
+    comba::seg::seg_init_kernel<<<(unsigned)(2 * bph), 256, 0, s>>>(RM, (long)bph);
+    if (cudaGetLastError() != cudaSuccess) return COMBA_ECUDA;
+    if (T == 0) return COMBA_OK;
+    return comba::launch_chunk_tc(q, k, v, log_alpha, beta, d, RM, nullptr, RM, B, T, H, s, 2 * B) == 0
+               ? COMBA_OK : COMBA_ECUDA;
+}
+
 extern "C" int comba_chunk_fwd_f32(const float* q, const float* k, const float* v,
                                    const float* log_alpha, const float* beta, const float* d,
                                    const float* S0, float* out, float* S_final, int B, int T,
@@ -300,9 +349,16 @@ HostLayout host_layout(int B, int T, int H, int dk, int dv) {
 // Copy streams of one device, created on first use and kept for the process.
 bool copy_streams(int dev, cudaStream_t* h2d, cudaStream_t* d2h) {
     static cudaStream_t s[kMaxDevices][2] = {};
+    std::lock_guard<std::mutex> lock(comba::init_mutex());
     if (!s[dev][0]) {
-        if (cudaStreamCreateWithFlags(&s[dev][0], cudaStreamNonBlocking) != cudaSuccess) return false;
-        if (cudaStreamCreateWithFlags(&s[dev][1], cudaStreamNonBlocking) != cudaSuccess) return false;
+        cudaStream_t a = nullptr, b = nullptr;
+        if (cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking) != cudaSuccess) return false;
+        if (cudaStreamCreateWithFlags(&b, cudaStreamNonBlocking) != cudaSuccess) {
+            cudaStreamDestroy(a);
+            return false;
+        }
+        s[dev][0] = a;
+        s[dev][1] = b;
     }
     *h2d = s[dev][0];
     *d2h = s[dev][1];
@@ -594,13 +650,30 @@ extern "C" int comba_state_compose(const float* RM, const float* S0, float* S_st
     return cudaGetLastError() == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
 }
 
+namespace {
+
+// Reads and clears the current device's status word with copies ordered on `s`.
+int read_clear_status(cudaStream_t s) {
+    int h = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&h, comba::g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyToSymbolAsync(comba::g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return COMBA_ECUDA;
+    return h;
+}
+
+}  // namespace
+
 extern "C" int comba_get_last_error(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return COMBA_ECUDA;
-    int h = 0;
-    if (cudaMemcpyFromSymbol(&h, comba::g_status, sizeof(int)) != cudaSuccess) return COMBA_ECUDA;
-    const int zero = 0;
-    if (cudaMemcpyToSymbol(comba::g_status, &zero, sizeof(int)) != cudaSuccess) return COMBA_ECUDA;
-    return h;
+    return read_clear_status(nullptr);
+}
+
+extern "C" int comba_get_last_error_stream(comba_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return COMBA_ECUDA;
+    return read_clear_status(s);
 }
 
 extern "C" const char* comba_status_string(int status) {

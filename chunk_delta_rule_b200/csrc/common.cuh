@@ -5,7 +5,17 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace comba {
+
+// Host side: guards the library's lazily initialised per-device state (kernel
+// attributes, cached device properties, copy streams), so that threads making their
+// first calls at the same time initialise it once.
+inline std::mutex& init_mutex() {
+    static std::mutex m;
+    return m;
+}
 
 // Per-device status word.  Kernels latch the first device-side error here
 // (atomicCAS from 0); comba_get_last_error() reads and clears it.

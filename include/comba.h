@@ -202,6 +202,45 @@ int comba_chunk_fwd_host(const void* q, const void* k, const void* v,
                          comba_stream_t stream);
 
 /*
+ * comba_chunk_fwd on the tensor-core kernel (dk = dv = 128, chunk 64; other shapes
+ * return COMBA_EUNSUPPORTED) with its per-wait limit set to `timeout_ns` instead of
+ * the default 2 s, and, when `stall` is nonzero, with one extra wait (the MMA-issue
+ * warp's, before the first chunk's state pass) on a barrier phase that nothing
+ * completes.  It exists to exercise the kernel's failure path without faulting the
+ * GPU: the wait runs out, COMBA_ETIMEOUT is latched in the device status word
+ * (comba_get_last_error), every thread leaves the chunk loop (the other waits run
+ * out too), the kernel waits (for at least 100 ms more) for the copies and MMAs it
+ * has already issued, releases its tensor memory and returns; the outputs are then
+ * undefined.  With stall == 0 it is comba_chunk_fwd with another wait limit.
+ */
+int comba_chunk_fwd_stall_test(const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta, const float* d,
+                               const float* S0, void* out, float* S_final,
+                               int B, int T, int H, int dk, int dv, int chunk,
+                               unsigned long long timeout_ns, int stall, comba_stream_t stream);
+
+/*
+ * The affine state transition of a piece of sequence: over tokens 0 .. T-1 the
+ * state pass maps a start state S to S M + R (the write-up's "recurrent across
+ * blocks, parallel inside" form, section "硬件高效的分块并行计算", one level up:
+ * R is the end state from S = 0, M the end state from S = I with V = 0).  Both
+ * come from one launch of the tensor-core kernel over the chains twice stacked,
+ * with no outputs written; a caller that holds pieces of a longer sequence (one
+ * per GPU, say) composes the pieces' start states from them (comba_state_compose)
+ * and reruns each piece with comba_chunk_fwd.
+ *
+ * q, k, v, log_alpha, beta, d: as comba_chunk_fwd (bf16, dk = dv = 128, chunk 64;
+ * other shapes return COMBA_EUNSUPPORTED).  RM: fp32 [2, B, H, 128, 128] device
+ * memory, 16-byte aligned, not overlapping an input: R of every chain, then M of
+ * every chain (the layout comba_state_compose reads, with P = 1).  T == 0 gives
+ * R = 0, M = I.
+ */
+int comba_chunk_fwd_transition(const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta, const float* d,
+                               float* RM, int B, int T, int H, int dk, int dv, int chunk,
+                               comba_stream_t stream);
+
+/*
  * Chunk-wise forward with fp32 q, k, v and out (same math, same layouts, same
  * size rules as comba_chunk_fwd); every product is an fp32 FMA, no reduced-
  * precision tensor-core arithmetic.
@@ -301,10 +340,20 @@ int comba_state_compose(const float* RM, const float* S0, float* S_start, int B,
 
 /*
  * Reads and clears the current device's status word (synchronises the
- * device first).  Returns COMBA_OK, COMBA_ETIMEOUT, COMBA_EDEVICE, or
+ * device first).  Returns COMBA_OK, COMBA_ETIMEOUT, COMBA_EDEVICE, COMBA_EINVAL
+ * (a malformed packed-sequence bound, see comba_chunk_fwd_varlen), or
  * COMBA_ECUDA if the synchronisation or the read itself failed.
  */
 int comba_get_last_error(void);
+
+/*
+ * The same status word, read after synchronising `stream` only (work on other
+ * streams keeps running).  The word is shared by every stream of the device: it
+ * holds the first error latched by any of this library's kernels since the last
+ * read, so a kernel still running on another stream may latch an error after this
+ * call returns.  The read and the clear are ordered on `stream`.
+ */
+int comba_get_last_error_stream(comba_stream_t stream);
 
 /* Static, NUL-terminated description of a status code. */
 const char* comba_status_string(int status);

@@ -34,7 +34,7 @@ def test_header_declares_entry_points():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert set(declared_functions()) <= set(cdr.EXPORTS) | set(declared_functions())
+    assert set(declared_functions()) == set(cdr.EXPORTS)
 
 
 def test_version_and_status_strings(lib):
@@ -296,3 +296,27 @@ def test_state_compose_rejects_bad_arguments(lib):
     assert call(RM, S0, RM + 4096) == -1                # S_start inside RM
     assert call(RM, S0, S0 + 64) == -1                  # S_start overlaps S0
     assert call(None, None, None, B=0) == 0             # empty
+
+
+def test_chunk_transition_rejects_bad_arguments(lib):
+    p = lambda x: ctypes.c_void_p(x)
+
+    def call(q=BASE, k=BASE + GB, v=BASE + 2 * GB, la=BASE + 3 * GB, be=BASE + 4 * GB, d=BASE + 5 * GB,
+             RM=BASE + 6 * GB, B=2, T=128, H=4, dk=128, dv=128, chunk=64):
+        return lib.comba_chunk_fwd_transition(p(q), p(k), p(v), p(la), p(be), p(d), p(RM), B, T, H, dk, dv,
+                                              chunk, ctypes.c_void_p(None))
+
+    assert call(B=-1) == -1
+    assert call(RM=None) == -1
+    assert call(RM=BASE + 6 * GB + 8) == -1          # misaligned
+    assert call(q=BASE + 2) == -1                     # misaligned input
+    assert call(v=None) == -1
+    assert call(RM=BASE + 2 * GB + 4096) == -1       # RM inside v
+    assert call(dk=64, dv=64) == -2                   # only the tensor-core shape
+    assert call(chunk=32) == -2
+    assert call(B=0) == 0                             # empty: nothing launched
+
+
+def test_stream_status_read_is_exported(lib):
+    assert hasattr(lib, "comba_get_last_error_stream")
+    assert "comba_get_last_error_stream" in cdr.EXPORTS

@@ -28,6 +28,15 @@ class OracleOps:
         return torch.from_numpy(o), torch.from_numpy(S)
 
     @staticmethod
+    def transition(q, k, v, log_alpha, beta, d, chunk):
+        B, T, H, dk = q.shape
+        dv = v.shape[-1]
+        _, R = oracle.recurrence(q, k, v, log_alpha, beta, d, None)
+        eye = torch.eye(dv, dk, dtype=torch.float64).expand(B, H, dv, dk).contiguous()
+        _, M = oracle.recurrence(q, k, torch.zeros_like(v), log_alpha, beta, d, eye)
+        return torch.from_numpy(R), torch.from_numpy(M)
+
+    @staticmethod
     def compose(R, M, S0):
         B, P, H = R.shape[:3]
         S = torch.zeros_like(R[:, 0]) if S0 is None else S0.to(torch.float64)
