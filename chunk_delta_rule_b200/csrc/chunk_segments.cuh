@@ -61,52 +61,75 @@ __global__ void seg_init_kernel(float* S, long n_half) {
 }
 
 constexpr int kComposeThreads = 256;
-constexpr size_t kComposeSmem = 2 * kStateFloats * sizeof(float);   // S and M tiles
+constexpr int kComposeRows = 16;                              // state rows per CTA
+constexpr int kComposeBlocks = kD / kComposeRows;             // CTAs per chain
+constexpr size_t kComposeSmem = (size_t)(kComposeRows + kD) * kD * sizeof(float);   // S rows, M
 
-// One CTA per (b, h) chain: S_start(0) = S0 (or 0), S_start(p+1) = S_start(p) M_p + R_p,
-// written for p = 0 .. P-1 to Sst[(b P + p) H + h].  R_p, M_p sit in RM at stacked
-// batch b P + p and B P + b P + p.  Each thread owns an 8 x 8 tile of the product.
+// S_start(0) = S0 (or 0), S_start(p+1) = S_start(p) M_p + R_p, written for p = 0 .. P-1
+// to Sst[(b P + p) H + h].  R_p, M_p sit in RM at stacked batch b P + p and B P + b P +
+// p.  A row of S_start(p+1) depends only on the same row of S_start(p), so each chain's
+// 128 rows are split over kComposeBlocks CTAs that never communicate: CTA
+// (b H + h) kComposeBlocks + rb owns rows 16 rb .. 16 rb + 15, and thread t the 8
+// columns 8 (t % 16) .. + 7 of row t / 16.  Every output element is the same fp32 FMA
+// chain (R first, then k = 0 .. 127) whichever CTA computes it.
 __global__ void __launch_bounds__(kComposeThreads)
 seg_compose_kernel(const float* __restrict__ RM, const float* __restrict__ S0, float* __restrict__ Sst,
                    int B, int H, int P) {
-    extern __shared__ float smem[];
-    float* Sc = smem;                  // current start state, row-major dv x dk
-    float* Mt = smem + kStateFloats;   // this segment's transition, dk x dk
-    const int b = blockIdx.x / H, h = blockIdx.x % H, tid = threadIdx.x;
+    extern __shared__ __align__(16) float smem[];
+    float* Sc = smem;                              // the CTA's rows of the current start state
+    float* Mt = smem + kComposeRows * kD;          // this segment's transition, dk x dk
+    const int chain = blockIdx.x / kComposeBlocks, rb = blockIdx.x % kComposeBlocks;
+    const int b = chain / H, h = chain % H, tid = threadIdx.x;
+    const int i = tid / 16, j0 = (tid % 16) * 8, row = rb * kComposeRows + i;
     const long BP = (long)B * P;
     const float* s0 = S0 ? S0 + ((size_t)b * H + h) * kStateFloats : nullptr;
-    for (int i = tid; i < (int)kStateFloats; i += kComposeThreads) Sc[i] = s0 ? s0[i] : 0.f;
-    const int i0 = (tid / 16) * 8, j0 = (tid % 16) * 8;
+    float sv[8];
+    {
+        const float4 a4 = s0 ? *reinterpret_cast<const float4*>(s0 + (size_t)row * kD + j0) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 b4 = s0 ? *reinterpret_cast<const float4*>(s0 + (size_t)row * kD + j0 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        sv[0] = a4.x; sv[1] = a4.y; sv[2] = a4.z; sv[3] = a4.w;
+        sv[4] = b4.x; sv[5] = b4.y; sv[6] = b4.z; sv[7] = b4.w;
+    }
     for (int p = 0; p < P; ++p) {
-        __syncthreads();
-        float* dst = Sst + ((size_t)(b * P + p) * H + h) * kStateFloats;
-        for (int i = tid; i < (int)kStateFloats; i += kComposeThreads) dst[i] = Sc[i];
+        float* dst = Sst + ((size_t)(b * P + p) * H + h) * kStateFloats + (size_t)row * kD + j0;
+        *reinterpret_cast<float4*>(dst) = make_float4(sv[0], sv[1], sv[2], sv[3]);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(sv[4], sv[5], sv[6], sv[7]);
         if (p + 1 == P) break;
         const float* Rp = RM + ((size_t)(b * P + p) * H + h) * kStateFloats;
         const float* Mp = RM + ((size_t)(BP + b * P + p) * H + h) * kStateFloats;
-        for (int i = tid; i < (int)kStateFloats; i += kComposeThreads) Mt[i] = Mp[i];
-        __syncthreads();
-        float acc[8][8];
+        __syncthreads();   // the previous product is done with Sc and Mt
 #pragma unroll
-        for (int a = 0; a < 8; ++a)
+        for (int c = 0; c < 8; ++c) Sc[i * kD + j0 + c] = sv[c];
+        {   // M_p into shared memory: every 16-byte load issued before the stores
+            constexpr int PER = (int)(kStateFloats / 4) / kComposeThreads;
+            float4 m4[PER];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) acc[a][c] = Rp[(size_t)(i0 + a) * kD + j0 + c];
-        for (int k = 0; k < kD; ++k) {
-            float sv[8], mv[8];
+            for (int it = 0; it < PER; ++it)
+                m4[it] = *reinterpret_cast<const float4*>(Mp + 4 * (size_t)(tid + it * kComposeThreads));
 #pragma unroll
-            for (int a = 0; a < 8; ++a) sv[a] = Sc[(i0 + a) * kD + k];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) mv[c] = Mt[k * kD + j0 + c];
-#pragma unroll
-            for (int a = 0; a < 8; ++a)
-#pragma unroll
-                for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(sv[a], mv[c], acc[a][c]);
+            for (int it = 0; it < PER; ++it)
+                *reinterpret_cast<float4*>(Mt + 4 * (tid + it * kComposeThreads)) = m4[it];
+        }
+        float acc[8];
+        {
+            const float4 a4 = *reinterpret_cast<const float4*>(Rp + (size_t)row * kD + j0);
+            const float4 b4 = *reinterpret_cast<const float4*>(Rp + (size_t)row * kD + j0 + 4);
+            acc[0] = a4.x; acc[1] = a4.y; acc[2] = a4.z; acc[3] = a4.w;
+            acc[4] = b4.x; acc[5] = b4.y; acc[6] = b4.z; acc[7] = b4.w;
         }
         __syncthreads();
+#pragma unroll 4
+        for (int k = 0; k < kD; ++k) {
+            const float s = Sc[i * kD + k];
+            const float4 ma = *reinterpret_cast<const float4*>(Mt + k * kD + j0);
+            const float4 mb = *reinterpret_cast<const float4*>(Mt + k * kD + j0 + 4);
+            acc[0] = fmaf(s, ma.x, acc[0]); acc[1] = fmaf(s, ma.y, acc[1]);
+            acc[2] = fmaf(s, ma.z, acc[2]); acc[3] = fmaf(s, ma.w, acc[3]);
+            acc[4] = fmaf(s, mb.x, acc[4]); acc[5] = fmaf(s, mb.y, acc[5]);
+            acc[6] = fmaf(s, mb.z, acc[6]); acc[7] = fmaf(s, mb.w, acc[7]);
+        }
 #pragma unroll
-        for (int a = 0; a < 8; ++a)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) Sc[(i0 + a) * kD + j0 + c] = acc[a][c];
+        for (int c = 0; c < 8; ++c) sv[c] = acc[c];
     }
 }
 
@@ -150,7 +173,7 @@ inline int launch_segmented(const void* q, const void* k, const void* v, const f
         attr_set[dev] = true;
     }
     lock.unlock();
-    seg_compose_kernel<<<B * H, kComposeThreads, kComposeSmem, stream>>>(RM, S0, Sst, B, H, P);
+    seg_compose_kernel<<<B * H * kComposeBlocks, kComposeThreads, kComposeSmem, stream>>>(RM, S0, Sst, B, H, P);
     if (cudaGetLastError() != cudaSuccess) return -3;
     if (int st = launch_chunk_tc(q, k, v, log_alpha, beta, d, Sst, out, Sfin, Bs, Ts, H, stream))
         return st;

@@ -638,14 +638,15 @@ extern "C" int comba_state_compose(const float* RM, const float* S0, float* S_st
     if (!aligned(RM, 16) || !aligned(S0, 16) || !aligned(S_start, 16)) return COMBA_EINVAL;
     const size_t st = comba::seg::kStateFloats * sizeof(float);
     const size_t bph = (size_t)B * P * H;
-    if (bph > (size_t)1 << 31) return COMBA_EINVAL;
+    if (bph > (size_t)1 << 31 || (size_t)B * H * comba::seg::kComposeBlocks > (size_t)0x7fffffff) return COMBA_EINVAL;
     if (overlap(S_start, bph * st, RM, 2 * bph * st) || overlap(S_start, bph * st, S0, (size_t)B * H * st))
         return COMBA_EINVAL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaFuncSetAttribute(comba::seg::seg_compose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)comba::seg::kComposeSmem) != cudaSuccess)
         return COMBA_ECUDA;
-    comba::seg::seg_compose_kernel<<<(unsigned)(B * H), comba::seg::kComposeThreads, comba::seg::kComposeSmem, s>>>(
+    comba::seg::seg_compose_kernel<<<(unsigned)(B * H * comba::seg::kComposeBlocks), comba::seg::kComposeThreads,
+                                        comba::seg::kComposeSmem, s>>>(
         RM, S0, S_start, B, H, P);
     return cudaGetLastError() == cudaSuccess ? COMBA_OK : COMBA_ECUDA;
 }
