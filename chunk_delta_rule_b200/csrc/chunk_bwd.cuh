@@ -33,7 +33,10 @@
 // plus bwd_dd_sum, which adds the dd partials per head in a fixed order.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
+#include "tc_primitives.cuh"
 
 namespace comba {
 namespace bwd {
@@ -460,6 +463,126 @@ struct GradSmem {
 
 enum { V_G, V_GP, V_BT, V_EG, V_EGP, V_DEC, V_T1, V_T2, V_ROWA, V_COLA, V_ROWP, V_COLP, V_QG, V_F, V_DQK, V_DG };
 
+// The grads kernel takes the tensor-core form of its dv x dk contractions for bf16
+// inputs with dk = dv = 128 (below); other inputs keep fp32 FMA throughout.
+template <typename Tin, int DK, int DV>
+__host__ __device__ constexpr bool grads_tc() { return std::is_same<Tin, __nv_bfloat16>::value && DK == 128 && DV == 128; }
+
+// ---- tensor-core form of the grads kernel's five dv x dk contractions (bf16 inputs,
+// dk = dv = 128).  Each contraction over the 128-wide state index has a 128-row side,
+// so it runs as an M = 128, N = 32 (tokens), K = 128 tcgen05 MMA with A taken from
+// TMEM: S and dS' as bf16 rows (lane = state row i) and columns (lane = state column
+// j), built from the workspace's fp32 states; B is a 32-token bf16 tile in shared
+// memory (128B-swizzled, K-major, two 64-column atoms):
+//   (a) (K S^T)^T    = S K^T       A = S rows,     B = K
+//   (b) (K dS'^T)^T  = dS' K^T     A = dS' rows,   B = K
+//   (c) (dO S)^T     = S^T dO^T    A = S columns,  B = dO
+//   (d) (X dS')^T    = dS'^T X^T   A = dS' columns, B = X
+//   (e) (dR S)^T     = S^T dR^T    A = S columns,  B = dR
+// The results (fp32, lane = state index, column = token) are written back transposed
+// into the kernel's fp32 tiles.  bf16 operands for the states, X and dR put every
+// gradient of a bf16-input backward within 2e-3 (rel-L2) of the float64 gradients on
+// the 1.3B-layer inputs.
+namespace gtc {
+constexpr uint32_t C_S = 0, C_ST = 64, C_DS = 128, C_DST = 192;     // TMEM A operands (64 columns each)
+constexpr uint32_t C_A = 256, C_B = 288, C_C = 320, C_D = 352, C_E = 384;   // results (32 columns each)
+constexpr uint32_t kCols = 512;
+constexpr uint32_t TILE = 8192;                                     // one 32 x 128 bf16 B tile
+constexpr uint32_t KB = 0, OB = TILE, XB = 2 * TILE, DRB = 3 * TILE, BARS = 4 * TILE, SLOT = BARS + 64;
+constexpr uint32_t kBytes = SLOT + 64;
+constexpr uint32_t ID = tc::idesc_bf16(128, 32, false, false);
+enum { B_ABC = 0, B_D = 1, B_E = 2, B_DRAIN = 3 };
+constexpr unsigned long long kWaitNs = 2000000000ull;   // bound on every wait for an MMA
+
+// waits for a commit (each barrier completes once per CTA: phase 0); a wait that runs
+// out latches COMBA_ETIMEOUT and goes on, so the kernel still ends
+__device__ __forceinline__ void wait(uint64_t* bar) {
+    if (!tc::mbar_wait(bar, 0, kWaitNs)) latch_status(-4 /* COMBA_ETIMEOUT */);
+    tc::tc_fence_after();
+}
+
+// 16-byte piece c (0..15) of row r of a K-major 32 x 128 bf16 tile: 64-column atoms
+// 4096 bytes apart, 128B-swizzled rows
+__device__ __forceinline__ uint32_t boff(int r, int c) {
+    return (uint32_t)(c >> 3) * 4096u + tc::sw128((uint32_t)r, (uint32_t)(c & 7));
+}
+// rows [32, 128] of a [B, T, H, 128] bf16 tensor into a tile (zero past Lc)
+__device__ __forceinline__ void rows_to_tile(uint32_t dst, const __nv_bfloat16* __restrict__ src, size_t row0,
+                                             int H, int Lc) {
+    uint4 w[2];
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+        const int e = threadIdx.x + it * kThreads, r = e >> 4, c = e & 15;
+        w[it] = (r < Lc) ? *reinterpret_cast<const uint4*>(src + (row0 + (size_t)r * H) * 128 + 8 * c)
+                         : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+        const int e = threadIdx.x + it * kThreads;
+        tc::sts_u32x4(dst + boff(e >> 4, e & 15), w[it]);
+    }
+}
+// a 32 x 128 fp32 shared-memory tile (row stride ld) into a bf16 tile
+__device__ __forceinline__ void f32_to_tile(uint32_t dst, const float* t, int ld) {
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+        const int e = threadIdx.x + it * kThreads, r = e >> 4, c = e & 15;
+        const float* x = t + r * ld + 8 * c;
+        uint4 w;
+        w.x = tc::pack_bf16(x[0], x[1]);
+        w.y = tc::pack_bf16(x[2], x[3]);
+        w.z = tc::pack_bf16(x[4], x[5]);
+        w.w = tc::pack_bf16(x[6], x[7]);
+        tc::sts_u32x4(dst + boff(r, c), w);
+    }
+}
+// a 128 x 128 fp32 state (row-major, global) into TMEM as bf16 A operands: its rows
+// (lane i, columns [rows, +64): pairs (j, j+1)) and its columns (lane j, columns
+// [cols, +64): pairs (i, i+1)); called by one warp per TMEM lane quarter
+__device__ __forceinline__ void state_to_tmem(uint32_t tl, int lane_row, const float* __restrict__ Sg,
+                                              uint32_t rows, uint32_t cols) {
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {   // row lane_row, state columns 64 hh .. + 63
+        float v[64];
+#pragma unroll
+        for (int e = 0; e < 64; e += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(Sg + (size_t)lane_row * 128 + 64 * hh + e);
+            v[e] = x.x; v[e + 1] = x.y; v[e + 2] = x.z; v[e + 3] = x.w;
+        }
+        float pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = __uint_as_float(tc::pack_bf16(v[2 * c], v[2 * c + 1]));
+        tc::tmem_st32(tl + rows + 32 * hh, pk);
+    }
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {   // column lane_row, state rows 64 hh .. + 63
+        float v[64];
+#pragma unroll
+        for (int e = 0; e < 64; ++e) v[e] = Sg[(size_t)(64 * hh + e) * 128 + lane_row];
+        float pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = __uint_as_float(tc::pack_bf16(v[2 * c], v[2 * c + 1]));
+        tc::tmem_st32(tl + cols + 32 * hh, pk);
+    }
+}
+// 32 result columns of this thread's TMEM lane (state index x) into the fp32 tile
+// column x: t[r][x] = f(r, value)
+template <typename F>
+__device__ __forceinline__ void result_to_tile(uint32_t taddr, int x, float* t, int ld, int rows, const F& f) {
+    float v[32];
+    tc::tmem_ld32(taddr, v);
+    tc::tmem_ld_wait();
+#pragma unroll
+    for (int r = 0; r < 32; ++r)
+        if (r < rows) t[r * ld + x] = f(r, v[r], t[r * ld + x]);
+}
+}  // namespace gtc
+
+template <typename Tin, int DK, int DV>
+__host__ __device__ constexpr size_t grads_smem_bytes() {
+    return GradSmem<DK, DV>::total * sizeof(float) + (grads_tc<Tin, DK, DV>() ? 1024 + gtc::kBytes : 0);
+}
+
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kThreads)
 bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
@@ -485,6 +608,24 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     const float dh = d[h];
     const float* S = ws.S + ci * DV * DK;      // chunk-start state
     const float* dSp = ws.dS + ci * DV * DK;   // gradient at the chunk's end state
+    constexpr bool kTC = grads_tc<Tin, DK, DV>();
+    // tensor-core form: B tiles, barriers and the TMEM address slot after the fp32
+    // layout (1024-byte aligned); TMEM for the A operands and results
+    uint32_t tcb = 0, tmem = 0, ttl = 0;
+    uint64_t* tbar = nullptr;
+    const int xrow = (warp & 3) * 32 + lane;   // this thread's TMEM lane
+    if constexpr (kTC) {
+        const uint32_t s0 = tc::smem_u32(sm);
+        tcb = (tc::smem_u32(sm + SM::total) + 1023u) & ~1023u;
+        tbar = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sm) + (tcb - s0) + gtc::BARS);
+        if (tid == 0) {
+            for (int i = 0; i < 4; ++i) tc::mbar_init(&tbar[i], 1);
+            tc::fence_mbar_init();
+        }
+        if (warp == 0)
+            tc::tmem_alloc(reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(sm) + (tcb - s0) + gtc::SLOT),
+                           gtc::kCols);
+    }
 
     // 1. tiles and decays
     load_rows<DK>(Ks, LD, k, row0, H, Lc);
@@ -492,7 +633,23 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     load_rows<DV>(Os, LD, dout, row0, H, Lc);
     load_rows<DV>(Vs, LD, v, row0, H, Lc);
     chunk_decays(log_alpha, beta, row0, H, Lc, g, gp, bt);
+    if constexpr (kTC) {
+        gtc::rows_to_tile(tcb + gtc::KB, k, row0, H, Lc);
+        gtc::rows_to_tile(tcb + gtc::OB, dout, row0, H, Lc);
+        tc::tc_fence_before();
+    }
     __syncthreads();
+    if constexpr (kTC) {
+        tc::tc_fence_after();
+        tmem = *reinterpret_cast<volatile uint32_t*>(reinterpret_cast<uint8_t*>(sm) + (tcb - tc::smem_u32(sm)) +
+                                                     gtc::SLOT);
+        ttl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        if (warp < 4) gtc::state_to_tmem(ttl, xrow, S, gtc::C_S, gtc::C_ST);
+        else gtc::state_to_tmem(ttl, xrow, dSp, gtc::C_DS, gtc::C_DST);
+        tc::tmem_st_wait();
+        tc::fence_proxy_async_smem();   // the B tiles, written by threads, for the tensor pipe
+        tc::tc_fence_before();
+    }
     for (int e = tid; e < kL * DK; e += kThreads) {
         const int r = e / DK, j = e % DK;
         Qs[r * LD + j] = fmaf(-dh, Ks[r * LD + j], Qs[r * LD + j]);
@@ -503,18 +660,43 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         dec[tid] = expf(g[kL - 1] - g[tid]);
     }
     // 2. K S^T, AF, dX = diag(e^{g_L - g}) K dS'^T (P^T dO added below)
-    bgemm_staged<kL, DV, DK, 4, 4, true>([&](int r, int j) { return Ks[r * LD + j]; }, S, stage,
-                                         [&](int r, int i, float x) { Rs[r * LD + i] = x; });
-    bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Ks[m * LD + x]; },
-                            [&](int x, int n) { return Ks[n * LD + x]; },
-                            [&](int m, int n, float s) { AF[m * kLDL + n] = (n < m) ? expf(gp[m] - g[n]) * s : 0.f; });
-    __syncthreads();   // q~, decays
-    bgemm_staged<kL, DV, DK, 4, 4, true>([&](int r, int j) { return Ks[r * LD + j]; }, dSp, stage,
-                                         [&](int r, int i, float x) { Ds[r * LD + i] = dec[r] * x; });
-    bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Qs[m * LD + x]; },
-                            [&](int x, int n) { return Ks[n * LD + x]; },
-                            [&](int m, int n, float s) { Pm[m * kLDL + n] = (n <= m) ? expf(g[m] - g[n]) * s : 0.f; });
-    __syncthreads();
+    if constexpr (kTC) {
+        __syncthreads();   // q~, decays, the TMEM operands and the K / dO tiles
+        if (warp == 0) {   // (a) S K^T, (b) dS' K^T, (c) S^T dO^T
+            tc::tc_fence_after();
+            tc::mma_bf16_ta_bk(tmem + gtc::C_A, tmem + gtc::C_S, tcb + gtc::KB, 4096, gtc::ID, 8, 0);
+            tc::mma_bf16_ta_bk(tmem + gtc::C_B, tmem + gtc::C_DS, tcb + gtc::KB, 4096, gtc::ID, 8, 0);
+            tc::mma_bf16_ta_bk(tmem + gtc::C_C, tmem + gtc::C_ST, tcb + gtc::OB, 4096, gtc::ID, 8, 0);
+            tc::mma_commit(&tbar[gtc::B_ABC]);
+        }
+        bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Ks[m * LD + x]; },
+                                [&](int x, int n) { return Ks[n * LD + x]; },
+                                [&](int m, int n, float s) { AF[m * kLDL + n] = (n < m) ? expf(gp[m] - g[n]) * s : 0.f; });
+        bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Qs[m * LD + x]; },
+                                [&](int x, int n) { return Ks[n * LD + x]; },
+                                [&](int m, int n, float s) { Pm[m * kLDL + n] = (n <= m) ? expf(g[m] - g[n]) * s : 0.f; });
+        gtc::wait(&tbar[gtc::B_ABC]);
+        if (warp < 4) {
+            gtc::result_to_tile(ttl + gtc::C_A, xrow, Rs, LD, kL, [&](int, float x, float) { return x; });
+            gtc::result_to_tile(ttl + gtc::C_C, xrow, Gs, LD, kL, [&](int r, float x, float) { return eg[r] * x; });
+        } else {
+            gtc::result_to_tile(ttl + gtc::C_B, xrow, Ds, LD, kL, [&](int r, float x, float) { return dec[r] * x; });
+        }
+        __syncthreads();
+    } else {
+        bgemm_staged<kL, DV, DK, 4, 4, true>([&](int r, int j) { return Ks[r * LD + j]; }, S, stage,
+                                             [&](int r, int i, float x) { Rs[r * LD + i] = x; });
+        bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Ks[m * LD + x]; },
+                                [&](int x, int n) { return Ks[n * LD + x]; },
+                                [&](int m, int n, float s) { AF[m * kLDL + n] = (n < m) ? expf(gp[m] - g[n]) * s : 0.f; });
+        __syncthreads();   // q~, decays
+        bgemm_staged<kL, DV, DK, 4, 4, true>([&](int r, int j) { return Ks[r * LD + j]; }, dSp, stage,
+                                             [&](int r, int i, float x) { Ds[r * LD + i] = dec[r] * x; });
+        bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Qs[m * LD + x]; },
+                                [&](int x, int n) { return Ks[n * LD + x]; },
+                                [&](int m, int n, float s) { Pm[m * kLDL + n] = (n <= m) ? expf(g[m] - g[n]) * s : 0.f; });
+        __syncthreads();
+    }
     // 3. X = T diag(beta) (V - diag(e^{g'}) K S^T) by forward substitution (one column
     //    per thread); dX += P^T dO
     for (int col = tid; col < DV; col += kThreads) {
@@ -546,8 +728,21 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
 #pragma unroll
         for (int r = 0; r < kL; ++r) Ds[r * LD + col] = x[r];
     }
+    if constexpr (kTC) {
+        gtc::f32_to_tile(tcb + gtc::XB, Xs, LD);
+        tc::fence_proxy_async_smem();
+    }
     __syncthreads();
     // 5. dA, dP; row dots dR.(V - e^{g'} K S^T) and dR.(K S^T); Gamma dO S
+    if constexpr (kTC) {
+        if (warp == 0) {   // (d) dS'^T X^T
+            tc::tc_fence_after();
+            tc::mma_bf16_ta_bk(tmem + gtc::C_D, tmem + gtc::C_DST, tcb + gtc::XB, 4096, gtc::ID, 8, 0);
+            tc::mma_commit(&tbar[gtc::B_D]);
+        }
+        gtc::f32_to_tile(tcb + gtc::DRB, Ds, LD);
+        tc::fence_proxy_async_smem();
+    }
     bgemm<kL, kL, DV, 4, 1>([&](int r, int i) { return Ds[r * LD + i]; },
                             [&](int i, int s) { return Xs[s * LD + i]; },
                             [&](int r, int s, float x) { dAm[r * kLDL + s] = (s < r) ? -x : 0.f; });
@@ -568,13 +763,30 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
             V_(V_T2)[r] = t2;
         }
     }
-    bgemm_staged<kL, DK, DV, 4, 4, false>([&](int r, int i) { return Os[r * LD + i]; }, S, stage,
-                                          [&](int r, int j, float x) { Gs[r * LD + j] = eg[r] * x; });
+    if constexpr (!kTC)
+        bgemm_staged<kL, DK, DV, 4, 4, false>([&](int r, int i) { return Os[r * LD + i]; }, S, stage,
+                                              [&](int r, int j, float x) { Gs[r * LD + j] = eg[r] * x; });
     __syncthreads();
     // 6. F = diag(e^{g_L - g}) X dS' (over K S^T); sums of dA o AF and dP o P by row
-    //    and column; q~_r . (Gamma dO S)_r
-    bgemm_staged<kL, DK, DV, 4, 4, false>([&](int s, int i) { return Xs[s * LD + i]; }, dSp, stage,
-                                          [&](int s, int j, float x) { Rs[s * LD + j] = dec[s] * x; });
+    //    and column; q~_r . (Gamma dO S)_r.  The tensor-core form also takes dR S here
+    //    (into the V tile, free after step 5).
+    if constexpr (kTC) {
+        if (warp == 0) {   // (e) S^T dR^T
+            tc::tc_fence_after();
+            tc::mma_bf16_ta_bk(tmem + gtc::C_E, tmem + gtc::C_ST, tcb + gtc::DRB, 4096, gtc::ID, 8, 0);
+            tc::mma_commit(&tbar[gtc::B_E]);
+        }
+        if (warp < 4) {
+            gtc::wait(&tbar[gtc::B_D]);
+            gtc::result_to_tile(ttl + gtc::C_D, xrow, Rs, LD, kL, [&](int s, float x, float) { return dec[s] * x; });
+        } else {
+            gtc::wait(&tbar[gtc::B_E]);
+            gtc::result_to_tile(ttl + gtc::C_E, xrow, Vs, LD, kL, [&](int, float x, float) { return x; });
+        }
+    } else {
+        bgemm_staged<kL, DK, DV, 4, 4, false>([&](int s, int i) { return Xs[s * LD + i]; }, dSp, stage,
+                                              [&](int s, int j, float x) { Rs[s * LD + j] = dec[s] * x; });
+    }
     if (tid < kL) {
         const int r = tid;
         float ra = 0.f, rp = 0.f;
@@ -626,9 +838,10 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     bgemm<kL, DK, kL, 4, 4>([&](int r, int s) { return dAm[r * kLDL + s] + dAm[s * kLDL + r]; },
                             [&](int s, int j) { return Ks[s * LD + j]; },
                             [&](int r, int j, float x) { TKs[r * LD + j] += x; });
-    bgemm_staged<kL, DK, DV, 4, 4, false>(
-        [&](int r, int i) { return Ds[r * LD + i]; }, S, stage,
-        [&](int r, int j, float x) { TKs[r * LD + j] = fmaf(-bt[r] * egp[r], x, TKs[r * LD + j]); });
+    if constexpr (!kTC)
+        bgemm_staged<kL, DK, DV, 4, 4, false>(
+            [&](int r, int i) { return Ds[r * LD + i]; }, S, stage,
+            [&](int r, int j, float x) { TKs[r * LD + j] = fmaf(-bt[r] * egp[r], x, TKs[r * LD + j]); });
     __syncthreads();
     // 9. outputs: dq, dk, dv; decay gradients; dd partial
     for (int e = tid; e < Lc * DK; e += kThreads) {
@@ -636,7 +849,9 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         const size_t o = (row0 + (size_t)r * H) * DK + j;
         const float dqt = Gs[r * LD + j];
         dq[o] = dqt;
-        dk[o] = fmaf(-dh, dqt, TKs[r * LD + j] + Rs[r * LD + j]);
+        float tk = TKs[r * LD + j];
+        if constexpr (kTC) tk = fmaf(-bt[r] * egp[r], Vs[r * LD + j], tk);
+        dk[o] = fmaf(-dh, dqt, tk + Rs[r * LD + j]);
     }
     for (int e = tid; e < Lc * DV; e += kThreads) {
         const int r = e / DV, i = e % DV;
@@ -661,7 +876,17 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         x = warp_sum(x);
         if (lane == 0) V_(V_DQK)[r] = x;
     }
+    if constexpr (kTC) tc::tc_fence_before();
     __syncthreads();
+    if constexpr (kTC) {
+        if (warp == 0) {   // every MMA has completed before TMEM is released
+            tc::tc_fence_after();
+            tc::mma_commit(&tbar[gtc::B_DRAIN]);
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&tbar[gtc::B_DRAIN], 0, gtc::kWaitNs)) && lane == 0)
+                latch_status(-4 /* COMBA_ETIMEOUT */);
+            tc::tmem_dealloc(tmem, gtc::kCols);
+        }
+    }
     if (warp == 0) {
         const int r = lane;
         float sdS = 0.f;

@@ -530,7 +530,7 @@ int launch_bwd(const BwdArgs& a, float* wsp, cudaStream_t s) {
     const size_t sp = bw::PrepSmem<Tin, DK, DV>::total * sizeof(float);
     const size_t ss = bw::StatesSmem<DK, DV>::total * sizeof(float);
     const size_t sd = bw::DStatesSmem<DK, DV>::total * sizeof(float);
-    const size_t sg = bw::GradSmem<DK, DV>::total * sizeof(float);
+    const size_t sg = bw::grads_smem_bytes<Tin, DK, DV>();
     if (cudaFuncSetAttribute(bw::bwd_prep_kernel<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sp) != cudaSuccess ||
         cudaFuncSetAttribute(bw::bwd_states_kernel<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -18,6 +18,15 @@ pytestmark = pytest.mark.gpu
 # 1e-5; the backward chains two triangular solves and the state passes per chunk,
 # about an order of magnitude more rounding steps per result).
 TOL_BWD = dict(rel=1e-4, abs=None)
+# bf16 inputs with dk = dv = 128 take the tensor-core form of the five state
+# contractions (S and dS' against 32-token tiles of K, dO, X and dR), with the
+# states, X and dR rounded to bf16 as MMA operands: held to the bf16 workload
+# bound of the forward, rel-L2 5e-3.
+TOL_BWD_TC = dict(rel=5e-3, abs=None)
+
+
+def tol_for(dtype, dk, dv):
+    return TOL_BWD_TC if (dtype == "bf16" and dk == 128 and dv == 128) else TOL_BWD
 GRADS = ("dq", "dk", "dv", "dlog_alpha", "dbeta", "dd", "dS0")
 
 
@@ -51,7 +60,7 @@ def test_bwd_against_oracle(B, H, T, dk, dv, dtype):
                                             decay="mamba")
     x = make_chunk_inputs(cfg, seed=1000 + T + dk)
     cot = make_cotangents(cfg, seed=2000 + T)
-    check(x, cot, run(x, cot))
+    check(x, cot, run(x, cot), tol=tol_for(dtype, dk, dv))
 
 
 def test_bwd_strong_decay_and_no_state_cotangent():
@@ -102,9 +111,10 @@ def test_bwd_full_layer_sampled_chains():
         ref = oracle.recurrence_bwd_np(xs["q"], xs["k"], xs["v"], xs["log_alpha"], xs["beta"], xs["d"],
                                        xs["S0"], cs["dout"], cs["dS_final"])
         for n in ("dq", "dk", "dv"):
-            assert_close(f"{n}[{b},{h}]", g[n][b:b + 1, :, h:h + 1], ref[n], TOL_BWD)
+            assert_close(f"{n}[{b},{h}]", g[n][b:b + 1, :, h:h + 1], ref[n], TOL_BWD_TC)
         for n in ("dlog_alpha", "dbeta"):
-            assert_close(f"{n}[{b},{h}]", g[n][b:b + 1, :, h:h + 1], ref[n], TOL_BWD)
+            assert_close(f"{n}[{b},{h}]", g[n][b:b + 1, :, h:h + 1], ref[n], TOL_BWD_TC)
+        # dS0 comes from the state passes alone (fp32 FMA)
         assert_close(f"dS0[{b},{h}]", g["dS0"][b:b + 1, h:h + 1], ref["dS0"], TOL_BWD)
 
 
