@@ -46,7 +46,9 @@ constexpr int kLDL = kL + 1;     // padded row stride of the L x L tiles
 constexpr int kThreads = 256;
 
 // Per-chain workspace, chunk-major: W [L, dk], U~ [L, dv], C [dv, dk], S_c [dv, dk],
-// dS'_c [dv, dk] per chunk, then one dd partial per chunk.
+// dS'_c [dv, dk] per chunk, then one dd partial per chunk (fp32 slots).  In the
+// tensor-core form the W and C slots hold the state passes' operand tiles and S_c,
+// dS'_c are bf16 (the first half of their slots).
 struct Workspace {
     float *W, *U, *C, *S, *dS, *ddp;
 };
@@ -263,8 +265,56 @@ __device__ __forceinline__ void tile_to_smem(float* dst, int lds, const float* _
     }
 }
 
+// The grads kernel and the state passes take a tensor-core form for bf16 inputs with
+// dk = dv = 128 (chunk_bwd_chain.cuh and bwd_grads_kernel); other inputs keep fp32 FMA
+// throughout.
+template <typename Tin, int DK, int DV>
+__host__ __device__ constexpr bool grads_tc() { return std::is_same<Tin, __nv_bfloat16>::value && DK == 128 && DV == 128; }
+
+// ---- bf16 32 x 128 tiles in the layout the tensor-core kernels read.  Row r (a token),
+// 16-byte piece c (elements 8c .. 8c+7) sits at byte (c / 8) 4096 + the 128B-swizzled
+// place of piece c % 8 in row r: two 64-column atoms of 32 rows x 128 B.  Copied to a
+// 1024-byte-aligned shared-memory address, a tile is a K-major MMA operand with the
+// tokens as rows, or an MN-major one with the tokens as its K index.
+namespace tile {
+constexpr uint32_t kBytes = 8192;
+__host__ __device__ constexpr uint32_t off(int r, int c) {
+    return (uint32_t)(c >> 3) * 4096u + (uint32_t)r * 128u + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
+}
+// an fp32 32 x 128 tile (row stride ld) into a bf16 tile at dst: its bf16 rounding, or
+// with kLo the rounding residual (x - bf16(x), rounded)
+template <bool kLo>
+__device__ __forceinline__ void from_f32(uint8_t* dst, const float* t, int ld) {
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+        const int e = threadIdx.x + it * kThreads, r = e >> 4, c = e & 15;
+        const float* x = t + r * ld + 8 * c;
+        uint32_t w[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            float a = x[2 * p], b = x[2 * p + 1];
+            if constexpr (kLo) {
+                a -= __bfloat162float(__float2bfloat16_rn(a));
+                b -= __bfloat162float(__float2bfloat16_rn(b));
+            }
+            const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+            w[p] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(dst + off(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+}  // namespace tile
+
+// Byte offset, inside a chunk's C slot of the workspace, of the decays the tensor-core
+// state passes read (e^{g_L - g_r} for the 32 positions, then e^{g_L}); before it: the
+// G hi, G lo and dO tiles.
+constexpr uint32_t kPrepDec = 3 * tile::kBytes;
+
 // ---------------------------------------------------------------------------------
-// bwd_prep: W, U~ and C = dO^T (Gamma Q~ - P W) of one chunk.
+// bwd_prep: W, U~ and C = dO^T (Gamma Q~ - P W) of one chunk.  In the tensor-core form
+// it leaves, instead of W and C in fp32, the operands of the state passes: the W and K
+// tiles (in W's slot), U~ (fp32, as before), the G = Gamma Q~ - P W hi and lo tiles, the
+// dO tile and the decays (in C's slot).
 template <typename Tin, int DK, int DV>
 struct PrepSmem {
     static constexpr int LDK = DK + 1, LDV = DV + 1;
@@ -294,6 +344,19 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     load_rows<DV>(Os, LDV, dout, row0, H, Lc);
     chunk_decays(log_alpha, beta, row0, H, Lc, g, gp, bt);
     __syncthreads();
+    constexpr bool kTC = grads_tc<Tin, DK, DV>();
+    const size_t ci = (size_t)bh * nch + c;
+    uint8_t* wk = reinterpret_cast<uint8_t*>(ws.W + ci * kL * DK);   // tensor-core form: W | K tiles
+    uint8_t* cs = reinterpret_cast<uint8_t*>(ws.C + ci * DV * DK);   // G hi | G lo | dO tiles, decays
+    if constexpr (kTC) {
+        tile::from_f32<false>(wk + tile::kBytes, Ks, LDK);
+        tile::from_f32<false>(cs + 2 * tile::kBytes, Os, LDV);
+        if (threadIdx.x < kL) {
+            float* dd = reinterpret_cast<float*>(cs + kPrepDec);
+            dd[threadIdx.x] = expf(g[kL - 1] - g[threadIdx.x]);
+            if (threadIdx.x == 0) dd[kL] = expf(g[kL - 1]);
+        }
+    }
     for (int e = threadIdx.x; e < kL * DK; e += kThreads) {   // q~ = q - d k
         const int r = e / DK, j = e % DK;
         Qs[r * LDK + j] = fmaf(-dh, Ks[r * LDK + j], Qs[r * LDK + j]);
@@ -332,15 +395,20 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
                             [&](int x, int n) { return Ks[x * LDK + n]; },
                             [&](int m, int n, float s) { Qs[m * LDK + n] = fmaf(expf(g[m]), Qs[m * LDK + n], -s); });
     __syncthreads();
-    const size_t ci = (size_t)bh * nch + c;
-    float* Cg = ws.C + ci * DV * DK;
-    bgemm<DV, DK, kL, 8, 8>([&](int i, int r) { return Os[r * LDV + i]; },
-                            [&](int r, int j) { return Qs[r * LDK + j]; },
-                            [&](int i, int j, float s) { Cg[(size_t)i * DK + j] = s; });
-    float* Wg = ws.W + ci * kL * DK;
     float* Ug = ws.U + ci * kL * DV;
-    for (int e = threadIdx.x; e < kL * DK; e += kThreads) Wg[e] = Ks[(e / DK) * LDK + e % DK];
     for (int e = threadIdx.x; e < kL * DV; e += kThreads) Ug[e] = Vs[(e / DV) * LDV + e % DV];
+    if constexpr (kTC) {
+        tile::from_f32<false>(wk, Ks, LDK);
+        tile::from_f32<false>(cs, Qs, LDK);
+        tile::from_f32<true>(cs + tile::kBytes, Qs, LDK);
+    } else {
+        float* Cg = ws.C + ci * DV * DK;
+        bgemm<DV, DK, kL, 8, 8>([&](int i, int r) { return Os[r * LDV + i]; },
+                                [&](int r, int j) { return Qs[r * LDK + j]; },
+                                [&](int i, int j, float s) { Cg[(size_t)i * DK + j] = s; });
+        float* Wg = ws.W + ci * kL * DK;
+        for (int e = threadIdx.x; e < kL * DK; e += kThreads) Wg[e] = Ks[(e / DK) * LDK + e % DK];
+    }
 }
 
 // ---------------------------------------------------------------------------------
@@ -463,10 +531,6 @@ struct GradSmem {
 
 enum { V_G, V_GP, V_BT, V_EG, V_EGP, V_DEC, V_T1, V_T2, V_ROWA, V_COLA, V_ROWP, V_COLP, V_QG, V_F, V_DQK, V_DG };
 
-// The grads kernel takes the tensor-core form of its dv x dk contractions for bf16
-// inputs with dk = dv = 128 (below); other inputs keep fp32 FMA throughout.
-template <typename Tin, int DK, int DV>
-__host__ __device__ constexpr bool grads_tc() { return std::is_same<Tin, __nv_bfloat16>::value && DK == 128 && DV == 128; }
 
 // ---- tensor-core form of the grads kernel's five dv x dk contractions (bf16 inputs,
 // dk = dv = 128).  Each contraction over the 128-wide state index has a 128-row side,
@@ -503,9 +567,7 @@ __device__ __forceinline__ void wait(uint64_t* bar) {
 
 // 16-byte piece c (0..15) of row r of a K-major 32 x 128 bf16 tile: 64-column atoms
 // 4096 bytes apart, 128B-swizzled rows
-__device__ __forceinline__ uint32_t boff(int r, int c) {
-    return (uint32_t)(c >> 3) * 4096u + tc::sw128((uint32_t)r, (uint32_t)(c & 7));
-}
+__device__ __forceinline__ uint32_t boff(int r, int c) { return tile::off(r, c); }
 // rows [32, 128] of a [B, T, H, 128] bf16 tensor into a tile (zero past Lc)
 __device__ __forceinline__ void rows_to_tile(uint32_t dst, const __nv_bfloat16* __restrict__ src, size_t row0,
                                              int H, int Lc) {
@@ -536,32 +598,32 @@ __device__ __forceinline__ void f32_to_tile(uint32_t dst, const float* t, int ld
         tc::sts_u32x4(dst + boff(r, c), w);
     }
 }
-// a 128 x 128 fp32 state (row-major, global) into TMEM as bf16 A operands: its rows
-// (lane i, columns [rows, +64): pairs (j, j+1)) and its columns (lane j, columns
-// [cols, +64): pairs (i, i+1)); called by one warp per TMEM lane quarter
-__device__ __forceinline__ void state_to_tmem(uint32_t tl, int lane_row, const float* __restrict__ Sg,
+// a 128 x 128 bf16 state (row-major, global: the state passes' output) into TMEM as
+// A operands: its rows (lane i, columns [rows, +64): pairs (j, j+1)) and its columns
+// (lane j, columns [cols, +64): pairs (i, i+1)); called by one warp per TMEM lane quarter
+__device__ __forceinline__ void state_to_tmem(uint32_t tl, int lane_row, const __nv_bfloat16* __restrict__ Sg,
                                               uint32_t rows, uint32_t cols) {
 #pragma unroll 1
-    for (int hh = 0; hh < 2; ++hh) {   // row lane_row, state columns 64 hh .. + 63
-        float v[64];
-#pragma unroll
-        for (int e = 0; e < 64; e += 4) {
-            const float4 x = *reinterpret_cast<const float4*>(Sg + (size_t)lane_row * 128 + 64 * hh + e);
-            v[e] = x.x; v[e + 1] = x.y; v[e + 2] = x.z; v[e + 3] = x.w;
-        }
+    for (int hh = 0; hh < 2; ++hh) {   // row lane_row, state columns 64 hh .. + 63: already pairs
         float pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = __uint_as_float(tc::pack_bf16(v[2 * c], v[2 * c + 1]));
+        for (int e = 0; e < 8; ++e) {
+            const uint4 x = *reinterpret_cast<const uint4*>(Sg + (size_t)lane_row * 128 + 64 * hh + 8 * e);
+            pk[4 * e] = __uint_as_float(x.x); pk[4 * e + 1] = __uint_as_float(x.y);
+            pk[4 * e + 2] = __uint_as_float(x.z); pk[4 * e + 3] = __uint_as_float(x.w);
+        }
         tc::tmem_st32(tl + rows + 32 * hh, pk);
     }
+    const unsigned short* Su = reinterpret_cast<const unsigned short*>(Sg);
 #pragma unroll 1
     for (int hh = 0; hh < 2; ++hh) {   // column lane_row, state rows 64 hh .. + 63
-        float v[64];
-#pragma unroll
-        for (int e = 0; e < 64; ++e) v[e] = Sg[(size_t)(64 * hh + e) * 128 + lane_row];
         float pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = __uint_as_float(tc::pack_bf16(v[2 * c], v[2 * c + 1]));
+        for (int c = 0; c < 32; ++c) {
+            const uint32_t lo = Su[(size_t)(64 * hh + 2 * c) * 128 + lane_row];
+            const uint32_t hi = Su[(size_t)(64 * hh + 2 * c + 1) * 128 + lane_row];
+            pk[c] = __uint_as_float(lo | (hi << 16));
+        }
         tc::tmem_st32(tl + cols + 32 * hh, pk);
     }
 }
@@ -644,8 +706,8 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         tmem = *reinterpret_cast<volatile uint32_t*>(reinterpret_cast<uint8_t*>(sm) + (tcb - tc::smem_u32(sm)) +
                                                      gtc::SLOT);
         ttl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        if (warp < 4) gtc::state_to_tmem(ttl, xrow, S, gtc::C_S, gtc::C_ST);
-        else gtc::state_to_tmem(ttl, xrow, dSp, gtc::C_DS, gtc::C_DST);
+        if (warp < 4) gtc::state_to_tmem(ttl, xrow, reinterpret_cast<const __nv_bfloat16*>(S), gtc::C_S, gtc::C_ST);
+        else gtc::state_to_tmem(ttl, xrow, reinterpret_cast<const __nv_bfloat16*>(dSp), gtc::C_DS, gtc::C_DST);
         tc::tmem_st_wait();
         tc::fence_proxy_async_smem();   // the B tiles, written by threads, for the tensor pipe
         tc::tc_fence_before();
@@ -859,7 +921,19 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     }
     // <dS', S> and sum_r dq~_r . k_r (block sums in a fixed order)
     float ss = 0.f;
-    {
+    if constexpr (kTC) {   // bf16 states
+        constexpr int PER = DV * DK / 8 / kThreads;   // 16-byte pieces of each matrix per thread
+        const uint4* x8 = reinterpret_cast<const uint4*>(dSp);
+        const uint4* y8 = reinterpret_cast<const uint4*>(S);
+#pragma unroll 4
+        for (int it = 0; it < PER; ++it) {
+            float fx[8], fy[8];
+            unpack16(x8[tid + it * kThreads], fx);
+            unpack16(y8[tid + it * kThreads], fy);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(fx[e], fy[e], ss);
+        }
+    } else {
         constexpr int PER = DV * DK / 4 / kThreads;   // float4s of each matrix per thread
 #pragma unroll 4
         for (int it = 0; it < PER; ++it) {

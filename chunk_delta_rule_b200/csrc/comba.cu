@@ -19,6 +19,7 @@
 #include "chunk_tc.cuh"
 #include "chunk_segments.cuh"
 #include "chunk_bwd.cuh"
+#include "chunk_bwd_chain.cuh"
 #include "recurrent_step.cuh"
 
 namespace {
@@ -540,14 +541,27 @@ int launch_bwd(const BwdArgs& a, float* wsp, cudaStream_t s) {
         cudaFuncSetAttribute(bw::bwd_grads_kernel<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sg) != cudaSuccess)
         return COMBA_ECUDA;
-    if (chains > 0 && nch > 0) {
+    if constexpr (bw::grads_tc<Tin, DK, DV>()) {
+        // prep, then both state passes in one launch (2 x chains CTAs), then the grads
+        if (cudaFuncSetAttribute(bw::chain::bwd_chain_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)bw::chain::kSmemBytes) != cudaSuccess)
+            return COMBA_ECUDA;
+        if (chains > 0 && nch > 0) {
+            const dim3 grid((unsigned)nch, (unsigned)chains);
+            bw::bwd_prep_kernel<Tin, DK, DV><<<grid, bw::kThreads, sp, s>>>(q, k, v, a.log_alpha, a.beta, a.d, o,
+                                                                             ws, a.T, a.H, nch);
+        }
+        if (chains > 0)
+            bw::chain::bwd_chain_tc_kernel<<<(unsigned)(2 * chains), bw::chain::kThreads, bw::chain::kSmemBytes, s>>>(
+                ws, a.S0, a.dS_final, a.dS0, (int)chains, nch);
+    } else if (chains > 0 && nch > 0) {
         const dim3 grid((unsigned)nch, (unsigned)chains);
         bw::bwd_prep_kernel<Tin, DK, DV><<<grid, bw::kThreads, sp, s>>>(q, k, v, a.log_alpha, a.beta, a.d, o, ws,
                                                                          a.T, a.H, nch);
         bw::bwd_states_kernel<Tin, DK, DV><<<(unsigned)(chains * (DV / bw::kRows)), bw::kThreads, ss, s>>>(k, a.log_alpha, a.beta, a.S0,
                                                                                        ws, a.T, a.H, nch);
     }
-    if (chains > 0)
+    if (!bw::grads_tc<Tin, DK, DV>() && chains > 0)
         bw::bwd_dstates_kernel<Tin, DK, DV><<<(unsigned)(chains * (DV / bw::kRows)), bw::kThreads, sd, s>>>(
             k, a.log_alpha, a.beta, a.dS_final, a.dS0, ws, a.T, a.H, nch);
     if (chains > 0 && nch > 0) {

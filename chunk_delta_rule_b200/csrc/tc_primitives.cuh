@@ -289,6 +289,15 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void*
         : "memory");
 }
 
+// Untiled bulk copy of `bytes` from global memory into this CTA's shared memory,
+// completing that many bytes of transaction count on `bar` (no multicast).  Both
+// addresses 16-byte aligned, `bytes` a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -393,6 +402,17 @@ __device__ __forceinline__ void mma_bf16_ta_bmn(uint32_t d, uint32_t a_tmem, uin
 #pragma unroll kMmaUnroll
     for (int ks = 0; ks < ksteps; ++ks)
         mma_bf16_ta(d, a_tmem + ks * 8, bd0 + (uint32_t)(ks * (2048 >> 4)), idesc, (ks > 0) ? 1u : acc0);
+}
+
+// bf16, A and B both MN-major from shared memory (M and N in 64-element atoms
+// `a_lbo` / `b_lbo` bytes apart; one 128 B row per K index in each).
+__device__ __forceinline__ void mma_amn_bmn(uint32_t d, uint32_t a, uint32_t a_lbo, uint32_t b,
+                                            uint32_t b_lbo, uint32_t idesc, int ksteps, uint32_t acc0) {
+    const uint64_t ad0 = sdesc_sw128(a, a_lbo, 1024), bd0 = sdesc_sw128(b, b_lbo, 1024);
+#pragma unroll kMmaUnroll
+    for (int ks = 0; ks < ksteps; ++ks)
+        mma_bf16(d, ad0 + (uint32_t)(ks * (2048 >> 4)), bd0 + (uint32_t)(ks * (2048 >> 4)), idesc,
+                 (ks > 0) ? 1u : acc0);
 }
 
 // ---------------------------------------------------------------- warp MMA (legacy)
