@@ -42,7 +42,7 @@ namespace comba {
 namespace bwd {
 
 constexpr int kL = 32;           // tokens per backward chunk (one warp's lanes)
-constexpr int kLDL = kL + 1;     // padded row stride of the L x L tiles
+constexpr int kLDL = kL + 4;     // padded row stride of the L x L tiles (4 mod 32: see wgemm)
 constexpr int kThreads = 256;
 
 // Per-chain workspace, chunk-major: W [L, dk], U~ [L, dv], C [dv, dk], S_c [dv, dk],
@@ -103,6 +103,50 @@ __device__ __forceinline__ void bgemm(const FA& a, const FB& b, const Epi& epi) 
         for (int i = 0; i < TM; ++i)
 #pragma unroll
             for (int j = 0; j < TN; ++j) epi(mt + i * MS, nt + j * NS, acc[i][j]);
+    }
+}
+
+// C(m, n) = sum_k a(m, k) b(k, n) on the warp tensor cores (m16n8k8 tf32 MMAs),
+// handed to epi(m, n, c).  kSa / kSb: that operand holds values with more than tf32
+// precision (fp32 results), so it is split into tf32 hi + lo and the product formed
+// as hi.lo + lo.hi + hi.hi, about fp32 accuracy; an operand exact in tf32 (bf16
+// inputs widened to fp32) skips the split.  Warp w takes the 16 x 8 output tiles w,
+// w + 8, ...; an element's owner depends only on <M, N>, so calls with the same M
+// and N may accumulate into one buffer without a barrier between them.  Fragment
+// loads hit distinct banks when the operands' row strides are 4 mod 32 (row g,
+// column t of a fragment: bank 4 g + t), in either orientation.
+template <int M, int N, int K, bool kSa, bool kSb, typename FA, typename FB, typename Epi>
+__device__ __forceinline__ void wgemm(const FA& a, const FB& b, const Epi& epi) {
+    static_assert(M % 16 == 0 && N % 8 == 0 && K % 8 == 0, "m16n8k8 tiles must divide the product");
+    constexpr int NT = N / 8, TILES = (M / 16) * NT;
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    for (int tt = threadIdx.x >> 5; tt < TILES; tt += kThreads / 32) {
+        const int m0 = (tt / NT) * 16, n0 = (tt % NT) * 8;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int k0 = 0; k0 < K; k0 += 8) {
+            const float av[4] = {a(m0 + g, k0 + t), a(m0 + g + 8, k0 + t), a(m0 + g, k0 + t + 4),
+                                 a(m0 + g + 8, k0 + t + 4)};
+            const float bv[2] = {b(k0 + t, n0 + g), b(k0 + t + 4, n0 + g)};
+            uint32_t ah[4], al[4], bh[2], bl[2];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                ah[e] = tc::f32_to_tf32(av[e]);
+                al[e] = kSa ? tc::f32_to_tf32(av[e] - __uint_as_float(ah[e])) : 0u;
+            }
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                bh[e] = tc::f32_to_tf32(bv[e]);
+                bl[e] = kSb ? tc::f32_to_tf32(bv[e] - __uint_as_float(bh[e])) : 0u;
+            }
+            if constexpr (kSb) tc::mma_sync_tf32(acc, ah[0], ah[1], ah[2], ah[3], bl[0], bl[1]);
+            if constexpr (kSa) tc::mma_sync_tf32(acc, al[0], al[1], al[2], al[3], bh[0], bh[1]);
+            tc::mma_sync_tf32(acc, ah[0], ah[1], ah[2], ah[3], bh[0], bh[1]);
+        }
+        epi(m0 + g, n0 + 2 * t, acc[0]);
+        epi(m0 + g, n0 + 2 * t + 1, acc[1]);
+        epi(m0 + g + 8, n0 + 2 * t, acc[2]);
+        epi(m0 + g + 8, n0 + 2 * t + 1, acc[3]);
     }
 }
 
@@ -242,6 +286,43 @@ __device__ __forceinline__ void load_rows(float* dst, int ld, const Tin* __restr
     }
 }
 
+// The same fill split in two, so several tensors' loads are in flight together:
+// rows_issue loads this thread's 16-byte pieces (zero past Lc) into registers,
+// rows_store writes them as fp32 rows (stride ld), rows_tile (bf16, D = 128) as a
+// bf16 MMA tile at a shared-memory address.
+template <int D, typename Tin>
+struct RowLoad {
+    static constexpr int VE = 16 / (int)sizeof(Tin), VPR = D / VE, NV = kL * VPR;
+    static constexpr int PER = (NV + kThreads - 1) / kThreads;
+    uint4 w[PER];
+};
+template <int D, typename Tin>
+__device__ __forceinline__ void rows_issue(RowLoad<D, Tin>& L, const Tin* __restrict__ src, size_t row0, int H,
+                                           int Lc) {
+    using R = RowLoad<D, Tin>;
+#pragma unroll
+    for (int it = 0; it < R::PER; ++it) {
+        const int e = threadIdx.x + it * kThreads, r = e / R::VPR;
+        L.w[it] = make_uint4(0u, 0u, 0u, 0u);
+        if ((R::NV % kThreads == 0 || e < R::NV) && r < Lc)
+            L.w[it] = *reinterpret_cast<const uint4*>(src + (row0 + (size_t)r * H) * D + (e % R::VPR) * R::VE);
+    }
+}
+template <int D, typename Tin>
+__device__ __forceinline__ void rows_store(const RowLoad<D, Tin>& L, float* dst, int ld) {
+    using R = RowLoad<D, Tin>;
+#pragma unroll
+    for (int it = 0; it < R::PER; ++it) {
+        const int e = threadIdx.x + it * kThreads;
+        if (R::NV % kThreads == 0 || e < R::NV) {
+            float f[R::VE];
+            unpack16(L.w[it], f);
+            float* o = dst + (e / R::VPR) * ld + (e % R::VPR) * R::VE;
+#pragma unroll
+            for (int x = 0; x < R::VE; ++x) o[x] = f[x];
+        }
+    }
+}
 // an R x C fp32 tile (global rows ldg floats apart, 16-byte aligned) into shared
 // memory (stride lds); src == nullptr fills zeros
 template <int R, int C>
@@ -305,6 +386,14 @@ __device__ __forceinline__ void from_f32(uint8_t* dst, const float* t, int ld) {
 }
 }  // namespace tile
 
+// The chunk states the tensor-core state passes store (S_c and dS'_c, bf16 128 x 128)
+// are laid out by 16-byte pieces: piece c (elements 8c .. 8c+7) of row i at byte
+// (128 c + i) 16, so that 32 threads holding 32 consecutive rows move 512 contiguous
+// bytes per access.
+namespace stl {
+__host__ __device__ constexpr uint32_t off(int i, int c) { return ((uint32_t)c * 128u + (uint32_t)i) * 16u; }
+}
+
 // Byte offset, inside a chunk's C slot of the workspace, of the decays the tensor-core
 // state passes read (e^{g_L - g_r} for the 32 positions, then e^{g_L}); before it: the
 // G hi, G lo and dO tiles.
@@ -317,7 +406,7 @@ constexpr uint32_t kPrepDec = 3 * tile::kBytes;
 // dO tile and the decays (in C's slot).
 template <typename Tin, int DK, int DV>
 struct PrepSmem {
-    static constexpr int LDK = DK + 1, LDV = DV + 1;
+    static constexpr int LDK = DK + 4, LDV = DV + 4;   // 4 mod 32 (wgemm)
     static constexpr size_t K = 0, Q = K + kL * LDK, V = Q + kL * LDK, O = V + kL * LDV, A = O + kL * LDV,
                             P = A + kL * kLDL, G = P + kL * kLDL, GP = G + kL, BT = GP + kL, CW = BT + kL,
                             total = CW + kL;
@@ -338,11 +427,19 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     const int t0 = c * kL, Lc = min(kL, T - t0);
     const size_t row0 = ((size_t)b * T + t0) * H + h;
     const float dh = d[h];
-    load_rows<DK>(Ks, LDK, k, row0, H, Lc);
-    load_rows<DK>(Qs, LDK, q, row0, H, Lc);
-    load_rows<DV>(Vs, LDV, v, row0, H, Lc);
-    load_rows<DV>(Os, LDV, dout, row0, H, Lc);
-    chunk_decays(log_alpha, beta, row0, H, Lc, g, gp, bt);
+    {
+        RowLoad<DK, Tin> lk, lq;
+        RowLoad<DV, Tin> lv, lo;
+        rows_issue(lk, k, row0, H, Lc);
+        rows_issue(lq, q, row0, H, Lc);
+        rows_issue(lv, v, row0, H, Lc);
+        rows_issue(lo, dout, row0, H, Lc);
+        chunk_decays(log_alpha, beta, row0, H, Lc, g, gp, bt);
+        rows_store(lk, Ks, LDK);
+        rows_store(lq, Qs, LDK);
+        rows_store(lv, Vs, LDV);
+        rows_store(lo, Os, LDV);
+    }
     __syncthreads();
     constexpr bool kTC = grads_tc<Tin, DK, DV>();
     const size_t ci = (size_t)bh * nch + c;
@@ -363,15 +460,16 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     }
     if (threadIdx.x < kL) cw[threadIdx.x] = bt[threadIdx.x] * expf(gp[threadIdx.x]);
     // A = diag(beta) AF (strictly lower) and P, both from the raw k rows
-    bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Ks[m * LDK + x]; },
-                            [&](int x, int n) { return Ks[n * LDK + x]; },
-                            [&](int m, int n, float s) {
-                                Am[m * kLDL + n] = (n < m) ? bt[m] * expf(gp[m] - g[n]) * s : 0.f;
-                            });
+    constexpr bool kIn = !std::is_same<Tin, __nv_bfloat16>::value;   // inputs not exact in tf32
+    wgemm<kL, kL, DK, kIn, kIn>([&](int m, int x) { return Ks[m * LDK + x]; },
+                                [&](int x, int n) { return Ks[n * LDK + x]; },
+                                [&](int m, int n, float s) {
+                                    Am[m * kLDL + n] = (n < m) ? bt[m] * expf(gp[m] - g[n]) * s : 0.f;
+                                });
     __syncthreads();   // q~ complete
-    bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Qs[m * LDK + x]; },
-                            [&](int x, int n) { return Ks[n * LDK + x]; },
-                            [&](int m, int n, float s) { Pm[m * kLDL + n] = (n <= m) ? expf(g[m] - g[n]) * s : 0.f; });
+    wgemm<kL, kL, DK, true, kIn>([&](int m, int x) { return Qs[m * LDK + x]; },
+                                 [&](int x, int n) { return Ks[n * LDK + x]; },
+                                 [&](int m, int n, float s) { Pm[m * kLDL + n] = (n <= m) ? expf(g[m] - g[n]) * s : 0.f; });
     __syncthreads();
     // [W | U~] = (I + A)^{-1} [diag(beta e^{g'}) K | diag(beta) V]: one column per
     // thread, forward substitution down the column, in place over K and V
@@ -391,9 +489,9 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     }
     __syncthreads();
     // Gamma Q~ - P W, in place over Q~
-    bgemm<kL, DK, kL, 2, 4>([&](int m, int x) { return Pm[m * kLDL + x]; },
-                            [&](int x, int n) { return Ks[x * LDK + n]; },
-                            [&](int m, int n, float s) { Qs[m * LDK + n] = fmaf(expf(g[m]), Qs[m * LDK + n], -s); });
+    wgemm<kL, DK, kL, true, true>([&](int m, int x) { return Pm[m * kLDL + x]; },
+                                  [&](int x, int n) { return Ks[x * LDK + n]; },
+                                  [&](int m, int n, float s) { Qs[m * LDK + n] = fmaf(expf(g[m]), Qs[m * LDK + n], -s); });
     __syncthreads();
     float* Ug = ws.U + ci * kL * DV;
     for (int e = threadIdx.x; e < kL * DV; e += kThreads) Ug[e] = Vs[(e / DV) * LDV + e % DV];
@@ -403,9 +501,9 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
         tile::from_f32<true>(cs + tile::kBytes, Qs, LDK);
     } else {
         float* Cg = ws.C + ci * DV * DK;
-        bgemm<DV, DK, kL, 8, 8>([&](int i, int r) { return Os[r * LDV + i]; },
-                                [&](int r, int j) { return Qs[r * LDK + j]; },
-                                [&](int i, int j, float s) { Cg[(size_t)i * DK + j] = s; });
+        wgemm<DV, DK, kL, kIn, true>([&](int i, int r) { return Os[r * LDV + i]; },
+                                     [&](int r, int j) { return Qs[r * LDK + j]; },
+                                     [&](int i, int j, float s) { Cg[(size_t)i * DK + j] = s; });
         float* Wg = ws.W + ci * kL * DK;
         for (int e = threadIdx.x; e < kL * DK; e += kThreads) Wg[e] = Ks[(e / DK) * LDK + e % DK];
     }
@@ -519,7 +617,7 @@ bwd_dstates_kernel(const Tin* __restrict__ k, const float* __restrict__ log_alph
 // bwd_grads: every input gradient of one chunk, from S_c and dS'_c.
 template <int DK, int DV>
 struct GradSmem {
-    static constexpr int DM = (DK > DV ? DK : DV), LD = DM + 1;
+    static constexpr int DM = (DK > DV ? DK : DV), LD = DM + 4;   // 4 mod 32 (wgemm)
     static constexpr int NV = 24;   // per-row vectors
     // [L, LD] tiles: K, Q~, dO, V, KS^T (then F), X, dX (then dR), Gamma dO S (then dq~), dk
     static constexpr size_t K = 0, Q = K + kL * LD, O = Q + kL * LD, V = O + kL * LD, R = V + kL * LD,
@@ -568,20 +666,12 @@ __device__ __forceinline__ void wait(uint64_t* bar) {
 // 16-byte piece c (0..15) of row r of a K-major 32 x 128 bf16 tile: 64-column atoms
 // 4096 bytes apart, 128B-swizzled rows
 __device__ __forceinline__ uint32_t boff(int r, int c) { return tile::off(r, c); }
-// rows [32, 128] of a [B, T, H, 128] bf16 tensor into a tile (zero past Lc)
-__device__ __forceinline__ void rows_to_tile(uint32_t dst, const __nv_bfloat16* __restrict__ src, size_t row0,
-                                             int H, int Lc) {
-    uint4 w[2];
+// bf16 rows already in registers (rows_issue, zero past Lc) as a tile at shared address dst
+__device__ __forceinline__ void rows_tile(const RowLoad<128, __nv_bfloat16>& L, uint32_t dst) {
 #pragma unroll
-    for (int it = 0; it < 2; ++it) {
-        const int e = threadIdx.x + it * kThreads, r = e >> 4, c = e & 15;
-        w[it] = (r < Lc) ? *reinterpret_cast<const uint4*>(src + (row0 + (size_t)r * H) * 128 + 8 * c)
-                         : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int it = 0; it < 2; ++it) {
+    for (int it = 0; it < RowLoad<128, __nv_bfloat16>::PER; ++it) {
         const int e = threadIdx.x + it * kThreads;
-        tc::sts_u32x4(dst + boff(e >> 4, e & 15), w[it]);
+        tc::sts_u32x4(dst + boff(e >> 4, e & 15), L.w[it]);
     }
 }
 // a 32 x 128 fp32 shared-memory tile (row stride ld) into a bf16 tile
@@ -598,34 +688,66 @@ __device__ __forceinline__ void f32_to_tile(uint32_t dst, const float* t, int ld
         tc::sts_u32x4(dst + boff(r, c), w);
     }
 }
-// a 128 x 128 bf16 state (row-major, global: the state passes' output) into TMEM as
-// A operands: its rows (lane i, columns [rows, +64): pairs (j, j+1)) and its columns
-// (lane j, columns [cols, +64): pairs (i, i+1)); called by one warp per TMEM lane quarter
-__device__ __forceinline__ void state_to_tmem(uint32_t tl, int lane_row, const __nv_bfloat16* __restrict__ Sg,
-                                              uint32_t rows, uint32_t cols) {
+// The chunk's S and dS' (bf16, the state passes' piece layout) into TMEM as A operands:
+// their rows (lane i, pairs (j, j+1): columns [C_S, +64) and [C_DS, +64)) and their
+// columns (lane j, pairs (i, i+1): [C_ST, +64) and [C_DST, +64)).  Warps 0-3 (thread =
+// row i) load both rows (coalesced), store them to TMEM and to two row-major scratch
+// tiles in shared memory (16-byte pieces XOR-swizzled by row: conflict-free both ways)
+// and return the row's part of <dS', S>.  After the barrier every thread takes a column
+// (lane j): warps 0-3 of dS', warps 4-7 of S, from the scratch.
+__device__ __forceinline__ uint32_t scr_off(int r, int c) {   // piece c of row r of a scratch tile
+    return (uint32_t)r * 256u + ((uint32_t)(c ^ (r & 7)) << 4);
+}
+__device__ __forceinline__ float states_to_tmem(uint32_t tl, int x, const uint8_t* __restrict__ Sg,
+                                                const uint8_t* __restrict__ dSg, uint8_t* scrS, uint8_t* scrD) {
+    const int warp = threadIdx.x >> 5;
+    float ss = 0.f;
+    if (warp < 4) {
 #pragma unroll 1
-    for (int hh = 0; hh < 2; ++hh) {   // row lane_row, state columns 64 hh .. + 63: already pairs
-        float pk[32];
+        for (int hh = 0; hh < 2; ++hh) {
+            uint4 a[8], b[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const uint4 x = *reinterpret_cast<const uint4*>(Sg + (size_t)lane_row * 128 + 64 * hh + 8 * e);
-            pk[4 * e] = __uint_as_float(x.x); pk[4 * e + 1] = __uint_as_float(x.y);
-            pk[4 * e + 2] = __uint_as_float(x.z); pk[4 * e + 3] = __uint_as_float(x.w);
+            for (int e = 0; e < 8; ++e) {
+                a[e] = *reinterpret_cast<const uint4*>(Sg + stl::off(x, 8 * hh + e));
+                b[e] = *reinterpret_cast<const uint4*>(dSg + stl::off(x, 8 * hh + e));
+            }
+            float pa[32], pb[32];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                float fa[8], fb[8];
+                unpack16(a[e], fa);
+                unpack16(b[e], fb);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) ss = fmaf(fa[q], fb[q], ss);
+                pa[4 * e] = __uint_as_float(a[e].x); pa[4 * e + 1] = __uint_as_float(a[e].y);
+                pa[4 * e + 2] = __uint_as_float(a[e].z); pa[4 * e + 3] = __uint_as_float(a[e].w);
+                pb[4 * e] = __uint_as_float(b[e].x); pb[4 * e + 1] = __uint_as_float(b[e].y);
+                pb[4 * e + 2] = __uint_as_float(b[e].z); pb[4 * e + 3] = __uint_as_float(b[e].w);
+                *reinterpret_cast<uint4*>(scrS + scr_off(x, 8 * hh + e)) = a[e];
+                *reinterpret_cast<uint4*>(scrD + scr_off(x, 8 * hh + e)) = b[e];
+            }
+            tc::tmem_st32(tl + C_S + 32 * hh, pa);
+            tc::tmem_st32(tl + C_DS + 32 * hh, pb);
         }
-        tc::tmem_st32(tl + rows + 32 * hh, pk);
     }
-    const unsigned short* Su = reinterpret_cast<const unsigned short*>(Sg);
+    __syncthreads();
+    const uint8_t* scr = (warp < 4) ? scrD : scrS;
+    const uint32_t col = (warp < 4) ? C_DST : C_ST;
+    const uint32_t sel = (x & 1) ? 0x7632u : 0x5410u;   // this column's half of each word
+    const uint32_t wo = (uint32_t)((x & 7) >> 1) * 4u;
 #pragma unroll 1
-    for (int hh = 0; hh < 2; ++hh) {   // column lane_row, state rows 64 hh .. + 63
+    for (int hh = 0; hh < 2; ++hh) {
         float pk[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-            const uint32_t lo = Su[(size_t)(64 * hh + 2 * c) * 128 + lane_row];
-            const uint32_t hi = Su[(size_t)(64 * hh + 2 * c + 1) * 128 + lane_row];
-            pk[c] = __uint_as_float(lo | (hi << 16));
+            const int r = 64 * hh + 2 * c;
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(scr + scr_off(r, x >> 3) + wo);
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(scr + scr_off(r + 1, x >> 3) + wo);
+            pk[c] = __uint_as_float(__byte_perm(w0, w1, sel));
         }
-        tc::tmem_st32(tl + cols + 32 * hh, pk);
+        tc::tmem_st32(tl + col + 32 * hh, pk);
     }
+    return ss;
 }
 // 32 result columns of this thread's TMEM lane (state index x) into the fp32 tile
 // column x: t[r][x] = f(r, value)
@@ -642,7 +764,9 @@ __device__ __forceinline__ void result_to_tile(uint32_t taddr, int x, float* t, 
 
 template <typename Tin, int DK, int DV>
 __host__ __device__ constexpr size_t grads_smem_bytes() {
-    return GradSmem<DK, DV>::total * sizeof(float) + (grads_tc<Tin, DK, DV>() ? 1024 + gtc::kBytes : 0);
+    // the tensor-core form has no global operand to stage: its region replaces STG
+    return grads_tc<Tin, DK, DV>() ? GradSmem<DK, DV>::STG * sizeof(float) + 1024 + gtc::kBytes
+                                   : GradSmem<DK, DV>::total * sizeof(float);
 }
 
 template <typename Tin, int DK, int DV>
@@ -671,14 +795,15 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     const float* S = ws.S + ci * DV * DK;      // chunk-start state
     const float* dSp = ws.dS + ci * DV * DK;   // gradient at the chunk's end state
     constexpr bool kTC = grads_tc<Tin, DK, DV>();
-    // tensor-core form: B tiles, barriers and the TMEM address slot after the fp32
-    // layout (1024-byte aligned); TMEM for the A operands and results
+    constexpr bool kIn = !std::is_same<Tin, __nv_bfloat16>::value;   // inputs not exact in tf32 (wgemm)
+    // tensor-core form: B tiles, barriers and the TMEM address slot in place of the
+    // staging slab (1024-byte aligned); TMEM for the A operands and results
     uint32_t tcb = 0, tmem = 0, ttl = 0;
     uint64_t* tbar = nullptr;
     const int xrow = (warp & 3) * 32 + lane;   // this thread's TMEM lane
     if constexpr (kTC) {
         const uint32_t s0 = tc::smem_u32(sm);
-        tcb = (tc::smem_u32(sm + SM::total) + 1023u) & ~1023u;
+        tcb = (tc::smem_u32(sm + SM::STG) + 1023u) & ~1023u;
         tbar = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sm) + (tcb - s0) + gtc::BARS);
         if (tid == 0) {
             for (int i = 0; i < 4; ++i) tc::mbar_init(&tbar[i], 1);
@@ -689,16 +814,25 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
                            gtc::kCols);
     }
 
-    // 1. tiles and decays
-    load_rows<DK>(Ks, LD, k, row0, H, Lc);
-    load_rows<DK>(Qs, LD, q, row0, H, Lc);
-    load_rows<DV>(Os, LD, dout, row0, H, Lc);
-    load_rows<DV>(Vs, LD, v, row0, H, Lc);
-    chunk_decays(log_alpha, beta, row0, H, Lc, g, gp, bt);
-    if constexpr (kTC) {
-        gtc::rows_to_tile(tcb + gtc::KB, k, row0, H, Lc);
-        gtc::rows_to_tile(tcb + gtc::OB, dout, row0, H, Lc);
-        tc::tc_fence_before();
+    // 1. tiles and decays (all four tensors' loads in flight together)
+    float ss = 0.f;   // this thread's part of <dS', S>
+    {
+        RowLoad<DK, Tin> lk, lq;
+        RowLoad<DV, Tin> lo, lv;
+        rows_issue(lk, k, row0, H, Lc);
+        rows_issue(lq, q, row0, H, Lc);
+        rows_issue(lo, dout, row0, H, Lc);
+        rows_issue(lv, v, row0, H, Lc);
+        chunk_decays(log_alpha, beta, row0, H, Lc, g, gp, bt);
+        rows_store(lk, Ks, LD);
+        rows_store(lq, Qs, LD);
+        rows_store(lo, Os, LD);
+        rows_store(lv, Vs, LD);
+        if constexpr (kTC) {
+            gtc::rows_tile(lk, tcb + gtc::KB);
+            gtc::rows_tile(lo, tcb + gtc::OB);
+            tc::tc_fence_before();
+        }
     }
     __syncthreads();
     if constexpr (kTC) {
@@ -706,8 +840,9 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         tmem = *reinterpret_cast<volatile uint32_t*>(reinterpret_cast<uint8_t*>(sm) + (tcb - tc::smem_u32(sm)) +
                                                      gtc::SLOT);
         ttl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        if (warp < 4) gtc::state_to_tmem(ttl, xrow, reinterpret_cast<const __nv_bfloat16*>(S), gtc::C_S, gtc::C_ST);
-        else gtc::state_to_tmem(ttl, xrow, reinterpret_cast<const __nv_bfloat16*>(dSp), gtc::C_DS, gtc::C_DST);
+        // scratch for the transposition: the R | X and G | TK tiles, not yet in use
+        ss = gtc::states_to_tmem(ttl, xrow, reinterpret_cast<const uint8_t*>(S), reinterpret_cast<const uint8_t*>(dSp),
+                                 reinterpret_cast<uint8_t*>(Rs), reinterpret_cast<uint8_t*>(Gs));
         tc::tmem_st_wait();
         tc::fence_proxy_async_smem();   // the B tiles, written by threads, for the tensor pipe
         tc::tc_fence_before();
@@ -731,10 +866,10 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
             tc::mma_bf16_ta_bk(tmem + gtc::C_C, tmem + gtc::C_ST, tcb + gtc::OB, 4096, gtc::ID, 8, 0);
             tc::mma_commit(&tbar[gtc::B_ABC]);
         }
-        bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Ks[m * LD + x]; },
+        wgemm<kL, kL, DK, kIn, kIn>([&](int m, int x) { return Ks[m * LD + x]; },
                                 [&](int x, int n) { return Ks[n * LD + x]; },
                                 [&](int m, int n, float s) { AF[m * kLDL + n] = (n < m) ? expf(gp[m] - g[n]) * s : 0.f; });
-        bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Qs[m * LD + x]; },
+        wgemm<kL, kL, DK, true, kIn>([&](int m, int x) { return Qs[m * LD + x]; },
                                 [&](int x, int n) { return Ks[n * LD + x]; },
                                 [&](int m, int n, float s) { Pm[m * kLDL + n] = (n <= m) ? expf(g[m] - g[n]) * s : 0.f; });
         gtc::wait(&tbar[gtc::B_ABC]);
@@ -748,13 +883,13 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     } else {
         bgemm_staged<kL, DV, DK, 4, 4, true>([&](int r, int j) { return Ks[r * LD + j]; }, S, stage,
                                              [&](int r, int i, float x) { Rs[r * LD + i] = x; });
-        bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Ks[m * LD + x]; },
+        wgemm<kL, kL, DK, kIn, kIn>([&](int m, int x) { return Ks[m * LD + x]; },
                                 [&](int x, int n) { return Ks[n * LD + x]; },
                                 [&](int m, int n, float s) { AF[m * kLDL + n] = (n < m) ? expf(gp[m] - g[n]) * s : 0.f; });
         __syncthreads();   // q~, decays
         bgemm_staged<kL, DV, DK, 4, 4, true>([&](int r, int j) { return Ks[r * LD + j]; }, dSp, stage,
                                              [&](int r, int i, float x) { Ds[r * LD + i] = dec[r] * x; });
-        bgemm<kL, kL, DK, 4, 1>([&](int m, int x) { return Qs[m * LD + x]; },
+        wgemm<kL, kL, DK, true, kIn>([&](int m, int x) { return Qs[m * LD + x]; },
                                 [&](int x, int n) { return Ks[n * LD + x]; },
                                 [&](int m, int n, float s) { Pm[m * kLDL + n] = (n <= m) ? expf(g[m] - g[n]) * s : 0.f; });
         __syncthreads();
@@ -773,7 +908,7 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
 #pragma unroll
         for (int r = 0; r < kL; ++r) Xs[r * LD + col] = x[r];
     }
-    bgemm<kL, DV, kL, 2, 4>([&](int r, int s) { return Pm[s * kLDL + r]; },
+    wgemm<kL, DV, kL, true, kIn>([&](int r, int s) { return Pm[s * kLDL + r]; },
                             [&](int s, int i) { return Os[s * LD + i]; },
                             [&](int r, int i, float s) { Ds[r * LD + i] += s; });
     __syncthreads();
@@ -805,10 +940,10 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         gtc::f32_to_tile(tcb + gtc::DRB, Ds, LD);
         tc::fence_proxy_async_smem();
     }
-    bgemm<kL, kL, DV, 4, 1>([&](int r, int i) { return Ds[r * LD + i]; },
+    wgemm<kL, kL, DV, true, true>([&](int r, int i) { return Ds[r * LD + i]; },
                             [&](int i, int s) { return Xs[s * LD + i]; },
                             [&](int r, int s, float x) { dAm[r * kLDL + s] = (s < r) ? -x : 0.f; });
-    bgemm<kL, kL, DV, 4, 1>([&](int r, int i) { return Os[r * LD + i]; },
+    wgemm<kL, kL, DV, kIn, true>([&](int r, int i) { return Os[r * LD + i]; },
                             [&](int i, int s) { return Xs[s * LD + i]; },
                             [&](int r, int s, float x) { dPm[r * kLDL + s] = (s <= r) ? x : 0.f; });
     for (int r = warp; r < kL; r += kThreads / 32) {
@@ -890,14 +1025,14 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     __syncthreads();
     // 8. dq~ = Gamma dO S + dZ K;  dk (without F and -d dq~) =
     //    dZ^T Q~ + (dY + dY^T) K - diag(beta e^{g'}) dR S
-    bgemm<kL, DK, kL, 2, 4>([&](int r, int s) { return dPm[r * kLDL + s]; },
+    wgemm<kL, DK, kL, true, kIn>([&](int r, int s) { return dPm[r * kLDL + s]; },
                             [&](int s, int j) { return Ks[s * LD + j]; },
                             [&](int r, int j, float x) { Gs[r * LD + j] += x; });
     // (the three dk terms share one tiling, so each element stays with one thread)
-    bgemm<kL, DK, kL, 4, 4>([&](int r, int s) { return dPm[s * kLDL + r]; },
+    wgemm<kL, DK, kL, true, true>([&](int r, int s) { return dPm[s * kLDL + r]; },
                             [&](int s, int j) { return Qs[s * LD + j]; },
                             [&](int r, int j, float x) { TKs[r * LD + j] = x; });
-    bgemm<kL, DK, kL, 4, 4>([&](int r, int s) { return dAm[r * kLDL + s] + dAm[s * kLDL + r]; },
+    wgemm<kL, DK, kL, true, kIn>([&](int r, int s) { return dAm[r * kLDL + s] + dAm[s * kLDL + r]; },
                             [&](int s, int j) { return Ks[s * LD + j]; },
                             [&](int r, int j, float x) { TKs[r * LD + j] += x; });
     if constexpr (!kTC)
@@ -906,34 +1041,45 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
             [&](int r, int j, float x) { TKs[r * LD + j] = fmaf(-bt[r] * egp[r], x, TKs[r * LD + j]); });
     __syncthreads();
     // 9. outputs: dq, dk, dv; decay gradients; dd partial
-    for (int e = tid; e < Lc * DK; e += kThreads) {
-        const int r = e / DK, j = e % DK;
-        const size_t o = (row0 + (size_t)r * H) * DK + j;
-        const float dqt = Gs[r * LD + j];
-        dq[o] = dqt;
-        float tk = TKs[r * LD + j];
-        if constexpr (kTC) tk = fmaf(-bt[r] * egp[r], Vs[r * LD + j], tk);
-        dk[o] = fmaf(-dh, dqt, tk + Rs[r * LD + j]);
-    }
-    for (int e = tid; e < Lc * DV; e += kThreads) {
-        const int r = e / DV, i = e % DV;
-        dv[(row0 + (size_t)r * H) * DV + i] = bt[r] * Ds[r * LD + i];
-    }
-    // <dS', S> and sum_r dq~_r . k_r (block sums in a fixed order)
-    float ss = 0.f;
-    if constexpr (kTC) {   // bf16 states
-        constexpr int PER = DV * DK / 8 / kThreads;   // 16-byte pieces of each matrix per thread
-        const uint4* x8 = reinterpret_cast<const uint4*>(dSp);
-        const uint4* y8 = reinterpret_cast<const uint4*>(S);
-#pragma unroll 4
-        for (int it = 0; it < PER; ++it) {
-            float fx[8], fy[8];
-            unpack16(x8[tid + it * kThreads], fx);
-            unpack16(y8[tid + it * kThreads], fy);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) ss = fmaf(fx[e], fy[e], ss);
+    // (16-byte stores when the three gradients allow them; the row stride LD keeps the
+    // shared-memory rows 16-byte aligned)
+    auto dk_of = [&](int r, float dqt, float tk, float rr, float vv) {
+        if constexpr (kTC) tk = fmaf(-bt[r] * egp[r], vv, tk);
+        return fmaf(-dh, dqt, tk + rr);
+    };
+    if (((reinterpret_cast<uintptr_t>(dq) | reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 15) == 0) {
+        for (int e = tid; e < Lc * (DK / 4); e += kThreads) {
+            const int r = e / (DK / 4), j = 4 * (e % (DK / 4));
+            const size_t o = (row0 + (size_t)r * H) * DK + j;
+            const float4 gq = *reinterpret_cast<const float4*>(Gs + r * LD + j);
+            const float4 tk = *reinterpret_cast<const float4*>(TKs + r * LD + j);
+            const float4 rr = *reinterpret_cast<const float4*>(Rs + r * LD + j);
+            const float4 vv = kTC ? *reinterpret_cast<const float4*>(Vs + r * LD + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4*>(dq + o) = gq;
+            *reinterpret_cast<float4*>(dk + o) = make_float4(dk_of(r, gq.x, tk.x, rr.x, vv.x), dk_of(r, gq.y, tk.y, rr.y, vv.y),
+                                                             dk_of(r, gq.z, tk.z, rr.z, vv.z), dk_of(r, gq.w, tk.w, rr.w, vv.w));
+        }
+        for (int e = tid; e < Lc * (DV / 4); e += kThreads) {
+            const int r = e / (DV / 4), i = 4 * (e % (DV / 4));
+            const float4 x = *reinterpret_cast<const float4*>(Ds + r * LD + i);
+            *reinterpret_cast<float4*>(dv + (row0 + (size_t)r * H) * DV + i) =
+                make_float4(bt[r] * x.x, bt[r] * x.y, bt[r] * x.z, bt[r] * x.w);
         }
     } else {
+        for (int e = tid; e < Lc * DK; e += kThreads) {
+            const int r = e / DK, j = e % DK;
+            const size_t o = (row0 + (size_t)r * H) * DK + j;
+            const float dqt = Gs[r * LD + j];
+            dq[o] = dqt;
+            dk[o] = dk_of(r, dqt, TKs[r * LD + j], Rs[r * LD + j], kTC ? Vs[r * LD + j] : 0.f);
+        }
+        for (int e = tid; e < Lc * DV; e += kThreads) {
+            const int r = e / DV, i = e % DV;
+            dv[(row0 + (size_t)r * H) * DV + i] = bt[r] * Ds[r * LD + i];
+        }
+    }
+    // <dS', S> and sum_r dq~_r . k_r (block sums in a fixed order)
+    if constexpr (!kTC) {   // (the tensor-core form took it while staging the states)
         constexpr int PER = DV * DK / 4 / kThreads;   // float4s of each matrix per thread
 #pragma unroll 4
         for (int it = 0; it < PER; ++it) {

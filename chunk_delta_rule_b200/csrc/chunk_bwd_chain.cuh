@@ -47,47 +47,62 @@ constexpr uint32_t ST_W = 0, ST_K = 8192, ST_U = 16384, ST_G = 16384, ST_GLO = 2
                    ST_DEC = 40960, ST_BYTES = 41984;
 constexpr uint32_t SM_BARS = 2 * ST_BYTES;     // 8 mbarriers, the TMEM slot, the abort flag
 constexpr uint32_t kSmemBytes = SM_BARS + 128 + 1024;   // + alignment slack
-enum { B_FULL0 = 0, B_FULL1 = 1, B_SREADY = 2, B_SPLIT = 3, B_MMA1 = 4, B_MMA2 = 5, B_DRAIN = 6 };
+enum { B_FULL0 = 0, B_FULL1 = 1, B_SREADY = 2, B_SPLIT = 3, B_MMA1 = 4, B_MMA2 = 5, B_DRAIN = 6, B_MREADY = 7 };
 
 constexpr uint32_t ID_N32 = tc::idesc_bf16(128, 32, false, false);    // S W^T, dS' K^T
 constexpr uint32_t ID_N128B = tc::idesc_bf16(128, 128, false, true);  // Xd^T K, Zd W (B MN-major)
 constexpr uint32_t ID_N128AB = tc::idesc_bf16(128, 128, true, true);  // dO^T G
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
-// the state row this thread owns, read out of the master: stored as bf16 to `row_out`
-// (if set) and as fp32 to `row_f32` (if set); unless `last`, the bf16 copy is refreshed
-// and the master scaled by `eL` for the next chunk's update
-__device__ __forceinline__ void read_out(uint32_t tl, bool last, float eL, __nv_bfloat16* row_out,
-                                         float* row_f32) {
+// Reading out the state row this thread owns (lane = row i) after a chunk's update,
+// in two passes so the next chunk's first MMA waits only for the first:
+//  copy_out: the bf16 copy (the next first MMA's A operand), unless `last`; returns
+//            the row as 64 packed bf16 pairs in `pk`
+//  store_out: the row to the workspace (bf16, piece layout) and, unless `last`, the
+//            master pre-scaled by `eL` for the next update; or, with `f32`, the row as
+//            fp32 (dS0)
+__device__ __forceinline__ void copy_out(uint32_t tl, bool last, uint32_t (&pk)[64]) {
+#pragma unroll
+    for (int pair = 0; pair < 2; ++pair) {
+        float v0[32], v1[32];
+        tc::tmem_ld32(tl + TM_S + 64 * pair, v0);
+        tc::tmem_ld32(tl + TM_S + 64 * pair + 32, v1);
+        tc::tmem_ld_wait();
+        float p[32];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            pk[32 * pair + c] = tc::pack_bf16(v0[2 * c], v0[2 * c + 1]);
+            pk[32 * pair + 16 + c] = tc::pack_bf16(v1[2 * c], v1[2 * c + 1]);
+            p[c] = __uint_as_float(pk[32 * pair + c]);
+            p[16 + c] = __uint_as_float(pk[32 * pair + 16 + c]);
+        }
+        if (!last) tc::tmem_st32(tl + TM_SB + 32 * pair, p);
+    }
+}
+__device__ __forceinline__ void store_out(uint32_t tl, int row, bool last, float eL, const uint32_t (&pk)[64],
+                                          uint8_t* slot, float* f32) {
+    if (slot) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+            *reinterpret_cast<uint4*>(slot + stl::off(row, c)) =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+    }
+    if (last && !f32) return;
 #pragma unroll 1
     for (int pair = 0; pair < 2; ++pair) {
         float v0[32], v1[32];
         tc::tmem_ld32(tl + TM_S + 64 * pair, v0);
         tc::tmem_ld32(tl + TM_S + 64 * pair + 32, v1);
         tc::tmem_ld_wait();
-        float pk[32];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            pk[c] = __uint_as_float(tc::pack_bf16(v0[2 * c], v0[2 * c + 1]));
-            pk[16 + c] = __uint_as_float(tc::pack_bf16(v1[2 * c], v1[2 * c + 1]));
-        }
-        if (row_out) {
-            uint4* o = reinterpret_cast<uint4*>(row_out + 64 * pair);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                o[e] = make_uint4(__float_as_uint(pk[4 * e]), __float_as_uint(pk[4 * e + 1]),
-                                  __float_as_uint(pk[4 * e + 2]), __float_as_uint(pk[4 * e + 3]));
-        }
-        if (row_f32) {
+        if (f32) {
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
-                *reinterpret_cast<float4*>(row_f32 + 64 * pair + e) = make_float4(v0[e], v0[e + 1], v0[e + 2], v0[e + 3]);
-                *reinterpret_cast<float4*>(row_f32 + 64 * pair + 32 + e) =
+                *reinterpret_cast<float4*>(f32 + 64 * pair + e) = make_float4(v0[e], v0[e + 1], v0[e + 2], v0[e + 3]);
+                *reinterpret_cast<float4*>(f32 + 64 * pair + 32 + e) =
                     make_float4(v1[e], v1[e + 1], v1[e + 2], v1[e + 3]);
             }
         }
         if (!last) {
-            tc::tmem_st32(tl + TM_SB + 32 * pair, pk);
 #pragma unroll
             for (int e = 0; e < 32; ++e) { v0[e] *= eL; v1[e] *= eL; }
             tc::tmem_st32(tl + TM_S + 64 * pair, v0);
@@ -97,12 +112,12 @@ __device__ __forceinline__ void read_out(uint32_t tl, bool last, float eL, __nv_
 }
 
 // the initial row (fp32 global, or zero) into the master (scaled by eL) and the bf16
-// copy, and stored as bf16 to `row_out`
-__device__ __forceinline__ void load_in(uint32_t tl, const float* __restrict__ src, bool need, float eL,
-                                        __nv_bfloat16* row_out) {
+// copy (if `need`), and stored as bf16 to the workspace slot
+__device__ __forceinline__ void load_in(uint32_t tl, int row, const float* __restrict__ src, bool need, float eL,
+                                        uint8_t* slot) {
 #pragma unroll 1
     for (int pair = 0; pair < 2; ++pair) {
-        float v0[32], v1[32], pk[32];
+        float v0[32], v1[32], p[32];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
             const float4 a = src ? *reinterpret_cast<const float4*>(src + 64 * pair + e) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -113,16 +128,16 @@ __device__ __forceinline__ void load_in(uint32_t tl, const float* __restrict__ s
         }
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-            pk[c] = __uint_as_float(tc::pack_bf16(v0[2 * c], v0[2 * c + 1]));
-            pk[16 + c] = __uint_as_float(tc::pack_bf16(v1[2 * c], v1[2 * c + 1]));
+            p[c] = __uint_as_float(tc::pack_bf16(v0[2 * c], v0[2 * c + 1]));
+            p[16 + c] = __uint_as_float(tc::pack_bf16(v1[2 * c], v1[2 * c + 1]));
         }
-        uint4* o = reinterpret_cast<uint4*>(row_out + 64 * pair);
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-            o[e] = make_uint4(__float_as_uint(pk[4 * e]), __float_as_uint(pk[4 * e + 1]), __float_as_uint(pk[4 * e + 2]),
-                              __float_as_uint(pk[4 * e + 3]));
+        for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(slot + stl::off(row, 8 * pair + c)) =
+                make_uint4(__float_as_uint(p[4 * c]), __float_as_uint(p[4 * c + 1]), __float_as_uint(p[4 * c + 2]),
+                           __float_as_uint(p[4 * c + 3]));
         if (need) {
-            tc::tmem_st32(tl + TM_SB + 32 * pair, pk);
+            tc::tmem_st32(tl + TM_SB + 32 * pair, p);
 #pragma unroll
             for (int e = 0; e < 32; ++e) { v0[e] *= eL; v1[e] *= eL; }
             tc::tmem_st32(tl + TM_S + 64 * pair, v0);
@@ -147,12 +162,12 @@ bwd_chain_tc_kernel(Workspace ws, const float* __restrict__ S0, const float* __r
     // dS'_{nch-1} .. dS'_0 and dS0 (nch updates)
     const int nit = rev ? nch : (nch > 0 ? nch - 1 : 0);
     auto chunk_of = [&](int n) { return rev ? nch - 1 - n : n; };
-    auto state_slot = [&](int c) {   // bf16 [128][128] in chunk c's fp32 slot
-        return reinterpret_cast<__nv_bfloat16*>((rev ? ws.dS : ws.S) + ((size_t)bh * nch + c) * kDS);
+    auto state_slot = [&](int c) {   // bf16 128 x 128 (piece layout) in chunk c's fp32 slot
+        return reinterpret_cast<uint8_t*>((rev ? ws.dS : ws.S) + ((size_t)bh * nch + c) * kDS);
     };
 
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) tc::mbar_init(&bars[i], (i == B_SREADY || i == B_SPLIT) ? 128u : 1u);
+        for (int i = 0; i < 8; ++i) tc::mbar_init(&bars[i], (i == B_SREADY || i == B_SPLIT || i == B_MREADY) ? 128u : 1u);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -190,7 +205,7 @@ bwd_chain_tc_kernel(Workspace ws, const float* __restrict__ S0, const float* __r
             } else {
                 const bool need = nit > 0;
                 if (need) ok = wait(B_FULL0, 0);
-                load_in(tl, src, need && ok, need && ok ? eL_of(0) : 1.f, state_slot(chunk_of(0)) + (size_t)row * kD);
+                load_in(tl, row, src, need && ok, need && ok ? eL_of(0) : 1.f, state_slot(chunk_of(0)));
                 tc::tmem_st_wait();
                 tc::tc_fence_before();
                 if (need && ok) tc::mbar_arrive(&bars[B_SREADY]);
@@ -222,21 +237,29 @@ bwd_chain_tc_kernel(Workspace ws, const float* __restrict__ S0, const float* __r
             tc::tmem_st_wait();
             tc::tc_fence_before();
             tc::mbar_arrive(&bars[B_SPLIT]);
-            // ---- the updated state: stored, then bf16 copy and pre-scaled master for the next
+            // ---- the updated state: the bf16 copy first (it releases the next chunk's
+            // first MMA), then the store and the pre-scaled master (before the next SPLIT)
             const bool more = n + 1 < nit;
             if (more && !(ok = wait((n + 1) & 1 ? B_FULL1 : B_FULL0, ((n + 1) >> 1) & 1))) break;
             if (!(ok = wait(B_MMA2, n & 1))) break;
             tc::tc_fence_after();
             const int c = chunk_of(n);
-            __nv_bfloat16* dst = nullptr;
+            uint8_t* slot = nullptr;
             float* f32 = nullptr;
-            if (!rev) dst = state_slot(c + 1) + (size_t)row * kD;
-            else if (c > 0) dst = state_slot(c - 1) + (size_t)row * kD;
+            if (!rev) slot = state_slot(c + 1);
+            else if (c > 0) slot = state_slot(c - 1);
             else if (dS0) f32 = dS0 + ((size_t)bh * kD + row) * kD;
-            read_out(tl, !more, more ? eL_of(n + 1) : 1.f, dst, f32);
+            uint32_t pk[64];
+            copy_out(tl, !more, pk);
+            if (more) {
+                tc::tmem_st_wait();
+                tc::tc_fence_before();
+                tc::mbar_arrive(&bars[B_SREADY]);
+            }
+            store_out(tl, row, !more, more ? eL_of(n + 1) : 1.f, pk, slot, f32);
             tc::tmem_st_wait();
             tc::tc_fence_before();
-            if (more) tc::mbar_arrive(&bars[B_SREADY]);
+            if (rev && more) tc::mbar_arrive(&bars[B_MREADY]);   // the master is scaled: dO^T G may add
         }
     } else {
         // ========================== copies and MMA issue (warp 4) ===================
@@ -268,11 +291,17 @@ bwd_chain_tc_kernel(Workspace ws, const float* __restrict__ S0, const float* __r
             ok = __all_sync(0xffffffffu, wait((n & 1) ? B_FULL1 : B_FULL0, (n >> 1) & 1) && wait(B_SREADY, n & 1)) != 0;
             if (!ok) break;
             tc::tc_fence_after();
-            // first product of the chunk; the reverse pass's dO^T G runs while the state
-            // group splits Z
+            // first product of the chunk; the reverse pass's dO^T G follows once the state
+            // group has pre-scaled the master (the chunk before's readout), and runs while
+            // the state group splits Z
             tc::mma_bf16_ta_bk(tmem + TM_X, tmem + TM_SB, st + (rev ? ST_K : ST_W), 4096, ID_N32, 8, 0);
             tc::mma_commit(&bars[B_MMA1]);
             if (rev) {
+                if (n > 0) {
+                    ok = __all_sync(0xffffffffu, wait(B_MREADY, (n - 1) & 1)) != 0;
+                    if (!ok) break;
+                    tc::tc_fence_after();
+                }
                 tc::mma_amn_bmn(tmem + TM_S, st + ST_DO, 4096, st + ST_G, 4096, ID_N128AB, 2, 1);
                 tc::mma_amn_bmn(tmem + TM_S, st + ST_DO, 4096, st + ST_GLO, 4096, ID_N128AB, 2, 1);
             }
