@@ -110,43 +110,70 @@ __device__ __forceinline__ void bgemm(const FA& a, const FB& b, const Epi& epi) 
 // handed to epi(m, n, c).  kSa / kSb: that operand holds values with more than tf32
 // precision (fp32 results), so it is split into tf32 hi + lo and the product formed
 // as hi.lo + lo.hi + hi.hi, about fp32 accuracy; an operand exact in tf32 (bf16
-// inputs widened to fp32) skips the split.  Warp w takes the 16 x 8 output tiles w,
-// w + 8, ...; an element's owner depends only on <M, N>, so calls with the same M
-// and N may accumulate into one buffer without a barrier between them.  Fragment
-// loads hit distinct banks when the operands' row strides are 4 mod 32 (row g,
-// column t of a fragment: bank 4 g + t), in either orientation.
+// inputs widened to fp32) skips the split.  Each warp takes 16 x 8 NB strips (NB
+// output tiles side by side, sharing the A fragment of every k step); strip w, w + 8,
+// ... goes to warp w.  An element's owner depends only on <M, N>, so calls with the
+// same M and N may accumulate into one buffer without a barrier between them.
+// Fragment loads hit distinct banks when the operands' row strides are 4 mod 32 (row
+// g, column t of a fragment: bank 4 g + t), in either orientation.
+template <int M, int N>
+__host__ __device__ constexpr int wgemm_nb() {
+    return ((M / 16) * (N / 8) >= 4 * (kThreads / 32) && (N / 8) % 4 == 0) ? 4
+         : ((M / 16) * (N / 8) >= 2 * (kThreads / 32) && (N / 8) % 2 == 0) ? 2 : 1;
+}
+__device__ __forceinline__ void tf32_split(float x, bool split, uint32_t& hi, uint32_t& lo) {
+    hi = tc::f32_to_tf32(x);
+    lo = split ? tc::f32_to_tf32(x - __uint_as_float(hi)) : 0u;
+}
 template <int M, int N, int K, bool kSa, bool kSb, typename FA, typename FB, typename Epi>
 __device__ __forceinline__ void wgemm(const FA& a, const FB& b, const Epi& epi) {
     static_assert(M % 16 == 0 && N % 8 == 0 && K % 8 == 0, "m16n8k8 tiles must divide the product");
-    constexpr int NT = N / 8, TILES = (M / 16) * NT;
+    constexpr int NB = wgemm_nb<M, N>(), NS = N / (8 * NB), STRIPS = (M / 16) * NS;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    for (int tt = threadIdx.x >> 5; tt < TILES; tt += kThreads / 32) {
-        const int m0 = (tt / NT) * 16, n0 = (tt % NT) * 8;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-        for (int k0 = 0; k0 < K; k0 += 8) {
-            const float av[4] = {a(m0 + g, k0 + t), a(m0 + g + 8, k0 + t), a(m0 + g, k0 + t + 4),
-                                 a(m0 + g + 8, k0 + t + 4)};
-            const float bv[2] = {b(k0 + t, n0 + g), b(k0 + t + 4, n0 + g)};
-            uint32_t ah[4], al[4], bh[2], bl[2];
+    for (int st = threadIdx.x >> 5; st < STRIPS; st += kThreads / 32) {
+        const int m0 = (st / NS) * 16, n0 = (st % NS) * 8 * NB;
+        // a single tile with a long K runs two accumulator chains (even and odd k steps)
+        constexpr int NA = (NB == 1 && K >= 64) ? 2 : 1;
+        float acc[NA][NB][4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                ah[e] = tc::f32_to_tf32(av[e]);
-                al[e] = kSa ? tc::f32_to_tf32(av[e] - __uint_as_float(ah[e])) : 0u;
-            }
+        for (int h = 0; h < NA; ++h)
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                bh[e] = tc::f32_to_tf32(bv[e]);
-                bl[e] = kSb ? tc::f32_to_tf32(bv[e] - __uint_as_float(bh[e])) : 0u;
+            for (int nb = 0; nb < NB; ++nb) acc[h][nb][0] = acc[h][nb][1] = acc[h][nb][2] = acc[h][nb][3] = 0.f;
+#pragma unroll 2
+        for (int kb = 0; kb < K; kb += 8 * NA) {
+#pragma unroll
+            for (int h = 0; h < NA; ++h) {
+                const int k0 = kb + 8 * h;
+                uint32_t ah[4], al[4];
+                tf32_split(a(m0 + g, k0 + t), kSa, ah[0], al[0]);
+                tf32_split(a(m0 + g + 8, k0 + t), kSa, ah[1], al[1]);
+                tf32_split(a(m0 + g, k0 + t + 4), kSa, ah[2], al[2]);
+                tf32_split(a(m0 + g + 8, k0 + t + 4), kSa, ah[3], al[3]);
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    uint32_t bh[2], bl[2];
+                    tf32_split(b(k0 + t, n0 + 8 * nb + g), kSb, bh[0], bl[0]);
+                    tf32_split(b(k0 + t + 4, n0 + 8 * nb + g), kSb, bh[1], bl[1]);
+                    if constexpr (kSb) tc::mma_sync_tf32(acc[h][nb], ah[0], ah[1], ah[2], ah[3], bl[0], bl[1]);
+                    if constexpr (kSa) tc::mma_sync_tf32(acc[h][nb], al[0], al[1], al[2], al[3], bh[0], bh[1]);
+                    tc::mma_sync_tf32(acc[h][nb], ah[0], ah[1], ah[2], ah[3], bh[0], bh[1]);
+                }
             }
-            if constexpr (kSb) tc::mma_sync_tf32(acc, ah[0], ah[1], ah[2], ah[3], bl[0], bl[1]);
-            if constexpr (kSa) tc::mma_sync_tf32(acc, al[0], al[1], al[2], al[3], bh[0], bh[1]);
-            tc::mma_sync_tf32(acc, ah[0], ah[1], ah[2], ah[3], bh[0], bh[1]);
         }
-        epi(m0 + g, n0 + 2 * t, acc[0]);
-        epi(m0 + g, n0 + 2 * t + 1, acc[1]);
-        epi(m0 + g + 8, n0 + 2 * t, acc[2]);
-        epi(m0 + g + 8, n0 + 2 * t + 1, acc[3]);
+        if constexpr (NA == 2) {
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[0][nb][e] += acc[1][nb][e];
+        }
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+            const int n = n0 + 8 * nb + 2 * t;
+            epi(m0 + g, n, acc[0][nb][0]);
+            epi(m0 + g, n + 1, acc[0][nb][1]);
+            epi(m0 + g + 8, n, acc[0][nb][2]);
+            epi(m0 + g + 8, n + 1, acc[0][nb][3]);
+        }
     }
 }
 
@@ -388,16 +415,22 @@ __device__ __forceinline__ void from_f32(uint8_t* dst, const float* t, int ld) {
 
 // The chunk states the tensor-core state passes store (S_c and dS'_c, bf16 128 x 128)
 // are laid out by 16-byte pieces: piece c (elements 8c .. 8c+7) of row i at byte
-// (128 c + i) 16, so that 32 threads holding 32 consecutive rows move 512 contiguous
-// bytes per access.
+// (128 c + (i ^ 2 (c % 4))) 16.  32 threads holding 32 consecutive rows move 512
+// contiguous bytes per access; copied whole into shared memory, a column read (32
+// consecutive columns of one row: four pieces 2 KB apart) hits distinct banks.
 namespace stl {
-__host__ __device__ constexpr uint32_t off(int i, int c) { return ((uint32_t)c * 128u + (uint32_t)i) * 16u; }
+__host__ __device__ constexpr uint32_t off(int i, int c) {
+    return ((uint32_t)c * 128u + (uint32_t)(i ^ (2 * (c & 3)))) * 16u;
+}
 }
 
 // Byte offset, inside a chunk's C slot of the workspace, of the decays the tensor-core
 // state passes read (e^{g_L - g_r} for the 32 positions, then e^{g_L}); before it: the
 // G hi, G lo and dO tiles.
 constexpr uint32_t kPrepDec = 3 * tile::kBytes;
+// ... and of the chunk's inverse T = (I + A)^{-1} (fp32 [32][32], row-major), which the
+// grads kernel applies as products instead of solving again.
+constexpr uint32_t kPrepT = 4 * tile::kBytes;
 
 // ---------------------------------------------------------------------------------
 // bwd_prep: W, U~ and C = dO^T (Gamma Q~ - P W) of one chunk.  In the tensor-core form
@@ -486,6 +519,22 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
         }
 #pragma unroll
         for (int r = 0; r < kL; ++r) base[r * ld] = x[r];
+    }
+    if constexpr (kTC) {
+        if (threadIdx.x < kL) {   // T = (I + A)^{-1}, lane = column, by forward substitution
+            const int sc = threadIdx.x;
+            float x[kL];
+#pragma unroll
+            for (int r = 0; r < kL; ++r) {
+                float acc = (r == sc) ? 1.f : 0.f;
+#pragma unroll
+                for (int m = 0; m < r; ++m) acc = fmaf(-Am[r * kLDL + m], x[m], acc);
+                x[r] = acc;
+            }
+            float* Tg = reinterpret_cast<float*>(cs + kPrepT);
+#pragma unroll
+            for (int r = 0; r < kL; ++r) Tg[r * kL + sc] = x[r];
+        }
     }
     __syncthreads();
     // Gamma Q~ - P W, in place over Q~
@@ -623,7 +672,7 @@ struct GradSmem {
     static constexpr size_t K = 0, Q = K + kL * LD, O = Q + kL * LD, V = O + kL * LD, R = V + kL * LD,
                             X = R + kL * LD, D = X + kL * LD, G = D + kL * LD, TK = G + kL * LD,
                             AF = TK + kL * LD, P = AF + kL * kLDL, DP = P + kL * kLDL, DA = DP + kL * kLDL,
-                            VEC = DA + kL * kLDL, RED = VEC + NV * kL, STG = RED + kThreads / 32,
+                            T = DA + kL * kLDL, VEC = T + kL * kLDL, RED = VEC + NV * kL, STG = RED + kThreads / 32,
                             total = STG + kL * LD;   // STG: staging of S / dS' slabs
 };
 
@@ -653,7 +702,7 @@ constexpr uint32_t TILE = 8192;                                     // one 32 x 
 constexpr uint32_t KB = 0, OB = TILE, XB = 2 * TILE, DRB = 3 * TILE, BARS = 4 * TILE, SLOT = BARS + 64;
 constexpr uint32_t kBytes = SLOT + 64;
 constexpr uint32_t ID = tc::idesc_bf16(128, 32, false, false);
-enum { B_ABC = 0, B_D = 1, B_E = 2, B_DRAIN = 3 };
+enum { B_ABC = 0, B_D = 1, B_E = 2, B_DRAIN = 3, B_ST = 4 };
 constexpr unsigned long long kWaitNs = 2000000000ull;   // bound on every wait for an MMA
 
 // waits for a commit (each barrier completes once per CTA: phase 0); a wait that runs
@@ -688,49 +737,37 @@ __device__ __forceinline__ void f32_to_tile(uint32_t dst, const float* t, int ld
         tc::sts_u32x4(dst + boff(r, c), w);
     }
 }
-// The chunk's S and dS' (bf16, the state passes' piece layout) into TMEM as A operands:
-// their rows (lane i, pairs (j, j+1): columns [C_S, +64) and [C_DS, +64)) and their
-// columns (lane j, pairs (i, i+1): [C_ST, +64) and [C_DST, +64)).  Warps 0-3 (thread =
-// row i) load both rows (coalesced), store them to TMEM and to two row-major scratch
-// tiles in shared memory (16-byte pieces XOR-swizzled by row: conflict-free both ways)
-// and return the row's part of <dS', S>.  After the barrier every thread takes a column
-// (lane j): warps 0-3 of dS', warps 4-7 of S, from the scratch.
-__device__ __forceinline__ uint32_t scr_off(int r, int c) {   // piece c of row r of a scratch tile
-    return (uint32_t)r * 256u + ((uint32_t)(c ^ (r & 7)) << 4);
-}
-__device__ __forceinline__ float states_to_tmem(uint32_t tl, int x, const uint8_t* __restrict__ Sg,
-                                                const uint8_t* __restrict__ dSg, uint8_t* scrS, uint8_t* scrD) {
+// The chunk's S and dS' (bf16, the state passes' piece layout, copied whole into
+// shared memory) into TMEM as A operands: their rows (lane i, pairs (j, j+1): columns
+// [C_S, +64) and [C_DS, +64)) and their columns (lane j, pairs (i, i+1): [C_ST, +64)
+// and [C_DST, +64)).  Warps 0-3 (thread = row i) take the rows and return the row's
+// part of <dS', S>; then every thread takes a column (lane j): warps 0-3 of dS', warps
+// 4-7 of S.  Both passes read the copies conflict-free.
+__device__ __forceinline__ float states_to_tmem(uint32_t tl, int x, const uint8_t* scrS, const uint8_t* scrD) {
     const int warp = threadIdx.x >> 5;
     float ss = 0.f;
     if (warp < 4) {
 #pragma unroll 1
         for (int hh = 0; hh < 2; ++hh) {
-            uint4 a[8], b[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                a[e] = *reinterpret_cast<const uint4*>(Sg + stl::off(x, 8 * hh + e));
-                b[e] = *reinterpret_cast<const uint4*>(dSg + stl::off(x, 8 * hh + e));
-            }
             float pa[32], pb[32];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
+                const uint4 a = *reinterpret_cast<const uint4*>(scrS + stl::off(x, 8 * hh + e));
+                const uint4 b = *reinterpret_cast<const uint4*>(scrD + stl::off(x, 8 * hh + e));
                 float fa[8], fb[8];
-                unpack16(a[e], fa);
-                unpack16(b[e], fb);
+                unpack16(a, fa);
+                unpack16(b, fb);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) ss = fmaf(fa[q], fb[q], ss);
-                pa[4 * e] = __uint_as_float(a[e].x); pa[4 * e + 1] = __uint_as_float(a[e].y);
-                pa[4 * e + 2] = __uint_as_float(a[e].z); pa[4 * e + 3] = __uint_as_float(a[e].w);
-                pb[4 * e] = __uint_as_float(b[e].x); pb[4 * e + 1] = __uint_as_float(b[e].y);
-                pb[4 * e + 2] = __uint_as_float(b[e].z); pb[4 * e + 3] = __uint_as_float(b[e].w);
-                *reinterpret_cast<uint4*>(scrS + scr_off(x, 8 * hh + e)) = a[e];
-                *reinterpret_cast<uint4*>(scrD + scr_off(x, 8 * hh + e)) = b[e];
+                pa[4 * e] = __uint_as_float(a.x); pa[4 * e + 1] = __uint_as_float(a.y);
+                pa[4 * e + 2] = __uint_as_float(a.z); pa[4 * e + 3] = __uint_as_float(a.w);
+                pb[4 * e] = __uint_as_float(b.x); pb[4 * e + 1] = __uint_as_float(b.y);
+                pb[4 * e + 2] = __uint_as_float(b.z); pb[4 * e + 3] = __uint_as_float(b.w);
             }
             tc::tmem_st32(tl + C_S + 32 * hh, pa);
             tc::tmem_st32(tl + C_DS + 32 * hh, pb);
         }
     }
-    __syncthreads();
     const uint8_t* scr = (warp < 4) ? scrD : scrS;
     const uint32_t col = (warp < 4) ? C_DST : C_ST;
     const uint32_t sel = (x & 1) ? 0x7632u : 0x5410u;   // this column's half of each word
@@ -741,8 +778,8 @@ __device__ __forceinline__ float states_to_tmem(uint32_t tl, int x, const uint8_
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
             const int r = 64 * hh + 2 * c;
-            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(scr + scr_off(r, x >> 3) + wo);
-            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(scr + scr_off(r + 1, x >> 3) + wo);
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(scr + stl::off(r, x >> 3) + wo);
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(scr + stl::off(r + 1, x >> 3) + wo);
             pk[c] = __uint_as_float(__byte_perm(w0, w1, sel));
         }
         tc::tmem_st32(tl + col + 32 * hh, pk);
@@ -781,7 +818,7 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     extern __shared__ float sm[];
     float *Ks = sm + SM::K, *Qs = sm + SM::Q, *Os = sm + SM::O, *Vs = sm + SM::V, *Rs = sm + SM::R;
     float *Xs = sm + SM::X, *Ds = sm + SM::D, *Gs = sm + SM::G, *TKs = sm + SM::TK;
-    float *AF = sm + SM::AF, *Pm = sm + SM::P, *dPm = sm + SM::DP, *dAm = sm + SM::DA;
+    float *AF = sm + SM::AF, *Pm = sm + SM::P, *dPm = sm + SM::DP, *dAm = sm + SM::DA, *Tm = sm + SM::T;
     float* vec = sm + SM::VEC;
     float* red = sm + SM::RED;
     float* stage = sm + SM::STG;
@@ -806,8 +843,12 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         tcb = (tc::smem_u32(sm + SM::STG) + 1023u) & ~1023u;
         tbar = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sm) + (tcb - s0) + gtc::BARS);
         if (tid == 0) {
-            for (int i = 0; i < 4; ++i) tc::mbar_init(&tbar[i], 1);
+            for (int i = 0; i < 5; ++i) tc::mbar_init(&tbar[i], 1);
             tc::fence_mbar_init();
+            // S and dS' whole, into the R | X and G | TK tiles (free until step 2)
+            tc::mbar_arrive_expect_tx(&tbar[gtc::B_ST], 2u * 32768u);
+            tc::bulk_load(Rs, S, 32768u, &tbar[gtc::B_ST]);
+            tc::bulk_load(Gs, dSp, 32768u, &tbar[gtc::B_ST]);
         }
         if (warp == 0)
             tc::tmem_alloc(reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(sm) + (tcb - s0) + gtc::SLOT),
@@ -831,6 +872,9 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         if constexpr (kTC) {
             gtc::rows_tile(lk, tcb + gtc::KB);
             gtc::rows_tile(lo, tcb + gtc::OB);
+            const float4 t4 = reinterpret_cast<const float4*>(reinterpret_cast<const uint8_t*>(ws.C + ci * DV * DK) +
+                                                              kPrepT)[tid];   // T, 8 float4 per row
+            *reinterpret_cast<float4*>(Tm + (tid >> 3) * kLDL + 4 * (tid & 7)) = t4;
             tc::tc_fence_before();
         }
     }
@@ -840,9 +884,8 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         tmem = *reinterpret_cast<volatile uint32_t*>(reinterpret_cast<uint8_t*>(sm) + (tcb - tc::smem_u32(sm)) +
                                                      gtc::SLOT);
         ttl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        // scratch for the transposition: the R | X and G | TK tiles, not yet in use
-        ss = gtc::states_to_tmem(ttl, xrow, reinterpret_cast<const uint8_t*>(S), reinterpret_cast<const uint8_t*>(dSp),
-                                 reinterpret_cast<uint8_t*>(Rs), reinterpret_cast<uint8_t*>(Gs));
+        if (!tc::mbar_wait(&tbar[gtc::B_ST], 0, gtc::kWaitNs)) latch_status(-4 /* COMBA_ETIMEOUT */);
+        ss = gtc::states_to_tmem(ttl, xrow, reinterpret_cast<const uint8_t*>(Rs), reinterpret_cast<const uint8_t*>(Gs));
         tc::tmem_st_wait();
         tc::fence_proxy_async_smem();   // the B tiles, written by threads, for the tensor pipe
         tc::tc_fence_before();
@@ -894,9 +937,19 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
                                 [&](int m, int n, float s) { Pm[m * kLDL + n] = (n <= m) ? expf(g[m] - g[n]) * s : 0.f; });
         __syncthreads();
     }
-    // 3. X = T diag(beta) (V - diag(e^{g'}) K S^T) by forward substitution (one column
-    //    per thread); dX += P^T dO
-    for (int col = tid; col < DV; col += kThreads) {
+    // 3. X = T diag(beta) (V - diag(e^{g'}) K S^T) (the tensor-core form as a product
+    //    with the prep kernel's T, else by forward substitution, one column per thread);
+    //    dX += P^T dO
+    if constexpr (kTC) {
+        for (int e = tid; e < kL * DV; e += kThreads) {   // the right-hand side, in the free dk tile
+            const int r = e / DV, col = e % DV;
+            TKs[r * LD + col] = bt[r] * fmaf(-egp[r], Rs[r * LD + col], Vs[r * LD + col]);
+        }
+        __syncthreads();
+        wgemm<kL, DV, kL, true, true>([&](int r, int s) { return Tm[r * kLDL + s]; },
+                                      [&](int s, int col) { return TKs[s * LD + col]; },
+                                      [&](int r, int col, float x) { Xs[r * LD + col] = x; });
+    } else for (int col = tid; col < DV; col += kThreads) {
         float x[kL];
 #pragma unroll
         for (int r = 0; r < kL; ++r) {
@@ -912,8 +965,13 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
                             [&](int s, int i) { return Os[s * LD + i]; },
                             [&](int r, int i, float s) { Ds[r * LD + i] += s; });
     __syncthreads();
-    // 4. dR = T^T dX by back substitution, in place
-    for (int col = tid; col < DV; col += kThreads) {
+    // 4. dR = T^T dX (the tensor-core form as a product into the free dk tile, which
+    //    then takes the dX tile's place; else by back substitution, in place)
+    if constexpr (kTC)
+        wgemm<kL, DV, kL, true, true>([&](int r, int s) { return Tm[s * kLDL + r]; },
+                                      [&](int s, int col) { return Ds[s * LD + col]; },
+                                      [&](int r, int col, float x) { TKs[r * LD + col] = x; });
+    else for (int col = tid; col < DV; col += kThreads) {
         float x[kL];
 #pragma unroll
         for (int r = kL - 1; r >= 0; --r) {
@@ -930,6 +988,11 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         tc::fence_proxy_async_smem();
     }
     __syncthreads();
+    if constexpr (kTC) {   // dR now sits in the former dk tile
+        float* t = Ds;
+        Ds = TKs;
+        TKs = t;
+    }
     // 5. dA, dP; row dots dR.(V - e^{g'} K S^T) and dR.(K S^T); Gamma dO S
     if constexpr (kTC) {
         if (warp == 0) {   // (d) dS'^T X^T
@@ -1028,13 +1091,11 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     wgemm<kL, DK, kL, true, kIn>([&](int r, int s) { return dPm[r * kLDL + s]; },
                             [&](int s, int j) { return Ks[s * LD + j]; },
                             [&](int r, int j, float x) { Gs[r * LD + j] += x; });
-    // (the three dk terms share one tiling, so each element stays with one thread)
-    wgemm<kL, DK, kL, true, true>([&](int r, int s) { return dPm[s * kLDL + r]; },
-                            [&](int s, int j) { return Qs[s * LD + j]; },
-                            [&](int r, int j, float x) { TKs[r * LD + j] = x; });
-    wgemm<kL, DK, kL, true, kIn>([&](int r, int s) { return dAm[r * kLDL + s] + dAm[s * kLDL + r]; },
-                            [&](int s, int j) { return Ks[s * LD + j]; },
-                            [&](int r, int j, float x) { TKs[r * LD + j] += x; });
+    // the two dk products as one over 2L: [dZ^T | dY + dY^T] [Q~; K]
+    wgemm<kL, DK, 2 * kL, true, true>(
+        [&](int r, int s) { return s < kL ? dPm[s * kLDL + r] : dAm[r * kLDL + s - kL] + dAm[(s - kL) * kLDL + r]; },
+        [&](int s, int j) { return s < kL ? Qs[s * LD + j] : Ks[(s - kL) * LD + j]; },
+        [&](int r, int j, float x) { TKs[r * LD + j] = x; });
     if constexpr (!kTC)
         bgemm_staged<kL, DK, DV, 4, 4, false>(
             [&](int r, int i) { return Ds[r * LD + i]; }, S, stage,
@@ -1102,7 +1163,8 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         if (warp == 0) {   // every MMA has completed before TMEM is released
             tc::tc_fence_after();
             tc::mma_commit(&tbar[gtc::B_DRAIN]);
-            if (!__all_sync(0xffffffffu, tc::mbar_wait(&tbar[gtc::B_DRAIN], 0, gtc::kWaitNs)) && lane == 0)
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&tbar[gtc::B_DRAIN], 0, gtc::kWaitNs) &&
+                                             tc::mbar_wait(&tbar[gtc::B_ST], 0, gtc::kWaitNs)) && lane == 0)
                 latch_status(-4 /* COMBA_ETIMEOUT */);
             tc::tmem_dealloc(tmem, gtc::kCols);
         }
