@@ -584,9 +584,16 @@ def bwd_algorithmic_flops(cfg):
     return chunks * (prep + states + dstates + grads)
 
 
-def fp32_alu_peak_tflops(sm_mhz: float, sms: int = 148) -> float:
-    """fp32 FMA peak: 148 SMs x 128 fp32 lanes x 2 flops x the SM clock."""
-    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+def bwd_algorithmic_bytes(cfg):
+    """Bytes one backward must move at the least: every input read once (bf16 q, k,
+    v, dout; fp32 gates, d, S0, dS_final) and every gradient written once (fp32 dq,
+    dk, dv, dlog_alpha, dbeta, dS0, dd).  The workspace round trips of the staged
+    design (per-chunk operand tiles, states and state gradients) are not counted."""
+    B, T, H, dk, dv = cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv
+    tok = B * T * H
+    inputs = tok * (2 * dk + 2 * dv) * 2 + tok * 2 * 4 + H * 4 + 2 * B * H * dv * dk * 4
+    grads = tok * (2 * dk + dv) * 4 + tok * 2 * 4 + B * H * dv * dk * 4 + H * 4
+    return inputs + grads
 
 
 def cpu_baseline_bwd(cfg, x, cot, target_s: float = 10.0):
@@ -682,21 +689,23 @@ def run_bwd(args):
     barrier(world)
     ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), world, dev) / args.steps
     flops = bwd_algorithmic_flops(cfg)
+    nbytes = bwd_algorithmic_bytes(cfg)
     ck = clocks.summary(th0, th1)
-    sm_max = ck.get("sm_max_mhz") or 1965.0
-    peak = fp32_alu_peak_tflops(sm_max)
-    tf = flops / (ms_step / 1e3) / 1e12
+    peaks = load_peaks()
+    peak = peaks["hbm_gbs"]
+    gbs = nbytes / (ms_step / 1e3) / 1e9
     line = {
-        "metric": "Comba chunk-bwd tokens/s (all input gradients) on 1 B200, % of fp32 ALU roofline",
+        "metric": "Comba chunk-bwd tokens/s (all input gradients) on 1 B200, % of HBM roofline",
         "value": weak_scaling_value(cfg.B * cfg.T, world, ms_step), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": dict(config_record(cfg), workload=BWD, chunk=BWD_CHUNK, inputs="bf16 q, k, v, dout"),
-        "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-                     "traffic": None,
-                     "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x max SM clock",
-                     "algorithmic_flops_per_launch": flops, "scope": "whole backward (5 kernels)"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                     "traffic": None, "peak_source": peaks["source"],
+                     "algorithmic_bytes_per_step": nbytes, "algorithmic_flops_per_step": flops,
+                     "tflops": flops / (ms_step / 1e3) / 1e12,
+                     "scope": "whole backward step (4 launches), against the bytes it must move at the least"},
         "e2e": {"value": weak_scaling_value(cfg.B * cfg.T, world, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in host.values()),
                 "d2h_bytes_per_step": sum(v.numel() * v.element_size() for v in outs_h.values()),

@@ -1,6 +1,5 @@
 // Chunk-wise Comba backward: gradients of the chunk forward with respect to q, k, v,
-// log_alpha, beta, d and S0, given the cotangents of out and S_final.  fp32 FMA
-// arithmetic throughout.
+// log_alpha, beta, d and S0, given the cotangents of out and S_final.
 //
 // The write-up (section "硬件高效的分块并行计算") says only that the backward pass
 // reuses the chunk-level states and the single inverse per chunk.  The algebra
@@ -22,15 +21,25 @@
 // and the decay gradients collect every exponent's sensitivity into dg_r, then
 // dlog_alpha_i = sum_{r >= i} dg_r inside the chunk.
 //
-// Four kernels, all over a fixed 32-token chunk (a tiling choice: the gradients are
-// the same function of the inputs for any chunk length):
+// Kernels, all over a fixed 32-token chunk (a tiling choice: the gradients are the
+// same function of the inputs for any chunk length):
 //   bwd_prep     (chunk, chain) in parallel: W, U~ and C = dO^T (Gamma Q~ - P W)
 //   bwd_states   one CTA per 32 state rows of a chain, chunks in order: chunk-start
 //                states S_c
 //   bwd_dstates  likewise, chunks in reverse: end-state gradients dS'_c, dS0
 //   bwd_grads    (chunk, chain) in parallel: dq, dk, dv, dlog_alpha, dbeta and a
 //                per-chunk partial of dd
-// plus bwd_dd_sum, which adds the dd partials per head in a fixed order.
+// plus bwd_dd_sum, which adds the dd partials per head in a fixed order.  The
+// shared-memory products run on warp MMAs (wgemm: tf32, fp32 operands split into
+// hi + lo, about fp32 accuracy).  For bf16 inputs with dk = dv = 128 the backward
+// takes its tensor-core form:
+//   bwd_prep     leaves the state passes' operands as bf16 MMA tiles (W, K, dO,
+//                G = Gamma Q~ - P W as hi + lo), U~, the decays and T, instead of C
+//   bwd_chain_tc (chunk_bwd_chain.cuh) both state passes in one launch, tcgen05 MMAs
+//                with the state in TMEM; S_c and dS'_c stored as bf16
+//   bwd_grads    the five state products (K S^T, K dS'^T, dO S, X dS', dR S) as
+//                tcgen05 MMAs with the bf16 states in TMEM, X and dR as products with T
+// whose bf16 state operands hold every gradient to the bf16 workloads' rel-L2 5e-3.
 #pragma once
 
 #include <type_traits>

@@ -284,13 +284,18 @@ int comba_recurrent_step_grouped(const void* q, const void* k, const void* v,
  * output above.  The write-up (section "硬件高效的分块并行计算") states only that
  * the backward pass reuses the chunk-level states and the per-chunk inverse; this
  * entry point computes the adjoint of the chunk form in four stages.
- *  1. Per chunk in parallel: W, U~ and dO^T (Gamma Q~ - P W).
+ *  1. Per chunk in parallel: W, U~, the inverse and dO^T (Gamma Q~ - P W).
  *  2. The chunk-start states, chunks in order.
  *  3. The end-state gradients, chunks in reverse.
  *  4. Per chunk in parallel: the input gradients.
  * It recomputes the states rather than reading saved ones.  Chunks are 32 tokens
  * (a tiling choice: the result is the same function of the inputs for any chunk
- * length).  fp32 arithmetic throughout.
+ * length).  Precision: fp32 inputs, and bf16 inputs with dk or dv below 128, are
+ * computed to about fp32 accuracy (warp MMAs on split tf32 operands; every gradient
+ * within rel-L2 1e-4 of the exact one).  bf16 inputs with dk = dv = 128 take the
+ * tensor-core form: stages 2 and 3 run as one launch on tcgen05 MMAs with the
+ * states in bf16, as do the state products of stage 4; every gradient, dS0
+ * included, is within rel-L2 5e-3 of the exact one (the bf16 workloads' bound).
  *
  * q, k [B, T, H, dk], v and dout [B, T, H, dv]: element type `dtype` (COMBA_BF16 or
  * COMBA_F32), the same values the forward read.  log_alpha, beta [B, T, H], d [H],
@@ -303,9 +308,9 @@ int comba_recurrent_step_grouped(const void* q, const void* k, const void* v,
  *  - dS0 [B, H, dv, dk] (NULL skips it).
  * dk, dv in {32, 64, 128}; any T >= 0 (T == 0: dS0 = dS_final, dd = 0); B * H <= 65535.
  * workspace: DEVICE memory, 16-byte aligned, at least
- * comba_chunk_bwd_workspace_size(B, T, H, dk, dv) bytes (per chunk: W, U~ and three
- * dv x dk fp32 matrices), owned by the caller and in use until `stream` has passed
- * the call.  q, k, v, dout, S0 and dS_final 16-byte aligned; everything else
+ * comba_chunk_bwd_workspace_size(B, T, H, dk, dv) bytes (per chunk: room for W, U~
+ * and three dv x dk fp32 matrices), owned by the caller and in use until `stream`
+ * has passed the call; its contents between calls are unspecified.  q, k, v, dout, S0 and dS_final 16-byte aligned; everything else
  * 4-byte aligned.  No output may overlap an input,
  * another output or the workspace.  Returns COMBA_EINVAL for a bad size, pointer,
  * alignment, overlap or workspace; COMBA_EUNSUPPORTED for B * H > 65535.
