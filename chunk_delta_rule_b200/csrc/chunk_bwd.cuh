@@ -353,9 +353,9 @@ __device__ __forceinline__ void rows_store(const RowLoad<D, Tin>& L, float* dst,
         if (R::NV % kThreads == 0 || e < R::NV) {
             float f[R::VE];
             unpack16(L.w[it], f);
-            float* o = dst + (e / R::VPR) * ld + (e % R::VPR) * R::VE;
+            float4* o = reinterpret_cast<float4*>(dst + (e / R::VPR) * ld + (e % R::VPR) * R::VE);   // ld % 4 == 0
 #pragma unroll
-            for (int x = 0; x < R::VE; ++x) o[x] = f[x];
+            for (int x = 0; x < R::VE / 4; ++x) o[x] = make_float4(f[4 * x], f[4 * x + 1], f[4 * x + 2], f[4 * x + 3]);
         }
     }
 }
@@ -405,7 +405,9 @@ __device__ __forceinline__ void from_f32(uint8_t* dst, const float* t, int ld) {
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
         const int e = threadIdx.x + it * kThreads, r = e >> 4, c = e & 15;
-        const float* x = t + r * ld + 8 * c;
+        const float4 x0 = *reinterpret_cast<const float4*>(t + r * ld + 8 * c);   // ld % 4 == 0
+        const float4 x1 = *reinterpret_cast<const float4*>(t + r * ld + 8 * c + 4);
+        const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
         uint32_t w[4];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
@@ -737,12 +739,13 @@ __device__ __forceinline__ void f32_to_tile(uint32_t dst, const float* t, int ld
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
         const int e = threadIdx.x + it * kThreads, r = e >> 4, c = e & 15;
-        const float* x = t + r * ld + 8 * c;
+        const float4 x0 = *reinterpret_cast<const float4*>(t + r * ld + 8 * c);   // ld % 4 == 0
+        const float4 x1 = *reinterpret_cast<const float4*>(t + r * ld + 8 * c + 4);
         uint4 w;
-        w.x = tc::pack_bf16(x[0], x[1]);
-        w.y = tc::pack_bf16(x[2], x[3]);
-        w.z = tc::pack_bf16(x[4], x[5]);
-        w.w = tc::pack_bf16(x[6], x[7]);
+        w.x = tc::pack_bf16(x0.x, x0.y);
+        w.y = tc::pack_bf16(x0.z, x0.w);
+        w.z = tc::pack_bf16(x1.x, x1.y);
+        w.w = tc::pack_bf16(x1.z, x1.w);
         tc::sts_u32x4(dst + boff(r, c), w);
     }
 }
