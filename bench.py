@@ -711,7 +711,7 @@ def run_bwd(args):
                 "d2h_bytes_per_step": sum(v.numel() * v.element_size() for v in outs_h.values()),
                 "ms_per_step": ms_e2e},
         "clocks": ck,
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": 4 * args.steps,   # prep, both state passes, grads, dd sum
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline_bwd(cfg, x, x).items() if k != "seconds"}
