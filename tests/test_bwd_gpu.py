@@ -94,6 +94,31 @@ def test_bwd_single_token_and_empty_sequence():
     assert np.array_equal(g["dd"], np.zeros(3))
 
 
+@pytest.mark.parametrize("T", [1, 32, 33, 45, 257])
+def test_bwd_tensor_core_form_edge_lengths(T):
+    """bf16, dk = dv = 128 (the tensor-core form): one token (the forward walk has no
+    update step), exactly one chunk, a ragged second chunk, and longer ragged tails;
+    with and without an initial state and a state cotangent."""
+    for s0, ds in ((0.0, 1.0), (0.2, 0.0), (0.2, 1.0)):
+        cfg = CONFIGS["layer340m_bf16"].replace(B=2, H=2, T=T, dk=128, dv=128, dtype="bf16", s0_std=s0,
+                                                decay="mamba")
+        x = make_chunk_inputs(cfg, seed=300 + T)
+        cot = make_cotangents(cfg, seed=400 + T, dS_std=ds)
+        check(x, cot, run(x, cot), tol=TOL_BWD_TC)
+
+
+def test_bwd_tensor_core_form_empty_sequence():
+    cfg = CONFIGS["layer340m_bf16"].replace(B=2, H=3, T=1, dk=128, dv=128, dtype="bf16", s0_std=0.3)
+    x = make_chunk_inputs(cfg, seed=13)
+    cot = make_cotangents(cfg, seed=14)
+    empty = {k: (v[:, :0].contiguous() if (v is not None and v.dim() >= 3 and k not in ("S0",)) else v)
+             for k, v in x.items()}
+    cot0 = {"dout": cot["dout"][:, :0].contiguous(), "dS_final": cot["dS_final"]}
+    g = run(empty, cot0)
+    assert np.array_equal(g["dS0"], cot["dS_final"].double().numpy())
+    assert np.array_equal(g["dd"], np.zeros(3))
+
+
 def test_bwd_full_layer_sampled_chains():
     """The 1.3B layer (B=8, T=4096, H=16, dk=dv=128, bf16): every output of three
     sampled (b, h) chains against the oracle run on those chains alone (chains are
