@@ -50,6 +50,18 @@
 namespace comba {
 namespace bwd {
 
+// Prefetch of `bytes` of global memory into L2 (16-byte aligned, a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t num_sms() {
+    uint32_t n;
+    asm("mov.u32 %0, %%nsmid;" : "=r"(n));
+    return n;
+}
+
 constexpr int kL = 32;           // tokens per backward chunk (one warp's lanes)
 constexpr int kLDL = kL + 4;     // padded row stride of the L x L tiles (4 mod 32: see wgemm)
 constexpr int kThreads = 256;
@@ -861,6 +873,22 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
             tc::mbar_arrive_expect_tx(&tbar[gtc::B_ST], 2u * 32768u);
             tc::bulk_load(Rs, S, 32768u, &tbar[gtc::B_ST]);
             tc::bulk_load(Gs, dSp, 32768u, &tbar[gtc::B_ST]);
+        }
+        // The CTA one wave ahead (one CTA per SM) finds its inputs in L2: its states,
+        // T and its rows of q, k, v and dout, prefetched now.
+        const long lin = (long)bh * nch + c, nxt = lin + num_sms();
+        if (nxt < (long)gridDim.y * nch) {
+            const int c2 = (int)(nxt % nch), bh2 = (int)(nxt / nch), t2 = c2 * kL, L2c = min(kL, T - t2);
+            const size_t ci2 = (size_t)bh2 * nch + c2, r2 = ((size_t)(bh2 / H) * T + t2) * H + bh2 % H;
+            if (tid == 32) {
+                prefetch_l2(ws.S + ci2 * DV * DK, 32768u);
+                prefetch_l2(ws.dS + ci2 * DV * DK, 32768u);
+                prefetch_l2(reinterpret_cast<const uint8_t*>(ws.C + ci2 * DV * DK) + kPrepT, 4096u);
+            } else if (tid >= 128 && tid - 128 < 4 * L2c) {   // one 256-byte row each
+                const int r = (tid - 128) >> 2, which = (tid - 128) & 3;
+                const Tin* base = which == 0 ? q : which == 1 ? k : which == 2 ? v : dout;
+                prefetch_l2(base + (r2 + (size_t)r * H) * 128, 256u);
+            }
         }
         if (warp == 0)
             tc::tmem_alloc(reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(sm) + (tcb - s0) + gtc::SLOT),
