@@ -463,9 +463,9 @@ constexpr uint32_t kPrepT = 4 * tile::kBytes;
 template <typename Tin, int DK, int DV>
 struct PrepSmem {
     static constexpr int LDK = DK + 4, LDV = DV + 4;   // 4 mod 32 (wgemm)
-    static constexpr size_t K = 0, Q = K + kL * LDK, V = Q + kL * LDK, O = V + kL * LDV, A = O + kL * LDV,
-                            P = A + kL * kLDL, G = P + kL * kLDL, GP = G + kL, BT = GP + kL, CW = BT + kL,
-                            total = CW + kL;
+    static constexpr size_t K = 0, Q = K + kL * LDK, V = Q + kL * LDK, O = V + kL * LDV, W = O + kL * LDV,
+                            A = W + kL * LDK, P = A + kL * kLDL, TI = P + kL * kLDL, G = TI + kL * kLDL,
+                            GP = G + kL, BT = GP + kL, CW = BT + kL, total = CW + kL;
 };
 
 template <typename Tin, int DK, int DV>
@@ -478,7 +478,7 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     extern __shared__ float sm[];
     float *Ks = sm + SM::K, *Qs = sm + SM::Q, *Vs = sm + SM::V, *Os = sm + SM::O;
     float *Am = sm + SM::A, *Pm = sm + SM::P, *g = sm + SM::G, *gp = sm + SM::GP, *bt = sm + SM::BT,
-          *cw = sm + SM::CW;
+          *cw = sm + SM::CW, *Ws = sm + SM::W, *Ti = sm + SM::TI;
     const int c = blockIdx.x, bh = blockIdx.y, b = bh / H, h = bh % H;
     const int t0 = c * kL, Lc = min(kL, T - t0);
     const size_t row0 = ((size_t)b * T + t0) * H + h;
@@ -527,48 +527,61 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
                                  [&](int x, int n) { return Ks[n * LDK + x]; },
                                  [&](int m, int n, float s) { Pm[m * kLDL + n] = (n <= m) ? expf(g[m] - g[n]) * s : 0.f; });
     __syncthreads();
-    // [W | U~] = (I + A)^{-1} [diag(beta e^{g'}) K | diag(beta) V]: one column per
-    // thread, forward substitution down the column, in place over K and V
-    for (int col = threadIdx.x; col < DK + DV; col += kThreads) {
-        float* base = (col < DK) ? Ks + col : Vs + (col - DK);
-        const int ld = (col < DK) ? LDK : LDV;
-        float x[kL];
+    // T = (I + A)^{-1} by 16 x 16 blocks: the diagonal blocks by forward substitution
+    // (lane = column), then T21 = -T22 A21 T11
+    const int tid = threadIdx.x;
+    if (tid < kL) {
+        const int o = (tid < 16) ? 0 : 16, sc = tid - o;
+        float x[16];
 #pragma unroll
-        for (int r = 0; r < kL; ++r) {
-            float acc = ((col < DK) ? cw[r] : bt[r]) * base[r * ld];
+        for (int r = 0; r < 16; ++r) {
+            float acc = (r == sc) ? 1.f : 0.f;
 #pragma unroll
-            for (int s = 0; s < r; ++s) acc = fmaf(-Am[r * kLDL + s], x[s], acc);
+            for (int m = 0; m < r; ++m) acc = fmaf(-Am[(o + r) * kLDL + o + m], x[m], acc);
             x[r] = acc;
         }
 #pragma unroll
-        for (int r = 0; r < kL; ++r) base[r * ld] = x[r];
+        for (int r = 0; r < 16; ++r) Ti[(o + r) * kLDL + o + sc] = x[r];
+    } else {
+        for (int e = tid - kL; e < 256; e += kThreads - kL) Ti[(e >> 4) * kLDL + 16 + (e & 15)] = 0.f;
     }
+    __syncthreads();
+    {   // A21 T11 into the W tile (scratch)
+        const int r = 16 + (tid >> 4), sc = tid & 15;
+        float acc = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) acc = fmaf(Am[r * kLDL + m], Ti[m * kLDL + sc], acc);
+        Ws[(tid >> 4) * LDK + sc] = acc;
+    }
+    __syncthreads();
+    {
+        const int r = 16 + (tid >> 4), sc = tid & 15;
+        float acc = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) acc = fmaf(Ti[r * kLDL + 16 + m], Ws[m * LDK + sc], acc);
+        Ti[r * kLDL + sc] = -acc;
+    }
+    __syncthreads();
+    // U~ = T diag(beta) V (to the workspace) and W = T diag(beta e^{g'}) K (to the W tile)
+    float* Ug = ws.U + ci * kL * DV;
+    wgemm<kL, DV, kL, true, true>([&](int r, int x) { return Ti[r * kLDL + x]; },
+                                  [&](int x, int col) { return bt[x] * Vs[x * LDV + col]; },
+                                  [&](int r, int col, float u) { Ug[r * DV + col] = u; });
+    wgemm<kL, DK, kL, true, true>([&](int r, int x) { return Ti[r * kLDL + x]; },
+                                  [&](int x, int col) { return cw[x] * Ks[x * LDK + col]; },
+                                  [&](int r, int col, float w) { Ws[r * LDK + col] = w; });
     if constexpr (kTC) {
-        if (threadIdx.x < kL) {   // T = (I + A)^{-1}, lane = column, by forward substitution
-            const int sc = threadIdx.x;
-            float x[kL];
-#pragma unroll
-            for (int r = 0; r < kL; ++r) {
-                float acc = (r == sc) ? 1.f : 0.f;
-#pragma unroll
-                for (int m = 0; m < r; ++m) acc = fmaf(-Am[r * kLDL + m], x[m], acc);
-                x[r] = acc;
-            }
-            float* Tg = reinterpret_cast<float*>(cs + kPrepT);
-#pragma unroll
-            for (int r = 0; r < kL; ++r) Tg[r * kL + sc] = x[r];
-        }
+        float* Tg = reinterpret_cast<float*>(cs + kPrepT);
+        for (int e = tid; e < kL * kL; e += kThreads) Tg[e] = Ti[(e >> 5) * kLDL + (e & 31)];
     }
     __syncthreads();
     // Gamma Q~ - P W, in place over Q~
     wgemm<kL, DK, kL, true, true>([&](int m, int x) { return Pm[m * kLDL + x]; },
-                                  [&](int x, int n) { return Ks[x * LDK + n]; },
+                                  [&](int x, int n) { return Ws[x * LDK + n]; },
                                   [&](int m, int n, float s) { Qs[m * LDK + n] = fmaf(expf(g[m]), Qs[m * LDK + n], -s); });
     __syncthreads();
-    float* Ug = ws.U + ci * kL * DV;
-    for (int e = threadIdx.x; e < kL * DV; e += kThreads) Ug[e] = Vs[(e / DV) * LDV + e % DV];
     if constexpr (kTC) {
-        tile::from_f32<false>(wk, Ks, LDK);
+        tile::from_f32<false>(wk, Ws, LDK);
         tile::from_f32<false>(cs, Qs, LDK);
         tile::from_f32<true>(cs + tile::kBytes, Qs, LDK);
     } else {
@@ -577,7 +590,7 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
                                      [&](int r, int j) { return Qs[r * LDK + j]; },
                                      [&](int i, int j, float s) { Cg[(size_t)i * DK + j] = s; });
         float* Wg = ws.W + ci * kL * DK;
-        for (int e = threadIdx.x; e < kL * DK; e += kThreads) Wg[e] = Ks[(e / DK) * LDK + e % DK];
+        for (int e = threadIdx.x; e < kL * DK; e += kThreads) Wg[e] = Ws[(e / DK) * LDK + e % DK];
     }
 }
 
