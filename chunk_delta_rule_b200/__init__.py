@@ -33,7 +33,7 @@ EXPORTS = ("comba_chunk_fwd", "comba_chunk_fwd_f32", "comba_chunk_fwd_varlen",
            "comba_chunk_fwd_workspace_size", "comba_chunk_fwd_ws", "comba_chunk_fwd_noalloc",
            "comba_chunk_fwd_host", "comba_chunk_fwd_host_workspace_size", "comba_chunk_fwd_gated",
            "comba_chunk_bwd", "comba_chunk_bwd_workspace_size", "comba_state_compose",
-           "comba_chunk_fwd_transition", "comba_chunk_fwd_stall_test",
+           "comba_chunk_fwd_transition", "comba_chunk_fwd_stall_test", "comba_chunk_bwd_stall_test",
            "comba_recurrent_step", "comba_recurrent_step_grouped", "comba_get_last_error",
            "comba_get_last_error_stream", "comba_status_string", "comba_version")
 
@@ -76,13 +76,15 @@ def library():
             lib.comba_state_compose.argtypes = [vp] * 3 + [i] * 3 + [vp]
             lib.comba_chunk_fwd_transition.argtypes = [vp] * 7 + [i] * 6 + [vp]
             lib.comba_chunk_fwd_stall_test.argtypes = [vp] * 9 + [i] * 6 + [ctypes.c_ulonglong, i, vp]
+            lib.comba_chunk_bwd_stall_test.argtypes = ([vp] * 16 + [i] * 6 + [vp, ctypes.c_size_t, ctypes.c_ulonglong, i,
+                                                        vp])
             lib.comba_chunk_bwd_workspace_size.restype = ctypes.c_size_t
             lib.comba_recurrent_step_grouped.argtypes = [vp] * 8 + [i] * 5 + [vp]
             for fn in (lib.comba_chunk_fwd, lib.comba_chunk_fwd_f32, lib.comba_chunk_fwd_ws,
                        lib.comba_chunk_fwd_noalloc, lib.comba_chunk_fwd_varlen,
                        lib.comba_recurrent_step_grouped, lib.comba_chunk_fwd_host,
                        lib.comba_chunk_fwd_gated, lib.comba_chunk_bwd, lib.comba_state_compose,
-                       lib.comba_chunk_fwd_transition, lib.comba_chunk_fwd_stall_test,
+                       lib.comba_chunk_fwd_transition, lib.comba_chunk_fwd_stall_test, lib.comba_chunk_bwd_stall_test,
                        lib.comba_recurrent_step, lib.comba_get_last_error,
                        lib.comba_get_last_error_stream, lib.comba_version):
                 fn.restype = ctypes.c_int

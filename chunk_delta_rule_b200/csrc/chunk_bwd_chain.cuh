@@ -52,7 +52,7 @@ enum { B_FULL0 = 0, B_FULL1 = 1, B_SREADY = 2, B_SPLIT = 3, B_MMA1 = 4, B_MMA2 =
 constexpr uint32_t ID_N32 = tc::idesc_bf16(128, 32, false, false);    // S W^T, dS' K^T
 constexpr uint32_t ID_N128B = tc::idesc_bf16(128, 128, false, true);  // Xd^T K, Zd W (B MN-major)
 constexpr uint32_t ID_N128AB = tc::idesc_bf16(128, 128, true, true);  // dO^T G
-constexpr unsigned long long kWaitNs = 2000000000ull;
+constexpr unsigned long long kWaitNs = 2000000000ull;   // the default per-wait limit
 
 // Reading out the state row this thread owns (lane = row i) after a chunk's update,
 // in two passes so the next chunk's first MMA waits only for the first:
@@ -148,7 +148,9 @@ __device__ __forceinline__ void load_in(uint32_t tl, int row, const float* __res
 
 __global__ void __launch_bounds__(kThreads)
 bwd_chain_tc_kernel(Workspace ws, const float* __restrict__ S0, const float* __restrict__ dS_final,
-                    float* __restrict__ dS0, int chains, int nch) {
+                    float* __restrict__ dS0, int chains, int nch, unsigned long long timeout_ns, int stall) {
+    // draining what was issued waits at least 100 ms, whatever the per-wait limit
+    const unsigned long long drain_ns = timeout_ns > 100000000ull ? timeout_ns : 100000000ull;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t base = (tc::smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t* sm = smem_raw + (base - tc::smem_u32(smem_raw));
@@ -182,7 +184,7 @@ bwd_chain_tc_kernel(Workspace ws, const float* __restrict__ S0, const float* __r
         latch_status(-4 /* COMBA_ETIMEOUT */);
     };
     auto wait = [&](int b, uint32_t parity) -> bool {
-        const bool ok = (*abort_flag == 0) && tc::mbar_wait(&bars[b], parity, kWaitNs);
+        const bool ok = (*abort_flag == 0) && tc::mbar_wait(&bars[b], parity, timeout_ns);
         if (!ok) fail();
         return ok;
     };
@@ -286,6 +288,9 @@ bwd_chain_tc_kernel(Workspace ws, const float* __restrict__ S0, const float* __r
             for (; issued < 2 && issued < nit; ++issued) load(issued);
         issued = __shfl_sync(0xffffffffu, issued, 0);
         bool ok = true;
+        // stall: a wait on a phase that nothing completes before the drain below (the
+        // failure-path test), so it runs out after timeout_ns and ends the walk
+        if (stall) ok = __all_sync(0xffffffffu, wait(B_DRAIN, 0)) != 0;
         for (int n = 0; n < nit && ok; ++n) {
             const uint32_t st = base + (n & 1) * ST_BYTES;
             ok = __all_sync(0xffffffffu, wait((n & 1) ? B_FULL1 : B_FULL0, (n >> 1) & 1) && wait(B_SREADY, n & 1)) != 0;
@@ -325,9 +330,9 @@ bwd_chain_tc_kernel(Workspace ws, const float* __restrict__ S0, const float* __r
         // the ring are released
         __syncwarp();
         tc::mma_commit(&bars[B_DRAIN]);
-        tc::mbar_wait(&bars[B_DRAIN], 0, kWaitNs);
+        tc::mbar_wait(&bars[B_DRAIN], 0, drain_ns);
         for (int m = (issued > 2 ? issued - 2 : 0); m < issued; ++m)
-            tc::mbar_wait(&bars[(m & 1) ? B_FULL1 : B_FULL0], (m >> 1) & 1, kWaitNs);
+            tc::mbar_wait(&bars[(m & 1) ? B_FULL1 : B_FULL0], (m >> 1) & 1, drain_ns);
     }
     tc::tc_fence_before();
     __syncthreads();

@@ -516,6 +516,8 @@ struct BwdArgs {
     const float *log_alpha, *beta, *d, *S0, *dS_final;
     float *dq, *dk, *dv, *dlog_alpha, *dbeta, *dd, *dS0;
     int B, T, H, DK, DV;
+    unsigned long long timeout_ns = comba::bwd::chain::kWaitNs;   // the state passes' per-wait limit
+    int stall = 0;                                                 // their failure-path test
 };
 
 template <typename Tin, int DK, int DV>
@@ -553,7 +555,7 @@ int launch_bwd(const BwdArgs& a, float* wsp, cudaStream_t s) {
         }
         if (chains > 0)
             bw::chain::bwd_chain_tc_kernel<<<(unsigned)(2 * chains), bw::chain::kThreads, bw::chain::kSmemBytes, s>>>(
-                ws, a.S0, a.dS_final, a.dS0, (int)chains, nch);
+                ws, a.S0, a.dS_final, a.dS0, (int)chains, nch, a.timeout_ns, a.stall);
     } else if (chains > 0 && nch > 0) {
         const dim3 grid((unsigned)nch, (unsigned)chains);
         bw::bwd_prep_kernel<Tin, DK, DV><<<grid, bw::kThreads, sp, s>>>(q, k, v, a.log_alpha, a.beta, a.d, o, ws,
@@ -603,11 +605,12 @@ extern "C" size_t comba_chunk_bwd_workspace_size(int B, int T, int H, int dk, in
     return comba::bwd::workspace_floats((long)B * H, nch, dk, dv) * sizeof(float);
 }
 
-extern "C" int comba_chunk_bwd(const void* q, const void* k, const void* v, const float* log_alpha,
-                               const float* beta, const float* d, const float* S0, const void* dout,
-                               const float* dS_final, float* dq, float* dk, float* dv, float* dlog_alpha,
-                               float* dbeta, float* dd, float* dS0, int B, int T, int H, int dk_, int dv_,
-                               int dtype, void* workspace, size_t workspace_bytes, comba_stream_t stream) {
+static int chunk_bwd_impl(const void* q, const void* k, const void* v, const float* log_alpha,
+                          const float* beta, const float* d, const float* S0, const void* dout,
+                          const float* dS_final, float* dq, float* dk, float* dv, float* dlog_alpha,
+                          float* dbeta, float* dd, float* dS0, int B, int T, int H, int dk_, int dv_,
+                          int dtype, void* workspace, size_t workspace_bytes, comba_stream_t stream,
+                          unsigned long long timeout_ns, int stall) {
     if (B < 0 || T < 0 || H < 0 || !bwd_dim(dk_) || !bwd_dim(dv_)) return COMBA_EINVAL;
     if (dtype != COMBA_BF16 && dtype != COMBA_F32) return COMBA_EINVAL;
     const size_t elt = (dtype == COMBA_BF16) ? 2 : 4;
@@ -638,10 +641,32 @@ extern "C" int comba_chunk_bwd(const void* q, const void* k, const void* v, cons
             if (overlap(outs[i], nout[i], outs[j], nout[j])) return COMBA_EINVAL;
     }
     const BwdArgs a{q, k, v, dout, log_alpha, beta, d, S0, dS_final, dq, dk, dv, dlog_alpha, dbeta, dd, dS0,
-                    B, T, H, dk_, dv_};
+                    B, T, H, dk_, dv_, timeout_ns, stall};
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     float* ws = static_cast<float*>(workspace);
     return dtype == COMBA_BF16 ? launch_bwd_dk<__nv_bfloat16>(a, ws, s) : launch_bwd_dk<float>(a, ws, s);
+}
+
+extern "C" int comba_chunk_bwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                               const float* beta, const float* d, const float* S0, const void* dout,
+                               const float* dS_final, float* dq, float* dk, float* dv, float* dlog_alpha,
+                               float* dbeta, float* dd, float* dS0, int B, int T, int H, int dk_, int dv_,
+                               int dtype, void* workspace, size_t workspace_bytes, comba_stream_t stream) {
+    return chunk_bwd_impl(q, k, v, log_alpha, beta, d, S0, dout, dS_final, dq, dk, dv, dlog_alpha, dbeta, dd, dS0,
+                          B, T, H, dk_, dv_, dtype, workspace, workspace_bytes, stream,
+                          comba::bwd::chain::kWaitNs, 0);
+}
+
+extern "C" int comba_chunk_bwd_stall_test(const void* q, const void* k, const void* v, const float* log_alpha,
+                                          const float* beta, const float* d, const float* S0, const void* dout,
+                                          const float* dS_final, float* dq, float* dk, float* dv,
+                                          float* dlog_alpha, float* dbeta, float* dd, float* dS0, int B, int T,
+                                          int H, int dk_, int dv_, int dtype, void* workspace,
+                                          size_t workspace_bytes, unsigned long long timeout_ns, int stall,
+                                          comba_stream_t stream) {
+    if (dtype != COMBA_BF16 || dk_ != 128 || dv_ != 128) return COMBA_EUNSUPPORTED;
+    return chunk_bwd_impl(q, k, v, log_alpha, beta, d, S0, dout, dS_final, dq, dk, dv, dlog_alpha, dbeta, dd, dS0,
+                          B, T, H, dk_, dv_, dtype, workspace, workspace_bytes, stream, timeout_ns, stall);
 }
 
 extern "C" int comba_state_compose(const float* RM, const float* S0, float* S_start, int B, int H, int P,

@@ -325,6 +325,28 @@ int comba_chunk_bwd(const void* q, const void* k, const void* v,
                     void* workspace, size_t workspace_bytes, comba_stream_t stream);
 
 /*
+ * comba_chunk_bwd in its tensor-core form (dtype COMBA_BF16, dk = dv = 128; other
+ * inputs return COMBA_EUNSUPPORTED) with the state passes' per-wait limit set to
+ * `timeout_ns` instead of the default 2 s, and, when `stall` is nonzero, with one
+ * extra wait in each state-pass CTA (its copy and MMA-issue warp's, before the first
+ * chunk) on a barrier phase that nothing completes.  It exists to exercise that
+ * kernel's failure path without faulting the GPU: the wait runs out, COMBA_ETIMEOUT
+ * is latched in the device status word (comba_get_last_error), every thread leaves
+ * the chunk walk (the other waits run out too), the kernel waits (for at least 100
+ * ms more) for the copies and MMAs it has already issued, releases its tensor memory
+ * and returns; the gradients are then undefined.  With stall == 0 it is
+ * comba_chunk_bwd with another wait limit.
+ */
+int comba_chunk_bwd_stall_test(const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta, const float* d,
+                               const float* S0, const void* dout, const float* dS_final,
+                               float* dq, float* dk, float* dv, float* dlog_alpha, float* dbeta,
+                               float* dd, float* dS0,
+                               int B, int T, int H, int dk_dim, int dv_dim, int dtype,
+                               void* workspace, size_t workspace_bytes,
+                               unsigned long long timeout_ns, int stall, comba_stream_t stream);
+
+/*
  * Start states of P consecutive sequence pieces from their affine state
  * transitions: over a piece, the state pass maps a start state S to S M + R (R: the
  * end state from S = 0; M: the end state from S = I with V = 0).  This is the

@@ -317,6 +317,20 @@ def test_chunk_transition_rejects_bad_arguments(lib):
     assert call(B=0) == 0                             # empty: nothing launched
 
 
+def test_chunk_bwd_stall_test_takes_only_the_tensor_core_form(lib):
+    p = lambda x: ctypes.c_void_p(x)
+    args = [p(BASE + i * GB) for i in range(16)]
+
+    def call(dk=128, dv=128, dtype=0):
+        return lib.comba_chunk_bwd_stall_test(*args, 2, 64, 2, dk, dv, dtype, p(BASE + 20 * GB),
+                                              ctypes.c_size_t(1 << 30), ctypes.c_ulonglong(1000), 1,
+                                              ctypes.c_void_p(None))
+
+    assert call(dtype=1) == -2          # fp32 inputs: not the tensor-core form
+    assert call(dk=64) == -2
+    assert call(dv=32) == -2
+
+
 def test_stream_status_read_is_exported(lib):
     assert hasattr(lib, "comba_get_last_error_stream")
     assert "comba_get_last_error_stream" in cdr.EXPORTS

@@ -65,3 +65,38 @@ def test_generous_limit_changes_nothing():
     torch.cuda.synchronize()
     assert lib.comba_get_last_error() == 0
     assert torch.equal(out, o) and torch.equal(Sf, S)
+
+
+def test_backward_state_pass_wait_that_runs_out_and_the_device_recovers():
+    """The same for the backward's tensor-core state passes (bf16, dk = dv = 128)."""
+    from comba_workloads import make_cotangents
+    cfg = CONFIGS["layer340m_bf16"].replace(B=1, H=2, T=200, dk=128, dv=128, s0_std=0.1)
+    x = make_chunk_inputs(cfg, seed=919)
+    cot = make_cotangents(cfg, seed=929)
+    xd = {k: (None if v is None else v.cuda()) for k, v in {**x, **cot}.items()}
+    lib = cdr.library()
+    assert lib.comba_get_last_error() == 0
+    B, T, H = 1, 200, 2
+    f32 = lambda *s: torch.zeros(*s, dtype=torch.float32, device="cuda")
+    g = dict(dq=f32(B, T, H, 128), dk=f32(B, T, H, 128), dv=f32(B, T, H, 128), dla=f32(B, T, H),
+             dbt=f32(B, T, H), dd=f32(H), dS0=f32(B, H, 128, 128))
+    need = int(lib.comba_chunk_bwd_workspace_size(B, T, H, 128, 128))
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    st = lib.comba_chunk_bwd_stall_test(
+        p(xd["q"]), p(xd["k"]), p(xd["v"]), p(xd["log_alpha"]), p(xd["beta"]), p(xd["d"]), p(xd["S0"]),
+        p(xd["dout"]), p(xd["dS_final"]), p(g["dq"]), p(g["dk"]), p(g["dv"]), p(g["dla"]), p(g["dbt"]),
+        p(g["dd"]), p(g["dS0"]), B, T, H, 128, 128, 0, p(ws), ctypes.c_size_t(need), ctypes.c_ulonglong(50_000),
+        1, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    assert lib.comba_get_last_error() == COMBA_ETIMEOUT
+    assert lib.comba_get_last_error() == 0
+    # a normal backward on the same device and process
+    res = cdr.chunk_bwd(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["d"], xd["dout"],
+                        S0=xd["S0"], dS_final=xd["dS_final"])
+    torch.cuda.synchronize()
+    assert lib.comba_get_last_error() == 0
+    ref = oracle.recurrence_bwd_np(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["d"], x["S0"],
+                                   cot["dout"], cot["dS_final"])
+    for n in ("dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0"):
+        assert_close(n, res[n].double().cpu().numpy(), ref[n], dict(rel=5e-3, abs=None))
