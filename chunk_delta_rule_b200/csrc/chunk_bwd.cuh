@@ -741,6 +741,16 @@ constexpr uint32_t ID = tc::idesc_bf16(128, 32, false, false);
 enum { B_ABC = 0, B_D = 1, B_E = 2, B_DRAIN = 3, B_ST = 4 };
 constexpr unsigned long long kWaitNs = 2000000000ull;   // bound on every wait for an MMA
 
+// one state product: D[128 x 32] = A (TMEM, K = 128) B^T (a 32-token tile), its eight
+// k steps issued from unrolled code (the issuing warp also has its share of the
+// warp-MMA products, so its issue time is on the phase's path)
+__device__ __forceinline__ void mma8(uint32_t d, uint32_t a_tmem, uint32_t b) {
+    const uint64_t bd0 = tc::sdesc_sw128(b, 16, 1024);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks)
+        tc::mma_bf16_ta(d, a_tmem + ks * 8, bd0 + (tc::katom_off(ks, 4096) >> 4), ID, ks > 0 ? 1u : 0u);
+}
+
 // waits for a commit (each barrier completes once per CTA: phase 0); a wait that runs
 // out latches COMBA_ETIMEOUT and goes on, so the kernel still ends
 __device__ __forceinline__ void wait(uint64_t* bar) {
@@ -957,9 +967,9 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
         __syncthreads();   // q~, decays, the TMEM operands and the K / dO tiles
         if (warp == 0) {   // (a) S K^T, (b) dS' K^T, (c) S^T dO^T
             tc::tc_fence_after();
-            tc::mma_bf16_ta_bk(tmem + gtc::C_A, tmem + gtc::C_S, tcb + gtc::KB, 4096, gtc::ID, 8, 0);
-            tc::mma_bf16_ta_bk(tmem + gtc::C_B, tmem + gtc::C_DS, tcb + gtc::KB, 4096, gtc::ID, 8, 0);
-            tc::mma_bf16_ta_bk(tmem + gtc::C_C, tmem + gtc::C_ST, tcb + gtc::OB, 4096, gtc::ID, 8, 0);
+            gtc::mma8(tmem + gtc::C_A, tmem + gtc::C_S, tcb + gtc::KB);
+            gtc::mma8(tmem + gtc::C_B, tmem + gtc::C_DS, tcb + gtc::KB);
+            gtc::mma8(tmem + gtc::C_C, tmem + gtc::C_ST, tcb + gtc::OB);
             tc::mma_commit(&tbar[gtc::B_ABC]);
         }
         wgemm<kL, kL, DK, kIn, kIn>([&](int m, int x) { return Ks[m * LD + x]; },
@@ -1050,7 +1060,7 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     if constexpr (kTC) {
         if (warp == 0) {   // (d) dS'^T X^T
             tc::tc_fence_after();
-            tc::mma_bf16_ta_bk(tmem + gtc::C_D, tmem + gtc::C_DST, tcb + gtc::XB, 4096, gtc::ID, 8, 0);
+            gtc::mma8(tmem + gtc::C_D, tmem + gtc::C_DST, tcb + gtc::XB);
             tc::mma_commit(&tbar[gtc::B_D]);
         }
         gtc::f32_to_tile(tcb + gtc::DRB, Ds, LD);
@@ -1086,7 +1096,7 @@ bwd_grads_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin
     if constexpr (kTC) {
         if (warp == 0) {   // (e) S^T dR^T
             tc::tc_fence_after();
-            tc::mma_bf16_ta_bk(tmem + gtc::C_E, tmem + gtc::C_ST, tcb + gtc::DRB, 4096, gtc::ID, 8, 0);
+            gtc::mma8(tmem + gtc::C_E, tmem + gtc::C_ST, tcb + gtc::DRB);
             tc::mma_commit(&tbar[gtc::B_E]);
         }
         if (warp < 4) {
