@@ -727,9 +727,9 @@ enum { V_G, V_GP, V_BT, V_EG, V_EGP, V_DEC, V_T1, V_T2, V_ROWA, V_COLA, V_ROWP, 
 //   (d) (X dS')^T    = dS'^T X^T   A = dS' columns, B = X
 //   (e) (dR S)^T     = S^T dR^T    A = S columns,  B = dR
 // The results (fp32, lane = state index, column = token) are written back transposed
-// into the kernel's fp32 tiles.  bf16 operands for the states, X and dR put every
-// gradient of a bf16-input backward within 2e-3 (rel-L2) of the float64 gradients on
-// the 1.3B-layer inputs.
+// into the kernel's fp32 tiles.  With these bf16 operands (and the state passes' bf16
+// states) every gradient of a bf16-input backward stays within 3e-3 (rel-L2) of the
+// float64 gradients on the test shapes, 2.1e-3 on sampled chains of the 1.3B layer.
 namespace gtc {
 constexpr uint32_t C_S = 0, C_ST = 64, C_DS = 128, C_DST = 192;     // TMEM A operands (64 columns each)
 constexpr uint32_t C_A = 256, C_B = 288, C_C = 320, C_D = 352, C_E = 384;   // results (32 columns each)

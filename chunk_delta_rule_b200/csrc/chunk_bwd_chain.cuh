@@ -14,10 +14,12 @@
 //            Xd^T = (U~^T - X'^T) diag(e^{g_L - g})  as bf16 hi + lo (state group)
 //            S   += Xd^T K           two M=128, N=128, K=32 MMAs (K: MN-major tile)
 //   reverse  Z    = dS' K^T          one M=128, N=32, K=128 MMA
-//            dS  += dO^T G           two SS MMAs (dO and G hi / lo tiles, both MN-major)
+//            dS  += dO^T G           two SS MMAs (dO and G hi / lo tiles, both MN-major),
+//                                    once the master has been pre-scaled
 //            -Z diag(e^{g_L - g}) as bf16 hi + lo; dS += that times W (two MMAs)
 // with the master pre-scaled by the chunk's e^{g_L} when the state is read out.  Each
-// state read out is stored (bf16, row-major) to the workspace for the grads kernel.
+// state read out is stored (bf16, in the piece layout of stl::off) to the workspace
+// for the grads kernel.
 // The prep kernel leaves every operand in the workspace in the layout the MMAs read
 // (bf16 32 x 128 tiles, U~ fp32, the decays), so a chunk's inputs are one or two untiled
 // bulk copies into a two-stage ring.  Warps 0-3 (the state group) own the TMEM lanes;
