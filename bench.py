@@ -630,6 +630,8 @@ def run_bwd(args):
     in the data path); times are the max over ranks."""
     import chunk_delta_rule_b200 as cdr
     cfg = CONFIGS["layer1p3b_bf16"]
+    if args.batch:   # a smaller batch of the same layer, for profiling captures
+        cfg = cfg.replace(B=args.batch)
     world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -731,6 +733,9 @@ def main():
     ap.add_argument("--workload", default="layer1p3b_bf16",
                     choices=sorted(CONFIGS) + [DECODE.name, VARLEN.name, GATED, BWD])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="backward workload only: run the 1.3B layer with this batch instead of 8 "
+                         "(for profiling captures; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
