@@ -562,11 +562,16 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
         Ti[r * kLDL + sc] = -acc;
     }
     __syncthreads();
-    // U~ = T diag(beta) V (to the workspace) and W = T diag(beta e^{g'}) K (to the W tile)
+    // U~ = T diag(beta) V (to the workspace; in the tensor-core form through the dO
+    // tile, whose bf16 copy is already out, for 16-byte stores) and
+    // W = T diag(beta e^{g'}) K (to the W tile)
     float* Ug = ws.U + ci * kL * DV;
     wgemm<kL, DV, kL, true, true>([&](int r, int x) { return Ti[r * kLDL + x]; },
                                   [&](int x, int col) { return bt[x] * Vs[x * LDV + col]; },
-                                  [&](int r, int col, float u) { Ug[r * DV + col] = u; });
+                                  [&](int r, int col, float u) {
+                                      if constexpr (kTC) Os[r * LDV + col] = u;
+                                      else Ug[r * DV + col] = u;
+                                  });
     wgemm<kL, DK, kL, true, true>([&](int r, int x) { return Ti[r * kLDL + x]; },
                                   [&](int x, int col) { return cw[x] * Ks[x * LDK + col]; },
                                   [&](int r, int col, float w) { Ws[r * LDK + col] = w; });
@@ -579,6 +584,9 @@ bwd_prep_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     wgemm<kL, DK, kL, true, true>([&](int m, int x) { return Pm[m * kLDL + x]; },
                                   [&](int x, int n) { return Ws[x * LDK + n]; },
                                   [&](int m, int n, float s) { Qs[m * LDK + n] = fmaf(expf(g[m]), Qs[m * LDK + n], -s); });
+    if constexpr (kTC)
+        for (int e = tid; e < kL * DV / 4; e += kThreads)
+            reinterpret_cast<float4*>(Ug)[e] = *reinterpret_cast<const float4*>(Os + (e / (DV / 4)) * LDV + 4 * (e % (DV / 4)));
     __syncthreads();
     if constexpr (kTC) {
         tile::from_f32<false>(wk, Ws, LDK);
