@@ -454,6 +454,11 @@ constexpr uint32_t kPrepDec = 3 * tile::kBytes;
 // ... and of the chunk's inverse T = (I + A)^{-1} (fp32 [32][32], row-major), which the
 // grads kernel applies as products instead of solving again.
 constexpr uint32_t kPrepT = 4 * tile::kBytes;
+// the tensor-core form's per-chunk operands fit the slots of the fp32 layout (dk = dv = 128)
+static_assert(2 * tile::kBytes <= kL * 128 * sizeof(float), "W | K tiles exceed the W slot");
+static_assert(kPrepDec + 33 * sizeof(float) <= kPrepT && kPrepT + kL * kL * sizeof(float) <= 128 * 128 * sizeof(float),
+              "G, dO tiles, decays and T exceed the C slot");
+static_assert(128 * 128 * 2 <= 128 * 128 * sizeof(float), "a bf16 state exceeds its slot");
 
 // ---------------------------------------------------------------------------------
 // bwd_prep: W, U~ and C = dO^T (Gamma Q~ - P W) of one chunk.  In the tensor-core form
@@ -860,6 +865,11 @@ __host__ __device__ constexpr size_t grads_smem_bytes() {
     return grads_tc<Tin, DK, DV>() ? GradSmem<DK, DV>::STG * sizeof(float) + 1024 + gtc::kBytes
                                    : GradSmem<DK, DV>::total * sizeof(float);
 }
+static_assert(grads_smem_bytes<__nv_bfloat16, 128, 128>() <= 227 * 1024 &&
+                  grads_smem_bytes<float, 128, 128>() <= 227 * 1024,
+              "the grads kernel exceeds the shared memory of one CTA");
+// the two 32 KB state copies land in the R | X and G | TK tiles
+static_assert(2 * kL * (128 + 4) * sizeof(float) >= 32768, "state staging does not fit two tiles");
 
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kThreads)

@@ -50,6 +50,10 @@ constexpr uint32_t ST_W = 0, ST_K = 8192, ST_U = 16384, ST_G = 16384, ST_GLO = 2
 constexpr uint32_t SM_BARS = 2 * ST_BYTES;     // 8 mbarriers, the TMEM slot, the abort flag
 constexpr uint32_t kSmemBytes = SM_BARS + 128 + 1024;   // + alignment slack
 enum { B_FULL0 = 0, B_FULL1 = 1, B_SREADY = 2, B_SPLIT = 3, B_MMA1 = 4, B_MMA2 = 5, B_DRAIN = 6, B_MREADY = 7 };
+static_assert(ST_DEC + 256 <= ST_BYTES && ST_BYTES % 1024 == 0, "ring stage layout");
+static_assert(ST_G + kPrepDec + 256 == ST_DEC + 256 && ST_DO == ST_G + 2 * tile::kBytes,
+              "the reverse walk's copy of the C slot lands G hi, G lo, dO and the decays in place");
+static_assert(2 * kSmemBytes <= 228 * 1024 - 2 * 1024, "two state-pass CTAs per SM");
 
 constexpr uint32_t ID_N32 = tc::idesc_bf16(128, 32, false, false);    // S W^T, dS' K^T
 constexpr uint32_t ID_N128B = tc::idesc_bf16(128, 128, false, true);  // Xd^T K, Zd W (B MN-major)
